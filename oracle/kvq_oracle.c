@@ -1,0 +1,581 @@
+/*
+ * kvq_oracle.c -- plain, slow CPU oracle for centroid-residual low-bit
+ * KV-cache compression.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Nothing on the product path may call, link or
+ * load this file; only the test suite, the smoke check and the benchmark's
+ * CPU-baseline leg do.  It shares no code with the CUDA library.
+ *
+ * Build: gcc -O2 -std=c11 -ffp-contract=off -fno-fast-math -fopenmp -shared -fPIC
+ * (strict IEEE binary32/binary64, no fused multiply-add, x86-64 SSE math).
+ *
+ * What it computes, and where the pages define it:
+ *
+ *  - nearest-centroid assignment of every key/value token of a head:
+ *    QuantWM: Temporally Consistent 2-Bit KV Cache Quantization for Video
+ *    World Models, Sec. 4.1 (QVG applies k-means to assign each key token to
+ *    its nearest centroid, then quantises the residual); TempoKV, Sec. 1
+ *    (QVG groups similar tokens and subtracts the group centroid).
+ *  - per-head k-means fitted online per cache block, separately for K and V:
+ *    CORAL-KV, Sec. 2 (QVG fits per-head centroid codebooks online for each
+ *    cache block); NanoKV page, Table 4 (QVG: 256 centres each for K/V, two
+ *    k-means iterations, BF16 centres) and Table 5 (centres fitted separately
+ *    for K and V).
+ *  - residual form X^ = X~ + D(Q(X - X~)) with the centroid as prediction:
+ *    TempoKV, Sec. 3.3, Eq. 2.
+ *  - asymmetric b-bit affine quantisation s = (max - min)/(2^b - 1),
+ *    z = round(-min/s), Q = round(X/s) + z, X^ = (Q - z) s: TempoKV, Sec. 3.1,
+ *    Eq. 1, applied per contiguous channel group (QuantWM Sec. 4.1: group
+ *    range R_g and step R_g/(2^b - 1)).
+ *  - packed INT2/INT4 storage: NanoKV page, Table 4 (packed INT2/INT4);
+ *    QuantWM, Fig. 9 (packed storage, on-demand reconstruction).
+ *  - joint head-channel linear encoder/decoder with INT4 coefficients, centres
+ *    added back after decoding: NanoKV page, abstract and Fig. 4(a,b).
+ *
+ * Readings taken where the pages are silent (each mirrored by the CUDA
+ * library and listed in the design notes):
+ *  - distance = squared Euclidean, evaluated as: widen to binary32; for
+ *    c = 0..d-1 in order, e = x_c - mu_c, acc = acc + e*e, each operation
+ *    rounded separately (no FMA); ties go to the lowest centroid index;
+ *  - k-means seeds = the first C tokens (rounded to bf16); each iteration
+ *    assigns, then sets mu_j = bf16(float(sum_fp64 / n_j)); empty clusters
+ *    keep their centre; a fixed iteration count, no convergence test;
+ *  - Eq. 1's round-to-nearest is round-half-to-even; X/s is evaluated as
+ *    X * inv with inv = 1/s (one IEEE division per group); codes are clamped
+ *    to [0, 2^b - 1];
+ *  - a group whose range is zero, or whose scale s underflows below the
+ *    smallest normal binary32, is "degenerate": s = |min|, z = -sign(min),
+ *    codes 0, which decodes to exactly min (and to 0 when min == 0);
+ *  - decode: x^_c = mu_c + (q_c - z) * s with the subtraction, multiply and
+ *    add each rounded to binary32.
+ */
+
+#include <float.h>
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+#define KVQO_OK 0
+#define KVQO_EINVAL 1
+#define KVQO_ENOMEM 2
+
+/* ------------------------------------------------------------------------ */
+/* bf16 storage conversions                                                  */
+/* ------------------------------------------------------------------------ */
+
+static float bf16_widen(uint16_t h)
+{
+    uint32_t u = ((uint32_t)h) << 16;
+    float f;
+    memcpy(&f, &u, sizeof f);
+    return f;
+}
+
+/* binary32 -> bf16, round to nearest, ties to even (NaN kept quiet). */
+static uint16_t bf16_round(float f)
+{
+    uint32_t u;
+    memcpy(&u, &f, sizeof u);
+    if ((u & 0x7f800000u) == 0x7f800000u && (u & 0x007fffffu) != 0u)
+        return (uint16_t)((u >> 16) | 0x0040u);
+    uint32_t keep_lsb = (u >> 16) & 1u;
+    u += 0x7fffu + keep_lsb;
+    return (uint16_t)(u >> 16);
+}
+
+uint16_t kvqo_bf16_round(float f) { return bf16_round(f); }
+
+/* x is either binary32 ([n]) or bf16 bit patterns ([n]); returns binary32. */
+static float load_x(const void *x, int x_is_bf16, int64_t i)
+{
+    if (x_is_bf16)
+        return bf16_widen(((const uint16_t *)x)[i]);
+    return ((const float *)x)[i];
+}
+
+/* ------------------------------------------------------------------------ */
+/* distance and assignment                                                   */
+/* ------------------------------------------------------------------------ */
+
+/* The specified squared distance: sequential over channels, no FMA. */
+float kvqo_distance(const float *x, const float *mu, int d)
+{
+    float acc = 0.0f;
+    for (int c = 0; c < d; ++c) {
+        float e = x[c] - mu[c];
+        float sq = e * e;
+        acc = acc + sq;
+    }
+    return acc;
+}
+
+/* Brute-force nearest centre of one vector; strict '<' keeps the lowest index
+ * among equal distances.  mu is [C][d] binary32. */
+static int nearest(const float *x, const float *mu, int C, int d, float *best_out)
+{
+    int best = 0;
+    float bd = kvqo_distance(x, mu, d);
+    for (int j = 1; j < C; ++j) {
+        float dj = kvqo_distance(x, mu + (int64_t)j * d, d);
+        if (dj < bd) {
+            bd = dj;
+            best = j;
+        }
+    }
+    if (best_out)
+        *best_out = bd;
+    return best;
+}
+
+/* Widen one head's centres [C][d] (bf16) to binary32. */
+static void widen_centres(const uint16_t *cent_h, int C, int d, float *out)
+{
+    for (int64_t i = 0; i < (int64_t)C * d; ++i)
+        out[i] = bf16_widen(cent_h[i]);
+}
+
+/* Gather token t of head h ([T][H][d] input) as binary32. */
+static void gather_token(const void *x, int x_is_bf16, int H, int d, int64_t t, int h, float *out)
+{
+    int64_t base = (t * H + h) * (int64_t)d;
+    for (int c = 0; c < d; ++c)
+        out[c] = load_x(x, x_is_bf16, base + c);
+}
+
+/*
+ * idx[h][t] = argmin_j D(x_{t,h}, mu_{h,j}).
+ * x: [T][H][d] (binary32 or bf16), cent: [H][C][d] bf16, idx: [H][T] uint16.
+ * dist_out (optional): [H][T] binary32 distance of the chosen centre.
+ */
+int kvqo_assign(const void *x, int x_is_bf16, int64_t T, int H, int d,
+                const uint16_t *cent, int C, uint16_t *idx, float *dist_out)
+{
+    if (T < 0 || H <= 0 || d <= 0 || C <= 0 || C > 65536)
+        return KVQO_EINVAL;
+    int rc = KVQO_OK;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int h = 0; h < H; ++h) {
+        float *mu = (float *)malloc(sizeof(float) * (size_t)C * d);
+        float *xv = (float *)malloc(sizeof(float) * (size_t)d);
+        if (!mu || !xv) {
+            rc = KVQO_ENOMEM;
+        } else {
+            widen_centres(cent + (int64_t)h * C * d, C, d, mu);
+            for (int64_t t = 0; t < T; ++t) {
+                gather_token(x, x_is_bf16, H, d, t, h, xv);
+                float bd;
+                int j = nearest(xv, mu, C, d, &bd);
+                idx[(int64_t)h * T + t] = (uint16_t)j;
+                if (dist_out)
+                    dist_out[(int64_t)h * T + t] = bd;
+            }
+        }
+        free(mu);
+        free(xv);
+    }
+    return rc;
+}
+
+/* ------------------------------------------------------------------------ */
+/* k-means fitting                                                           */
+/* ------------------------------------------------------------------------ */
+
+/*
+ * Per head: seed mu_j = bf16(x_j) for the first C tokens; then `iters` times:
+ * assign every token, mu_j = bf16(float(sum_{t in j} x_t / n_j)) with the sum
+ * in binary64 in token order; a centre with no tokens keeps its value.
+ * inertia_out (optional): [H][iters + 1] binary64 sum of exact squared
+ * distances of every token to its assigned centre, measured with the centres
+ * in force before each iteration's update (index 0..iters-1) and with the
+ * final centres (index iters).
+ */
+int kvqo_fit(const void *x, int x_is_bf16, int64_t T, int H, int d, int C, int iters,
+             uint16_t *cent_out, double *inertia_out)
+{
+    if (T < C || H <= 0 || d <= 0 || C <= 0 || C > 65536 || iters < 0)
+        return KVQO_EINVAL;
+    int rc = KVQO_OK;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int h = 0; h < H; ++h) {
+        uint16_t *cent_h = cent_out + (int64_t)h * C * d;
+        float *mu = (float *)malloc(sizeof(float) * (size_t)C * d);
+        float *xv = (float *)malloc(sizeof(float) * (size_t)d);
+        double *sums = (double *)malloc(sizeof(double) * (size_t)C * d);
+        int64_t *counts = (int64_t *)malloc(sizeof(int64_t) * (size_t)C);
+        if (!mu || !xv || !sums || !counts) {
+            rc = KVQO_ENOMEM;
+            goto done;
+        }
+        for (int j = 0; j < C; ++j) {
+            gather_token(x, x_is_bf16, H, d, j, h, xv);
+            for (int c = 0; c < d; ++c)
+                cent_h[(int64_t)j * d + c] = bf16_round(xv[c]);
+        }
+        for (int it = 0; it <= iters; ++it) {
+            widen_centres(cent_h, C, d, mu);
+            memset(sums, 0, sizeof(double) * (size_t)C * d);
+            memset(counts, 0, sizeof(int64_t) * (size_t)C);
+            double inertia = 0.0;
+            for (int64_t t = 0; t < T; ++t) {
+                gather_token(x, x_is_bf16, H, d, t, h, xv);
+                int j = nearest(xv, mu, C, d, NULL);
+                counts[j] += 1;
+                for (int c = 0; c < d; ++c) {
+                    sums[(int64_t)j * d + c] += (double)xv[c];
+                    double e = (double)xv[c] - (double)mu[(int64_t)j * d + c];
+                    inertia += e * e;
+                }
+            }
+            if (inertia_out)
+                inertia_out[(int64_t)h * (iters + 1) + it] = inertia;
+            if (it == iters)
+                break;
+            for (int j = 0; j < C; ++j) {
+                if (counts[j] == 0)
+                    continue;
+                for (int c = 0; c < d; ++c) {
+                    double mean = sums[(int64_t)j * d + c] / (double)counts[j];
+                    cent_h[(int64_t)j * d + c] = bf16_round((float)mean);
+                }
+            }
+        }
+    done:
+        free(mu);
+        free(xv);
+        free(sums);
+        free(counts);
+    }
+    return rc;
+}
+
+/* ------------------------------------------------------------------------ */
+/* Eq. 1 quantisation of one group                                           */
+/* ------------------------------------------------------------------------ */
+
+/*
+ * r: G residuals.  Writes scale s, zero z and G codes in [0, 2^bits - 1].
+ */
+void kvqo_quant_group(const float *r, int G, int bits, float *s_out, float *z_out, uint8_t *q)
+{
+    float mn = r[0], mx = r[0];
+    for (int c = 1; c < G; ++c) {
+        if (r[c] < mn)
+            mn = r[c];
+        if (r[c] > mx)
+            mx = r[c];
+    }
+    const float qmax = (float)((1 << bits) - 1);
+    float s = 0.0f;
+    if (mx != mn)
+        s = (mx - mn) / qmax;
+    if (mx == mn || !(s >= FLT_MIN)) {
+        /* degenerate group: decodes to exactly mn */
+        if (mn == 0.0f) {
+            *s_out = 0.0f;
+            *z_out = 0.0f;
+        } else {
+            *s_out = fabsf(mn);
+            *z_out = (mn > 0.0f) ? -1.0f : 1.0f;
+        }
+        for (int c = 0; c < G; ++c)
+            q[c] = 0;
+        return;
+    }
+    float inv = 1.0f / s;
+    float z = rintf(-mn * inv);
+    for (int c = 0; c < G; ++c) {
+        float v = rintf(r[c] * inv) + z;
+        if (v < 0.0f)
+            v = 0.0f;
+        if (v > qmax)
+            v = qmax;
+        q[c] = (uint8_t)v;
+    }
+    *s_out = s;
+    *z_out = z;
+}
+
+/* x^ = (q - z) * s, each step rounded to binary32. */
+float kvqo_dequant(uint8_t q, float s, float z)
+{
+    float t = (float)q - z;
+    return t * s;
+}
+
+/* ------------------------------------------------------------------------ */
+/* packing                                                                   */
+/* ------------------------------------------------------------------------ */
+
+/* n codes of `bits` (2 or 4) into n*bits/8 bytes, least significant first. */
+void kvqo_pack(const uint8_t *q, int n, int bits, uint8_t *out)
+{
+    int per = 8 / bits;
+    for (int k = 0; k < n / per; ++k) {
+        unsigned byte = 0;
+        for (int i = 0; i < per; ++i)
+            byte |= ((unsigned)q[k * per + i] & ((1u << bits) - 1u)) << (i * bits);
+        out[k] = (uint8_t)byte;
+    }
+}
+
+void kvqo_unpack(const uint8_t *in, int n, int bits, uint8_t *q)
+{
+    int per = 8 / bits;
+    for (int c = 0; c < n; ++c)
+        q[c] = (uint8_t)((in[c / per] >> ((c % per) * bits)) & ((1u << bits) - 1u));
+}
+
+/* ------------------------------------------------------------------------ */
+/* per-head encode / decode                                                  */
+/* ------------------------------------------------------------------------ */
+
+static int check_codec(int H, int d, int C, int bits, int G)
+{
+    if (H <= 0 || d <= 0 || C <= 0 || C > 65536)
+        return 0;
+    if (bits != 2 && bits != 4)
+        return 0;
+    if (G <= 0 || d % G != 0 || (d * bits) % 8 != 0 || G > 256)
+        return 0;
+    return 1;
+}
+
+/*
+ * Encode one K or V history.
+ *   x     [T][H][d]  binary32 or bf16
+ *   cent  [H][C][d]  bf16
+ *   idx   [H][T]     uint16 (out)
+ *   codes [H][T][d*bits/8]  packed (out)
+ *   meta  [H][T][d/G][2]    {s, z} binary32 (out)
+ */
+int kvqo_encode(const void *x, int x_is_bf16, int64_t T, int H, int d, const uint16_t *cent, int C,
+                int bits, int G, uint16_t *idx, uint8_t *codes, float *meta)
+{
+    if (T < 0 || !check_codec(H, d, C, bits, G))
+        return KVQO_EINVAL;
+    const int cb = d * bits / 8, ng = d / G;
+    int rc = KVQO_OK;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int h = 0; h < H; ++h) {
+        float *mu = (float *)malloc(sizeof(float) * (size_t)C * d);
+        float *xv = (float *)malloc(sizeof(float) * (size_t)d);
+        float *r = (float *)malloc(sizeof(float) * (size_t)d);
+        uint8_t *q = (uint8_t *)malloc((size_t)d);
+        if (!mu || !xv || !r || !q) {
+            rc = KVQO_ENOMEM;
+        } else {
+            widen_centres(cent + (int64_t)h * C * d, C, d, mu);
+            for (int64_t t = 0; t < T; ++t) {
+                int64_t th = (int64_t)h * T + t;
+                gather_token(x, x_is_bf16, H, d, t, h, xv);
+                int j = nearest(xv, mu, C, d, NULL);
+                idx[th] = (uint16_t)j;
+                for (int c = 0; c < d; ++c)
+                    r[c] = xv[c] - mu[(int64_t)j * d + c];
+                for (int g = 0; g < ng; ++g) {
+                    float s, z;
+                    kvqo_quant_group(r + g * G, G, bits, &s, &z, q + g * G);
+                    meta[(th * ng + g) * 2 + 0] = s;
+                    meta[(th * ng + g) * 2 + 1] = z;
+                }
+                kvqo_pack(q, d, bits, codes + th * cb);
+            }
+        }
+        free(mu);
+        free(xv);
+        free(r);
+        free(q);
+    }
+    return rc;
+}
+
+/* Reconstruct [T][H][d] binary32 from the encoded form. */
+int kvqo_decode(const uint16_t *idx, const uint8_t *codes, const float *meta, const uint16_t *cent,
+                int64_t T, int H, int d, int C, int bits, int G, float *out)
+{
+    if (T < 0 || !check_codec(H, d, C, bits, G))
+        return KVQO_EINVAL;
+    const int cb = d * bits / 8, ng = d / G;
+    int rc = KVQO_OK;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int h = 0; h < H; ++h) {
+        uint8_t *q = (uint8_t *)malloc((size_t)d);
+        if (!q) {
+            rc = KVQO_ENOMEM;
+            continue;
+        }
+        for (int64_t t = 0; t < T; ++t) {
+            int64_t th = (int64_t)h * T + t;
+            int j = idx[th];
+            if (j >= C) {
+                rc = KVQO_EINVAL;
+                break;
+            }
+            kvqo_unpack(codes + th * cb, d, bits, q);
+            for (int c = 0; c < d; ++c) {
+                int g = c / G;
+                float s = meta[(th * ng + g) * 2 + 0];
+                float z = meta[(th * ng + g) * 2 + 1];
+                float mu = bf16_widen(cent[((int64_t)h * C + j) * d + c]);
+                out[(t * H + h) * (int64_t)d + c] = mu + kvqo_dequant(q[c], s, z);
+            }
+        }
+        free(q);
+    }
+    return rc;
+}
+
+/* ------------------------------------------------------------------------ */
+/* joint head-channel path                                                   */
+/* ------------------------------------------------------------------------ */
+
+/*
+ * Quantise a [T][r] binary32 coefficient matrix with Eq. 1 per contiguous
+ * group of G coefficients: codes [T][r*bits/8], meta [T][r/G][2].
+ */
+int kvqo_quant_rows(const float *coef, int64_t T, int r, int bits, int G, uint8_t *codes, float *meta)
+{
+    if (T < 0 || r <= 0 || (bits != 2 && bits != 4) || G <= 0 || r % G != 0 || (r * bits) % 8 != 0)
+        return KVQO_EINVAL;
+    const int cb = r * bits / 8, ng = r / G;
+    int rc = KVQO_OK;
+#pragma omp parallel for schedule(static)
+    for (int64_t t = 0; t < T; ++t) {
+        uint8_t *q = (uint8_t *)malloc((size_t)r);
+        if (!q) {
+            rc = KVQO_ENOMEM;
+            continue;
+        }
+        for (int g = 0; g < ng; ++g) {
+            float s, z;
+            kvqo_quant_group(coef + t * r + g * G, G, bits, &s, &z, q + g * G);
+            meta[(t * ng + g) * 2 + 0] = s;
+            meta[(t * ng + g) * 2 + 1] = z;
+        }
+        kvqo_pack(q, r, bits, codes + t * cb);
+        free(q);
+    }
+    return rc;
+}
+
+/*
+ * Joint encoder.  Per token: assign each head to its nearest centre (as the
+ * per-head codec), form the residual over all H*d channels, round it to bf16,
+ * project with W_enc ([H*d][r] bf16) in binary64, round to binary32, and
+ * quantise the r coefficients per group of G.
+ *   idx [H][T], codes [T][r*bits/8], meta [T][r/G][2]; coef_out (optional)
+ *   [T][r] binary32 coefficients before quantisation.
+ */
+int kvqo_joint_encode(const void *x, int x_is_bf16, int64_t T, int H, int d, const uint16_t *cent, int C,
+                      const uint16_t *w_enc, int r, int bits, int G,
+                      uint16_t *idx, uint8_t *codes, float *meta, float *coef_out)
+{
+    if (T < 0 || H <= 0 || d <= 0 || C <= 0 || C > 65536 || r <= 0)
+        return KVQO_EINVAL;
+    if ((bits != 2 && bits != 4) || G <= 0 || r % G != 0 || (r * bits) % 8 != 0)
+        return KVQO_EINVAL;
+    const int64_t n = (int64_t)H * d;
+    float *coef = (float *)malloc(sizeof(float) * (size_t)(T > 0 ? T : 1) * r);
+    float *w = (float *)malloc(sizeof(float) * (size_t)n * r);
+    float *mu = (float *)malloc(sizeof(float) * (size_t)H * C * d);
+    if (!coef || !w || !mu) {
+        free(coef);
+        free(w);
+        free(mu);
+        return KVQO_ENOMEM;
+    }
+    for (int64_t i = 0; i < n * r; ++i)
+        w[i] = bf16_widen(w_enc[i]);
+    for (int64_t i = 0; i < (int64_t)H * C * d; ++i)
+        mu[i] = bf16_widen(cent[i]);
+    int rc = KVQO_OK;
+#pragma omp parallel for schedule(static)
+    for (int64_t t = 0; t < T; ++t) {
+        float *xv = (float *)malloc(sizeof(float) * (size_t)d);
+        float *res = (float *)malloc(sizeof(float) * (size_t)n);
+        if (!xv || !res) {
+            rc = KVQO_ENOMEM;
+            free(xv);
+            free(res);
+            continue;
+        }
+        for (int h = 0; h < H; ++h) {
+            const float *mu_h = mu + (int64_t)h * C * d;
+            gather_token(x, x_is_bf16, H, d, t, h, xv);
+            int j = nearest(xv, mu_h, C, d, NULL);
+            idx[(int64_t)h * T + t] = (uint16_t)j;
+            for (int c = 0; c < d; ++c) {
+                float e = xv[c] - mu_h[(int64_t)j * d + c];
+                res[h * d + c] = bf16_widen(bf16_round(e));
+            }
+        }
+        for (int k = 0; k < r; ++k) {
+            double acc = 0.0;
+            for (int64_t i = 0; i < n; ++i)
+                acc += (double)res[i] * (double)w[i * r + k];
+            coef[t * r + k] = (float)acc;
+        }
+        free(xv);
+        free(res);
+    }
+    if (rc == KVQO_OK)
+        rc = kvqo_quant_rows(coef, T, r, bits, G, codes, meta);
+    if (coef_out && rc == KVQO_OK)
+        memcpy(coef_out, coef, sizeof(float) * (size_t)T * r);
+    free(coef);
+    free(w);
+    free(mu);
+    return rc;
+}
+
+/*
+ * Joint decoder: c^ = (q - z) s per coefficient (binary32), R^ = c^ W_dec in
+ * binary64 with W_dec [r][H*d] bf16, rounded to binary32, then
+ * x^_{t,h,c} = mu_{h, idx}[c] + R^[h*d + c] in binary32.  out [T][H][d].
+ */
+int kvqo_joint_decode(const uint16_t *idx, const uint8_t *codes, const float *meta, const uint16_t *cent,
+                      const uint16_t *w_dec, int64_t T, int H, int d, int C, int r, int bits, int G,
+                      float *out)
+{
+    if (T < 0 || H <= 0 || d <= 0 || C <= 0 || r <= 0 || (bits != 2 && bits != 4) || G <= 0 || r % G != 0)
+        return KVQO_EINVAL;
+    const int64_t n = (int64_t)H * d;
+    const int cb = r * bits / 8, ng = r / G;
+    float *w = (float *)malloc(sizeof(float) * (size_t)n * r);
+    if (!w)
+        return KVQO_ENOMEM;
+    for (int64_t i = 0; i < n * r; ++i)
+        w[i] = bf16_widen(w_dec[i]);
+    int rc = KVQO_OK;
+#pragma omp parallel for schedule(static)
+    for (int64_t t = 0; t < T; ++t) {
+        uint8_t *q = (uint8_t *)malloc((size_t)r);
+        float *ch = (float *)malloc(sizeof(float) * (size_t)r);
+        if (!q || !ch) {
+            rc = KVQO_ENOMEM;
+            free(q);
+            free(ch);
+            continue;
+        }
+        kvqo_unpack(codes + t * cb, r, bits, q);
+        for (int k = 0; k < r; ++k) {
+            int g = k / G;
+            ch[k] = kvqo_dequant(q[k], meta[(t * ng + g) * 2 + 0], meta[(t * ng + g) * 2 + 1]);
+        }
+        for (int h = 0; h < H; ++h) {
+            int j = idx[(int64_t)h * T + t];
+            for (int c = 0; c < d; ++c) {
+                double acc = 0.0;
+                for (int k = 0; k < r; ++k)
+                    acc += (double)ch[k] * (double)w[(int64_t)k * n + h * d + c];
+                float mu = bf16_widen(cent[((int64_t)h * C + j) * d + c]);
+                out[(t * H + h) * (int64_t)d + c] = mu + (float)acc;
+            }
+        }
+        free(q);
+        free(ch);
+    }
+    free(w);
+    return rc;
+}

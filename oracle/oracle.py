@@ -1,0 +1,308 @@
+"""Python face of the CPU oracle.
+
+TEST INFRASTRUCTURE ONLY.  Only the test suite, ``__graft_entry__.smoke()``
+and the benchmark's CPU-baseline / reference leg may import this module.  It
+shares no code with the CUDA library: the codec steps run in the plain C file
+next to it (strict IEEE, no FMA) and attention / log-sum-exp merging run here
+in NumPy float64.
+
+Functions and the passages they follow:
+
+* ``assign``, ``fit``, ``encode``, ``decode``: centroid-residual codec -- see
+  the header of kvq_oracle.c (QuantWM Sec. 4.1; TempoKV Sec. 3.1 Eq. 1 and
+  Sec. 3.3 Eq. 2; CORAL-KV Sec. 2; NanoKV page Tables 4-5).
+* ``joint_encode``, ``joint_decode``, ``quant_rows``: joint head-channel
+  encoder/decoder with INT4 coefficients (NanoKV page, abstract, Fig. 4(b)).
+* ``attention``: softmax attention of the current chunk's queries over the
+  reconstructed history, returning the output and the natural-log
+  log-sum-exp of the logits (NanoKV page, Fig. 4(a,d)).
+* ``lse_merge``: combination of partial attention results over history parts
+  by their log-sum-exp (NanoKV page, Fig. 4(d)).
+* ``stored_bytes_per_token_head`` / ``bits_per_value``: storage accounting.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+from typing import List, Optional, Sequence, Tuple
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_LIB_PATH = os.path.join(_HERE, "libkvq_oracle.so")
+_lib = None
+
+
+def _load():
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(_LIB_PATH) or os.path.getmtime(_LIB_PATH) < os.path.getmtime(
+            os.path.join(_HERE, "kvq_oracle.c")):
+        from . import build as _b  # type: ignore
+        _b.build()
+    lib = ctypes.CDLL(_LIB_PATH)
+    vp, i64, i32 = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int
+    lib.kvqo_assign.argtypes = [vp, i32, i64, i32, i32, vp, i32, vp, vp]
+    lib.kvqo_fit.argtypes = [vp, i32, i64, i32, i32, i32, i32, vp, vp]
+    lib.kvqo_encode.argtypes = [vp, i32, i64, i32, i32, vp, i32, i32, i32, vp, vp, vp]
+    lib.kvqo_decode.argtypes = [vp, vp, vp, vp, i64, i32, i32, i32, i32, i32, vp]
+    lib.kvqo_quant_rows.argtypes = [vp, i64, i32, i32, i32, vp, vp]
+    lib.kvqo_joint_encode.argtypes = [vp, i32, i64, i32, i32, vp, i32, vp, i32, i32, i32, vp, vp, vp, vp]
+    lib.kvqo_joint_decode.argtypes = [vp, vp, vp, vp, vp, i64, i32, i32, i32, i32, i32, i32, vp]
+    lib.kvqo_distance.argtypes = [vp, vp, i32]
+    lib.kvqo_distance.restype = ctypes.c_float
+    lib.kvqo_quant_group.argtypes = [vp, i32, i32, vp, vp, vp]
+    lib.kvqo_dequant.argtypes = [ctypes.c_uint8, ctypes.c_float, ctypes.c_float]
+    lib.kvqo_dequant.restype = ctypes.c_float
+    lib.kvqo_pack.argtypes = [vp, i32, i32, vp]
+    lib.kvqo_unpack.argtypes = [vp, i32, i32, vp]
+    lib.kvqo_bf16_round.argtypes = [ctypes.c_float]
+    lib.kvqo_bf16_round.restype = ctypes.c_uint16
+    _lib = lib
+    return lib
+
+
+def _ptr(a: np.ndarray) -> int:
+    assert a.flags["C_CONTIGUOUS"]
+    return a.ctypes.data
+
+
+def _x_arg(x: np.ndarray) -> Tuple[np.ndarray, int]:
+    if x.dtype == np.float32:
+        return np.ascontiguousarray(x), 0
+    if x.dtype == np.uint16:
+        return np.ascontiguousarray(x), 1
+    raise TypeError("history must be float32 or uint16 bf16 bits")
+
+
+def _check(rc: int, what: str):
+    if rc != 0:
+        raise RuntimeError(f"oracle {what} failed with code {rc}")
+
+
+# ----------------------------------------------------------------------------
+# scalar helpers (exposed for pinning)
+# ----------------------------------------------------------------------------
+
+def distance(x: np.ndarray, mu: np.ndarray) -> float:
+    """The specified binary32 squared distance of two float32 vectors."""
+    x = np.ascontiguousarray(x, dtype=np.float32)
+    mu = np.ascontiguousarray(mu, dtype=np.float32)
+    return float(_load().kvqo_distance(_ptr(x), _ptr(mu), x.shape[0]))
+
+
+def quant_group(r: np.ndarray, bits: int) -> Tuple[float, float, np.ndarray]:
+    """Eq. 1 on one group of residuals: (scale, zero, codes)."""
+    r = np.ascontiguousarray(r, dtype=np.float32)
+    s = np.zeros(1, np.float32)
+    z = np.zeros(1, np.float32)
+    q = np.zeros(r.shape[0], np.uint8)
+    _load().kvqo_quant_group(_ptr(r), r.shape[0], bits, _ptr(s), _ptr(z), _ptr(q))
+    return float(s[0]), float(z[0]), q
+
+
+def dequant(q: int, s: float, z: float) -> float:
+    return float(_load().kvqo_dequant(q, s, z))
+
+
+def pack(q: np.ndarray, bits: int) -> np.ndarray:
+    q = np.ascontiguousarray(q, dtype=np.uint8)
+    out = np.zeros(q.shape[0] * bits // 8, np.uint8)
+    _load().kvqo_pack(_ptr(q), q.shape[0], bits, _ptr(out))
+    return out
+
+
+def unpack(b: np.ndarray, n: int, bits: int) -> np.ndarray:
+    b = np.ascontiguousarray(b, dtype=np.uint8)
+    out = np.zeros(n, np.uint8)
+    _load().kvqo_unpack(_ptr(b), n, bits, _ptr(out))
+    return out
+
+
+def bf16_round(f: float) -> int:
+    return int(_load().kvqo_bf16_round(f))
+
+
+# ----------------------------------------------------------------------------
+# codec
+# ----------------------------------------------------------------------------
+
+def assign(x: np.ndarray, cent: np.ndarray, return_dist: bool = False):
+    """idx [H][T] of the nearest centre per token-head.  x [T][H][d], cent [H][C][d] bf16 bits."""
+    x, xb = _x_arg(x)
+    T, H, d = x.shape
+    C = cent.shape[1]
+    cent = np.ascontiguousarray(cent, dtype=np.uint16)
+    idx = np.zeros((H, T), np.uint16)
+    dist = np.zeros((H, T), np.float32)
+    _check(_load().kvqo_assign(_ptr(x), xb, T, H, d, _ptr(cent), C, _ptr(idx), _ptr(dist)), "assign")
+    return (idx, dist) if return_dist else idx
+
+
+def fit(x: np.ndarray, num_centroids: int, iters: int, return_inertia: bool = False):
+    """Per-head k-means centres [H][C][d] (bf16 bits)."""
+    x, xb = _x_arg(x)
+    T, H, d = x.shape
+    cent = np.zeros((H, num_centroids, d), np.uint16)
+    inertia = np.zeros((H, iters + 1), np.float64)
+    _check(_load().kvqo_fit(_ptr(x), xb, T, H, d, num_centroids, iters, _ptr(cent), _ptr(inertia)), "fit")
+    return (cent, inertia) if return_inertia else cent
+
+
+def encode(x: np.ndarray, cent: np.ndarray, bits: int, group: int):
+    """(idx [H][T] u16, codes [H][T][d*bits/8] u8, meta [H][T][d/G][2] f32)."""
+    x, xb = _x_arg(x)
+    T, H, d = x.shape
+    C = cent.shape[1]
+    cent = np.ascontiguousarray(cent, dtype=np.uint16)
+    idx = np.zeros((H, T), np.uint16)
+    codes = np.zeros((H, T, d * bits // 8), np.uint8)
+    meta = np.zeros((H, T, d // group, 2), np.float32)
+    _check(_load().kvqo_encode(_ptr(x), xb, T, H, d, _ptr(cent), C, bits, group,
+                               _ptr(idx), _ptr(codes), _ptr(meta)), "encode")
+    return idx, codes, meta
+
+
+def decode(idx: np.ndarray, codes: np.ndarray, meta: np.ndarray, cent: np.ndarray,
+           bits: int, group: int) -> np.ndarray:
+    """Reconstruction [T][H][d] float32."""
+    H, T = idx.shape
+    C, d = cent.shape[1], cent.shape[2]
+    out = np.zeros((T, H, d), np.float32)
+    args = [np.ascontiguousarray(a) for a in (idx, codes, meta, cent)]
+    _check(_load().kvqo_decode(*(_ptr(a) for a in args), T, H, d, C, bits, group, _ptr(out)), "decode")
+    return out
+
+
+def quant_rows(coef: np.ndarray, bits: int, group: int):
+    """Eq. 1 per contiguous group along rows of a [T][r] float32 matrix."""
+    coef = np.ascontiguousarray(coef, dtype=np.float32)
+    T, r = coef.shape
+    codes = np.zeros((T, r * bits // 8), np.uint8)
+    meta = np.zeros((T, r // group, 2), np.float32)
+    _check(_load().kvqo_quant_rows(_ptr(coef), T, r, bits, group, _ptr(codes), _ptr(meta)), "quant_rows")
+    return codes, meta
+
+
+def joint_encode(x: np.ndarray, cent: np.ndarray, w_enc: np.ndarray, bits: int, group: int):
+    """(idx [H][T], codes [T][r*bits/8], meta [T][r/G][2], coef [T][r] f32)."""
+    x, xb = _x_arg(x)
+    T, H, d = x.shape
+    C = cent.shape[1]
+    r = w_enc.shape[1]
+    cent = np.ascontiguousarray(cent, dtype=np.uint16)
+    w_enc = np.ascontiguousarray(w_enc, dtype=np.uint16)
+    idx = np.zeros((H, T), np.uint16)
+    codes = np.zeros((T, r * bits // 8), np.uint8)
+    meta = np.zeros((T, r // group, 2), np.float32)
+    coef = np.zeros((T, r), np.float32)
+    _check(_load().kvqo_joint_encode(_ptr(x), xb, T, H, d, _ptr(cent), C, _ptr(w_enc), r, bits, group,
+                                     _ptr(idx), _ptr(codes), _ptr(meta), _ptr(coef)), "joint_encode")
+    return idx, codes, meta, coef
+
+
+def joint_decode(idx, codes, meta, cent, w_dec, bits: int, group: int) -> np.ndarray:
+    H, T = idx.shape
+    C, d = cent.shape[1], cent.shape[2]
+    r = w_dec.shape[0]
+    out = np.zeros((T, H, d), np.float32)
+    args = [np.ascontiguousarray(a) for a in (idx, codes, meta, cent, w_dec)]
+    _check(_load().kvqo_joint_decode(*(_ptr(a) for a in args), T, H, d, C, r, bits, group, _ptr(out)),
+           "joint_decode")
+    return out
+
+
+# ----------------------------------------------------------------------------
+# attention and merging (NumPy float64)
+# ----------------------------------------------------------------------------
+
+def _widen(a: np.ndarray) -> np.ndarray:
+    if a.dtype == np.uint16:  # bf16 bit patterns
+        return (a.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    return a.astype(np.float64)
+
+
+def attention(q: np.ndarray, k: np.ndarray, v: np.ndarray, scale: Optional[float] = None,
+              rows: Optional[np.ndarray] = None) -> Tuple[np.ndarray, np.ndarray]:
+    """Softmax attention of queries over a (reconstructed) history.
+
+    q [Tq][H][d] (bf16 bits or float), k, v [T][H][d] float32 reconstructions.
+    Logits s_ij = scale * q_i . k_j with scale = 1/sqrt(d) unless given; no
+    mask (the history strictly precedes the current chunk).
+    Returns O [n][H][d] float64 and lse [H][n] float64 (natural log), where n
+    = Tq or len(rows) when only some query rows are evaluated.  An empty
+    history gives O = 0 and lse = -inf.
+    """
+    qf = _widen(q)
+    if rows is not None:
+        qf = qf[rows]
+    kf = k.astype(np.float64)
+    vf = v.astype(np.float64)
+    n, H, d = qf.shape
+    T = kf.shape[0]
+    sc = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    O = np.zeros((n, H, d), np.float64)
+    lse = np.full((H, n), -np.inf, np.float64)
+    if T == 0:
+        return O, lse
+    for h in range(H):
+        s = (qf[:, h, :] @ kf[:, h, :].T) * sc          # [n][T]
+        m = s.max(axis=1, keepdims=True)
+        p = np.exp(s - m)
+        l = p.sum(axis=1, keepdims=True)
+        O[:, h, :] = (p @ vf[:, h, :]) / l
+        lse[h, :] = (m + np.log(l))[:, 0]
+    return O, lse
+
+
+def lse_merge(o_parts: Sequence[np.ndarray], lse_parts: Sequence[np.ndarray]) -> Tuple[np.ndarray, np.ndarray]:
+    """Merge partial attention results over disjoint history parts.
+
+    lse = m + ln sum_b exp(lse_b - m), m = max_b lse_b;
+    O = sum_b exp(lse_b - lse) O_b.  Parts with lse = -inf carry weight 0; if
+    every part is empty the result is O = 0, lse = -inf.
+    o_parts[b] [Tq][H][d], lse_parts[b] [H][Tq].
+    """
+    L = np.stack([np.asarray(l, np.float64) for l in lse_parts])     # [n][H][Tq]
+    Os = np.stack([np.asarray(o, np.float64) for o in o_parts])      # [n][Tq][H][d]
+    m = L.max(axis=0)                                                # [H][Tq]
+    finite = np.isfinite(m)
+    msafe = np.where(finite, m, 0.0)
+    w = np.where(np.isfinite(L), np.exp(L - msafe[None]), 0.0)       # [n][H][Tq]
+    tot = w.sum(axis=0)
+    lse = np.where(finite, msafe + np.log(np.where(finite, tot, 1.0)), -np.inf)
+    wn = np.where(finite[None], w / np.where(finite, tot, 1.0)[None], 0.0)
+    O = np.einsum("nht,nthd->thd", wn, Os)
+    return O, lse
+
+
+# ----------------------------------------------------------------------------
+# storage accounting
+# ----------------------------------------------------------------------------
+
+def stored_bytes_per_token_head(d: int, bits: int, group: int, meta_bytes_per_group: int = 8,
+                                index_bytes: int = 2) -> float:
+    """Bytes stored per d-vector: packed codes + per-group {scale, zero} + index."""
+    return d * bits / 8 + (d // group) * meta_bytes_per_group + index_bytes
+
+
+def bits_per_value(bits: int, group: int, meta_bits_per_group: int) -> float:
+    """Stored bits per cached value for b-bit codes with per-group metadata."""
+    return bits + meta_bits_per_group / group
+
+
+def compression_ratio(bits: int, group: int, meta_bits_per_group: int, base_bits: int = 16) -> float:
+    return base_bits / bits_per_value(bits, group, meta_bits_per_group)
+
+
+def joint_nominal_ratio(channels: int, rank: int, coef_bits: int = 4, base_bits: int = 16) -> float:
+    """Nominal coefficient compression: channels*16 / (rank*coef_bits)."""
+    return channels * base_bits / (rank * coef_bits)
+
+
+def kv_cache_bytes(layers: int, tokens: int, width: int, bits: int = 16) -> float:
+    """Uncompressed K+V storage: 2 * L * T * C * bits / 8 bytes."""
+    return 2 * layers * tokens * width * bits / 8

@@ -1,0 +1,446 @@
+"""Pins for the CPU oracle: each check ties an oracle function to something
+other than itself -- hand-worked examples of the pages' formulas, exact
+rational arithmetic, closed forms, invariants, and library routines."""
+
+import json
+import math
+import os
+from fractions import Fraction
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import oracle as O
+
+GOLDEN = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden")
+
+
+def _golden(name):
+    with open(os.path.join(GOLDEN, name)) as f:
+        return json.load(f)
+
+
+def _bf16(a):
+    """float -> bf16 bits via torch (an implementation independent of the oracle)."""
+    t = torch.from_numpy(np.ascontiguousarray(a, dtype=np.float32))
+    return t.to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+
+
+def _widen(bits):
+    return (bits.astype(np.uint32) << 16).view(np.float32)
+
+
+# ----------------------------------------------------------------------------
+# distance
+# ----------------------------------------------------------------------------
+
+def test_distance_channel_order_golden():
+    for case in _golden("distance_order.json")["cases"]:
+        got = O.distance(np.array(case["x"], np.float32), np.array(case["mu"], np.float32))
+        assert got == np.float32(case["spec"])
+        exact = sum((Fraction(a) - Fraction(b)) ** 2 for a, b in zip(case["x"], case["mu"]))
+        assert float(exact) == case["exact"]
+
+
+def test_distance_within_rounding_bound_of_exact():
+    rng = np.random.default_rng(1)
+    u = 2.0 ** -24
+    for _ in range(300):
+        d = int(rng.integers(1, 130))
+        x = _widen(_bf16(rng.normal(size=d) * rng.uniform(0.1, 10)))
+        mu = _widen(_bf16(rng.normal(size=d) * rng.uniform(0.1, 10)))
+        exact = sum((Fraction(float(a)) - Fraction(float(b))) ** 2 for a, b in zip(x, mu))
+        got = Fraction(O.distance(x, mu))
+        k = d + 2
+        gamma = Fraction(k) * Fraction(u) / (1 - Fraction(k) * Fraction(u))
+        assert abs(got - exact) <= gamma * exact
+
+
+# ----------------------------------------------------------------------------
+# assignment
+# ----------------------------------------------------------------------------
+
+def test_assign_matches_exact_rational_argmin():
+    rng = np.random.default_rng(2)
+    checked = 0
+    for trial in range(40):
+        T, H, d, C = int(rng.integers(1, 64)), int(rng.integers(1, 3)), int(rng.integers(1, 9)), int(rng.integers(1, 9))
+        x = _bf16(rng.normal(size=(T, H, d)))
+        cent = _bf16(rng.normal(size=(H, C, d)))
+        idx = O.assign(x, cent)
+        xf, cf = _widen(x), _widen(cent)
+        for h in range(H):
+            for t in range(T):
+                ds = [sum((Fraction(float(a)) - Fraction(float(b))) ** 2 for a, b in zip(xf[t, h], cf[h, j]))
+                      for j in range(C)]
+                best = min(range(C), key=lambda j: (ds[j], j))
+                others = [ds[j] for j in range(C) if j != best]
+                if others and min(others) - ds[best] <= Fraction(1, 10 ** 5) * (ds[best] + 1):
+                    continue  # near tie: the binary32 specification may legitimately differ
+                assert idx[h, t] == best
+                checked += 1
+    assert checked > 500
+
+
+def test_assign_ties_go_to_lowest_index():
+    # duplicated centres and exactly equidistant centres
+    x = _bf16(np.array([[[0.0, 0.0]], [[1.0, 1.0]]], np.float32))  # T=2, H=1, d=2
+    cent = _bf16(np.array([[[1.0, 0.0], [0.0, 1.0], [1.0, 0.0]]], np.float32))
+    idx = O.assign(x, cent)
+    assert idx.tolist() == [[0, 0]]
+    cent2 = _bf16(np.array([[[5.0, 5.0], [0.0, 1.0], [1.0, 0.0]]], np.float32))
+    assert O.assign(x, cent2).tolist() == [[1, 1]]
+
+
+# ----------------------------------------------------------------------------
+# Eq. 1 quantisation and packing
+# ----------------------------------------------------------------------------
+
+def test_eq1_worked_examples():
+    for g in _golden("eq1_worked_examples.json")["groups"]:
+        s, z, q = O.quant_group(np.array(g["r"], np.float32), g["bits"])
+        assert s == g["s"] and z == g["z"], g
+        assert math.copysign(1.0, z) == math.copysign(1.0, g["z"]), g
+        assert q.tolist() == g["q"], g
+        dec = [O.dequant(int(c), s, z) for c in q]
+        assert dec == g["decoded"], g
+        assert O.pack(q, g["bits"]).tolist() == g["packed"], g
+
+
+def test_quant_error_bound_and_nearest_level():
+    rng = np.random.default_rng(3)
+    for _ in range(400):
+        bits = int(rng.choice([2, 4]))
+        G = int(rng.choice([4, 16, 32, 64]))
+        r = (rng.standard_t(3, size=G) * rng.uniform(1e-3, 50)).astype(np.float32)
+        s, z, q = O.quant_group(r, bits)
+        qmax = (1 << bits) - 1
+        assert q.min() >= 0 and q.max() <= qmax
+        dec = np.array([O.dequant(int(c), s, z) for c in q], np.float64)
+        err = np.abs(dec - r.astype(np.float64))
+        # rounding to the nearest level leaves at most half a step, plus the
+        # binary32 error of forming r*inv, z and (q - z)*s
+        slack = 4 * np.finfo(np.float32).eps * (np.abs(r).max() + s * (qmax + abs(z)))
+        assert np.all(err <= s / 2 + slack)
+        # every code is (one of) the nearest representable level(s)
+        levels = (np.arange(qmax + 1) - z) * np.float64(s)
+        best = np.min(np.abs(levels[None, :] - r.astype(np.float64)[:, None]), axis=1)
+        assert np.all(err <= best + slack)
+        # the group's extremes land on the end codes (generic data)
+        if np.ptp(r) > 0:
+            assert q[np.argmin(r)] == 0 and q[np.argmax(r)] == qmax
+
+
+def test_pack_layout_and_roundtrip():
+    assert O.pack(np.array([0, 1, 2, 3], np.uint8), 2).tolist() == [0xE4]
+    assert O.pack(np.array([3, 10], np.uint8), 4).tolist() == [0xA3]
+    rng = np.random.default_rng(4)
+    for bits in (2, 4):
+        q = rng.integers(0, 1 << bits, size=128).astype(np.uint8)
+        b = O.pack(q, bits)
+        assert b.shape == (128 * bits // 8,)
+        assert np.array_equal(O.unpack(b, 128, bits), q)
+        # independent unpack with numpy bit arithmetic
+        per = 8 // bits
+        manual = np.array([(b[c // per] >> ((c % per) * bits)) & ((1 << bits) - 1) for c in range(128)])
+        assert np.array_equal(manual, q)
+
+
+# ----------------------------------------------------------------------------
+# storage accounting vs figures printed on the pages
+# ----------------------------------------------------------------------------
+
+def test_storage_ratios_printed_on_pages():
+    g = _golden("storage_ratios.json")
+    for row in g["rtn"]:
+        assert round(O.compression_ratio(row["bits"], row["group"], row["meta_bits"]), 2) == row["ratio"]
+    for row in g["bits_per_value"]:
+        assert O.bits_per_value(row["bits"], row["group"], row["meta_bits"]) == row["value"]
+    for row in g["joint_nominal"]:
+        assert O.joint_nominal_ratio(row["heads"] * row["head_dim"], row["rank"]) == row["ratio"]
+    # the joint workload: 12 heads x 128 channels, rank 192 -> 32x nominal
+    assert O.joint_nominal_ratio(1536, 192) == 32
+    # per token-head bytes of the stored format: 128 ch, INT2, group 16:
+    # 32 B codes + 8 groups x 8 B {s, z} + 2 B index
+    assert O.stored_bytes_per_token_head(128, 2, 16) == 98
+
+
+# ----------------------------------------------------------------------------
+# encode / decode
+# ----------------------------------------------------------------------------
+
+def test_identical_tokens_collapse_to_centre():
+    rng = np.random.default_rng(5)
+    H, d, T, C = 2, 64, 40, 4
+    tok = _bf16(rng.normal(size=(H, d)))
+    x = np.broadcast_to(tok[None], (T, H, d)).copy()
+    cent = O.fit(x, C, 3)
+    for h in range(H):
+        for j in range(C):
+            assert np.array_equal(cent[h, j], tok[h])
+    idx, codes, meta = O.encode(x, cent, 2, 32)
+    assert np.all(idx == 0)
+    assert np.all(codes == 0)
+    assert np.all(meta == 0.0)
+    dec = O.decode(idx, codes, meta, cent, 2, 32)
+    assert np.array_equal(dec, np.broadcast_to(_widen(tok)[None], (T, H, d)))
+
+
+def test_zero_centre_reduces_to_plain_groupwise_rtn():
+    rng = np.random.default_rng(6)
+    T, H, d, G = 33, 3, 64, 16
+    x = _bf16(rng.normal(size=(T, H, d)) * 3)
+    cent = np.zeros((H, 1, d), np.uint16)
+    idx, codes, meta = O.encode(x, cent, 4, G)
+    assert np.all(idx == 0)
+    xf = _widen(x)
+    for h in range(H):
+        c2, m2 = O.quant_rows(np.ascontiguousarray(xf[:, h, :]), 4, G)
+        assert np.array_equal(codes[h], c2)
+        assert np.array_equal(meta[h], m2)
+
+
+def test_encode_decode_error_bound_and_residual_form():
+    rng = np.random.default_rng(7)
+    T, H, d, C, G = 200, 2, 64, 8, 16
+    x = _bf16(rng.normal(size=(T, H, d)) * 2)
+    cent = O.fit(x, C, 2)
+    for bits in (2, 4):
+        idx, codes, meta = O.encode(x, cent, bits, G)
+        assert np.array_equal(idx, O.assign(x, cent))
+        dec = O.decode(idx, codes, meta, cent, bits, G)
+        xf = _widen(x).astype(np.float64)
+        s = np.repeat(meta[..., 0], G, axis=2)  # [H][T][d]
+        s = np.transpose(s, (1, 0, 2))
+        err = np.abs(dec - xf)
+        assert np.all(err <= s / 2 + 1e-5 * (np.abs(xf) + 1))
+        # the decoded vector is centre + dequantised residual: removing the
+        # centre leaves a value on the group's quantisation grid
+        cf = _widen(cent).astype(np.float64)
+        mu = np.stack([cf[h][idx[h]] for h in range(H)], axis=1)  # [T][H][d]
+        z = np.transpose(np.repeat(meta[..., 1], G, axis=2), (1, 0, 2))
+        with np.errstate(divide="ignore", invalid="ignore"):
+            lvl = np.where(s > 0, (dec - mu) / s + z, 0.0)
+        assert np.all(np.abs(lvl - np.round(lvl)) < 1e-3)
+        assert np.all((np.round(lvl) >= -1e-9) & (np.round(lvl) <= (1 << bits) - 1))
+
+
+def test_decode_uses_each_stored_field():
+    """Hand-built encoded form: decode = centre + (q - z) s per group."""
+    H, T, d, C, G, bits = 1, 2, 8, 2, 4, 2
+    cent = _bf16(np.array([[[1, 2, 3, 4, 5, 6, 7, 8], [-1, -1, -1, -1, 0.5, 0.5, 0.5, 0.5]]], np.float32))
+    idx = np.array([[1, 0]], np.uint16)
+    q = np.array([[0, 1, 2, 3, 3, 2, 1, 0], [1, 1, 1, 1, 0, 0, 0, 0]], np.uint8)
+    codes = np.stack([O.pack(q[t], bits) for t in range(T)])[None]
+    meta = np.array([[[[0.5, 1.0], [2.0, 0.0]], [[0.25, 2.0], [1.0, -1.0]]]], np.float32)
+    dec = O.decode(idx, codes, meta, cent, bits, G)
+    want_t0 = [-1 + (0 - 1) * 0.5, -1 + 0, -1 + 0.5, -1 + 1.0, 0.5 + 6, 0.5 + 4, 0.5 + 2, 0.5 + 0]
+    want_t1 = [1 + (1 - 2) * 0.25, 2 - 0.25, 3 - 0.25, 4 - 0.25, 5 + 1, 6 + 1, 7 + 1, 8 + 1]
+    assert dec[0, 0].tolist() == want_t0
+    assert dec[1, 0].tolist() == want_t1
+
+
+# ----------------------------------------------------------------------------
+# k-means fitting
+# ----------------------------------------------------------------------------
+
+def test_fit_seeds_from_first_tokens():
+    rng = np.random.default_rng(8)
+    x = rng.normal(size=(50, 2, 16)).astype(np.float32)
+    cent = O.fit(x, 5, 0)
+    for h in range(2):
+        assert np.array_equal(cent[h], _bf16(x[:5, h, :]))
+
+
+def test_fit_recovers_planted_centres_with_exact_update():
+    rng = np.random.default_rng(9)
+    H, d, C, per = 2, 32, 6, 40
+    planted = (rng.integers(-8, 9, size=(H, C, d)) * 4).astype(np.float64)
+    members = []
+    for j in range(C):
+        members.append(planted[:, j, :][None] + rng.normal(0, 0.05, size=(per, H, d)))
+    # first C tokens: one per blob, so the seeds land in distinct blobs
+    first = np.stack([m[0] for m in members])
+    rest = np.concatenate([m[1:] for m in members])
+    order = rng.permutation(rest.shape[0])
+    x = _bf16(np.concatenate([first, rest[order]]).astype(np.float32))
+    blob = np.concatenate([np.arange(C), np.repeat(np.arange(C), per - 1)[order]])
+    cent = O.fit(x, C, 1)
+    xf = _widen(x).astype(np.float64)
+    for h in range(H):
+        for j in range(C):
+            mean = xf[blob == j, h, :].mean(axis=0)
+            assert np.array_equal(cent[h, j], _bf16(mean.astype(np.float32)))
+
+
+def test_fit_inertia_non_increasing_up_to_centre_rounding():
+    rng = np.random.default_rng(10)
+    x = _bf16(rng.normal(size=(400, 2, 32)))
+    iters = 5
+    cent, inertia = O.fit(x, 12, iters, return_inertia=True)
+    xmax = float(np.abs(_widen(x)).max())
+    # rounding a mean to bf16 moves it by <= 2^-8 relative per channel; by the
+    # parallel-axis identity that can add at most sum_j n_j |mu_j - mean_j|^2
+    bound = 400 * 32 * (2.0 ** -8 * xmax) ** 2
+    for h in range(2):
+        for i in range(iters):
+            assert inertia[h, i + 1] <= inertia[h, i] + bound
+        assert inertia[h, -1] < inertia[h, 0]
+
+
+def test_fit_c_equals_t_each_point_is_its_centre():
+    rng = np.random.default_rng(11)
+    T = 24
+    x = _bf16(rng.normal(size=(T, 1, 8)))
+    cent, inertia = O.fit(x, T, 3, return_inertia=True)
+    assert np.array_equal(cent[0], x[:, 0, :])
+    assert inertia[0, -1] == 0.0
+
+
+def test_fit_empty_cluster_keeps_centre():
+    # tokens 0 and 1 identical -> seeds 0 and 1 coincide and, by the
+    # lowest-index tie rule, centre 1 receives no token in the first round
+    x = np.array([[[1.0, 1.0]], [[1.0, 1.0]], [[5.0, 5.0]], [[1.5, 1.0]], [[5.5, 5.0]]], np.float32)
+    cent = O.fit(x, 3, 1)
+    assert _widen(cent[0, 1]).tolist() == [1.0, 1.0]          # empty: kept
+    assert _widen(cent[0, 0]).tolist() == [1.1640625, 1.0]    # bf16(3.5/3)
+    assert _widen(cent[0, 2]).tolist() == [5.25, 5.0]
+    # second round: tokens 0 and 1 now sit exactly on centre 1
+    cent = O.fit(x, 3, 2)
+    assert _widen(cent[0, 0]).tolist() == [1.5, 1.0]
+    assert _widen(cent[0, 1]).tolist() == [1.0, 1.0]
+    assert _widen(cent[0, 2]).tolist() == [5.25, 5.0]
+
+
+# ----------------------------------------------------------------------------
+# joint head-channel path
+# ----------------------------------------------------------------------------
+
+def test_joint_identity_encoder_is_channel_quantisation():
+    rng = np.random.default_rng(12)
+    T, H, d, C, r, G = 20, 3, 64, 4, 96, 32
+    x = _bf16(rng.normal(size=(T, H, d)))
+    cent = O.fit(x, C, 1)
+    w = np.zeros((H * d, r), np.float32)
+    w[np.arange(r), np.arange(r)] = 1.0
+    idx, codes, meta, coef = O.joint_encode(x, cent, _bf16(w), 4, G)
+    assert np.array_equal(idx, O.assign(x, cent))
+    xf, cf = _widen(x), _widen(cent)
+    res = np.stack([xf[:, h, :] - cf[h][idx[h]] for h in range(H)], axis=1).reshape(T, H * d)
+    want = _widen(_bf16(res[:, :r]))
+    assert np.array_equal(coef, want)
+    c2, m2 = O.quant_rows(coef, 4, G)
+    assert np.array_equal(codes, c2) and np.array_equal(meta, m2)
+
+
+def test_joint_decode_is_projection_when_coefficients_are_on_grid():
+    rng = np.random.default_rng(13)
+    T, H, d, C, r, G = 10, 2, 64, 3, 64, 32
+    cent = _bf16(rng.normal(size=(H, C, d)))
+    idx = rng.integers(0, C, size=(H, T)).astype(np.uint16)
+    coef = rng.integers(-7, 8, size=(T, r)).astype(np.float32)
+    for t in range(T):  # force a full 15-step span in every group -> s = 1
+        for g in range(r // G):
+            coef[t, g * G] = -7.0
+            coef[t, g * G + 1] = 8.0
+    codes, meta = O.quant_rows(coef, 4, G)
+    assert np.all(meta[..., 0] == 1.0)
+    rng2 = np.random.default_rng(14)
+    q_, _ = np.linalg.qr(rng2.normal(size=(H * d, r)))
+    w_dec = _bf16(q_.T)
+    out = O.joint_decode(idx, codes, meta, cent, w_dec, 4, G)
+    proj = coef.astype(np.float64) @ _widen(w_dec).astype(np.float64)  # [T][H*d]
+    cf = _widen(cent).astype(np.float64)
+    want = np.stack([cf[h][idx[h]] for h in range(H)], axis=1) + proj.reshape(T, H, d)
+    assert np.max(np.abs(out - want)) < 1e-5 * (np.abs(want).max() + 1)
+
+
+# ----------------------------------------------------------------------------
+# attention and log-sum-exp merging
+# ----------------------------------------------------------------------------
+
+def test_attention_single_key_returns_its_value():
+    rng = np.random.default_rng(15)
+    q = _bf16(rng.normal(size=(5, 2, 64)))
+    k = rng.normal(size=(1, 2, 64)).astype(np.float32)
+    v = rng.normal(size=(1, 2, 64)).astype(np.float32)
+    o, lse = O.attention(q, k, v)
+    qf = _widen(q).astype(np.float64)
+    for h in range(2):
+        assert np.allclose(o[:, h, :], v[0, h][None], rtol=0, atol=1e-15)
+        want = qf[:, h, :] @ k[0, h].astype(np.float64) / 8.0
+        assert np.allclose(lse[h], want, rtol=1e-14, atol=1e-14)
+
+
+def test_attention_identical_keys_mean_value_and_log_n():
+    rng = np.random.default_rng(16)
+    n = 7
+    q = _bf16(rng.normal(size=(3, 1, 64)))
+    k = np.broadcast_to(rng.normal(size=(1, 1, 64)).astype(np.float32), (n, 1, 64)).copy()
+    v = rng.normal(size=(n, 1, 64)).astype(np.float32)
+    o, lse = O.attention(q, k, v)
+    s = _widen(q)[:, 0, :].astype(np.float64) @ k[0, 0].astype(np.float64) / 8.0
+    assert np.allclose(o[:, 0, :], v[:, 0, :].astype(np.float64).mean(axis=0)[None], atol=1e-14)
+    assert np.allclose(lse[0], s + math.log(n), atol=1e-13)
+
+
+def test_attention_two_keys_logistic():
+    rng = np.random.default_rng(17)
+    q = _bf16(rng.normal(size=(4, 1, 64)))
+    k = rng.normal(size=(2, 1, 64)).astype(np.float32)
+    v = rng.normal(size=(2, 1, 64)).astype(np.float32)
+    o, lse = O.attention(q, k, v)
+    qf = _widen(q).astype(np.float64)
+    for i in range(4):
+        s1 = float(qf[i, 0] @ k[0, 0].astype(np.float64)) / 8.0
+        s2 = float(qf[i, 0] @ k[1, 0].astype(np.float64)) / 8.0
+        w1 = 1.0 / (1.0 + math.exp(s2 - s1))
+        want = w1 * v[0, 0].astype(np.float64) + (1 - w1) * v[1, 0].astype(np.float64)
+        assert np.allclose(o[i, 0], want, atol=1e-14)
+        assert abs(lse[0, i] - (max(s1, s2) + math.log1p(math.exp(-abs(s1 - s2))))) < 1e-13
+
+
+def test_attention_matches_library_sdpa_and_logsumexp():
+    from scipy.special import logsumexp
+
+    rng = np.random.default_rng(18)
+    Tq, T, H, d = 37, 300, 3, 64
+    q = _bf16(rng.normal(size=(Tq, H, d)))
+    k = rng.normal(size=(T, H, d)).astype(np.float32)
+    v = rng.normal(size=(T, H, d)).astype(np.float32)
+    o, lse = O.attention(q, k, v)
+    qt = torch.from_numpy(_widen(q).astype(np.float64)).permute(1, 0, 2)
+    kt = torch.from_numpy(k.astype(np.float64)).permute(1, 0, 2)
+    vt = torch.from_numpy(v.astype(np.float64)).permute(1, 0, 2)
+    ref = torch.nn.functional.scaled_dot_product_attention(qt, kt, vt).permute(1, 0, 2).numpy()
+    assert np.max(np.abs(o - ref)) < 1e-12
+    s = np.einsum("qhd,khd->hqk", _widen(q).astype(np.float64), k.astype(np.float64)) / math.sqrt(d)
+    assert np.max(np.abs(lse - logsumexp(s, axis=2))) < 1e-12
+
+
+def test_merge_of_split_history_equals_unsplit():
+    rng = np.random.default_rng(19)
+    Tq, T, H, d = 20, 333, 2, 64
+    q = _bf16(rng.normal(size=(Tq, H, d)))
+    k = (rng.normal(size=(T, H, d)) * 2).astype(np.float32)
+    v = rng.normal(size=(T, H, d)).astype(np.float32)
+    o_full, lse_full = O.attention(q, k, v)
+    cuts = [0, 1, 100, 101, 250, T]
+    parts = [O.attention(q, k[a:b], v[a:b]) for a, b in zip(cuts[:-1], cuts[1:])]
+    o, lse = O.lse_merge([p[0] for p in parts], [p[1] for p in parts])
+    assert np.max(np.abs(o - o_full)) < 1e-12
+    assert np.max(np.abs(lse - lse_full)) < 1e-12
+
+
+def test_merge_with_empty_parts():
+    rng = np.random.default_rng(20)
+    o1 = rng.normal(size=(5, 2, 8))
+    l1 = rng.normal(size=(2, 5))
+    o_empty, l_empty = O.attention(_bf16(rng.normal(size=(5, 2, 8))), np.zeros((0, 2, 8), np.float32),
+                                   np.zeros((0, 2, 8), np.float32))
+    assert np.all(l_empty == -np.inf) and np.all(o_empty == 0)
+    o, l = O.lse_merge([o1, o_empty], [l1, l_empty])
+    assert np.allclose(o, o1, atol=1e-15) and np.allclose(l, l1, atol=1e-15)
+    o, l = O.lse_merge([o_empty, o_empty], [l_empty, l_empty])
+    assert np.all(l == -np.inf) and np.all(o == 0)

@@ -1,0 +1,228 @@
+/*
+ * kvq.h -- C ABI of libkvq: centroid-residual low-bit compression of an
+ * autoregressive video model's historical KV cache, and attention of the
+ * current chunk's queries over that compressed history (NVIDIA B200, sm_100a).
+ *
+ * The method, as the pages state it:
+ *  - QVG-style codec: every key/value token of a head is assigned to its
+ *    nearest centroid (k-means fitted online per head, per cache block,
+ *    separately for K and V) and only the residual is quantised to low bit
+ *    width (QuantWM: Temporally Consistent 2-Bit KV Cache Quantization for
+ *    Video World Models, Sec. 4.1; CORAL-KV, Sec. 2; TempoKV, Sec. 1 and
+ *    Sec. 3.3 Eq. 2; NanoKV page, Table 4).
+ *  - asymmetric affine b-bit quantisation per channel group (TempoKV, Sec. 3.1,
+ *    Eq. 1), packed storage (NanoKV page, Table 4; QuantWM, Fig. 9).
+ *  - optional joint head-channel linear encoder/decoder of the residual with
+ *    INT4 coefficients, centres added back after decoding (NanoKV page,
+ *    abstract, Fig. 4(a,b)).
+ *  - attention over the compressed history with the reconstruction done on
+ *    demand, and log-sum-exp merging of partial results (NanoKV page,
+ *    Fig. 4(a,d); QuantWM, Fig. 9).
+ *
+ * Conventions for every call:
+ *  - All tensor pointers are DEVICE pointers owned by the caller; the library
+ *    allocates no device memory and keeps no state across calls apart from a
+ *    per-device status word (see kvq_last_device_status).  Pointers must be
+ *    16-byte aligned unless stated otherwise (KVQ_ERR_ALIGNMENT).
+ *  - Calls are asynchronous on `stream` (NULL = the legacy default stream).
+ *  - Arguments are validated on the host before anything is launched; a
+ *    rejected call launches nothing and returns the error.  No call aborts
+ *    or throws.  Launch failures return KVQ_ERR_CUDA.
+ *  - bf16 values are stored as raw 16-bit patterns (same bits as
+ *    __nv_bfloat16); float is IEEE binary32.
+ *  - Layouts (T = history tokens, H = heads, d = head dim, C = centroids,
+ *    b = bits, G = group size, r = joint rank, Tq = query tokens):
+ *      history   x      [T][H][d]        (token t = frame * S + position)
+ *      centroids        [H][C][d]        bf16
+ *      idx              [H][T]           uint16
+ *      codes (per-head) [H][T][d*b/8]    uint8, code of channel c of a byte
+ *                                         holds bits (c % (8/b)) * b ..; low
+ *                                         bits first
+ *      meta  (per-head) [H][T][d/G][2]   float {scale s, zero z}
+ *      codes (joint)    [T][r*b/8]       meta (joint) [T][r/G][2]
+ *      queries q        [Tq][H][d]       bf16;  output o [Tq][H][d]
+ *      lse              [H][Tq]          float, natural logarithm
+ */
+#ifndef KVQ_H_
+#define KVQ_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define KVQ_API __attribute__((visibility("default")))
+#else
+#define KVQ_API
+#endif
+
+struct CUstream_st;
+/* Same type as cudaStream_t. */
+typedef struct CUstream_st *kvq_stream_t;
+
+typedef enum {
+    KVQ_OK = 0,
+    KVQ_ERR_INVALID_ARG = 1,    /* null pointer, bad size or shape */
+    KVQ_ERR_UNSUPPORTED = 2,    /* a valid request this build does not serve */
+    KVQ_ERR_ALIGNMENT = 3,      /* a pointer is not 16-byte aligned */
+    KVQ_ERR_WORKSPACE = 4,      /* workspace missing or smaller than required */
+    KVQ_ERR_CUDA = 5,           /* a CUDA runtime call or launch failed */
+    KVQ_ERR_DEVICE_TIMEOUT = 6  /* a kernel gave up a bounded wait (device status) */
+} kvq_status;
+
+typedef enum { KVQ_F32 = 0, KVQ_BF16 = 1 } kvq_dtype;
+
+typedef enum {
+    KVQ_OP_FIT = 0,
+    KVQ_OP_ENCODE = 1,
+    KVQ_OP_DECODE = 2,
+    KVQ_OP_ATTENTION = 3
+} kvq_op;
+
+/* Codec of one K or V branch.  K and V are described separately, which is
+ * how mixed bit widths (k4v2 etc.; TempoKV, Sec. 4.2, Table 4) are set. */
+typedef struct {
+    int32_t num_heads;     /* H >= 1 */
+    int32_t head_dim;      /* d: 64 or 128 */
+    int32_t num_centroids; /* C: 1 .. 65536 */
+    int32_t bits;          /* b: 2 or 4 */
+    int32_t group_size;    /* G: multiple of 8 dividing d (per-head) or r (joint) */
+    int32_t joint_rank;    /* 0: per-head codec; r > 0: joint head-channel code */
+} kvq_codec_desc;
+
+/* A compressed K or V history as produced by kvq_encode (read-only view). */
+typedef struct {
+    kvq_codec_desc desc;
+    int64_t num_tokens;     /* T */
+    const void *centroids;  /* [H][C][d] bf16 */
+    const uint16_t *idx;    /* [H][T] */
+    const uint8_t *codes;   /* per-head [H][T][d*b/8]; joint [T][r*b/8] */
+    const float *meta;      /* per-head [H][T][d/G][2]; joint [T][r/G][2] */
+    const void *w_dec;      /* joint only: decoder [r][H*d] bf16; else NULL */
+} kvq_compressed_view;
+
+/* Human-readable name of a status code (static string, never NULL). */
+KVQ_API const char *kvq_status_string(kvq_status s);
+
+/* Byte sizes of the three encoded arrays for T tokens of this codec (host
+ * only; no device work).  Any output pointer may be NULL. */
+KVQ_API kvq_status kvq_encoded_sizes(const kvq_codec_desc *desc, int64_t num_tokens, size_t *idx_bytes,
+                             size_t *code_bytes, size_t *meta_bytes);
+
+/* Device workspace (bytes) an operation needs for these sizes; 0 means the
+ * call accepts workspace = NULL.  Tq is used by KVQ_OP_ATTENTION only. */
+KVQ_API kvq_status kvq_workspace_size(kvq_op op, const kvq_codec_desc *desc, int64_t num_tokens,
+                              int64_t num_queries, size_t *bytes);
+
+/*
+ * Fit per-head centroids to one K or V history (k-means; CORAL-KV, Sec. 2:
+ * per-head codebooks fitted online for each cache block; NanoKV page,
+ * Table 4: QVG uses 256 centres and two k-means iterations, BF16 centres).
+ *   x            [T][H][d] float or bf16 (x_dtype); T >= C
+ *   iters        >= 0 rounds of {assign every token to its nearest centre;
+ *                move each centre to the mean of its tokens}
+ *   centroids_out [H][C][d] bf16.  Seeds are the first C tokens.  A centre
+ *                 that receives no token keeps its value.  Means are summed
+ *                 in binary64 and rounded to binary32, then to bf16.
+ *   workspace    >= kvq_workspace_size(KVQ_OP_FIT, ...) bytes.
+ */
+KVQ_API kvq_status kvq_fit_centroids(const kvq_codec_desc *desc, const void *x, kvq_dtype x_dtype, int64_t num_tokens,
+                             int32_t iters, void *centroids_out, void *workspace, size_t workspace_bytes,
+                             kvq_stream_t stream);
+
+/*
+ * Encode one K or V history against fitted centroids.
+ * Per-head codec (desc->joint_rank == 0, w_enc == NULL):
+ *   idx[h][t]  = nearest centre (squared Euclidean distance evaluated in
+ *                binary32 channel by channel without FMA; ties go to the
+ *                lowest index) -- QuantWM, Sec. 4.1;
+ *   residual   r = x - mu[idx] (binary32; TempoKV, Sec. 3.3, Eq. 2);
+ *   per group of G channels: s = (max - min)/(2^b - 1), z = rint(-min/s),
+ *   q = clamp(rint(r/s) + z, 0, 2^b - 1) with 1/s formed once per group
+ *   (TempoKV, Sec. 3.1, Eq. 1); a zero-range (or underflowing) group stores
+ *   s = |min|, z = -sign(min), q = 0.  Codes packed low bits first.
+ * Joint codec (desc->joint_rank = r > 0, w_enc = [H*d][r] bf16):
+ *   idx as above per head; the residual of all H*d channels of a token is
+ *   rounded to bf16 and projected, c = R W_enc (tensor-core GEMM, binary32
+ *   accumulation), and the r coefficients are quantised per group of G as
+ *   above (NanoKV page, Fig. 4(b)).
+ * Outputs: idx [H][T], codes, meta as in the layout table.  No workspace is
+ * needed by the per-head codec; the joint codec needs
+ * kvq_workspace_size(KVQ_OP_ENCODE, ...) bytes.
+ */
+KVQ_API kvq_status kvq_encode(const kvq_codec_desc *desc, const void *x, kvq_dtype x_dtype, int64_t num_tokens,
+                      const void *centroids, const void *w_enc, uint16_t *idx, uint8_t *codes, float *meta,
+                      void *workspace, size_t workspace_bytes, kvq_stream_t stream);
+
+/*
+ * Joint codec only: the binary32 coefficient matrix c = R W_enc [T][r] that
+ * kvq_encode quantises, and idx [H][T].  Lets a caller quantise the same
+ * coefficients independently.  Workspace as for kvq_encode.
+ */
+KVQ_API kvq_status kvq_joint_coefficients(const kvq_codec_desc *desc, const void *x, kvq_dtype x_dtype,
+                                  int64_t num_tokens, const void *centroids, const void *w_enc, uint16_t *idx,
+                                  float *coef_out, void *workspace, size_t workspace_bytes,
+                                  kvq_stream_t stream);
+
+/*
+ * Reconstruct a history from its compressed view (NanoKV page, Fig. 4(b):
+ * the decoder reconstructs the residual and adds back the centres).
+ * Per-head: x^ = mu[idx] + (q - z) * s, each step rounded to binary32
+ * (subtract, multiply, add; no FMA), then stored as float or bf16 (RNE).
+ * Joint: c^ = (q - z) s; R^ = c^ W_dec (tensor-core GEMM); x^ = mu[idx] + R^.
+ *   x_out [T][H][d] in out_dtype.  The joint decoder needs
+ *   kvq_workspace_size(KVQ_OP_DECODE, ...) bytes of workspace.
+ */
+KVQ_API kvq_status kvq_decode(const kvq_compressed_view *view, void *x_out, kvq_dtype out_dtype, void *workspace,
+                      size_t workspace_bytes, kvq_stream_t stream);
+
+/*
+ * Attention of the current chunk's queries over history tokens
+ * [t_begin, t_end) of a compressed K and V (per-head codec), with the
+ * reconstruction fused into the kernel (NanoKV page, Fig. 4(a); QuantWM,
+ * Fig. 9: on-demand reconstruction):
+ *   s_ij = softmax_scale * q_i . k^_j   (softmax_scale <= 0 selects 1/sqrt(d))
+ *   o_i  = sum_j softmax(s_i)_j v^_j,  lse_i = ln sum_j exp(s_ij)
+ * k^ and v^ are rounded to bf16 for the tensor cores; logits, softmax and the
+ * output accumulate in binary32.  No mask: the history precedes the chunk.
+ *   q     [Tq][H][d] bf16;  o_out [Tq][H][d] (o_dtype);  lse_out [H][Tq]
+ * k and v must have the same H, d and num_tokens; their bits, group sizes and
+ * centroid counts may differ.  An empty range gives o = 0, lse = -inf.
+ * Workspace: none (pass NULL / 0).
+ */
+KVQ_API kvq_status kvq_attention_lse(const void *q, int64_t num_queries, const kvq_compressed_view *k,
+                             const kvq_compressed_view *v, int64_t t_begin, int64_t t_end, float softmax_scale,
+                             void *o_out, kvq_dtype o_dtype, float *lse_out, void *workspace,
+                             size_t workspace_bytes, kvq_stream_t stream);
+
+/*
+ * Merge n partial attention results over disjoint history parts by their
+ * log-sum-exp (NanoKV page, Fig. 4(d)):
+ *   m = max_b lse_b;  lse = m + ln sum_b exp(lse_b - m);
+ *   o = sum_b exp(lse_b - lse) o_b;  parts with lse_b = -inf weigh 0; if all
+ *   parts are empty, o = 0 and lse = -inf.
+ *   o_parts / lse_parts: HOST arrays of n (1..64) DEVICE pointers to
+ *   o_b [Tq][H][d] float and lse_b [H][Tq] float.
+ *   o_out [Tq][H][d] (o_dtype), lse_out [H][Tq] float.  The outputs must not
+ *   overlap any part.
+ */
+KVQ_API kvq_status kvq_lse_merge(int32_t n_parts, const float *const *o_parts, const float *const *lse_parts,
+                         int64_t num_queries, int32_t num_heads, int32_t head_dim, void *o_out,
+                         kvq_dtype o_dtype, float *lse_out, kvq_stream_t stream);
+
+/*
+ * Synchronise `stream`, then read and clear this device's status word.
+ * Returns KVQ_ERR_DEVICE_TIMEOUT if any kernel since the last read gave up a
+ * bounded wait (its outputs are then undefined), KVQ_ERR_CUDA if the stream
+ * reports an error, else KVQ_OK.
+ */
+KVQ_API kvq_status kvq_last_device_status(kvq_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* KVQ_H_ */

@@ -1,0 +1,439 @@
+// kvq_lib.cu -- the C ABI of libkvq (declared in include/kvq.h): argument
+// validation, workspace accounting and kernel launches.  Built as a single
+// translation unit for sm_100a.
+#include <stdint.h>
+#include <string.h>
+
+#include "attention.cuh"
+#include "codec.cuh"
+#include "common.cuh"
+#include "merge.cuh"
+
+using namespace kvq;
+
+namespace {
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
+
+size_t round_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+bool supported_dim(int d) { return d == 64 || d == 128; }
+
+// Shared checks of a per-head codec description.
+kvq_status check_desc(const kvq_codec_desc *d, bool allow_joint)
+{
+    if (!d)
+        return KVQ_ERR_INVALID_ARG;
+    if (d->num_heads < 1 || d->num_centroids < 1 || d->num_centroids > 65536)
+        return KVQ_ERR_INVALID_ARG;
+    if (!supported_dim(d->head_dim))
+        return KVQ_ERR_UNSUPPORTED;
+    if (d->bits != 2 && d->bits != 4)
+        return KVQ_ERR_UNSUPPORTED;
+    if (d->joint_rank < 0)
+        return KVQ_ERR_INVALID_ARG;
+    if (d->joint_rank > 0 && !allow_joint)
+        return KVQ_ERR_UNSUPPORTED;
+    const int span = d->joint_rank > 0 ? d->joint_rank : d->head_dim;
+    if (d->group_size < 8 || d->group_size % 8 != 0 || span % d->group_size != 0)
+        return KVQ_ERR_INVALID_ARG;
+    if (d->joint_rank == 0 && d->group_size != 16 && d->group_size != 32 && d->group_size != 64)
+        return KVQ_ERR_UNSUPPORTED;
+    return KVQ_OK;
+}
+
+kvq_status launch_status()
+{
+    return cudaGetLastError() == cudaSuccess ? KVQ_OK : KVQ_ERR_CUDA;
+}
+
+// ---------------------------------------------------------------------------
+// per-head encode dispatch
+// ---------------------------------------------------------------------------
+template <int D, int BITS>
+kvq_status launch_encode_direct_g(const EncodeArgs &a, cudaStream_t s)
+{
+    const dim3 grid((unsigned)ceil_div(a.T, kDirectTokens), (unsigned)a.H);
+    switch (a.G) {
+    case 16: encode_direct_kernel<D, BITS, 16><<<grid, kDirectTokens, 0, s>>>(a); break;
+    case 32: encode_direct_kernel<D, BITS, 32><<<grid, kDirectTokens, 0, s>>>(a); break;
+    case 64: encode_direct_kernel<D, BITS, 64><<<grid, kDirectTokens, 0, s>>>(a); break;
+    default: return KVQ_ERR_UNSUPPORTED;
+    }
+    return launch_status();
+}
+
+kvq_status launch_encode_direct(int D, const EncodeArgs &a, cudaStream_t s)
+{
+    if (a.T == 0)
+        return KVQ_OK;
+    if (D == 128)
+        return a.bits == 2 ? launch_encode_direct_g<128, 2>(a, s) : launch_encode_direct_g<128, 4>(a, s);
+    return a.bits == 2 ? launch_encode_direct_g<64, 2>(a, s) : launch_encode_direct_g<64, 4>(a, s);
+}
+
+size_t fit_workspace(const kvq_codec_desc *d, int64_t T)
+{
+    const size_t idx_b = round_up((size_t)d->num_heads * (size_t)T * 2, 256);
+    const size_t cnt_b = round_up((size_t)d->num_heads * d->num_centroids * 4, 256);
+    const size_t sum_b = (size_t)d->num_heads * d->num_centroids * d->head_dim * 8;
+    return idx_b + cnt_b + sum_b;
+}
+
+kvq_status check_view(const kvq_compressed_view *v)
+{
+    if (!v)
+        return KVQ_ERR_INVALID_ARG;
+    kvq_status st = check_desc(&v->desc, true);
+    if (st != KVQ_OK)
+        return st;
+    if (v->num_tokens < 0)
+        return KVQ_ERR_INVALID_ARG;
+    if (v->num_tokens > 0 && (!v->centroids || !v->idx || !v->codes || !v->meta))
+        return KVQ_ERR_INVALID_ARG;
+    if (!aligned16(v->centroids) || !aligned16(v->codes) || !aligned16(v->meta) ||
+        (reinterpret_cast<uintptr_t>(v->idx) & 1u))
+        return KVQ_ERR_ALIGNMENT;
+    return KVQ_OK;
+}
+
+CodecView to_codec_view(const kvq_compressed_view *v)
+{
+    CodecView cv;
+    cv.cent = static_cast<const uint16_t *>(v->centroids);
+    cv.idx = v->idx;
+    cv.codes = v->codes;
+    cv.meta = v->meta;
+    cv.T = v->num_tokens;
+    cv.C = v->desc.num_centroids;
+    cv.bits = v->desc.bits;
+    cv.G = v->desc.group_size;
+    return cv;
+}
+
+template <int D>
+kvq_status launch_attention(const AttnArgs &a, cudaStream_t s)
+{
+    using L = AttnSmem<D>;
+    // the dynamic shared-memory opt-in is a per-device function attribute
+    static bool configured[64] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64)
+        return KVQ_ERR_CUDA;
+    if (!configured[dev]) {
+        if (cudaFuncSetAttribute(attention_lse_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)L::kLaunchBytes) != cudaSuccess)
+            return KVQ_ERR_CUDA;
+        configured[dev] = true;
+    }
+    const dim3 grid((unsigned)ceil_div(a.Tq, kAttnRows), (unsigned)a.H);
+    attention_lse_kernel<D><<<grid, kAttnThreads, L::kLaunchBytes, s>>>(a);
+    return launch_status();
+}
+
+}  // namespace
+
+extern "C" {
+
+const char *kvq_status_string(kvq_status s)
+{
+    switch (s) {
+    case KVQ_OK: return "KVQ_OK";
+    case KVQ_ERR_INVALID_ARG: return "KVQ_ERR_INVALID_ARG";
+    case KVQ_ERR_UNSUPPORTED: return "KVQ_ERR_UNSUPPORTED";
+    case KVQ_ERR_ALIGNMENT: return "KVQ_ERR_ALIGNMENT";
+    case KVQ_ERR_WORKSPACE: return "KVQ_ERR_WORKSPACE";
+    case KVQ_ERR_CUDA: return "KVQ_ERR_CUDA";
+    case KVQ_ERR_DEVICE_TIMEOUT: return "KVQ_ERR_DEVICE_TIMEOUT";
+    }
+    return "KVQ_ERR_UNKNOWN";
+}
+
+kvq_status kvq_encoded_sizes(const kvq_codec_desc *desc, int64_t T, size_t *idx_bytes, size_t *code_bytes,
+                             size_t *meta_bytes)
+{
+    kvq_status st = check_desc(desc, true);
+    if (st != KVQ_OK)
+        return st;
+    if (T < 0)
+        return KVQ_ERR_INVALID_ARG;
+    const size_t H = (size_t)desc->num_heads, d = (size_t)desc->head_dim;
+    size_t ib = H * (size_t)T * 2, cb, mb;
+    if (desc->joint_rank > 0) {
+        const size_t r = (size_t)desc->joint_rank;
+        cb = (size_t)T * r * desc->bits / 8;
+        mb = (size_t)T * (r / desc->group_size) * 8;
+    } else {
+        cb = H * (size_t)T * d * desc->bits / 8;
+        mb = H * (size_t)T * (d / desc->group_size) * 8;
+    }
+    if (idx_bytes) *idx_bytes = ib;
+    if (code_bytes) *code_bytes = cb;
+    if (meta_bytes) *meta_bytes = mb;
+    return KVQ_OK;
+}
+
+kvq_status kvq_workspace_size(kvq_op op, const kvq_codec_desc *desc, int64_t T, int64_t Tq, size_t *bytes)
+{
+    if (!bytes)
+        return KVQ_ERR_INVALID_ARG;
+    kvq_status st = check_desc(desc, true);
+    if (st != KVQ_OK)
+        return st;
+    if (T < 0 || Tq < 0)
+        return KVQ_ERR_INVALID_ARG;
+    switch (op) {
+    case KVQ_OP_FIT: *bytes = fit_workspace(desc, T); return KVQ_OK;
+    case KVQ_OP_ENCODE:
+    case KVQ_OP_DECODE:
+        *bytes = 0;
+        return desc->joint_rank > 0 ? KVQ_ERR_UNSUPPORTED : KVQ_OK;
+    case KVQ_OP_ATTENTION: *bytes = 0; return KVQ_OK;
+    }
+    return KVQ_ERR_INVALID_ARG;
+}
+
+kvq_status kvq_fit_centroids(const kvq_codec_desc *desc, const void *x, kvq_dtype x_dtype, int64_t T, int32_t iters,
+                             void *centroids_out, void *workspace, size_t workspace_bytes, kvq_stream_t stream)
+{
+    kvq_status st = check_desc(desc, true);
+    if (st != KVQ_OK)
+        return st;
+    if (desc->joint_rank > 0)
+        return KVQ_ERR_INVALID_ARG;  // centres are per head; fit with joint_rank = 0
+    if (!x || !centroids_out || iters < 0 || T < desc->num_centroids || (x_dtype != KVQ_F32 && x_dtype != KVQ_BF16))
+        return KVQ_ERR_INVALID_ARG;
+    if (!aligned16(x) || !aligned16(centroids_out) || !aligned16(workspace))
+        return KVQ_ERR_ALIGNMENT;
+    const size_t need = fit_workspace(desc, T);
+    if (!workspace || workspace_bytes < need)
+        return KVQ_ERR_WORKSPACE;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    const int H = desc->num_heads, D = desc->head_dim, C = desc->num_centroids;
+    uint8_t *ws = static_cast<uint8_t *>(workspace);
+    FitArgs f;
+    f.x = x;
+    f.x_bf16 = x_dtype == KVQ_BF16;
+    f.T = T;
+    f.H = H;
+    f.D = D;
+    f.C = C;
+    f.cent = static_cast<uint16_t *>(centroids_out);
+    f.idx = reinterpret_cast<uint16_t *>(ws);
+    const size_t idx_b = round_up((size_t)H * (size_t)T * 2, 256);
+    const size_t cnt_b = round_up((size_t)H * C * 4, 256);
+    f.counts = reinterpret_cast<unsigned int *>(ws + idx_b);
+    f.sums = reinterpret_cast<double *>(ws + idx_b + cnt_b);
+
+    const int64_t n_cent = (int64_t)H * C * D;
+    fit_seed_kernel<<<(unsigned)ceil_div(n_cent, 256), 256, 0, s>>>(f);
+    if ((st = launch_status()) != KVQ_OK)
+        return st;
+    EncodeArgs e;
+    memset(&e, 0, sizeof e);
+    e.x = x;
+    e.x_bf16 = f.x_bf16;
+    e.T = T;
+    e.H = H;
+    e.C = C;
+    e.bits = 2;
+    e.G = 16;
+    e.cent = f.cent;
+    e.idx = reinterpret_cast<uint16_t *>(ws);
+    e.assign_only = 1;
+    const int64_t n_units = T * H * (D / 8);
+    for (int it = 0; it < iters; ++it) {
+        if ((st = launch_encode_direct(D, e, s)) != KVQ_OK)
+            return st;
+        if (cudaMemsetAsync(ws + idx_b, 0, cnt_b + (size_t)H * C * D * 8, s) != cudaSuccess)
+            return KVQ_ERR_CUDA;
+        fit_accumulate_kernel<<<(unsigned)ceil_div(n_units, 256), 256, 0, s>>>(f);
+        if ((st = launch_status()) != KVQ_OK)
+            return st;
+        fit_update_kernel<<<(unsigned)ceil_div(n_cent, 256), 256, 0, s>>>(f);
+        if ((st = launch_status()) != KVQ_OK)
+            return st;
+    }
+    return KVQ_OK;
+}
+
+kvq_status kvq_encode(const kvq_codec_desc *desc, const void *x, kvq_dtype x_dtype, int64_t T,
+                      const void *centroids, const void *w_enc, uint16_t *idx, uint8_t *codes, float *meta,
+                      void *workspace, size_t workspace_bytes, kvq_stream_t stream)
+{
+    (void)workspace;
+    (void)workspace_bytes;
+    kvq_status st = check_desc(desc, true);
+    if (st != KVQ_OK)
+        return st;
+    if (desc->joint_rank > 0 || w_enc)
+        return KVQ_ERR_UNSUPPORTED;
+    if (T < 0 || (x_dtype != KVQ_F32 && x_dtype != KVQ_BF16))
+        return KVQ_ERR_INVALID_ARG;
+    if (T == 0)
+        return KVQ_OK;
+    if (!x || !centroids || !idx || !codes || !meta)
+        return KVQ_ERR_INVALID_ARG;
+    if (!aligned16(x) || !aligned16(centroids) || !aligned16(codes) || !aligned16(meta) ||
+        (reinterpret_cast<uintptr_t>(idx) & 1u))
+        return KVQ_ERR_ALIGNMENT;
+    EncodeArgs e;
+    e.x = x;
+    e.x_bf16 = x_dtype == KVQ_BF16;
+    e.T = T;
+    e.H = desc->num_heads;
+    e.C = desc->num_centroids;
+    e.bits = desc->bits;
+    e.G = desc->group_size;
+    e.cent = static_cast<const uint16_t *>(centroids);
+    e.idx = idx;
+    e.codes = codes;
+    e.meta = meta;
+    e.assign_only = 0;
+    return launch_encode_direct(desc->head_dim, e, reinterpret_cast<cudaStream_t>(stream));
+}
+
+kvq_status kvq_joint_coefficients(const kvq_codec_desc *desc, const void *x, kvq_dtype x_dtype, int64_t T,
+                                  const void *centroids, const void *w_enc, uint16_t *idx, float *coef_out,
+                                  void *workspace, size_t workspace_bytes, kvq_stream_t stream)
+{
+    (void)desc; (void)x; (void)x_dtype; (void)T; (void)centroids; (void)w_enc; (void)idx; (void)coef_out;
+    (void)workspace; (void)workspace_bytes; (void)stream;
+    return KVQ_ERR_UNSUPPORTED;
+}
+
+kvq_status kvq_decode(const kvq_compressed_view *view, void *x_out, kvq_dtype out_dtype, void *workspace,
+                      size_t workspace_bytes, kvq_stream_t stream)
+{
+    (void)workspace;
+    (void)workspace_bytes;
+    kvq_status st = check_view(view);
+    if (st != KVQ_OK)
+        return st;
+    if (view->desc.joint_rank > 0)
+        return KVQ_ERR_UNSUPPORTED;
+    if (out_dtype != KVQ_F32 && out_dtype != KVQ_BF16)
+        return KVQ_ERR_INVALID_ARG;
+    if (view->num_tokens == 0)
+        return KVQ_OK;
+    if (!x_out)
+        return KVQ_ERR_INVALID_ARG;
+    if (!aligned16(x_out))
+        return KVQ_ERR_ALIGNMENT;
+    DecodeArgs a;
+    a.cent = static_cast<const uint16_t *>(view->centroids);
+    a.idx = view->idx;
+    a.codes = view->codes;
+    a.meta = view->meta;
+    a.T = view->num_tokens;
+    a.H = view->desc.num_heads;
+    a.D = view->desc.head_dim;
+    a.C = view->desc.num_centroids;
+    a.bits = view->desc.bits;
+    a.G = view->desc.group_size;
+    a.out = x_out;
+    a.out_bf16 = out_dtype == KVQ_BF16;
+    const int64_t n = a.T * a.H * (a.D / 8);
+    decode_kernel<<<(unsigned)ceil_div(n, 256), 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(a);
+    return launch_status();
+}
+
+kvq_status kvq_attention_lse(const void *q, int64_t Tq, const kvq_compressed_view *k, const kvq_compressed_view *v,
+                             int64_t t_begin, int64_t t_end, float softmax_scale, void *o_out, kvq_dtype o_dtype,
+                             float *lse_out, void *workspace, size_t workspace_bytes, kvq_stream_t stream)
+{
+    (void)workspace;
+    (void)workspace_bytes;
+    kvq_status st;
+    if ((st = check_view(k)) != KVQ_OK || (st = check_view(v)) != KVQ_OK)
+        return st;
+    if (k->desc.joint_rank > 0 || v->desc.joint_rank > 0)
+        return KVQ_ERR_UNSUPPORTED;
+    if (k->desc.num_heads != v->desc.num_heads || k->desc.head_dim != v->desc.head_dim ||
+        k->num_tokens != v->num_tokens)
+        return KVQ_ERR_INVALID_ARG;
+    if (Tq < 0 || t_begin < 0 || t_end < t_begin || t_end > k->num_tokens)
+        return KVQ_ERR_INVALID_ARG;
+    if (o_dtype != KVQ_F32 && o_dtype != KVQ_BF16)
+        return KVQ_ERR_INVALID_ARG;
+    if (Tq == 0)
+        return KVQ_OK;
+    if (!q || !o_out || !lse_out)
+        return KVQ_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(o_out) || !aligned16(lse_out))
+        return KVQ_ERR_ALIGNMENT;
+    const int D = k->desc.head_dim;
+    AttnArgs a;
+    a.q = static_cast<const uint16_t *>(q);
+    a.Tq = Tq;
+    a.H = k->desc.num_heads;
+    a.k = to_codec_view(k);
+    a.v = to_codec_view(v);
+    a.t_begin = t_begin;
+    a.t_end = t_end;
+    const float scale = softmax_scale > 0.0f ? softmax_scale : 1.0f / sqrtf((float)D);
+    a.scale_log2 = scale * 1.4426950408889634f;
+    a.o_out = o_out;
+    a.o_bf16 = o_dtype == KVQ_BF16;
+    a.lse_out = lse_out;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    return D == 128 ? launch_attention<128>(a, s) : launch_attention<64>(a, s);
+}
+
+kvq_status kvq_lse_merge(int32_t n_parts, const float *const *o_parts, const float *const *lse_parts, int64_t Tq,
+                         int32_t H, int32_t d, void *o_out, kvq_dtype o_dtype, float *lse_out, kvq_stream_t stream)
+{
+    if (n_parts < 1 || n_parts > kMaxMergeParts || !o_parts || !lse_parts || Tq < 0 || H < 1)
+        return KVQ_ERR_INVALID_ARG;
+    if (!supported_dim(d))
+        return KVQ_ERR_UNSUPPORTED;
+    if (o_dtype != KVQ_F32 && o_dtype != KVQ_BF16)
+        return KVQ_ERR_INVALID_ARG;
+    if (Tq == 0)
+        return KVQ_OK;
+    if (!o_out || !lse_out)
+        return KVQ_ERR_INVALID_ARG;
+    MergeArgs a;
+    memset(&a, 0, sizeof a);
+    for (int b = 0; b < n_parts; ++b) {
+        if (!o_parts[b] || !lse_parts[b])
+            return KVQ_ERR_INVALID_ARG;
+        if (!aligned16(o_parts[b]) || (reinterpret_cast<uintptr_t>(lse_parts[b]) & 3u))
+            return KVQ_ERR_ALIGNMENT;
+        a.o[b] = o_parts[b];
+        a.lse[b] = lse_parts[b];
+    }
+    if (!aligned16(o_out) || (reinterpret_cast<uintptr_t>(lse_out) & 3u))
+        return KVQ_ERR_ALIGNMENT;
+    a.n = n_parts;
+    a.Tq = Tq;
+    a.H = H;
+    a.D = d;
+    a.o_out = o_out;
+    a.o_bf16 = o_dtype == KVQ_BF16;
+    a.lse_out = lse_out;
+    const int64_t n = Tq * H * (d / 4);
+    lse_merge_kernel<<<(unsigned)ceil_div(n, 256), 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(a);
+    return launch_status();
+}
+
+kvq_status kvq_last_device_status(kvq_stream_t stream)
+{
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (cudaStreamSynchronize(s) != cudaSuccess)
+        return KVQ_ERR_CUDA;
+    unsigned int word = 0, zero = 0;
+    if (cudaMemcpyFromSymbol(&word, g_device_status, sizeof word) != cudaSuccess)
+        return KVQ_ERR_CUDA;
+    if (word != 0 && cudaMemcpyToSymbol(g_device_status, &zero, sizeof zero) != cudaSuccess)
+        return KVQ_ERR_CUDA;
+    if (word & DEVSTAT_TIMEOUT)
+        return KVQ_ERR_DEVICE_TIMEOUT;
+    if (word & DEVSTAT_BAD_INDEX)
+        return KVQ_ERR_INVALID_ARG;
+    return KVQ_OK;
+}
+
+}  // extern "C"

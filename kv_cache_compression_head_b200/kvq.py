@@ -1,0 +1,271 @@
+"""ctypes binding of libkvq (include/kvq.h).
+
+Argument marshalling only: every step of the codec and of the attention runs
+in the CUDA library.  Tensors are torch CUDA tensors (device memory and the
+current stream come from torch); the functions take the same names as the C
+entry points.  If libkvq.so is missing or fails to load, importing this module
+raises -- there is no fallback.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import dataclasses
+import os
+from typing import Optional, Sequence, Tuple
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libkvq.so")
+
+KVQ_OK = 0
+KVQ_ERR_INVALID_ARG = 1
+KVQ_ERR_UNSUPPORTED = 2
+KVQ_ERR_ALIGNMENT = 3
+KVQ_ERR_WORKSPACE = 4
+KVQ_ERR_CUDA = 5
+KVQ_ERR_DEVICE_TIMEOUT = 6
+
+KVQ_F32 = 0
+KVQ_BF16 = 1
+
+KVQ_OP_FIT = 0
+KVQ_OP_ENCODE = 1
+KVQ_OP_DECODE = 2
+KVQ_OP_ATTENTION = 3
+
+EXPORTED = (
+    "kvq_status_string", "kvq_encoded_sizes", "kvq_workspace_size", "kvq_fit_centroids", "kvq_encode",
+    "kvq_joint_coefficients", "kvq_decode", "kvq_attention_lse", "kvq_lse_merge", "kvq_last_device_status",
+)
+
+
+class KvqError(RuntimeError):
+    def __init__(self, code: int, what: str):
+        self.code = code
+        super().__init__(f"{what} failed: {status_string(code)} ({code})")
+
+
+class CodecDesc(ctypes.Structure):
+    _fields_ = [("num_heads", ctypes.c_int32), ("head_dim", ctypes.c_int32), ("num_centroids", ctypes.c_int32),
+                ("bits", ctypes.c_int32), ("group_size", ctypes.c_int32), ("joint_rank", ctypes.c_int32)]
+
+
+class CompressedView(ctypes.Structure):
+    _fields_ = [("desc", CodecDesc), ("num_tokens", ctypes.c_int64), ("centroids", ctypes.c_void_p),
+                ("idx", ctypes.c_void_p), ("codes", ctypes.c_void_p), ("meta", ctypes.c_void_p),
+                ("w_dec", ctypes.c_void_p)]
+
+
+def _load():
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"libkvq.so not built ({LIB_PATH}); run python -m kv_cache_compression_head_b200.build")
+    lib = ctypes.CDLL(LIB_PATH)
+    vp, i32, i64, sz = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_size_t
+    pdesc, pview = ctypes.POINTER(CodecDesc), ctypes.POINTER(CompressedView)
+    lib.kvq_status_string.argtypes = [ctypes.c_int]
+    lib.kvq_status_string.restype = ctypes.c_char_p
+    sig = {
+        "kvq_encoded_sizes": [pdesc, i64, ctypes.POINTER(sz), ctypes.POINTER(sz), ctypes.POINTER(sz)],
+        "kvq_workspace_size": [ctypes.c_int, pdesc, i64, i64, ctypes.POINTER(sz)],
+        "kvq_fit_centroids": [pdesc, vp, ctypes.c_int, i64, i32, vp, vp, sz, vp],
+        "kvq_encode": [pdesc, vp, ctypes.c_int, i64, vp, vp, vp, vp, vp, vp, sz, vp],
+        "kvq_joint_coefficients": [pdesc, vp, ctypes.c_int, i64, vp, vp, vp, vp, vp, sz, vp],
+        "kvq_decode": [pview, vp, ctypes.c_int, vp, sz, vp],
+        "kvq_attention_lse": [vp, i64, pview, pview, i64, i64, ctypes.c_float, vp, ctypes.c_int, vp, vp, sz, vp],
+        "kvq_lse_merge": [i32, ctypes.POINTER(vp), ctypes.POINTER(vp), i64, i32, i32, vp, ctypes.c_int, vp, vp],
+        "kvq_last_device_status": [vp],
+    }
+    for name, args in sig.items():
+        fn = getattr(lib, name)
+        fn.argtypes = args
+        fn.restype = ctypes.c_int
+    return lib
+
+
+_lib = _load()
+
+
+def status_string(code: int) -> str:
+    return _lib.kvq_status_string(code).decode()
+
+
+def _check(code: int, what: str):
+    if code != KVQ_OK:
+        raise KvqError(code, what)
+
+
+def _ptr(t: Optional[torch.Tensor]) -> Optional[int]:
+    if t is None:
+        return None
+    return t.data_ptr()
+
+
+def _stream(stream=None) -> Optional[int]:
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return s.cuda_stream or None
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return KVQ_BF16
+    if t.dtype == torch.float32:
+        return KVQ_F32
+    raise TypeError(f"unsupported dtype {t.dtype}")
+
+
+# ----------------------------------------------------------------------------
+# descriptors
+# ----------------------------------------------------------------------------
+
+@dataclasses.dataclass
+class Codec:
+    """One K or V branch: heads, head dim, centroids, bits, group size, joint rank."""
+
+    num_heads: int
+    head_dim: int
+    num_centroids: int
+    bits: int
+    group_size: int
+    joint_rank: int = 0
+
+    def c(self) -> CodecDesc:
+        return CodecDesc(self.num_heads, self.head_dim, self.num_centroids, self.bits, self.group_size,
+                         self.joint_rank)
+
+
+@dataclasses.dataclass
+class Compressed:
+    """Device tensors of one encoded K or V history."""
+
+    codec: Codec
+    num_tokens: int
+    centroids: torch.Tensor  # [H][C][d] bf16
+    idx: torch.Tensor        # [H][T] int16 (uint16 bits)
+    codes: torch.Tensor      # uint8
+    meta: torch.Tensor       # float32
+    w_dec: Optional[torch.Tensor] = None
+
+    def view(self) -> CompressedView:
+        return CompressedView(self.codec.c(), self.num_tokens, _ptr(self.centroids), _ptr(self.idx),
+                              _ptr(self.codes), _ptr(self.meta), _ptr(self.w_dec))
+
+
+def encoded_sizes(codec: Codec, num_tokens: int) -> Tuple[int, int, int]:
+    a, b, c = ctypes.c_size_t(), ctypes.c_size_t(), ctypes.c_size_t()
+    d = codec.c()
+    _check(_lib.kvq_encoded_sizes(ctypes.byref(d), num_tokens, ctypes.byref(a), ctypes.byref(b), ctypes.byref(c)),
+           "kvq_encoded_sizes")
+    return a.value, b.value, c.value
+
+
+def workspace_size(op: int, codec: Codec, num_tokens: int, num_queries: int = 0) -> int:
+    out = ctypes.c_size_t()
+    d = codec.c()
+    _check(_lib.kvq_workspace_size(op, ctypes.byref(d), num_tokens, num_queries, ctypes.byref(out)),
+           "kvq_workspace_size")
+    return out.value
+
+
+def alloc_encoded(codec: Codec, num_tokens: int, device) -> Tuple[torch.Tensor, torch.Tensor, torch.Tensor]:
+    """Allocate idx, codes and meta tensors of the sizes kvq_encoded_sizes reports."""
+    ib, cb, mb = encoded_sizes(codec, num_tokens)
+    idx = torch.empty(ib // 2, dtype=torch.int16, device=device)
+    codes = torch.empty(cb, dtype=torch.uint8, device=device)
+    meta = torch.empty(mb // 4, dtype=torch.float32, device=device)
+    return idx, codes, meta
+
+
+def alloc_workspace(op: int, codec: Codec, num_tokens: int, device, num_queries: int = 0) -> Optional[torch.Tensor]:
+    n = workspace_size(op, codec, num_tokens, num_queries)
+    if n == 0:
+        return None
+    return torch.empty(n, dtype=torch.uint8, device=device)
+
+
+# ----------------------------------------------------------------------------
+# entry points
+# ----------------------------------------------------------------------------
+
+def kvq_fit_centroids(codec: Codec, x: torch.Tensor, iters: int, centroids_out: torch.Tensor,
+                      workspace: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    T = x.shape[0]
+    if workspace is None:
+        workspace = alloc_workspace(KVQ_OP_FIT, codec, T, x.device)
+    d = codec.c()
+    _check(_lib.kvq_fit_centroids(ctypes.byref(d), _ptr(x), _dtype_code(x), T, iters, _ptr(centroids_out),
+                                  _ptr(workspace), workspace.numel() if workspace is not None else 0,
+                                  _stream(stream)), "kvq_fit_centroids")
+    return centroids_out
+
+
+def kvq_encode(codec: Codec, x: torch.Tensor, centroids: torch.Tensor, idx: torch.Tensor, codes: torch.Tensor,
+               meta: torch.Tensor, w_enc: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None,
+               stream=None) -> None:
+    d = codec.c()
+    _check(_lib.kvq_encode(ctypes.byref(d), _ptr(x), _dtype_code(x), x.shape[0], _ptr(centroids), _ptr(w_enc),
+                           _ptr(idx), _ptr(codes), _ptr(meta), _ptr(workspace),
+                           workspace.numel() if workspace is not None else 0, _stream(stream)), "kvq_encode")
+
+
+def kvq_joint_coefficients(codec: Codec, x: torch.Tensor, centroids: torch.Tensor, w_enc: torch.Tensor,
+                           idx: torch.Tensor, coef_out: torch.Tensor, workspace: Optional[torch.Tensor] = None,
+                           stream=None) -> None:
+    d = codec.c()
+    _check(_lib.kvq_joint_coefficients(ctypes.byref(d), _ptr(x), _dtype_code(x), x.shape[0], _ptr(centroids),
+                                       _ptr(w_enc), _ptr(idx), _ptr(coef_out), _ptr(workspace),
+                                       workspace.numel() if workspace is not None else 0, _stream(stream)),
+           "kvq_joint_coefficients")
+
+
+def kvq_decode(comp: Compressed, x_out: torch.Tensor, workspace: Optional[torch.Tensor] = None,
+               stream=None) -> torch.Tensor:
+    v = comp.view()
+    _check(_lib.kvq_decode(ctypes.byref(v), _ptr(x_out), _dtype_code(x_out), _ptr(workspace),
+                           workspace.numel() if workspace is not None else 0, _stream(stream)), "kvq_decode")
+    return x_out
+
+
+def kvq_attention_lse(q: torch.Tensor, k: Compressed, v: Compressed, o_out: torch.Tensor, lse_out: torch.Tensor,
+                      t_begin: int = 0, t_end: Optional[int] = None, softmax_scale: float = 0.0,
+                      workspace: Optional[torch.Tensor] = None, stream=None) -> None:
+    if t_end is None:
+        t_end = k.num_tokens
+    kv, vv = k.view(), v.view()
+    _check(_lib.kvq_attention_lse(_ptr(q), q.shape[0], ctypes.byref(kv), ctypes.byref(vv), t_begin, t_end,
+                                  softmax_scale, _ptr(o_out), _dtype_code(o_out), _ptr(lse_out), _ptr(workspace),
+                                  workspace.numel() if workspace is not None else 0, _stream(stream)),
+           "kvq_attention_lse")
+
+
+def kvq_lse_merge(o_parts: Sequence[torch.Tensor], lse_parts: Sequence[torch.Tensor], o_out: torch.Tensor,
+                  lse_out: torch.Tensor, stream=None) -> None:
+    n = len(o_parts)
+    Tq, H, d = o_parts[0].shape
+    arr_o = (ctypes.c_void_p * n)(*[t.data_ptr() for t in o_parts])
+    arr_l = (ctypes.c_void_p * n)(*[t.data_ptr() for t in lse_parts])
+    _check(_lib.kvq_lse_merge(n, arr_o, arr_l, Tq, H, d, _ptr(o_out), _dtype_code(o_out), _ptr(lse_out),
+                              _stream(stream)), "kvq_lse_merge")
+
+
+def kvq_last_device_status(stream=None) -> int:
+    return _lib.kvq_last_device_status(_stream(stream))
+
+
+# ----------------------------------------------------------------------------
+# convenience: fit + encode one history into a Compressed record
+# ----------------------------------------------------------------------------
+
+def compress(codec: Codec, x: torch.Tensor, iters: int, centroids: Optional[torch.Tensor] = None,
+             fit_workspace: Optional[torch.Tensor] = None, stream=None) -> Compressed:
+    """Fit (unless centroids are given) and encode one K or V history."""
+    T = x.shape[0]
+    dev = x.device
+    if centroids is None:
+        centroids = torch.empty((codec.num_heads, codec.num_centroids, codec.head_dim), dtype=torch.bfloat16,
+                                device=dev)
+        kvq_fit_centroids(codec, x, iters, centroids, fit_workspace, stream)
+    idx, codes, meta = alloc_encoded(codec, T, dev)
+    kvq_encode(codec, x, centroids, idx, codes, meta, stream=stream)
+    return Compressed(codec, T, centroids, idx, codes, meta)

@@ -1,0 +1,117 @@
+"""Host-side checks of the C ABI: the library loads, exports every entry point
+include/kvq.h declares, reports sizes, and rejects bad arguments before any
+device work (these calls never reach the GPU, so they run without one)."""
+
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def K():
+    from kv_cache_compression_head_b200 import build
+
+    build.build()
+    from kv_cache_compression_head_b200 import kvq
+
+    return kvq
+
+
+def _declared():
+    src = open(os.path.join(ROOT, "include", "kvq.h")).read()
+    return sorted(set(re.findall(r"KVQ_API\s+[\w\s\*]*?\b(kvq_\w+)\s*\(", src)))
+
+
+def test_header_symbols_exported(K):
+    names = _declared()
+    assert len(names) >= 10
+    lib = ctypes.CDLL(K.LIB_PATH)
+    for n in names:
+        assert hasattr(lib, n), n
+    assert set(names) == set(K.EXPORTED)
+
+
+def test_status_strings(K):
+    for code in range(7):
+        assert K.status_string(code).startswith("KVQ_")
+    assert K.status_string(99) == "KVQ_ERR_UNKNOWN"
+
+
+def test_encoded_sizes_and_workspace(K):
+    c = K.Codec(12, 128, 256, 2, 16)
+    ib, cb, mb = K.encoded_sizes(c, 32760)
+    assert ib == 12 * 32760 * 2
+    assert cb == 12 * 32760 * 32
+    assert mb == 12 * 32760 * 8 * 8
+    # 98 bytes per token-head: 2 index + 32 codes + 64 metadata
+    assert (ib + cb + mb) == 12 * 32760 * 98
+    c4 = K.Codec(40, 128, 512, 4, 32)
+    assert K.encoded_sizes(c4, 10)[1] == 40 * 10 * 64
+    assert K.workspace_size(K.KVQ_OP_FIT, c, 32760) > 12 * 256 * 128 * 8
+    assert K.workspace_size(K.KVQ_OP_ATTENTION, c, 32760, 4680) == 0
+    assert K.workspace_size(K.KVQ_OP_ENCODE, c, 32760) == 0
+
+
+def _err(K, fn, *args):
+    return getattr(K._lib, fn)(*args)
+
+
+def test_bad_descriptors_rejected(K):
+    sz = ctypes.c_size_t()
+    for bad, want in [((12, 96, 256, 2, 16, 0), K.KVQ_ERR_UNSUPPORTED), ((12, 128, 256, 3, 16, 0), K.KVQ_ERR_UNSUPPORTED),
+                      ((12, 128, 256, 2, 24, 0), K.KVQ_ERR_INVALID_ARG), ((12, 128, 0, 2, 16, 0), K.KVQ_ERR_INVALID_ARG),
+                      ((0, 128, 256, 2, 16, 0), K.KVQ_ERR_INVALID_ARG), ((12, 128, 70000, 2, 16, 0), K.KVQ_ERR_INVALID_ARG),
+                      ((12, 128, 256, 2, 8, 0), K.KVQ_ERR_UNSUPPORTED), ((12, 128, 256, 4, 20, 192), K.KVQ_ERR_INVALID_ARG)]:
+        d = K.CodecDesc(*bad)
+        assert _err(K, "kvq_encoded_sizes", ctypes.byref(d), 10, ctypes.byref(sz), None, None) == want, bad
+    d = K.CodecDesc(12, 128, 256, 2, 16, 0)
+    assert _err(K, "kvq_encoded_sizes", ctypes.byref(d), -1, None, None, None) == K.KVQ_ERR_INVALID_ARG
+    assert _err(K, "kvq_encoded_sizes", None, 10, None, None, None) == K.KVQ_ERR_INVALID_ARG
+
+
+def test_bad_pointers_and_sizes_rejected_on_host(K):
+    d = K.CodecDesc(12, 128, 256, 2, 16, 0)
+    A = 1 << 20  # a fake, 16-byte-aligned address: never dereferenced
+    # encode: null input, misaligned codes
+    assert _err(K, "kvq_encode", ctypes.byref(d), None, K.KVQ_BF16, 100, A, None, A, A, A, None, 0, None) \
+        == K.KVQ_ERR_INVALID_ARG
+    assert _err(K, "kvq_encode", ctypes.byref(d), A, K.KVQ_BF16, 100, A, None, A, A + 8, A, None, 0, None) \
+        == K.KVQ_ERR_ALIGNMENT
+    assert _err(K, "kvq_encode", ctypes.byref(d), A, 7, 100, A, None, A, A, A, None, 0, None) \
+        == K.KVQ_ERR_INVALID_ARG
+    # fit: T < C, too little workspace
+    assert _err(K, "kvq_fit_centroids", ctypes.byref(d), A, K.KVQ_BF16, 100, 2, A, A, 1 << 30, None) \
+        == K.KVQ_ERR_INVALID_ARG
+    assert _err(K, "kvq_fit_centroids", ctypes.byref(d), A, K.KVQ_BF16, 1000, 2, A, A, 16, None) \
+        == K.KVQ_ERR_WORKSPACE
+    assert _err(K, "kvq_fit_centroids", ctypes.byref(d), A, K.KVQ_BF16, 1000, -1, A, A, 1 << 30, None) \
+        == K.KVQ_ERR_INVALID_ARG
+    # attention: range outside the history, mismatched views
+    v = K.CompressedView(d, 1000, A, A, A, A, None)
+    v2 = K.CompressedView(K.CodecDesc(8, 128, 256, 2, 16, 0), 1000, A, A, A, A, None)
+    assert _err(K, "kvq_attention_lse", A, 10, ctypes.byref(v), ctypes.byref(v), 0, 1001, ctypes.c_float(0),
+                A, K.KVQ_F32, A, None, 0, None) == K.KVQ_ERR_INVALID_ARG
+    assert _err(K, "kvq_attention_lse", A, 10, ctypes.byref(v), ctypes.byref(v), 5, 4, ctypes.c_float(0),
+                A, K.KVQ_F32, A, None, 0, None) == K.KVQ_ERR_INVALID_ARG
+    assert _err(K, "kvq_attention_lse", A, 10, ctypes.byref(v), ctypes.byref(v2), 0, 10, ctypes.c_float(0),
+                A, K.KVQ_F32, A, None, 0, None) == K.KVQ_ERR_INVALID_ARG
+    assert _err(K, "kvq_attention_lse", A + 4, 10, ctypes.byref(v), ctypes.byref(v), 0, 10, ctypes.c_float(0),
+                A, K.KVQ_F32, A, None, 0, None) == K.KVQ_ERR_ALIGNMENT
+    # zero query rows is a no-op even with null outputs
+    assert _err(K, "kvq_attention_lse", None, 0, ctypes.byref(v), ctypes.byref(v), 0, 10, ctypes.c_float(0),
+                None, K.KVQ_F32, None, None, 0, None) == K.KVQ_OK
+    # merge: part counts out of range, null part
+    arr = (ctypes.c_void_p * 65)(*([A] * 65))
+    assert _err(K, "kvq_lse_merge", 0, arr, arr, 10, 2, 128, A, K.KVQ_F32, A, None) == K.KVQ_ERR_INVALID_ARG
+    assert _err(K, "kvq_lse_merge", 65, arr, arr, 10, 2, 128, A, K.KVQ_F32, A, None) == K.KVQ_ERR_INVALID_ARG
+    arr_null = (ctypes.c_void_p * 2)(A, None)
+    assert _err(K, "kvq_lse_merge", 2, arr_null, arr, 10, 2, 128, A, K.KVQ_F32, A, None) == K.KVQ_ERR_INVALID_ARG
+    assert _err(K, "kvq_lse_merge", 2, arr, arr, 10, 2, 96, A, K.KVQ_F32, A, None) == K.KVQ_ERR_UNSUPPORTED
+    # decode: joint view not served yet by the per-head decoder arguments
+    vj = K.CompressedView(K.CodecDesc(12, 128, 256, 4, 32, 192), 10, A, A, A, A, A)
+    assert _err(K, "kvq_decode", ctypes.byref(vj), A, K.KVQ_F32, None, 0, None) in (K.KVQ_ERR_UNSUPPORTED,
+                                                                                     K.KVQ_ERR_WORKSPACE)

@@ -1,0 +1,492 @@
+#!/usr/bin/env python
+"""Benchmark of the compressed-KV hot path on B200.
+
+One step = one pass of every step of the path over the Wan-1.3B-like layer
+(12 heads x 128, bf16, history 21 frames x 1,560 = 32,760 tokens, query chunk
+4,680 tokens, 256 centroids per head, K INT2 / V INT2, group 16):
+
+  fit centroids (K, V; 2 k-means rounds) -> encode (K, V) -> decode (K, V)
+  -> attention of the chunk over the compressed history in 2 blocks
+  -> LSE merge of the 2 partial results.
+
+Inputs are seeded synthetic tensors resident in HBM before timing starts;
+L2 is flushed (256 MiB write) before every timed step, outside the step's
+events.  The headline value is history tokens per second of whole steps,
+summed over ranks.  ``--impl reference`` times the CPU oracle instead on a
+bounded sample of the same workload.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+"""
+
+from __future__ import annotations
+
+import argparse
+import datetime
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "encode history-tokens/s (HBM GB/s) and compressed-KV attention TFLOP/s, 1×B200"
+UNIT = "history-tokens/s"
+WORKLOAD = "wan13b"
+HISTORY_BLOCKS = 2
+FLUSH_BYTES = 256 << 20
+
+
+def parse_args():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=10)
+    p.add_argument("--warmup", type=int, default=3)
+    p.add_argument("--impl", default="kvq", choices=["kvq", "reference"])
+    p.add_argument("--no-e2e", action="store_true")
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    return p.parse_args()
+
+
+# ----------------------------------------------------------------------------
+# distributed plumbing (replicas: every rank runs the full workload)
+# ----------------------------------------------------------------------------
+
+def dist_env():
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return rank, world, local
+
+
+def init_dist(world, backend):
+    import torch.distributed as dist
+
+    if world > 1 and not dist.is_initialized():
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    return dist
+
+
+def max_over_ranks(x: float, world: int, device) -> float:
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.barrier()
+
+
+# ----------------------------------------------------------------------------
+# clocks during the timed region
+# ----------------------------------------------------------------------------
+
+class ClockSampler:
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        fd, self.path = tempfile.mkstemp(prefix="kvq_clocks_", suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.QUERY}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        rows = []
+        for line in open(self.path):
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                rows.append((float(f[1]), float(f[2]), float(f[3]) if f[3] not in ("[N/A]", "N/A") else 0.0,
+                             f[5:9]))
+            except ValueError:
+                continue
+        os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        sm_max = max(r[1] for r in rows)
+        loaded = [r for r in rows if r[2] > 200.0] or rows
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in loaded for i, v in enumerate(r[3]) if v.lower() == "active"})
+        return {"sm_mhz": statistics.median(r[0] for r in loaded), "sm_max_mhz": sm_max, "reasons": reasons,
+                "samples": len(rows), "samples_under_load": len(loaded),
+                "power_w_max": max(r[2] for r in rows)}
+
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        return p["hbm_gbs"], p["bf16_tflops"], "measured"
+    return 6650.0, 1590.0, "fallback"
+
+
+# ----------------------------------------------------------------------------
+# algorithmic work per step (roofline numerators)
+# ----------------------------------------------------------------------------
+
+def work_model(w):
+    T, H, d, Tq, C, G = w.history_tokens, w.num_heads, w.head_dim, w.query_tokens, w.num_centroids, w.group_size
+    th = T * H
+
+    def stored(bits):  # bytes written per token-head by encode
+        return d * bits // 8 + 8 * (d // G) + 2
+
+    enc_bytes = sum(th * (2 * d + stored(b)) for b in (w.bits_k, w.bits_v))
+    dec_bytes = sum(th * (stored(b) + 2 * d) for b in (w.bits_k, w.bits_v))  # read compressed, write bf16
+    attn_flops = 4.0 * Tq * T * d * H
+    merge_bytes = (HISTORY_BLOCKS + 1) * Tq * H * d * 4 + (HISTORY_BLOCKS + 1) * Tq * H * 4
+    assign_ops = 3.0 * th * C * d * 2  # exact distance: sub, mul, add per channel per centre (K and V)
+    return {"encode_bytes": enc_bytes, "decode_bytes": dec_bytes, "attention_flops": attn_flops,
+            "merge_bytes": merge_bytes, "assign_ops": assign_ops}
+
+
+# ----------------------------------------------------------------------------
+# GPU arm
+# ----------------------------------------------------------------------------
+
+class Pipeline:
+    """Device buffers and the per-step call sequence through the public API."""
+
+    ROWS = ("fit", "encode", "decode", "attention", "merge")
+
+    def __init__(self, w, device):
+        import torch
+
+        from kv_cache_compression_head_b200 import kvq as K
+
+        self.K = K
+        self.w = w
+        self.dev = device
+        T, H, d, Tq = w.history_tokens, w.num_heads, w.head_dim, w.query_tokens
+        self.codec_k = K.Codec(H, d, w.num_centroids, w.bits_k, w.group_size)
+        self.codec_v = K.Codec(H, d, w.num_centroids, w.bits_v, w.group_size)
+        bf = torch.bfloat16
+        self.xk = torch.empty((T, H, d), dtype=bf, device=device)
+        self.xv = torch.empty((T, H, d), dtype=bf, device=device)
+        self.q = torch.empty((Tq, H, d), dtype=bf, device=device)
+        self.cent = [torch.empty((H, w.num_centroids, d), dtype=bf, device=device) for _ in range(2)]
+        self.enc = [K.alloc_encoded(c, T, device) for c in (self.codec_k, self.codec_v)]
+        self.ws = K.alloc_workspace(K.KVQ_OP_FIT, self.codec_k, T, device)
+        self.dec = [torch.empty((T, H, d), dtype=bf, device=device) for _ in range(2)]
+        self.o_parts = [torch.empty((Tq, H, d), dtype=torch.float32, device=device) for _ in range(HISTORY_BLOCKS)]
+        self.l_parts = [torch.empty((H, Tq), dtype=torch.float32, device=device) for _ in range(HISTORY_BLOCKS)]
+        self.o = torch.empty((Tq, H, d), dtype=bf, device=device)
+        self.lse = torch.empty((H, Tq), dtype=torch.float32, device=device)
+        self.edges = [T * i // HISTORY_BLOCKS for i in range(HISTORY_BLOCKS + 1)]
+        self.comp = [K.Compressed(c, T, self.cent[i], *self.enc[i])
+                     for i, c in enumerate((self.codec_k, self.codec_v))]
+        self.launches_per_step = (2 * (1 + 3 * w.kmeans_iters) + 2 + 2 + HISTORY_BLOCKS + 1)
+
+    def outputs(self):
+        outs = [self.o, self.lse]
+        for i in range(2):
+            outs += [self.cent[i], *self.enc[i]]
+        return outs
+
+    def step(self, ev=None):
+        """Run one step; ev (optional) is a dict row -> (start, end) events."""
+        K, w = self.K, self.w
+
+        def mark(row, i):
+            if ev is not None:
+                ev[row][i].record()
+
+        mark("fit", 0)
+        K.kvq_fit_centroids(self.codec_k, self.xk, w.kmeans_iters, self.cent[0], self.ws)
+        K.kvq_fit_centroids(self.codec_v, self.xv, w.kmeans_iters, self.cent[1], self.ws)
+        mark("fit", 1)
+        mark("encode", 0)
+        K.kvq_encode(self.codec_k, self.xk, self.cent[0], *self.enc[0])
+        K.kvq_encode(self.codec_v, self.xv, self.cent[1], *self.enc[1])
+        mark("encode", 1)
+        mark("decode", 0)
+        K.kvq_decode(self.comp[0], self.dec[0])
+        K.kvq_decode(self.comp[1], self.dec[1])
+        mark("decode", 1)
+        mark("attention", 0)
+        for b in range(HISTORY_BLOCKS):
+            K.kvq_attention_lse(self.q, self.comp[0], self.comp[1], self.o_parts[b], self.l_parts[b],
+                                t_begin=self.edges[b], t_end=self.edges[b + 1])
+        mark("attention", 1)
+        mark("merge", 0)
+        K.kvq_lse_merge(self.o_parts, self.l_parts, self.o, self.lse)
+        mark("merge", 1)
+
+
+def run_gpu(args):
+    import torch
+
+    from kv_cache_compression_head_b200 import synth
+
+    rank, world, local = dist_env()
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    init_dist(world, "nccl")
+    w = synth.workload(WORKLOAD)
+
+    # seeded inputs: generated on the host, staged in pinned memory
+    hk = synth.make_history(w, "K")
+    hv = synth.make_history(w, "V")
+    hq = synth.make_queries(w)
+    pin = lambda a: torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).pin_memory()
+    pk, pv, pq = pin(hk), pin(hv), pin(hq)
+
+    pipe = Pipeline(w, device)
+    pipe.xk.copy_(pk)
+    pipe.xv.copy_(pv)
+    pipe.q.copy_(pq)
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=device)
+    torch.cuda.synchronize()
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        pipe.step()
+    torch.cuda.synchronize()
+    st = pipe.K.kvq_last_device_status()
+    if st != 0:
+        raise RuntimeError(f"device status after warm-up: {pipe.K.status_string(st)}")
+
+    ev = [{r: (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for r in Pipeline.ROWS}
+          for _ in range(args.steps)]
+    clocks = ClockSampler(local)
+    barrier(world)
+    torch.cuda.synchronize()
+    clocks.start()
+    t_wall = time.perf_counter()
+    for k in range(args.steps):
+        flush.zero_()
+        pipe.step(ev[k])
+    torch.cuda.synchronize()
+    wall = time.perf_counter() - t_wall
+    barrier(world)
+    clk = clocks.stop()
+    st = pipe.K.kvq_last_device_status()
+    if st != 0:
+        raise RuntimeError(f"device status after timing: {pipe.K.status_string(st)}")
+
+    row_ms = {r: [e[r][0].elapsed_time(e[r][1]) for e in ev] for r in Pipeline.ROWS}
+    step_ms = [ev[k]["fit"][0].elapsed_time(ev[k]["merge"][1]) for k in range(args.steps)]
+    ms_step_local = statistics.mean(step_ms)
+    ms_step = max_over_ranks(ms_step_local, world, device)
+    row_mean = {r: statistics.mean(v) for r, v in row_ms.items()}
+
+    # end-to-end through the public API with host buffers
+    e2e = None
+    if not args.no_e2e:
+        outs = pipe.outputs()
+        host_outs = [torch.empty(o.shape, dtype=o.dtype, pin_memory=True) for o in outs]
+        h2d = sum(t.numel() * t.element_size() for t in (pk, pv, pq))
+        d2h = sum(t.numel() * t.element_size() for t in outs)
+        e_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                for _ in range(args.steps)]
+        for k in range(args.steps + 1):  # first pass untimed
+            if k > 0:
+                e_ev[k - 1][0].record()
+            pipe.xk.copy_(pk, non_blocking=True)
+            pipe.xv.copy_(pv, non_blocking=True)
+            pipe.q.copy_(pq, non_blocking=True)
+            pipe.step()
+            for ho, o in zip(host_outs, outs):
+                ho.copy_(o, non_blocking=True)
+            if k > 0:
+                e_ev[k - 1][1].record()
+        torch.cuda.synchronize()
+        e2e_ms = max_over_ranks(statistics.mean(a.elapsed_time(b) for a, b in e_ev), world, device)
+        e2e = {"value": world * w.history_tokens / (e2e_ms / 1e3), "unit": UNIT, "ms_per_step": e2e_ms,
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+
+    if rank == 0:
+        wm = work_model(w)
+        hbm, tfl, peak_kind = measured_peaks()
+        attn_launch_ms = row_mean["attention"] / HISTORY_BLOCKS
+        attn_launch_flops = wm["attention_flops"] / HISTORY_BLOCKS
+        attn_tflops = attn_launch_flops / (attn_launch_ms / 1e3) / 1e12
+        enc_gbps = wm["encode_bytes"] / (row_mean["encode"] / 1e3) / 1e9
+        dec_gbps = wm["decode_bytes"] / (row_mean["decode"] / 1e3) / 1e9
+        merge_gbps = wm["merge_bytes"] / (row_mean["merge"] / 1e3) / 1e9
+        # exact assignment on CUDA cores: separately rounded sub, mul, add per
+        # channel per centre; peak = 148 SMs x 128 FP32 lanes x 1.965 GHz
+        alu_peak_tops = 148 * 128 * 1.965e9 / 1e12
+        fit_tops = wm["assign_ops"] * (w.kmeans_iters) / (row_mean["fit"] / 1e3) / 1e12
+        rows = {
+            "fit": {"ms": row_mean["fit"], "bound": "alu", "achieved": fit_tops, "peak": alu_peak_tops,
+                    "unit": "Top/s", "frac": fit_tops / alu_peak_tops},
+            "encode": {"ms": row_mean["encode"], "tokens_per_s": w.history_tokens / (row_mean["encode"] / 1e3),
+                       "gbps": enc_gbps, "hbm_frac": enc_gbps / hbm},
+            "decode": {"ms": row_mean["decode"], "gbps": dec_gbps, "hbm_frac": dec_gbps / hbm},
+            "attention": {"ms": row_mean["attention"], "launches": HISTORY_BLOCKS, "tflops": attn_tflops,
+                          "frac": attn_tflops / tfl},
+            "merge": {"ms": row_mean["merge"], "gbps": merge_gbps, "hbm_frac": merge_gbps / hbm},
+        }
+        line = {
+            "metric": METRIC,
+            "value": world * w.history_tokens / (ms_step / 1e3),
+            "unit": UNIT,
+            "n_gpus": world,
+            "steps": args.steps,
+            "warmup": args.warmup,
+            "ms_per_step": ms_step,
+            "higher_is_better": True,
+            "scaling": "weak",
+            "vs_baseline": None,
+            "dtype": "bf16",
+            "data": "synthetic (seeded AR(1) frames + heavy-tailed outlier channels)",
+            "config": {"workload": "wan13b-like layer: 12 heads x 128, history 32760 tokens (21 frames x 1560), "
+                                   "query chunk 4680, C=256, K2V2, group 16, fit 2 rounds, 2 history blocks",
+                       "history_tokens": w.history_tokens, "query_tokens": w.query_tokens,
+                       "heads": w.num_heads, "head_dim": w.head_dim, "centroids": w.num_centroids,
+                       "bits_k": w.bits_k, "bits_v": w.bits_v, "group": w.group_size,
+                       "parallelism": f"replicas x{world}", "l2": "flushed (256 MiB write) before each step"},
+            "roofline": {"kernel": "attention_lse_kernel<128>", "bound": "tensor", "achieved": attn_tflops,
+                         "peak": tfl, "unit": "TFLOP/s", "frac": attn_tflops / tfl, "peak_kind": peak_kind,
+                         "traffic": None},
+            "rows": rows,
+            "clocks": clk,
+            "gpu_launches": pipe.launches_per_step * args.steps,
+            "wall_s_timed_region": wall,
+            "e2e": e2e,
+        }
+        if not args.no_cpu_baseline:
+            line["cpu_baseline"] = cpu_baseline(w)
+        print(json.dumps(line), flush=True)
+    barrier(world)
+
+
+# ----------------------------------------------------------------------------
+# CPU oracle: baseline leg and reference arm
+# ----------------------------------------------------------------------------
+
+CPU_SAMPLE_T = 4096
+CPU_SAMPLE_TQ = 256
+
+
+def oracle_step_times(w):
+    """Time the oracle on a bounded sample of the workload: fit+encode+decode
+    of the first CPU_SAMPLE_T history tokens (all heads, K and V) and attention
+    (2 blocks) + merge of CPU_SAMPLE_TQ queries over them.  Returns the
+    extrapolated seconds of one full step and the raw sample times."""
+    from kv_cache_compression_head_b200 import synth
+    from oracle import oracle as O
+
+    Ts, Tqs = CPU_SAMPLE_T, CPU_SAMPLE_TQ
+    xk = synth.make_history(w, "K", max_tokens=Ts)
+    xv = synth.make_history(w, "V", max_tokens=Ts)
+    q = synth.make_queries(w, max_tokens=Tqs)
+    t0 = time.perf_counter()
+    decs = []
+    for x, bits in ((xk, w.bits_k), (xv, w.bits_v)):
+        cent = O.fit(x, w.num_centroids, w.kmeans_iters)
+        e = O.encode(x, cent, bits, w.group_size)
+        decs.append(O.decode(*e, cent, bits, w.group_size))
+    t1 = time.perf_counter()
+    edges = [Ts * i // HISTORY_BLOCKS for i in range(HISTORY_BLOCKS + 1)]
+    parts = [O.attention(q, decs[0][a:b], decs[1][a:b]) for a, b in zip(edges[:-1], edges[1:])]
+    O.lse_merge([p[0] for p in parts], [p[1] for p in parts])
+    t2 = time.perf_counter()
+    codec_s, attn_s = t1 - t0, t2 - t1
+    full = codec_s * (w.history_tokens / Ts) + attn_s * (w.history_tokens * w.query_tokens) / (Ts * Tqs)
+    return full, codec_s, attn_s
+
+
+def _omp_threads():
+    return int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
+
+
+def cpu_baseline(w):
+    full, codec_s, attn_s = oracle_step_times(w)
+    return {"value": w.history_tokens / full, "unit": UNIT, "cores": _omp_threads(), "kind": "oracle",
+            "sample": f"fit+encode+decode of {CPU_SAMPLE_T}/{w.history_tokens} history tokens (12 heads, K and V): "
+                      f"{codec_s:.2f}s; attention (2 blocks)+merge of {CPU_SAMPLE_TQ}/{w.query_tokens} queries "
+                      f"over them: {attn_s:.2f}s; scaled per history token and per query x history token",
+            "extrapolated_s_per_step": full}
+
+
+def run_reference(args):
+    rank, world, _ = dist_env()
+    if world > 1:
+        init_dist(world, "gloo")
+    if rank != 0:
+        barrier(world)
+        return
+    from kv_cache_compression_head_b200 import synth
+
+    w = synth.workload(WORKLOAD)
+    for _ in range(args.warmup):
+        oracle_step_times(w)
+    fulls = []
+    t_wall = time.perf_counter()
+    for _ in range(args.steps):
+        fulls.append(oracle_step_times(w)[0])
+    wall = time.perf_counter() - t_wall
+    s = statistics.mean(fulls)
+    value = w.history_tokens / s
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": s * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f32/f64 (CPU oracle)", "data": "synthetic",
+        "config": {"workload": "wan13b-like layer (bounded sample per step, extrapolated)",
+                   "history_tokens": w.history_tokens, "query_tokens": w.query_tokens,
+                   "parallelism": "rank 0 only"},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": _omp_threads(), "kind": "oracle",
+                         "sample": f"each step: fit+encode+decode of {CPU_SAMPLE_T} history tokens and attention "
+                                   f"of {CPU_SAMPLE_TQ} queries over them, extrapolated to the full step"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "wall_s_timed_region": wall,
+    }
+    print(json.dumps(line), flush=True)
+    barrier(world)
+
+
+def main():
+    args = parse_args()
+    if args.warmup < 0 or args.steps < 1:
+        raise SystemExit("need --steps >= 1 and --warmup >= 0")
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_gpu(args)
+    rank, world, _ = dist_env()
+    if world > 1:
+        import torch.distributed as dist
+
+        if dist.is_initialized():
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -39,6 +39,15 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi)
     return *reinterpret_cast<uint32_t *>(&v);
 }
 
+// Two floats -> packed fp16x2 (round to nearest; out-of-range values saturate
+// to the largest finite fp16).
+__device__ __forceinline__ uint32_t pack_f16x2_sat(float lo, float hi)
+{
+    uint32_t r;
+    asm("cvt.rn.satfinite.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+    return r;
+}
+
 __device__ __forceinline__ float ex2_approx(float x)
 {
     float y;
@@ -126,16 +135,22 @@ __device__ __forceinline__ uint64_t sdesc_sw128(uint32_t saddr, uint32_t lbo, ui
            ((uint64_t)((sbo >> 4) & 0x3FFFu) << 32) | (1ull << 46) | (2ull << 61);
 }
 
-// Instruction descriptor, kind::f16 with bf16 A/B and fp32 accumulation.
-__host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, bool a_mn_major, bool b_mn_major)
+// Instruction descriptor, kind::f16 with fp32 accumulation; A and B share one
+// 16-bit type: bf16 (bf16 = true) or fp16.
+__host__ __device__ constexpr uint32_t idesc_f32acc(int M, int N, bool bf16, bool a_mn_major, bool b_mn_major)
 {
     return (1u << 4)                              // D format: f32
-           | (1u << 7)                            // A format: bf16
-           | (1u << 10)                           // B format: bf16
+           | ((bf16 ? 1u : 0u) << 7)              // A format: bf16 (1) / f16 (0)
+           | ((bf16 ? 1u : 0u) << 10)             // B format
            | ((a_mn_major ? 1u : 0u) << 15)       // A major
            | ((b_mn_major ? 1u : 0u) << 16)       // B major
            | ((uint32_t)(N >> 3) << 17)           // N / 8
            | ((uint32_t)(M >> 4) << 24);          // M / 16
+}
+
+__host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, bool a_mn_major, bool b_mn_major)
+{
+    return idesc_f32acc(M, N, true, a_mn_major, b_mn_major);
 }
 
 // D[tmem] (+)= A[smem] * B[smem]^T ; issued by one thread.

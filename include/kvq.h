@@ -133,6 +133,39 @@ KVQ_API kvq_status kvq_fit_centroids(const kvq_codec_desc *desc, const void *x, 
                              int32_t iters, void *centroids_out, void *workspace, size_t workspace_bytes,
                              kvq_stream_t stream);
 
+/* Size of the fixed device scratch behind kvq_fit_centroids_static. */
+#define KVQ_FIT_STATIC_SCRATCH_BYTES (16u << 20)
+
+/*
+ * kvq_fit_centroids without a caller-supplied workspace: the same fit, with
+ * its scratch in a fixed device array inside the library.  No passage of the
+ * pages corresponds to this call; it exists for callers that cannot
+ * allocate device memory on demand -- for example a serving runtime that
+ * reserves nearly all HBM up front for its KV cache and routes every
+ * allocation through its own pool, or a plain C caller with no allocator
+ * handle at the point of the call.  Such callers still pass x and
+ * centroids_out; nothing is allocated, and no cudaMalloc / cudaFree or
+ * allocating library routine is called.
+ *
+ *  - Limit: the scratch kvq_workspace_size(KVQ_OP_FIT, desc, T, ...) reports
+ *    must not exceed KVQ_FIT_STATIC_SCRATCH_BYTES (16 MiB: e.g. 12 heads x
+ *    32,760 tokens x 256 centres needs 3.9 MB); larger requests return
+ *    KVQ_ERR_WORKSPACE before anything is launched.
+ *  - The array is one per GPU that loads the library and is held until the
+ *    process exits.  Every call on a device shares it: two calls whose work
+ *    overlaps on that GPU (different streams, no ordering between them) race
+ *    and corrupt each other's results.  Order them on one stream or with
+ *    events.  Sums and counts are cleared at the start of every round, so
+ *    no state carries over from an earlier call.
+ *  - The first call on each device looks up the array's device address
+ *    (cudaGetSymbolAddress with that device current); make that first call
+ *    before any stream capture.
+ * Other arguments, validation and results are those of kvq_fit_centroids.
+ */
+KVQ_API kvq_status kvq_fit_centroids_static(const kvq_codec_desc *desc, const void *x, kvq_dtype x_dtype,
+                                            int64_t num_tokens, int32_t iters, void *centroids_out,
+                                            kvq_stream_t stream);
+
 /*
  * Encode one K or V history against fitted centroids.
  * Per-head codec (desc->joint_rank == 0, w_enc == NULL):

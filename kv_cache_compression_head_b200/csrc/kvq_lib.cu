@@ -259,6 +259,57 @@ kvq_status kvq_fit_centroids(const kvq_codec_desc *desc, const void *x, kvq_dtyp
     return KVQ_OK;
 }
 
+}  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Fit with a fixed device scratch array instead of a caller workspace.
+// Host code only ever uses the array's device address, looked up once per
+// device with that device current; the symbol itself is a host-side stand-in.
+// ---------------------------------------------------------------------------
+static __device__ __align__(256) unsigned char g_fit_static_scratch[KVQ_FIT_STATIC_SCRATCH_BYTES];
+
+namespace {
+
+void *fit_static_scratch(kvq_status *st)
+{
+    static void *by_device[64] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) {
+        *st = KVQ_ERR_CUDA;
+        return nullptr;
+    }
+    if (!by_device[dev]) {
+        void *p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_fit_static_scratch) != cudaSuccess || !p) {
+            *st = KVQ_ERR_CUDA;
+            return nullptr;
+        }
+        by_device[dev] = p;
+    }
+    return by_device[dev];
+}
+
+}  // namespace
+
+extern "C" {
+
+kvq_status kvq_fit_centroids_static(const kvq_codec_desc *desc, const void *x, kvq_dtype x_dtype, int64_t T,
+                                    int32_t iters, void *centroids_out, kvq_stream_t stream)
+{
+    kvq_status st = check_desc(desc, true);
+    if (st != KVQ_OK)
+        return st;
+    if (desc->joint_rank > 0 || T < 0)
+        return KVQ_ERR_INVALID_ARG;
+    if (fit_workspace(desc, T) > (size_t)KVQ_FIT_STATIC_SCRATCH_BYTES)
+        return KVQ_ERR_WORKSPACE;
+    void *scratch = fit_static_scratch(&st);
+    if (!scratch)
+        return st;
+    return kvq_fit_centroids(desc, x, x_dtype, T, iters, centroids_out, scratch, KVQ_FIT_STATIC_SCRATCH_BYTES,
+                             stream);
+}
+
 kvq_status kvq_encode(const kvq_codec_desc *desc, const void *x, kvq_dtype x_dtype, int64_t T,
                       const void *centroids, const void *w_enc, uint16_t *idx, uint8_t *codes, float *meta,
                       void *workspace, size_t workspace_bytes, kvq_stream_t stream)

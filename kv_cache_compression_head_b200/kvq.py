@@ -36,7 +36,8 @@ KVQ_OP_DECODE = 2
 KVQ_OP_ATTENTION = 3
 
 EXPORTED = (
-    "kvq_status_string", "kvq_encoded_sizes", "kvq_workspace_size", "kvq_fit_centroids", "kvq_encode",
+    "kvq_status_string", "kvq_encoded_sizes", "kvq_workspace_size", "kvq_fit_centroids",
+    "kvq_fit_centroids_static", "kvq_encode",
     "kvq_joint_coefficients", "kvq_decode", "kvq_attention_lse", "kvq_lse_merge", "kvq_last_device_status",
 )
 
@@ -70,6 +71,7 @@ def _load():
         "kvq_encoded_sizes": [pdesc, i64, ctypes.POINTER(sz), ctypes.POINTER(sz), ctypes.POINTER(sz)],
         "kvq_workspace_size": [ctypes.c_int, pdesc, i64, i64, ctypes.POINTER(sz)],
         "kvq_fit_centroids": [pdesc, vp, ctypes.c_int, i64, i32, vp, vp, sz, vp],
+        "kvq_fit_centroids_static": [pdesc, vp, ctypes.c_int, i64, i32, vp, vp],
         "kvq_encode": [pdesc, vp, ctypes.c_int, i64, vp, vp, vp, vp, vp, vp, sz, vp],
         "kvq_joint_coefficients": [pdesc, vp, ctypes.c_int, i64, vp, vp, vp, vp, vp, sz, vp],
         "kvq_decode": [pview, vp, ctypes.c_int, vp, sz, vp],
@@ -197,6 +199,15 @@ def kvq_fit_centroids(codec: Codec, x: torch.Tensor, iters: int, centroids_out: 
     _check(_lib.kvq_fit_centroids(ctypes.byref(d), _ptr(x), _dtype_code(x), T, iters, _ptr(centroids_out),
                                   _ptr(workspace), workspace.numel() if workspace is not None else 0,
                                   _stream(stream)), "kvq_fit_centroids")
+    return centroids_out
+
+
+def kvq_fit_centroids_static(codec: Codec, x: torch.Tensor, iters: int, centroids_out: torch.Tensor,
+                             stream=None) -> torch.Tensor:
+    """kvq_fit_centroids with the library's fixed device scratch (no workspace)."""
+    d = codec.c()
+    _check(_lib.kvq_fit_centroids_static(ctypes.byref(d), _ptr(x), _dtype_code(x), x.shape[0], iters,
+                                         _ptr(centroids_out), _stream(stream)), "kvq_fit_centroids_static")
     return centroids_out
 
 

@@ -93,6 +93,25 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity)
     return ok != 0;
 }
 
+// Arrive on an mbarrier and announce `bytes` of asynchronous transfer that
+// the current phase must also wait for.
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t bytes)
+{
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
+}
+
+// TMA tiled load of a 3-D box (coordinates innermost first) into shared
+// memory, completing `bytes` on the mbarrier.  `tmap` is the generic address
+// of a __grid_constant__ CUtensorMap.  No multicast.
+__device__ __forceinline__ void tma_load_3d(uint32_t dst, const void *tmap, uint32_t bar, int c0, int c1, int c2)
+{
+    asm volatile(
+        "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], "
+        "[%5];" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(tmap)), "r"(c0), "r"(c1), "r"(c2), "r"(bar)
+        : "memory");
+}
+
 // Bounded wait for phase `parity` of an mbarrier.  On expiry the device status
 // word records a timeout and false is returned; callers then stop issuing work.
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity)

@@ -1,0 +1,380 @@
+// encode_filter.cuh -- nearest-centroid assignment + residual quantisation with
+// a tensor-core distance filter (bf16 history, C <= 512 centres per head).
+//
+// Method: QuantWM: Temporally Consistent 2-Bit KV Cache Quantization for
+// Video World Models, Sec. 4.1 (nearest centroid, then residual
+// quantisation); TempoKV, Sec. 3.1 Eq. 1 (quantiser).  The result is
+// bit-identical to the exact kernel in codec.cuh: the tensor cores only narrow
+// the search, the decision is taken by the specified binary32 distance.
+//
+// For a tile of 128 tokens of head h:
+//   1. TMA loads the tile X [128][d] (bf16, 128-byte swizzle) from [T][H][d];
+//   2. one thread issues P = X mu^T (M=128, N=C, K=d, fp32 in TMEM); the
+//      centres of the head stay resident in shared memory for every tile the
+//      CTA processes;
+//   3. two threads per token (one per half of the TMEM columns and of the
+//      channels) compute v_j = |mu_j|^2 - 2 p_j, the row minimum m and the
+//      candidate window  v_j <= m + kappa (|x| + max_j |mu_j|)^2,  which
+//      provably contains the specified argmin: kappa covers the tensor-core
+//      accumulation error, the rounding of |mu_j|^2 and of v_j, and the
+//      rounding of the specified distance.  A single candidate is the
+//      answer; otherwise the candidates are re-scored with the specified
+//      distance (lowest index wins ties);
+//   4. the residual against the chosen centre is quantised (Eq. 1) per group
+//      and packed, each thread covering its half of the channels.
+#pragma once
+
+#include <cuda.h>
+
+#include "codec.cuh"
+#include "common.cuh"
+
+namespace kvq {
+
+constexpr int kFltRows = 128;
+constexpr int kFltThreads = 256;
+constexpr int kFltMaxC = 512;
+
+struct FilterArgs {
+    int64_t T;
+    int H;
+    int C;
+    int Cpad;          // C rounded up to a multiple of 32
+    int tmem_cols;     // power of two >= max(32, Cpad)
+    const uint16_t *cent;
+    uint16_t *idx;
+    uint8_t *codes;
+    float *meta;
+    int assign_only;
+    float kappa;       // window = kappa * (|x| + M)^2
+};
+
+__host__ __device__ constexpr uint32_t flt_smem_bytes(int D, int Cpad)
+{
+    // X tile | centres | norms | pair exchange (2 x 128 x 16 B) | 2 barriers + slots
+    return (uint32_t)(D * 2 * kFltRows) + (uint32_t)(Cpad * D * 2) + (uint32_t)(Cpad * 4) + 4096u + 64u;
+}
+
+// Specified binary32 distance of row `row` of the X tile to centre j of the
+// resident centre tile (both 128-byte swizzled bf16).
+template <int D>
+__device__ __forceinline__ float spec_distance_smem(const uint8_t *sX, const uint8_t *sMu, int Cpad, int row, int j)
+{
+    float acc = 0.0f;
+#pragma unroll 2
+    for (int u = 0; u < D / 8; ++u) {
+        const uint4 xw = *reinterpret_cast<const uint4 *>(sX + sw128_unit_offset(row, u, kFltRows));
+        const uint4 mw = *reinterpret_cast<const uint4 *>(sMu + sw128_unit_offset(j, u, Cpad));
+        const uint32_t xa[4] = {xw.x, xw.y, xw.z, xw.w}, ma[4] = {mw.x, mw.y, mw.z, mw.w};
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            float e = __fsub_rn(bf16_lo(xa[k]), bf16_lo(ma[k]));
+            acc = __fadd_rn(acc, __fmul_rn(e, e));
+            e = __fsub_rn(bf16_hi(xa[k]), bf16_hi(ma[k]));
+            acc = __fadd_rn(acc, __fmul_rn(e, e));
+        }
+    }
+    return acc;
+}
+
+// Residual r = x - mu[best] of channels [half*CH, half*CH + CH) of one token,
+// read from the swizzled tiles, quantised per group (Eq. 1) and packed.  Two
+// passes over shared memory (min/max, then codes) keep r out of registers.
+// Group min/max use strict comparisons in channel order, as specified.
+template <int CH, int BITS, int G>
+__device__ __forceinline__ void encode_residual_smem(const uint8_t *sX, const uint8_t *sMu, int Cpad, int row,
+                                                     int best, int half, uint8_t *codes_dst, float2 *meta_dst)
+{
+    constexpr int kPerWord = 32 / BITS;
+    constexpr int kWords = CH * BITS / 32;
+    uint32_t words[kWords];
+#pragma unroll
+    for (int w = 0; w < kWords; ++w)
+        words[w] = 0u;
+#pragma unroll
+    for (int g = 0; g < CH / G; ++g) {
+        float mn = 0.0f, mx = 0.0f;
+#pragma unroll
+        for (int uu = 0; uu < G / 8; ++uu) {
+            const int u = half * (CH / 8) + g * (G / 8) + uu;
+            const uint4 xw = *reinterpret_cast<const uint4 *>(sX + sw128_unit_offset(row, u, kFltRows));
+            const uint4 mw = *reinterpret_cast<const uint4 *>(sMu + sw128_unit_offset(best, u, Cpad));
+            const uint32_t xa[4] = {xw.x, xw.y, xw.z, xw.w}, ma[4] = {mw.x, mw.y, mw.z, mw.w};
+#pragma unroll
+            for (int k = 0; k < 8; ++k) {
+                const float r = __fsub_rn((k & 1) ? bf16_hi(xa[k >> 1]) : bf16_lo(xa[k >> 1]),
+                                          (k & 1) ? bf16_hi(ma[k >> 1]) : bf16_lo(ma[k >> 1]));
+                if (uu == 0 && k == 0) {
+                    mn = r;
+                    mx = r;
+                } else {
+                    if (r < mn) mn = r;
+                    if (r > mx) mx = r;
+                }
+            }
+        }
+        const GroupQ gq = group_params(mn, mx, BITS);
+        meta_dst[g] = make_float2(gq.s, gq.z);
+#pragma unroll
+        for (int uu = 0; uu < G / 8; ++uu) {
+            const int u = half * (CH / 8) + g * (G / 8) + uu;
+            const uint4 xw = *reinterpret_cast<const uint4 *>(sX + sw128_unit_offset(row, u, kFltRows));
+            const uint4 mw = *reinterpret_cast<const uint4 *>(sMu + sw128_unit_offset(best, u, Cpad));
+            const uint32_t xa[4] = {xw.x, xw.y, xw.z, xw.w}, ma[4] = {mw.x, mw.y, mw.z, mw.w};
+#pragma unroll
+            for (int k = 0; k < 8; ++k) {
+                const float r = __fsub_rn((k & 1) ? bf16_hi(xa[k >> 1]) : bf16_lo(xa[k >> 1]),
+                                          (k & 1) ? bf16_hi(ma[k >> 1]) : bf16_lo(ma[k >> 1]));
+                const int c = g * G + uu * 8 + k;
+                words[c / kPerWord] |= quant_code(r, gq, BITS) << ((c % kPerWord) * BITS);
+            }
+        }
+    }
+    if constexpr (kWords >= 4) {
+        uint4 *dst = reinterpret_cast<uint4 *>(codes_dst);
+#pragma unroll
+        for (int v = 0; v < kWords / 4; ++v)
+            dst[v] = make_uint4(words[4 * v], words[4 * v + 1], words[4 * v + 2], words[4 * v + 3]);
+    } else {
+        uint32_t *dst = reinterpret_cast<uint32_t *>(codes_dst);
+#pragma unroll
+        for (int v = 0; v < kWords; ++v)
+            dst[v] = words[v];
+    }
+}
+
+template <int D, int BITS, int G>
+__global__ void __launch_bounds__(kFltThreads, 2)
+    encode_filter_kernel(const __grid_constant__ CUtensorMap tmap_x, FilterArgs a)
+{
+    static_assert(G <= D / 2, "a group must lie inside one half of the channels");
+    constexpr int CH = D / 2;             // channels per thread
+    constexpr int kMaxChunks = kFltMaxC / 32 / 2;
+
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const int Cpad = a.Cpad;
+    uint8_t *sX = smem;
+    uint8_t *sMu = smem + D * 2 * kFltRows;
+    float *sNrm = reinterpret_cast<float *>(sMu + Cpad * D * 2);
+    float4 *sPair = reinterpret_cast<float4 *>(sNrm + Cpad);  // [2][128]
+    uint64_t *bars = reinterpret_cast<uint64_t *>(reinterpret_cast<uint8_t *>(sPair) + 4096);
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 2);
+    uint32_t *sMaxNrm = tmem_slot + 1;
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int half = warp >> 2;
+    const int row = (warp & 3) * 32 + lane;
+    const int h = blockIdx.y;
+    const uint32_t bar_x = smem_u32(bars), bar_m = smem_u32(bars + 1);
+
+    if (warp == 0)
+        tmem_alloc(smem_u32(tmem_slot), a.tmem_cols);
+    if (tid == 0) {
+        mbar_init(bar_x, 1);
+        mbar_init(bar_m, 1);
+        fence_mbar_init();
+        *sMaxNrm = 0u;
+    }
+    __syncthreads();
+
+    // centres of head h -> swizzled K-major tile [D/64][Cpad][128 B]; norms
+    const uint16_t *cent_h = a.cent + (int64_t)h * a.C * D;
+    for (int e = tid; e < Cpad * (D / 8); e += kFltThreads) {
+        const int j = e / (D / 8), u = e % (D / 8);
+        const uint4 w = j < a.C ? __ldg(reinterpret_cast<const uint4 *>(cent_h + (int64_t)j * D) + u)
+                                : make_uint4(0, 0, 0, 0);
+        *reinterpret_cast<uint4 *>(sMu + sw128_unit_offset(j, u, Cpad)) = w;
+    }
+    for (int j = tid; j < Cpad; j += kFltThreads) {
+        float nrm = INFINITY;
+        if (j < a.C) {
+            nrm = 0.0f;
+            for (int u = 0; u < D / 8; ++u) {
+                float m8[8];
+                load_bf16x8(cent_h + (int64_t)j * D + u * 8, m8);
+#pragma unroll
+                for (int k = 0; k < 8; ++k)
+                    nrm = fmaf(m8[k], m8[k], nrm);
+            }
+            atomicMax(sMaxNrm, __float_as_uint(nrm));
+        }
+        sNrm[j] = nrm;
+    }
+    fence_proxy_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    const float Mnorm = sqrtf(__uint_as_float(*sMaxNrm));
+    const uint32_t lane_off = ((uint32_t)(warp & 3) * 32u) << 16;
+    const uint32_t aX = smem_u32(sX), aMu = smem_u32(sMu);
+
+    // this thread's 32-column chunks of the TMEM row
+    const int nchunks = Cpad / 32;
+    const int c_lo = half == 0 ? 0 : (nchunks + 1) / 2;
+    const int c_hi = half == 0 ? (nchunks + 1) / 2 : nchunks;
+
+    const int64_t ntiles = (a.T + kFltRows - 1) / kFltRows;
+    uint32_t ph_x = 0, ph_m = 0;
+    bool ok = true;
+    for (int64_t tile = blockIdx.x; tile < ntiles; tile += gridDim.x) {
+        const int64_t t0 = tile * kFltRows;
+        if (tid == 0) {
+            mbar_arrive_expect_tx(bar_x, D * 2 * kFltRows);
+#pragma unroll
+            for (int ch = 0; ch < D / 64; ++ch)
+                tma_load_3d(aX + ch * (kFltRows * 128), &tmap_x, bar_x, ch * 64, h, (int)t0);
+        }
+        ok = mbar_wait(bar_x, ph_x) && ok;
+        ph_x ^= 1u;
+        if (tid == 0) {
+            tc_fence_after();
+            for (int n0 = 0; n0 < Cpad; n0 += 256) {
+                const int N = min(256, Cpad - n0);
+                const uint32_t idesc = idesc_f32acc(128, N, true, false, false);
+#pragma unroll
+                for (int ks = 0; ks < D / 16; ++ks) {
+                    const uint32_t aoff = (uint32_t)(ks >> 2) * (kFltRows * 128u) + (uint32_t)(ks & 3) * 32u;
+                    const uint32_t boff =
+                        (uint32_t)(ks >> 2) * (uint32_t)(Cpad * 128) + (uint32_t)n0 * 128u + (uint32_t)(ks & 3) * 32u;
+                    umma_ss(tmem + (uint32_t)n0, sdesc_sw128(aX + aoff, 16, 1024), sdesc_sw128(aMu + boff, 16, 1024),
+                            idesc, ks > 0 ? 1u : 0u);
+                }
+            }
+            umma_commit(bar_m);
+        }
+        ok = mbar_wait(bar_m, ph_m) && ok;
+        ph_m ^= 1u;
+        tc_fence_after();
+
+        // (1) |x|^2 over this thread's channel half
+        float xx = 0.0f;
+#pragma unroll
+        for (int u = half * (CH / 8); u < (half + 1) * (CH / 8); ++u) {
+            const uint4 w = *reinterpret_cast<const uint4 *>(sX + sw128_unit_offset(row, u, kFltRows));
+            const uint32_t wa[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                xx = fmaf(bf16_lo(wa[k]), bf16_lo(wa[k]), xx);
+                xx = fmaf(bf16_hi(wa[k]), bf16_hi(wa[k]), xx);
+            }
+        }
+        // (2) v_j = |mu_j|^2 - 2 p_j over this thread's chunks: per-chunk minima
+        float cmin[kMaxChunks];
+        float tmin = INFINITY;
+#pragma unroll
+        for (int k = 0; k < kMaxChunks; ++k) {
+            cmin[k] = INFINITY;
+            const int c = c_lo + k;
+            if (c < c_hi) {
+                float p[32];
+                tmem_ld32(tmem + lane_off + (uint32_t)(c * 32), p);
+                float mn = INFINITY;
+#pragma unroll
+                for (int i = 0; i < 32; ++i)
+                    mn = fminf(mn, fmaf(-2.0f, p[i], sNrm[c * 32 + i]));
+                cmin[k] = mn;
+                tmin = fminf(tmin, mn);
+            }
+        }
+        sPair[half * 128 + row] = make_float4(xx, tmin, 0.f, 0.f);
+        __syncthreads();
+        const float4 other = sPair[(half ^ 1) * 128 + row];
+        const float m = fminf(tmin, other.y);
+        const float xn = sqrtf(xx + other.x);
+        const float thr = m + a.kappa * (xn + Mnorm) * (xn + Mnorm);
+        // (3) candidates inside the window.  tcgen05.ld is warp-collective, so
+        // a chunk is re-read when any lane of the warp needs it.
+        int count = 0, first = -1;
+#pragma unroll
+        for (int k = 0; k < kMaxChunks; ++k) {
+            const int c = c_lo + k;
+            const bool need = c < c_hi && cmin[k] <= thr;
+            if (c < c_hi && __any_sync(0xffffffffu, need)) {
+                float p[32];
+                tmem_ld32(tmem + lane_off + (uint32_t)(c * 32), p);
+                if (need) {
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) {
+                        const float v = fmaf(-2.0f, p[i], sNrm[c * 32 + i]);
+                        if (v <= thr) {
+                            if (count == 0)
+                                first = c * 32 + i;
+                            ++count;
+                        }
+                    }
+                }
+            }
+        }
+        __syncthreads();  // both halves have read sPair
+        sPair[half * 128 + row] = make_float4(__int_as_float(count), __int_as_float(first), 0.f, 0.f);
+        __syncthreads();
+        const float4 o2 = sPair[(half ^ 1) * 128 + row];
+        const int count_all = count + __float_as_int(o2.x);
+        int best = half == 0 ? (count > 0 ? first : __float_as_int(o2.y))
+                             : (__float_as_int(o2.x) > 0 ? __float_as_int(o2.y) : first);
+        const bool exact = count_all != 1 || !(thr < INFINITY);
+        __syncthreads();  // both halves have read the counts
+        // rare: re-score the window (or every centre when the window is not
+        // finite) with the specified distance; the half-0 thread decides.  The
+        // warp reads TMEM together whenever one of its rows needs this.
+        if (half == 0 && __any_sync(0xffffffffu, exact)) {
+            float bd = INFINITY;
+            int bj = -1;
+            const bool all = !(thr < INFINITY);
+            for (int c = 0; c < nchunks; ++c) {
+                float p[32];
+                tmem_ld32(tmem + lane_off + (uint32_t)(c * 32), p);
+                uint32_t cand = 0u;
+#pragma unroll
+                for (int i = 0; i < 32; ++i) {
+                    const int j = c * 32 + i;
+                    const float v = fmaf(-2.0f, p[i], sNrm[j]);
+                    if (exact && j < a.C && (all || v <= thr))
+                        cand |= 1u << i;
+                }
+                while (cand) {  // increasing index order
+                    const int i = __ffs(cand) - 1;
+                    cand &= cand - 1u;
+                    const int j = c * 32 + i;
+                    const float dj = spec_distance_smem<D>(sX, sMu, Cpad, row, j);
+                    if (bj < 0 || dj < bd) {
+                        bd = dj;
+                        bj = j;
+                    }
+                }
+            }
+            if (exact)
+                sPair[row] = make_float4(__int_as_float(bj), 0.f, 0.f, 0.f);
+        }
+        __syncthreads();
+        if (exact)
+            best = __float_as_int(sPair[row].x);
+        if (best < 0 || best >= a.C)
+            best = 0;  // unreachable for finite inputs
+
+        // (4) residual + Eq. 1 + packing for this thread's channel half
+        const int64_t t = t0 + row;
+        if (t < a.T) {
+            const int64_t th = (int64_t)h * a.T + t;
+            if (half == 0)
+                a.idx[th] = (uint16_t)best;
+            if (!a.assign_only)
+                encode_residual_smem<CH, BITS, G>(sX, sMu, Cpad, row, best, half,
+                                                  a.codes + th * (D * BITS / 8) + half * (CH * BITS / 8),
+                                                  reinterpret_cast<float2 *>(a.meta) + th * (D / G) + half * (CH / G));
+        }
+        tc_fence_before();
+        ok = __syncthreads_and(ok) != 0;
+        if (!ok)
+            break;
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 0)
+        tmem_dealloc(tmem, a.tmem_cols);
+}
+
+}  // namespace kvq

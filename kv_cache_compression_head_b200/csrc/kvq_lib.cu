@@ -1,12 +1,16 @@
 // kvq_lib.cu -- the C ABI of libkvq (declared in include/kvq.h): argument
 // validation, workspace accounting and kernel launches.  Built as a single
 // translation unit for sm_100a.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <math.h>
 #include <stdint.h>
 #include <string.h>
 
 #include "attention.cuh"
 #include "codec.cuh"
 #include "common.cuh"
+#include "encode_filter.cuh"
 #include "merge.cuh"
 
 using namespace kvq;
@@ -72,6 +76,140 @@ kvq_status launch_encode_direct(int D, const EncodeArgs &a, cudaStream_t s)
     if (D == 128)
         return a.bits == 2 ? launch_encode_direct_g<128, 2>(a, s) : launch_encode_direct_g<128, 4>(a, s);
     return a.bits == 2 ? launch_encode_direct_g<64, 2>(a, s) : launch_encode_direct_g<64, 4>(a, s);
+}
+
+// ---------------------------------------------------------------------------
+// tensor-core filtered encode (bf16 history, C <= 512, G <= d/2)
+// ---------------------------------------------------------------------------
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder()
+{
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    if (!fn) {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) != cudaSuccess ||
+            q != cudaDriverEntryPointSuccess)
+            return nullptr;
+        fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    }
+    return fn;
+}
+
+// 3-D map of a [T][H][D] bf16 history: box = 64 channels x 1 head x 128 tokens,
+// 128-byte swizzle (the K-major operand layout), zero fill past T.
+bool make_history_map(CUtensorMap *m, const void *x, int64_t T, int H, int D)
+{
+    PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
+    if (!enc)
+        return false;
+    cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)H, (cuuint64_t)T};
+    cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)H * D * 2};
+    cuuint32_t box[3] = {64, 1, (cuuint32_t)kFltRows};
+    cuuint32_t estr[3] = {1, 1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(x), dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+int sm_count()
+{
+    int dev = 0, n = 148;
+    if (cudaGetDevice(&dev) == cudaSuccess)
+        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    return n;
+}
+
+bool filter_applies(int D, int C, int G, bool x_bf16)
+{
+    return x_bf16 && C <= kFltMaxC && G <= D / 2 && (D == 64 || D == 128);
+}
+
+template <int D, int BITS, int G>
+kvq_status launch_filter_t(const CUtensorMap &m, const FilterArgs &a, cudaStream_t s)
+{
+    const uint32_t smem = flt_smem_bytes(D, a.Cpad) + 1024;
+    static bool configured[64] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64)
+        return KVQ_ERR_CUDA;
+    if (!configured[dev]) {
+        if (cudaFuncSetAttribute(encode_filter_kernel<D, BITS, G>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 227 * 1024) != cudaSuccess)
+            return KVQ_ERR_CUDA;
+        configured[dev] = true;
+    }
+    // CTAs per SM: bounded by shared memory and by TMEM (512 columns)
+    const int by_smem = (int)((228u * 1024u) / (smem + 1024u));
+    const int by_tmem = 512 / a.tmem_cols;
+    const int per_sm = max(1, min(min(by_smem, by_tmem), 8));
+    const int64_t ntiles = (a.T + kFltRows - 1) / kFltRows;
+    const int64_t want = ((int64_t)per_sm * sm_count() + a.H - 1) / a.H;
+    const int64_t gx64 = ntiles < want ? ntiles : want;
+    const unsigned gx = (unsigned)(gx64 > 0 ? gx64 : 1);
+    encode_filter_kernel<D, BITS, G><<<dim3(gx, (unsigned)a.H), kFltThreads, smem, s>>>(m, a);
+    return launch_status();
+}
+
+template <int D, int BITS>
+kvq_status launch_filter_g(int G, const CUtensorMap &m, const FilterArgs &a, cudaStream_t s)
+{
+    switch (G) {
+    case 16: return launch_filter_t<D, BITS, 16>(m, a, s);
+    case 32: return launch_filter_t<D, BITS, 32>(m, a, s);
+    case 64:
+        if constexpr (D >= 128)
+            return launch_filter_t<D, BITS, 64>(m, a, s);
+        return KVQ_ERR_UNSUPPORTED;
+    default: return KVQ_ERR_UNSUPPORTED;
+    }
+}
+
+// Window factor of the certified candidate set (see encode_filter.cuh):
+// kappa = 4 (eps_tc + gamma_d + 2u + gamma_{d+2}), eps_tc = d 2^-21 bounding
+// the tensor-core accumulation error relative to sum |x_c mu_c|.
+float filter_kappa(int D)
+{
+    const double u = ldexp(1.0, -24);
+    const double eps_tc = D * ldexp(1.0, -21);
+    const double g_d = D * u / (1.0 - D * u), g_d2 = (D + 2) * u / (1.0 - (D + 2) * u);
+    return (float)(4.0 * (eps_tc + g_d + 2.0 * u + g_d2));
+}
+
+kvq_status launch_encode_filter(int D, int bits, int G, const void *x, const EncodeArgs &e, cudaStream_t s)
+{
+    CUtensorMap m;
+    if (!make_history_map(&m, x, e.T, e.H, D))
+        return KVQ_ERR_CUDA;
+    FilterArgs a;
+    a.T = e.T;
+    a.H = e.H;
+    a.C = e.C;
+    a.Cpad = (e.C + 31) / 32 * 32;
+    int cols = 32;
+    while (cols < a.Cpad)
+        cols <<= 1;
+    a.tmem_cols = cols;
+    a.cent = e.cent;
+    a.idx = e.idx;
+    a.codes = e.codes;
+    a.meta = e.meta;
+    a.assign_only = e.assign_only;
+    a.kappa = filter_kappa(D);
+    if (D == 128)
+        return bits == 2 ? launch_filter_g<128, 2>(G, m, a, s) : launch_filter_g<128, 4>(G, m, a, s);
+    return bits == 2 ? launch_filter_g<64, 2>(G, m, a, s) : launch_filter_g<64, 4>(G, m, a, s);
+}
+
+// Assignment (+ residual quantisation unless assign_only): the filtered
+// tensor-core kernel where it applies, else the exact CUDA-core kernel.  Both
+// produce identical results.
+kvq_status launch_encode(int D, const EncodeArgs &e, cudaStream_t s)
+{
+    if (e.T == 0)
+        return KVQ_OK;
+    if (filter_applies(D, e.C, e.G, e.x_bf16 != 0))
+        return launch_encode_filter(D, e.bits, e.G, e.x, e, s);
+    return launch_encode_direct(D, e, s);
 }
 
 size_t fit_workspace(const kvq_codec_desc *d, int64_t T)
@@ -245,7 +383,7 @@ kvq_status kvq_fit_centroids(const kvq_codec_desc *desc, const void *x, kvq_dtyp
     e.assign_only = 1;
     const int64_t n_units = T * H * (D / 8);
     for (int it = 0; it < iters; ++it) {
-        if ((st = launch_encode_direct(D, e, s)) != KVQ_OK)
+        if ((st = launch_encode(D, e, s)) != KVQ_OK)
             return st;
         if (cudaMemsetAsync(ws + idx_b, 0, cnt_b + (size_t)H * C * D * 8, s) != cudaSuccess)
             return KVQ_ERR_CUDA;
@@ -343,7 +481,7 @@ kvq_status kvq_encode(const kvq_codec_desc *desc, const void *x, kvq_dtype x_dty
     e.codes = codes;
     e.meta = meta;
     e.assign_only = 0;
-    return launch_encode_direct(desc->head_dim, e, reinterpret_cast<cudaStream_t>(stream));
+    return launch_encode(desc->head_dim, e, reinterpret_cast<cudaStream_t>(stream));
 }
 
 kvq_status kvq_joint_coefficients(const kvq_codec_desc *desc, const void *x, kvq_dtype x_dtype, int64_t T,

@@ -323,3 +323,31 @@ def test_identical_tokens_and_constant_groups():
         _assert_encoded_equal(comp, H, T, d, bits, G, *e)
         assert np.all(e[1][:, :, : 64 * bits // 8] == 0) and np.all(e[2][:, :, : 64 // G] == 0)
     _status_ok()
+
+
+def test_encode_ties_and_near_ties():
+    """Duplicated centres (exact ties) and tokens half-way between two centres:
+    the tensor-core filter's window then holds several candidates and the
+    specified distance decides, lowest index first."""
+    K = _K()
+    rng = np.random.default_rng(41)
+    H, d, C, T = 2, 128, 64, 700
+    base = rng.integers(-4, 5, size=(H, C // 2, d)).astype(np.float64)
+    cent = _bf16_bits(np.concatenate([base, base], axis=1))  # centre j == centre j + 32
+    cf = synth.bf16_bits_to_f32(cent).astype(np.float64)
+    x = rng.normal(size=(T, H, d)) * 2
+    for t in range(0, T, 3):  # midpoints of centre pairs (exact in bf16: half-integers)
+        for h in range(H):
+            a, b = rng.choice(C // 2, size=2, replace=False)
+            x[t, h] = 0.5 * (cf[h, a] + cf[h, b])
+    for t in range(1, T, 7):  # exactly on a centre
+        for h in range(H):
+            x[t, h] = cf[h, rng.integers(C)]
+    x = _bf16_bits(x)
+    for bits, G in ((2, 16), (4, 32)):
+        codec = K.Codec(H, d, C, bits, G)
+        e = O.encode(x, cent, bits, G)
+        comp = _gpu_encode(codec, x, cent)
+        _assert_encoded_equal(comp, H, T, d, bits, G, *e)
+        assert np.all(e[0] < C // 2)  # ties resolved to the lower duplicate
+    _status_ok()

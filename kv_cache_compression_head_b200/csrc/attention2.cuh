@@ -1,0 +1,432 @@
+// attention2.cuh -- warp-specialised attention over a compressed K/V history
+// (tcgen05 / TMEM), two 128-row query tiles per CTA.
+//
+// Method: NanoKV page, Fig. 4(a,d) (history read through the decoder: centres
+// added back to the dequantised residual; partial results carry their
+// log-sum-exp); QuantWM, Fig. 9 (on-demand reconstruction during attention).
+//
+// Roles (416 threads):
+//   warps 0-3  producer: load the two Q tiles, then for every 128-token history
+//              tile rebuild k^ (bf16 hi + lo tiles) and v^ (fp16 tile) from
+//              codes, {s, z}, idx and the bf16 centres straight into the
+//              128-byte-swizzled operand layout; one thread per history row.
+//   warp 4     MMA issuer (one thread): S_i = Q_i K_hi^T + Q_i K_lo^T into
+//              TMEM for both query tiles, then O_i += P_i V^ (fp16) once the
+//              softmax has published P_i.
+//   warps 5-8  softmax for query tile 0, warps 9-12 for query tile 1: one
+//              thread per query row (its TMEM lane); online softmax in the
+//              exp2 domain with lazy rescaling (O in TMEM is rescaled only when
+//              the running maximum grows by more than 2^8); P (fp16) goes to
+//              the shared buffers of the K stage the tile came from.
+// Shared memory: Q tiles 2 x 32 KB, two K stages of 2 x 32 KB (K_hi, K_lo,
+// later P_0, P_1), one V tile of 32 KB (d = 128).  TMEM: S_0, S_1 (128 columns
+// each) and O_0, O_1 (d columns each).
+//
+// Ordering (mbarriers; parity = use count & 1):
+//   kfull[s]  producer -> MMA   K stage s holds tile j (j = s mod 2)
+//   vfull     producer -> MMA   V tile j written
+//   sfull[i]  MMA -> softmax    S_i(j) complete.  The QK MMAs run hi(0),
+//             hi(1), lo(0), lo(1), so S_0 completes after K_hi's last read and
+//             S_1 after K_lo's: each P_i can overwrite its slot at once
+//   pfull[i]  softmax -> MMA    P_i(j) written, O_i rescaled
+//   pvdone    MMA -> producer   PV_0(j), PV_1(j) complete: V and K stage j free
+//   ofull     MMA -> softmax    last PV complete
+// Every wait is bounded and also polls a shared abort flag, so that one
+// role giving up releases the others; the MMA thread drains its tcgen05 work
+// before TMEM is freed.
+#pragma once
+
+#include "attention.cuh"
+#include "codec.cuh"
+#include "common.cuh"
+
+namespace kvq {
+
+constexpr int kA2Threads = 416;
+constexpr int kA2Rows = 256;  // query rows per CTA (two tiles)
+
+template <int D>
+struct A2Smem {
+    static constexpr uint32_t kQ = D * 2 * 128;
+    static constexpr uint32_t kKt = D * 2 * 128;           // one K_hi / K_lo tile
+    static constexpr uint32_t kPt = 2 * 128 * 128;         // one P tile (fp16)
+    static constexpr uint32_t kSlot = kKt > kPt ? kKt : kPt;
+    static constexpr uint32_t offQ0 = 0, offQ1 = kQ;
+    static constexpr uint32_t offStage = 2 * kQ;          // stage s slot t at offStage + (2s + t) kSlot
+    static constexpr uint32_t offV = offStage + 4 * kSlot;
+    static constexpr uint32_t offBar = offV + kKt;
+    static constexpr uint32_t kBytes = offBar + 128;
+    static constexpr uint32_t kLaunchBytes = kBytes + 1024;
+};
+
+enum { B_QREADY = 0, B_KFULL0, B_KFULL1, B_VFULL, B_SFULL0, B_SFULL1, B_PFULL0, B_PFULL1, B_PVDONE, B_OFULL, B_COUNT };
+
+// Bounded wait that also gives up when another role has raised `abort`.
+__device__ __forceinline__ bool a2_wait(uint32_t bar, uint32_t parity, volatile int *abort)
+{
+    for (uint32_t i = 0; i < kSpinLimit; ++i) {
+        if (mbar_try_wait(bar, parity))
+            return true;
+        if ((i & 255u) == 255u && *abort)
+            return false;
+    }
+    raise_status(DEVSTAT_TIMEOUT);
+    *abort = 1;
+    return false;
+}
+
+__device__ __forceinline__ void mbar_arrive(uint32_t bar)
+{
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+
+// Rebuild history row `tok` of a compressed K (SPLIT: bf16 hi + lo tiles) or
+// V (fp16 tile) into the swizzled tiles.  k^ = fma(f, 2^b s, mu - (2^b + z) s)
+// with f = 1 + q 2^-b built directly in the float's mantissa, the decoder's
+// value up to one rounding.
+template <int D, bool SPLIT>
+__device__ __forceinline__ void a2_dequant_row(const CodecView &cv, int h, int64_t tok, bool valid, uint8_t *tile,
+                                               uint8_t *tile_lo, uint32_t row)
+{
+    if (!valid) {
+#pragma unroll
+        for (int u = 0; u < D / 8; ++u) {
+            *reinterpret_cast<uint4 *>(tile + sw128_unit_offset(row, u, 128)) = make_uint4(0, 0, 0, 0);
+            if (SPLIT)
+                *reinterpret_cast<uint4 *>(tile_lo + sw128_unit_offset(row, u, 128)) = make_uint4(0, 0, 0, 0);
+        }
+        return;
+    }
+    const int64_t th = (int64_t)h * cv.T + tok;
+    int j = __ldg(cv.idx + th);
+    if (j >= cv.C) {
+        raise_status(DEVSTAT_BAD_INDEX);
+        j = 0;
+    }
+    const uint4 *mu_row = reinterpret_cast<const uint4 *>(cv.cent + ((int64_t)h * cv.C + j) * D);
+    const float2 *meta_row = reinterpret_cast<const float2 *>(cv.meta) + th * (D / cv.G);
+    const int bits = cv.bits;
+    const float two_b = (float)(1 << bits);
+    const uint32_t qshift = 23u - (uint32_t)bits;
+    const uint32_t qmask = ((1u << bits) - 1u) << qshift;
+#pragma unroll 4
+    for (int u = 0; u < D / 8; ++u) {
+        const int c0 = u * 8;
+        const float2 sz = __ldg(meta_row + c0 / cv.G);
+        const float sc = two_b * sz.x;                  // 2^b s (exact)
+        const float nb = -__fmul_rn(two_b + sz.y, sz.x); // -(2^b + z) s
+        uint32_t cw;
+        if (bits == 2)
+            cw = __ldg(reinterpret_cast<const uint16_t *>(cv.codes + th * (D / 4)) + u);
+        else
+            cw = __ldg(reinterpret_cast<const uint32_t *>(cv.codes + th * (D / 2)) + u);
+        const uint4 mw = __ldg(mu_row + u);
+        const uint32_t ma[4] = {mw.x, mw.y, mw.z, mw.w};
+        float val[8];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+            const int sh = (int)qshift - k * bits;
+            const uint32_t qb = (sh >= 0 ? (cw << sh) : (cw >> -sh)) & qmask;
+            const float f = __uint_as_float(0x3F800000u | qb);
+            const float mu = (k & 1) ? bf16_hi(ma[k >> 1]) : bf16_lo(ma[k >> 1]);
+            val[k] = fmaf(f, sc, mu + nb);
+        }
+        const uint32_t off = sw128_unit_offset(row, u, 128);
+        if (SPLIT) {
+            uint32_t hi[4], lo[4];
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                const uint32_t a0 = __float_as_uint(val[2 * k]) & 0xffff0000u;
+                const uint32_t a1 = __float_as_uint(val[2 * k + 1]) & 0xffff0000u;
+                hi[k] = (a0 >> 16) | a1;
+                lo[k] = pack_bf16x2(val[2 * k] - __uint_as_float(a0), val[2 * k + 1] - __uint_as_float(a1));
+            }
+            *reinterpret_cast<uint4 *>(tile + off) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+            *reinterpret_cast<uint4 *>(tile_lo + off) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+        } else {
+            *reinterpret_cast<uint4 *>(tile + off) =
+                make_uint4(pack_f16x2_sat(val[0], val[1]), pack_f16x2_sat(val[2], val[3]),
+                           pack_f16x2_sat(val[4], val[5]), pack_f16x2_sat(val[6], val[7]));
+        }
+    }
+}
+
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const float *v)
+{
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
+        "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
+        "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
+        "r"(__float_as_uint(v[0])), "r"(__float_as_uint(v[1])), "r"(__float_as_uint(v[2])),
+        "r"(__float_as_uint(v[3])), "r"(__float_as_uint(v[4])), "r"(__float_as_uint(v[5])),
+        "r"(__float_as_uint(v[6])), "r"(__float_as_uint(v[7])), "r"(__float_as_uint(v[8])),
+        "r"(__float_as_uint(v[9])), "r"(__float_as_uint(v[10])), "r"(__float_as_uint(v[11])),
+        "r"(__float_as_uint(v[12])), "r"(__float_as_uint(v[13])), "r"(__float_as_uint(v[14])),
+        "r"(__float_as_uint(v[15])), "r"(__float_as_uint(v[16])), "r"(__float_as_uint(v[17])),
+        "r"(__float_as_uint(v[18])), "r"(__float_as_uint(v[19])), "r"(__float_as_uint(v[20])),
+        "r"(__float_as_uint(v[21])), "r"(__float_as_uint(v[22])), "r"(__float_as_uint(v[23])),
+        "r"(__float_as_uint(v[24])), "r"(__float_as_uint(v[25])), "r"(__float_as_uint(v[26])),
+        "r"(__float_as_uint(v[27])), "r"(__float_as_uint(v[28])), "r"(__float_as_uint(v[29])),
+        "r"(__float_as_uint(v[30])), "r"(__float_as_uint(v[31]))
+        : "memory");
+    asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
+
+template <int D>
+__global__ void __maxnreg__(152) attention2_kernel(AttnArgs a)
+{
+    using L = A2Smem<D>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + L::offBar);
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + B_COUNT);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
+    auto bar = [&](int i) { return smem_u32(bars + i); };
+    auto slot = [&](int s, int t) { return smem + L::offStage + (uint32_t)(2 * s + t) * L::kSlot; };
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int h = blockIdx.y;
+    const int64_t q0 = (int64_t)blockIdx.x * kA2Rows;
+    const int64_t span = a.t_end - a.t_begin;
+    const int ntiles = (int)((span + 127) / 128);
+
+    if (warp == 0)
+        tmem_alloc(smem_u32(tmem_slot), 512);
+    if (tid == 0) {
+        mbar_init(bar(B_QREADY), 128);
+        mbar_init(bar(B_KFULL0), 128);
+        mbar_init(bar(B_KFULL1), 128);
+        mbar_init(bar(B_VFULL), 128);
+        mbar_init(bar(B_SFULL0), 1);
+        mbar_init(bar(B_SFULL1), 1);
+        mbar_init(bar(B_PFULL0), 128);
+        mbar_init(bar(B_PFULL1), 128);
+        mbar_init(bar(B_PVDONE), 1);
+        mbar_init(bar(B_OFULL), 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp < 4) {
+        // ------------------------------------------------------------ producer
+        const uint32_t r = (uint32_t)tid;
+        for (int qt = 0; qt < 2; ++qt) {
+            const int64_t qr = q0 + qt * 128 + r;
+            const bool valid = qr < a.Tq;
+            const uint16_t *src = a.q + (qr * a.H + h) * D;
+            uint8_t *dst = smem + (qt ? L::offQ1 : L::offQ0);
+#pragma unroll
+            for (int u = 0; u < D / 8; ++u) {
+                const uint4 w = valid ? __ldg(reinterpret_cast<const uint4 *>(src) + u) : make_uint4(0, 0, 0, 0);
+                *reinterpret_cast<uint4 *>(dst + sw128_unit_offset(r, u, 128)) = w;
+            }
+        }
+        fence_proxy_async_smem();
+        mbar_arrive(bar(B_QREADY));
+        if (ntiles > 0) {
+            {
+                const int64_t tok = a.t_begin + r;
+                a2_dequant_row<D, true>(a.k, h, tok, tok < a.t_end, slot(0, 0), slot(0, 1), r);
+                fence_proxy_async_smem();
+                mbar_arrive(bar(B_KFULL0));
+            }
+            for (int j = 0; j < ntiles; ++j) {
+                if (j >= 1 && !a2_wait(bar(B_PVDONE), (uint32_t)((j - 1) & 1), abort_flag))
+                    break;
+                const int64_t tok = a.t_begin + (int64_t)j * 128 + r;
+                a2_dequant_row<D, false>(a.v, h, tok, tok < a.t_end, smem + L::offV, nullptr, r);
+                fence_proxy_async_smem();
+                mbar_arrive(bar(B_VFULL));
+                if (j + 1 < ntiles) {
+                    const int s = (j + 1) & 1;
+                    const int64_t tk = tok + 128;
+                    a2_dequant_row<D, true>(a.k, h, tk, tk < a.t_end, slot(s, 0), slot(s, 1), r);
+                    fence_proxy_async_smem();
+                    mbar_arrive(bar(s ? B_KFULL1 : B_KFULL0));
+                }
+            }
+        }
+    } else if (warp == 4) {
+        // ------------------------------------------------------------ MMA issuer
+        if (lane == 0 && ntiles > 0) {
+            constexpr uint32_t idescS = idesc_f32acc(128, 128, true, false, false);
+            constexpr uint32_t idescO = idesc_f32acc(128, D, false, false, true);
+            const uint32_t aQ[2] = {smem_u32(smem + L::offQ0), smem_u32(smem + L::offQ1)};
+            const uint32_t aV = smem_u32(smem + L::offV);
+            const uint32_t tS[2] = {tmem, tmem + 128}, tO[2] = {tmem + 256, tmem + 256 + D};
+            bool ok = a2_wait(bar(B_QREADY), 0, abort_flag);
+            for (int j = 0; ok && j < ntiles; ++j) {
+                const int s = j & 1;
+                ok = a2_wait(bar(s ? B_KFULL1 : B_KFULL0), (uint32_t)((j >> 1) & 1), abort_flag);
+                if (!ok)
+                    break;
+                tc_fence_after();
+                const uint32_t aKh = smem_u32(slot(s, 0)), aKl = smem_u32(slot(s, 1));
+                // order hi(0), hi(1), lo(0), lo(1): when S_0 completes, K_hi is no
+                // longer read and can take P_0; S_1 completes last (K_lo -> P_1)
+#pragma unroll
+                for (int part = 0; part < 2; ++part) {
+#pragma unroll
+                    for (int qt = 0; qt < 2; ++qt) {
+#pragma unroll
+                        for (int ks = 0; ks < D / 16; ++ks) {
+                            const uint32_t off = (uint32_t)(ks >> 2) * (128u * 128u) + (uint32_t)(ks & 3) * 32u;
+                            umma_ss(tS[qt], sdesc_sw128(aQ[qt] + off, 16, 1024),
+                                    sdesc_sw128((part ? aKl : aKh) + off, 16, 1024), idescS, (part | ks) ? 1u : 0u);
+                        }
+                        if (part == 1)
+                            umma_commit(bar(qt ? B_SFULL1 : B_SFULL0));
+                    }
+                }
+                ok = a2_wait(bar(B_VFULL), (uint32_t)(j & 1), abort_flag);
+                for (int qt = 0; ok && qt < 2; ++qt) {
+                    ok = a2_wait(bar(qt ? B_PFULL1 : B_PFULL0), (uint32_t)(j & 1), abort_flag);
+                    if (!ok)
+                        break;
+                    tc_fence_after();
+                    const uint32_t aP = smem_u32(slot(s, qt));
+#pragma unroll
+                    for (int ks = 0; ks < 128 / 16; ++ks) {
+                        const uint32_t poff = (uint32_t)(ks >> 2) * (128u * 128u) + (uint32_t)(ks & 3) * 32u;
+                        umma_ss(tO[qt], sdesc_sw128(aP + poff, 16, 1024),
+                                sdesc_sw128(aV + (uint32_t)ks * 2048u, 128u * 128u, 1024), idescO,
+                                (j > 0 || ks > 0) ? 1u : 0u);
+                    }
+                }
+                if (!ok)
+                    break;
+                umma_commit(bar(B_PVDONE));
+            }
+            if (ok) {
+                umma_commit(bar(B_OFULL));
+            } else {
+                // drain: everything issued so far must finish before TMEM is freed
+                umma_commit(bar(B_OFULL));
+                uint32_t spins = 0;
+                while (!mbar_try_wait(bar(B_OFULL), 0) && ++spins < kSpinLimit) {
+                }
+            }
+        }
+    } else {
+        // ------------------------------------------------------------ softmax
+        const int grp = (warp - 5) >> 2;            // query tile 0 or 1
+        const uint32_t quarter = (uint32_t)(warp & 3);
+        const uint32_t r = quarter * 32u + (uint32_t)lane;  // row in the tile == TMEM lane
+        const uint32_t lane_off = (quarter * 32u) << 16;
+        const uint32_t tS = tmem + (grp ? 128u : 0u), tO = tmem + 256u + (grp ? (uint32_t)D : 0u);
+        float m_used = -INFINITY, l = 0.0f;
+        bool ok = true;
+        for (int j = 0; j < ntiles; ++j) {
+            ok = __all_sync(0xffffffffu, a2_wait(bar(grp ? B_SFULL1 : B_SFULL0), (uint32_t)(j & 1), abort_flag));
+            if (!ok)
+                break;
+            tc_fence_after();
+            const int64_t t0 = a.t_begin + (int64_t)j * 128;
+            const int64_t rem = a.t_end - t0;
+            const int nvalid = rem < 128 ? (int)rem : 128;
+            float tmax = -INFINITY;
+#pragma unroll
+            for (int cb = 0; cb < 4; ++cb) {
+                float sv[32];
+                tmem_ld32(tS + lane_off + (uint32_t)(cb * 32), sv);
+#pragma unroll
+                for (int i = 0; i < 32; ++i)
+                    if (cb * 32 + i < nvalid)
+                        tmax = fmaxf(tmax, sv[i]);
+            }
+            const float m_tile = tmax * a.scale_log2;
+            // lazy rescale: keep the stale maximum while exp2 stays below 2^8
+            const bool grow = m_tile > m_used + 8.0f;
+            if (__any_sync(0xffffffffu, grow)) {
+                const float m_new = grow ? fmaxf(m_tile, m_used) : m_used;
+                const float alpha = (m_used == -INFINITY) ? 0.0f : ex2_approx(m_used - m_new);
+                if (j > 0) {
+#pragma unroll 1
+                    for (int cb = 0; cb < D / 32; ++cb) {
+                        float ov[32];
+                        tmem_ld32(tO + lane_off + (uint32_t)(cb * 32), ov);
+#pragma unroll
+                        for (int i = 0; i < 32; ++i)
+                            ov[i] *= alpha;
+                        tmem_st32(tO + lane_off + (uint32_t)(cb * 32), ov);
+                    }
+                }
+                l *= alpha;
+                m_used = m_new;
+            }
+            // P = exp2(s * scale - m_used), fp16, into the stage's slot (K_hi
+            // for tile 0, K_lo for tile 1; both already consumed by the MMAs)
+            uint8_t *pt = slot(j & 1, grp);
+            float lt = 0.0f;
+#pragma unroll
+            for (int cb = 0; cb < 4; ++cb) {
+                float sv[32];
+                tmem_ld32(tS + lane_off + (uint32_t)(cb * 32), sv);
+                uint32_t pk[16];
+#pragma unroll
+                for (int i = 0; i < 32; i += 2) {
+                    const float p0 = (cb * 32 + i < nvalid) ? ex2_approx(fmaf(sv[i], a.scale_log2, -m_used)) : 0.0f;
+                    const float p1 =
+                        (cb * 32 + i + 1 < nvalid) ? ex2_approx(fmaf(sv[i + 1], a.scale_log2, -m_used)) : 0.0f;
+                    lt += p0 + p1;
+                    pk[i / 2] = pack_f16x2_sat(p0, p1);
+                }
+#pragma unroll
+                for (int uu = 0; uu < 4; ++uu)
+                    *reinterpret_cast<uint4 *>(pt + sw128_unit_offset(r, cb * 4 + uu, 128)) =
+                        make_uint4(pk[4 * uu], pk[4 * uu + 1], pk[4 * uu + 2], pk[4 * uu + 3]);
+            }
+            l += lt;
+            fence_proxy_async_smem();
+            tc_fence_before();
+            mbar_arrive(bar(grp ? B_PFULL1 : B_PFULL0));
+        }
+        // epilogue
+        const int64_t qr = q0 + grp * 128 + r;
+        const bool have =
+            __all_sync(0xffffffffu, ntiles > 0 && ok && a2_wait(bar(B_OFULL), 0, abort_flag));
+        if (have)
+            tc_fence_after();
+        const bool empty = !(l > 0.0f);
+        const float inv_l = empty ? 0.0f : 1.0f / l;
+#pragma unroll 1
+        for (int cb = 0; cb < D / 32; ++cb) {
+            float ov[32];
+            if (have)
+                tmem_ld32(tO + lane_off + (uint32_t)(cb * 32), ov);
+            if (qr < a.Tq) {
+#pragma unroll
+                for (int i = 0; i < 32; ++i)
+                    ov[i] = have ? ov[i] * inv_l : 0.0f;
+                if (a.o_bf16) {
+                    uint4 *dst = reinterpret_cast<uint4 *>(static_cast<uint16_t *>(a.o_out) + (qr * a.H + h) * D + cb * 32);
+#pragma unroll
+                    for (int u = 0; u < 4; ++u)
+                        dst[u] = make_uint4(pack_bf16x2(ov[8 * u], ov[8 * u + 1]), pack_bf16x2(ov[8 * u + 2], ov[8 * u + 3]),
+                                            pack_bf16x2(ov[8 * u + 4], ov[8 * u + 5]),
+                                            pack_bf16x2(ov[8 * u + 6], ov[8 * u + 7]));
+                } else {
+                    float4 *dst = reinterpret_cast<float4 *>(static_cast<float *>(a.o_out) + (qr * a.H + h) * D + cb * 32);
+#pragma unroll
+                    for (int u = 0; u < 8; ++u)
+                        dst[u] = make_float4(ov[4 * u], ov[4 * u + 1], ov[4 * u + 2], ov[4 * u + 3]);
+                }
+            }
+        }
+        if (qr < a.Tq)
+            a.lse_out[(int64_t)h * a.Tq + qr] =
+                (empty || !have) ? -INFINITY : (m_used + log2f(l)) * 0.69314718055994531f;
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 0)
+        tmem_dealloc(tmem, 512);
+}
+
+}  // namespace kvq

@@ -8,6 +8,7 @@
 #include <string.h>
 
 #include "attention.cuh"
+#include "attention2.cuh"
 #include "codec.cuh"
 #include "common.cuh"
 #include "encode_filter.cuh"
@@ -249,6 +250,25 @@ CodecView to_codec_view(const kvq_compressed_view *v)
     cv.bits = v->desc.bits;
     cv.G = v->desc.group_size;
     return cv;
+}
+
+template <int D>
+kvq_status launch_attention2(const AttnArgs &a, cudaStream_t s)
+{
+    using L = A2Smem<D>;
+    static bool configured[64] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64)
+        return KVQ_ERR_CUDA;
+    if (!configured[dev]) {
+        if (cudaFuncSetAttribute(attention2_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)L::kLaunchBytes) != cudaSuccess)
+            return KVQ_ERR_CUDA;
+        configured[dev] = true;
+    }
+    const dim3 grid((unsigned)ceil_div(a.Tq, kA2Rows), (unsigned)a.H);
+    attention2_kernel<D><<<grid, kA2Threads, L::kLaunchBytes, s>>>(a);
+    return launch_status();
 }
 
 template <int D>
@@ -568,7 +588,7 @@ kvq_status kvq_attention_lse(const void *q, int64_t Tq, const kvq_compressed_vie
     a.o_bf16 = o_dtype == KVQ_BF16;
     a.lse_out = lse_out;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    return D == 128 ? launch_attention<128>(a, s) : launch_attention<64>(a, s);
+    return D == 128 ? launch_attention2<128>(a, s) : launch_attention2<64>(a, s);
 }
 
 kvq_status kvq_lse_merge(int32_t n_parts, const float *const *o_parts, const float *const *lse_parts, int64_t Tq,

@@ -173,7 +173,7 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const float *v)
 }
 
 template <int D>
-__global__ void __maxnreg__(152) attention2_kernel(AttnArgs a)
+__global__ void __launch_bounds__(kA2Threads, 1) attention2_kernel(AttnArgs a)
 {
     using L = A2Smem<D>;
     extern __shared__ uint8_t smem_raw[];

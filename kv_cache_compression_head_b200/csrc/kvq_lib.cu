@@ -5,6 +5,8 @@
 #include <cudaTypedefs.h>
 #include <math.h>
 #include <stdint.h>
+#include <stdio.h>
+#include <stdlib.h>
 #include <string.h>
 
 #include "attention.cuh"
@@ -49,9 +51,16 @@ kvq_status check_desc(const kvq_codec_desc *d, bool allow_joint)
     return KVQ_OK;
 }
 
+// A failed launch is reported as KVQ_ERR_CUDA; with KVQ_DEBUG set in the
+// environment the CUDA error string is also printed to stderr.
 kvq_status launch_status()
 {
-    return cudaGetLastError() == cudaSuccess ? KVQ_OK : KVQ_ERR_CUDA;
+    const cudaError_t e = cudaGetLastError();
+    if (e == cudaSuccess)
+        return KVQ_OK;
+    if (getenv("KVQ_DEBUG"))
+        fprintf(stderr, "libkvq: CUDA error %d: %s\n", (int)e, cudaGetErrorString(e));
+    return KVQ_ERR_CUDA;
 }
 
 // ---------------------------------------------------------------------------

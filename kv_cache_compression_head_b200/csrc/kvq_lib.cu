@@ -153,7 +153,8 @@ kvq_status launch_filter_t(const CUtensorMap &m, const FilterArgs &a, cudaStream
     const int by_tmem = 512 / a.tmem_cols;
     const int per_sm = max(1, min(min(by_smem, by_tmem), 8));
     const int64_t ntiles = (a.T + kFltRows - 1) / kFltRows;
-    const int64_t want = ((int64_t)per_sm * sm_count() + a.H - 1) / a.H;
+    // one resident wave: per_sm CTAs on every SM, split evenly across heads
+    const int64_t want = ((int64_t)per_sm * sm_count()) / a.H > 0 ? ((int64_t)per_sm * sm_count()) / a.H : 1;
     const int64_t gx64 = ntiles < want ? ntiles : want;
     const unsigned gx = (unsigned)(gx64 > 0 ? gx64 : 1);
     encode_filter_kernel<D, BITS, G><<<dim3(gx, (unsigned)a.H), kFltThreads, smem, s>>>(m, a);

@@ -202,6 +202,7 @@ class Pipeline:
         self.cent = [torch.empty((H, w.num_centroids, d), dtype=bf, device=device) for _ in range(2)]
         self.enc = [K.alloc_encoded(c, T, device) for c in (self.codec_k, self.codec_v)]
         self.ws = K.alloc_workspace(K.KVQ_OP_FIT, self.codec_k, T, device)
+        self.ws_attn = K.alloc_workspace(K.KVQ_OP_ATTENTION, self.codec_k, T, device, num_queries=Tq)
         self.dec = [torch.empty((T, H, d), dtype=bf, device=device) for _ in range(2)]
         self.o_parts = [torch.empty((Tq, H, d), dtype=torch.float32, device=device) for _ in range(HISTORY_BLOCKS)]
         self.l_parts = [torch.empty((H, Tq), dtype=torch.float32, device=device) for _ in range(HISTORY_BLOCKS)]
@@ -241,7 +242,7 @@ class Pipeline:
         mark("attention", 0)
         for b in range(HISTORY_BLOCKS):
             K.kvq_attention_lse(self.q, self.comp[0], self.comp[1], self.o_parts[b], self.l_parts[b],
-                                t_begin=self.edges[b], t_end=self.edges[b + 1])
+                                t_begin=self.edges[b], t_end=self.edges[b + 1], workspace=self.ws_attn)
         mark("attention", 1)
         mark("merge", 0)
         K.kvq_lse_merge(self.o_parts, self.l_parts, self.o, self.lse)

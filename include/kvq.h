@@ -224,7 +224,11 @@ KVQ_API kvq_status kvq_decode(const kvq_compressed_view *view, void *x_out, kvq_
  *   q     [Tq][H][d] bf16;  o_out [Tq][H][d] (o_dtype);  lse_out [H][Tq]
  * k and v must have the same H, d and num_tokens; their bits, group sizes and
  * centroid counts may differ.  An empty range gives o = 0, lse = -inf.
- * Workspace: none (pass NULL / 0).
+ * Workspace (optional): with at least kvq_workspace_size(KVQ_OP_ATTENTION, k
+ * desc, T, Tq) bytes (16-byte aligned), the call may split the history range
+ * into up to 4 sub-ranges processed by separate CTAs when that fills the GPU
+ * better, writing binary32 partial results to the workspace and merging them
+ * by LSE as kvq_lse_merge does.  With NULL / 0 it runs unsplit.
  */
 KVQ_API kvq_status kvq_attention_lse(const void *q, int64_t num_queries, const kvq_compressed_view *k,
                              const kvq_compressed_view *v, int64_t t_begin, int64_t t_end, float softmax_scale,

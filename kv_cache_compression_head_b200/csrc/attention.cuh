@@ -54,6 +54,8 @@ struct AttnArgs {
     void *o_out;
     int o_bf16;
     float *lse_out;  // [H][Tq]
+    int nsplit;      // > 1: blockIdx.z selects a sub-range; o_out / lse_out
+                     // then hold nsplit float partials [z][Tq][H][D], [z][H][Tq]
 };
 
 constexpr int kAttnRows = 128;     // query rows per CTA

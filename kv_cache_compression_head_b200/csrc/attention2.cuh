@@ -5,19 +5,20 @@
 // added back to the dequantised residual; partial results carry their
 // log-sum-exp); QuantWM, Fig. 9 (on-demand reconstruction during attention).
 //
-// Roles (416 threads):
-//   warps 0-3  producer: load the two Q tiles, then for every 128-token history
-//              tile rebuild k^ (bf16 hi + lo tiles) and v^ (fp16 tile) from
-//              codes, {s, z}, idx and the bf16 centres straight into the
-//              128-byte-swizzled operand layout; one thread per history row.
-//   warp 4     MMA issuer (one thread): S_i = Q_i K_hi^T + Q_i K_lo^T into
-//              TMEM for both query tiles, then O_i += P_i V^ (fp16) once the
-//              softmax has published P_i.
-//   warps 5-8  softmax for query tile 0, warps 9-12 for query tile 1: one
-//              thread per query row (its TMEM lane); online softmax in the
-//              exp2 domain with lazy rescaling (O in TMEM is rescaled only when
-//              the running maximum grows by more than 2^8); P (fp16) goes to
-//              the shared buffers of the K stage the tile came from.
+// Roles (544 threads):
+//   warps 0-7   producer: load the two Q tiles, then for every 128-token
+//               history tile rebuild k^ (bf16 hi + lo tiles) and v^ (fp16
+//               tile) from codes, {s, z}, idx and the bf16 centres straight
+//               into the 128-byte-swizzled operand layout; two threads per
+//               history row, one per half of the channels.
+//   warp 8      MMA issuer (one thread): S_i = Q_i K_hi^T + Q_i K_lo^T into
+//               TMEM for both query tiles, then O_i += P_i V^ (fp16) once the
+//               softmax has published P_i.
+//   warps 9-12  softmax for query tile 0, warps 13-16 for query tile 1: one
+//               thread per query row (its TMEM lane); online softmax in the
+//               exp2 domain with lazy rescaling (O in TMEM is rescaled only
+//               when the running maximum grows by more than 2^8); P (fp16)
+//               goes to the shared buffers of the K stage the tile came from.
 // Shared memory: Q tiles 2 x 32 KB, two K stages of 2 x 32 KB (K_hi, K_lo,
 // later P_0, P_1), one V tile of 32 KB (d = 128).  TMEM: S_0, S_1 (128 columns
 // each) and O_0, O_1 (d columns each).
@@ -42,7 +43,8 @@
 
 namespace kvq {
 
-constexpr int kA2Threads = 416;
+constexpr int kA2Threads = 544;
+constexpr int kA2Producers = 256;
 constexpr int kA2Rows = 256;  // query rows per CTA (two tiles)
 
 template <int D>
@@ -80,20 +82,36 @@ __device__ __forceinline__ void mbar_arrive(uint32_t bar)
     asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
 }
 
-// Rebuild history row `tok` of a compressed K (SPLIT: bf16 hi + lo tiles) or
-// V (fp16 tile) into the swizzled tiles.  k^ = fma(f, 2^b s, mu - (2^b + z) s)
-// with f = 1 + q 2^-b built directly in the float's mantissa, the decoder's
-// value up to one rounding.
-template <int D, bool SPLIT>
-__device__ __forceinline__ void a2_dequant_row(const CodecView &cv, int h, int64_t tok, bool valid, uint8_t *tile,
-                                               uint8_t *tile_lo, uint32_t row)
+// f = 1 + q 2^-b for the code of channel k (0..7) of a unit: the code bits are
+// moved into the top of the mantissa of 1.0f.
+template <int BITS>
+__device__ __forceinline__ float code_as_unit_float(uint32_t cw, int k)
 {
+    constexpr int kShift = 23 - BITS;
+    constexpr uint32_t kMask = ((1u << BITS) - 1u) << kShift;
+    const int sh = kShift - k * BITS;
+    const uint32_t qb = (sh >= 0 ? (cw << sh) : (cw >> -sh)) & kMask;
+    return __uint_as_float(0x3F800000u | qb);
+}
+
+// Rebuild channels [d/2 half, d/2 half + d/2) of history row `tok` of a
+// compressed K (SPLIT: bf16 hi + lo tiles) or V (fp16 tile) into the swizzled
+// tiles:  x^ = fma(f, 2^b s, mu - (2^b + z) s),  f = 1 + q 2^-b,  which is the
+// decoder's mu + (q - z) s up to one rounding.  The loads of the half row are
+// issued together before any arithmetic.
+template <int D, int BITS, bool SPLIT>
+__device__ __forceinline__ void a2_dequant_half(const CodecView &cv, int h, int64_t tok, bool valid, int half,
+                                                uint8_t *tile, uint8_t *tile_lo, uint32_t row)
+{
+    constexpr int kUnits = D / 16;  // 8-channel units in a half row
+    const int u0 = half * kUnits;
     if (!valid) {
 #pragma unroll
-        for (int u = 0; u < D / 8; ++u) {
-            *reinterpret_cast<uint4 *>(tile + sw128_unit_offset(row, u, 128)) = make_uint4(0, 0, 0, 0);
+        for (int uu = 0; uu < kUnits; ++uu) {
+            const uint32_t off = sw128_unit_offset(row, u0 + uu, 128);
+            *reinterpret_cast<uint4 *>(tile + off) = make_uint4(0, 0, 0, 0);
             if (SPLIT)
-                *reinterpret_cast<uint4 *>(tile_lo + sw128_unit_offset(row, u, 128)) = make_uint4(0, 0, 0, 0);
+                *reinterpret_cast<uint4 *>(tile_lo + off) = make_uint4(0, 0, 0, 0);
         }
         return;
     }
@@ -103,52 +121,69 @@ __device__ __forceinline__ void a2_dequant_row(const CodecView &cv, int h, int64
         raise_status(DEVSTAT_BAD_INDEX);
         j = 0;
     }
-    const uint4 *mu_row = reinterpret_cast<const uint4 *>(cv.cent + ((int64_t)h * cv.C + j) * D);
-    const float2 *meta_row = reinterpret_cast<const float2 *>(cv.meta) + th * (D / cv.G);
-    const int bits = cv.bits;
-    const float two_b = (float)(1 << bits);
-    const uint32_t qshift = 23u - (uint32_t)bits;
-    const uint32_t qmask = ((1u << bits) - 1u) << qshift;
-#pragma unroll 4
-    for (int u = 0; u < D / 8; ++u) {
-        const int c0 = u * 8;
-        const float2 sz = __ldg(meta_row + c0 / cv.G);
-        const float sc = two_b * sz.x;                  // 2^b s (exact)
-        const float nb = -__fmul_rn(two_b + sz.y, sz.x); // -(2^b + z) s
-        uint32_t cw;
-        if (bits == 2)
-            cw = __ldg(reinterpret_cast<const uint16_t *>(cv.codes + th * (D / 4)) + u);
-        else
-            cw = __ldg(reinterpret_cast<const uint32_t *>(cv.codes + th * (D / 2)) + u);
-        const uint4 mw = __ldg(mu_row + u);
-        const uint32_t ma[4] = {mw.x, mw.y, mw.z, mw.w};
-        float val[8];
+    const uint4 *mu_row = reinterpret_cast<const uint4 *>(cv.cent + ((int64_t)h * cv.C + j) * D) + u0;
+    uint4 mw[kUnits];
 #pragma unroll
-        for (int k = 0; k < 8; ++k) {
-            const int sh = (int)qshift - k * bits;
-            const uint32_t qb = (sh >= 0 ? (cw << sh) : (cw >> -sh)) & qmask;
-            const float f = __uint_as_float(0x3F800000u | qb);
-            const float mu = (k & 1) ? bf16_hi(ma[k >> 1]) : bf16_lo(ma[k >> 1]);
-            val[k] = fmaf(f, sc, mu + nb);
+    for (int uu = 0; uu < kUnits; ++uu)
+        mw[uu] = __ldg(mu_row + uu);
+    uint32_t cws[kUnits];
+    if (BITS == 2) {
+        const uint16_t *cr = reinterpret_cast<const uint16_t *>(cv.codes + th * (D / 4)) + u0;
+#pragma unroll
+        for (int uu = 0; uu < kUnits; ++uu)
+            cws[uu] = __ldg(cr + uu);
+    } else {
+        const uint32_t *cr = reinterpret_cast<const uint32_t *>(cv.codes + th * (D / 2)) + u0;
+#pragma unroll
+        for (int uu = 0; uu < kUnits; ++uu)
+            cws[uu] = __ldg(cr + uu);
+    }
+    const float2 *meta_row = reinterpret_cast<const float2 *>(cv.meta) + th * (D / cv.G);
+    constexpr float kTwoB = (float)(1 << BITS);
+#pragma unroll
+    for (int uu = 0; uu < kUnits; ++uu) {
+        const int c0 = (u0 + uu) * 8;
+        const float2 sz = __ldg(meta_row + c0 / cv.G);
+        const float sc = kTwoB * sz.x;                  // 2^b s (exact)
+        const float nb = -__fmul_rn(kTwoB + sz.y, sz.x); // -(2^b + z) s
+        const uint32_t ma[4] = {mw[uu].x, mw[uu].y, mw[uu].z, mw[uu].w};
+        float2 val[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            const float2 f = make_float2(code_as_unit_float<BITS>(cws[uu], 2 * k),
+                                         code_as_unit_float<BITS>(cws[uu], 2 * k + 1));
+            const float2 b = add2(make_float2(bf16_lo(ma[k]), bf16_hi(ma[k])), make_float2(nb, nb));
+            val[k] = fma2(f, make_float2(sc, sc), b);
         }
-        const uint32_t off = sw128_unit_offset(row, u, 128);
+        const uint32_t off = sw128_unit_offset(row, u0 + uu, 128);
         if (SPLIT) {
             uint32_t hi[4], lo[4];
 #pragma unroll
             for (int k = 0; k < 4; ++k) {
-                const uint32_t a0 = __float_as_uint(val[2 * k]) & 0xffff0000u;
-                const uint32_t a1 = __float_as_uint(val[2 * k + 1]) & 0xffff0000u;
-                hi[k] = (a0 >> 16) | a1;
-                lo[k] = pack_bf16x2(val[2 * k] - __uint_as_float(a0), val[2 * k + 1] - __uint_as_float(a1));
+                const uint32_t a0 = __float_as_uint(val[k].x) & 0xffff0000u;
+                const uint32_t a1 = __float_as_uint(val[k].y) & 0xffff0000u;
+                hi[k] = __byte_perm(a0, a1, 0x7632);
+                const float2 r = sub2(val[k], make_float2(__uint_as_float(a0), __uint_as_float(a1)));
+                lo[k] = pack_bf16x2(r.x, r.y);
             }
             *reinterpret_cast<uint4 *>(tile + off) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
             *reinterpret_cast<uint4 *>(tile_lo + off) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
         } else {
             *reinterpret_cast<uint4 *>(tile + off) =
-                make_uint4(pack_f16x2_sat(val[0], val[1]), pack_f16x2_sat(val[2], val[3]),
-                           pack_f16x2_sat(val[4], val[5]), pack_f16x2_sat(val[6], val[7]));
+                make_uint4(pack_f16x2_sat(val[0].x, val[0].y), pack_f16x2_sat(val[1].x, val[1].y),
+                           pack_f16x2_sat(val[2].x, val[2].y), pack_f16x2_sat(val[3].x, val[3].y));
         }
     }
+}
+
+template <int D, bool SPLIT>
+__device__ __forceinline__ void a2_dequant(const CodecView &cv, int h, int64_t tok, bool valid, int half, uint8_t *tile,
+                                           uint8_t *tile_lo, uint32_t row)
+{
+    if (cv.bits == 2)
+        a2_dequant_half<D, 2, SPLIT>(cv, h, tok, valid, half, tile, tile_lo, row);
+    else
+        a2_dequant_half<D, 4, SPLIT>(cv, h, tok, valid, half, tile, tile_lo, row);
 }
 
 __device__ __forceinline__ void tmem_st32(uint32_t taddr, const float *v)
@@ -172,6 +207,32 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const float *v)
     asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
 
+// One 32-column chunk of P = exp2(s * scale - m), packed fp16, into 4 swizzled
+// 16-byte units of the P tile; returns the chunk's sum of the (unrounded) p.
+template <bool MASKED>
+__device__ __forceinline__ float a2_softmax_chunk(const float *sv, float scale, float m, int cbase, int nvalid,
+                                                  uint8_t *pt, uint32_t r, int cb)
+{
+    float lt = 0.0f;
+    uint32_t pk[16];
+#pragma unroll
+    for (int i = 0; i < 32; i += 2) {
+        float p0 = ex2_approx(fmaf(sv[i], scale, -m));
+        float p1 = ex2_approx(fmaf(sv[i + 1], scale, -m));
+        if (MASKED) {
+            p0 = (cbase + i < nvalid) ? p0 : 0.0f;
+            p1 = (cbase + i + 1 < nvalid) ? p1 : 0.0f;
+        }
+        lt += p0 + p1;
+        pk[i / 2] = pack_f16x2_sat(p0, p1);
+    }
+#pragma unroll
+    for (int uu = 0; uu < 4; ++uu)
+        *reinterpret_cast<uint4 *>(pt + sw128_unit_offset(r, cb * 4 + uu, 128)) =
+            make_uint4(pk[4 * uu], pk[4 * uu + 1], pk[4 * uu + 2], pk[4 * uu + 3]);
+    return lt;
+}
+
 template <int D>
 __global__ void __launch_bounds__(kA2Threads, 1) attention2_kernel(AttnArgs a)
 {
@@ -187,16 +248,29 @@ __global__ void __launch_bounds__(kA2Threads, 1) attention2_kernel(AttnArgs a)
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int h = blockIdx.y;
     const int64_t q0 = (int64_t)blockIdx.x * kA2Rows;
+    if (a.nsplit > 1) {
+        // sub-range z of the history, split at 128-token tile boundaries; the
+        // partial result (binary32) goes to slice z of the partial buffers
+        const int64_t tiles_all = (a.t_end - a.t_begin + 127) / 128;
+        const int z = blockIdx.z;
+        const int64_t b0 = a.t_begin + (tiles_all * z / a.nsplit) * 128;
+        const int64_t b1 = a.t_begin + (tiles_all * (z + 1) / a.nsplit) * 128;
+        a.t_end = b1 < a.t_end ? b1 : a.t_end;
+        a.t_begin = b0 < a.t_end ? b0 : a.t_end;
+        a.o_out = static_cast<float *>(a.o_out) + (int64_t)z * a.Tq * a.H * D;
+        a.lse_out += (int64_t)z * a.H * a.Tq;
+        a.o_bf16 = 0;
+    }
     const int64_t span = a.t_end - a.t_begin;
     const int ntiles = (int)((span + 127) / 128);
 
     if (warp == 0)
         tmem_alloc(smem_u32(tmem_slot), 512);
     if (tid == 0) {
-        mbar_init(bar(B_QREADY), 128);
-        mbar_init(bar(B_KFULL0), 128);
-        mbar_init(bar(B_KFULL1), 128);
-        mbar_init(bar(B_VFULL), 128);
+        mbar_init(bar(B_QREADY), kA2Producers);
+        mbar_init(bar(B_KFULL0), kA2Producers);
+        mbar_init(bar(B_KFULL1), kA2Producers);
+        mbar_init(bar(B_VFULL), kA2Producers);
         mbar_init(bar(B_SFULL0), 1);
         mbar_init(bar(B_SFULL1), 1);
         mbar_init(bar(B_PFULL0), 128);
@@ -211,10 +285,11 @@ __global__ void __launch_bounds__(kA2Threads, 1) attention2_kernel(AttnArgs a)
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
 
-    if (warp < 4) {
+    if (warp < kA2Producers / 32) {
         // ------------------------------------------------------------ producer
-        const uint32_t r = (uint32_t)tid;
-        for (int qt = 0; qt < 2; ++qt) {
+        {
+            const int qt = tid >> 7;
+            const uint32_t r = (uint32_t)(tid & 127);
             const int64_t qr = q0 + qt * 128 + r;
             const bool valid = qr < a.Tq;
             const uint16_t *src = a.q + (qr * a.H + h) * D;
@@ -227,10 +302,12 @@ __global__ void __launch_bounds__(kA2Threads, 1) attention2_kernel(AttnArgs a)
         }
         fence_proxy_async_smem();
         mbar_arrive(bar(B_QREADY));
+        const uint32_t r = (uint32_t)(tid & 127);
+        const int half = tid >> 7;
         if (ntiles > 0) {
             {
                 const int64_t tok = a.t_begin + r;
-                a2_dequant_row<D, true>(a.k, h, tok, tok < a.t_end, slot(0, 0), slot(0, 1), r);
+                a2_dequant<D, true>(a.k, h, tok, tok < a.t_end, half, slot(0, 0), slot(0, 1), r);
                 fence_proxy_async_smem();
                 mbar_arrive(bar(B_KFULL0));
             }
@@ -238,19 +315,19 @@ __global__ void __launch_bounds__(kA2Threads, 1) attention2_kernel(AttnArgs a)
                 if (j >= 1 && !a2_wait(bar(B_PVDONE), (uint32_t)((j - 1) & 1), abort_flag))
                     break;
                 const int64_t tok = a.t_begin + (int64_t)j * 128 + r;
-                a2_dequant_row<D, false>(a.v, h, tok, tok < a.t_end, smem + L::offV, nullptr, r);
+                a2_dequant<D, false>(a.v, h, tok, tok < a.t_end, half, smem + L::offV, nullptr, r);
                 fence_proxy_async_smem();
                 mbar_arrive(bar(B_VFULL));
                 if (j + 1 < ntiles) {
                     const int s = (j + 1) & 1;
                     const int64_t tk = tok + 128;
-                    a2_dequant_row<D, true>(a.k, h, tk, tk < a.t_end, slot(s, 0), slot(s, 1), r);
+                    a2_dequant<D, true>(a.k, h, tk, tk < a.t_end, half, slot(s, 0), slot(s, 1), r);
                     fence_proxy_async_smem();
                     mbar_arrive(bar(s ? B_KFULL1 : B_KFULL0));
                 }
             }
         }
-    } else if (warp == 4) {
+    } else if (warp == kA2Producers / 32) {
         // ------------------------------------------------------------ MMA issuer
         if (lane == 0 && ntiles > 0) {
             constexpr uint32_t idescS = idesc_f32acc(128, 128, true, false, false);
@@ -301,11 +378,10 @@ __global__ void __launch_bounds__(kA2Threads, 1) attention2_kernel(AttnArgs a)
                     break;
                 umma_commit(bar(B_PVDONE));
             }
-            if (ok) {
-                umma_commit(bar(B_OFULL));
-            } else {
-                // drain: everything issued so far must finish before TMEM is freed
-                umma_commit(bar(B_OFULL));
+            // on success this signals the epilogue; on failure it drains every
+            // MMA issued so far before TMEM is freed
+            umma_commit(bar(B_OFULL));
+            if (!ok) {
                 uint32_t spins = 0;
                 while (!mbar_try_wait(bar(B_OFULL), 0) && ++spins < kSpinLimit) {
                 }
@@ -313,9 +389,9 @@ __global__ void __launch_bounds__(kA2Threads, 1) attention2_kernel(AttnArgs a)
         }
     } else {
         // ------------------------------------------------------------ softmax
-        const int grp = (warp - 5) >> 2;            // query tile 0 or 1
+        const int grp = (warp - kA2Producers / 32 - 1) >> 2;  // query tile 0 or 1
         const uint32_t quarter = (uint32_t)(warp & 3);
-        const uint32_t r = quarter * 32u + (uint32_t)lane;  // row in the tile == TMEM lane
+        const uint32_t r = quarter * 32u + (uint32_t)lane;    // row in the tile == TMEM lane
         const uint32_t lane_off = (quarter * 32u) << 16;
         const uint32_t tS = tmem + (grp ? 128u : 0u), tO = tmem + 256u + (grp ? (uint32_t)D : 0u);
         float m_used = -INFINITY, l = 0.0f;
@@ -333,10 +409,16 @@ __global__ void __launch_bounds__(kA2Threads, 1) attention2_kernel(AttnArgs a)
             for (int cb = 0; cb < 4; ++cb) {
                 float sv[32];
                 tmem_ld32(tS + lane_off + (uint32_t)(cb * 32), sv);
+                if (nvalid == 128) {
 #pragma unroll
-                for (int i = 0; i < 32; ++i)
-                    if (cb * 32 + i < nvalid)
+                    for (int i = 0; i < 32; ++i)
                         tmax = fmaxf(tmax, sv[i]);
+                } else {
+#pragma unroll
+                    for (int i = 0; i < 32; ++i)
+                        if (cb * 32 + i < nvalid)
+                            tmax = fmaxf(tmax, sv[i]);
+                }
             }
             const float m_tile = tmax * a.scale_log2;
             // lazy rescale: keep the stale maximum while exp2 stays below 2^8
@@ -366,19 +448,10 @@ __global__ void __launch_bounds__(kA2Threads, 1) attention2_kernel(AttnArgs a)
             for (int cb = 0; cb < 4; ++cb) {
                 float sv[32];
                 tmem_ld32(tS + lane_off + (uint32_t)(cb * 32), sv);
-                uint32_t pk[16];
-#pragma unroll
-                for (int i = 0; i < 32; i += 2) {
-                    const float p0 = (cb * 32 + i < nvalid) ? ex2_approx(fmaf(sv[i], a.scale_log2, -m_used)) : 0.0f;
-                    const float p1 =
-                        (cb * 32 + i + 1 < nvalid) ? ex2_approx(fmaf(sv[i + 1], a.scale_log2, -m_used)) : 0.0f;
-                    lt += p0 + p1;
-                    pk[i / 2] = pack_f16x2_sat(p0, p1);
-                }
-#pragma unroll
-                for (int uu = 0; uu < 4; ++uu)
-                    *reinterpret_cast<uint4 *>(pt + sw128_unit_offset(r, cb * 4 + uu, 128)) =
-                        make_uint4(pk[4 * uu], pk[4 * uu + 1], pk[4 * uu + 2], pk[4 * uu + 3]);
+                if (nvalid == 128)
+                    lt += a2_softmax_chunk<false>(sv, a.scale_log2, m_used, cb * 32, nvalid, pt, r, cb);
+                else
+                    lt += a2_softmax_chunk<true>(sv, a.scale_log2, m_used, cb * 32, nvalid, pt, r, cb);
             }
             l += lt;
             fence_proxy_async_smem();
@@ -403,14 +476,16 @@ __global__ void __launch_bounds__(kA2Threads, 1) attention2_kernel(AttnArgs a)
                 for (int i = 0; i < 32; ++i)
                     ov[i] = have ? ov[i] * inv_l : 0.0f;
                 if (a.o_bf16) {
-                    uint4 *dst = reinterpret_cast<uint4 *>(static_cast<uint16_t *>(a.o_out) + (qr * a.H + h) * D + cb * 32);
+                    uint4 *dst =
+                        reinterpret_cast<uint4 *>(static_cast<uint16_t *>(a.o_out) + (qr * a.H + h) * D + cb * 32);
 #pragma unroll
                     for (int u = 0; u < 4; ++u)
                         dst[u] = make_uint4(pack_bf16x2(ov[8 * u], ov[8 * u + 1]), pack_bf16x2(ov[8 * u + 2], ov[8 * u + 3]),
                                             pack_bf16x2(ov[8 * u + 4], ov[8 * u + 5]),
                                             pack_bf16x2(ov[8 * u + 6], ov[8 * u + 7]));
                 } else {
-                    float4 *dst = reinterpret_cast<float4 *>(static_cast<float *>(a.o_out) + (qr * a.H + h) * D + cb * 32);
+                    float4 *dst =
+                        reinterpret_cast<float4 *>(static_cast<float *>(a.o_out) + (qr * a.H + h) * D + cb * 32);
 #pragma unroll
                     for (int u = 0; u < 8; ++u)
                         dst[u] = make_float4(ov[4 * u], ov[4 * u + 1], ov[4 * u + 2], ov[4 * u + 3]);

@@ -262,6 +262,39 @@ CodecView to_codec_view(const kvq_compressed_view *v)
     return cv;
 }
 
+constexpr int kMaxAttnSplit = 4;
+
+size_t attention_workspace(const kvq_codec_desc *d, int64_t Tq)
+{
+    const size_t o = (size_t)kMaxAttnSplit * (size_t)Tq * d->num_heads * d->head_dim * 4;
+    return round_up(o, 256) + (size_t)kMaxAttnSplit * d->num_heads * (size_t)Tq * 4;
+}
+
+// Number of history sub-ranges for one attention call: the CTA count
+// (query-tile pairs x heads x splits) should fill whole waves of one CTA per
+// SM, and every sub-range should keep at least 8 history tiles.
+int attention_splits(int64_t Tq, int H, int64_t span, size_t ws_bytes, size_t ws_need)
+{
+    if (ws_bytes < ws_need)
+        return 1;
+    const int64_t base = ((Tq + kA2Rows - 1) / kA2Rows) * H;
+    const int64_t sms = sm_count();
+    const int64_t tiles = (span + 127) / 128;
+    int best = 1;
+    double best_eff = (double)base / (double)(((base + sms - 1) / sms) * sms);
+    for (int k = 2; k <= kMaxAttnSplit; ++k) {
+        if (tiles / k < 8)
+            break;
+        const int64_t n = base * k;
+        const double eff = (double)n / (double)(((n + sms - 1) / sms) * sms);
+        if (eff > best_eff + 0.02) {
+            best = k;
+            best_eff = eff;
+        }
+    }
+    return best;
+}
+
 template <int D>
 kvq_status launch_attention2(const AttnArgs &a, cudaStream_t s)
 {
@@ -276,7 +309,7 @@ kvq_status launch_attention2(const AttnArgs &a, cudaStream_t s)
             return KVQ_ERR_CUDA;
         configured[dev] = true;
     }
-    const dim3 grid((unsigned)ceil_div(a.Tq, kA2Rows), (unsigned)a.H);
+    const dim3 grid((unsigned)ceil_div(a.Tq, kA2Rows), (unsigned)a.H, (unsigned)(a.nsplit > 1 ? a.nsplit : 1));
     attention2_kernel<D><<<grid, kA2Threads, L::kLaunchBytes, s>>>(a);
     return launch_status();
 }
@@ -358,7 +391,7 @@ kvq_status kvq_workspace_size(kvq_op op, const kvq_codec_desc *desc, int64_t T, 
     case KVQ_OP_DECODE:
         *bytes = 0;
         return desc->joint_rank > 0 ? KVQ_ERR_UNSUPPORTED : KVQ_OK;
-    case KVQ_OP_ATTENTION: *bytes = 0; return KVQ_OK;
+    case KVQ_OP_ATTENTION: *bytes = attention_workspace(desc, Tq); return KVQ_OK;
     }
     return KVQ_ERR_INVALID_ARG;
 }
@@ -597,8 +630,42 @@ kvq_status kvq_attention_lse(const void *q, int64_t Tq, const kvq_compressed_vie
     a.o_out = o_out;
     a.o_bf16 = o_dtype == KVQ_BF16;
     a.lse_out = lse_out;
+    a.nsplit = 1;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    return D == 128 ? launch_attention2<128>(a, s) : launch_attention2<64>(a, s);
+    const size_t need = attention_workspace(&k->desc, Tq);
+    const int nsplit = (workspace && aligned16(workspace))
+                           ? attention_splits(Tq, a.H, t_end - t_begin, workspace_bytes, need)
+                           : 1;
+    if (nsplit == 1)
+        return D == 128 ? launch_attention2<128>(a, s) : launch_attention2<64>(a, s);
+    // history split across CTAs: binary32 partials in the workspace, merged by LSE
+    float *o_part = static_cast<float *>(workspace);
+    float *l_part = reinterpret_cast<float *>(static_cast<uint8_t *>(workspace) +
+                                              round_up((size_t)kMaxAttnSplit * (size_t)Tq * a.H * D * 4, 256));
+    AttnArgs ap = a;
+    ap.o_out = o_part;
+    ap.lse_out = l_part;
+    ap.o_bf16 = 0;
+    ap.nsplit = nsplit;
+    st = D == 128 ? launch_attention2<128>(ap, s) : launch_attention2<64>(ap, s);
+    if (st != KVQ_OK)
+        return st;
+    MergeArgs m;
+    memset(&m, 0, sizeof m);
+    for (int z = 0; z < nsplit; ++z) {
+        m.o[z] = o_part + (int64_t)z * Tq * a.H * D;
+        m.lse[z] = l_part + (int64_t)z * a.H * Tq;
+    }
+    m.n = nsplit;
+    m.Tq = Tq;
+    m.H = a.H;
+    m.D = D;
+    m.o_out = o_out;
+    m.o_bf16 = a.o_bf16;
+    m.lse_out = lse_out;
+    const int64_t n = Tq * a.H * (D / 4);
+    lse_merge_kernel<<<(unsigned)ceil_div(n, 256), 256, 0, s>>>(m);
+    return launch_status();
 }
 
 kvq_status kvq_lse_merge(int32_t n_parts, const float *const *o_parts, const float *const *lse_parts, int64_t Tq,

@@ -47,13 +47,14 @@ def _assert_encoded_equal(comp, H, T, d, bits, G, idx_ref, codes_ref, meta_ref, 
     assert np.array_equal(meta, f32_bits(meta_ref)), "meta mismatch"
 
 
-def _attention(q_np, kc, vc, t0=None, t1=None, o_dtype=torch.float32):
+def _attention(q_np, kc, vc, t0=None, t1=None, o_dtype=torch.float32, split=False):
     K = _K()
     q = to_dev(q_np)
     Tq, H, d = q_np.shape
     o = torch.empty((Tq, H, d), dtype=o_dtype, device="cuda")
     lse = torch.empty((H, Tq), dtype=torch.float32, device="cuda")
-    K.kvq_attention_lse(q, kc, vc, o, lse, t_begin=0 if t0 is None else t0, t_end=t1)
+    ws = K.alloc_workspace(K.KVQ_OP_ATTENTION, kc.codec, kc.num_tokens, "cuda", num_queries=Tq) if split else None
+    K.kvq_attention_lse(q, kc, vc, o, lse, t_begin=0 if t0 is None else t0, t_end=t1, workspace=ws)
     return o, lse
 
 
@@ -102,6 +103,8 @@ def test_tiny_end_to_end():
     o_ref, lse_ref = O.attention(q, decs[0], decs[1])
     o, lse = _attention(q, comps[0], comps[1])
     assert_attention_close(o.cpu().numpy(), lse.cpu().numpy(), o_ref, lse_ref, "tiny")
+    o2, lse2 = _attention(q, comps[0], comps[1], split=True)
+    assert_attention_close(o2.cpu().numpy(), lse2.cpu().numpy(), o_ref, lse_ref, "tiny split")
     # the bf16 output is the binary32 result rounded to nearest-even
     ob, lseb = _attention(q, comps[0], comps[1], o_dtype=torch.bfloat16)
     assert torch.equal(ob.cpu().view(torch.int16), o.cpu().to(torch.bfloat16).view(torch.int16))
@@ -170,6 +173,7 @@ def test_wan_attention_full_size_sampled(wan):
     ck = _gpu_encode(K.Codec(H, d, w.num_centroids, w.bits_k, w.group_size), xk, seeds_k)
     cv = _gpu_encode(K.Codec(H, d, w.num_centroids, w.bits_v, w.group_size), xv, seeds_v)
     o, lse = _attention(q, ck, cv)
+    o_s, lse_s = _attention(q, ck, cv, split=True)  # history split inside the call
     heads = [3, 11]
     rows = _sample_tokens(w.query_tokens, 256, 5)
     sub = lambda a: np.ascontiguousarray(a[:, heads])
@@ -181,6 +185,8 @@ def test_wan_attention_full_size_sampled(wan):
     o_g = o.cpu().numpy()[rows][:, heads]
     l_g = lse.cpu().numpy()[heads][:, rows]
     assert_attention_close(o_g, l_g, o_ref, lse_ref, "wan full")
+    assert_attention_close(o_s.cpu().numpy()[rows][:, heads], lse_s.cpu().numpy()[heads][:, rows], o_ref, lse_ref,
+                           "wan full, split history")
     _status_ok()
 
 

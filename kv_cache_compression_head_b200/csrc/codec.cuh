@@ -346,6 +346,40 @@ __global__ void __launch_bounds__(256) fit_accumulate_kernel(FitArgs a)
         atomicAdd(a.counts + (int64_t)h * a.C + j, 1u);
 }
 
+// Same sums with far fewer global atomics: a block owns one head, one slice
+// of W channels and a contiguous token range; it accumulates into binary64
+// shared-memory sums [C][W] and adds them to the global sums once at the end.
+// Token counts are added by the slice-0 blocks.
+template <int W>
+__global__ void __launch_bounds__(256) fit_accumulate_smem_kernel(FitArgs a, int64_t tokens_per_block)
+{
+    extern __shared__ double s_sum[];  // [C][W]
+    const int h = blockIdx.y, slice = blockIdx.z;
+    const int64_t t_lo = (int64_t)blockIdx.x * tokens_per_block;
+    const int64_t t_hi = min(a.T, t_lo + tokens_per_block);
+    for (int e = threadIdx.x; e < a.C * W; e += blockDim.x)
+        s_sum[e] = 0.0;
+    __syncthreads();
+    // a group of W lanes handles one token; lane c adds channel slice*W + c
+    constexpr int kGroups = 256 / W;
+    const int grp = threadIdx.x / W, c = threadIdx.x % W;
+    for (int64_t t = t_lo + grp; t < t_hi; t += kGroups) {
+        const int j = a.idx[(int64_t)h * a.T + t];
+        const int64_t e = (t * a.H + h) * a.D + slice * W + c;
+        const float v = a.x_bf16 ? __uint_as_float((uint32_t)static_cast<const uint16_t *>(a.x)[e] << 16)
+                                 : static_cast<const float *>(a.x)[e];
+        atomicAdd(&s_sum[j * W + c], (double)v);
+        if (slice == 0 && c == 0)
+            atomicAdd(a.counts + (int64_t)h * a.C + j, 1u);
+    }
+    __syncthreads();
+    for (int e = threadIdx.x; e < a.C * W; e += blockDim.x) {
+        const double v = s_sum[e];
+        if (v != 0.0)
+            atomicAdd(a.sums + ((int64_t)h * a.C + e / W) * a.D + slice * W + e % W, v);
+    }
+}
+
 // mu_j = bf16(float(sum_j / n_j)) where n_j > 0; empty centres keep mu_j.
 __global__ void __launch_bounds__(256) fit_update_kernel(FitArgs a)
 {

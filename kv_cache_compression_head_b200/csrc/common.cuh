@@ -158,6 +158,25 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity)
     return false;
 }
 
+// Named barrier ID (1..15, a compile-time constant so that only the barriers
+// used are reserved) over `count` threads (whole warps).
+template <int ID>
+__device__ __forceinline__ void named_barrier_sync(int count)
+{
+    asm volatile("bar.sync %0, %1;" ::"n"(ID), "r"(count) : "memory");
+}
+
+// Named barrier 1 + q (q = 0..3) over `count` threads.
+__device__ __forceinline__ void named_barrier_sync_q(int q, int count)
+{
+    switch (q & 3) {
+    case 0: named_barrier_sync<1>(count); break;
+    case 1: named_barrier_sync<2>(count); break;
+    case 2: named_barrier_sync<3>(count); break;
+    default: named_barrier_sync<4>(count); break;
+    }
+}
+
 // ---------------------------------------------------------------------------
 // tcgen05: tensor memory, MMA, loads
 // ---------------------------------------------------------------------------

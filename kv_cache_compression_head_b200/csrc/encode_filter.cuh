@@ -16,10 +16,11 @@
 //      channels) compute v_j = |mu_j|^2 - 2 p_j, the row minimum m and the
 //      candidate window  v_j <= m + kappa (|x| + max_j |mu_j|)^2,  which
 //      provably contains the specified argmin: kappa covers the tensor-core
-//      accumulation error, the rounding of |mu_j|^2 and of v_j, and the
-//      rounding of the specified distance.  A single candidate is the
-//      answer; otherwise the candidates are re-scored with the specified
-//      distance (lowest index wins ties);
+//      accumulation error, the rounding of |mu_j|^2 and of v_j, the rounding
+//      of the specified distance and the index bits carried in v.  When the
+//      second smallest v lies outside the window the smallest is the answer;
+//      otherwise the window is re-scored with the specified distance (lowest
+//      index wins ties);
 //   4. the residual against the chosen centre is quantised (Eq. 1) per group
 //      and packed, each thread covering its half of the channels.
 #pragma once
@@ -51,8 +52,8 @@ struct FilterArgs {
 
 __host__ __device__ constexpr uint32_t flt_smem_bytes(int D, int Cpad)
 {
-    // X tile | centres | norms | pair exchange (2 x 128 x 16 B) | 2 barriers + slots
-    return (uint32_t)(D * 2 * kFltRows) + (uint32_t)(Cpad * D * 2) + (uint32_t)(Cpad * 4) + 4096u + 64u;
+    // X tile | centres | norms | pair exchange (3 x 128 x 16 B) | 2 barriers + slots
+    return (uint32_t)(D * 2 * kFltRows) + (uint32_t)(Cpad * D * 2) + (uint32_t)(Cpad * 4) + 6144u + 64u;
 }
 
 // Specified binary32 distance of row `row` of the X tile to centre j of the
@@ -93,6 +94,48 @@ __device__ __forceinline__ void encode_residual_smem(const uint8_t *sX, const ui
         words[w] = 0u;
 #pragma unroll
     for (int g = 0; g < CH / G; ++g) {
+        if constexpr (G <= 32) {
+            // the group's residuals stay in registers
+            float r[G];
+#pragma unroll
+            for (int uu = 0; uu < G / 8; ++uu) {
+                const int u = half * (CH / 8) + g * (G / 8) + uu;
+                const uint4 xw = *reinterpret_cast<const uint4 *>(sX + sw128_unit_offset(row, u, kFltRows));
+                const uint4 mw = *reinterpret_cast<const uint4 *>(sMu + sw128_unit_offset(best, u, Cpad));
+                const uint32_t xa[4] = {xw.x, xw.y, xw.z, xw.w}, ma[4] = {mw.x, mw.y, mw.z, mw.w};
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    const float2 d = sub2(make_float2(bf16_lo(xa[k]), bf16_hi(xa[k])),
+                                          make_float2(bf16_lo(ma[k]), bf16_hi(ma[k])));
+                    r[uu * 8 + 2 * k] = d.x;
+                    r[uu * 8 + 2 * k + 1] = d.y;
+                }
+            }
+            float mn = r[0], mx = r[0];
+#pragma unroll
+            for (int c = 1; c < G; ++c) {
+                mn = fminf(mn, r[c]);
+                mx = fmaxf(mx, r[c]);
+            }
+            if (mn == 0.0f || mx == 0.0f) {
+                // a zero extreme: take its sign exactly as the ordered strict scan does
+                mn = r[0];
+                mx = r[0];
+#pragma unroll
+                for (int c = 1; c < G; ++c) {
+                    if (r[c] < mn) mn = r[c];
+                    if (r[c] > mx) mx = r[c];
+                }
+            }
+            const GroupQ gq = group_params(mn, mx, BITS);
+            meta_dst[g] = make_float2(gq.s, gq.z);
+#pragma unroll
+            for (int c = 0; c < G; ++c) {
+                const int cc = g * G + c;
+                words[cc / kPerWord] |= quant_code(r[c], gq, BITS) << ((cc % kPerWord) * BITS);
+            }
+            continue;
+        }
         float mn = 0.0f, mx = 0.0f;
 #pragma unroll
         for (int uu = 0; uu < G / 8; ++uu) {
@@ -157,8 +200,8 @@ __global__ void __launch_bounds__(kFltThreads, 2)
     uint8_t *sX = smem;
     uint8_t *sMu = smem + D * 2 * kFltRows;
     float *sNrm = reinterpret_cast<float *>(sMu + Cpad * D * 2);
-    float4 *sPair = reinterpret_cast<float4 *>(sNrm + Cpad);  // [2][128]
-    uint64_t *bars = reinterpret_cast<uint64_t *>(reinterpret_cast<uint8_t *>(sPair) + 4096);
+    float4 *sPair = reinterpret_cast<float4 *>(sNrm + Cpad);  // [3][128]: pair exchange, exact winners
+    uint64_t *bars = reinterpret_cast<uint64_t *>(reinterpret_cast<uint8_t *>(sPair) + 6144);
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 2);
     uint32_t *sMaxNrm = tmem_slot + 1;
 
@@ -260,97 +303,92 @@ __global__ void __launch_bounds__(kFltThreads, 2)
                 xx = fmaf(bf16_hi(wa[k]), bf16_hi(wa[k]), xx);
             }
         }
-        // (2) v_j = |mu_j|^2 - 2 p_j over this thread's chunks: per-chunk minima
-        float cmin[kMaxChunks];
-        float tmin = INFINITY;
+        // (2) v_j = |mu_j|^2 - 2 p_j over this thread's chunks.  The chunk-local
+        // column index rides in the low 5 mantissa bits of v, so one pass keeps
+        // the smallest and the second smallest value (the window below absorbs
+        // the <= 31 ulp this perturbs v).
+        float b1 = INFINITY, b2 = INFINITY;  // best and second best of this thread
+        int bchunk = 0;
 #pragma unroll
         for (int k = 0; k < kMaxChunks; ++k) {
-            cmin[k] = INFINITY;
             const int c = c_lo + k;
             if (c < c_hi) {
                 float p[32];
                 tmem_ld32(tmem + lane_off + (uint32_t)(c * 32), p);
-                float mn = INFINITY;
+                float m1 = INFINITY, m2 = INFINITY;
+                const float4 *nrm4 = reinterpret_cast<const float4 *>(sNrm + c * 32);
 #pragma unroll
-                for (int i = 0; i < 32; ++i)
-                    mn = fminf(mn, fmaf(-2.0f, p[i], sNrm[c * 32 + i]));
-                cmin[k] = mn;
-                tmin = fminf(tmin, mn);
+                for (int i4 = 0; i4 < 8; ++i4) {
+                    const float4 n4 = nrm4[i4];
+                    const float nn[4] = {n4.x, n4.y, n4.z, n4.w};
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const int i = i4 * 4 + e;
+                        const float v = fmaf(-2.0f, p[i], nn[e]);
+                        const float vp = __uint_as_float((__float_as_uint(v) & ~31u) | (uint32_t)i);
+                        m2 = fminf(m2, fmaxf(m1, vp));
+                        m1 = fminf(m1, vp);
+                    }
+                }
+                // fold the chunk into the thread's (best, second best)
+                if (m1 < b1) {
+                    b2 = fminf(b1, m2);
+                    b1 = m1;
+                    bchunk = c;
+                } else {
+                    b2 = fminf(b2, m1);
+                }
             }
         }
-        sPair[half * 128 + row] = make_float4(xx, tmin, 0.f, 0.f);
-        __syncthreads();
+        // (3) exchange with the partner thread of this row (warps w and w+4)
+        sPair[half * 128 + row] = make_float4(xx, b1, b2, __int_as_float(bchunk));
+        named_barrier_sync_q(warp & 3, 64);
         const float4 other = sPair[(half ^ 1) * 128 + row];
-        const float m = fminf(tmin, other.y);
         const float xn = sqrtf(xx + other.x);
-        const float thr = m + a.kappa * (xn + Mnorm) * (xn + Mnorm);
-        // (3) candidates inside the window.  tcgen05.ld is warp-collective, so
-        // a chunk is re-read when any lane of the warp needs it.
-        int count = 0, first = -1;
-#pragma unroll
-        for (int k = 0; k < kMaxChunks; ++k) {
-            const int c = c_lo + k;
-            const bool need = c < c_hi && cmin[k] <= thr;
-            if (c < c_hi && __any_sync(0xffffffffu, need)) {
-                float p[32];
-                tmem_ld32(tmem + lane_off + (uint32_t)(c * 32), p);
-                if (need) {
+        const float thr = fminf(b1, other.y) + a.kappa * (xn + Mnorm) * (xn + Mnorm);
+        const bool mine = b1 < other.y || (b1 == other.y && half == 0);
+        const float best_v = mine ? b1 : other.y;
+        const float second = fminf(fminf(b2, other.z), mine ? other.y : b1);
+        const int best_chunk = mine ? bchunk : __float_as_int(other.w);
+        int best = best_chunk * 32 + (int)(__float_as_uint(best_v) & 31u);
+        const bool exact = !(second > thr) || !(thr < INFINITY);
+        // rare: re-score the window (or every centre when the window is not
+        // finite) with the specified distance; the half-0 thread decides and
+        // hands the result to its partner.  Both warps of the pair see the same
+        // `exact` flags, so they take the branch together.
+        if (__any_sync(0xffffffffu, exact)) {
+            if (half == 0) {
+                float bd = INFINITY;
+                int bj = -1;
+                const bool all = !(thr < INFINITY);
+                for (int c = 0; c < nchunks; ++c) {
+                    float p[32];
+                    tmem_ld32(tmem + lane_off + (uint32_t)(c * 32), p);
+                    uint32_t cand = 0u;
 #pragma unroll
                     for (int i = 0; i < 32; ++i) {
-                        const float v = fmaf(-2.0f, p[i], sNrm[c * 32 + i]);
-                        if (v <= thr) {
-                            if (count == 0)
-                                first = c * 32 + i;
-                            ++count;
+                        const int j = c * 32 + i;
+                        const float v = fmaf(-2.0f, p[i], sNrm[j]);
+                        if (exact && j < a.C && (all || v <= thr))
+                            cand |= 1u << i;
+                    }
+                    while (cand) {  // increasing index order
+                        const int i = __ffs(cand) - 1;
+                        cand &= cand - 1u;
+                        const int j = c * 32 + i;
+                        const float dj = spec_distance_smem<D>(sX, sMu, Cpad, row, j);
+                        if (bj < 0 || dj < bd) {
+                            bd = dj;
+                            bj = j;
                         }
                     }
                 }
+                sPair[2 * 128 + row] = make_float4(__int_as_float(bj), 0.f, 0.f, 0.f);
             }
-        }
-        __syncthreads();  // both halves have read sPair
-        sPair[half * 128 + row] = make_float4(__int_as_float(count), __int_as_float(first), 0.f, 0.f);
-        __syncthreads();
-        const float4 o2 = sPair[(half ^ 1) * 128 + row];
-        const int count_all = count + __float_as_int(o2.x);
-        int best = half == 0 ? (count > 0 ? first : __float_as_int(o2.y))
-                             : (__float_as_int(o2.x) > 0 ? __float_as_int(o2.y) : first);
-        const bool exact = count_all != 1 || !(thr < INFINITY);
-        __syncthreads();  // both halves have read the counts
-        // rare: re-score the window (or every centre when the window is not
-        // finite) with the specified distance; the half-0 thread decides.  The
-        // warp reads TMEM together whenever one of its rows needs this.
-        if (half == 0 && __any_sync(0xffffffffu, exact)) {
-            float bd = INFINITY;
-            int bj = -1;
-            const bool all = !(thr < INFINITY);
-            for (int c = 0; c < nchunks; ++c) {
-                float p[32];
-                tmem_ld32(tmem + lane_off + (uint32_t)(c * 32), p);
-                uint32_t cand = 0u;
-#pragma unroll
-                for (int i = 0; i < 32; ++i) {
-                    const int j = c * 32 + i;
-                    const float v = fmaf(-2.0f, p[i], sNrm[j]);
-                    if (exact && j < a.C && (all || v <= thr))
-                        cand |= 1u << i;
-                }
-                while (cand) {  // increasing index order
-                    const int i = __ffs(cand) - 1;
-                    cand &= cand - 1u;
-                    const int j = c * 32 + i;
-                    const float dj = spec_distance_smem<D>(sX, sMu, Cpad, row, j);
-                    if (bj < 0 || dj < bd) {
-                        bd = dj;
-                        bj = j;
-                    }
-                }
-            }
+            named_barrier_sync_q(warp & 3, 64);
             if (exact)
-                sPair[row] = make_float4(__int_as_float(bj), 0.f, 0.f, 0.f);
+                best = __float_as_int(sPair[2 * 128 + row].x);
         }
-        __syncthreads();
-        if (exact)
-            best = __float_as_int(sPair[row].x);
         if (best < 0 || best >= a.C)
             best = 0;  // unreachable for finite inputs
 

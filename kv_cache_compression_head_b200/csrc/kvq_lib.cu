@@ -178,12 +178,14 @@ kvq_status launch_filter_g(int G, const CUtensorMap &m, const FilterArgs &a, cud
 // Window factor of the certified candidate set (see encode_filter.cuh):
 // kappa = 4 (eps_tc + gamma_d + 2u + gamma_{d+2}), eps_tc = d 2^-21 bounding
 // the tensor-core accumulation error relative to sum |x_c mu_c|.
+// Plus 2^-16 for the column index carried in the low 5 mantissa bits of v
+// (<= 31 ulp each on the smallest and on the compared value, |v| <= (|x|+M)^2).
 float filter_kappa(int D)
 {
     const double u = ldexp(1.0, -24);
     const double eps_tc = D * ldexp(1.0, -21);
     const double g_d = D * u / (1.0 - D * u), g_d2 = (D + 2) * u / (1.0 - (D + 2) * u);
-    return (float)(4.0 * (eps_tc + g_d + 2.0 * u + g_d2));
+    return (float)(4.0 * (eps_tc + g_d + 2.0 * u + g_d2) + ldexp(1.0, -16));
 }
 
 kvq_status launch_encode_filter(int D, int bits, int G, const void *x, const EncodeArgs &e, cudaStream_t s)
@@ -221,6 +223,52 @@ kvq_status launch_encode(int D, const EncodeArgs &e, cudaStream_t s)
     if (filter_applies(D, e.C, e.G, e.x_bf16 != 0))
         return launch_encode_filter(D, e.bits, e.G, e.x, e, s);
     return launch_encode_direct(D, e, s);
+}
+
+// Per-centre sums of one k-means round: shared-memory binary64 partial sums
+// per (head, 32- or 16-channel slice, token range) where they fit, else one
+// global binary64 atomic per channel of every token.
+kvq_status launch_fit_accumulate(const FitArgs &f, cudaStream_t s)
+{
+    const int64_t n_units = f.T * f.H * (f.D / 8);
+    const size_t smem32 = (size_t)f.C * 32 * 8, smem16 = (size_t)f.C * 16 * 8;
+    static bool configured[64][2] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64)
+        return KVQ_ERR_CUDA;
+    const int W = smem32 <= 160 * 1024 ? 32 : (smem16 <= 160 * 1024 ? 16 : 0);
+    if (W == 0) {
+        fit_accumulate_kernel<<<(unsigned)ceil_div(n_units, 256), 256, 0, s>>>(f);
+        return launch_status();
+    }
+    const size_t smem = (size_t)f.C * W * 8;
+    const int slices = f.D / W;
+    // about four blocks per SM overall
+    const int64_t want = (int64_t)4 * sm_count();
+    int64_t chunks = want / ((int64_t)f.H * slices);
+    if (chunks < 1)
+        chunks = 1;
+    const int64_t per = (f.T + chunks - 1) / chunks;
+    chunks = (f.T + per - 1) / per;
+    const dim3 grid((unsigned)chunks, (unsigned)f.H, (unsigned)slices);
+    if (W == 32) {
+        if (!configured[dev][0]) {
+            if (cudaFuncSetAttribute(fit_accumulate_smem_kernel<32>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     160 * 1024) != cudaSuccess)
+                return KVQ_ERR_CUDA;
+            configured[dev][0] = true;
+        }
+        fit_accumulate_smem_kernel<32><<<grid, 256, smem, s>>>(f, per);
+    } else {
+        if (!configured[dev][1]) {
+            if (cudaFuncSetAttribute(fit_accumulate_smem_kernel<16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     160 * 1024) != cudaSuccess)
+                return KVQ_ERR_CUDA;
+            configured[dev][1] = true;
+        }
+        fit_accumulate_smem_kernel<16><<<grid, 256, smem, s>>>(f, per);
+    }
+    return launch_status();
 }
 
 size_t fit_workspace(const kvq_codec_desc *d, int64_t T)
@@ -444,14 +492,12 @@ kvq_status kvq_fit_centroids(const kvq_codec_desc *desc, const void *x, kvq_dtyp
     e.cent = f.cent;
     e.idx = reinterpret_cast<uint16_t *>(ws);
     e.assign_only = 1;
-    const int64_t n_units = T * H * (D / 8);
     for (int it = 0; it < iters; ++it) {
         if ((st = launch_encode(D, e, s)) != KVQ_OK)
             return st;
         if (cudaMemsetAsync(ws + idx_b, 0, cnt_b + (size_t)H * C * D * 8, s) != cudaSuccess)
             return KVQ_ERR_CUDA;
-        fit_accumulate_kernel<<<(unsigned)ceil_div(n_units, 256), 256, 0, s>>>(f);
-        if ((st = launch_status()) != KVQ_OK)
+        if ((st = launch_fit_accumulate(f, s)) != KVQ_OK)
             return st;
         fit_update_kernel<<<(unsigned)ceil_div(n_cent, 256), 256, 0, s>>>(f);
         if ((st = launch_status()) != KVQ_OK)

@@ -170,9 +170,11 @@ def work_model(w):
     dec_bytes = sum(th * (stored(b) + 2 * d) for b in (w.bits_k, w.bits_v))  # read compressed, write bf16
     attn_flops = 4.0 * Tq * T * d * H
     merge_bytes = (HISTORY_BLOCKS + 1) * Tq * H * d * 4 + (HISTORY_BLOCKS + 1) * Tq * H * 4
-    assign_ops = 3.0 * th * C * d * 2  # exact distance: sub, mul, add per channel per centre (K and V)
+    # fit, per k-means round and token-head: the assignment reads x and writes
+    # its index, the accumulation reads x and the index (K and V)
+    fit_bytes = 2 * w.kmeans_iters * th * (2 * d + 2 + 2 * d + 2)
     return {"encode_bytes": enc_bytes, "decode_bytes": dec_bytes, "attention_flops": attn_flops,
-            "merge_bytes": merge_bytes, "assign_ops": assign_ops}
+            "merge_bytes": merge_bytes, "fit_bytes": fit_bytes}
 
 
 # ----------------------------------------------------------------------------
@@ -340,13 +342,9 @@ def run_gpu(args):
         enc_gbps = wm["encode_bytes"] / (row_mean["encode"] / 1e3) / 1e9
         dec_gbps = wm["decode_bytes"] / (row_mean["decode"] / 1e3) / 1e9
         merge_gbps = wm["merge_bytes"] / (row_mean["merge"] / 1e3) / 1e9
-        # exact assignment on CUDA cores: separately rounded sub, mul, add per
-        # channel per centre; peak = 148 SMs x 128 FP32 lanes x 1.965 GHz
-        alu_peak_tops = 148 * 128 * 1.965e9 / 1e12
-        fit_tops = wm["assign_ops"] * (w.kmeans_iters) / (row_mean["fit"] / 1e3) / 1e12
+        fit_gbps = wm["fit_bytes"] / (row_mean["fit"] / 1e3) / 1e9
         rows = {
-            "fit": {"ms": row_mean["fit"], "bound": "alu", "achieved": fit_tops, "peak": alu_peak_tops,
-                    "unit": "Top/s", "frac": fit_tops / alu_peak_tops},
+            "fit": {"ms": row_mean["fit"], "gbps": fit_gbps, "hbm_frac": fit_gbps / hbm},
             "encode": {"ms": row_mean["encode"], "tokens_per_s": w.history_tokens / (row_mean["encode"] / 1e3),
                        "gbps": enc_gbps, "hbm_frac": enc_gbps / hbm},
             "decode": {"ms": row_mean["decode"], "gbps": dec_gbps, "hbm_frac": dec_gbps / hbm},

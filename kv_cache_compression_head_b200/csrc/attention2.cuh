@@ -17,19 +17,21 @@
 //   warps 9-12  softmax for query tile 0, warps 13-16 for query tile 1: one
 //               thread per query row (its TMEM lane); online softmax in the
 //               exp2 domain with lazy rescaling (O in TMEM is rescaled only
-//               when the running maximum grows by more than 2^8); P (fp16)
-//               goes to the shared buffers of the K stage the tile came from.
-// Shared memory: Q tiles 2 x 32 KB, two K stages of 2 x 32 KB (K_hi, K_lo,
-// later P_0, P_1), one V tile of 32 KB (d = 128).  TMEM: S_0, S_1 (128 columns
-// each) and O_0, O_1 (d columns each).
+//               when the running maximum grows by more than 2^8); P (fp16
+//               pairs) is written back over the S tile it came from and read
+//               by the P V MMA straight from TMEM.
+// Shared memory: Q tiles 2 x 32 KB, two K stages of 2 x 32 KB (K_hi, K_lo),
+// one V tile of 32 KB (d = 128).  TMEM: S_0, S_1 (128 columns each; P_i in the
+// first 64 columns of S_i) and O_0, O_1 (d columns each).
 //
 // Ordering (mbarriers; parity = use count & 1):
 //   kfull[s]  producer -> MMA   K stage s holds tile j (j = s mod 2)
 //   vfull     producer -> MMA   V tile j written
-//   sfull[i]  MMA -> softmax    S_i(j) complete.  The QK MMAs run hi(0),
-//             hi(1), lo(0), lo(1), so S_0 completes after K_hi's last read and
-//             S_1 after K_lo's: each P_i can overwrite its slot at once
-//   pfull[i]  softmax -> MMA    P_i(j) written, O_i rescaled
+//   sfull[i]  MMA -> softmax    S_i(j) complete (QK MMAs run hi(0), hi(1),
+//             lo(0), lo(1))
+//   pfull[i]  softmax -> MMA    P_i(j) in TMEM, O_i rescaled.  The next
+//             QK_i overwrites S_i only after P V_i(j), issued before it, has
+//             read P_i (tcgen05 MMAs of one thread execute in order)
 //   pvdone    MMA -> producer   PV_0(j), PV_1(j) complete: V and K stage j free
 //   ofull     MMA -> softmax    last PV complete
 // Every wait is bounded and also polls a shared abort flag, so that one
@@ -51,8 +53,7 @@ template <int D>
 struct A2Smem {
     static constexpr uint32_t kQ = D * 2 * 128;
     static constexpr uint32_t kKt = D * 2 * 128;           // one K_hi / K_lo tile
-    static constexpr uint32_t kPt = 2 * 128 * 128;         // one P tile (fp16)
-    static constexpr uint32_t kSlot = kKt > kPt ? kKt : kPt;
+    static constexpr uint32_t kSlot = kKt;
     static constexpr uint32_t offQ0 = 0, offQ1 = kQ;
     static constexpr uint32_t offStage = 2 * kQ;          // stage s slot t at offStage + (2s + t) kSlot
     static constexpr uint32_t offV = offStage + 4 * kSlot;
@@ -207,11 +208,37 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const float *v)
     asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
 
-// One 32-column chunk of P = exp2(s * scale - m), packed fp16, into 4 swizzled
-// 16-byte units of the P tile; returns the chunk's sum of the (unrounded) p.
+// 16 consecutive 32-bit TMEM columns of this thread's lane.
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t *v)
+{
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+        "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(taddr),
+        "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]), "r"(v[8]),
+        "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15])
+        : "memory");
+}
+
+// D[tmem] (+)= A[tmem] * B[smem]; A is M rows (lanes) x K 16-bit elements, two
+// per 32-bit column (even element in the low half).
+__device__ __forceinline__ void umma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc, uint32_t idesc,
+                                        uint32_t accumulate)
+{
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}\n" ::"r"(d_tmem),
+        "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+// One 32-column chunk of P = exp2(s * scale - m), packed fp16 pairs, written
+// back into TMEM as 16 columns of the A operand of P V (columns 16 cb ..
+// 16 cb + 15 of the S tile, which this thread has already read); returns the
+// chunk's sum of the (unrounded) p.
 template <bool MASKED>
 __device__ __forceinline__ float a2_softmax_chunk(const float *sv, float scale, float m, int cbase, int nvalid,
-                                                  uint8_t *pt, uint32_t r, int cb)
+                                                  uint32_t tp)
 {
     float lt = 0.0f;
     uint32_t pk[16];
@@ -226,10 +253,7 @@ __device__ __forceinline__ float a2_softmax_chunk(const float *sv, float scale, 
         lt += p0 + p1;
         pk[i / 2] = pack_f16x2_sat(p0, p1);
     }
-#pragma unroll
-    for (int uu = 0; uu < 4; ++uu)
-        *reinterpret_cast<uint4 *>(pt + sw128_unit_offset(r, cb * 4 + uu, 128)) =
-            make_uint4(pk[4 * uu], pk[4 * uu + 1], pk[4 * uu + 2], pk[4 * uu + 3]);
+    tmem_st16(tp, pk);
     return lt;
 }
 
@@ -365,14 +389,11 @@ __global__ void __launch_bounds__(kA2Threads, 1) attention2_kernel(AttnArgs a)
                     if (!ok)
                         break;
                     tc_fence_after();
-                    const uint32_t aP = smem_u32(slot(s, qt));
 #pragma unroll
-                    for (int ks = 0; ks < 128 / 16; ++ks) {
-                        const uint32_t poff = (uint32_t)(ks >> 2) * (128u * 128u) + (uint32_t)(ks & 3) * 32u;
-                        umma_ss(tO[qt], sdesc_sw128(aP + poff, 16, 1024),
+                    for (int ks = 0; ks < 128 / 16; ++ks)
+                        umma_ts(tO[qt], tS[qt] + (uint32_t)ks * 8u,
                                 sdesc_sw128(aV + (uint32_t)ks * 2048u, 128u * 128u, 1024), idescO,
                                 (j > 0 || ks > 0) ? 1u : 0u);
-                    }
                 }
                 if (!ok)
                     break;
@@ -440,21 +461,21 @@ __global__ void __launch_bounds__(kA2Threads, 1) attention2_kernel(AttnArgs a)
                 l *= alpha;
                 m_used = m_new;
             }
-            // P = exp2(s * scale - m_used), fp16, into the stage's slot (K_hi
-            // for tile 0, K_lo for tile 1; both already consumed by the MMAs)
-            uint8_t *pt = slot(j & 1, grp);
+            // P = exp2(s * scale - m_used), fp16 pairs, back into the first 64
+            // columns of S_i: the A operand of P V, read from TMEM
             float lt = 0.0f;
 #pragma unroll
             for (int cb = 0; cb < 4; ++cb) {
                 float sv[32];
                 tmem_ld32(tS + lane_off + (uint32_t)(cb * 32), sv);
+                const uint32_t tp = tS + lane_off + (uint32_t)(cb * 16);
                 if (nvalid == 128)
-                    lt += a2_softmax_chunk<false>(sv, a.scale_log2, m_used, cb * 32, nvalid, pt, r, cb);
+                    lt += a2_softmax_chunk<false>(sv, a.scale_log2, m_used, cb * 32, nvalid, tp);
                 else
-                    lt += a2_softmax_chunk<true>(sv, a.scale_log2, m_used, cb * 32, nvalid, pt, r, cb);
+                    lt += a2_softmax_chunk<true>(sv, a.scale_log2, m_used, cb * 32, nvalid, tp);
             }
+            asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
             l += lt;
-            fence_proxy_async_smem();
             tc_fence_before();
             mbar_arrive(bar(grp ? B_PFULL1 : B_PFULL0));
         }

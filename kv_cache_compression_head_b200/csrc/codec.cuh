@@ -360,17 +360,35 @@ __global__ void __launch_bounds__(256) fit_accumulate_smem_kernel(FitArgs a, int
     for (int e = threadIdx.x; e < a.C * W; e += blockDim.x)
         s_sum[e] = 0.0;
     __syncthreads();
-    // a group of W lanes handles one token; lane c adds channel slice*W + c
-    constexpr int kGroups = 256 / W;
+    // a group of W lanes handles one token; lane c adds channel slice*W + c.
+    // Tokens go in batches of 8 so that their loads are in flight together.
+    constexpr int kGroups = 256 / W, kBatch = 8;
     const int grp = threadIdx.x / W, c = threadIdx.x % W;
-    for (int64_t t = t_lo + grp; t < t_hi; t += kGroups) {
-        const int j = a.idx[(int64_t)h * a.T + t];
-        const int64_t e = (t * a.H + h) * a.D + slice * W + c;
-        const float v = a.x_bf16 ? __uint_as_float((uint32_t)static_cast<const uint16_t *>(a.x)[e] << 16)
-                                 : static_cast<const float *>(a.x)[e];
-        atomicAdd(&s_sum[j * W + c], (double)v);
-        if (slice == 0 && c == 0)
-            atomicAdd(a.counts + (int64_t)h * a.C + j, 1u);
+    for (int64_t t0 = t_lo + grp; t0 < t_hi; t0 += (int64_t)kGroups * kBatch) {
+        int j[kBatch];
+        float v[kBatch];
+#pragma unroll
+        for (int b = 0; b < kBatch; ++b) {
+            const int64_t t = t0 + (int64_t)b * kGroups;
+            j[b] = t < t_hi ? __ldg(a.idx + (int64_t)h * a.T + t) : -1;
+        }
+#pragma unroll
+        for (int b = 0; b < kBatch; ++b) {
+            const int64_t t = t0 + (int64_t)b * kGroups;
+            const int64_t e = (t * a.H + h) * a.D + slice * W + c;
+            v[b] = 0.0f;
+            if (j[b] >= 0)
+                v[b] = a.x_bf16 ? __uint_as_float((uint32_t)__ldg(static_cast<const uint16_t *>(a.x) + e) << 16)
+                                : __ldg(static_cast<const float *>(a.x) + e);
+        }
+#pragma unroll
+        for (int b = 0; b < kBatch; ++b) {
+            if (j[b] < 0)
+                continue;
+            atomicAdd(&s_sum[j[b] * W + c], (double)v[b]);
+            if (slice == 0 && c == 0)
+                atomicAdd(a.counts + (int64_t)h * a.C + j[b], 1u);
+        }
     }
     __syncthreads();
     for (int e = threadIdx.x; e < a.C * W; e += blockDim.x) {

@@ -298,10 +298,7 @@ struct FitArgs {
     int H;
     int D;
     int C;
-    uint16_t *cent;          // [H][C][D]
-    const uint16_t *idx;     // [H][T]
-    double *sums;            // [H][C][D]
-    unsigned int *counts;    // [H][C]
+    uint16_t *cent;  // [H][C][D]
 };
 
 // mu_j = bf16(x_j) for the first C tokens.
@@ -322,95 +319,161 @@ __global__ void __launch_bounds__(256) fit_seed_kernel(FitArgs a)
     a.cent[gid] = *reinterpret_cast<const uint16_t *>(&b);
 }
 
-// sums[h][idx][c] += x (binary64), counts[h][idx] += 1; one thread per
-// 8 channels of a token-head.
-__global__ void __launch_bounds__(256) fit_accumulate_kernel(FitArgs a)
+// ---------------------------------------------------------------------------
+// Deterministic centre update by bucket sort: every centre's tokens are
+// gathered in token order and summed sequentially in binary64, exactly as the
+// specification's sequential sum does, so the new centres do not depend on
+// thread timing.
+//   fit_hist:    per (head, token chunk) centre counts            [H][nch][C]
+//   fit_scan:    per head, bucket starts and per-chunk bases       [H][C], [H][nch][C]
+//   fit_scatter: per (head, chunk), stable placement of token ids  order[H][T]
+//   fit_bucket_update: one warp per (head, centre): sum in token order,
+//                mean in binary64, round to binary32 then bf16 (empty: keep)
+// ---------------------------------------------------------------------------
+constexpr int kFitChunk = 2048;
+
+struct FitSortArgs {
+    const void *x;
+    int x_bf16;
+    int64_t T;
+    int H;
+    int D;
+    int C;
+    int nchunks;
+    uint16_t *cent;          // [H][C][D]
+    const uint16_t *idx;     // [H][T]
+    int *chunk_counts;       // [H][nchunks][C] (counts, then bases)
+    int *bucket_start;       // [H][C + 1]
+    int *order;              // [H][T]
+};
+
+__global__ void __launch_bounds__(256) fit_hist_kernel(FitSortArgs a)
 {
-    const int units = a.D / 8;
-    const int64_t gid = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-    const int64_t total = a.T * a.H * units;
-    if (gid >= total)
-        return;
-    const int u = (int)(gid % units);
-    const int64_t th_in = gid / units;  // t * H + h
-    const int h = (int)(th_in % a.H);
-    const int64_t t = th_in / a.H;
-    const int j = a.idx[(int64_t)h * a.T + t];
-    float xv[8];
-    load_x8(a.x, a.x_bf16, th_in * a.D + u * 8, xv);
-    double *dst = a.sums + ((int64_t)h * a.C + j) * a.D + u * 8;
-#pragma unroll
-    for (int k = 0; k < 8; ++k)
-        atomicAdd(dst + k, (double)xv[k]);
-    if (u == 0)
-        atomicAdd(a.counts + (int64_t)h * a.C + j, 1u);
+    extern __shared__ int s_cnt[];  // [C]
+    const int h = blockIdx.y, ch = blockIdx.x;
+    for (int j = threadIdx.x; j < a.C; j += blockDim.x)
+        s_cnt[j] = 0;
+    __syncthreads();
+    const int64_t t0 = (int64_t)ch * kFitChunk;
+    const int64_t t1 = min(a.T, t0 + kFitChunk);
+    for (int64_t t = t0 + threadIdx.x; t < t1; t += blockDim.x)
+        atomicAdd(&s_cnt[a.idx[(int64_t)h * a.T + t]], 1);
+    __syncthreads();
+    int *dst = a.chunk_counts + ((int64_t)h * a.nchunks + ch) * a.C;
+    for (int j = threadIdx.x; j < a.C; j += blockDim.x)
+        dst[j] = s_cnt[j];
 }
 
-// Same sums with far fewer global atomics: a block owns one head, one slice
-// of W channels and a contiguous token range; it accumulates into binary64
-// shared-memory sums [C][W] and adds them to the global sums once at the end.
-// Token counts are added by the slice-0 blocks.
-template <int W>
-__global__ void __launch_bounds__(256) fit_accumulate_smem_kernel(FitArgs a, int64_t tokens_per_block)
+// One block per head.  Bucket totals -> exclusive prefix over centres (bucket
+// starts); then each chunk's count is replaced by the chunk's base inside the
+// centre's bucket (prefix over chunks).
+__global__ void __launch_bounds__(1024) fit_scan_kernel(FitSortArgs a)
 {
-    extern __shared__ double s_sum[];  // [C][W]
-    const int h = blockIdx.y, slice = blockIdx.z;
-    const int64_t t_lo = (int64_t)blockIdx.x * tokens_per_block;
-    const int64_t t_hi = min(a.T, t_lo + tokens_per_block);
-    for (int e = threadIdx.x; e < a.C * W; e += blockDim.x)
-        s_sum[e] = 0.0;
-    __syncthreads();
-    // a group of W lanes handles one token; lane c adds channel slice*W + c.
-    // Tokens go in batches of 8 so that their loads are in flight together.
-    constexpr int kGroups = 256 / W, kBatch = 8;
-    const int grp = threadIdx.x / W, c = threadIdx.x % W;
-    for (int64_t t0 = t_lo + grp; t0 < t_hi; t0 += (int64_t)kGroups * kBatch) {
-        int j[kBatch];
-        float v[kBatch];
-#pragma unroll
-        for (int b = 0; b < kBatch; ++b) {
-            const int64_t t = t0 + (int64_t)b * kGroups;
-            j[b] = t < t_hi ? __ldg(a.idx + (int64_t)h * a.T + t) : -1;
+    extern __shared__ int s_tot[];  // [C]
+    const int h = blockIdx.x;
+    int *cc = a.chunk_counts + (int64_t)h * a.nchunks * a.C;
+    for (int j = threadIdx.x; j < a.C; j += blockDim.x) {
+        int run = 0;
+        for (int ch = 0; ch < a.nchunks; ++ch) {
+            const int c = cc[(int64_t)ch * a.C + j];
+            cc[(int64_t)ch * a.C + j] = run;
+            run += c;
         }
-#pragma unroll
-        for (int b = 0; b < kBatch; ++b) {
-            const int64_t t = t0 + (int64_t)b * kGroups;
-            const int64_t e = (t * a.H + h) * a.D + slice * W + c;
-            v[b] = 0.0f;
-            if (j[b] >= 0)
-                v[b] = a.x_bf16 ? __uint_as_float((uint32_t)__ldg(static_cast<const uint16_t *>(a.x) + e) << 16)
-                                : __ldg(static_cast<const float *>(a.x) + e);
-        }
-#pragma unroll
-        for (int b = 0; b < kBatch; ++b) {
-            if (j[b] < 0)
-                continue;
-            atomicAdd(&s_sum[j[b] * W + c], (double)v[b]);
-            if (slice == 0 && c == 0)
-                atomicAdd(a.counts + (int64_t)h * a.C + j[b], 1u);
-        }
+        s_tot[j] = run;
     }
     __syncthreads();
-    for (int e = threadIdx.x; e < a.C * W; e += blockDim.x) {
-        const double v = s_sum[e];
-        if (v != 0.0)
-            atomicAdd(a.sums + ((int64_t)h * a.C + e / W) * a.D + slice * W + e % W, v);
+    if (threadIdx.x == 0) {
+        int run = 0;
+        int *bs = a.bucket_start + (int64_t)h * (a.C + 1);
+        for (int j = 0; j < a.C; ++j) {
+            bs[j] = run;
+            run += s_tot[j];
+        }
+        bs[a.C] = run;
     }
 }
 
-// mu_j = bf16(float(sum_j / n_j)) where n_j > 0; empty centres keep mu_j.
-__global__ void __launch_bounds__(256) fit_update_kernel(FitArgs a)
+// One warp per (head, chunk): tokens in order, 32 at a time; lanes holding the
+// same centre get consecutive slots in lane order, so every bucket lists its
+// tokens in increasing token order.
+__global__ void __launch_bounds__(32) fit_scatter_kernel(FitSortArgs a)
 {
-    const int64_t gid = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-    const int64_t total = (int64_t)a.H * a.C * a.D;
-    if (gid >= total)
+    extern __shared__ int s_cur[];  // [C] running offset of each centre in this chunk
+    const int h = blockIdx.y, ch = blockIdx.x, lane = threadIdx.x;
+    const int *base = a.chunk_counts + ((int64_t)h * a.nchunks + ch) * a.C;
+    const int *bs = a.bucket_start + (int64_t)h * (a.C + 1);
+    for (int j = lane; j < a.C; j += 32)
+        s_cur[j] = bs[j] + base[j];
+    __syncwarp();
+    const int64_t t0 = (int64_t)ch * kFitChunk;
+    const int64_t t1 = min(a.T, t0 + kFitChunk);
+    for (int64_t tb = t0; tb < t1; tb += 32) {
+        const int64_t t = tb + lane;
+        const bool on = t < t1;
+        const int j = on ? (int)a.idx[(int64_t)h * a.T + t] : -1;
+        const unsigned peers = __match_any_sync(0xffffffffu, j);
+        const int rank = __popc(peers & ((1u << lane) - 1u));
+        const int leader = __ffs(peers) - 1;
+        int slot = 0;
+        if (on)
+            slot = s_cur[j] + rank;
+        __syncwarp();
+        if (on && lane == leader)
+            s_cur[j] += __popc(peers);
+        __syncwarp();
+        if (on)
+            a.order[(int64_t)h * a.T + slot] = (int)t;
+    }
+}
+
+// One warp per (head, centre); lane l owns channels 4l .. 4l+3 (D = 128) or
+// 2l .. 2l+1 (D = 64).  Sums in binary64 in token order.
+template <int D>
+__global__ void __launch_bounds__(256) fit_bucket_update_kernel(FitSortArgs a)
+{
+    constexpr int kPer = D / 32;
+    const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
+    if (warp >= a.H * a.C)
         return;
-    const unsigned n = a.counts[gid / a.D];
-    if (n == 0)
-        return;
-    const double mean = __ddiv_rn(a.sums[gid], (double)n);
-    const __nv_bfloat16 b = __float2bfloat16_rn(__double2float_rn(mean));
-    a.cent[gid] = *reinterpret_cast<const uint16_t *>(&b);
+    const int h = warp / a.C, j = warp % a.C;
+    const int *bs = a.bucket_start + (int64_t)h * (a.C + 1);
+    const int b0 = bs[j], b1 = bs[j + 1];
+    if (b1 == b0)
+        return;  // empty: the centre keeps its value
+    const int *ord = a.order + (int64_t)h * a.T;
+    double acc[kPer];
+#pragma unroll
+    for (int k = 0; k < kPer; ++k)
+        acc[k] = 0.0;
+    for (int i = b0; i < b1; ++i) {
+        const int64_t t = ord[i];
+        const int64_t e = (t * a.H + h) * D + lane * kPer;
+        float v[kPer];
+        if (a.x_bf16) {
+            if (kPer == 4) {
+                const uint2 w = __ldg(reinterpret_cast<const uint2 *>(static_cast<const uint16_t *>(a.x) + e));
+                v[0] = bf16_lo(w.x); v[1] = bf16_hi(w.x);
+                v[2 % kPer] = bf16_lo(w.y); v[3 % kPer] = bf16_hi(w.y);
+            } else {
+                const uint32_t w = __ldg(reinterpret_cast<const uint32_t *>(static_cast<const uint16_t *>(a.x) + e));
+                v[0] = bf16_lo(w); v[1 % kPer] = bf16_hi(w);
+            }
+        } else {
+#pragma unroll
+            for (int k = 0; k < kPer; ++k)
+                v[k] = __ldg(static_cast<const float *>(a.x) + e + k);
+        }
+#pragma unroll
+        for (int k = 0; k < kPer; ++k)
+            acc[k] = __dadd_rn(acc[k], (double)v[k]);
+    }
+    const double n = (double)(b1 - b0);
+    uint16_t *dst = a.cent + ((int64_t)h * a.C + j) * D + lane * kPer;
+#pragma unroll
+    for (int k = 0; k < kPer; ++k) {
+        const __nv_bfloat16 b = __float2bfloat16_rn(__double2float_rn(__ddiv_rn(acc[k], n)));
+        dst[k] = *reinterpret_cast<const uint16_t *>(&b);
+    }
 }
 
 }  // namespace kvq

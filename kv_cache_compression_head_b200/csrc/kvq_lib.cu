@@ -225,58 +225,41 @@ kvq_status launch_encode(int D, const EncodeArgs &e, cudaStream_t s)
     return launch_encode_direct(D, e, s);
 }
 
-// Per-centre sums of one k-means round: shared-memory binary64 partial sums
-// per (head, 32- or 16-channel slice, token range) where they fit, else one
-// global binary64 atomic per channel of every token.
-kvq_status launch_fit_accumulate(const FitArgs &f, cudaStream_t s)
+// Fit workspace: idx [H][T] u16 | per-chunk centre counts [H][nch][C] i32 |
+// bucket starts [H][C+1] i32 | token order [H][T] i32.
+struct FitLayout {
+    size_t idx, counts, starts, order, total;
+    int nchunks;
+};
+
+FitLayout fit_layout(const kvq_codec_desc *d, int64_t T)
 {
-    const int64_t n_units = f.T * f.H * (f.D / 8);
-    const size_t smem32 = (size_t)f.C * 32 * 8, smem16 = (size_t)f.C * 16 * 8;
-    static bool configured[64][2] = {};
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64)
-        return KVQ_ERR_CUDA;
-    const int W = smem32 <= 160 * 1024 ? 32 : (smem16 <= 160 * 1024 ? 16 : 0);
-    if (W == 0) {
-        fit_accumulate_kernel<<<(unsigned)ceil_div(n_units, 256), 256, 0, s>>>(f);
-        return launch_status();
-    }
-    const size_t smem = (size_t)f.C * W * 8;
-    const int slices = f.D / W;
-    // about four blocks per SM overall
-    const int64_t want = (int64_t)4 * sm_count();
-    int64_t chunks = want / ((int64_t)f.H * slices);
-    if (chunks < 1)
-        chunks = 1;
-    const int64_t per = (f.T + chunks - 1) / chunks;
-    chunks = (f.T + per - 1) / per;
-    const dim3 grid((unsigned)chunks, (unsigned)f.H, (unsigned)slices);
-    if (W == 32) {
-        if (!configured[dev][0]) {
-            if (cudaFuncSetAttribute(fit_accumulate_smem_kernel<32>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                     160 * 1024) != cudaSuccess)
-                return KVQ_ERR_CUDA;
-            configured[dev][0] = true;
-        }
-        fit_accumulate_smem_kernel<32><<<grid, 256, smem, s>>>(f, per);
-    } else {
-        if (!configured[dev][1]) {
-            if (cudaFuncSetAttribute(fit_accumulate_smem_kernel<16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                     160 * 1024) != cudaSuccess)
-                return KVQ_ERR_CUDA;
-            configured[dev][1] = true;
-        }
-        fit_accumulate_smem_kernel<16><<<grid, 256, smem, s>>>(f, per);
-    }
-    return launch_status();
+    FitLayout L;
+    const size_t H = (size_t)d->num_heads, C = (size_t)d->num_centroids;
+    L.nchunks = (int)((T + kFitChunk - 1) / kFitChunk);
+    if (L.nchunks < 1)
+        L.nchunks = 1;
+    L.idx = 0;
+    L.counts = round_up(H * (size_t)T * 2, 256);
+    L.starts = L.counts + round_up(H * (size_t)L.nchunks * C * 4, 256);
+    L.order = L.starts + round_up(H * (C + 1) * 4, 256);
+    L.total = L.order + H * (size_t)T * 4;
+    return L;
 }
 
-size_t fit_workspace(const kvq_codec_desc *d, int64_t T)
+size_t fit_workspace(const kvq_codec_desc *d, int64_t T) { return fit_layout(d, T).total; }
+
+// Largest centre count the fit's shared-memory histograms take.
+constexpr int kFitMaxC = 32768;
+
+template <typename K>
+kvq_status smem_opt_in(K kernel, size_t bytes)
 {
-    const size_t idx_b = round_up((size_t)d->num_heads * (size_t)T * 2, 256);
-    const size_t cnt_b = round_up((size_t)d->num_heads * d->num_centroids * 4, 256);
-    const size_t sum_b = (size_t)d->num_heads * d->num_centroids * d->head_dim * 8;
-    return idx_b + cnt_b + sum_b;
+    if (bytes <= 48 * 1024)
+        return KVQ_OK;
+    return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes) == cudaSuccess
+               ? KVQ_OK
+               : KVQ_ERR_CUDA;
 }
 
 kvq_status check_view(const kvq_compressed_view *v)
@@ -456,8 +439,10 @@ kvq_status kvq_fit_centroids(const kvq_codec_desc *desc, const void *x, kvq_dtyp
         return KVQ_ERR_INVALID_ARG;
     if (!aligned16(x) || !aligned16(centroids_out) || !aligned16(workspace))
         return KVQ_ERR_ALIGNMENT;
-    const size_t need = fit_workspace(desc, T);
-    if (!workspace || workspace_bytes < need)
+    if (desc->num_centroids > kFitMaxC)
+        return KVQ_ERR_UNSUPPORTED;
+    const FitLayout Lw = fit_layout(desc, T);
+    if (!workspace || workspace_bytes < Lw.total)
         return KVQ_ERR_WORKSPACE;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     const int H = desc->num_heads, D = desc->head_dim, C = desc->num_centroids;
@@ -470,15 +455,27 @@ kvq_status kvq_fit_centroids(const kvq_codec_desc *desc, const void *x, kvq_dtyp
     f.D = D;
     f.C = C;
     f.cent = static_cast<uint16_t *>(centroids_out);
-    f.idx = reinterpret_cast<uint16_t *>(ws);
-    const size_t idx_b = round_up((size_t)H * (size_t)T * 2, 256);
-    const size_t cnt_b = round_up((size_t)H * C * 4, 256);
-    f.counts = reinterpret_cast<unsigned int *>(ws + idx_b);
-    f.sums = reinterpret_cast<double *>(ws + idx_b + cnt_b);
+    FitSortArgs fs;
+    fs.x = x;
+    fs.x_bf16 = f.x_bf16;
+    fs.T = T;
+    fs.H = H;
+    fs.D = D;
+    fs.C = C;
+    fs.nchunks = Lw.nchunks;
+    fs.cent = f.cent;
+    fs.idx = reinterpret_cast<const uint16_t *>(ws + Lw.idx);
+    fs.chunk_counts = reinterpret_cast<int *>(ws + Lw.counts);
+    fs.bucket_start = reinterpret_cast<int *>(ws + Lw.starts);
+    fs.order = reinterpret_cast<int *>(ws + Lw.order);
 
     const int64_t n_cent = (int64_t)H * C * D;
     fit_seed_kernel<<<(unsigned)ceil_div(n_cent, 256), 256, 0, s>>>(f);
     if ((st = launch_status()) != KVQ_OK)
+        return st;
+    const size_t cbytes = (size_t)C * 4;
+    if ((st = smem_opt_in(fit_hist_kernel, cbytes)) != KVQ_OK || (st = smem_opt_in(fit_scan_kernel, cbytes)) != KVQ_OK ||
+        (st = smem_opt_in(fit_scatter_kernel, cbytes)) != KVQ_OK)
         return st;
     EncodeArgs e;
     memset(&e, 0, sizeof e);
@@ -490,16 +487,20 @@ kvq_status kvq_fit_centroids(const kvq_codec_desc *desc, const void *x, kvq_dtyp
     e.bits = 2;
     e.G = 16;
     e.cent = f.cent;
-    e.idx = reinterpret_cast<uint16_t *>(ws);
+    e.idx = reinterpret_cast<uint16_t *>(ws + Lw.idx);
     e.assign_only = 1;
+    const dim3 chunks((unsigned)Lw.nchunks, (unsigned)H);
     for (int it = 0; it < iters; ++it) {
         if ((st = launch_encode(D, e, s)) != KVQ_OK)
             return st;
-        if (cudaMemsetAsync(ws + idx_b, 0, cnt_b + (size_t)H * C * D * 8, s) != cudaSuccess)
-            return KVQ_ERR_CUDA;
-        if ((st = launch_fit_accumulate(f, s)) != KVQ_OK)
-            return st;
-        fit_update_kernel<<<(unsigned)ceil_div(n_cent, 256), 256, 0, s>>>(f);
+        fit_hist_kernel<<<chunks, 256, cbytes, s>>>(fs);
+        fit_scan_kernel<<<(unsigned)H, 1024, cbytes, s>>>(fs);
+        fit_scatter_kernel<<<chunks, 32, cbytes, s>>>(fs);
+        const int64_t warps = (int64_t)H * C;
+        if (D == 128)
+            fit_bucket_update_kernel<128><<<(unsigned)ceil_div(warps * 32, 256), 256, 0, s>>>(fs);
+        else
+            fit_bucket_update_kernel<64><<<(unsigned)ceil_div(warps * 32, 256), 256, 0, s>>>(fs);
         if ((st = launch_status()) != KVQ_OK)
             return st;
     }

@@ -51,7 +51,7 @@ def test_encoded_sizes_and_workspace(K):
     assert (ib + cb + mb) == 12 * 32760 * 98
     c4 = K.Codec(40, 128, 512, 4, 32)
     assert K.encoded_sizes(c4, 10)[1] == 40 * 10 * 64
-    assert K.workspace_size(K.KVQ_OP_FIT, c, 32760) > 12 * 256 * 128 * 8
+    assert K.workspace_size(K.KVQ_OP_FIT, c, 32760) >= 12 * 32760 * (2 + 4)
     assert K.workspace_size(K.KVQ_OP_ATTENTION, c, 32760, 4680) >= 4 * 4680 * 12 * 128 * 4
     assert K.workspace_size(K.KVQ_OP_ENCODE, c, 32760) == 0
 

@@ -357,3 +357,20 @@ def test_encode_ties_and_near_ties():
         _assert_encoded_equal(comp, H, T, d, bits, G, *e)
         assert np.all(e[0] < C // 2)  # ties resolved to the lower duplicate
     _status_ok()
+
+
+def test_fit_token_order_sums_with_inexact_binary64():
+    """Values spanning ~33 decades make the binary64 centre sums inexact; the
+    fit still matches the oracle bit for bit because both sum every centre's
+    tokens sequentially in token order."""
+    K = _K()
+    rng = np.random.default_rng(43)
+    T, H, d, C = 3000, 2, 128, 16
+    mag = 10.0 ** rng.uniform(-30, 3, size=(T, H, d))
+    x = _bf16_bits(rng.normal(size=(T, H, d)) * mag)
+    for it in (1, 3):
+        codec = K.Codec(H, d, C, 2, 16)
+        cent = torch.empty((H, C, d), dtype=torch.bfloat16, device="cuda")
+        K.kvq_fit_centroids(codec, to_dev(x), it, cent)
+        assert np.array_equal(bits_u16(cent), O.fit(x, C, it))
+    _status_ok()

@@ -518,6 +518,7 @@ __global__ void __launch_bounds__(kA2Threads, 1) attention2_kernel(AttnArgs a)
                 (empty || !have) ? -INFINITY : (m_used + log2f(l)) * 0.69314718055994531f;
     }
 
+    __syncwarp();  // the MMA lane rejoins its warp before the block barrier
     tc_fence_before();
     __syncthreads();
     tc_fence_after();

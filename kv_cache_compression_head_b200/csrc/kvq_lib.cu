@@ -11,6 +11,7 @@
 
 #include "attention.cuh"
 #include "attention2.cuh"
+#include "attention_pair.cuh"
 #include "codec.cuh"
 #include "common.cuh"
 #include "encode_filter.cuh"
@@ -304,11 +305,12 @@ size_t attention_workspace(const kvq_codec_desc *d, int64_t Tq)
 // Number of history sub-ranges for one attention call: the CTA count
 // (query-tile pairs x heads x splits) should fill whole waves of one CTA per
 // SM, and every sub-range should keep at least 8 history tiles.
-int attention_splits(int64_t Tq, int H, int64_t span, size_t ws_bytes, size_t ws_need)
+int attention_splits(int64_t Tq, int H, int64_t span, size_t ws_bytes, size_t ws_need, int rows_per_unit,
+                     int ctas_per_unit)
 {
     if (ws_bytes < ws_need)
         return 1;
-    const int64_t base = ((Tq + kA2Rows - 1) / kA2Rows) * H;
+    const int64_t base = ((Tq + rows_per_unit - 1) / rows_per_unit) * ctas_per_unit * H;
     const int64_t sms = sm_count();
     const int64_t tiles = (span + 127) / 128;
     int best = 1;
@@ -324,6 +326,24 @@ int attention_splits(int64_t Tq, int H, int64_t span, size_t ws_bytes, size_t ws
         }
     }
     return best;
+}
+
+kvq_status launch_attention_pair(const AttnArgs &a, cudaStream_t s)
+{
+    static bool configured[64] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64)
+        return KVQ_ERR_CUDA;
+    if (!configured[dev]) {
+        if (cudaFuncSetAttribute(attention_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)APSmem::kLaunchBytes) != cudaSuccess)
+            return KVQ_ERR_CUDA;
+        configured[dev] = true;
+    }
+    const dim3 grid((unsigned)(2 * ceil_div(a.Tq, kAPRowsPerPair)), (unsigned)a.H,
+                    (unsigned)(a.nsplit > 1 ? a.nsplit : 1));
+    attention_pair_kernel<<<grid, kAPThreads, APSmem::kLaunchBytes, s>>>(a);
+    return launch_status();
 }
 
 template <int D>
@@ -680,11 +700,17 @@ kvq_status kvq_attention_lse(const void *q, int64_t Tq, const kvq_compressed_vie
     a.nsplit = 1;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     const size_t need = attention_workspace(&k->desc, Tq);
+    // d = 128 runs on CTA pairs (512 query rows per pair), d = 64 on single CTAs
+    const bool pair = D == 128;
+    auto launch = [&](const AttnArgs &x) {
+        return pair ? launch_attention_pair(x, s) : launch_attention2<64>(x, s);
+    };
     const int nsplit = (workspace && aligned16(workspace))
-                           ? attention_splits(Tq, a.H, t_end - t_begin, workspace_bytes, need)
+                           ? attention_splits(Tq, a.H, t_end - t_begin, workspace_bytes, need,
+                                              pair ? kAPRowsPerPair : kA2Rows, pair ? 2 : 1)
                            : 1;
     if (nsplit == 1)
-        return D == 128 ? launch_attention2<128>(a, s) : launch_attention2<64>(a, s);
+        return launch(a);
     // history split across CTAs: binary32 partials in the workspace, merged by LSE
     float *o_part = static_cast<float *>(workspace);
     float *l_part = reinterpret_cast<float *>(static_cast<uint8_t *>(workspace) +
@@ -694,7 +720,7 @@ kvq_status kvq_attention_lse(const void *q, int64_t Tq, const kvq_compressed_vie
     ap.lse_out = l_part;
     ap.o_bf16 = 0;
     ap.nsplit = nsplit;
-    st = D == 128 ? launch_attention2<128>(ap, s) : launch_attention2<64>(ap, s);
+    st = launch(ap);
     if (st != KVQ_OK)
         return st;
     MergeArgs m;

@@ -330,7 +330,7 @@ __global__ void __launch_bounds__(256) fit_seed_kernel(FitArgs a)
 //   fit_bucket_update: one warp per (head, centre): sum in token order,
 //                mean in binary64, round to binary32 then bf16 (empty: keep)
 // ---------------------------------------------------------------------------
-constexpr int kFitChunk = 2048;
+constexpr int kFitChunk = 256;
 
 struct FitSortArgs {
     const void *x;
@@ -445,27 +445,48 @@ __global__ void __launch_bounds__(256) fit_bucket_update_kernel(FitSortArgs a)
 #pragma unroll
     for (int k = 0; k < kPer; ++k)
         acc[k] = 0.0;
-    for (int i = b0; i < b1; ++i) {
-        const int64_t t = ord[i];
-        const int64_t e = (t * a.H + h) * D + lane * kPer;
-        float v[kPer];
-        if (a.x_bf16) {
-            if (kPer == 4) {
-                const uint2 w = __ldg(reinterpret_cast<const uint2 *>(static_cast<const uint16_t *>(a.x) + e));
-                v[0] = bf16_lo(w.x); v[1] = bf16_hi(w.x);
-                v[2 % kPer] = bf16_lo(w.y); v[3 % kPer] = bf16_hi(w.y);
-            } else {
-                const uint32_t w = __ldg(reinterpret_cast<const uint32_t *>(static_cast<const uint16_t *>(a.x) + e));
-                v[0] = bf16_lo(w); v[1 % kPer] = bf16_hi(w);
-            }
-        } else {
+    // tokens in batches of 8: loads of a batch are issued together, the adds
+    // then run in token order
+    constexpr int kBatch = 8;
+    for (int i0 = b0; i0 < b1; i0 += kBatch) {
+        float v[kBatch][kPer];
+#pragma unroll
+        for (int b = 0; b < kBatch; ++b) {
+            const int i = i0 + b;
 #pragma unroll
             for (int k = 0; k < kPer; ++k)
-                v[k] = __ldg(static_cast<const float *>(a.x) + e + k);
+                v[b][k] = 0.0f;
+            if (i >= b1)
+                continue;
+            const int64_t t = ord[i];
+            const int64_t e = (t * a.H + h) * D + lane * kPer;
+            if (a.x_bf16) {
+                if constexpr (kPer == 4) {
+                    const uint2 w = __ldg(reinterpret_cast<const uint2 *>(static_cast<const uint16_t *>(a.x) + e));
+                    v[b][0] = bf16_lo(w.x);
+                    v[b][1] = bf16_hi(w.x);
+                    v[b][2] = bf16_lo(w.y);
+                    v[b][3] = bf16_hi(w.y);
+                } else {
+                    const uint32_t w =
+                        __ldg(reinterpret_cast<const uint32_t *>(static_cast<const uint16_t *>(a.x) + e));
+                    v[b][0] = bf16_lo(w);
+                    v[b][1] = bf16_hi(w);
+                }
+            } else {
+#pragma unroll
+                for (int k = 0; k < kPer; ++k)
+                    v[b][k] = __ldg(static_cast<const float *>(a.x) + e + k);
+            }
         }
 #pragma unroll
-        for (int k = 0; k < kPer; ++k)
-            acc[k] = __dadd_rn(acc[k], (double)v[k]);
+        for (int b = 0; b < kBatch; ++b) {
+            if (i0 + b >= b1)
+                break;
+#pragma unroll
+            for (int k = 0; k < kPer; ++k)
+                acc[k] = __dadd_rn(acc[k], (double)v[b][k]);
+        }
     }
     const double n = (double)(b1 - b0);
     uint16_t *dst = a.cent + ((int64_t)h * a.C + j) * D + lane * kPer;

@@ -371,7 +371,8 @@ def run_gpu(args):
                        "heads": w.num_heads, "head_dim": w.head_dim, "centroids": w.num_centroids,
                        "bits_k": w.bits_k, "bits_v": w.bits_v, "group": w.group_size,
                        "parallelism": f"replicas x{world}", "l2": "flushed (256 MiB write) before each step"},
-            "roofline": {"kernel": "attention_lse_kernel<128>", "bound": "tensor", "achieved": attn_tflops,
+            "roofline": {"kernel": "attention_pair_kernel (time of the whole kvq_attention_lse call, incl. its "
+                                   "in-call LSE merge)", "bound": "tensor", "achieved": attn_tflops,
                          "peak": tfl, "unit": "TFLOP/s", "frac": attn_tflops / tfl, "peak_kind": peak_kind,
                          "traffic": None},
             "rows": rows,

@@ -181,10 +181,13 @@ KVQ_API kvq_status kvq_fit_centroids_static(const kvq_codec_desc *desc, const vo
  *   idx as above per head; the residual of all H*d channels of a token is
  *   rounded to bf16 and projected, c = R W_enc (tensor-core GEMM, binary32
  *   accumulation), and the r coefficients are quantised per group of G as
- *   above (NanoKV page, Fig. 4(b)).
- * Outputs: idx [H][T], codes, meta as in the layout table.  No workspace is
- * needed by the per-head codec; the joint codec needs
- * kvq_workspace_size(KVQ_OP_ENCODE, ...) bytes.
+ *   above (NanoKV page, Fig. 4(b)).  Needs x in bf16 (KVQ_ERR_UNSUPPORTED
+ *   otherwise), r a multiple of 64 up to 256 and G in {16, 32, 64}
+ *   (KVQ_ERR_UNSUPPORTED otherwise); w_enc 16-byte aligned.  w_enc given
+ *   without joint_rank, or joint_rank without w_enc, is KVQ_ERR_INVALID_ARG.
+ * Outputs: idx [H][T], codes, meta as in the layout table.  Neither codec
+ * needs workspace (kvq_workspace_size(KVQ_OP_ENCODE, ...) reports 0; the
+ * arguments are accepted and ignored).
  */
 KVQ_API kvq_status kvq_encode(const kvq_codec_desc *desc, const void *x, kvq_dtype x_dtype, int64_t num_tokens,
                       const void *centroids, const void *w_enc, uint16_t *idx, uint8_t *codes, float *meta,
@@ -193,7 +196,9 @@ KVQ_API kvq_status kvq_encode(const kvq_codec_desc *desc, const void *x, kvq_dty
 /*
  * Joint codec only: the binary32 coefficient matrix c = R W_enc [T][r] that
  * kvq_encode quantises, and idx [H][T].  Lets a caller quantise the same
- * coefficients independently.  Workspace as for kvq_encode.
+ * coefficients independently: they are bit-identical to the ones kvq_encode
+ * quantises for the same inputs.  coef_out 16-byte aligned; requirements and
+ * workspace as for the joint kvq_encode.
  */
 KVQ_API kvq_status kvq_joint_coefficients(const kvq_codec_desc *desc, const void *x, kvq_dtype x_dtype,
                                   int64_t num_tokens, const void *centroids, const void *w_enc, uint16_t *idx,
@@ -205,9 +210,12 @@ KVQ_API kvq_status kvq_joint_coefficients(const kvq_codec_desc *desc, const void
  * the decoder reconstructs the residual and adds back the centres).
  * Per-head: x^ = mu[idx] + (q - z) * s, each step rounded to binary32
  * (subtract, multiply, add; no FMA), then stored as float or bf16 (RNE).
- * Joint: c^ = (q - z) s; R^ = c^ W_dec (tensor-core GEMM); x^ = mu[idx] + R^.
- *   x_out [T][H][d] in out_dtype.  The joint decoder needs
- *   kvq_workspace_size(KVQ_OP_DECODE, ...) bytes of workspace.
+ * Joint: c^ = (q - z) s (binary32); R^ = c^ W_dec (tensor-core GEMM: c^ is
+ *   carried as a bf16 high part plus a bf16 remainder, about 16 significant
+ *   bits, against bf16 W_dec with binary32 accumulation); x^ = mu[idx] + R^
+ *   rounded to binary32.  view->w_dec [r][H*d] bf16, 16-byte aligned.
+ *   x_out [T][H][d] in out_dtype.  No workspace is needed (the arguments are
+ *   accepted and ignored).
  */
 KVQ_API kvq_status kvq_decode(const kvq_compressed_view *view, void *x_out, kvq_dtype out_dtype, void *workspace,
                       size_t workspace_bytes, kvq_stream_t stream);

@@ -1,0 +1,358 @@
+// joint.cuh -- joint head-channel linear encoder / decoder of the residual
+// (NanoKV page, abstract and Fig. 4(a,b): joint head-channel residuals are
+// encoded into low-bit (INT4) coefficients; the decoder reconstructs them and
+// adds back the centres).
+//
+// Encoder, per 128-token tile (one CTA):
+//   R[t][i] = bf16( x[t][h][c] - mu_h[idx[h][t]][c] ),  i = h d + c
+//   Coef[t][n] = sum_i R[t][i] W_enc[i][n]    (tcgen05, M = 128, N = r, K = H d,
+//                bf16 operands, binary32 accumulation in TMEM)
+//   per row, Eq. 1 on each group of G coefficients -> packed codes, {s, z}
+// The A operand (R) is built in shared memory by the CTA's threads, 64
+// channels per K-block; W_enc [H d][r] (r contiguous) is the MN-major B
+// operand.  Two stages: the threads build K-block k+1 while the MMAs of block
+// k run.
+//
+// Decoder, per 128-token tile and 128 output channels (one head):
+//   c^[t][n] = (q - z) s                       (binary32, the quantiser's grid)
+//   R^[t][i] = sum_n c^[t][n] W_dec[n][i]      (tcgen05, c^ as bf16 hi + lo
+//                parts against bf16 W_dec, binary32 accumulation)
+//   x^[t][h][c] = mu_h[idx[h][t]][c] + R^[t][h d + c]
+#pragma once
+
+#include "codec.cuh"
+#include "common.cuh"
+
+namespace kvq {
+
+constexpr int kJRows = 128;      // tokens per CTA
+constexpr int kJThreads = 128;   // one thread per token row (TMEM lane)
+constexpr int kJKBlock = 64;     // channels per K-block
+
+struct JointEncArgs {
+    const uint16_t *x;     // [T][H][D] bf16
+    const uint16_t *cent;  // [H][C][D]
+    const uint16_t *idx;   // [H][T]
+    const uint16_t *w;     // [H*D][r] bf16
+    int64_t T;
+    int H, D, C, r, bits, G;
+    uint8_t *codes;        // [T][r*bits/8]
+    float *meta;           // [T][r/G][2]
+    float *coef_out;       // [T][r] or null
+};
+
+// shared memory: two stages of {A: 128 x 64 bf16 (16 KB), B: 64 x r bf16}
+__host__ __device__ constexpr uint32_t joint_enc_stage_bytes(int r) { return 16384u + 64u * (uint32_t)r * 2u; }
+__host__ __device__ constexpr uint32_t joint_enc_smem_bytes(int r) { return 2u * joint_enc_stage_bytes(r) + 64u; }
+
+__host__ __device__ constexpr uint32_t pow2_cols(int n)
+{
+    uint32_t c = 32;
+    while (c < (uint32_t)n)
+        c <<= 1;
+    return c;
+}
+
+// Quantise one row's r coefficients held in TMEM (columns [0, r) of this
+// thread's lane) with Eq. 1 per group of G, and store codes / {s, z}
+// (and the binary32 coefficients themselves when coef_row is set).
+template <int G, int BITS>
+__device__ __forceinline__ void joint_quant_row(uint32_t trow, int r, uint8_t *codes_row, float2 *meta_row,
+                                                float *coef_row)
+{
+    static_assert(G % 16 == 0 && G <= 64, "group of 16, 32 or 64 coefficients");
+    constexpr int kPerWord = 32 / BITS;
+    constexpr int kWords = G * BITS / 32;
+    for (int g = 0; g < r / G; ++g) {
+        float v[G];
+#pragma unroll
+        for (int c = 0; c < G; c += 16) {
+            uint32_t w16[16];
+            asm volatile(
+                "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, "
+                "[%16];"
+                : "=r"(w16[0]), "=r"(w16[1]), "=r"(w16[2]), "=r"(w16[3]), "=r"(w16[4]), "=r"(w16[5]), "=r"(w16[6]),
+                  "=r"(w16[7]), "=r"(w16[8]), "=r"(w16[9]), "=r"(w16[10]), "=r"(w16[11]), "=r"(w16[12]),
+                  "=r"(w16[13]), "=r"(w16[14]), "=r"(w16[15])
+                : "r"(trow + (uint32_t)(g * G + c)));
+            asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+            for (int k = 0; k < 16; ++k)
+                v[c + k] = __uint_as_float(w16[k]);
+        }
+        if (coef_row) {
+#pragma unroll
+            for (int c = 0; c < G; c += 4)
+                *reinterpret_cast<float4 *>(coef_row + g * G + c) = make_float4(v[c], v[c + 1], v[c + 2], v[c + 3]);
+        }
+        if (!codes_row)
+            continue;
+        float mn = v[0], mx = v[0];
+#pragma unroll
+        for (int c = 1; c < G; ++c) {
+            if (v[c] < mn) mn = v[c];
+            if (v[c] > mx) mx = v[c];
+        }
+        const GroupQ gq = group_params(mn, mx, BITS);
+        meta_row[g] = make_float2(gq.s, gq.z);
+        uint32_t *words = reinterpret_cast<uint32_t *>(codes_row) + g * kWords;
+#pragma unroll
+        for (int w = 0; w < kWords; ++w) {
+            uint32_t word = 0;
+#pragma unroll
+            for (int c = 0; c < kPerWord; ++c)
+                word |= quant_code(v[w * kPerWord + c], gq, BITS) << (c * BITS);
+            words[w] = word;
+        }
+    }
+}
+
+// One CTA per 128-token tile.  All 128 threads build the A stage (each thread
+// one token row, 64 channels) and copy the B stage; thread 0 issues the MMAs.
+template <int G, int BITS>
+__global__ void __launch_bounds__(kJThreads, 1) joint_encode_kernel(JointEncArgs a)
+{
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const uint32_t stage_bytes = joint_enc_stage_bytes(a.r);
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + 2 * stage_bytes);
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 3);
+    const int tid = threadIdx.x, warp = tid >> 5;
+    const int64_t t0 = (int64_t)blockIdx.x * kJRows;
+    const int64_t t = t0 + tid;
+    const bool valid = t < a.T;
+    const uint32_t ncols = pow2_cols(a.r);
+
+    if (warp == 0)
+        tmem_alloc(smem_u32(tmem_slot), ncols);
+    if (tid == 0) {
+        mbar_init(smem_u32(bars + 0), 1);
+        mbar_init(smem_u32(bars + 1), 1);
+        fence_mbar_init();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    const int nk = a.H * a.D / kJKBlock;
+    const uint32_t idesc = idesc_f32acc(128, a.r, true, false, true);  // bf16, B MN-major
+    uint32_t phase[2] = {0u, 0u};
+    bool ok = true;
+
+    for (int kb = 0; kb < nk; ++kb) {
+        const int s = kb & 1;
+        uint8_t *sA = smem + (uint32_t)s * stage_bytes;
+        uint8_t *sB = sA + 16384;
+        if (kb >= 2) {  // the MMAs of block kb - 2 read this stage
+            ok = mbar_wait(smem_u32(bars + s), phase[s]) && ok;
+            phase[s] ^= 1u;
+        }
+        // A: residual of channels [64 kb, 64 kb + 64) of this token, bf16
+        const int i0 = kb * kJKBlock;
+        const int h = i0 / a.D, c0 = i0 % a.D;
+        int j = 0;
+        if (valid) {
+            j = a.idx[(int64_t)h * a.T + t];
+            if (j >= a.C) {
+                raise_status(DEVSTAT_BAD_INDEX);
+                j = 0;
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < kJKBlock / 8; ++u) {
+            uint4 w = make_uint4(0, 0, 0, 0);
+            if (valid) {
+                float xv[8], mv[8];
+                load_bf16x8(a.x + (t * a.H + h) * a.D + c0 + u * 8, xv);
+                load_bf16x8(a.cent + ((int64_t)h * a.C + j) * a.D + c0 + u * 8, mv);
+                w = make_uint4(pack_bf16x2(__fsub_rn(xv[0], mv[0]), __fsub_rn(xv[1], mv[1])),
+                               pack_bf16x2(__fsub_rn(xv[2], mv[2]), __fsub_rn(xv[3], mv[3])),
+                               pack_bf16x2(__fsub_rn(xv[4], mv[4]), __fsub_rn(xv[5], mv[5])),
+                               pack_bf16x2(__fsub_rn(xv[6], mv[6]), __fsub_rn(xv[7], mv[7])));
+            }
+            *reinterpret_cast<uint4 *>(sA + sw128_unit_offset(tid, u, kJRows)) = w;
+        }
+        // B: W rows [i0, i0 + 64), all r columns -> MN-major [r/64][64][128 B]
+        for (int e = tid; e < kJKBlock * (a.r / 8); e += kJThreads) {
+            const int k = e / (a.r / 8), u = e % (a.r / 8);
+            const uint4 w = __ldg(reinterpret_cast<const uint4 *>(a.w + (int64_t)(i0 + k) * a.r) + u);
+            *reinterpret_cast<uint4 *>(sB + sw128_unit_offset(k, u, kJKBlock)) = w;
+        }
+        fence_proxy_async_smem();
+        tc_fence_before();
+        __syncthreads();
+        if (tid == 0) {
+            tc_fence_after();
+            const uint32_t aA = smem_u32(sA), aB = smem_u32(sB);
+#pragma unroll
+            for (int ks = 0; ks < kJKBlock / 16; ++ks)
+                umma_ss(tmem, sdesc_sw128(aA + (uint32_t)ks * 32u, 16, 1024),
+                        sdesc_sw128(aB + (uint32_t)ks * 2048u, kJKBlock * 128u, 1024), idesc,
+                        (kb > 0 || ks > 0) ? 1u : 0u);
+            umma_commit(smem_u32(bars + s));
+        }
+    }
+    // each stage has one commit outstanding (its last block); wait for both
+    {
+        const int s_last = (nk - 1) & 1;
+        if (nk >= 2)
+            ok = mbar_wait(smem_u32(bars + (s_last ^ 1)), phase[s_last ^ 1]) && ok;
+        ok = mbar_wait(smem_u32(bars + s_last), phase[s_last]) && ok;
+    }
+    tc_fence_after();
+    const uint32_t trow = tmem + (((uint32_t)warp * 32u) << 16);
+    ok = __all_sync(0xffffffffu, ok);  // tcgen05.ld below is warp-collective
+    if (ok) {
+        uint8_t *codes_row = (valid && a.codes) ? a.codes + t * (a.r * a.bits / 8) : nullptr;
+        float2 *meta_row = (valid && a.meta) ? reinterpret_cast<float2 *>(a.meta) + t * (a.r / G) : nullptr;
+        float *coef_row = (valid && a.coef_out) ? a.coef_out + t * a.r : nullptr;
+        joint_quant_row<G, BITS>(trow, a.r, codes_row, meta_row, coef_row);
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 0)
+        tmem_dealloc(tmem, ncols);
+}
+
+struct JointDecArgs {
+    const uint16_t *cent;  // [H][C][D]
+    const uint16_t *idx;   // [H][T]
+    const uint8_t *codes;  // [T][r*bits/8]
+    const float *meta;     // [T][r/G][2]
+    const uint16_t *w;     // [r][H*D] bf16
+    int64_t T;
+    int H, D, C, r, bits, G;
+    void *out;             // [T][H][D]
+    int out_bf16;
+};
+
+// shared memory: A hi + lo (128 x r bf16 each) and B (r x 128 bf16, MN-major)
+__host__ __device__ constexpr uint32_t joint_dec_smem_bytes(int r)
+{
+    return 3u * 128u * (uint32_t)r * 2u + 64u;
+}
+
+// One CTA per (128-token tile, head): O[128][D] = c^ W_dec[:, h D .. h D + D).
+__global__ void __launch_bounds__(kJThreads, 1) joint_decode_kernel(JointDecArgs a)
+{
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const uint32_t abytes = 128u * (uint32_t)a.r * 2u;
+    uint8_t *sAh = smem, *sAl = smem + abytes, *sB = smem + 2 * abytes;
+    uint64_t *bar = reinterpret_cast<uint64_t *>(smem + 3 * abytes);
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bar + 1);
+    const int tid = threadIdx.x, warp = tid >> 5;
+    const int64_t t0 = (int64_t)blockIdx.x * kJRows;
+    const int h = blockIdx.y;
+    const int64_t t = t0 + tid;
+    const bool valid = t < a.T;
+
+    if (warp == 0)
+        tmem_alloc(smem_u32(tmem_slot), 128);
+    if (tid == 0) {
+        mbar_init(smem_u32(bar), 1);
+        fence_mbar_init();
+    }
+    // A: c^ of this token, split into bf16 hi + lo, K-major [r/64][128][128 B]
+    const int ng = a.r / a.G;
+    const uint32_t mask = (1u << a.bits) - 1u;
+    for (int u = 0; u < a.r / 8; ++u) {
+        uint4 wh = make_uint4(0, 0, 0, 0), wl = make_uint4(0, 0, 0, 0);
+        if (valid) {
+            const int c0 = u * 8;
+            const float2 sz = reinterpret_cast<const float2 *>(a.meta)[t * ng + c0 / a.G];
+            uint32_t cw;
+            if (a.bits == 4)
+                cw = *reinterpret_cast<const uint32_t *>(a.codes + t * (a.r / 2) + c0 / 2);
+            else
+                cw = *reinterpret_cast<const uint16_t *>(a.codes + t * (a.r / 4) + c0 / 4);
+            uint32_t hi[4], lo[4];
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                const float v0 = __fmul_rn(__fsub_rn((float)((cw >> (2 * k * a.bits)) & mask), sz.y), sz.x);
+                const float v1 = __fmul_rn(__fsub_rn((float)((cw >> ((2 * k + 1) * a.bits)) & mask), sz.y), sz.x);
+                const uint32_t a0 = __float_as_uint(v0) & 0xffff0000u, a1 = __float_as_uint(v1) & 0xffff0000u;
+                hi[k] = __byte_perm(a0, a1, 0x7632);
+                lo[k] = pack_bf16x2(v0 - __uint_as_float(a0), v1 - __uint_as_float(a1));
+            }
+            wh = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+            wl = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+        }
+        const uint32_t off = sw128_unit_offset(tid, u, kJRows);
+        *reinterpret_cast<uint4 *>(sAh + off) = wh;
+        *reinterpret_cast<uint4 *>(sAl + off) = wl;
+    }
+    // B: W_dec rows n (K), columns [h D, h D + D) (N) -> MN-major [D/64][r][128 B]
+    const int HD = a.H * a.D;
+    for (int e = tid; e < a.r * (a.D / 8); e += kJThreads) {
+        const int n = e / (a.D / 8), u = e % (a.D / 8);
+        const uint4 w = __ldg(reinterpret_cast<const uint4 *>(a.w + (int64_t)n * HD + (int64_t)h * a.D) + u);
+        *reinterpret_cast<uint4 *>(sB + sw128_unit_offset(n, u, a.r)) = w;
+    }
+    fence_proxy_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    bool ok = true;
+    if (tid == 0) {
+        const uint32_t idesc = idesc_f32acc(128, a.D, true, false, true);
+        const uint32_t aAh = smem_u32(sAh), aAl = smem_u32(sAl), aB = smem_u32(sB);
+        const int nks = a.r / 16;
+        for (int part = 0; part < 2; ++part)
+            for (int ks = 0; ks < nks; ++ks) {
+                const uint32_t aoff = (uint32_t)(ks >> 2) * (128u * 128u) + (uint32_t)(ks & 3) * 32u;
+                umma_ss(tmem, sdesc_sw128((part ? aAl : aAh) + aoff, 16, 1024),
+                        sdesc_sw128(aB + (uint32_t)ks * 2048u, (uint32_t)a.r * 128u, 1024), idesc,
+                        (part || ks) ? 1u : 0u);
+            }
+        umma_commit(smem_u32(bar));
+    }
+    ok = mbar_wait(smem_u32(bar), 0);
+    tc_fence_after();
+    const uint32_t trow = tmem + (((uint32_t)warp * 32u) << 16);
+    int j = 0;
+    if (valid) {
+        j = a.idx[(int64_t)h * a.T + t];
+        if (j >= a.C) {
+            raise_status(DEVSTAT_BAD_INDEX);
+            j = 0;
+        }
+    }
+    for (int cb = 0; cb < a.D / 32; ++cb) {
+        float v[32];
+        tmem_ld32(trow + (uint32_t)(cb * 32), v);
+        if (!valid || !ok)
+            continue;
+        const uint16_t *mu = a.cent + ((int64_t)h * a.C + j) * a.D + cb * 32;
+        float m8[8];
+        const int64_t o = (t * a.H + h) * a.D + cb * 32;
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            load_bf16x8(mu + u * 8, m8);
+#pragma unroll
+            for (int k = 0; k < 8; ++k)
+                v[u * 8 + k] = __fadd_rn(m8[k], v[u * 8 + k]);
+        }
+        if (a.out_bf16) {
+            uint4 *dst = reinterpret_cast<uint4 *>(static_cast<uint16_t *>(a.out) + o);
+#pragma unroll
+            for (int u = 0; u < 4; ++u)
+                dst[u] = make_uint4(pack_bf16x2(v[8 * u], v[8 * u + 1]), pack_bf16x2(v[8 * u + 2], v[8 * u + 3]),
+                                    pack_bf16x2(v[8 * u + 4], v[8 * u + 5]), pack_bf16x2(v[8 * u + 6], v[8 * u + 7]));
+        } else {
+            float4 *dst = reinterpret_cast<float4 *>(static_cast<float *>(a.out) + o);
+#pragma unroll
+            for (int u = 0; u < 8; ++u)
+                dst[u] = make_float4(v[4 * u], v[4 * u + 1], v[4 * u + 2], v[4 * u + 3]);
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 0)
+        tmem_dealloc(tmem, 128);
+}
+
+}  // namespace kvq

@@ -15,6 +15,7 @@
 #include "codec.cuh"
 #include "common.cuh"
 #include "encode_filter.cuh"
+#include "joint.cuh"
 #include "merge.cuh"
 
 using namespace kvq;
@@ -47,7 +48,10 @@ kvq_status check_desc(const kvq_codec_desc *d, bool allow_joint)
     const int span = d->joint_rank > 0 ? d->joint_rank : d->head_dim;
     if (d->group_size < 8 || d->group_size % 8 != 0 || span % d->group_size != 0)
         return KVQ_ERR_INVALID_ARG;
-    if (d->joint_rank == 0 && d->group_size != 16 && d->group_size != 32 && d->group_size != 64)
+    if (d->group_size != 16 && d->group_size != 32 && d->group_size != 64)
+        return KVQ_ERR_UNSUPPORTED;
+    // joint code: rank a multiple of 64 up to 256 (one MMA N extent)
+    if (d->joint_rank > 0 && (d->joint_rank % 64 != 0 || d->joint_rank > 256))
         return KVQ_ERR_UNSUPPORTED;
     return KVQ_OK;
 }
@@ -226,6 +230,111 @@ kvq_status launch_encode(int D, const EncodeArgs &e, cudaStream_t s)
     return launch_encode_direct(D, e, s);
 }
 
+// ---------------------------------------------------------------------------
+// joint head-channel code
+// ---------------------------------------------------------------------------
+template <int G, int BITS>
+kvq_status launch_joint_encode_t(const JointEncArgs &a, cudaStream_t s)
+{
+    const uint32_t smem = joint_enc_smem_bytes(a.r) + 1024;
+    static bool configured[64] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64)
+        return KVQ_ERR_CUDA;
+    if (!configured[dev]) {
+        if (cudaFuncSetAttribute(joint_encode_kernel<G, BITS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)(joint_enc_smem_bytes(256) + 1024)) != cudaSuccess)
+            return KVQ_ERR_CUDA;
+        configured[dev] = true;
+    }
+    joint_encode_kernel<G, BITS><<<(unsigned)ceil_div(a.T, kJRows), kJThreads, smem, s>>>(a);
+    return launch_status();
+}
+
+kvq_status launch_joint_encode(const JointEncArgs &a, cudaStream_t s)
+{
+    if (a.T == 0)
+        return KVQ_OK;
+    switch (a.G * 8 + a.bits) {
+    case 16 * 8 + 2: return launch_joint_encode_t<16, 2>(a, s);
+    case 16 * 8 + 4: return launch_joint_encode_t<16, 4>(a, s);
+    case 32 * 8 + 2: return launch_joint_encode_t<32, 2>(a, s);
+    case 32 * 8 + 4: return launch_joint_encode_t<32, 4>(a, s);
+    case 64 * 8 + 2: return launch_joint_encode_t<64, 2>(a, s);
+    case 64 * 8 + 4: return launch_joint_encode_t<64, 4>(a, s);
+    default: return KVQ_ERR_UNSUPPORTED;
+    }
+}
+
+kvq_status launch_joint_decode(const JointDecArgs &a, cudaStream_t s)
+{
+    if (a.T == 0)
+        return KVQ_OK;
+    static bool configured[64] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64)
+        return KVQ_ERR_CUDA;
+    if (!configured[dev]) {
+        if (cudaFuncSetAttribute(joint_decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)(joint_dec_smem_bytes(256) + 1024)) != cudaSuccess)
+            return KVQ_ERR_CUDA;
+        configured[dev] = true;
+    }
+    const dim3 grid((unsigned)ceil_div(a.T, kJRows), (unsigned)a.H);
+    joint_decode_kernel<<<grid, kJThreads, joint_dec_smem_bytes(a.r) + 1024, s>>>(a);
+    return launch_status();
+}
+
+// Validates and runs the joint encoder: per-head assignment into idx, then the
+// projection + quantisation (codes/meta) and/or the binary32 coefficients.
+kvq_status joint_encode_call(const kvq_codec_desc *desc, const void *x, kvq_dtype x_dtype, int64_t T,
+                             const void *centroids, const void *w_enc, uint16_t *idx, uint8_t *codes, float *meta,
+                             float *coef_out, cudaStream_t s)
+{
+    if (x_dtype != KVQ_BF16)
+        return KVQ_ERR_UNSUPPORTED;  // the joint residual is formed from a bf16 history
+    if (T < 0)
+        return KVQ_ERR_INVALID_ARG;
+    if (T == 0)
+        return KVQ_OK;
+    if (!x || !centroids || !w_enc || !idx || (!coef_out && (!codes || !meta)))
+        return KVQ_ERR_INVALID_ARG;
+    if (!aligned16(x) || !aligned16(centroids) || !aligned16(w_enc) || (codes && !aligned16(codes)) ||
+        (meta && !aligned16(meta)) || (coef_out && !aligned16(coef_out)) || (reinterpret_cast<uintptr_t>(idx) & 1u))
+        return KVQ_ERR_ALIGNMENT;
+    EncodeArgs e;
+    memset(&e, 0, sizeof e);
+    e.x = x;
+    e.x_bf16 = 1;
+    e.T = T;
+    e.H = desc->num_heads;
+    e.C = desc->num_centroids;
+    e.bits = 2;
+    e.G = 16;
+    e.cent = static_cast<const uint16_t *>(centroids);
+    e.idx = idx;
+    e.assign_only = 1;
+    kvq_status st = launch_encode(desc->head_dim, e, s);
+    if (st != KVQ_OK)
+        return st;
+    JointEncArgs a;
+    a.x = static_cast<const uint16_t *>(x);
+    a.cent = e.cent;
+    a.idx = idx;
+    a.w = static_cast<const uint16_t *>(w_enc);
+    a.T = T;
+    a.H = desc->num_heads;
+    a.D = desc->head_dim;
+    a.C = desc->num_centroids;
+    a.r = desc->joint_rank;
+    a.bits = desc->bits;
+    a.G = desc->group_size;
+    a.codes = codes;
+    a.meta = meta;
+    a.coef_out = coef_out;
+    return launch_joint_encode(a, s);
+}
+
 // Fit workspace: idx [H][T] u16 | per-chunk centre counts [H][nch][C] i32 |
 // bucket starts [H][C+1] i32 | token order [H][T] i32.
 struct FitLayout {
@@ -365,26 +474,6 @@ kvq_status launch_attention2(const AttnArgs &a, cudaStream_t s)
     return launch_status();
 }
 
-template <int D>
-kvq_status launch_attention(const AttnArgs &a, cudaStream_t s)
-{
-    using L = AttnSmem<D>;
-    // the dynamic shared-memory opt-in is a per-device function attribute
-    static bool configured[64] = {};
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64)
-        return KVQ_ERR_CUDA;
-    if (!configured[dev]) {
-        if (cudaFuncSetAttribute(attention_lse_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)L::kLaunchBytes) != cudaSuccess)
-            return KVQ_ERR_CUDA;
-        configured[dev] = true;
-    }
-    const dim3 grid((unsigned)ceil_div(a.Tq, kAttnRows), (unsigned)a.H);
-    attention_lse_kernel<D><<<grid, kAttnThreads, L::kLaunchBytes, s>>>(a);
-    return launch_status();
-}
-
 }  // namespace
 
 extern "C" {
@@ -439,9 +528,7 @@ kvq_status kvq_workspace_size(kvq_op op, const kvq_codec_desc *desc, int64_t T, 
     switch (op) {
     case KVQ_OP_FIT: *bytes = fit_workspace(desc, T); return KVQ_OK;
     case KVQ_OP_ENCODE:
-    case KVQ_OP_DECODE:
-        *bytes = 0;
-        return desc->joint_rank > 0 ? KVQ_ERR_UNSUPPORTED : KVQ_OK;
+    case KVQ_OP_DECODE: *bytes = 0; return KVQ_OK;
     case KVQ_OP_ATTENTION: *bytes = attention_workspace(desc, Tq); return KVQ_OK;
     }
     return KVQ_ERR_INVALID_ARG;
@@ -587,8 +674,14 @@ kvq_status kvq_encode(const kvq_codec_desc *desc, const void *x, kvq_dtype x_dty
     kvq_status st = check_desc(desc, true);
     if (st != KVQ_OK)
         return st;
-    if (desc->joint_rank > 0 || w_enc)
-        return KVQ_ERR_UNSUPPORTED;
+    if (desc->joint_rank > 0 || w_enc) {
+        if (desc->joint_rank == 0 || !w_enc)
+            return KVQ_ERR_INVALID_ARG;  // w_enc is given exactly for the joint code
+        if (x_dtype != KVQ_F32 && x_dtype != KVQ_BF16)
+            return KVQ_ERR_INVALID_ARG;
+        return joint_encode_call(desc, x, x_dtype, T, centroids, w_enc, idx, codes, meta, nullptr,
+                                 reinterpret_cast<cudaStream_t>(stream));
+    }
     if (T < 0 || (x_dtype != KVQ_F32 && x_dtype != KVQ_BF16))
         return KVQ_ERR_INVALID_ARG;
     if (T == 0)
@@ -618,9 +711,19 @@ kvq_status kvq_joint_coefficients(const kvq_codec_desc *desc, const void *x, kvq
                                   const void *centroids, const void *w_enc, uint16_t *idx, float *coef_out,
                                   void *workspace, size_t workspace_bytes, kvq_stream_t stream)
 {
-    (void)desc; (void)x; (void)x_dtype; (void)T; (void)centroids; (void)w_enc; (void)idx; (void)coef_out;
-    (void)workspace; (void)workspace_bytes; (void)stream;
-    return KVQ_ERR_UNSUPPORTED;
+    (void)workspace;
+    (void)workspace_bytes;
+    kvq_status st = check_desc(desc, true);
+    if (st != KVQ_OK)
+        return st;
+    if (desc->joint_rank == 0 || !w_enc)
+        return KVQ_ERR_INVALID_ARG;
+    if (x_dtype != KVQ_F32 && x_dtype != KVQ_BF16)
+        return KVQ_ERR_INVALID_ARG;
+    if (T > 0 && !coef_out)
+        return KVQ_ERR_INVALID_ARG;
+    return joint_encode_call(desc, x, x_dtype, T, centroids, w_enc, idx, nullptr, nullptr, coef_out,
+                             reinterpret_cast<cudaStream_t>(stream));
 }
 
 kvq_status kvq_decode(const kvq_compressed_view *view, void *x_out, kvq_dtype out_dtype, void *workspace,
@@ -631,8 +734,6 @@ kvq_status kvq_decode(const kvq_compressed_view *view, void *x_out, kvq_dtype ou
     kvq_status st = check_view(view);
     if (st != KVQ_OK)
         return st;
-    if (view->desc.joint_rank > 0)
-        return KVQ_ERR_UNSUPPORTED;
     if (out_dtype != KVQ_F32 && out_dtype != KVQ_BF16)
         return KVQ_ERR_INVALID_ARG;
     if (view->num_tokens == 0)
@@ -641,6 +742,28 @@ kvq_status kvq_decode(const kvq_compressed_view *view, void *x_out, kvq_dtype ou
         return KVQ_ERR_INVALID_ARG;
     if (!aligned16(x_out))
         return KVQ_ERR_ALIGNMENT;
+    if (view->desc.joint_rank > 0) {
+        if (!view->w_dec)
+            return KVQ_ERR_INVALID_ARG;
+        if (!aligned16(view->w_dec))
+            return KVQ_ERR_ALIGNMENT;
+        JointDecArgs j;
+        j.cent = static_cast<const uint16_t *>(view->centroids);
+        j.idx = view->idx;
+        j.codes = view->codes;
+        j.meta = view->meta;
+        j.w = static_cast<const uint16_t *>(view->w_dec);
+        j.T = view->num_tokens;
+        j.H = view->desc.num_heads;
+        j.D = view->desc.head_dim;
+        j.C = view->desc.num_centroids;
+        j.r = view->desc.joint_rank;
+        j.bits = view->desc.bits;
+        j.G = view->desc.group_size;
+        j.out = x_out;
+        j.out_bf16 = out_dtype == KVQ_BF16;
+        return launch_joint_decode(j, reinterpret_cast<cudaStream_t>(stream));
+    }
     DecodeArgs a;
     a.cent = static_cast<const uint16_t *>(view->centroids);
     a.idx = view->idx;

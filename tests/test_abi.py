@@ -111,7 +111,24 @@ def test_bad_pointers_and_sizes_rejected_on_host(K):
     arr_null = (ctypes.c_void_p * 2)(A, None)
     assert _err(K, "kvq_lse_merge", 2, arr_null, arr, 10, 2, 128, A, K.KVQ_F32, A, None) == K.KVQ_ERR_INVALID_ARG
     assert _err(K, "kvq_lse_merge", 2, arr, arr, 10, 2, 96, A, K.KVQ_F32, A, None) == K.KVQ_ERR_UNSUPPORTED
-    # decode: joint view not served yet by the per-head decoder arguments
-    vj = K.CompressedView(K.CodecDesc(12, 128, 256, 4, 32, 192), 10, A, A, A, A, A)
-    assert _err(K, "kvq_decode", ctypes.byref(vj), A, K.KVQ_F32, None, 0, None) in (K.KVQ_ERR_UNSUPPORTED,
-                                                                                     K.KVQ_ERR_WORKSPACE)
+    # joint codec: decoder matrix missing or misaligned, unsupported rank,
+    # encoder matrix without a rank (and the reverse), f32 input
+    dj = K.CodecDesc(12, 128, 256, 4, 32, 192)
+    vj = K.CompressedView(dj, 10, A, A, A, A, None)
+    assert _err(K, "kvq_decode", ctypes.byref(vj), A, K.KVQ_F32, None, 0, None) == K.KVQ_ERR_INVALID_ARG
+    vj = K.CompressedView(dj, 10, A, A, A, A, A + 8)
+    assert _err(K, "kvq_decode", ctypes.byref(vj), A, K.KVQ_F32, None, 0, None) == K.KVQ_ERR_ALIGNMENT
+    d96 = K.CodecDesc(12, 128, 256, 4, 32, 96)
+    assert _err(K, "kvq_encoded_sizes", ctypes.byref(d96), 10, ctypes.byref(ctypes.c_size_t()), None, None) \
+        == K.KVQ_ERR_UNSUPPORTED
+    assert _err(K, "kvq_encode", ctypes.byref(d), A, K.KVQ_BF16, 100, A, A, A, A, A, None, 0, None) \
+        == K.KVQ_ERR_INVALID_ARG
+    assert _err(K, "kvq_encode", ctypes.byref(dj), A, K.KVQ_BF16, 100, A, None, A, A, A, None, 0, None) \
+        == K.KVQ_ERR_INVALID_ARG
+    assert _err(K, "kvq_encode", ctypes.byref(dj), A, K.KVQ_F32, 100, A, A, A, A, A, None, 0, None) \
+        == K.KVQ_ERR_UNSUPPORTED
+    assert _err(K, "kvq_joint_coefficients", ctypes.byref(dj), A, K.KVQ_BF16, 100, A, A, A, None, None, 0, None) \
+        == K.KVQ_ERR_INVALID_ARG
+    assert _err(K, "kvq_joint_coefficients", ctypes.byref(dj), A, K.KVQ_BF16, 100, A, A, A, A + 4, None, 0, None) \
+        == K.KVQ_ERR_ALIGNMENT
+    assert K.workspace_size(K.KVQ_OP_ENCODE, K.Codec(12, 128, 256, 4, 32, 192), 32760) == 0

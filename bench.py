@@ -6,6 +6,8 @@ One step = one pass of every step of the path over the Wan-1.3B-like layer
 4,680 tokens, 256 centroids per head, K INT2 / V INT2, group 16):
 
   fit centroids (K, V; 2 k-means rounds) -> encode (K, V) -> decode (K, V)
+  -> joint head-channel code of the same history (K, V: rank 192, INT4,
+     group 32, orthonormal W_enc): encode, then decode
   -> attention of the chunk over the compressed history in 2 blocks
   -> LSE merge of the 2 partial results.
 
@@ -42,6 +44,13 @@ UNIT = "history-tokens/s"
 WORKLOAD = "wan13b"
 HISTORY_BLOCKS = 2
 FLUSH_BYTES = 256 << 20
+
+
+def _joint():
+    """The joint head-channel workload (same history shape as WORKLOAD)."""
+    from kv_cache_compression_head_b200 import synth
+
+    return synth.workload("joint")
 
 
 def parse_args():
@@ -173,8 +182,17 @@ def work_model(w):
     # fit, per k-means round and token-head: the assignment reads x and writes
     # its index, the accumulation reads x and the index (K and V)
     fit_bytes = 2 * w.kmeans_iters * th * (2 * d + 2 + 2 * d + 2)
+    # joint code, K and V: the assignment pass reads x and writes idx; the
+    # projection pass reads x and idx and writes r*b/8 code bytes and r/G
+    # {s, z} pairs per token; the decoder reads those and writes bf16 x^
+    wj = _joint()
+    jstored = wj.joint_rank * wj.bits_k // 8 + 8 * (wj.joint_rank // wj.joint_group)
+    joint_enc_bytes = 2 * T * (2 * (2 * H * d + 2 * H) + jstored)
+    joint_dec_bytes = 2 * T * (2 * H + jstored + 2 * H * d)
+    joint_flops = 2 * T * 2.0 * H * d * wj.joint_rank  # one GEMM per direction, K and V
     return {"encode_bytes": enc_bytes, "decode_bytes": dec_bytes, "attention_flops": attn_flops,
-            "merge_bytes": merge_bytes, "fit_bytes": fit_bytes}
+            "merge_bytes": merge_bytes, "fit_bytes": fit_bytes, "joint_enc_bytes": joint_enc_bytes,
+            "joint_dec_bytes": joint_dec_bytes, "joint_gemm_flops": joint_flops}
 
 
 # ----------------------------------------------------------------------------
@@ -184,7 +202,7 @@ def work_model(w):
 class Pipeline:
     """Device buffers and the per-step call sequence through the public API."""
 
-    ROWS = ("fit", "encode", "decode", "attention", "merge")
+    ROWS = ("fit", "encode", "decode", "joint_encode", "joint_decode", "attention", "merge")
 
     def __init__(self, w, device):
         import torch
@@ -213,12 +231,27 @@ class Pipeline:
         self.edges = [T * i // HISTORY_BLOCKS for i in range(HISTORY_BLOCKS + 1)]
         self.comp = [K.Compressed(c, T, self.cent[i], *self.enc[i])
                      for i, c in enumerate((self.codec_k, self.codec_v))]
-        self.launches_per_step = (2 * (1 + 3 * w.kmeans_iters) + 2 + 2 + HISTORY_BLOCKS + 1)
+        # joint head-channel code of the same history (same centres)
+        from kv_cache_compression_head_b200 import synth
+
+        wj = _joint()
+        self.codec_j = [K.Codec(H, d, w.num_centroids, b, wj.joint_group, wj.joint_rank)
+                        for b in (wj.bits_k, wj.bits_v)]
+        w_enc = synth.make_orthonormal_encoder(wj)
+        self.w_enc = torch.from_numpy(w_enc.view(np.int16)).view(bf).to(device)
+        self.w_dec = self.w_enc.t().contiguous()
+        self.enc_j = [K.alloc_encoded(c, T, device) for c in self.codec_j]
+        self.comp_j = [K.Compressed(c, T, self.cent[i], *self.enc_j[i], w_dec=self.w_dec)
+                       for i, c in enumerate(self.codec_j)]
+        # fit: seed + (assign + 4 sort/update kernels) per round; encode 1;
+        # decode 1; joint encode 2 (assign, projection), joint decode 1;
+        # attention 2 per block (split + its merge); final merge 1 -- K and V
+        self.launches_per_step = (2 * (1 + 5 * w.kmeans_iters) + 2 + 2 + 2 * 2 + 2 + 2 * HISTORY_BLOCKS + 1)
 
     def outputs(self):
         outs = [self.o, self.lse]
         for i in range(2):
-            outs += [self.cent[i], *self.enc[i]]
+            outs += [self.cent[i], *self.enc[i], *self.enc_j[i]]
         return outs
 
     def step(self, ev=None):
@@ -241,6 +274,14 @@ class Pipeline:
         K.kvq_decode(self.comp[0], self.dec[0])
         K.kvq_decode(self.comp[1], self.dec[1])
         mark("decode", 1)
+        mark("joint_encode", 0)
+        K.kvq_encode(self.codec_j[0], self.xk, self.cent[0], *self.enc_j[0], w_enc=self.w_enc)
+        K.kvq_encode(self.codec_j[1], self.xv, self.cent[1], *self.enc_j[1], w_enc=self.w_enc)
+        mark("joint_encode", 1)
+        mark("joint_decode", 0)
+        K.kvq_decode(self.comp_j[0], self.dec[0])
+        K.kvq_decode(self.comp_j[1], self.dec[1])
+        mark("joint_decode", 1)
         mark("attention", 0)
         for b in range(HISTORY_BLOCKS):
             K.kvq_attention_lse(self.q, self.comp[0], self.comp[1], self.o_parts[b], self.l_parts[b],
@@ -343,11 +384,19 @@ def run_gpu(args):
         dec_gbps = wm["decode_bytes"] / (row_mean["decode"] / 1e3) / 1e9
         merge_gbps = wm["merge_bytes"] / (row_mean["merge"] / 1e3) / 1e9
         fit_gbps = wm["fit_bytes"] / (row_mean["fit"] / 1e3) / 1e9
+        jenc_gbps = wm["joint_enc_bytes"] / (row_mean["joint_encode"] / 1e3) / 1e9
+        jdec_gbps = wm["joint_dec_bytes"] / (row_mean["joint_decode"] / 1e3) / 1e9
+        jdec_tflops = wm["joint_gemm_flops"] / 2 / (row_mean["joint_decode"] / 1e3) / 1e12
+        jenc_tflops = wm["joint_gemm_flops"] / 2 / (row_mean["joint_encode"] / 1e3) / 1e12
         rows = {
             "fit": {"ms": row_mean["fit"], "gbps": fit_gbps, "hbm_frac": fit_gbps / hbm},
             "encode": {"ms": row_mean["encode"], "tokens_per_s": w.history_tokens / (row_mean["encode"] / 1e3),
                        "gbps": enc_gbps, "hbm_frac": enc_gbps / hbm},
             "decode": {"ms": row_mean["decode"], "gbps": dec_gbps, "hbm_frac": dec_gbps / hbm},
+            "joint_encode": {"ms": row_mean["joint_encode"], "gbps": jenc_gbps, "hbm_frac": jenc_gbps / hbm,
+                             "gemm_tflops": jenc_tflops},
+            "joint_decode": {"ms": row_mean["joint_decode"], "gbps": jdec_gbps, "hbm_frac": jdec_gbps / hbm,
+                             "gemm_tflops": jdec_tflops},
             "attention": {"ms": row_mean["attention"], "launches": HISTORY_BLOCKS, "tflops": attn_tflops,
                           "frac": attn_tflops / tfl},
             "merge": {"ms": row_mean["merge"], "gbps": merge_gbps, "hbm_frac": merge_gbps / hbm},
@@ -366,7 +415,8 @@ def run_gpu(args):
             "dtype": "bf16",
             "data": "synthetic (seeded AR(1) frames + heavy-tailed outlier channels)",
             "config": {"workload": "wan13b-like layer: 12 heads x 128, history 32760 tokens (21 frames x 1560), "
-                                   "query chunk 4680, C=256, K2V2, group 16, fit 2 rounds, 2 history blocks",
+                                   "query chunk 4680, C=256, K2V2, group 16, fit 2 rounds, 2 history blocks; "
+                                   "joint code of the same history: rank 192, K4V4, group 32",
                        "history_tokens": w.history_tokens, "query_tokens": w.query_tokens,
                        "heads": w.num_heads, "head_dim": w.head_dim, "centroids": w.num_centroids,
                        "bits_k": w.bits_k, "bits_v": w.bits_v, "group": w.group_size,

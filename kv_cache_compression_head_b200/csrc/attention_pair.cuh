@@ -20,15 +20,28 @@
 // online softmax for query tile 0 / 1 (one thread per row = TMEM lane, lazy
 // rescaling of O in TMEM, P written back over S as fp16 pairs).
 //
-// Barriers (parity = use count & 1).  Counted on the leader, arrived on from
-// both CTAs (release.cluster): qready (512), kfull[s], vfull[s] (512 each:
-// the producers of both CTAs), pfull[i] (256: the softmax threads of both
-// CTAs).  Signalled by multicast tcgen05.commit into both CTAs: sfull[i]
-// (S_i ready), kfree[s] (QK of the tile in K stage s done), vfree[s] (P V of
-// the tile in V stage s done), ofull (last P V done).  No waiter can fall two
-// phases behind: every barrier's next completion needs an action of the
-// waiting role.  Waits are bounded and poll a per-CTA abort flag; before TMEM
-// is freed the leader drains its MMAs and both CTAs meet at a cluster barrier.
+// MMA issue order (the two query tiles run half a tile apart, so that the
+// softmax of one overlaps the tensor-core work of the other):
+//   S(0,0) S(0,1) | P V(0,0) S(1,0) P V(0,1) S(1,1) | P V(1,0) S(2,0) ...
+// where S(j,i) = Q_i K_j^T (hi and lo) and P V(j,i) needs the softmax of
+// S(j,i).  tcgen05 MMAs of one issuer run in order, so S(j+1,i) overwrites
+// P(j,i) in TMEM only after P V(j,i) has read it.
+//
+// Producers: each thread rebuilds 4 units (32 channels) of one K row and of
+// one V row per tile.  The global loads of the next item (its centre row,
+// codes and {s, z}) are issued before the current item is rebuilt, and the
+// centre index two items ahead, so the gather latency overlaps arithmetic.
+//
+// Barriers (parity = use count & 1).  Counted on the leader, arrived on once
+// per warp from both CTAs (release.cluster, after each lane's proxy fence and
+// a warp barrier): qready, kfull[s], vfull[s] (16 each: the producer warps of
+// both CTAs), pfull[i] (8: the softmax warps of both CTAs).  Signalled by
+// multicast tcgen05.commit into both CTAs: sfull[i] (S_i ready), kfree[s] (QK
+// of the tile in K stage s done), vfree[s] (P V of the tile in V stage s
+// done), ofull (last P V done).  No waiter can fall two phases behind: every
+// barrier's next completion needs an action of the waiting role.  Waits are
+// bounded and poll a per-CTA abort flag; before TMEM is freed the leader
+// drains its MMAs and both CTAs meet at a cluster barrier.
 #pragma once
 
 #include "attention.cuh"
@@ -142,66 +155,85 @@ __device__ __forceinline__ void umma2_commit_both(uint32_t bar)
         : "memory");
 }
 
-// Rebuild 8-channel units [u0, u0 + n) of history row `tok` (K: bf16 hi + lo
-// split; V: fp16) into `tile` at swizzled row `row` of a tile with `rows`
-// rows.  Unit u of the row lands at unit (u - ubase) of the tile row.
-template <int BITS, bool SPLIT, int NU>
-__device__ __forceinline__ void ap_dequant_units(const CodecView &cv, int h, int64_t tok, bool valid, int u0,
-                                                 int ubase, uint8_t *tile, uint8_t *tile_lo, uint32_t row,
-                                                 uint32_t rows)
+// One thread's share of one history row: 4 units (8 channels each) of the
+// centre row, their code words and their groups' {s, z}.
+struct APRow {
+    uint4 mu[4];
+    uint32_t cw[4];
+    float2 sz[4];
+};
+
+// Centre index of history row `tok` (0 for rows past the range).
+__device__ __forceinline__ int ap_index(const CodecView &cv, int h, int64_t tok, bool valid)
+{
+    return valid ? (int)__ldg(cv.idx + (int64_t)h * cv.T + tok) : 0;
+}
+
+// Issue the loads of units [u0, u0 + 4) of row `tok` (centre j).
+template <int BITS>
+__device__ __forceinline__ void ap_load(const CodecView &cv, int h, int64_t tok, bool valid, int j, int u0,
+                                        APRow &r)
 {
     constexpr int D = 128;
-    if (!valid) {
-#pragma unroll
-        for (int uu = 0; uu < NU; ++uu) {
-            const uint32_t off = sw128_unit_offset(row, u0 + uu - ubase, rows);
-            *reinterpret_cast<uint4 *>(tile + off) = make_uint4(0, 0, 0, 0);
-            if (SPLIT)
-                *reinterpret_cast<uint4 *>(tile_lo + off) = make_uint4(0, 0, 0, 0);
-        }
+    if (!valid)
         return;
-    }
-    const int64_t th = (int64_t)h * cv.T + tok;
-    int j = __ldg(cv.idx + th);
     if (j >= cv.C) {
         raise_status(DEVSTAT_BAD_INDEX);
         j = 0;
     }
+    const int64_t th = (int64_t)h * cv.T + tok;
     const uint4 *mu_row = reinterpret_cast<const uint4 *>(cv.cent + ((int64_t)h * cv.C + j) * D) + u0;
-    uint4 mw[NU];
 #pragma unroll
-    for (int uu = 0; uu < NU; ++uu)
-        mw[uu] = __ldg(mu_row + uu);
-    uint32_t cws[NU];
+    for (int uu = 0; uu < 4; ++uu)
+        r.mu[uu] = __ldg(mu_row + uu);
     if (BITS == 2) {
         const uint16_t *cr = reinterpret_cast<const uint16_t *>(cv.codes + th * (D / 4)) + u0;
 #pragma unroll
-        for (int uu = 0; uu < NU; ++uu)
-            cws[uu] = __ldg(cr + uu);
+        for (int uu = 0; uu < 4; ++uu)
+            r.cw[uu] = __ldg(cr + uu);
     } else {
         const uint32_t *cr = reinterpret_cast<const uint32_t *>(cv.codes + th * (D / 2)) + u0;
 #pragma unroll
-        for (int uu = 0; uu < NU; ++uu)
-            cws[uu] = __ldg(cr + uu);
+        for (int uu = 0; uu < 4; ++uu)
+            r.cw[uu] = __ldg(cr + uu);
     }
     const float2 *meta_row = reinterpret_cast<const float2 *>(cv.meta) + th * (D / cv.G);
+#pragma unroll
+    for (int uu = 0; uu < 4; ++uu)
+        r.sz[uu] = __ldg(meta_row + (u0 + uu) * 8 / cv.G);
+}
+
+// Rebuild the loaded units into `tile` at swizzled row `row` of a tile with
+// `rows` rows (unit u0 + uu lands at unit u0 + uu - ubase):
+//   x^ = fma(f, 2^b s, mu - (2^b + z) s),  f = 1 + q 2^-b
+// which is the decoder's mu + (q - z) s up to one rounding.  K (SPLIT): bf16
+// hi (truncated) + lo (the rounded remainder) tiles; V: one fp16 tile.
+template <int BITS, bool SPLIT>
+__device__ __forceinline__ void ap_store(const APRow &r, bool valid, int u0, int ubase, uint8_t *tile,
+                                         uint8_t *tile_lo, uint32_t row, uint32_t rows)
+{
     constexpr float kTwoB = (float)(1 << BITS);
 #pragma unroll
-    for (int uu = 0; uu < NU; ++uu) {
-        const int c0 = (u0 + uu) * 8;
-        const float2 sz = __ldg(meta_row + c0 / cv.G);
+    for (int uu = 0; uu < 4; ++uu) {
+        const uint32_t off = sw128_unit_offset(row, u0 + uu - ubase, rows);
+        if (!valid) {
+            *reinterpret_cast<uint4 *>(tile + off) = make_uint4(0, 0, 0, 0);
+            if (SPLIT)
+                *reinterpret_cast<uint4 *>(tile_lo + off) = make_uint4(0, 0, 0, 0);
+            continue;
+        }
+        const float2 sz = r.sz[uu];
         const float sc = kTwoB * sz.x;
         const float nb = -__fmul_rn(kTwoB + sz.y, sz.x);
-        const uint32_t ma[4] = {mw[uu].x, mw[uu].y, mw[uu].z, mw[uu].w};
+        const uint32_t ma[4] = {r.mu[uu].x, r.mu[uu].y, r.mu[uu].z, r.mu[uu].w};
         float2 val[4];
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
-            const float2 f = make_float2(code_as_unit_float<BITS>(cws[uu], 2 * k),
-                                         code_as_unit_float<BITS>(cws[uu], 2 * k + 1));
+            const float2 f = make_float2(code_as_unit_float<BITS>(r.cw[uu], 2 * k),
+                                         code_as_unit_float<BITS>(r.cw[uu], 2 * k + 1));
             const float2 b = add2(make_float2(bf16_lo(ma[k]), bf16_hi(ma[k])), make_float2(nb, nb));
             val[k] = fma2(f, make_float2(sc, sc), b);
         }
-        const uint32_t off = sw128_unit_offset(row, u0 + uu - ubase, rows);
         if (SPLIT) {
             uint32_t hi[4], lo[4];
 #pragma unroll
@@ -209,8 +241,8 @@ __device__ __forceinline__ void ap_dequant_units(const CodecView &cv, int h, int
                 const uint32_t a0 = __float_as_uint(val[k].x) & 0xffff0000u;
                 const uint32_t a1 = __float_as_uint(val[k].y) & 0xffff0000u;
                 hi[k] = __byte_perm(a0, a1, 0x7632);
-                const float2 r = sub2(val[k], make_float2(__uint_as_float(a0), __uint_as_float(a1)));
-                lo[k] = pack_bf16x2(r.x, r.y);
+                const float2 d = sub2(val[k], make_float2(__uint_as_float(a0), __uint_as_float(a1)));
+                lo[k] = pack_bf16x2(d.x, d.y);
             }
             *reinterpret_cast<uint4 *>(tile + off) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
             *reinterpret_cast<uint4 *>(tile_lo + off) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
@@ -219,6 +251,63 @@ __device__ __forceinline__ void ap_dequant_units(const CodecView &cv, int h, int
                 make_uint4(pack_f16x2_sat(val[0].x, val[0].y), pack_f16x2_sat(val[1].x, val[1].y),
                            pack_f16x2_sat(val[2].x, val[2].y), pack_f16x2_sat(val[3].x, val[3].y));
         }
+    }
+}
+
+// Make the warp's generic-proxy writes visible to the tensor core, then one
+// lane arrives on the leader's barrier (cluster address).
+__device__ __forceinline__ void ap_publish(uint32_t lead_bar)
+{
+    fence_proxy_async_smem();
+    __syncwarp();
+    if ((threadIdx.x & 31) == 0)
+        mbar_arrive_cluster(lead_bar);
+}
+
+// Producer loop: items K(0), V(0), K(1), V(1), ...; K(i) and V(i) reuse the
+// stage of tile i - 2 once its MMAs are done.
+template <int BK, int BV>
+__device__ __forceinline__ void ap_produce(const AttnArgs &a, int h, uint32_t rank, int tid, int ntiles,
+                                           uint8_t *smem, uint64_t *bars, volatile int *abort_flag)
+{
+    using L = APSmem;
+    auto bar = [&](int i) { return smem_u32(bars + i); };
+    auto lead = [&](int i) { return mapa_shared(bar(i), 0); };
+    // K: history rows [64 rank, 64 rank + 64) of the tile; thread -> (row
+    // tid & 63, channel quarter tid >> 6: units 4q .. 4q + 3)
+    const uint32_t krow = (uint32_t)(tid & 63);
+    const int ku0 = 4 * (tid >> 6);
+    // V: channels [64 rank, 64 rank + 64); thread -> (row tid & 127, units
+    // 8 rank + 4 (tid >> 7) .. + 3)
+    const uint32_t vrow = (uint32_t)(tid & 127);
+    const int vu0 = 8 * (int)rank + 4 * (tid >> 7);
+    auto ktok = [&](int i) { return a.t_begin + (int64_t)i * 128 + 64 * rank + krow; };
+    auto vtok = [&](int i) { return a.t_begin + (int64_t)i * 128 + vrow; };
+
+    APRow rk, rv;
+    int jk = ap_index(a.k, h, ktok(0), ktok(0) < a.t_end);
+    int jv = ap_index(a.v, h, vtok(0), vtok(0) < a.t_end);
+    ap_load<BK>(a.k, h, ktok(0), ktok(0) < a.t_end, jk, ku0, rk);
+    jk = (ntiles > 1) ? ap_index(a.k, h, ktok(1), ktok(1) < a.t_end) : 0;
+    for (int i = 0; i < ntiles; ++i) {
+        const int s = i & 1;
+        const uint32_t par = (uint32_t)(((i - 2) >> 1) & 1);
+        ap_load<BV>(a.v, h, vtok(i), vtok(i) < a.t_end, jv, vu0, rv);
+        jv = (i + 1 < ntiles) ? ap_index(a.v, h, vtok(i + 1), vtok(i + 1) < a.t_end) : 0;
+        if (i >= 2 && !__all_sync(0xffffffffu, ap_wait(bar(s ? P_KFREE1 : P_KFREE0), par, abort_flag)))
+            return;
+        ap_store<BK, true>(rk, ktok(i) < a.t_end, ku0, 0, smem + L::offK + (uint32_t)(2 * s) * L::kKh,
+                           smem + L::offK + (uint32_t)(2 * s + 1) * L::kKh, krow, 64);
+        ap_publish(lead(s ? P_KFULL1 : P_KFULL0));
+        if (i + 1 < ntiles) {
+            ap_load<BK>(a.k, h, ktok(i + 1), ktok(i + 1) < a.t_end, jk, ku0, rk);
+            jk = (i + 2 < ntiles) ? ap_index(a.k, h, ktok(i + 2), ktok(i + 2) < a.t_end) : 0;
+        }
+        if (i >= 2 && !__all_sync(0xffffffffu, ap_wait(bar(s ? P_VFREE1 : P_VFREE0), par, abort_flag)))
+            return;
+        ap_store<BV, false>(rv, vtok(i) < a.t_end, vu0, 8 * (int)rank, smem + L::offV + (uint32_t)s * L::kV,
+                            nullptr, vrow, 128);
+        ap_publish(lead(s ? P_VFULL1 : P_VFULL0));
     }
 }
 
@@ -260,15 +349,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAPThreads, 1) atten
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
     }
     if (tid == 0) {
-        mbar_init(bar(P_QREADY), 2 * kAPProducers);
-        mbar_init(bar(P_KFULL0), 2 * kAPProducers);
-        mbar_init(bar(P_KFULL1), 2 * kAPProducers);
-        mbar_init(bar(P_VFULL0), 2 * kAPProducers);
-        mbar_init(bar(P_VFULL1), 2 * kAPProducers);
+        constexpr uint32_t kProdWarps = 2 * kAPProducers / 32;  // both CTAs
+        mbar_init(bar(P_QREADY), kProdWarps);
+        mbar_init(bar(P_KFULL0), kProdWarps);
+        mbar_init(bar(P_KFULL1), kProdWarps);
+        mbar_init(bar(P_VFULL0), kProdWarps);
+        mbar_init(bar(P_VFULL1), kProdWarps);
         mbar_init(bar(P_SFULL0), 1);
         mbar_init(bar(P_SFULL1), 1);
-        mbar_init(bar(P_PFULL0), 256);
-        mbar_init(bar(P_PFULL1), 256);
+        mbar_init(bar(P_PFULL0), 8);  // 4 softmax warps per CTA and query tile
+        mbar_init(bar(P_PFULL1), 8);
         mbar_init(bar(P_KFREE0), 1);
         mbar_init(bar(P_KFREE1), 1);
         mbar_init(bar(P_VFREE0), 1);
@@ -299,55 +389,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAPThreads, 1) atten
                 *reinterpret_cast<uint4 *>(dst + sw128_unit_offset(r, u, 128)) = w;
             }
         }
-        fence_proxy_async_smem();
-        mbar_arrive_cluster(lead(P_QREADY));
-        // K half: history rows [64 rank, 64 rank + 64) of the tile; thread ->
-        // (row p & 63, channel quarter p >> 6: units 4q .. 4q+3)
-        const uint32_t krow = (uint32_t)(tid & 63);
-        const int kq = tid >> 6;
-        // V half: channels [64 rank, 64 rank + 64); thread -> (row p & 127,
-        // units 8 rank + 4 hh .. + 3, hh = p >> 7)
-        const uint32_t vrow = (uint32_t)(tid & 127);
-        const int vu0 = 8 * (int)rank + 4 * (tid >> 7);
-        auto make_k = [&](int jt, int s) {
-            const int64_t tok = a.t_begin + (int64_t)jt * 128 + 64 * rank + krow;
-            if (a.k.bits == 2)
-                ap_dequant_units<2, true, 4>(a.k, h, tok, tok < a.t_end, 4 * kq, 0, ksl(s, 0), ksl(s, 1), krow, 64);
-            else
-                ap_dequant_units<4, true, 4>(a.k, h, tok, tok < a.t_end, 4 * kq, 0, ksl(s, 0), ksl(s, 1), krow, 64);
-            fence_proxy_async_smem();
-            mbar_arrive_cluster(lead(s ? P_KFULL1 : P_KFULL0));
-        };
-        auto make_v = [&](int jt, int s) {
-            const int64_t tok = a.t_begin + (int64_t)jt * 128 + vrow;
-            if (a.v.bits == 2)
-                ap_dequant_units<2, false, 4>(a.v, h, tok, tok < a.t_end, vu0, 8 * (int)rank, vsl(s), nullptr, vrow,
-                                              128);
-            else
-                ap_dequant_units<4, false, 4>(a.v, h, tok, tok < a.t_end, vu0, 8 * (int)rank, vsl(s), nullptr, vrow,
-                                              128);
-            fence_proxy_async_smem();
-            mbar_arrive_cluster(lead(s ? P_VFULL1 : P_VFULL0));
-        };
+        ap_publish(lead(P_QREADY));
         if (ntiles > 0) {
-            make_k(0, 0);
-            make_v(0, 0);
-            if (ntiles > 1)
-                make_k(1, 1);
-            for (int j = 0; j < ntiles; ++j) {
-                if (j + 1 < ntiles) {
-                    const int s = (j + 1) & 1;
-                    if (j >= 1 && !ap_wait(bar(s ? P_VFREE1 : P_VFREE0), (uint32_t)(((j - 1) >> 1) & 1), abort_flag))
-                        break;
-                    make_v(j + 1, s);
-                }
-                if (j + 2 < ntiles) {
-                    const int s = j & 1;
-                    if (!ap_wait(bar(s ? P_KFREE1 : P_KFREE0), (uint32_t)((j >> 1) & 1), abort_flag))
-                        break;
-                    make_k(j + 2, s);
-                }
-            }
+            if (a.k.bits == 2 && a.v.bits == 2)
+                ap_produce<2, 2>(a, h, rank, tid, ntiles, smem, bars, abort_flag);
+            else if (a.k.bits == 2)
+                ap_produce<2, 4>(a, h, rank, tid, ntiles, smem, bars, abort_flag);
+            else if (a.v.bits == 2)
+                ap_produce<4, 2>(a, h, rank, tid, ntiles, smem, bars, abort_flag);
+            else
+                ap_produce<4, 4>(a, h, rank, tid, ntiles, smem, bars, abort_flag);
         }
     } else if (warp == kAPProducers / 32) {
         // ------------------------------------------------------------ MMA issuer (leader)
@@ -356,30 +407,32 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAPThreads, 1) atten
             constexpr uint32_t idescO = idesc_f32acc(256, D, false, false, true);
             const uint32_t aQ[2] = {smem_u32(smem + L::offQ), smem_u32(smem + L::offQ + L::kQ)};
             const uint32_t tS[2] = {tmem, tmem + 128}, tO[2] = {tmem + 256, tmem + 384};
-            bool ok = ap_wait(bar(P_QREADY), 0, abort_flag);
-            for (int j = 0; ok && j < ntiles; ++j) {
-                const int s = j & 1;
-                ok = ap_wait(bar(s ? P_KFULL1 : P_KFULL0), (uint32_t)((j >> 1) & 1), abort_flag);
-                if (!ok)
-                    break;
-                tc_fence_after();
-                const uint32_t aK[2] = {smem_u32(ksl(s, 0)), smem_u32(ksl(s, 1))};
+            // S(j, qt) = Q_qt (K_j hi + K_j lo)^T into tS[qt]
+            auto issue_s = [&](int j, int qt) {
+                const int ks_ = j & 1;
+                const uint32_t aK[2] = {smem_u32(ksl(ks_, 0)), smem_u32(ksl(ks_, 1))};
 #pragma unroll
                 for (int part = 0; part < 2; ++part) {
 #pragma unroll
-                    for (int qt = 0; qt < 2; ++qt) {
-#pragma unroll
-                        for (int ks = 0; ks < D / 16; ++ks) {
-                            const uint32_t offa = (uint32_t)(ks >> 2) * (128u * 128u) + (uint32_t)(ks & 3) * 32u;
-                            const uint32_t offb = (uint32_t)(ks >> 2) * (64u * 128u) + (uint32_t)(ks & 3) * 32u;
-                            umma2_ss(tS[qt], sdesc_sw128(aQ[qt] + offa, 16, 1024),
-                                     sdesc_sw128(aK[part] + offb, 16, 1024), idescS, (part | ks) ? 1u : 0u);
-                        }
-                        if (part == 1)
-                            umma2_commit_both(bar(qt ? P_SFULL1 : P_SFULL0));
+                    for (int ks = 0; ks < D / 16; ++ks) {
+                        const uint32_t offa = (uint32_t)(ks >> 2) * (128u * 128u) + (uint32_t)(ks & 3) * 32u;
+                        const uint32_t offb = (uint32_t)(ks >> 2) * (64u * 128u) + (uint32_t)(ks & 3) * 32u;
+                        umma2_ss(tS[qt], sdesc_sw128(aQ[qt] + offa, 16, 1024), sdesc_sw128(aK[part] + offb, 16, 1024),
+                                 idescS, (part | ks) ? 1u : 0u);
                     }
                 }
-                umma2_commit_both(bar(s ? P_KFREE1 : P_KFREE0));
+                umma2_commit_both(bar(qt ? P_SFULL1 : P_SFULL0));
+                if (qt == 1)
+                    umma2_commit_both(bar(ks_ ? P_KFREE1 : P_KFREE0));
+            };
+            bool ok = ap_wait(bar(P_QREADY), 0, abort_flag) && ap_wait(bar(P_KFULL0), 0, abort_flag);
+            if (ok) {
+                tc_fence_after();
+                issue_s(0, 0);
+                issue_s(0, 1);
+            }
+            for (int j = 0; ok && j < ntiles; ++j) {
+                const int s = j & 1;
                 ok = ap_wait(bar(s ? P_VFULL1 : P_VFULL0), (uint32_t)((j >> 1) & 1), abort_flag);
                 const uint32_t aV = smem_u32(vsl(s));
                 for (int qt = 0; ok && qt < 2; ++qt) {
@@ -391,10 +444,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAPThreads, 1) atten
                     for (int ks = 0; ks < 128 / 16; ++ks)
                         umma2_ts(tO[qt], tS[qt] + (uint32_t)ks * 8u, sdesc_sw128(aV + (uint32_t)ks * 2048u, 16384, 1024),
                                  idescO, (j > 0 || ks > 0) ? 1u : 0u);
+                    if (qt == 1)
+                        umma2_commit_both(bar(s ? P_VFREE1 : P_VFREE0));
+                    if (j + 1 < ntiles) {
+                        if (qt == 0) {
+                            const int s1 = (j + 1) & 1;
+                            ok = ap_wait(bar(s1 ? P_KFULL1 : P_KFULL0), (uint32_t)(((j + 1) >> 1) & 1), abort_flag);
+                            if (!ok)
+                                break;
+                            tc_fence_after();
+                        }
+                        issue_s(j + 1, qt);
+                    }
                 }
-                if (!ok)
-                    break;
-                umma2_commit_both(bar(s ? P_VFREE1 : P_VFREE0));
             }
             // success: signals the epilogues; failure: drains every MMA issued
             umma2_commit_both(bar(P_OFULL));
@@ -471,7 +533,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAPThreads, 1) atten
             asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
             l += lt;
             tc_fence_before();
-            mbar_arrive_cluster(pfull);
+            __syncwarp();
+            if (lane == 0)
+                mbar_arrive_cluster(pfull);
         }
         const int64_t qr = q0 + grp * 128 + r;
         const bool have =

@@ -78,11 +78,6 @@ __device__ __forceinline__ bool a2_wait(uint32_t bar, uint32_t parity, volatile 
     return false;
 }
 
-__device__ __forceinline__ void mbar_arrive(uint32_t bar)
-{
-    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
-}
-
 // f = 1 + q 2^-b for the code of channel k (0..7) of a unit: the code bits are
 // moved into the top of the mantissa of 1.0f.
 template <int BITS>

@@ -20,6 +20,7 @@
 #pragma once
 
 #include <float.h>
+#include <limits.h>
 
 #include "common.cuh"
 
@@ -301,8 +302,57 @@ struct FitArgs {
     uint16_t *cent;  // [H][C][D]
 };
 
-// mu_j = bf16(x_j) for the first C tokens.
-__global__ void __launch_bounds__(256) fit_seed_kernel(FitArgs a)
+// ---------------------------------------------------------------------------
+// Deterministic centre update.  The specification sums every centre's tokens
+// sequentially in token order in binary64.  That sum is exact -- and then
+// equal to the sum in any order -- whenever every value is a multiple of 2^L
+// and every partial sum stays below 2^(53 + L) in magnitude: all partial sums
+// are then integers times 2^L representable in 53 bits.  So:
+//   fit_hist:    per (head, token chunk) centre counts            [H][C][nch]
+//   fit_scan:    per head, bucket starts and per-chunk bases       [H][C+1], [H][C][nch]
+//   fit_scatter: per (head, chunk), stable placement of token ids  order[H][T]
+//   fit_segsum:  one warp per 64 consecutive slots of the sorted order: per
+//                run of one centre, binary64 sums per channel, a bound Q on
+//                every channel's sum of |x| and the smallest exponent L of
+//                any value's last significand bit; added to the centre's
+//                totals with atomics (exact sums are order independent)
+//   fit_finalize: one warp per (head, centre): if Q <= 2^(52 + L) the sums
+//                are exact: mean in binary64, binary32, then bf16 (empty:
+//                keep); otherwise the centre is marked for
+//   fit_bucket_update: the sequential token-order sum (marked centres only).
+// ---------------------------------------------------------------------------
+constexpr int kFitChunk = 256;
+constexpr int kFitSegSlots = 64;
+
+struct FitSortArgs {
+    const void *x;
+    int x_bf16;
+    int64_t T;
+    int H;
+    int D;
+    int C;
+    int nchunks;
+    uint16_t *cent;          // [H][C][D]
+    const uint16_t *idx;     // [H][T]
+    int *chunk_counts;       // [H][C][nchunks] (counts, then bases)
+    int *bucket_start;       // [H][C + 1]
+    int *order;              // [H][T]
+    double *sums;            // [H][C][D]
+    double *qsum;            // [H][C]
+    int *lmin;               // [H][C]
+    int *redo;               // [H][C]
+};
+
+// Exponent of the last significand bit of a nonzero binary32 value.
+__device__ __forceinline__ int lsb_exponent(float v)
+{
+    const uint32_t b = __float_as_uint(v);
+    const uint32_t e = (b >> 23) & 0xffu, m = b & 0x7fffffu;
+    return e == 0u ? -149 + (__ffs((int)m) - 1) : (int)e - 150 + (__ffs((int)(m | 0x800000u)) - 1);
+}
+
+// mu_j = bf16(x_j) for the first C tokens; the update totals start cleared.
+__global__ void __launch_bounds__(256) fit_seed_kernel(FitArgs a, FitSortArgs fs)
 {
     const int64_t gid = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
     const int64_t total = (int64_t)a.H * a.C * a.D;
@@ -317,35 +367,13 @@ __global__ void __launch_bounds__(256) fit_seed_kernel(FitArgs a)
                        : static_cast<const float *>(a.x)[e];
     const __nv_bfloat16 b = __float2bfloat16_rn(v);
     a.cent[gid] = *reinterpret_cast<const uint16_t *>(&b);
+    fs.sums[gid] = 0.0;
+    if (c == 0) {
+        fs.qsum[hj] = 0.0;
+        fs.lmin[hj] = INT_MAX;
+        fs.redo[hj] = 0;
+    }
 }
-
-// ---------------------------------------------------------------------------
-// Deterministic centre update by bucket sort: every centre's tokens are
-// gathered in token order and summed sequentially in binary64, exactly as the
-// specification's sequential sum does, so the new centres do not depend on
-// thread timing.
-//   fit_hist:    per (head, token chunk) centre counts            [H][nch][C]
-//   fit_scan:    per head, bucket starts and per-chunk bases       [H][C], [H][nch][C]
-//   fit_scatter: per (head, chunk), stable placement of token ids  order[H][T]
-//   fit_bucket_update: one warp per (head, centre): sum in token order,
-//                mean in binary64, round to binary32 then bf16 (empty: keep)
-// ---------------------------------------------------------------------------
-constexpr int kFitChunk = 256;
-
-struct FitSortArgs {
-    const void *x;
-    int x_bf16;
-    int64_t T;
-    int H;
-    int D;
-    int C;
-    int nchunks;
-    uint16_t *cent;          // [H][C][D]
-    const uint16_t *idx;     // [H][T]
-    int *chunk_counts;       // [H][nchunks][C] (counts, then bases)
-    int *bucket_start;       // [H][C + 1]
-    int *order;              // [H][T]
-};
 
 __global__ void __launch_bounds__(256) fit_hist_kernel(FitSortArgs a)
 {
@@ -359,38 +387,78 @@ __global__ void __launch_bounds__(256) fit_hist_kernel(FitSortArgs a)
     for (int64_t t = t0 + threadIdx.x; t < t1; t += blockDim.x)
         atomicAdd(&s_cnt[a.idx[(int64_t)h * a.T + t]], 1);
     __syncthreads();
-    int *dst = a.chunk_counts + ((int64_t)h * a.nchunks + ch) * a.C;
+    int *dst = a.chunk_counts + (int64_t)h * a.C * a.nchunks + ch;
     for (int j = threadIdx.x; j < a.C; j += blockDim.x)
-        dst[j] = s_cnt[j];
+        dst[(int64_t)j * a.nchunks] = s_cnt[j];
 }
 
-// One block per head.  Bucket totals -> exclusive prefix over centres (bucket
-// starts); then each chunk's count is replaced by the chunk's base inside the
-// centre's bucket (prefix over chunks).
+// One block (1024 threads) per head.  Each warp turns the chunk counts of its
+// centres into chunk bases (prefix over chunks); then a block-wide exclusive
+// prefix over the centre totals gives the bucket starts.
 __global__ void __launch_bounds__(1024) fit_scan_kernel(FitSortArgs a)
 {
     extern __shared__ int s_tot[];  // [C]
-    const int h = blockIdx.x;
-    int *cc = a.chunk_counts + (int64_t)h * a.nchunks * a.C;
-    for (int j = threadIdx.x; j < a.C; j += blockDim.x) {
+    __shared__ int s_warp[32];
+    const int h = blockIdx.x, lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    int *cc = a.chunk_counts + (int64_t)h * a.C * a.nchunks;
+    for (int j = warp; j < a.C; j += 32) {
+        int *row = cc + (int64_t)j * a.nchunks;
         int run = 0;
-        for (int ch = 0; ch < a.nchunks; ++ch) {
-            const int c = cc[(int64_t)ch * a.C + j];
-            cc[(int64_t)ch * a.C + j] = run;
-            run += c;
+        for (int c0 = 0; c0 < a.nchunks; c0 += 32) {
+            const int c = c0 + lane;
+            const int v = c < a.nchunks ? row[c] : 0;
+            int incl = v;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int n = __shfl_up_sync(0xffffffffu, incl, o);
+                if (lane >= o)
+                    incl += n;
+            }
+            if (c < a.nchunks)
+                row[c] = run + incl - v;
+            run += __shfl_sync(0xffffffffu, incl, 31);
         }
-        s_tot[j] = run;
+        if (lane == 0)
+            s_tot[j] = run;
     }
     __syncthreads();
-    if (threadIdx.x == 0) {
-        int run = 0;
-        int *bs = a.bucket_start + (int64_t)h * (a.C + 1);
-        for (int j = 0; j < a.C; ++j) {
-            bs[j] = run;
-            run += s_tot[j];
-        }
-        bs[a.C] = run;
+    // exclusive prefix of s_tot: thread k owns entries [k per, (k + 1) per)
+    const int per = (a.C + 1023) / 1024;
+    const int j0 = threadIdx.x * per, j1 = min(a.C, j0 + per);
+    int local = 0;
+    for (int j = j0; j < j1; ++j)
+        local += s_tot[j];
+    int incl = local;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int n = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o)
+            incl += n;
     }
+    if (lane == 31)
+        s_warp[warp] = incl;
+    __syncthreads();
+    if (warp == 0) {
+        const int v = s_warp[lane];
+        int wi = v;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int n = __shfl_up_sync(0xffffffffu, wi, o);
+            if (lane >= o)
+                wi += n;
+        }
+        s_warp[lane] = wi - v;
+    }
+    __syncthreads();
+    int run = s_warp[warp] + incl - local;
+    int *bs = a.bucket_start + (int64_t)h * (a.C + 1);
+    for (int j = j0; j < j1; ++j) {
+        const int t = s_tot[j];
+        bs[j] = run;
+        run += t;
+    }
+    if (threadIdx.x == 1023)
+        bs[a.C] = run;
 }
 
 // One warp per (head, chunk): tokens in order, 32 at a time; lanes holding the
@@ -400,10 +468,10 @@ __global__ void __launch_bounds__(32) fit_scatter_kernel(FitSortArgs a)
 {
     extern __shared__ int s_cur[];  // [C] running offset of each centre in this chunk
     const int h = blockIdx.y, ch = blockIdx.x, lane = threadIdx.x;
-    const int *base = a.chunk_counts + ((int64_t)h * a.nchunks + ch) * a.C;
+    const int *base = a.chunk_counts + (int64_t)h * a.C * a.nchunks + ch;
     const int *bs = a.bucket_start + (int64_t)h * (a.C + 1);
     for (int j = lane; j < a.C; j += 32)
-        s_cur[j] = bs[j] + base[j];
+        s_cur[j] = bs[j] + base[(int64_t)j * a.nchunks];
     __syncwarp();
     const int64_t t0 = (int64_t)ch * kFitChunk;
     const int64_t t1 = min(a.T, t0 + kFitChunk);
@@ -426,8 +494,156 @@ __global__ void __launch_bounds__(32) fit_scatter_kernel(FitSortArgs a)
     }
 }
 
-// One warp per (head, centre); lane l owns channels 4l .. 4l+3 (D = 128) or
-// 2l .. 2l+1 (D = 64).  Sums in binary64 in token order.
+// Lane l owns channels kPer l .. kPer l + kPer - 1 of token t.
+template <int D>
+__device__ __forceinline__ void fit_load_row(const FitSortArgs &a, int h, int64_t t, int lane, float *v)
+{
+    constexpr int kPer = D / 32;
+    const int64_t e = (t * a.H + h) * D + lane * kPer;
+    if (a.x_bf16) {
+        if constexpr (kPer == 4) {
+            const uint2 w = __ldg(reinterpret_cast<const uint2 *>(static_cast<const uint16_t *>(a.x) + e));
+            v[0] = bf16_lo(w.x);
+            v[1] = bf16_hi(w.x);
+            v[2] = bf16_lo(w.y);
+            v[3] = bf16_hi(w.y);
+        } else {
+            const uint32_t w = __ldg(reinterpret_cast<const uint32_t *>(static_cast<const uint16_t *>(a.x) + e));
+            v[0] = bf16_lo(w);
+            v[1] = bf16_hi(w);
+        }
+    } else {
+#pragma unroll
+        for (int k = 0; k < kPer; ++k)
+            v[k] = __ldg(static_cast<const float *>(a.x) + e + k);
+    }
+}
+
+template <int D>
+__global__ void __launch_bounds__(256) fit_segsum_kernel(FitSortArgs a)
+{
+    constexpr int kPer = D / 32;
+    const int lane = threadIdx.x & 31;
+    const int64_t segs = (a.T + kFitSegSlots - 1) / kFitSegSlots;
+    const int64_t gw = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    if (gw >= segs * a.H)
+        return;
+    const int h = (int)(gw / segs);
+    const int64_t i0 = (gw % segs) * kFitSegSlots;
+    const int64_t i1 = min(a.T, i0 + kFitSegSlots);
+    const int *ord = a.order + (int64_t)h * a.T;
+    const uint16_t *idx = a.idx + (int64_t)h * a.T;
+
+    double acc[kPer], q = 0.0;
+    int lm = INT_MAX, cur = -1;
+#pragma unroll
+    for (int k = 0; k < kPer; ++k)
+        acc[k] = 0.0;
+    auto flush = [&]() {
+        double* dst = a.sums + ((int64_t)h * a.C + cur) * D + lane * kPer;
+#pragma unroll
+        for (int k = 0; k < kPer; ++k)
+            atomicAdd(dst + k, acc[k]);
+        // Q: every channel's sum of |x| is at most its lane's q, so at most
+        // the largest q; L: the smallest last-bit exponent
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            q = fmax(q, __shfl_xor_sync(0xffffffffu, q, o));
+            lm = min(lm, __shfl_xor_sync(0xffffffffu, lm, o));
+        }
+        if (lane == 0) {
+            atomicAdd(a.qsum + (int64_t)h * a.C + cur, q);
+            atomicMin(a.lmin + (int64_t)h * a.C + cur, lm);
+        }
+#pragma unroll
+        for (int k = 0; k < kPer; ++k)
+            acc[k] = 0.0;
+        q = 0.0;
+        lm = INT_MAX;
+    };
+    for (int64_t ib = i0; ib < i1; ib += 32) {
+        const int nb = (int)min((int64_t)32, i1 - ib);
+        int t_l = 0, j_l = -1;
+        if (lane < nb) {
+            t_l = ord[ib + lane];
+            j_l = idx[t_l];
+        }
+        for (int b0 = 0; b0 < nb; b0 += 8) {
+            float v[8][kPer];
+            int jj[8];
+#pragma unroll
+            for (int b = 0; b < 8; ++b) {
+                const int t = __shfl_sync(0xffffffffu, t_l, (b0 + b) & 31);
+                jj[b] = __shfl_sync(0xffffffffu, j_l, (b0 + b) & 31);
+                if (b0 + b < nb)
+                    fit_load_row<D>(a, h, t, lane, v[b]);
+                else
+                    jj[b] = -1;
+            }
+#pragma unroll
+            for (int b = 0; b < 8; ++b) {
+                if (jj[b] < 0)
+                    break;
+                if (jj[b] != cur) {
+                    if (cur >= 0)
+                        flush();
+                    cur = jj[b];
+                }
+                float mx = 0.0f;
+#pragma unroll
+                for (int k = 0; k < kPer; ++k) {
+                    const float x = v[b][k];
+                    acc[k] = __dadd_rn(acc[k], (double)x);
+                    mx = fmaxf(mx, fabsf(x));
+                    if (x != 0.0f)
+                        lm = min(lm, lsb_exponent(x));
+                }
+                q = __dadd_ru(q, (double)mx);
+            }
+        }
+    }
+    if (cur >= 0)
+        flush();
+}
+
+// One warp per (head, centre): exact totals -> new centre; otherwise mark the
+// centre for the sequential pass.  Clears the totals for the next round.
+template <int D>
+__global__ void __launch_bounds__(256) fit_finalize_kernel(FitSortArgs a)
+{
+    constexpr int kPer = D / 32;
+    const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
+    if (warp >= a.H * a.C)
+        return;
+    const int h = warp / a.C, j = warp % a.C;
+    const int64_t hj = (int64_t)h * a.C + j;
+    const int *bs = a.bucket_start + (int64_t)h * (a.C + 1);
+    const int n = bs[j + 1] - bs[j];
+    const double q = a.qsum[hj];
+    const int L = a.lmin[hj];
+    // every partial sum is a multiple of 2^L below 2^(53 + L) in magnitude
+    const bool exact = L == INT_MAX || q <= ldexp(1.0, 52 + L);
+    double *sum = a.sums + hj * D + lane * kPer;
+    if (n > 0 && exact) {
+        uint16_t *dst = a.cent + hj * D + lane * kPer;
+#pragma unroll
+        for (int k = 0; k < kPer; ++k) {
+            const __nv_bfloat16 b = __float2bfloat16_rn(__double2float_rn(__ddiv_rn(sum[k], (double)n)));
+            dst[k] = *reinterpret_cast<const uint16_t *>(&b);
+        }
+    }
+#pragma unroll
+    for (int k = 0; k < kPer; ++k)
+        sum[k] = 0.0;
+    if (lane == 0) {
+        a.redo[hj] = (n > 0 && !exact) ? 1 : 0;
+        a.qsum[hj] = 0.0;
+        a.lmin[hj] = INT_MAX;
+    }
+}
+
+// One warp per (head, centre) marked by fit_finalize; lane l owns channels
+// kPer l .. kPer l + kPer - 1.  Sums in binary64 in token order.
 template <int D>
 __global__ void __launch_bounds__(256) fit_bucket_update_kernel(FitSortArgs a)
 {
@@ -436,6 +652,8 @@ __global__ void __launch_bounds__(256) fit_bucket_update_kernel(FitSortArgs a)
     if (warp >= a.H * a.C)
         return;
     const int h = warp / a.C, j = warp % a.C;
+    if (!a.redo[(int64_t)h * a.C + j])
+        return;
     const int *bs = a.bucket_start + (int64_t)h * (a.C + 1);
     const int b0 = bs[j], b1 = bs[j + 1];
     if (b1 == b0)
@@ -456,28 +674,8 @@ __global__ void __launch_bounds__(256) fit_bucket_update_kernel(FitSortArgs a)
 #pragma unroll
             for (int k = 0; k < kPer; ++k)
                 v[b][k] = 0.0f;
-            if (i >= b1)
-                continue;
-            const int64_t t = ord[i];
-            const int64_t e = (t * a.H + h) * D + lane * kPer;
-            if (a.x_bf16) {
-                if constexpr (kPer == 4) {
-                    const uint2 w = __ldg(reinterpret_cast<const uint2 *>(static_cast<const uint16_t *>(a.x) + e));
-                    v[b][0] = bf16_lo(w.x);
-                    v[b][1] = bf16_hi(w.x);
-                    v[b][2] = bf16_lo(w.y);
-                    v[b][3] = bf16_hi(w.y);
-                } else {
-                    const uint32_t w =
-                        __ldg(reinterpret_cast<const uint32_t *>(static_cast<const uint16_t *>(a.x) + e));
-                    v[b][0] = bf16_lo(w);
-                    v[b][1] = bf16_hi(w);
-                }
-            } else {
-#pragma unroll
-                for (int k = 0; k < kPer; ++k)
-                    v[b][k] = __ldg(static_cast<const float *>(a.x) + e + k);
-            }
+            if (i < b1)
+                fit_load_row<D>(a, h, ord[i], lane, v[b]);
         }
 #pragma unroll
         for (int b = 0; b < kBatch; ++b) {

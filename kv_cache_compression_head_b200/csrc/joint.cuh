@@ -220,139 +220,231 @@ struct JointDecArgs {
     const uint16_t *idx;   // [H][T]
     const uint8_t *codes;  // [T][r*bits/8]
     const float *meta;     // [T][r/G][2]
-    const uint16_t *w;     // [r][H*D] bf16
     int64_t T;
     int H, D, C, r, bits, G;
     void *out;             // [T][H][D]
     int out_bf16;
 };
 
-// shared memory: A hi + lo (128 x r bf16 each) and B (r x 128 bf16, MN-major)
-__host__ __device__ constexpr uint32_t joint_dec_smem_bytes(int r)
-{
-    return 3u * 128u * (uint32_t)r * 2u + 64u;
-}
+// Decoder roles (288 threads): warps 0-3 and 4-7 are two epilogue groups
+// (even and odd heads; each thread one token row = TMEM lane), warp 8 lane 0
+// loads W_dec slices with TMA and issues the MMAs.  All 256 epilogue threads
+// first build c^ (two threads per token, half the coefficients each).
+constexpr int kJDThreads = 288;
 
-// One CTA per (128-token tile, head): O[128][D] = c^ W_dec[:, h D .. h D + D).
-__global__ void __launch_bounds__(kJThreads, 1) joint_decode_kernel(JointDecArgs a)
+constexpr uint32_t kJDSmemLimit = 227u * 1024u - 1024u;  // less the alignment slack
+
+struct JDLayout {
+    uint32_t a_bytes;  // one of A hi / A lo: [r/64][128][128 B]
+    uint32_t w_bytes;  // one W stage: [D/64][r][128 B]
+    int nst;           // W stages: 2 where they fit, else 1
+    uint32_t off_lo, off_w, off_bar, total;
+    __host__ __device__ JDLayout(int r, int D)
+    {
+        a_bytes = 128u * (uint32_t)r * 2u;
+        w_bytes = (uint32_t)(D / 64) * (uint32_t)r * 128u;
+        nst = (2u * a_bytes + 2u * w_bytes + 128u <= kJDSmemLimit) ? 2 : 1;
+        off_lo = a_bytes;
+        off_w = 2u * a_bytes;
+        off_bar = off_w + (uint32_t)nst * w_bytes;
+        total = off_bar + 128u;
+    }
+};
+
+enum { JD_WFULL0 = 0, JD_WFULL1, JD_DONE0, JD_FREE0 = JD_DONE0 + 4, JD_DRAIN = JD_FREE0 + 4, JD_COUNT };
+
+// One CTA per 128-token tile; head h: TMEM buffer h & 3 (D columns) and
+// W stage h & 1.  The MMA of head h overlaps the epilogue of head h - 1.
+__global__ void __launch_bounds__(kJDThreads, 1)
+    joint_decode_kernel(const __grid_constant__ CUtensorMap tmap_w, JointDecArgs a)
 {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    const uint32_t abytes = 128u * (uint32_t)a.r * 2u;
-    uint8_t *sAh = smem, *sAl = smem + abytes, *sB = smem + 2 * abytes;
-    uint64_t *bar = reinterpret_cast<uint64_t *>(smem + 3 * abytes);
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bar + 1);
-    const int tid = threadIdx.x, warp = tid >> 5;
+    const JDLayout L(a.r, a.D);
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + L.off_bar);
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + JD_COUNT);
+    auto bar = [&](int i) { return smem_u32(bars + i); };
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int64_t t0 = (int64_t)blockIdx.x * kJRows;
-    const int h = blockIdx.y;
-    const int64_t t = t0 + tid;
-    const bool valid = t < a.T;
+    const uint32_t tcols = (uint32_t)(a.D == 128 ? 512 : 256);
 
     if (warp == 0)
-        tmem_alloc(smem_u32(tmem_slot), 128);
+        tmem_alloc(smem_u32(tmem_slot), tcols);
     if (tid == 0) {
-        mbar_init(smem_u32(bar), 1);
+        mbar_init(bar(JD_WFULL0), 1);
+        mbar_init(bar(JD_WFULL1), 1);
+        for (int b = 0; b < 4; ++b) {
+            mbar_init(bar(JD_DONE0 + b), 1);
+            mbar_init(bar(JD_FREE0 + b), 4);  // the 4 warps of one epilogue group
+        }
+        mbar_init(bar(JD_DRAIN), 1);
         fence_mbar_init();
     }
-    // A: c^ of this token, split into bf16 hi + lo, K-major [r/64][128][128 B]
-    const int ng = a.r / a.G;
-    const uint32_t mask = (1u << a.bits) - 1u;
-    for (int u = 0; u < a.r / 8; ++u) {
-        uint4 wh = make_uint4(0, 0, 0, 0), wl = make_uint4(0, 0, 0, 0);
-        if (valid) {
-            const int c0 = u * 8;
-            const float2 sz = reinterpret_cast<const float2 *>(a.meta)[t * ng + c0 / a.G];
-            uint32_t cw;
-            if (a.bits == 4)
-                cw = *reinterpret_cast<const uint32_t *>(a.codes + t * (a.r / 2) + c0 / 2);
-            else
-                cw = *reinterpret_cast<const uint16_t *>(a.codes + t * (a.r / 4) + c0 / 4);
-            uint32_t hi[4], lo[4];
-#pragma unroll
-            for (int k = 0; k < 4; ++k) {
-                const float v0 = __fmul_rn(__fsub_rn((float)((cw >> (2 * k * a.bits)) & mask), sz.y), sz.x);
-                const float v1 = __fmul_rn(__fsub_rn((float)((cw >> ((2 * k + 1) * a.bits)) & mask), sz.y), sz.x);
-                const uint32_t a0 = __float_as_uint(v0) & 0xffff0000u, a1 = __float_as_uint(v1) & 0xffff0000u;
-                hi[k] = __byte_perm(a0, a1, 0x7632);
-                lo[k] = pack_bf16x2(v0 - __uint_as_float(a0), v1 - __uint_as_float(a1));
-            }
-            wh = make_uint4(hi[0], hi[1], hi[2], hi[3]);
-            wl = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+    if (warp == 8 && lane == 0) {
+        // W slices of the first heads while c^ is being built
+        for (int h = 0; h < L.nst && h < a.H; ++h) {
+            mbar_arrive_expect_tx(bar(JD_WFULL0 + h), L.w_bytes);
+            for (int c = 0; c < a.D / 64; ++c)
+                tma_load_2d(smem_u32(smem + L.off_w + (uint32_t)h * L.w_bytes + (uint32_t)c * (uint32_t)a.r * 128u),
+                            &tmap_w, bar(JD_WFULL0 + h), h * a.D + c * 64, 0);
         }
-        const uint32_t off = sw128_unit_offset(tid, u, kJRows);
-        *reinterpret_cast<uint4 *>(sAh + off) = wh;
-        *reinterpret_cast<uint4 *>(sAl + off) = wl;
     }
-    // B: W_dec rows n (K), columns [h D, h D + D) (N) -> MN-major [D/64][r][128 B]
-    const int HD = a.H * a.D;
-    for (int e = tid; e < a.r * (a.D / 8); e += kJThreads) {
-        const int n = e / (a.D / 8), u = e % (a.D / 8);
-        const uint4 w = __ldg(reinterpret_cast<const uint4 *>(a.w + (int64_t)n * HD + (int64_t)h * a.D) + u);
-        *reinterpret_cast<uint4 *>(sB + sw128_unit_offset(n, u, a.r)) = w;
+    if (warp < 8) {
+        // A: c^ = (q - z) s, split into bf16 hi (truncated) + lo (rounded
+        // remainder), K-major [r/64][128][128 B]
+        const int row = tid & 127, half = tid >> 7;
+        const int64_t t = t0 + row;
+        const bool valid = t < a.T;
+        const int ng = a.r / a.G;
+        const uint32_t mask = (1u << a.bits) - 1u;
+        for (int u = half * (a.r / 16); u < (half + 1) * (a.r / 16); ++u) {
+            uint4 wh = make_uint4(0, 0, 0, 0), wl = make_uint4(0, 0, 0, 0);
+            if (valid) {
+                const int c0 = u * 8;
+                const float2 sz = __ldg(reinterpret_cast<const float2 *>(a.meta) + t * ng + c0 / a.G);
+                uint32_t cw;
+                if (a.bits == 4)
+                    cw = __ldg(reinterpret_cast<const uint32_t *>(a.codes + t * (a.r / 2) + c0 / 2));
+                else
+                    cw = __ldg(reinterpret_cast<const uint16_t *>(a.codes + t * (a.r / 4) + c0 / 4));
+                uint32_t hi[4], lo[4];
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    const float v0 = __fmul_rn(__fsub_rn((float)((cw >> (2 * k * a.bits)) & mask), sz.y), sz.x);
+                    const float v1 = __fmul_rn(__fsub_rn((float)((cw >> ((2 * k + 1) * a.bits)) & mask), sz.y), sz.x);
+                    const uint32_t a0 = __float_as_uint(v0) & 0xffff0000u, a1 = __float_as_uint(v1) & 0xffff0000u;
+                    hi[k] = __byte_perm(a0, a1, 0x7632);
+                    lo[k] = pack_bf16x2(v0 - __uint_as_float(a0), v1 - __uint_as_float(a1));
+                }
+                wh = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+                wl = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+            }
+            const uint32_t off = sw128_unit_offset(row, u, kJRows);
+            *reinterpret_cast<uint4 *>(smem + off) = wh;
+            *reinterpret_cast<uint4 *>(smem + L.off_lo + off) = wl;
+        }
+        fence_proxy_async_smem();
     }
-    fence_proxy_async_smem();
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
     bool ok = true;
-    if (tid == 0) {
-        const uint32_t idesc = idesc_f32acc(128, a.D, true, false, true);
-        const uint32_t aAh = smem_u32(sAh), aAl = smem_u32(sAl), aB = smem_u32(sB);
-        const int nks = a.r / 16;
-        for (int part = 0; part < 2; ++part)
-            for (int ks = 0; ks < nks; ++ks) {
-                const uint32_t aoff = (uint32_t)(ks >> 2) * (128u * 128u) + (uint32_t)(ks & 3) * 32u;
-                umma_ss(tmem, sdesc_sw128((part ? aAl : aAh) + aoff, 16, 1024),
-                        sdesc_sw128(aB + (uint32_t)ks * 2048u, (uint32_t)a.r * 128u, 1024), idesc,
-                        (part || ks) ? 1u : 0u);
+
+    if (warp == 8) {
+        // ------------------------------------------------ W loads + MMAs
+        if (lane == 0) {
+            const uint32_t idesc = idesc_f32acc(128, a.D, true, false, true);
+            const uint32_t aAh = smem_u32(smem), aAl = smem_u32(smem + L.off_lo);
+            const int nks = a.r / 16;
+            const int nst = L.nst;
+            int h = 0;
+            for (; ok && h < a.H; ++h) {
+                const int s = h % nst, b = h & 3;
+                ok = mbar_wait(bar(JD_WFULL0 + s), (uint32_t)((h / nst) & 1));
+                if (ok && h >= 4)
+                    ok = mbar_wait(bar(JD_FREE0 + b), (uint32_t)(((h - 4) >> 2) & 1));
+                if (!ok)
+                    break;
+                tc_fence_after();
+                const uint32_t aB = smem_u32(smem + L.off_w + (uint32_t)s * L.w_bytes);
+                for (int part = 0; part < 2; ++part)
+                    for (int ks = 0; ks < nks; ++ks) {
+                        const uint32_t aoff = (uint32_t)(ks >> 2) * (128u * 128u) + (uint32_t)(ks & 3) * 32u;
+                        umma_ss(tmem + (uint32_t)(b * a.D), sdesc_sw128((part ? aAl : aAh) + aoff, 16, 1024),
+                                sdesc_sw128(aB + (uint32_t)ks * 2048u, (uint32_t)a.r * 128u, 1024), idesc,
+                                (part || ks) ? 1u : 0u);
+                    }
+                umma_commit(bar(JD_DONE0 + b));
+                if (h + nst < a.H) {
+                    // stage s is free once this head's MMAs are done
+                    ok = mbar_wait(bar(JD_DONE0 + b), (uint32_t)((h >> 2) & 1));
+                    if (!ok)
+                        break;
+                    mbar_arrive_expect_tx(bar(JD_WFULL0 + s), L.w_bytes);
+                    for (int c = 0; c < a.D / 64; ++c)
+                        tma_load_2d(smem_u32(smem + L.off_w + (uint32_t)s * L.w_bytes +
+                                             (uint32_t)c * (uint32_t)a.r * 128u),
+                                    &tmap_w, bar(JD_WFULL0 + s), (h + nst) * a.D + c * 64, 0);
+                }
             }
-        umma_commit(smem_u32(bar));
-    }
-    ok = mbar_wait(smem_u32(bar), 0);
-    tc_fence_after();
-    const uint32_t trow = tmem + (((uint32_t)warp * 32u) << 16);
-    int j = 0;
-    if (valid) {
-        j = a.idx[(int64_t)h * a.T + t];
-        if (j >= a.C) {
-            raise_status(DEVSTAT_BAD_INDEX);
-            j = 0;
+            // wait for every MMA issued before teardown; after a give-up also
+            // for the W loads already issued (heads h .. h + nst - 1)
+            umma_commit(bar(JD_DRAIN));
+            mbar_wait(bar(JD_DRAIN), 0);
+            if (!ok)
+                for (int hh = h; hh < a.H && hh < h + nst; ++hh)
+                    mbar_wait(bar(JD_WFULL0 + hh % nst), (uint32_t)((hh / nst) & 1));
         }
-    }
-    for (int cb = 0; cb < a.D / 32; ++cb) {
-        float v[32];
-        tmem_ld32(trow + (uint32_t)(cb * 32), v);
-        if (!valid || !ok)
-            continue;
-        const uint16_t *mu = a.cent + ((int64_t)h * a.C + j) * a.D + cb * 32;
-        float m8[8];
-        const int64_t o = (t * a.H + h) * a.D + cb * 32;
+        __syncwarp();
+    } else {
+        // ------------------------------------------------ epilogue
+        const int g = warp >> 2;
+        const int row = (warp & 3) * 32 + lane;
+        const int64_t t = t0 + row;
+        const bool valid = t < a.T;
+        const uint32_t lane_off = ((uint32_t)(warp & 3) * 32u) << 16;
+        for (int h = g; h < a.H; h += 2) {
+            const int b = h & 3;
+            int j = 0;
+            if (valid) {
+                j = __ldg(a.idx + (int64_t)h * a.T + t);
+                if (j >= a.C) {
+                    raise_status(DEVSTAT_BAD_INDEX);
+                    j = 0;
+                }
+            }
+            const uint16_t *mu = a.cent + ((int64_t)h * a.C + j) * a.D;
+            ok = __all_sync(0xffffffffu, ok && mbar_wait(bar(JD_DONE0 + b), (uint32_t)((h >> 2) & 1)));
+            if (!ok)
+                break;
+            tc_fence_after();
+            for (int cb = 0; cb < a.D / 32; ++cb) {
+                uint4 mw[4];
+                if (valid) {
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
-            load_bf16x8(mu + u * 8, m8);
+                    for (int u = 0; u < 4; ++u)
+                        mw[u] = __ldg(reinterpret_cast<const uint4 *>(mu + cb * 32) + u);
+                }
+                float v[32];
+                tmem_ld32(tmem + lane_off + (uint32_t)(b * a.D + cb * 32), v);
+                if (!valid)
+                    continue;
 #pragma unroll
-            for (int k = 0; k < 8; ++k)
-                v[u * 8 + k] = __fadd_rn(m8[k], v[u * 8 + k]);
-        }
-        if (a.out_bf16) {
-            uint4 *dst = reinterpret_cast<uint4 *>(static_cast<uint16_t *>(a.out) + o);
+                for (int u = 0; u < 4; ++u) {
+                    const uint32_t m[4] = {mw[u].x, mw[u].y, mw[u].z, mw[u].w};
 #pragma unroll
-            for (int u = 0; u < 4; ++u)
-                dst[u] = make_uint4(pack_bf16x2(v[8 * u], v[8 * u + 1]), pack_bf16x2(v[8 * u + 2], v[8 * u + 3]),
-                                    pack_bf16x2(v[8 * u + 4], v[8 * u + 5]), pack_bf16x2(v[8 * u + 6], v[8 * u + 7]));
-        } else {
-            float4 *dst = reinterpret_cast<float4 *>(static_cast<float *>(a.out) + o);
+                    for (int k = 0; k < 4; ++k) {
+                        v[u * 8 + 2 * k] = __fadd_rn(bf16_lo(m[k]), v[u * 8 + 2 * k]);
+                        v[u * 8 + 2 * k + 1] = __fadd_rn(bf16_hi(m[k]), v[u * 8 + 2 * k + 1]);
+                    }
+                }
+                const int64_t o = (t * a.H + h) * a.D + cb * 32;
+                if (a.out_bf16) {
+                    uint4 *dst = reinterpret_cast<uint4 *>(static_cast<uint16_t *>(a.out) + o);
 #pragma unroll
-            for (int u = 0; u < 8; ++u)
-                dst[u] = make_float4(v[4 * u], v[4 * u + 1], v[4 * u + 2], v[4 * u + 3]);
+                    for (int u = 0; u < 4; ++u)
+                        dst[u] = make_uint4(pack_bf16x2(v[8 * u], v[8 * u + 1]), pack_bf16x2(v[8 * u + 2], v[8 * u + 3]),
+                                            pack_bf16x2(v[8 * u + 4], v[8 * u + 5]),
+                                            pack_bf16x2(v[8 * u + 6], v[8 * u + 7]));
+                } else {
+                    float4 *dst = reinterpret_cast<float4 *>(static_cast<float *>(a.out) + o);
+#pragma unroll
+                    for (int u = 0; u < 8; ++u)
+                        dst[u] = make_float4(v[4 * u], v[4 * u + 1], v[4 * u + 2], v[4 * u + 3]);
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0)
+                mbar_arrive(bar(JD_FREE0 + b));
         }
     }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     if (warp == 0)
-        tmem_dealloc(tmem, 128);
+        tmem_dealloc(tmem, tcols);
 }
 
 }  // namespace kvq

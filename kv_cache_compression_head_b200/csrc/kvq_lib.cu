@@ -266,7 +266,23 @@ kvq_status launch_joint_encode(const JointEncArgs &a, cudaStream_t s)
     }
 }
 
-kvq_status launch_joint_decode(const JointDecArgs &a, cudaStream_t s)
+// 2-D map of W_dec [r][H*D] bf16: box = 64 output channels x r rows,
+// 128-byte swizzle (the MN-major B layout of the decoder's MMA).
+bool make_wdec_map(CUtensorMap *m, const void *w, int r, int HD)
+{
+    PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
+    if (!enc)
+        return false;
+    cuuint64_t dims[2] = {(cuuint64_t)HD, (cuuint64_t)r};
+    cuuint64_t strides[1] = {(cuuint64_t)HD * 2};
+    cuuint32_t box[2] = {64, (cuuint32_t)r};
+    cuuint32_t estr[2] = {1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(w), dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+kvq_status launch_joint_decode(const JointDecArgs &a, const void *w_dec, cudaStream_t s)
 {
     if (a.T == 0)
         return KVQ_OK;
@@ -276,12 +292,15 @@ kvq_status launch_joint_decode(const JointDecArgs &a, cudaStream_t s)
         return KVQ_ERR_CUDA;
     if (!configured[dev]) {
         if (cudaFuncSetAttribute(joint_decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)(joint_dec_smem_bytes(256) + 1024)) != cudaSuccess)
+                                 (int)(kJDSmemLimit + 1024)) != cudaSuccess)
             return KVQ_ERR_CUDA;
         configured[dev] = true;
     }
-    const dim3 grid((unsigned)ceil_div(a.T, kJRows), (unsigned)a.H);
-    joint_decode_kernel<<<grid, kJThreads, joint_dec_smem_bytes(a.r) + 1024, s>>>(a);
+    CUtensorMap m;
+    if (!make_wdec_map(&m, w_dec, a.r, a.H * a.D))
+        return KVQ_ERR_CUDA;
+    const JDLayout L(a.r, a.D);
+    joint_decode_kernel<<<(unsigned)ceil_div(a.T, kJRows), kJDThreads, L.total + 1024, s>>>(m, a);
     return launch_status();
 }
 
@@ -338,7 +357,7 @@ kvq_status joint_encode_call(const kvq_codec_desc *desc, const void *x, kvq_dtyp
 // Fit workspace: idx [H][T] u16 | per-chunk centre counts [H][nch][C] i32 |
 // bucket starts [H][C+1] i32 | token order [H][T] i32.
 struct FitLayout {
-    size_t idx, counts, starts, order, total;
+    size_t idx, counts, starts, order, sums, qsum, lmin, redo, total;
     int nchunks;
 };
 
@@ -353,7 +372,11 @@ FitLayout fit_layout(const kvq_codec_desc *d, int64_t T)
     L.counts = round_up(H * (size_t)T * 2, 256);
     L.starts = L.counts + round_up(H * (size_t)L.nchunks * C * 4, 256);
     L.order = L.starts + round_up(H * (C + 1) * 4, 256);
-    L.total = L.order + H * (size_t)T * 4;
+    L.sums = L.order + round_up(H * (size_t)T * 4, 256);
+    L.qsum = L.sums + round_up(H * C * (size_t)d->head_dim * 8, 256);
+    L.lmin = L.qsum + round_up(H * C * 8, 256);
+    L.redo = L.lmin + round_up(H * C * 4, 256);
+    L.total = L.redo + H * C * 4;
     return L;
 }
 
@@ -575,9 +598,13 @@ kvq_status kvq_fit_centroids(const kvq_codec_desc *desc, const void *x, kvq_dtyp
     fs.chunk_counts = reinterpret_cast<int *>(ws + Lw.counts);
     fs.bucket_start = reinterpret_cast<int *>(ws + Lw.starts);
     fs.order = reinterpret_cast<int *>(ws + Lw.order);
+    fs.sums = reinterpret_cast<double *>(ws + Lw.sums);
+    fs.qsum = reinterpret_cast<double *>(ws + Lw.qsum);
+    fs.lmin = reinterpret_cast<int *>(ws + Lw.lmin);
+    fs.redo = reinterpret_cast<int *>(ws + Lw.redo);
 
     const int64_t n_cent = (int64_t)H * C * D;
-    fit_seed_kernel<<<(unsigned)ceil_div(n_cent, 256), 256, 0, s>>>(f);
+    fit_seed_kernel<<<(unsigned)ceil_div(n_cent, 256), 256, 0, s>>>(f, fs);
     if ((st = launch_status()) != KVQ_OK)
         return st;
     const size_t cbytes = (size_t)C * 4;
@@ -604,10 +631,17 @@ kvq_status kvq_fit_centroids(const kvq_codec_desc *desc, const void *x, kvq_dtyp
         fit_scan_kernel<<<(unsigned)H, 1024, cbytes, s>>>(fs);
         fit_scatter_kernel<<<chunks, 32, cbytes, s>>>(fs);
         const int64_t warps = (int64_t)H * C;
-        if (D == 128)
-            fit_bucket_update_kernel<128><<<(unsigned)ceil_div(warps * 32, 256), 256, 0, s>>>(fs);
-        else
-            fit_bucket_update_kernel<64><<<(unsigned)ceil_div(warps * 32, 256), 256, 0, s>>>(fs);
+        const unsigned seg_blocks = (unsigned)ceil_div((int64_t)H * ceil_div(T, kFitSegSlots) * 32, 256);
+        const unsigned cent_blocks = (unsigned)ceil_div(warps * 32, 256);
+        if (D == 128) {
+            fit_segsum_kernel<128><<<seg_blocks, 256, 0, s>>>(fs);
+            fit_finalize_kernel<128><<<cent_blocks, 256, 0, s>>>(fs);
+            fit_bucket_update_kernel<128><<<cent_blocks, 256, 0, s>>>(fs);
+        } else {
+            fit_segsum_kernel<64><<<seg_blocks, 256, 0, s>>>(fs);
+            fit_finalize_kernel<64><<<cent_blocks, 256, 0, s>>>(fs);
+            fit_bucket_update_kernel<64><<<cent_blocks, 256, 0, s>>>(fs);
+        }
         if ((st = launch_status()) != KVQ_OK)
             return st;
     }
@@ -752,7 +786,6 @@ kvq_status kvq_decode(const kvq_compressed_view *view, void *x_out, kvq_dtype ou
         j.idx = view->idx;
         j.codes = view->codes;
         j.meta = view->meta;
-        j.w = static_cast<const uint16_t *>(view->w_dec);
         j.T = view->num_tokens;
         j.H = view->desc.num_heads;
         j.D = view->desc.head_dim;
@@ -762,7 +795,7 @@ kvq_status kvq_decode(const kvq_compressed_view *view, void *x_out, kvq_dtype ou
         j.G = view->desc.group_size;
         j.out = x_out;
         j.out_bf16 = out_dtype == KVQ_BF16;
-        return launch_joint_decode(j, reinterpret_cast<cudaStream_t>(stream));
+        return launch_joint_decode(j, view->w_dec, reinterpret_cast<cudaStream_t>(stream));
     }
     DecodeArgs a;
     a.cent = static_cast<const uint16_t *>(view->centroids);

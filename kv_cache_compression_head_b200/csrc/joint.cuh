@@ -280,6 +280,7 @@ __global__ void __launch_bounds__(kJDThreads, 1)
         mbar_init(bar(JD_DRAIN), 1);
         fence_mbar_init();
     }
+    __syncthreads();  // barriers initialised before any TMA names them
     if (warp == 8 && lane == 0) {
         // W slices of the first heads while c^ is being built
         for (int h = 0; h < L.nst && h < a.H; ++h) {

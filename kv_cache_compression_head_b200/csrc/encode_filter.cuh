@@ -19,8 +19,9 @@
 //      accumulation error, the rounding of |mu_j|^2 and of v_j, the rounding
 //      of the specified distance and the index bits carried in v.  When the
 //      second smallest v lies outside the window the smallest is the answer;
-//      otherwise the window is re-scored with the specified distance (lowest
-//      index wins ties);
+//      when only the two smallest lie inside it, the two threads of the token
+//      each score one of them with the specified distance; otherwise the
+//      whole window is re-scored (lowest index wins ties everywhere);
 //   4. the residual against the chosen centre is quantised (Eq. 1) per group
 //      and packed, each thread covering its half of the channels.
 #pragma once
@@ -50,10 +51,37 @@ struct FilterArgs {
     float kappa;       // window = kappa * (|x| + M)^2
 };
 
+constexpr uint32_t kFltPairBytes = 7168u;  // pair exchange: float4 [2][128] | int [2][128] | float4 [128]
+
 __host__ __device__ constexpr uint32_t flt_smem_bytes(int D, int Cpad)
 {
-    // X tile | centres | norms | pair exchange (3 x 128 x 16 B) | 2 barriers + slots
-    return (uint32_t)(D * 2 * kFltRows) + (uint32_t)(Cpad * D * 2) + (uint32_t)(Cpad * 4) + 6144u + 64u;
+    // X tile | centres | norms | pair exchange | 2 barriers + slots
+    return (uint32_t)(D * 2 * kFltRows) + (uint32_t)(Cpad * D * 2) + (uint32_t)(Cpad * 4) + kFltPairBytes + 64u;
+}
+
+// Insert (v, c) into the ascending list (b1, c1) <= (b2, c2) <= (b3, c3);
+// on equal values the entry already present stays first.
+__device__ __forceinline__ void top3_insert(float v, int c, float &b1, int &c1, float &b2, int &c2, float &b3,
+                                            int &c3)
+{
+    if (v < b3) {
+        if (v < b2) {
+            b3 = b2;
+            c3 = c2;
+            if (v < b1) {
+                b2 = b1;
+                c2 = c1;
+                b1 = v;
+                c1 = c;
+            } else {
+                b2 = v;
+                c2 = c;
+            }
+        } else {
+            b3 = v;
+            c3 = c;
+        }
+    }
 }
 
 // Specified binary32 distance of row `row` of the X tile to centre j of the
@@ -200,8 +228,10 @@ __global__ void __launch_bounds__(kFltThreads, 2)
     uint8_t *sX = smem;
     uint8_t *sMu = smem + D * 2 * kFltRows;
     float *sNrm = reinterpret_cast<float *>(sMu + Cpad * D * 2);
-    float4 *sPair = reinterpret_cast<float4 *>(sNrm + Cpad);  // [3][128]: pair exchange, exact winners
-    uint64_t *bars = reinterpret_cast<uint64_t *>(reinterpret_cast<uint8_t *>(sPair) + 6144);
+    float4 *sPair = reinterpret_cast<float4 *>(sNrm + Cpad);               // [2][128] {|x|^2 part, top 3}
+    int *sPairC = reinterpret_cast<int *>(sPair + 2 * 128);                  // [2][128] top-3 chunk ids
+    float4 *sWin = reinterpret_cast<float4 *>(sPairC + 2 * 128);             // [128] exact winners / distances
+    uint64_t *bars = reinterpret_cast<uint64_t *>(reinterpret_cast<uint8_t *>(sPair) + kFltPairBytes);
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 2);
     uint32_t *sMaxNrm = tmem_slot + 1;
 
@@ -305,17 +335,17 @@ __global__ void __launch_bounds__(kFltThreads, 2)
         }
         // (2) v_j = |mu_j|^2 - 2 p_j over this thread's chunks.  The chunk-local
         // column index rides in the low 5 mantissa bits of v, so one pass keeps
-        // the smallest and the second smallest value (the window below absorbs
-        // the <= 31 ulp this perturbs v).
-        float b1 = INFINITY, b2 = INFINITY;  // best and second best of this thread
-        int bchunk = 0;
+        // the three smallest values (the window below absorbs the <= 31 ulp
+        // this perturbs v); chunk ids are kept beside them.
+        float b1 = INFINITY, b2 = INFINITY, b3 = INFINITY;
+        int k1 = 0, k2 = 0, k3 = 0;
 #pragma unroll
         for (int k = 0; k < kMaxChunks; ++k) {
             const int c = c_lo + k;
             if (c < c_hi) {
                 float p[32];
                 tmem_ld32(tmem + lane_off + (uint32_t)(c * 32), p);
-                float m1 = INFINITY, m2 = INFINITY;
+                float m1 = INFINITY, m2 = INFINITY, m3 = INFINITY;
                 const float4 *nrm4 = reinterpret_cast<const float4 *>(sNrm + c * 32);
 #pragma unroll
                 for (int i4 = 0; i4 < 8; ++i4) {
@@ -326,41 +356,81 @@ __global__ void __launch_bounds__(kFltThreads, 2)
                         const int i = i4 * 4 + e;
                         const float v = fmaf(-2.0f, p[i], nn[e]);
                         const float vp = __uint_as_float((__float_as_uint(v) & ~31u) | (uint32_t)i);
+                        m3 = fminf(m3, fmaxf(m2, vp));
                         m2 = fminf(m2, fmaxf(m1, vp));
                         m1 = fminf(m1, vp);
                     }
                 }
-                // fold the chunk into the thread's (best, second best)
-                if (m1 < b1) {
-                    b2 = fminf(b1, m2);
-                    b1 = m1;
-                    bchunk = c;
-                } else {
-                    b2 = fminf(b2, m1);
-                }
+                top3_insert(m1, c, b1, k1, b2, k2, b3, k3);
+                top3_insert(m2, c, b1, k1, b2, k2, b3, k3);
+                top3_insert(m3, c, b1, k1, b2, k2, b3, k3);
             }
         }
-        // (3) exchange with the partner thread of this row (warps w and w+4)
-        sPair[half * 128 + row] = make_float4(xx, b1, b2, __int_as_float(bchunk));
+        // (3) exchange with the partner thread of this row (warps w and w+4);
+        // both threads then hold the row's three smallest values, half-0
+        // entries first on equal values
+        sPair[half * 128 + row] = make_float4(xx, b1, b2, b3);
+        sPairC[half * 128 + row] = k1 | (k2 << 8) | (k3 << 16);
         named_barrier_sync_q(warp & 3, 64);
         const float4 other = sPair[(half ^ 1) * 128 + row];
+        const int oc = sPairC[(half ^ 1) * 128 + row];
+        float g1, g2, g3;
+        int h1, h2, h3;
+        {
+            // list of half 0, then insert half 1's entries
+            const bool h0 = half == 0;
+            g1 = h0 ? b1 : other.y;
+            g2 = h0 ? b2 : other.z;
+            g3 = h0 ? b3 : other.w;
+            const int cc = h0 ? (k1 | (k2 << 8) | (k3 << 16)) : oc;
+            h1 = cc & 0xff;
+            h2 = (cc >> 8) & 0xff;
+            h3 = (cc >> 16) & 0xff;
+            const int dc = h0 ? oc : (k1 | (k2 << 8) | (k3 << 16));
+            top3_insert(h0 ? other.y : b1, dc & 0xff, g1, h1, g2, h2, g3, h3);
+            top3_insert(h0 ? other.z : b2, (dc >> 8) & 0xff, g1, h1, g2, h2, g3, h3);
+            top3_insert(h0 ? other.w : b3, (dc >> 16) & 0xff, g1, h1, g2, h2, g3, h3);
+        }
         const float xn = sqrtf(xx + other.x);
-        const float thr = fminf(b1, other.y) + a.kappa * (xn + Mnorm) * (xn + Mnorm);
-        const bool mine = b1 < other.y || (b1 == other.y && half == 0);
-        const float best_v = mine ? b1 : other.y;
-        const float second = fminf(fminf(b2, other.z), mine ? other.y : b1);
-        const int best_chunk = mine ? bchunk : __float_as_int(other.w);
-        int best = best_chunk * 32 + (int)(__float_as_uint(best_v) & 31u);
-        const bool exact = !(second > thr) || !(thr < INFINITY);
-        // rare: re-score the window (or every centre when the window is not
-        // finite) with the specified distance; the half-0 thread decides and
-        // hands the result to its partner.  Both warps of the pair see the same
-        // `exact` flags, so they take the branch together.
-        if (__any_sync(0xffffffffu, exact)) {
+        const float thr = g1 + a.kappa * (xn + Mnorm) * (xn + Mnorm);
+        int best = h1 * 32 + (int)(__float_as_uint(g1) & 31u);
+        const bool finite = thr < INFINITY;
+        const bool pair_case = finite && !(g2 > thr) && g3 > thr;    // two candidates
+        const bool wide_case = !finite || (!(g2 > thr) && !(g3 > thr));  // three or more
+        // two candidates: each thread of the pair scores one with the specified
+        // distance; the smaller wins, the lower index on a tie
+        if (__any_sync(0xffffffffu, pair_case)) {
+            const int j1 = best, j2 = h2 * 32 + (int)(__float_as_uint(g2) & 31u);
+            float dmine = 0.0f;
+            if (pair_case)
+                dmine = spec_distance_smem<D>(sX, sMu, Cpad, row, half == 0 ? j1 : j2);
+            if (pair_case) {
+                if (half == 0)
+                    sWin[row].x = dmine;
+            }
+            named_barrier_sync_q(warp & 3, 64);
+            if (pair_case) {
+                const float d1 = half == 0 ? dmine : sWin[row].x;
+                const float d2 = half == 0 ? 0.0f : dmine;
+                if (half == 1) {
+                    const int lo = j1 < j2 ? j1 : j2;
+                    const int hi = j1 < j2 ? j2 : j1;
+                    const float dlo = j1 < j2 ? d1 : d2, dhi = j1 < j2 ? d2 : d1;
+                    sWin[row].y = __int_as_float(dhi < dlo ? hi : lo);
+                }
+            }
+            named_barrier_sync_q(warp & 3, 64);
+            if (pair_case)
+                best = __float_as_int(sWin[row].y);
+        }
+        // three or more candidates (rare): re-score the window (or every centre
+        // when the window is not finite) with the specified distance; the
+        // half-0 thread decides and hands the result to its partner.  Both
+        // warps of the pair see the same flags, so they take the branch together.
+        if (__any_sync(0xffffffffu, wide_case)) {
             if (half == 0) {
                 float bd = INFINITY;
                 int bj = -1;
-                const bool all = !(thr < INFINITY);
                 for (int c = 0; c < nchunks; ++c) {
                     float p[32];
                     tmem_ld32(tmem + lane_off + (uint32_t)(c * 32), p);
@@ -369,7 +439,7 @@ __global__ void __launch_bounds__(kFltThreads, 2)
                     for (int i = 0; i < 32; ++i) {
                         const int j = c * 32 + i;
                         const float v = fmaf(-2.0f, p[i], sNrm[j]);
-                        if (exact && j < a.C && (all || v <= thr))
+                        if (wide_case && j < a.C && (!finite || v <= thr))
                             cand |= 1u << i;
                     }
                     while (cand) {  // increasing index order
@@ -383,11 +453,11 @@ __global__ void __launch_bounds__(kFltThreads, 2)
                         }
                     }
                 }
-                sPair[2 * 128 + row] = make_float4(__int_as_float(bj), 0.f, 0.f, 0.f);
+                sWin[row] = make_float4(__int_as_float(bj), 0.f, 0.f, 0.f);
             }
             named_barrier_sync_q(warp & 3, 64);
-            if (exact)
-                best = __float_as_int(sPair[2 * 128 + row].x);
+            if (wide_case)
+                best = __float_as_int(sWin[row].x);
         }
         if (best < 0 || best >= a.C)
             best = 0;  // unreachable for finite inputs

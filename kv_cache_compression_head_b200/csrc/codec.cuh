@@ -71,6 +71,51 @@ __device__ __forceinline__ uint32_t quant_code(float r, const GroupQ &g, int bit
     return (uint32_t)v;
 }
 
+// Eq. 1 codes of a group whose every |r * inv| is below 2^22 (checked once
+// per group), without the conversion unit: t + 1.5 2^23 rounds t to the
+// nearest integer, ties to even -- rint(t) -- in the low significand bits, so
+// rint(t) + z is an integer add on those bits.  Equal to quant_code.
+struct GroupFast {
+    float inv;
+    int zoff;  // z - bits(1.5 2^23)
+    bool fast;
+};
+
+__device__ __forceinline__ GroupFast group_fast(const GroupQ &g, float mn, float mx)
+{
+    GroupFast f;
+    f.inv = g.inv;
+    f.fast = !g.degenerate && __fmul_rn(fmaxf(fabsf(mn), fabsf(mx)), g.inv) < 4194304.0f;
+    f.zoff = f.fast ? (int)g.z - 0x4B400000 : 0;
+    return f;
+}
+
+template <int BITS>
+__device__ __forceinline__ uint32_t quant_code_fast(float r, const GroupFast &f)
+{
+    const int v = __float_as_int(__fadd_rn(__fmul_rn(r, f.inv), 12582912.0f)) + f.zoff;
+    return (uint32_t)min(max(v, 0), (1 << BITS) - 1);
+}
+
+// Codes of the G values r[0..G) of one group, added (the bit fields are
+// disjoint) into words at channel offset c0 (low bits first).
+template <int G, int BITS>
+__device__ __forceinline__ void quant_group_into(const float *r, const GroupQ &g, float mn, float mx, uint32_t *words,
+                                                 int c0)
+{
+    constexpr int kPerWord = 32 / BITS;
+    const GroupFast f = group_fast(g, mn, mx);
+    if (f.fast) {
+#pragma unroll
+        for (int c = 0; c < G; ++c)
+            words[(c0 + c) / kPerWord] += quant_code_fast<BITS>(r[c], f) << (((c0 + c) % kPerWord) * BITS);
+    } else {
+#pragma unroll
+        for (int c = 0; c < G; ++c)
+            words[(c0 + c) / kPerWord] += quant_code(r[c], g, BITS) << (((c0 + c) % kPerWord) * BITS);
+    }
+}
+
 __device__ __forceinline__ float dequant_spec(uint32_t q, float s, float z, float mu)
 {
     return __fadd_rn(mu, __fmul_rn(__fsub_rn((float)q, z), s));
@@ -109,7 +154,6 @@ template <int D, int BITS, int G>
 __device__ __forceinline__ void encode_residual_row(const float *r, uint8_t *codes_row, float2 *meta_row)
 {
     constexpr int kWords = D * BITS / 32;
-    constexpr int kPerWord = 32 / BITS;
     uint32_t words[kWords];
 #pragma unroll
     for (int w = 0; w < kWords; ++w)
@@ -124,9 +168,7 @@ __device__ __forceinline__ void encode_residual_row(const float *r, uint8_t *cod
         }
         const GroupQ gq = group_params(mn, mx, BITS);
         meta_row[g] = make_float2(gq.s, gq.z);
-#pragma unroll
-        for (int c = g * G; c < (g + 1) * G; ++c)
-            words[c / kPerWord] |= quant_code(r[c], gq, BITS) << ((c % kPerWord) * BITS);
+        quant_group_into<G, BITS>(r + g * G, gq, mn, mx, words, g * G);
     }
     uint4 *dst = reinterpret_cast<uint4 *>(codes_row);
 #pragma unroll

@@ -157,11 +157,7 @@ __device__ __forceinline__ void encode_residual_smem(const uint8_t *sX, const ui
             }
             const GroupQ gq = group_params(mn, mx, BITS);
             meta_dst[g] = make_float2(gq.s, gq.z);
-#pragma unroll
-            for (int c = 0; c < G; ++c) {
-                const int cc = g * G + c;
-                words[cc / kPerWord] |= quant_code(r[c], gq, BITS) << ((cc % kPerWord) * BITS);
-            }
+            quant_group_into<G, BITS>(r, gq, mn, mx, words, g * G);
             continue;
         }
         float mn = 0.0f, mx = 0.0f;
@@ -186,6 +182,7 @@ __device__ __forceinline__ void encode_residual_smem(const uint8_t *sX, const ui
         }
         const GroupQ gq = group_params(mn, mx, BITS);
         meta_dst[g] = make_float2(gq.s, gq.z);
+        const GroupFast gf = group_fast(gq, mn, mx);
 #pragma unroll
         for (int uu = 0; uu < G / 8; ++uu) {
             const int u = half * (CH / 8) + g * (G / 8) + uu;
@@ -197,7 +194,8 @@ __device__ __forceinline__ void encode_residual_smem(const uint8_t *sX, const ui
                 const float r = __fsub_rn((k & 1) ? bf16_hi(xa[k >> 1]) : bf16_lo(xa[k >> 1]),
                                           (k & 1) ? bf16_hi(ma[k >> 1]) : bf16_lo(ma[k >> 1]));
                 const int c = g * G + uu * 8 + k;
-                words[c / kPerWord] |= quant_code(r, gq, BITS) << ((c % kPerWord) * BITS);
+                words[c / kPerWord] += (gf.fast ? quant_code_fast<BITS>(r, gf) : quant_code(r, gq, BITS))
+                                       << ((c % kPerWord) * BITS);
             }
         }
     }

@@ -61,7 +61,6 @@ __device__ __forceinline__ void joint_quant_row(uint32_t trow, int r, uint8_t *c
                                                 float *coef_row)
 {
     static_assert(G % 16 == 0 && G <= 64, "group of 16, 32 or 64 coefficients");
-    constexpr int kPerWord = 32 / BITS;
     constexpr int kWords = G * BITS / 32;
     for (int g = 0; g < r / G; ++g) {
         float v[G];
@@ -95,15 +94,15 @@ __device__ __forceinline__ void joint_quant_row(uint32_t trow, int r, uint8_t *c
         }
         const GroupQ gq = group_params(mn, mx, BITS);
         meta_row[g] = make_float2(gq.s, gq.z);
+        uint32_t wv[kWords];
+#pragma unroll
+        for (int w = 0; w < kWords; ++w)
+            wv[w] = 0u;
+        quant_group_into<G, BITS>(v, gq, mn, mx, wv, 0);
         uint32_t *words = reinterpret_cast<uint32_t *>(codes_row) + g * kWords;
 #pragma unroll
-        for (int w = 0; w < kWords; ++w) {
-            uint32_t word = 0;
-#pragma unroll
-            for (int c = 0; c < kPerWord; ++c)
-                word |= quant_code(v[w * kPerWord + c], gq, BITS) << (c * BITS);
-            words[w] = word;
-        }
+        for (int w = 0; w < kWords; ++w)
+            words[w] = wv[w];
     }
 }
 

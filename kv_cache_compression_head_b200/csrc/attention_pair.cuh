@@ -28,9 +28,11 @@
 // P(j,i) in TMEM only after P V(j,i) has read it.
 //
 // Producers: each thread rebuilds 4 units (32 channels) of one K row and of
-// one V row per tile.  The global loads of the next item (its centre row,
-// codes and {s, z}) are issued before the current item is rebuilt, and the
-// centre index two items ahead, so the gather latency overlaps arithmetic.
+// one V row per tile.  Two tiles ahead it stages, with per-thread
+// asynchronous copies, the centre rows of its units directly into their
+// swizzled slots of the operand tiles (K hi, V) and its code words and
+// {s, z} into its own slots of the K lo tile; when the tile's turn comes it
+// rebuilds the values in place.  Three stages of K and V tiles.
 //
 // Barriers (parity = use count & 1).  Counted on the leader, arrived on once
 // per warp from both CTAs (release.cluster, after each lane's proxy fence and
@@ -56,21 +58,23 @@ constexpr int kAPProducers = 256;
 constexpr int kAPRowsPerCta = 256;
 constexpr int kAPRowsPerPair = 512;
 
+constexpr int kAPStages = 3;
+
 struct APSmem {
     static constexpr uint32_t kQ = 128 * 2 * 128;     // one 128-row Q tile (d = 128)
     static constexpr uint32_t kKh = 64 * 2 * 128;     // 64 history rows x 128 channels, bf16
     static constexpr uint32_t kV = 128 * 2 * 64;      // 128 history rows x 64 channels, fp16
     static constexpr uint32_t offQ = 0;               // Q tile t at offQ + t kQ
     static constexpr uint32_t offK = 2 * kQ;          // K stage s part p at offK + (2 s + p) kKh
-    static constexpr uint32_t offV = offK + 4 * kKh;  // V stage s at offV + s kV
-    static constexpr uint32_t offBar = offV + 2 * kV;
+    static constexpr uint32_t offV = offK + 2 * kAPStages * kKh;  // V stage s at offV + s kV
+    static constexpr uint32_t offBar = offV + kAPStages * kV;
     static constexpr uint32_t kBytes = offBar + 256;
     static constexpr uint32_t kLaunchBytes = kBytes + 1024;
 };
 
 enum {
-    P_QREADY = 0, P_KFULL0, P_KFULL1, P_VFULL0, P_VFULL1, P_SFULL0, P_SFULL1, P_PFULL0, P_PFULL1,
-    P_KFREE0, P_KFREE1, P_VFREE0, P_VFREE1, P_OFULL, P_COUNT
+    P_QREADY = 0, P_KFULL0, P_VFULL0 = P_KFULL0 + kAPStages, P_SFULL0 = P_VFULL0 + kAPStages, P_SFULL1,
+    P_PFULL0, P_PFULL1, P_KFREE0, P_VFREE0 = P_KFREE0 + kAPStages, P_OFULL = P_VFREE0 + kAPStages, P_COUNT
 };
 
 __device__ __forceinline__ uint32_t cluster_ctarank()
@@ -155,102 +159,109 @@ __device__ __forceinline__ void umma2_commit_both(uint32_t bar)
         : "memory");
 }
 
-// One thread's share of one history row: 4 units (8 channels each) of the
-// centre row, their code words and their groups' {s, z}.
-struct APRow {
-    uint4 mu[4];
-    uint32_t cw[4];
-    float2 sz[4];
-};
-
-// Centre index of history row `tok` (0 for rows past the range).
-__device__ __forceinline__ int ap_index(const CodecView &cv, int h, int64_t tok, bool valid)
-{
-    return valid ? (int)__ldg(cv.idx + (int64_t)h * cv.T + tok) : 0;
-}
-
-// Issue the loads of units [u0, u0 + 4) of row `tok` (centre j).
-template <int BITS>
-__device__ __forceinline__ void ap_load(const CodecView &cv, int h, int64_t tok, bool valid, int j, int u0,
-                                        APRow &r)
-{
-    constexpr int D = 128;
-    if (!valid)
-        return;
-    if (j >= cv.C) {
-        raise_status(DEVSTAT_BAD_INDEX);
-        j = 0;
-    }
-    const int64_t th = (int64_t)h * cv.T + tok;
-    const uint4 *mu_row = reinterpret_cast<const uint4 *>(cv.cent + ((int64_t)h * cv.C + j) * D) + u0;
-#pragma unroll
-    for (int uu = 0; uu < 4; ++uu)
-        r.mu[uu] = __ldg(mu_row + uu);
-    if (BITS == 2) {
-        const uint16_t *cr = reinterpret_cast<const uint16_t *>(cv.codes + th * (D / 4)) + u0;
-#pragma unroll
-        for (int uu = 0; uu < 4; ++uu)
-            r.cw[uu] = __ldg(cr + uu);
-    } else {
-        const uint32_t *cr = reinterpret_cast<const uint32_t *>(cv.codes + th * (D / 2)) + u0;
-#pragma unroll
-        for (int uu = 0; uu < 4; ++uu)
-            r.cw[uu] = __ldg(cr + uu);
-    }
-    const float2 *meta_row = reinterpret_cast<const float2 *>(cv.meta) + th * (D / cv.G);
-#pragma unroll
-    for (int uu = 0; uu < 4; ++uu)
-        r.sz[uu] = __ldg(meta_row + (u0 + uu) * 8 / cv.G);
-}
-
-// Rebuild the loaded units into `tile` at swizzled row `row` of a tile with
-// `rows` rows (unit u0 + uu lands at unit u0 + uu - ubase):
-//   x^ = fma(f, 2^b s, mu - (2^b + z) s),  f = 1 + q 2^-b
-// which is the decoder's mu + (q - z) s up to one rounding.  K (SPLIT): bf16
-// hi (truncated) + lo (the rounded remainder) tiles; V: one fp16 tile.
+// Rebuild 4 units of one row in place: the centre units were staged at
+// `tile + off[uu]`; codes `cw` and each unit's {s, z} come from the staging
+// slots.  x^ = fma(f, 2^b s, mu - (2^b + z) s),  f = 1 + q 2^-b, which is the
+// decoder's mu + (q - z) s up to one rounding.  K (SPLIT): bf16 hi
+// (truncated) in place + lo (the rounded remainder) at `lo + off[uu]`; V: fp16.
 template <int BITS, bool SPLIT>
-__device__ __forceinline__ void ap_store(const APRow &r, bool valid, int u0, int ubase, uint8_t *tile,
-                                         uint8_t *tile_lo, uint32_t row, uint32_t rows)
+__device__ __forceinline__ void ap_rebuild(uint8_t *tile, uint8_t *lo, const uint32_t *off, const uint32_t *cw,
+                                           const float2 *sz, bool valid)
 {
     constexpr float kTwoB = (float)(1 << BITS);
 #pragma unroll
     for (int uu = 0; uu < 4; ++uu) {
-        const uint32_t off = sw128_unit_offset(row, u0 + uu - ubase, rows);
+        uint4 *dst = reinterpret_cast<uint4 *>(tile + off[uu]);
         if (!valid) {
-            *reinterpret_cast<uint4 *>(tile + off) = make_uint4(0, 0, 0, 0);
+            *dst = make_uint4(0, 0, 0, 0);
             if (SPLIT)
-                *reinterpret_cast<uint4 *>(tile_lo + off) = make_uint4(0, 0, 0, 0);
+                *reinterpret_cast<uint4 *>(lo + off[uu]) = make_uint4(0, 0, 0, 0);
             continue;
         }
-        const float2 sz = r.sz[uu];
-        const float sc = kTwoB * sz.x;
-        const float nb = -__fmul_rn(kTwoB + sz.y, sz.x);
-        const uint32_t ma[4] = {r.mu[uu].x, r.mu[uu].y, r.mu[uu].z, r.mu[uu].w};
+        const uint4 mw = *dst;
+        const float sc = kTwoB * sz[uu].x;
+        const float nb = -__fmul_rn(kTwoB + sz[uu].y, sz[uu].x);
+        const uint32_t ma[4] = {mw.x, mw.y, mw.z, mw.w};
         float2 val[4];
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
-            const float2 f = make_float2(code_as_unit_float<BITS>(r.cw[uu], 2 * k),
-                                         code_as_unit_float<BITS>(r.cw[uu], 2 * k + 1));
+            const float2 f = make_float2(code_as_unit_float<BITS>(cw[uu], 2 * k),
+                                         code_as_unit_float<BITS>(cw[uu], 2 * k + 1));
             const float2 b = add2(make_float2(bf16_lo(ma[k]), bf16_hi(ma[k])), make_float2(nb, nb));
             val[k] = fma2(f, make_float2(sc, sc), b);
         }
         if (SPLIT) {
-            uint32_t hi[4], lo[4];
+            uint32_t hi[4], lw[4];
 #pragma unroll
             for (int k = 0; k < 4; ++k) {
                 const uint32_t a0 = __float_as_uint(val[k].x) & 0xffff0000u;
                 const uint32_t a1 = __float_as_uint(val[k].y) & 0xffff0000u;
                 hi[k] = __byte_perm(a0, a1, 0x7632);
                 const float2 d = sub2(val[k], make_float2(__uint_as_float(a0), __uint_as_float(a1)));
-                lo[k] = pack_bf16x2(d.x, d.y);
+                lw[k] = pack_bf16x2(d.x, d.y);
             }
-            *reinterpret_cast<uint4 *>(tile + off) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
-            *reinterpret_cast<uint4 *>(tile_lo + off) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+            *dst = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+            *reinterpret_cast<uint4 *>(lo + off[uu]) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
         } else {
-            *reinterpret_cast<uint4 *>(tile + off) =
-                make_uint4(pack_f16x2_sat(val[0].x, val[0].y), pack_f16x2_sat(val[1].x, val[1].y),
-                           pack_f16x2_sat(val[2].x, val[2].y), pack_f16x2_sat(val[3].x, val[3].y));
+            *dst = make_uint4(pack_f16x2_sat(val[0].x, val[0].y), pack_f16x2_sat(val[1].x, val[1].y),
+                              pack_f16x2_sat(val[2].x, val[2].y), pack_f16x2_sat(val[3].x, val[3].y));
         }
+    }
+}
+
+// Stage units [u0, u0 + 4) of history row `tok` (centre j) of one codec: the
+// centre units into `tile + off[uu]`, the code words (8 or 16 B) into
+// `stage_cw` and the {s, z} of their groups (8 or 16 B) into `stage_sz`.
+template <int BITS>
+__device__ __forceinline__ void ap_stage(const CodecView &cv, int h, int64_t tok, int j, int u0, uint32_t tile,
+                                         const uint32_t *off, uint32_t stage_cw, uint32_t stage_sz)
+{
+    constexpr int D = 128;
+    if (j >= cv.C) {
+        raise_status(DEVSTAT_BAD_INDEX);
+        j = 0;
+    }
+    const int64_t th = (int64_t)h * cv.T + tok;
+    const uint16_t *mu = cv.cent + ((int64_t)h * cv.C + j) * D + u0 * 8;
+#pragma unroll
+    for (int uu = 0; uu < 4; ++uu)
+        cp_async16(tile + off[uu], mu + uu * 8);
+    if (BITS == 2)
+        cp_async8(stage_cw, cv.codes + th * (D / 4) + u0 * 2);
+    else
+        cp_async16(stage_cw, cv.codes + th * (D / 2) + u0 * 4);
+    const float *meta = cv.meta + (th * (D / cv.G) + (u0 * 8) / cv.G) * 2;
+    if (cv.G == 16)
+        cp_async16(stage_sz, meta);
+    else
+        cp_async8(stage_sz, meta);
+}
+
+// Code words and per-unit {s, z} of 4 units from the staging slots.
+template <int BITS>
+__device__ __forceinline__ void ap_read_stage(const uint8_t *stage_cw, const uint8_t *stage_sz, int G, uint32_t *cw,
+                                              float2 *sz)
+{
+    if (BITS == 2) {
+        const uint2 w = *reinterpret_cast<const uint2 *>(stage_cw);
+        cw[0] = w.x & 0xffffu;
+        cw[1] = w.x >> 16;
+        cw[2] = w.y & 0xffffu;
+        cw[3] = w.y >> 16;
+    } else {
+        const uint4 w = *reinterpret_cast<const uint4 *>(stage_cw);
+        cw[0] = w.x;
+        cw[1] = w.y;
+        cw[2] = w.z;
+        cw[3] = w.w;
+    }
+    if (G == 16) {
+        const float4 m = *reinterpret_cast<const float4 *>(stage_sz);
+        sz[0] = sz[1] = make_float2(m.x, m.y);
+        sz[2] = sz[3] = make_float2(m.z, m.w);
+    } else {
+        const float2 m = *reinterpret_cast<const float2 *>(stage_sz);
+        sz[0] = sz[1] = sz[2] = sz[3] = m;
     }
 }
 
@@ -264,8 +275,11 @@ __device__ __forceinline__ void ap_publish(uint32_t lead_bar)
         mbar_arrive_cluster(lead_bar);
 }
 
-// Producer loop: items K(0), V(0), K(1), V(1), ...; K(i) and V(i) reuse the
-// stage of tile i - 2 once its MMAs are done.
+// Producer loop over tiles i: stage K(i + 2) once the QK of tile i - 1 has
+// freed its stage, rebuild K(i), stage V(i + 2) once the P V of tile i - 1
+// has freed its stage, rebuild V(i).  One commit group per staging step
+// (empty past the end), so "all but the newest three groups" is always the
+// pair K(i), V(i).
 template <int BK, int BV>
 __device__ __forceinline__ void ap_produce(const AttnArgs &a, int h, uint32_t rank, int tid, int ntiles,
                                            uint8_t *smem, uint64_t *bars, volatile int *abort_flag)
@@ -273,42 +287,100 @@ __device__ __forceinline__ void ap_produce(const AttnArgs &a, int h, uint32_t ra
     using L = APSmem;
     auto bar = [&](int i) { return smem_u32(bars + i); };
     auto lead = [&](int i) { return mapa_shared(bar(i), 0); };
+    auto khi = [&](int s) { return smem + L::offK + (uint32_t)(2 * s) * L::kKh; };
+    auto klo = [&](int s) { return smem + L::offK + (uint32_t)(2 * s + 1) * L::kKh; };
+    auto vst = [&](int s) { return smem + L::offV + (uint32_t)s * L::kV; };
     // K: history rows [64 rank, 64 rank + 64) of the tile; thread -> (row
-    // tid & 63, channel quarter tid >> 6: units 4q .. 4q + 3)
+    // tid & 63, channel quarter tid >> 6: units 4q .. 4q + 3).  Its 4 K lo
+    // slots double as staging: K codes, K {s, z}, V codes, V {s, z}.
     const uint32_t krow = (uint32_t)(tid & 63);
     const int ku0 = 4 * (tid >> 6);
     // V: channels [64 rank, 64 rank + 64); thread -> (row tid & 127, units
     // 8 rank + 4 (tid >> 7) .. + 3)
     const uint32_t vrow = (uint32_t)(tid & 127);
     const int vu0 = 8 * (int)rank + 4 * (tid >> 7);
+    uint32_t koff[4], voff[4];
+#pragma unroll
+    for (int uu = 0; uu < 4; ++uu) {
+        koff[uu] = sw128_unit_offset(krow, ku0 + uu, 64);
+        voff[uu] = sw128_unit_offset(vrow, vu0 - 8 * (int)rank + uu, 128);
+    }
     auto ktok = [&](int i) { return a.t_begin + (int64_t)i * 128 + 64 * rank + krow; };
     auto vtok = [&](int i) { return a.t_begin + (int64_t)i * 128 + vrow; };
+    auto kidx = [&](int i) {
+        const int64_t t = ktok(i);
+        return (i < ntiles && t < a.t_end) ? (int)__ldg(a.k.idx + (int64_t)h * a.k.T + t) : 0;
+    };
+    auto vidx = [&](int i) {
+        const int64_t t = vtok(i);
+        return (i < ntiles && t < a.t_end) ? (int)__ldg(a.v.idx + (int64_t)h * a.v.T + t) : 0;
+    };
+    auto stage_k = [&](int i, int j) {
+        const int s = i % kAPStages;
+        if (ktok(i) < a.t_end)
+            ap_stage<BK>(a.k, h, ktok(i), j, ku0, smem_u32(khi(s)), koff, smem_u32(klo(s) + koff[0]),
+                         smem_u32(klo(s) + koff[1]));
+    };
+    auto stage_v = [&](int i, int j) {
+        const int s = i % kAPStages;
+        if (vtok(i) < a.t_end)
+            ap_stage<BV>(a.v, h, vtok(i), j, vu0, smem_u32(vst(s)), voff, smem_u32(klo(s) + koff[2]),
+                         smem_u32(klo(s) + koff[3]));
+    };
 
-    APRow rk, rv;
-    int jk = ap_index(a.k, h, ktok(0), ktok(0) < a.t_end);
-    int jv = ap_index(a.v, h, vtok(0), vtok(0) < a.t_end);
-    ap_load<BK>(a.k, h, ktok(0), ktok(0) < a.t_end, jk, ku0, rk);
-    jk = (ntiles > 1) ? ap_index(a.k, h, ktok(1), ktok(1) < a.t_end) : 0;
-    for (int i = 0; i < ntiles; ++i) {
-        const int s = i & 1;
-        const uint32_t par = (uint32_t)(((i - 2) >> 1) & 1);
-        ap_load<BV>(a.v, h, vtok(i), vtok(i) < a.t_end, jv, vu0, rv);
-        jv = (i + 1 < ntiles) ? ap_index(a.v, h, vtok(i + 1), vtok(i + 1) < a.t_end) : 0;
-        if (i >= 2 && !__all_sync(0xffffffffu, ap_wait(bar(s ? P_KFREE1 : P_KFREE0), par, abort_flag)))
-            return;
-        ap_store<BK, true>(rk, ktok(i) < a.t_end, ku0, 0, smem + L::offK + (uint32_t)(2 * s) * L::kKh,
-                           smem + L::offK + (uint32_t)(2 * s + 1) * L::kKh, krow, 64);
-        ap_publish(lead(s ? P_KFULL1 : P_KFULL0));
-        if (i + 1 < ntiles) {
-            ap_load<BK>(a.k, h, ktok(i + 1), ktok(i + 1) < a.t_end, jk, ku0, rk);
-            jk = (i + 2 < ntiles) ? ap_index(a.k, h, ktok(i + 2), ktok(i + 2) < a.t_end) : 0;
-        }
-        if (i >= 2 && !__all_sync(0xffffffffu, ap_wait(bar(s ? P_VFREE1 : P_VFREE0), par, abort_flag)))
-            return;
-        ap_store<BV, false>(rv, vtok(i) < a.t_end, vu0, 8 * (int)rank, smem + L::offV + (uint32_t)s * L::kV,
-                            nullptr, vrow, 128);
-        ap_publish(lead(s ? P_VFULL1 : P_VFULL0));
+    // prologue: tiles 0 and 1
+    {
+        const int jk0 = kidx(0), jv0 = vidx(0), jk1 = kidx(1), jv1 = vidx(1);
+        stage_k(0, jk0);
+        cp_async_commit();
+        stage_v(0, jv0);
+        cp_async_commit();
+        if (ntiles > 1)
+            stage_k(1, jk1);
+        cp_async_commit();
+        if (ntiles > 1)
+            stage_v(1, jv1);
+        cp_async_commit();
     }
+    int jk = kidx(2), jv = vidx(2);
+    for (int i = 0; i < ntiles; ++i) {
+        const int s = i % kAPStages;
+        const int sp = (i + 2) % kAPStages;  // stage of tile i + 2 = stage of tile i - 1
+        const uint32_t par_prev = (uint32_t)(((i - 1) / kAPStages) & 1);
+        // (1) stage K(i + 2)
+        if (i + 2 < ntiles) {
+            if (i >= 1 && !__all_sync(0xffffffffu, ap_wait(bar(P_KFREE0 + sp), par_prev, abort_flag))) {
+                cp_async_wait<0>();
+                return;
+            }
+            stage_k(i + 2, jk);
+            jk = kidx(i + 3);
+        }
+        cp_async_commit();
+        // (2) rebuild K(i) (V(i)'s staged words are read first: K lo is
+        // overwritten below)
+        cp_async_wait<3>();
+        uint32_t kcw[4], vcw[4];
+        float2 ksz[4], vsz[4];
+        ap_read_stage<BK>(klo(s) + koff[0], klo(s) + koff[1], a.k.G, kcw, ksz);
+        ap_read_stage<BV>(klo(s) + koff[2], klo(s) + koff[3], a.v.G, vcw, vsz);
+        ap_rebuild<BK, true>(khi(s), klo(s), koff, kcw, ksz, ktok(i) < a.t_end);
+        ap_publish(lead(P_KFULL0 + s));
+        // (3) stage V(i + 2)
+        if (i + 2 < ntiles) {
+            if (i >= 1 && !__all_sync(0xffffffffu, ap_wait(bar(P_VFREE0 + sp), par_prev, abort_flag))) {
+                cp_async_wait<0>();
+                return;
+            }
+            stage_v(i + 2, jv);
+            jv = vidx(i + 3);
+        }
+        cp_async_commit();
+        // (4) rebuild V(i)
+        ap_rebuild<BV, false>(vst(s), nullptr, voff, vcw, vsz, vtok(i) < a.t_end);
+        ap_publish(lead(P_VFULL0 + s));
+    }
+    cp_async_wait<0>();
 }
 
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAPThreads, 1) attention_pair_kernel(AttnArgs a)
@@ -321,8 +393,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAPThreads, 1) atten
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + P_COUNT);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
     auto bar = [&](int i) { return smem_u32(bars + i); };
-    auto ksl = [&](int s, int part) { return smem + L::offK + (uint32_t)(2 * s + part) * L::kKh; };
-    auto vsl = [&](int s) { return smem + L::offV + (uint32_t)s * L::kV; };
+    auto ksl = [&](int st, int part) { return smem + L::offK + (uint32_t)(2 * st + part) * L::kKh; };
+    auto vsl = [&](int st) { return smem + L::offV + (uint32_t)st * L::kV; };
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const uint32_t rank = cluster_ctarank();
@@ -351,18 +423,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAPThreads, 1) atten
     if (tid == 0) {
         constexpr uint32_t kProdWarps = 2 * kAPProducers / 32;  // both CTAs
         mbar_init(bar(P_QREADY), kProdWarps);
-        mbar_init(bar(P_KFULL0), kProdWarps);
-        mbar_init(bar(P_KFULL1), kProdWarps);
-        mbar_init(bar(P_VFULL0), kProdWarps);
-        mbar_init(bar(P_VFULL1), kProdWarps);
+        for (int st = 0; st < kAPStages; ++st) {
+            mbar_init(bar(P_KFULL0 + st), kProdWarps);
+            mbar_init(bar(P_VFULL0 + st), kProdWarps);
+            mbar_init(bar(P_KFREE0 + st), 1);
+            mbar_init(bar(P_VFREE0 + st), 1);
+        }
         mbar_init(bar(P_SFULL0), 1);
         mbar_init(bar(P_SFULL1), 1);
         mbar_init(bar(P_PFULL0), 8);  // 4 softmax warps per CTA and query tile
         mbar_init(bar(P_PFULL1), 8);
-        mbar_init(bar(P_KFREE0), 1);
-        mbar_init(bar(P_KFREE1), 1);
-        mbar_init(bar(P_VFREE0), 1);
-        mbar_init(bar(P_VFREE1), 1);
         mbar_init(bar(P_OFULL), 1);
         *abort_flag = 0;
         fence_mbar_init();
@@ -409,7 +479,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAPThreads, 1) atten
             const uint32_t tS[2] = {tmem, tmem + 128}, tO[2] = {tmem + 256, tmem + 384};
             // S(j, qt) = Q_qt (K_j hi + K_j lo)^T into tS[qt]
             auto issue_s = [&](int j, int qt) {
-                const int ks_ = j & 1;
+                const int ks_ = j % kAPStages;
                 const uint32_t aK[2] = {smem_u32(ksl(ks_, 0)), smem_u32(ksl(ks_, 1))};
 #pragma unroll
                 for (int part = 0; part < 2; ++part) {
@@ -423,7 +493,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAPThreads, 1) atten
                 }
                 umma2_commit_both(bar(qt ? P_SFULL1 : P_SFULL0));
                 if (qt == 1)
-                    umma2_commit_both(bar(ks_ ? P_KFREE1 : P_KFREE0));
+                    umma2_commit_both(bar(P_KFREE0 + ks_));
             };
             bool ok = ap_wait(bar(P_QREADY), 0, abort_flag) && ap_wait(bar(P_KFULL0), 0, abort_flag);
             if (ok) {
@@ -432,8 +502,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAPThreads, 1) atten
                 issue_s(0, 1);
             }
             for (int j = 0; ok && j < ntiles; ++j) {
-                const int s = j & 1;
-                ok = ap_wait(bar(s ? P_VFULL1 : P_VFULL0), (uint32_t)((j >> 1) & 1), abort_flag);
+                const int s = j % kAPStages;
+                ok = ap_wait(bar(P_VFULL0 + s), (uint32_t)((j / kAPStages) & 1), abort_flag);
                 const uint32_t aV = smem_u32(vsl(s));
                 for (int qt = 0; ok && qt < 2; ++qt) {
                     ok = ap_wait(bar(qt ? P_PFULL1 : P_PFULL0), (uint32_t)(j & 1), abort_flag);
@@ -445,11 +515,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAPThreads, 1) atten
                         umma2_ts(tO[qt], tS[qt] + (uint32_t)ks * 8u, sdesc_sw128(aV + (uint32_t)ks * 2048u, 16384, 1024),
                                  idescO, (j > 0 || ks > 0) ? 1u : 0u);
                     if (qt == 1)
-                        umma2_commit_both(bar(s ? P_VFREE1 : P_VFREE0));
+                        umma2_commit_both(bar(P_VFREE0 + s));
                     if (j + 1 < ntiles) {
                         if (qt == 0) {
-                            const int s1 = (j + 1) & 1;
-                            ok = ap_wait(bar(s1 ? P_KFULL1 : P_KFULL0), (uint32_t)(((j + 1) >> 1) & 1), abort_flag);
+                            const int s1 = (j + 1) % kAPStages;
+                            ok = ap_wait(bar(P_KFULL0 + s1), (uint32_t)(((j + 1) / kAPStages) & 1), abort_flag);
                             if (!ok)
                                 break;
                             tc_fence_after();

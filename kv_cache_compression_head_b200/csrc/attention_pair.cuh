@@ -275,11 +275,10 @@ __device__ __forceinline__ void ap_publish(uint32_t lead_bar)
         mbar_arrive_cluster(lead_bar);
 }
 
-// Producer loop over tiles i: stage K(i + 2) once the QK of tile i - 1 has
-// freed its stage, rebuild K(i), stage V(i + 2) once the P V of tile i - 1
-// has freed its stage, rebuild V(i).  One commit group per staging step
-// (empty past the end), so "all but the newest three groups" is always the
-// pair K(i), V(i).
+// Producer loop over tiles i: rebuild K(i) and V(i), then stage K(i + 2)
+// once the QK of tile i - 1 has freed its stage and V(i + 2) once its P V
+// has.  One commit group per staging step (empty past the end), so "all but
+// the newest two groups" is always the pair K(i), V(i).
 template <int BK, int BV>
 __device__ __forceinline__ void ap_produce(const AttnArgs &a, int h, uint32_t rank, int tid, int ntiles,
                                            uint8_t *smem, uint64_t *bars, volatile int *abort_flag)
@@ -345,9 +344,23 @@ __device__ __forceinline__ void ap_produce(const AttnArgs &a, int h, uint32_t ra
     int jk = kidx(2), jv = vidx(2);
     for (int i = 0; i < ntiles; ++i) {
         const int s = i % kAPStages;
-        const int sp = (i + 2) % kAPStages;  // stage of tile i + 2 = stage of tile i - 1
+        // (1) rebuild K(i) and V(i) from their staged data (all but the newest
+        // two commit groups); V's staged words are read first: K lo is
+        // overwritten by the K rebuild
+        cp_async_wait<2>();
+        uint32_t kcw[4], vcw[4];
+        float2 ksz[4], vsz[4];
+        ap_read_stage<BK>(klo(s) + koff[0], klo(s) + koff[1], a.k.G, kcw, ksz);
+        ap_read_stage<BV>(klo(s) + koff[2], klo(s) + koff[3], a.v.G, vcw, vsz);
+        ap_rebuild<BK, true>(khi(s), klo(s), koff, kcw, ksz, ktok(i) < a.t_end);
+        ap_publish(lead(P_KFULL0 + s));
+        ap_rebuild<BV, false>(vst(s), nullptr, voff, vcw, vsz, vtok(i) < a.t_end);
+        ap_publish(lead(P_VFULL0 + s));
+        // (2) stage tile i + 2 into the stage of tile i - 1 once its QK (K) and
+        // its P V (V) are done.  Issued after the publications above, whose
+        // proxy fences then need not wait for these copies.
+        const int sp = (i + 2) % kAPStages;
         const uint32_t par_prev = (uint32_t)(((i - 1) / kAPStages) & 1);
-        // (1) stage K(i + 2)
         if (i + 2 < ntiles) {
             if (i >= 1 && !__all_sync(0xffffffffu, ap_wait(bar(P_KFREE0 + sp), par_prev, abort_flag))) {
                 cp_async_wait<0>();
@@ -357,16 +370,6 @@ __device__ __forceinline__ void ap_produce(const AttnArgs &a, int h, uint32_t ra
             jk = kidx(i + 3);
         }
         cp_async_commit();
-        // (2) rebuild K(i) (V(i)'s staged words are read first: K lo is
-        // overwritten below)
-        cp_async_wait<3>();
-        uint32_t kcw[4], vcw[4];
-        float2 ksz[4], vsz[4];
-        ap_read_stage<BK>(klo(s) + koff[0], klo(s) + koff[1], a.k.G, kcw, ksz);
-        ap_read_stage<BV>(klo(s) + koff[2], klo(s) + koff[3], a.v.G, vcw, vsz);
-        ap_rebuild<BK, true>(khi(s), klo(s), koff, kcw, ksz, ktok(i) < a.t_end);
-        ap_publish(lead(P_KFULL0 + s));
-        // (3) stage V(i + 2)
         if (i + 2 < ntiles) {
             if (i >= 1 && !__all_sync(0xffffffffu, ap_wait(bar(P_VFREE0 + sp), par_prev, abort_flag))) {
                 cp_async_wait<0>();
@@ -376,9 +379,6 @@ __device__ __forceinline__ void ap_produce(const AttnArgs &a, int h, uint32_t ra
             jv = vidx(i + 3);
         }
         cp_async_commit();
-        // (4) rebuild V(i)
-        ap_rebuild<BV, false>(vst(s), nullptr, voff, vcw, vsz, vtok(i) < a.t_end);
-        ap_publish(lead(P_VFULL0 + s));
     }
     cp_async_wait<0>();
 }

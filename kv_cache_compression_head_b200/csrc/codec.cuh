@@ -349,16 +349,19 @@ struct FitArgs {
 // sequentially in token order in binary64.  That sum is exact -- and then
 // equal to the sum in any order -- whenever every value is a multiple of 2^L
 // and every partial sum stays below 2^(53 + L) in magnitude: all partial sums
-// are then integers times 2^L representable in 53 bits.  So:
+// are then integers times 2^L representable in 53 bits.  With A the largest
+// |x| of the head and n the centre's token count, n A <= 2^(52 + L) suffices;
+// L is bounded below by the exponent of the smallest nonzero |x| of the head
+// less 134 (bf16 values: 8 significant bits) or 150 (binary32).  So:
 //   fit_hist:    per (head, token chunk) centre counts            [H][C][nch]
 //   fit_scan:    per head, bucket starts and per-chunk bases       [H][C+1], [H][C][nch]
 //   fit_scatter: per (head, chunk), stable placement of token ids  order[H][T]
 //   fit_segsum:  one warp per 64 consecutive slots of the sorted order: per
-//                run of one centre, binary64 sums per channel, a bound Q on
-//                every channel's sum of |x| and the smallest exponent L of
-//                any value's last significand bit; added to the centre's
-//                totals with atomics (exact sums are order independent)
-//   fit_finalize: one warp per (head, centre): if Q <= 2^(52 + L) the sums
+//                run of one centre, binary64 sums per channel, added to the
+//                centre's totals with atomics (exact sums are order
+//                independent); in the first round also the head's largest
+//                and smallest nonzero |x|
+//   fit_finalize: one warp per (head, centre): if n A <= 2^(52 + L) the sums
 //                are exact: mean in binary64, binary32, then bf16 (empty:
 //                keep); otherwise the centre is marked for
 //   fit_bucket_update: the sequential token-order sum (marked centres only).
@@ -380,18 +383,11 @@ struct FitSortArgs {
     int *bucket_start;       // [H][C + 1]
     int *order;              // [H][T]
     double *sums;            // [H][C][D]
-    double *qsum;            // [H][C]
-    int *lmin;               // [H][C]
+    unsigned *abs_max;       // [H] bits of the largest |x|
+    unsigned *abs_min;       // [H] bits of the smallest nonzero |x| (+inf: none)
     int *redo;               // [H][C]
+    int track;               // segsum also updates abs_max / abs_min
 };
-
-// Exponent of the last significand bit of a nonzero binary32 value.
-__device__ __forceinline__ int lsb_exponent(float v)
-{
-    const uint32_t b = __float_as_uint(v);
-    const uint32_t e = (b >> 23) & 0xffu, m = b & 0x7fffffu;
-    return e == 0u ? -149 + (__ffs((int)m) - 1) : (int)e - 150 + (__ffs((int)(m | 0x800000u)) - 1);
-}
 
 // mu_j = bf16(x_j) for the first C tokens; the update totals start cleared.
 __global__ void __launch_bounds__(256) fit_seed_kernel(FitArgs a, FitSortArgs fs)
@@ -410,10 +406,11 @@ __global__ void __launch_bounds__(256) fit_seed_kernel(FitArgs a, FitSortArgs fs
     const __nv_bfloat16 b = __float2bfloat16_rn(v);
     a.cent[gid] = *reinterpret_cast<const uint16_t *>(&b);
     fs.sums[gid] = 0.0;
-    if (c == 0) {
-        fs.qsum[hj] = 0.0;
-        fs.lmin[hj] = INT_MAX;
+    if (c == 0)
         fs.redo[hj] = 0;
+    if (c == 0 && j == 0) {
+        fs.abs_max[h] = 0u;
+        fs.abs_min[h] = 0x7f800000u;
     }
 }
 
@@ -576,32 +573,19 @@ __global__ void __launch_bounds__(256) fit_segsum_kernel(FitSortArgs a)
     const int *ord = a.order + (int64_t)h * a.T;
     const uint16_t *idx = a.idx + (int64_t)h * a.T;
 
-    double acc[kPer], q = 0.0;
-    int lm = INT_MAX, cur = -1;
+    double acc[kPer];
+    unsigned amax = 0u, amin = 0x7f800000u;
+    int cur = -1;
 #pragma unroll
     for (int k = 0; k < kPer; ++k)
         acc[k] = 0.0;
     auto flush = [&]() {
-        double* dst = a.sums + ((int64_t)h * a.C + cur) * D + lane * kPer;
+        double *dst = a.sums + ((int64_t)h * a.C + cur) * D + lane * kPer;
 #pragma unroll
-        for (int k = 0; k < kPer; ++k)
+        for (int k = 0; k < kPer; ++k) {
             atomicAdd(dst + k, acc[k]);
-        // Q: every channel's sum of |x| is at most its lane's q, so at most
-        // the largest q; L: the smallest last-bit exponent
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) {
-            q = fmax(q, __shfl_xor_sync(0xffffffffu, q, o));
-            lm = min(lm, __shfl_xor_sync(0xffffffffu, lm, o));
-        }
-        if (lane == 0) {
-            atomicAdd(a.qsum + (int64_t)h * a.C + cur, q);
-            atomicMin(a.lmin + (int64_t)h * a.C + cur, lm);
-        }
-#pragma unroll
-        for (int k = 0; k < kPer; ++k)
             acc[k] = 0.0;
-        q = 0.0;
-        lm = INT_MAX;
+        }
     };
     for (int64_t ib = i0; ib < i1; ib += 32) {
         const int nb = (int)min((int64_t)32, i1 - ib);
@@ -631,21 +615,31 @@ __global__ void __launch_bounds__(256) fit_segsum_kernel(FitSortArgs a)
                         flush();
                     cur = jj[b];
                 }
-                float mx = 0.0f;
 #pragma unroll
                 for (int k = 0; k < kPer; ++k) {
-                    const float x = v[b][k];
-                    acc[k] = __dadd_rn(acc[k], (double)x);
-                    mx = fmaxf(mx, fabsf(x));
-                    if (x != 0.0f)
-                        lm = min(lm, lsb_exponent(x));
+                    acc[k] = __dadd_rn(acc[k], (double)v[b][k]);
+                    if (a.track) {
+                        const unsigned u = __float_as_uint(v[b][k]) & 0x7fffffffu;
+                        amax = max(amax, u);
+                        amin = min(amin, u ? u : 0x7f800000u);
+                    }
                 }
-                q = __dadd_ru(q, (double)mx);
             }
         }
     }
     if (cur >= 0)
         flush();
+    if (a.track) {
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            amax = max(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+            amin = min(amin, __shfl_xor_sync(0xffffffffu, amin, o));
+        }
+        if (lane == 0) {
+            atomicMax(a.abs_max + h, amax);
+            atomicMin(a.abs_min + h, amin);
+        }
+    }
 }
 
 // One warp per (head, centre): exact totals -> new centre; otherwise mark the
@@ -661,10 +655,11 @@ __global__ void __launch_bounds__(256) fit_finalize_kernel(FitSortArgs a)
     const int64_t hj = (int64_t)h * a.C + j;
     const int *bs = a.bucket_start + (int64_t)h * (a.C + 1);
     const int n = bs[j + 1] - bs[j];
-    const double q = a.qsum[hj];
-    const int L = a.lmin[hj];
     // every partial sum is a multiple of 2^L below 2^(53 + L) in magnitude
-    const bool exact = L == INT_MAX || q <= ldexp(1.0, 52 + L);
+    const unsigned amin = a.abs_min[h];
+    const int L = (int)(amin >> 23) - (a.x_bf16 ? 134 : 150);
+    const bool exact =
+        amin >= 0x7f800000u || (double)n * (double)__uint_as_float(a.abs_max[h]) <= ldexp(1.0, 52 + L);
     double *sum = a.sums + hj * D + lane * kPer;
     if (n > 0 && exact) {
         uint16_t *dst = a.cent + hj * D + lane * kPer;
@@ -677,11 +672,8 @@ __global__ void __launch_bounds__(256) fit_finalize_kernel(FitSortArgs a)
 #pragma unroll
     for (int k = 0; k < kPer; ++k)
         sum[k] = 0.0;
-    if (lane == 0) {
+    if (lane == 0)
         a.redo[hj] = (n > 0 && !exact) ? 1 : 0;
-        a.qsum[hj] = 0.0;
-        a.lmin[hj] = INT_MAX;
-    }
 }
 
 // One warp per (head, centre) marked by fit_finalize; lane l owns channels

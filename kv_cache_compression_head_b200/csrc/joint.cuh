@@ -384,35 +384,41 @@ __global__ void __launch_bounds__(kJDThreads, 1)
         const int64_t t = t0 + row;
         const bool valid = t < a.T;
         const uint32_t lane_off = ((uint32_t)(warp & 3) * 32u) << 16;
+        // the centre row of the next head is fetched before its MMAs are awaited
+        auto centre_row = [&](int h, uint4 *mw) {
+            if (!valid || h >= a.H)
+                return;
+            int j = __ldg(a.idx + (int64_t)h * a.T + t);
+            if (j >= a.C) {
+                raise_status(DEVSTAT_BAD_INDEX);
+                j = 0;
+            }
+            const uint4 *mu = reinterpret_cast<const uint4 *>(a.cent + ((int64_t)h * a.C + j) * a.D);
+#pragma unroll
+            for (int u = 0; u < 16; ++u)
+                if (u < a.D / 8)
+                    mw[u] = __ldg(mu + u);
+        };
+        uint4 mw[16];
+        centre_row(g, mw);
         for (int h = g; h < a.H; h += 2) {
             const int b = h & 3;
-            int j = 0;
-            if (valid) {
-                j = __ldg(a.idx + (int64_t)h * a.T + t);
-                if (j >= a.C) {
-                    raise_status(DEVSTAT_BAD_INDEX);
-                    j = 0;
-                }
-            }
-            const uint16_t *mu = a.cent + ((int64_t)h * a.C + j) * a.D;
             ok = __all_sync(0xffffffffu, ok && mbar_wait(bar(JD_DONE0 + b), (uint32_t)((h >> 2) & 1)));
             if (!ok)
                 break;
             tc_fence_after();
-            for (int cb = 0; cb < a.D / 32; ++cb) {
-                uint4 mw[4];
-                if (valid) {
 #pragma unroll
-                    for (int u = 0; u < 4; ++u)
-                        mw[u] = __ldg(reinterpret_cast<const uint4 *>(mu + cb * 32) + u);
-                }
+            for (int cb = 0; cb < 4; ++cb) {
+                if (cb >= a.D / 32)
+                    break;
                 float v[32];
                 tmem_ld32(tmem + lane_off + (uint32_t)(b * a.D + cb * 32), v);
                 if (!valid)
                     continue;
 #pragma unroll
                 for (int u = 0; u < 4; ++u) {
-                    const uint32_t m[4] = {mw[u].x, mw[u].y, mw[u].z, mw[u].w};
+                    const uint4 m4 = mw[cb * 4 + u];
+                    const uint32_t m[4] = {m4.x, m4.y, m4.z, m4.w};
 #pragma unroll
                     for (int k = 0; k < 4; ++k) {
                         v[u * 8 + 2 * k] = __fadd_rn(bf16_lo(m[k]), v[u * 8 + 2 * k]);
@@ -434,6 +440,7 @@ __global__ void __launch_bounds__(kJDThreads, 1)
                         dst[u] = make_float4(v[4 * u], v[4 * u + 1], v[4 * u + 2], v[4 * u + 3]);
                 }
             }
+            centre_row(h + 2, mw);
             tc_fence_before();
             __syncwarp();
             if (lane == 0)

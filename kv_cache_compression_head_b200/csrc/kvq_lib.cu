@@ -357,7 +357,7 @@ kvq_status joint_encode_call(const kvq_codec_desc *desc, const void *x, kvq_dtyp
 // Fit workspace: idx [H][T] u16 | per-chunk centre counts [H][nch][C] i32 |
 // bucket starts [H][C+1] i32 | token order [H][T] i32.
 struct FitLayout {
-    size_t idx, counts, starts, order, sums, qsum, lmin, redo, total;
+    size_t idx, counts, starts, order, sums, bounds, redo, total;
     int nchunks;
 };
 
@@ -373,9 +373,8 @@ FitLayout fit_layout(const kvq_codec_desc *d, int64_t T)
     L.starts = L.counts + round_up(H * (size_t)L.nchunks * C * 4, 256);
     L.order = L.starts + round_up(H * (C + 1) * 4, 256);
     L.sums = L.order + round_up(H * (size_t)T * 4, 256);
-    L.qsum = L.sums + round_up(H * C * (size_t)d->head_dim * 8, 256);
-    L.lmin = L.qsum + round_up(H * C * 8, 256);
-    L.redo = L.lmin + round_up(H * C * 4, 256);
+    L.bounds = L.sums + round_up(H * C * (size_t)d->head_dim * 8, 256);
+    L.redo = L.bounds + round_up(H * 8, 256);
     L.total = L.redo + H * C * 4;
     return L;
 }
@@ -599,8 +598,9 @@ kvq_status kvq_fit_centroids(const kvq_codec_desc *desc, const void *x, kvq_dtyp
     fs.bucket_start = reinterpret_cast<int *>(ws + Lw.starts);
     fs.order = reinterpret_cast<int *>(ws + Lw.order);
     fs.sums = reinterpret_cast<double *>(ws + Lw.sums);
-    fs.qsum = reinterpret_cast<double *>(ws + Lw.qsum);
-    fs.lmin = reinterpret_cast<int *>(ws + Lw.lmin);
+    fs.abs_max = reinterpret_cast<unsigned *>(ws + Lw.bounds);
+    fs.abs_min = fs.abs_max + H;
+    fs.track = 1;
     fs.redo = reinterpret_cast<int *>(ws + Lw.redo);
 
     const int64_t n_cent = (int64_t)H * C * D;
@@ -633,6 +633,7 @@ kvq_status kvq_fit_centroids(const kvq_codec_desc *desc, const void *x, kvq_dtyp
         const int64_t warps = (int64_t)H * C;
         const unsigned seg_blocks = (unsigned)ceil_div((int64_t)H * ceil_div(T, kFitSegSlots) * 32, 256);
         const unsigned cent_blocks = (unsigned)ceil_div(warps * 32, 256);
+        fs.track = it == 0 ? 1 : 0;  // the head bounds need one pass over x
         if (D == 128) {
             fit_segsum_kernel<128><<<seg_blocks, 256, 0, s>>>(fs);
             fit_finalize_kernel<128><<<cent_blocks, 256, 0, s>>>(fs);

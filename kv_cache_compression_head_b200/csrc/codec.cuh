@@ -287,17 +287,19 @@ struct DecodeArgs {
     int out_bf16;
 };
 
+// One block per (tile of 256 / (D/8) tokens, head); thread = 8 channels of
+// one token: the encoded rows of the head are read contiguously and every
+// token-head's output row is one contiguous run of D values.
+template <int D>
 __global__ void __launch_bounds__(256) decode_kernel(DecodeArgs a)
 {
-    const int units = a.D / 8;
-    const int64_t gid = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-    const int64_t total = a.T * a.H * units;
-    if (gid >= total)
+    constexpr int kUnits = D / 8;
+    constexpr int kTokens = 256 / kUnits;
+    const int u = threadIdx.x % kUnits;
+    const int64_t t = (int64_t)blockIdx.x * kTokens + threadIdx.x / kUnits;
+    const int h = blockIdx.y;
+    if (t >= a.T)
         return;
-    const int u = (int)(gid % units);
-    const int64_t th_out = gid / units;       // t * H + h
-    const int h = (int)(th_out % a.H);
-    const int64_t t = th_out / a.H;
     const int64_t th = (int64_t)h * a.T + t;  // encoded-row index
     int j = a.idx[th];
     if (j >= a.C) {
@@ -305,21 +307,20 @@ __global__ void __launch_bounds__(256) decode_kernel(DecodeArgs a)
         j = 0;
     }
     const int c0 = u * 8;
-    const int g = c0 / a.G;
-    const float2 sz = reinterpret_cast<const float2 *>(a.meta)[th * (a.D / a.G) + g];
+    const float2 sz = reinterpret_cast<const float2 *>(a.meta)[th * (D / a.G) + c0 / a.G];
     uint32_t cw;
     if (a.bits == 2)
-        cw = *reinterpret_cast<const uint16_t *>(a.codes + th * (a.D / 4) + c0 / 4);
+        cw = *reinterpret_cast<const uint16_t *>(a.codes + th * (D / 4) + c0 / 4);
     else
-        cw = *reinterpret_cast<const uint32_t *>(a.codes + th * (a.D / 2) + c0 / 2);
+        cw = *reinterpret_cast<const uint32_t *>(a.codes + th * (D / 2) + c0 / 2);
     float mu[8];
-    load_bf16x8(a.cent + ((int64_t)h * a.C + j) * a.D + c0, mu);
+    load_bf16x8(a.cent + ((int64_t)h * a.C + j) * D + c0, mu);
     const uint32_t mask = (1u << a.bits) - 1u;
     float v[8];
 #pragma unroll
     for (int k = 0; k < 8; ++k)
         v[k] = dequant_spec((cw >> (k * a.bits)) & mask, sz.x, sz.y, mu[k]);
-    const int64_t o = th_out * a.D + c0;
+    const int64_t o = (t * a.H + h) * D + c0;
     if (a.out_bf16) {
         uint4 w = make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]), pack_bf16x2(v[4], v[5]),
                              pack_bf16x2(v[6], v[7]));

@@ -459,6 +459,14 @@ int attention_splits(int64_t Tq, int H, int64_t span, size_t ws_bytes, size_t ws
     return best;
 }
 
+void launch_merge(const MergeArgs &m, cudaStream_t s)
+{
+    if (m.D == 128)
+        lse_merge_kernel<128><<<dim3((unsigned)ceil_div(m.Tq, 256 / 32), (unsigned)m.H), 256, 0, s>>>(m);
+    else
+        lse_merge_kernel<64><<<dim3((unsigned)ceil_div(m.Tq, 256 / 16), (unsigned)m.H), 256, 0, s>>>(m);
+}
+
 kvq_status launch_attention_pair(const AttnArgs &a, cudaStream_t s)
 {
     static bool configured[64] = {};
@@ -811,8 +819,11 @@ kvq_status kvq_decode(const kvq_compressed_view *view, void *x_out, kvq_dtype ou
     a.G = view->desc.group_size;
     a.out = x_out;
     a.out_bf16 = out_dtype == KVQ_BF16;
-    const int64_t n = a.T * a.H * (a.D / 8);
-    decode_kernel<<<(unsigned)ceil_div(n, 256), 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(a);
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (a.D == 128)
+        decode_kernel<128><<<dim3((unsigned)ceil_div(a.T, 256 / 16), (unsigned)a.H), 256, 0, s>>>(a);
+    else
+        decode_kernel<64><<<dim3((unsigned)ceil_div(a.T, 256 / 8), (unsigned)a.H), 256, 0, s>>>(a);
     return launch_status();
 }
 
@@ -893,8 +904,7 @@ kvq_status kvq_attention_lse(const void *q, int64_t Tq, const kvq_compressed_vie
     m.o_out = o_out;
     m.o_bf16 = a.o_bf16;
     m.lse_out = lse_out;
-    const int64_t n = Tq * a.H * (D / 4);
-    lse_merge_kernel<<<(unsigned)ceil_div(n, 256), 256, 0, s>>>(m);
+    launch_merge(m, s);
     return launch_status();
 }
 
@@ -930,8 +940,7 @@ kvq_status kvq_lse_merge(int32_t n_parts, const float *const *o_parts, const flo
     a.o_out = o_out;
     a.o_bf16 = o_dtype == KVQ_BF16;
     a.lse_out = lse_out;
-    const int64_t n = Tq * H * (d / 4);
-    lse_merge_kernel<<<(unsigned)ceil_div(n, 256), 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(a);
+    launch_merge(a, reinterpret_cast<cudaStream_t>(stream));
     return launch_status();
 }
 

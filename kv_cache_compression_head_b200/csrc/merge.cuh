@@ -24,20 +24,21 @@ struct MergeArgs {
     float *lse_out;
 };
 
-// One thread per 4 channels of a (query, head) row.  Every thread of a row
-// recomputes the row's weights (n exps), which keeps the kernel a single
-// pass over the o_b reads and the output write.
+// One block per (tile of 256 / (D/4) queries, head); thread = 4 channels of
+// one (query, head) row.  Every thread of a row recomputes the row's weights
+// (n exps), which keeps the kernel a single pass over the o_b reads and the
+// output write.
+template <int D>
 __global__ void __launch_bounds__(256) lse_merge_kernel(MergeArgs a)
 {
-    const int units = a.D / 4;
-    const int64_t gid = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-    const int64_t total = a.Tq * a.H * units;
-    if (gid >= total)
+    constexpr int kUnits = D / 4;
+    constexpr int kRows = 256 / kUnits;
+    const int u = threadIdx.x % kUnits;
+    const int64_t t = (int64_t)blockIdx.x * kRows + threadIdx.x / kUnits;
+    const int h = blockIdx.y;
+    if (t >= a.Tq)
         return;
-    const int u = (int)(gid % units);
-    const int64_t row = gid / units;  // t * H + h
-    const int h = (int)(row % a.H);
-    const int64_t t = row / a.H;
+    const int64_t row = t * a.H + h;
     const int64_t li = (int64_t)h * a.Tq + t;
 
     float m = -INFINITY;
@@ -58,7 +59,7 @@ __global__ void __launch_bounds__(256) lse_merge_kernel(MergeArgs a)
             if (l == -INFINITY)
                 continue;
             const float w = expf(l - lse);
-            const float4 v = *reinterpret_cast<const float4 *>(a.o[b] + row * a.D + u * 4);
+            const float4 v = *reinterpret_cast<const float4 *>(a.o[b] + row * D + u * 4);
             acc.x = fmaf(w, v.x, acc.x);
             acc.y = fmaf(w, v.y, acc.y);
             acc.z = fmaf(w, v.z, acc.z);
@@ -67,9 +68,9 @@ __global__ void __launch_bounds__(256) lse_merge_kernel(MergeArgs a)
     }
     if (a.o_bf16) {
         uint2 w = make_uint2(pack_bf16x2(acc.x, acc.y), pack_bf16x2(acc.z, acc.w));
-        *reinterpret_cast<uint2 *>(static_cast<uint16_t *>(a.o_out) + row * a.D + u * 4) = w;
+        *reinterpret_cast<uint2 *>(static_cast<uint16_t *>(a.o_out) + row * D + u * 4) = w;
     } else {
-        *reinterpret_cast<float4 *>(static_cast<float *>(a.o_out) + row * a.D + u * 4) = acc;
+        *reinterpret_cast<float4 *>(static_cast<float *>(a.o_out) + row * D + u * 4) = acc;
     }
     if (u == 0)
         a.lse_out[li] = lse;

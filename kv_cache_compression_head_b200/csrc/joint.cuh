@@ -26,7 +26,8 @@
 namespace kvq {
 
 constexpr int kJRows = 128;      // tokens per CTA
-constexpr int kJThreads = 128;   // one thread per token row (TMEM lane)
+constexpr int kJThreads = 128;   // decoder helpers: one thread per token row (TMEM lane)
+constexpr int kJEThreads = 256;  // encoder: two threads per token row
 constexpr int kJKBlock = 64;     // channels per K-block
 
 struct JointEncArgs {
@@ -53,16 +54,17 @@ __host__ __device__ constexpr uint32_t pow2_cols(int n)
     return c;
 }
 
-// Quantise one row's r coefficients held in TMEM (columns [0, r) of this
-// thread's lane) with Eq. 1 per group of G, and store codes / {s, z}
-// (and the binary32 coefficients themselves when coef_row is set).
+// Quantise groups g0, g0 + gstep, ... of one row's r coefficients held in
+// TMEM (columns [0, r) of this thread's lane) with Eq. 1 per group of G, and
+// store codes / {s, z} (and the binary32 coefficients themselves when
+// coef_row is set).
 template <int G, int BITS>
 __device__ __forceinline__ void joint_quant_row(uint32_t trow, int r, uint8_t *codes_row, float2 *meta_row,
-                                                float *coef_row)
+                                                float *coef_row, int g0, int gstep)
 {
     static_assert(G % 16 == 0 && G <= 64, "group of 16, 32 or 64 coefficients");
     constexpr int kWords = G * BITS / 32;
-    for (int g = 0; g < r / G; ++g) {
+    for (int g = g0; g < r / G; g += gstep) {
         float v[G];
 #pragma unroll
         for (int c = 0; c < G; c += 16) {
@@ -106,10 +108,12 @@ __device__ __forceinline__ void joint_quant_row(uint32_t trow, int r, uint8_t *c
     }
 }
 
-// One CTA per 128-token tile.  All 128 threads build the A stage (each thread
-// one token row, 64 channels) and copy the B stage; thread 0 issues the MMAs.
+// One CTA per 128-token tile.  All 256 threads build the A stage (two threads
+// per token row, 32 channels each) and copy the B stage; thread 0 issues the
+// MMAs; in the epilogue the two threads of a row (warps w and w + 4 share the
+// TMEM lanes) quantise alternate groups.
 template <int G, int BITS>
-__global__ void __launch_bounds__(kJThreads, 1) joint_encode_kernel(JointEncArgs a)
+__global__ void __launch_bounds__(kJEThreads, 1) joint_encode_kernel(JointEncArgs a)
 {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -117,8 +121,9 @@ __global__ void __launch_bounds__(kJThreads, 1) joint_encode_kernel(JointEncArgs
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + 2 * stage_bytes);
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 3);
     const int tid = threadIdx.x, warp = tid >> 5;
+    const int row = tid & 127, half = tid >> 7;
     const int64_t t0 = (int64_t)blockIdx.x * kJRows;
-    const int64_t t = t0 + tid;
+    const int64_t t = t0 + row;
     const bool valid = t < a.T;
     const uint32_t ncols = pow2_cols(a.r);
 
@@ -158,7 +163,7 @@ __global__ void __launch_bounds__(kJThreads, 1) joint_encode_kernel(JointEncArgs
             }
         }
 #pragma unroll
-        for (int u = 0; u < kJKBlock / 8; ++u) {
+        for (int u = half * (kJKBlock / 16); u < (half + 1) * (kJKBlock / 16); ++u) {
             uint4 w = make_uint4(0, 0, 0, 0);
             if (valid) {
                 float xv[8], mv[8];
@@ -169,10 +174,10 @@ __global__ void __launch_bounds__(kJThreads, 1) joint_encode_kernel(JointEncArgs
                                pack_bf16x2(__fsub_rn(xv[4], mv[4]), __fsub_rn(xv[5], mv[5])),
                                pack_bf16x2(__fsub_rn(xv[6], mv[6]), __fsub_rn(xv[7], mv[7])));
             }
-            *reinterpret_cast<uint4 *>(sA + sw128_unit_offset(tid, u, kJRows)) = w;
+            *reinterpret_cast<uint4 *>(sA + sw128_unit_offset(row, u, kJRows)) = w;
         }
         // B: W rows [i0, i0 + 64), all r columns -> MN-major [r/64][64][128 B]
-        for (int e = tid; e < kJKBlock * (a.r / 8); e += kJThreads) {
+        for (int e = tid; e < kJKBlock * (a.r / 8); e += kJEThreads) {
             const int k = e / (a.r / 8), u = e % (a.r / 8);
             const uint4 w = __ldg(reinterpret_cast<const uint4 *>(a.w + (int64_t)(i0 + k) * a.r) + u);
             *reinterpret_cast<uint4 *>(sB + sw128_unit_offset(k, u, kJKBlock)) = w;
@@ -199,13 +204,13 @@ __global__ void __launch_bounds__(kJThreads, 1) joint_encode_kernel(JointEncArgs
         ok = mbar_wait(smem_u32(bars + s_last), phase[s_last]) && ok;
     }
     tc_fence_after();
-    const uint32_t trow = tmem + (((uint32_t)warp * 32u) << 16);
+    const uint32_t trow = tmem + (((uint32_t)(warp & 3) * 32u) << 16);
     ok = __all_sync(0xffffffffu, ok);  // tcgen05.ld below is warp-collective
     if (ok) {
         uint8_t *codes_row = (valid && a.codes) ? a.codes + t * (a.r * a.bits / 8) : nullptr;
         float2 *meta_row = (valid && a.meta) ? reinterpret_cast<float2 *>(a.meta) + t * (a.r / G) : nullptr;
         float *coef_row = (valid && a.coef_out) ? a.coef_out + t * a.r : nullptr;
-        joint_quant_row<G, BITS>(trow, a.r, codes_row, meta_row, coef_row);
+        joint_quant_row<G, BITS>(trow, a.r, codes_row, meta_row, coef_row, half, 2);
     }
     tc_fence_before();
     __syncthreads();

@@ -247,7 +247,7 @@ kvq_status launch_joint_encode_t(const JointEncArgs &a, cudaStream_t s)
             return KVQ_ERR_CUDA;
         configured[dev] = true;
     }
-    joint_encode_kernel<G, BITS><<<(unsigned)ceil_div(a.T, kJRows), kJThreads, smem, s>>>(a);
+    joint_encode_kernel<G, BITS><<<(unsigned)ceil_div(a.T, kJRows), kJEThreads, smem, s>>>(a);
     return launch_status();
 }
 

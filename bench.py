@@ -243,10 +243,10 @@ class Pipeline:
         self.enc_j = [K.alloc_encoded(c, T, device) for c in self.codec_j]
         self.comp_j = [K.Compressed(c, T, self.cent[i], *self.enc_j[i], w_dec=self.w_dec)
                        for i, c in enumerate(self.codec_j)]
-        # fit: seed + (assign + 3 sort + 3 update kernels) per round; encode 1;
+        # fit: seed + (assign + 4 sort + 3 update kernels) per round; encode 1;
         # decode 1; joint encode 2 (assign, projection), joint decode 1;
         # attention 2 per block (split + its merge); final merge 1 -- K and V
-        self.launches_per_step = (2 * (1 + 7 * w.kmeans_iters) + 2 + 2 + 2 * 2 + 2 + 2 * HISTORY_BLOCKS + 1)
+        self.launches_per_step = (2 * (1 + 8 * w.kmeans_iters) + 2 + 2 + 2 * 2 + 2 + 2 * HISTORY_BLOCKS + 1)
 
     def outputs(self):
         outs = [self.o, self.lse]

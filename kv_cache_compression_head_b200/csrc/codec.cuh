@@ -317,9 +317,20 @@ __global__ void __launch_bounds__(256) decode_kernel(DecodeArgs a)
     load_bf16x8(a.cent + ((int64_t)h * a.C + j) * D + c0, mu);
     const uint32_t mask = (1u << a.bits) - 1u;
     float v[8];
+    if (fabsf(sz.y) < 4194304.0f) {
+        // q - z = (2^23 + q) - (2^23 + z), both terms and the difference exact:
+        // the same value dequant_spec forms, without the int -> float convert
+        const float zz = __fadd_rn(8388608.0f, sz.y);
 #pragma unroll
-    for (int k = 0; k < 8; ++k)
-        v[k] = dequant_spec((cw >> (k * a.bits)) & mask, sz.x, sz.y, mu[k]);
+        for (int k = 0; k < 8; ++k) {
+            const float d = __fsub_rn(__uint_as_float(0x4B000000u | ((cw >> (k * a.bits)) & mask)), zz);
+            v[k] = __fadd_rn(mu[k], __fmul_rn(d, sz.x));
+        }
+    } else {
+#pragma unroll
+        for (int k = 0; k < 8; ++k)
+            v[k] = dequant_spec((cw >> (k * a.bits)) & mask, sz.x, sz.y, mu[k]);
+    }
     const int64_t o = (t * a.H + h) * D + c0;
     if (a.out_bf16) {
         uint4 w = make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]), pack_bf16x2(v[4], v[5]),
@@ -355,7 +366,8 @@ struct FitArgs {
 // L is bounded below by the exponent of the smallest nonzero |x| of the head
 // less 134 (bf16 values: 8 significant bits) or 150 (binary32).  So:
 //   fit_hist:    per (head, token chunk) centre counts            [H][C][nch]
-//   fit_scan:    per head, bucket starts and per-chunk bases       [H][C+1], [H][C][nch]
+//   fit_scan:    per (head, centre), per-chunk bases and totals    [H][C][nch], [H][C]
+//   fit_starts:  per head, bucket starts (prefix of the totals)    [H][C+1]
 //   fit_scatter: per (head, chunk), stable placement of token ids  order[H][T]
 //   fit_segsum:  one warp per 64 consecutive slots of the sorted order: per
 //                run of one centre, binary64 sums per channel, added to the
@@ -432,42 +444,48 @@ __global__ void __launch_bounds__(256) fit_hist_kernel(FitSortArgs a)
         dst[(int64_t)j * a.nchunks] = s_cnt[j];
 }
 
-// One block (1024 threads) per head.  Each warp turns the chunk counts of its
-// centres into chunk bases (prefix over chunks); then a block-wide exclusive
-// prefix over the centre totals gives the bucket starts.
-__global__ void __launch_bounds__(1024) fit_scan_kernel(FitSortArgs a)
+// One warp per (head, centre): the centre's chunk counts become chunk bases
+// (prefix over chunks) and its total goes to bucket_start[h][j] (turned into
+// bucket starts by fit_starts_kernel).
+__global__ void __launch_bounds__(256) fit_scan_kernel(FitSortArgs a)
 {
-    extern __shared__ int s_tot[];  // [C]
+    const int lane = threadIdx.x & 31;
+    const int j = blockIdx.x * 8 + (threadIdx.x >> 5), h = blockIdx.y;
+    if (j >= a.C)
+        return;
+    int *row = a.chunk_counts + ((int64_t)h * a.C + j) * a.nchunks;
+    int run = 0;
+    for (int c0 = 0; c0 < a.nchunks; c0 += 32) {
+        const int c = c0 + lane;
+        const int v = c < a.nchunks ? row[c] : 0;
+        int incl = v;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int n = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o)
+                incl += n;
+        }
+        if (c < a.nchunks)
+            row[c] = run + incl - v;
+        run += __shfl_sync(0xffffffffu, incl, 31);
+    }
+    if (lane == 0)
+        a.bucket_start[(int64_t)h * (a.C + 1) + j] = run;
+}
+
+// One block (1024 threads) per head: exclusive prefix of the centre totals
+// in bucket_start[h][0..C) in place, total in bucket_start[h][C].
+__global__ void __launch_bounds__(1024) fit_starts_kernel(FitSortArgs a)
+{
     __shared__ int s_warp[32];
     const int h = blockIdx.x, lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    int *cc = a.chunk_counts + (int64_t)h * a.C * a.nchunks;
-    for (int j = warp; j < a.C; j += 32) {
-        int *row = cc + (int64_t)j * a.nchunks;
-        int run = 0;
-        for (int c0 = 0; c0 < a.nchunks; c0 += 32) {
-            const int c = c0 + lane;
-            const int v = c < a.nchunks ? row[c] : 0;
-            int incl = v;
-#pragma unroll
-            for (int o = 1; o < 32; o <<= 1) {
-                const int n = __shfl_up_sync(0xffffffffu, incl, o);
-                if (lane >= o)
-                    incl += n;
-            }
-            if (c < a.nchunks)
-                row[c] = run + incl - v;
-            run += __shfl_sync(0xffffffffu, incl, 31);
-        }
-        if (lane == 0)
-            s_tot[j] = run;
-    }
-    __syncthreads();
-    // exclusive prefix of s_tot: thread k owns entries [k per, (k + 1) per)
+    int *bs = a.bucket_start + (int64_t)h * (a.C + 1);
+    // thread k owns entries [k per, (k + 1) per)
     const int per = (a.C + 1023) / 1024;
     const int j0 = threadIdx.x * per, j1 = min(a.C, j0 + per);
     int local = 0;
     for (int j = j0; j < j1; ++j)
-        local += s_tot[j];
+        local += bs[j];
     int incl = local;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
@@ -491,9 +509,8 @@ __global__ void __launch_bounds__(1024) fit_scan_kernel(FitSortArgs a)
     }
     __syncthreads();
     int run = s_warp[warp] + incl - local;
-    int *bs = a.bucket_start + (int64_t)h * (a.C + 1);
     for (int j = j0; j < j1; ++j) {
-        const int t = s_tot[j];
+        const int t = bs[j];
         bs[j] = run;
         run += t;
     }

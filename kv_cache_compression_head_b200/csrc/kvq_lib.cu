@@ -616,7 +616,7 @@ kvq_status kvq_fit_centroids(const kvq_codec_desc *desc, const void *x, kvq_dtyp
     if ((st = launch_status()) != KVQ_OK)
         return st;
     const size_t cbytes = (size_t)C * 4;
-    if ((st = smem_opt_in(fit_hist_kernel, cbytes)) != KVQ_OK || (st = smem_opt_in(fit_scan_kernel, cbytes)) != KVQ_OK ||
+    if ((st = smem_opt_in(fit_hist_kernel, cbytes)) != KVQ_OK ||
         (st = smem_opt_in(fit_scatter_kernel, cbytes)) != KVQ_OK)
         return st;
     EncodeArgs e;
@@ -636,7 +636,8 @@ kvq_status kvq_fit_centroids(const kvq_codec_desc *desc, const void *x, kvq_dtyp
         if ((st = launch_encode(D, e, s)) != KVQ_OK)
             return st;
         fit_hist_kernel<<<chunks, 256, cbytes, s>>>(fs);
-        fit_scan_kernel<<<(unsigned)H, 1024, cbytes, s>>>(fs);
+        fit_scan_kernel<<<dim3((unsigned)ceil_div(C, 8), (unsigned)H), 256, 0, s>>>(fs);
+        fit_starts_kernel<<<(unsigned)H, 1024, 0, s>>>(fs);
         fit_scatter_kernel<<<chunks, 32, cbytes, s>>>(fs);
         const int64_t warps = (int64_t)H * C;
         const unsigned seg_blocks = (unsigned)ceil_div((int64_t)H * ceil_div(T, kFitSegSlots) * 32, 256);

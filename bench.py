@@ -44,6 +44,10 @@ UNIT = "history-tokens/s"
 WORKLOAD = "wan13b"
 HISTORY_BLOCKS = 2
 FLUSH_BYTES = 256 << 20
+# DRAM bytes (read + write) of one attention_pair_kernel launch of this
+# workload, from the ncu capture summarised in profiles/attention_pair_wan13b.md;
+# None whenever the kernel has changed since that capture.
+ATTN_NCU_TRAFFIC_BYTES = 56_144_640 + 37_984_000
 
 
 def _joint():
@@ -424,7 +428,8 @@ def run_gpu(args):
             "roofline": {"kernel": "attention_pair_kernel (time of the whole kvq_attention_lse call, incl. its "
                                    "in-call LSE merge)", "bound": "tensor", "achieved": attn_tflops,
                          "peak": tfl, "unit": "TFLOP/s", "frac": attn_tflops / tfl, "peak_kind": peak_kind,
-                         "traffic": None},
+                         "traffic": ATTN_NCU_TRAFFIC_BYTES,
+                         "traffic_unit": "bytes per launch (ncu dram__bytes_read.sum + dram__bytes_write.sum)"},
             "rows": rows,
             "clocks": clk,
             "gpu_launches": pipe.launches_per_step * args.steps,

@@ -100,6 +100,21 @@ __device__ __forceinline__ uint32_t smem_u32(const void *p)
 
 // Make this thread's generic-proxy shared-memory writes visible to the async
 // proxy (tensor-core operand reads).
+// Three-input binary32 min / max (one instruction on sm_100).
+__device__ __forceinline__ float fmin3(float a, float b, float c)
+{
+    float r;
+    asm("min.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+    return r;
+}
+
+__device__ __forceinline__ float fmax3(float a, float b, float c)
+{
+    float r;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+    return r;
+}
+
 // Per-thread asynchronous global -> shared copies (completion tracked per
 // thread with commit / wait groups).
 __device__ __forceinline__ void cp_async16(uint32_t dst, const void *src)

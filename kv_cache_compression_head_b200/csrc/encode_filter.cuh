@@ -139,11 +139,11 @@ __device__ __forceinline__ void encode_residual_smem(const uint8_t *sX, const ui
                     r[uu * 8 + 2 * k + 1] = d.y;
                 }
             }
-            float mn = r[0], mx = r[0];
+            float mn = fminf(r[0], r[1]), mx = fmaxf(r[0], r[1]);
 #pragma unroll
-            for (int c = 1; c < G; ++c) {
-                mn = fminf(mn, r[c]);
-                mx = fmaxf(mx, r[c]);
+            for (int c = 2; c < G; c += 2) {
+                mn = fmin3(mn, r[c], r[c + 1]);
+                mx = fmax3(mx, r[c], r[c + 1]);
             }
             if (mn == 0.0f || mx == 0.0f) {
                 // a zero extreme: take its sign exactly as the ordered strict scan does
@@ -343,22 +343,40 @@ __global__ void __launch_bounds__(kFltThreads, 2)
             if (c < c_hi) {
                 float p[32];
                 tmem_ld32(tmem + lane_off + (uint32_t)(c * 32), p);
-                float m1 = INFINITY, m2 = INFINITY, m3 = INFINITY;
+                // two independent chains (pairs 4q and 4q + 2 / 4q + 1 and 4q + 3
+                // of the chunk) so consecutive updates do not wait on each other
+                float a1 = INFINITY, a2 = INFINITY, a3 = INFINITY;
+                float c1 = INFINITY, c2 = INFINITY, c3 = INFINITY;
                 const float4 *nrm4 = reinterpret_cast<const float4 *>(sNrm + c * 32);
+                auto pair_into = [](float pa, float pb, float &m1, float &m2, float &m3) {
+                    // sort the pair, then merge it into the three smallest
+                    // (k-th smallest of two sorted lists = min over i + j = k
+                    // of max(a_i, b_j))
+                    const float lo = fminf(pa, pb), hi = fmaxf(pa, pb);
+                    const float n3 = fmin3(m3, fmaxf(m2, lo), fmaxf(m1, hi));
+                    const float n2 = fmin3(fmaxf(m1, lo), m2, hi);
+                    m1 = fminf(m1, lo);
+                    m2 = n2;
+                    m3 = n3;
+                };
 #pragma unroll
                 for (int i4 = 0; i4 < 8; ++i4) {
                     const float4 n4 = nrm4[i4];
                     const float nn[4] = {n4.x, n4.y, n4.z, n4.w};
+                    float pk[4];
 #pragma unroll
                     for (int e = 0; e < 4; ++e) {
                         const int i = i4 * 4 + e;
                         const float v = fmaf(-2.0f, p[i], nn[e]);
-                        const float vp = __uint_as_float((__float_as_uint(v) & ~31u) | (uint32_t)i);
-                        m3 = fminf(m3, fmaxf(m2, vp));
-                        m2 = fminf(m2, fmaxf(m1, vp));
-                        m1 = fminf(m1, vp);
+                        pk[e] = __uint_as_float((__float_as_uint(v) & ~31u) | (uint32_t)i);
                     }
+                    pair_into(pk[0], pk[1], a1, a2, a3);
+                    pair_into(pk[2], pk[3], c1, c2, c3);
                 }
+                // merge the two chains' three smallest
+                const float m1 = fminf(a1, c1);
+                const float m2 = fmin3(a2, fmaxf(a1, c1), c2);
+                const float m3 = fminf(fmin3(a3, fmaxf(a2, c1), fmaxf(a1, c2)), c3);
                 top3_insert(m1, c, b1, k1, b2, k2, b3, k3);
                 top3_insert(m2, c, b1, k1, b2, k2, b3, k3);
                 top3_insert(m3, c, b1, k1, b2, k2, b3, k3);

@@ -605,23 +605,27 @@ __global__ void __launch_bounds__(256) fit_segsum_kernel(FitSortArgs a)
             acc[k] = 0.0;
         }
     };
+    // the next 32 slots' token ids are fetched one round ahead; a round's rows
+    // are requested before its centre indices are consumed
+    int t_next = (i0 + lane < i1) ? ord[i0 + lane] : 0;
     for (int64_t ib = i0; ib < i1; ib += 32) {
         const int nb = (int)min((int64_t)32, i1 - ib);
-        int t_l = 0, j_l = -1;
-        if (lane < nb) {
-            t_l = ord[ib + lane];
-            j_l = idx[t_l];
-        }
+        const int t_l = t_next;
+        t_next = (ib + 32 + lane < i1) ? ord[ib + 32 + lane] : 0;
+        const int j_l = lane < nb ? (int)idx[t_l] : -1;
         for (int b0 = 0; b0 < nb; b0 += 8) {
             float v[8][kPer];
             int jj[8];
 #pragma unroll
             for (int b = 0; b < 8; ++b) {
                 const int t = __shfl_sync(0xffffffffu, t_l, (b0 + b) & 31);
-                jj[b] = __shfl_sync(0xffffffffu, j_l, (b0 + b) & 31);
                 if (b0 + b < nb)
                     fit_load_row<D>(a, h, t, lane, v[b]);
-                else
+            }
+#pragma unroll
+            for (int b = 0; b < 8; ++b) {
+                jj[b] = __shfl_sync(0xffffffffu, j_l, (b0 + b) & 31);
+                if (b0 + b >= nb)
                     jj[b] = -1;
             }
 #pragma unroll

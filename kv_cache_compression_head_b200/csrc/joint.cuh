@@ -238,20 +238,25 @@ constexpr int kJDThreads = 288;
 
 constexpr uint32_t kJDSmemLimit = 227u * 1024u - 1024u;  // less the alignment slack
 
+constexpr uint32_t kJDStageRow = 80;                 // staged output row: 32 bf16 + 16 B pad
+constexpr uint32_t kJDStageWarp = 32u * kJDStageRow;  // per epilogue warp
+
 struct JDLayout {
     uint32_t a_bytes;  // one of A hi / A lo: [r/64][128][128 B]
     uint32_t w_bytes;  // one W stage: [D/64][r][128 B]
     int nst;           // W stages: 2 where they fit, else 1
-    uint32_t off_lo, off_w, off_bar, total;
+    uint32_t off_lo, off_w, off_bar, off_stg, total;
     __host__ __device__ JDLayout(int r, int D)
     {
         a_bytes = 128u * (uint32_t)r * 2u;
         w_bytes = (uint32_t)(D / 64) * (uint32_t)r * 128u;
-        nst = (2u * a_bytes + 2u * w_bytes + 128u <= kJDSmemLimit) ? 2 : 1;
+        const uint32_t fixed = 2u * a_bytes + 128u + 8u * kJDStageWarp;
+        nst = (fixed + 2u * w_bytes <= kJDSmemLimit) ? 2 : 1;
         off_lo = a_bytes;
         off_w = 2u * a_bytes;
         off_bar = off_w + (uint32_t)nst * w_bytes;
-        total = off_bar + 128u;
+        off_stg = off_bar + 128u;
+        total = off_stg + 8u * kJDStageWarp;
     }
 };
 
@@ -418,27 +423,44 @@ __global__ void __launch_bounds__(kJDThreads, 1)
                     break;
                 float v[32];
                 tmem_ld32(tmem + lane_off + (uint32_t)(b * a.D + cb * 32), v);
-                if (!valid)
-                    continue;
+                if (valid) {
 #pragma unroll
-                for (int u = 0; u < 4; ++u) {
-                    const uint4 m4 = mw[cb * 4 + u];
-                    const uint32_t m[4] = {m4.x, m4.y, m4.z, m4.w};
+                    for (int u = 0; u < 4; ++u) {
+                        const uint4 m4 = mw[cb * 4 + u];
+                        const uint32_t m[4] = {m4.x, m4.y, m4.z, m4.w};
 #pragma unroll
-                    for (int k = 0; k < 4; ++k) {
-                        v[u * 8 + 2 * k] = __fadd_rn(bf16_lo(m[k]), v[u * 8 + 2 * k]);
-                        v[u * 8 + 2 * k + 1] = __fadd_rn(bf16_hi(m[k]), v[u * 8 + 2 * k + 1]);
+                        for (int k = 0; k < 4; ++k) {
+                            v[u * 8 + 2 * k] = __fadd_rn(bf16_lo(m[k]), v[u * 8 + 2 * k]);
+                            v[u * 8 + 2 * k + 1] = __fadd_rn(bf16_hi(m[k]), v[u * 8 + 2 * k + 1]);
+                        }
                     }
                 }
-                const int64_t o = (t * a.H + h) * a.D + cb * 32;
                 if (a.out_bf16) {
-                    uint4 *dst = reinterpret_cast<uint4 *>(static_cast<uint16_t *>(a.out) + o);
+                    // through the warp's staging rows, so the stores of a warp
+                    // cover whole 64-byte row pieces of 8 rows at a time
+                    uint8_t *stg = smem + L.off_stg + (uint32_t)warp * kJDStageWarp;
+                    if (valid) {
 #pragma unroll
-                    for (int u = 0; u < 4; ++u)
-                        dst[u] = make_uint4(pack_bf16x2(v[8 * u], v[8 * u + 1]), pack_bf16x2(v[8 * u + 2], v[8 * u + 3]),
-                                            pack_bf16x2(v[8 * u + 4], v[8 * u + 5]),
-                                            pack_bf16x2(v[8 * u + 6], v[8 * u + 7]));
-                } else {
+                        for (int u = 0; u < 4; ++u)
+                            *reinterpret_cast<uint4 *>(stg + (uint32_t)lane * kJDStageRow + 16u * (uint32_t)u) =
+                                make_uint4(pack_bf16x2(v[8 * u], v[8 * u + 1]),
+                                           pack_bf16x2(v[8 * u + 2], v[8 * u + 3]),
+                                           pack_bf16x2(v[8 * u + 4], v[8 * u + 5]),
+                                           pack_bf16x2(v[8 * u + 6], v[8 * u + 7]));
+                    }
+                    __syncwarp();
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        const int rr = 8 * i + (lane >> 2), uu = lane & 3;
+                        const int64_t tr = t0 + 32 * (warp & 3) + rr;
+                        if (tr < a.T)
+                            *reinterpret_cast<uint4 *>(static_cast<uint16_t *>(a.out) + (tr * a.H + h) * a.D +
+                                                       cb * 32 + 8 * uu) =
+                                *reinterpret_cast<const uint4 *>(stg + (uint32_t)rr * kJDStageRow + 16u * (uint32_t)uu);
+                    }
+                    __syncwarp();
+                } else if (valid) {
+                    const int64_t o = (t * a.H + h) * a.D + cb * 32;
                     float4 *dst = reinterpret_cast<float4 *>(static_cast<float *>(a.out) + o);
 #pragma unroll
                     for (int u = 0; u < 8; ++u)

@@ -42,9 +42,13 @@ struct JointEncArgs {
     float *coef_out;       // [T][r] or null
 };
 
-// shared memory: two stages of {A: 128 x 64 bf16 (16 KB), B: 64 x r bf16}
+// shared memory: kJEStages stages of {A: 128 x 64 bf16 (16 KB), B: 64 x r bf16}
+constexpr int kJEStages = 4;
 __host__ __device__ constexpr uint32_t joint_enc_stage_bytes(int r) { return 16384u + 64u * (uint32_t)r * 2u; }
-__host__ __device__ constexpr uint32_t joint_enc_smem_bytes(int r) { return 2u * joint_enc_stage_bytes(r) + 64u; }
+__host__ __device__ constexpr uint32_t joint_enc_smem_bytes(int r)
+{
+    return (uint32_t)kJEStages * joint_enc_stage_bytes(r) + 128u;
+}
 
 __host__ __device__ constexpr uint32_t pow2_cols(int n)
 {
@@ -108,101 +112,136 @@ __device__ __forceinline__ void joint_quant_row(uint32_t trow, int r, uint8_t *c
     }
 }
 
-// One CTA per 128-token tile.  All 256 threads build the A stage (two threads
-// per token row, 32 channels each) and copy the B stage; thread 0 issues the
-// MMAs; in the epilogue the two threads of a row (warps w and w + 4 share the
-// TMEM lanes) quantise alternate groups.
+// One CTA per 128-token tile, K-blocks of 64 channels in a ring of kJEStages
+// stages.  Thread 0 loads each block's x tile (3-D map over [T][H][D], 128-byte
+// swizzle: already the K-major A layout) and W_enc rows (2-D map, MN-major B)
+// with TMA three blocks ahead and issues the MMAs.  All 256 threads (two per
+// token row, 32 channels each) rewrite their units of the x tile in place as
+// A = bf16(x - mu[idx]), the centre units fetched one block ahead.  In the
+// epilogue the two threads of a row (warps w and w + 4 share the TMEM lanes)
+// quantise alternate groups.
 template <int G, int BITS>
-__global__ void __launch_bounds__(kJEThreads, 1) joint_encode_kernel(JointEncArgs a)
+__global__ void __launch_bounds__(kJEThreads, 1)
+    joint_encode_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_w,
+                        JointEncArgs a)
 {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const uint32_t stage_bytes = joint_enc_stage_bytes(a.r);
-    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + 2 * stage_bytes);
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 3);
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + kJEStages * stage_bytes);  // full[4], done[4]
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 2 * kJEStages);
+    auto full = [&](int st) { return smem_u32(bars + st); };
+    auto done = [&](int st) { return smem_u32(bars + kJEStages + st); };
     const int tid = threadIdx.x, warp = tid >> 5;
     const int row = tid & 127, half = tid >> 7;
     const int64_t t0 = (int64_t)blockIdx.x * kJRows;
     const int64_t t = t0 + row;
     const bool valid = t < a.T;
     const uint32_t ncols = pow2_cols(a.r);
+    const int nk = a.H * a.D / kJKBlock;
+    const uint32_t tx_bytes = stage_bytes;
 
     if (warp == 0)
         tmem_alloc(smem_u32(tmem_slot), ncols);
     if (tid == 0) {
-        mbar_init(smem_u32(bars + 0), 1);
-        mbar_init(smem_u32(bars + 1), 1);
+        for (int st = 0; st < kJEStages; ++st) {
+            mbar_init(full(st), 1);
+            mbar_init(done(st), 1);
+        }
         fence_mbar_init();
     }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
-    const int nk = a.H * a.D / kJKBlock;
     const uint32_t idesc = idesc_f32acc(128, a.r, true, false, true);  // bf16, B MN-major
-    uint32_t phase[2] = {0u, 0u};
-    bool ok = true;
-
-    for (int kb = 0; kb < nk; ++kb) {
-        const int s = kb & 1;
-        uint8_t *sA = smem + (uint32_t)s * stage_bytes;
-        uint8_t *sB = sA + 16384;
-        if (kb >= 2) {  // the MMAs of block kb - 2 read this stage
-            ok = mbar_wait(smem_u32(bars + s), phase[s]) && ok;
-            phase[s] ^= 1u;
-        }
-        // A: residual of channels [64 kb, 64 kb + 64) of this token, bf16
+    auto issue_loads = [&](int kb) {  // thread 0: TMA of block kb into its stage
+        const int st = kb % kJEStages;
+        uint8_t *sA = smem + (uint32_t)st * stage_bytes;
         const int i0 = kb * kJKBlock;
-        const int h = i0 / a.D, c0 = i0 % a.D;
-        int j = 0;
-        if (valid) {
+        mbar_arrive_expect_tx(full(st), tx_bytes);
+        tma_load_3d(smem_u32(sA), &tmap_x, full(st), i0 % a.D, i0 / a.D, (int)t0);
+        for (int c = 0; c < a.r / 64; ++c)
+            tma_load_2d(smem_u32(sA + 16384u + (uint32_t)c * 8192u), &tmap_w, full(st), c * 64, i0);
+    };
+    if (tid == 0)
+        for (int kb = 0; kb < kJEStages - 1 && kb < nk; ++kb)
+            issue_loads(kb);
+
+    // centre units of this thread's 32 channels of block kb (one block ahead)
+    int jh = -1, j = 0;
+    auto fetch_mu = [&](int kb, uint4 *mu) {
+        const int i0 = kb * kJKBlock, h = i0 / a.D, c0 = i0 % a.D;
+        if (!valid)
+            return;
+        if (h != jh) {
+            jh = h;
             j = a.idx[(int64_t)h * a.T + t];
             if (j >= a.C) {
                 raise_status(DEVSTAT_BAD_INDEX);
                 j = 0;
             }
         }
+        const uint4 *src = reinterpret_cast<const uint4 *>(a.cent + ((int64_t)h * a.C + j) * a.D + c0) + 4 * half;
 #pragma unroll
-        for (int u = half * (kJKBlock / 16); u < (half + 1) * (kJKBlock / 16); ++u) {
+        for (int u = 0; u < 4; ++u)
+            mu[u] = __ldg(src + u);
+    };
+    uint4 mu_next[4];
+    fetch_mu(0, mu_next);
+    bool ok = true;
+
+    for (int kb = 0; kb < nk; ++kb) {
+        const int s = kb % kJEStages;
+        uint8_t *sA = smem + (uint32_t)s * stage_bytes;
+        uint4 mu[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+            mu[u] = mu_next[u];
+        if (kb + 1 < nk)
+            fetch_mu(kb + 1, mu_next);
+        ok = mbar_wait(full(s), (uint32_t)((kb / kJEStages) & 1)) && ok;
+        // A in place: this thread's 4 units of its row
+#pragma unroll
+        for (int uu = 0; uu < 4; ++uu) {
+            const int u = 4 * half + uu;
+            uint4 *p = reinterpret_cast<uint4 *>(sA + sw128_unit_offset(row, u, kJRows));
             uint4 w = make_uint4(0, 0, 0, 0);
             if (valid) {
-                float xv[8], mv[8];
-                load_bf16x8(a.x + (t * a.H + h) * a.D + c0 + u * 8, xv);
-                load_bf16x8(a.cent + ((int64_t)h * a.C + j) * a.D + c0 + u * 8, mv);
-                w = make_uint4(pack_bf16x2(__fsub_rn(xv[0], mv[0]), __fsub_rn(xv[1], mv[1])),
-                               pack_bf16x2(__fsub_rn(xv[2], mv[2]), __fsub_rn(xv[3], mv[3])),
-                               pack_bf16x2(__fsub_rn(xv[4], mv[4]), __fsub_rn(xv[5], mv[5])),
-                               pack_bf16x2(__fsub_rn(xv[6], mv[6]), __fsub_rn(xv[7], mv[7])));
+                const uint4 xw = *p;
+                const uint32_t xa[4] = {xw.x, xw.y, xw.z, xw.w}, ma[4] = {mu[uu].x, mu[uu].y, mu[uu].z, mu[uu].w};
+                uint32_t o[4];
+#pragma unroll
+                for (int k = 0; k < 4; ++k)
+                    o[k] = pack_bf16x2(__fsub_rn(bf16_lo(xa[k]), bf16_lo(ma[k])),
+                                       __fsub_rn(bf16_hi(xa[k]), bf16_hi(ma[k])));
+                w = make_uint4(o[0], o[1], o[2], o[3]);
             }
-            *reinterpret_cast<uint4 *>(sA + sw128_unit_offset(row, u, kJRows)) = w;
-        }
-        // B: W rows [i0, i0 + 64), all r columns -> MN-major [r/64][64][128 B]
-        for (int e = tid; e < kJKBlock * (a.r / 8); e += kJEThreads) {
-            const int k = e / (a.r / 8), u = e % (a.r / 8);
-            const uint4 w = __ldg(reinterpret_cast<const uint4 *>(a.w + (int64_t)(i0 + k) * a.r) + u);
-            *reinterpret_cast<uint4 *>(sB + sw128_unit_offset(k, u, kJKBlock)) = w;
+            *p = w;
         }
         fence_proxy_async_smem();
         tc_fence_before();
         __syncthreads();
         if (tid == 0) {
             tc_fence_after();
-            const uint32_t aA = smem_u32(sA), aB = smem_u32(sB);
+            const uint32_t aA = smem_u32(sA), aB = smem_u32(sA + 16384u);
 #pragma unroll
             for (int ks = 0; ks < kJKBlock / 16; ++ks)
                 umma_ss(tmem, sdesc_sw128(aA + (uint32_t)ks * 32u, 16, 1024),
                         sdesc_sw128(aB + (uint32_t)ks * 2048u, kJKBlock * 128u, 1024), idesc,
                         (kb > 0 || ks > 0) ? 1u : 0u);
-            umma_commit(smem_u32(bars + s));
+            umma_commit(done(s));
+            // block kb + 3 goes into the stage of block kb - 1 once its MMAs are done
+            const int kn = kb + kJEStages - 1;
+            if (kn < nk) {
+                if (kb >= 1)
+                    ok = mbar_wait(done((kb - 1) % kJEStages), (uint32_t)(((kb - 1) / kJEStages) & 1)) && ok;
+                issue_loads(kn);
+            }
         }
     }
-    // each stage has one commit outstanding (its last block); wait for both
-    {
-        const int s_last = (nk - 1) & 1;
-        if (nk >= 2)
-            ok = mbar_wait(smem_u32(bars + (s_last ^ 1)), phase[s_last ^ 1]) && ok;
-        ok = mbar_wait(smem_u32(bars + s_last), phase[s_last]) && ok;
-    }
+    // the last block's MMAs complete after all earlier ones: wait for them
+    ok = mbar_wait(done((nk - 1) % kJEStages), (uint32_t)(((nk - 1) / kJEStages) & 1)) && ok;
     tc_fence_after();
     const uint32_t trow = tmem + (((uint32_t)(warp & 3) * 32u) << 16);
     ok = __all_sync(0xffffffffu, ok);  // tcgen05.ld below is warp-collective

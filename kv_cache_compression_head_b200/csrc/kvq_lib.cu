@@ -247,7 +247,23 @@ kvq_status launch_joint_encode_t(const JointEncArgs &a, cudaStream_t s)
             return KVQ_ERR_CUDA;
         configured[dev] = true;
     }
-    joint_encode_kernel<G, BITS><<<(unsigned)ceil_div(a.T, kJRows), kJEThreads, smem, s>>>(a);
+    CUtensorMap mx, mw;
+    if (!make_history_map(&mx, a.x, a.T, a.H, a.D))
+        return KVQ_ERR_CUDA;
+    PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
+    if (!enc)
+        return KVQ_ERR_CUDA;
+    // W_enc [H d][r] bf16: box = 64 coefficients x 64 rows, 128-byte swizzle
+    // (the MN-major B layout of the encoder's MMA)
+    cuuint64_t dims[2] = {(cuuint64_t)a.r, (cuuint64_t)a.H * a.D};
+    cuuint64_t strides[1] = {(cuuint64_t)a.r * 2};
+    cuuint32_t box[2] = {64, (cuuint32_t)kJKBlock};
+    cuuint32_t estr[2] = {1, 1};
+    if (enc(&mw, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<uint16_t *>(a.w), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+        return KVQ_ERR_CUDA;
+    joint_encode_kernel<G, BITS><<<(unsigned)ceil_div(a.T, kJRows), kJEThreads, smem, s>>>(mx, mw, a);
     return launch_status();
 }
 

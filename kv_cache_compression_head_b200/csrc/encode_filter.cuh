@@ -440,40 +440,42 @@ __global__ void __launch_bounds__(kFltThreads, 2)
                 best = __float_as_int(sWin[row].y);
         }
         // three or more candidates (rare): re-score the window (or every centre
-        // when the window is not finite) with the specified distance; the
-        // half-0 thread decides and hands the result to its partner.  Both
-        // warps of the pair see the same flags, so they take the branch together.
+        // when the window is not finite) with the specified distance.  Each
+        // thread of the pair scans its own half of the columns in increasing
+        // index order; the lower half wins ties.  Both warps of the pair see
+        // the same flags, so they take the branch together.
         if (__any_sync(0xffffffffu, wide_case)) {
-            if (half == 0) {
-                float bd = INFINITY;
-                int bj = -1;
-                for (int c = 0; c < nchunks; ++c) {
-                    float p[32];
-                    tmem_ld32(tmem + lane_off + (uint32_t)(c * 32), p);
-                    uint32_t cand = 0u;
+            float bd = INFINITY;
+            int bj = -1;
+            for (int c = c_lo; c < c_hi; ++c) {
+                float p[32];
+                tmem_ld32(tmem + lane_off + (uint32_t)(c * 32), p);
+                uint32_t cand = 0u;
 #pragma unroll
-                    for (int i = 0; i < 32; ++i) {
-                        const int j = c * 32 + i;
-                        const float v = fmaf(-2.0f, p[i], sNrm[j]);
-                        if (wide_case && j < a.C && (!finite || v <= thr))
-                            cand |= 1u << i;
-                    }
-                    while (cand) {  // increasing index order
-                        const int i = __ffs(cand) - 1;
-                        cand &= cand - 1u;
-                        const int j = c * 32 + i;
-                        const float dj = spec_distance_smem<D>(sX, sMu, Cpad, row, j);
-                        if (bj < 0 || dj < bd) {
-                            bd = dj;
-                            bj = j;
-                        }
+                for (int i = 0; i < 32; ++i) {
+                    const int j = c * 32 + i;
+                    const float v = fmaf(-2.0f, p[i], sNrm[j]);
+                    if (wide_case && j < a.C && (!finite || v <= thr))
+                        cand |= 1u << i;
+                }
+                while (cand) {  // increasing index order
+                    const int i = __ffs(cand) - 1;
+                    cand &= cand - 1u;
+                    const int j = c * 32 + i;
+                    const float dj = spec_distance_smem<D>(sX, sMu, Cpad, row, j);
+                    if (bj < 0 || dj < bd) {
+                        bd = dj;
+                        bj = j;
                     }
                 }
-                sWin[row] = make_float4(__int_as_float(bj), 0.f, 0.f, 0.f);
             }
+            reinterpret_cast<float2 *>(sWin + row)[half] = make_float2(bd, __int_as_float(bj));
             named_barrier_sync_q(warp & 3, 64);
-            if (wide_case)
-                best = __float_as_int(sWin[row].x);
+            if (wide_case) {
+                const float4 w = sWin[row];
+                const int j0 = __float_as_int(w.y), j1 = __float_as_int(w.w);
+                best = (j0 < 0 || (j1 >= 0 && w.z < w.x)) ? j1 : j0;
+            }
         }
         if (best < 0 || best >= a.C)
             best = 0;  // unreachable for finite inputs

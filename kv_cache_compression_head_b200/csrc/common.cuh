@@ -271,11 +271,6 @@ __host__ __device__ constexpr uint32_t idesc_f32acc(int M, int N, bool bf16, boo
            | ((uint32_t)(M >> 4) << 24);          // M / 16
 }
 
-__host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, bool a_mn_major, bool b_mn_major)
-{
-    return idesc_f32acc(M, N, true, a_mn_major, b_mn_major);
-}
-
 // D[tmem] (+)= A[smem] * B[smem]^T ; issued by one thread.
 __device__ __forceinline__ void umma_ss(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
                                         uint32_t accumulate)

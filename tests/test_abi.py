@@ -132,3 +132,20 @@ def test_bad_pointers_and_sizes_rejected_on_host(K):
     assert _err(K, "kvq_joint_coefficients", ctypes.byref(dj), A, K.KVQ_BF16, 100, A, A, A, A + 4, None, 0, None) \
         == K.KVQ_ERR_ALIGNMENT
     assert K.workspace_size(K.KVQ_OP_ENCODE, K.Codec(12, 128, 256, 4, 32, 192), 32760) == 0
+
+
+def test_binding_refuses_to_load_without_the_library(tmp_path):
+    """A copy of the package without libkvq.so: importing the binding raises
+    (the product path has no fallback)."""
+    import shutil
+    import subprocess
+    import sys
+
+    pkg = tmp_path / "kv_cache_compression_head_b200"
+    pkg.mkdir()
+    for name in ("__init__.py", "kvq.py"):
+        shutil.copy(os.path.join(ROOT, "kv_cache_compression_head_b200", name), pkg / name)
+    r = subprocess.run([sys.executable, "-c", "import kv_cache_compression_head_b200.kvq"], cwd=tmp_path,
+                       capture_output=True, text=True, env={**os.environ, "PYTHONPATH": str(tmp_path)})
+    assert r.returncode != 0
+    assert "ImportError" in r.stderr and "libkvq.so not built" in r.stderr

@@ -1,0 +1,78 @@
+"""The oracle's pins catch plausible mistakes: each case below plants one
+mistake in a copy of the C oracle (a dropped term, a flipped sign, a wrong
+index or bit order, a wrong tie rule, a skipped rounding), builds it, points
+the oracle wrapper at it and checks that at least one pin of
+tests/test_oracle_pins.py fails.  CPU only; the real oracle is restored after
+every case."""
+
+import inspect
+import os
+import subprocess
+import tempfile
+
+import pytest
+
+from oracle import build as OB
+from oracle import oracle as O
+from tests import test_oracle_pins as P
+
+# (name, text in kvq_oracle.c, replacement)
+MUTATIONS = [
+    ("distance drops the last channel",
+     "for (int c = 0; c < d; ++c) {\n        float e = x[c] - mu[c];",
+     "for (int c = 0; c < d - 1; ++c) {\n        float e = x[c] - mu[c];"),
+    ("distance subtracts the squared term", "acc = acc + sq;", "acc = acc - sq;"),
+    ("argmin ties go to the highest index", "        if (dj < bd) {\n            bd = dj;",
+     "        if (dj <= bd) {\n            bd = dj;"),
+    ("zero point with the wrong sign", "float z = rintf(-mn * inv);", "float z = rintf(mn * inv);"),
+    ("codes without the zero point", "float v = rintf(r[c] * inv) + z;", "float v = rintf(r[c] * inv);"),
+    ("dequantisation adds the zero point", "float t = (float)q - z;", "float t = (float)q + z;"),
+    ("codes packed high bits first", "<< (i * bits);", "<< ((per - 1 - i) * bits);"),
+    ("k-means mean over n + 1", "/ (double)counts[j];", "/ (double)(counts[j] + 1);"),
+    ("empty centre zeroed instead of kept",
+     "                if (counts[j] == 0)\n                    continue;",
+     "                if (counts[j] == 0) {\n                    for (int c = 0; c < d; ++c)\n"
+     "                        cent_h[(int64_t)j * d + c] = 0;\n                    continue;\n                }"),
+    ("joint residual not rounded to bf16", "res[h * d + c] = bf16_widen(bf16_round(e));", "res[h * d + c] = e;"),
+    ("joint decoder forgets the centre", "out[(t * H + h) * (int64_t)d + c] = mu + (float)acc;",
+     "out[(t * H + h) * (int64_t)d + c] = (float)acc;"),
+]
+
+
+def _pins():
+    return [(n, f) for n, f in inspect.getmembers(P, inspect.isfunction)
+            if n.startswith("test_") and not inspect.signature(f).parameters]
+
+
+def _build_mutant(src: str, out_dir: str) -> str:
+    path_c = os.path.join(out_dir, "kvq_oracle_mutant.c")
+    with open(path_c, "w") as f:
+        f.write(src)
+    path_so = os.path.join(out_dir, "libkvq_oracle_mutant.so")
+    subprocess.run(["gcc", *OB.CFLAGS, "-o", path_so, path_c, "-lm"], check=True)
+    return path_so
+
+
+@pytest.mark.parametrize("name,old,new", MUTATIONS, ids=[m[0] for m in MUTATIONS])
+def test_pins_catch_planted_mistake(name, old, new):
+    src = open(OB.SRC).read()
+    assert src.count(old) == 1, f"mutation site not unique or missing: {name}"
+    saved_path, saved_lib = O._LIB_PATH, O._lib
+    failed = []
+    with tempfile.TemporaryDirectory() as d:
+        so = _build_mutant(src.replace(old, new), d)
+        try:
+            O._LIB_PATH, O._lib = so, None
+            for pin_name, pin in _pins():
+                try:
+                    pin()
+                except (AssertionError, RuntimeError, ValueError):
+                    failed.append(pin_name)
+        finally:
+            O._LIB_PATH, O._lib = saved_path, saved_lib
+    assert failed, f"no pin fails with the planted mistake: {name}"
+
+
+def test_unmutated_oracle_passes_every_pin():
+    for _, pin in _pins():
+        pin()

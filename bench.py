@@ -265,6 +265,14 @@ class Pipeline:
         self.enc_j = [K.alloc_encoded(c, T, device) for c in self.codec_j]
         self.comp_j = [K.Compressed(c, T, self.cent[i], *self.enc_j[i], w_dec=self.w_dec)
                        for i, c in enumerate(self.codec_j)]
+        # full-layer attention (outside the step): the chunk's own keys and
+        # values follow the history; one call = compressed part + dense part
+        # + their merge
+        self.kc = torch.empty((Tq, H, d), dtype=bf, device=device)
+        self.vc = torch.empty((Tq, H, d), dtype=bf, device=device)
+        self.ws_layer = K.alloc_workspace(K.KVQ_OP_LAYER_ATTENTION, self.codec_k, T, device, num_queries=Tq)
+        self.o_layer = torch.empty((Tq, H, d), dtype=bf, device=device)
+        self.lse_layer = torch.empty((H, Tq), dtype=torch.float32, device=device)
         # fit: seed + (assign + 4 sort + 3 update kernels) per round; encode 1;
         # decode 1; joint encode 2 (assign, projection), joint decode 1;
         # attention 2 per block (split + its merge); final merge 1 -- K and V
@@ -314,6 +322,32 @@ class Pipeline:
         mark("merge", 1)
 
 
+    def layer_attention(self):
+        self.K.kvq_layer_attention(self.q, self.comp[0], self.comp[1], self.kc, self.vc, self.o_layer,
+                                   self.lse_layer, self.ws_layer)
+
+    def dense_attention(self):
+        self.K.kvq_attention_dense_lse(self.q, self.kc, self.vc, self.o_layer, self.lse_layer,
+                                       workspace=self.ws_attn)
+
+
+def time_calls(fn, reps, warmup, flush):
+    """Mean device time (ms) of fn() over reps calls, L2 flushed before each."""
+    import torch
+
+    for _ in range(warmup):
+        flush.zero_()
+        fn()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(reps)]
+    for a, b in ev:
+        flush.zero_()
+        a.record()
+        fn()
+        b.record()
+    torch.cuda.synchronize()
+    return statistics.mean(a.elapsed_time(b) for a, b in ev)
+
+
 def run_gpu(args):
     import torch
 
@@ -336,6 +370,8 @@ def run_gpu(args):
     pipe.xk.copy_(pk)
     pipe.xv.copy_(pv)
     pipe.q.copy_(pq)
+    pipe.kc.copy_(pin(synth.make_chunk(w, "K")))
+    pipe.vc.copy_(pin(synth.make_chunk(w, "V")))
     flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=device)
     torch.cuda.synchronize()
 
@@ -364,6 +400,15 @@ def run_gpu(args):
     st = pipe.K.kvq_last_device_status()
     if st != 0:
         raise RuntimeError(f"device status after timing: {pipe.K.status_string(st)}")
+
+    # next to the step: the current chunk's full-layer attention (compressed
+    # history + its own uncompressed keys, merged by LSE) and the dense part
+    # alone, on the step's freshly encoded history
+    layer_ms = max_over_ranks(time_calls(pipe.layer_attention, args.steps, args.warmup, flush), world, device)
+    dense_ms = max_over_ranks(time_calls(pipe.dense_attention, args.steps, args.warmup, flush), world, device)
+    st = pipe.K.kvq_last_device_status()
+    if st != 0:
+        raise RuntimeError(f"device status after the layer attention: {pipe.K.status_string(st)}")
 
     row_ms = {r: [e[r][0].elapsed_time(e[r][1]) for e in ev] for r in Pipeline.ROWS}
     step_ms = [ev[k]["fit"][0].elapsed_time(ev[k]["merge"][1]) for k in range(args.steps)]
@@ -423,6 +468,20 @@ def run_gpu(args):
                           "frac": attn_tflops / tfl},
             "merge": {"ms": row_mean["merge"], "gbps": merge_gbps, "hbm_frac": merge_gbps / hbm},
         }
+        Tq, H, d = w.query_tokens, w.num_heads, w.head_dim
+        layer_flops = 4.0 * Tq * (w.history_tokens + Tq) * d * H
+        dense_flops = 4.0 * Tq * Tq * d * H
+        next_rows = {
+            "layer_attention": {"ms": layer_ms, "calls": 1, "keys": w.history_tokens + Tq,
+                                "tflops": layer_flops / (layer_ms / 1e3) / 1e12,
+                                "frac": layer_flops / (layer_ms / 1e3) / 1e12 / tfl,
+                                "what": "kvq_layer_attention: 32760 compressed history keys + the 4680-key chunk "
+                                        "(bf16), one softmax, LSE merge inside the call"},
+            "dense_attention": {"ms": dense_ms, "calls": 1, "keys": Tq,
+                                "tflops": dense_flops / (dense_ms / 1e3) / 1e12,
+                                "frac": dense_flops / (dense_ms / 1e3) / 1e12 / tfl,
+                                "what": "kvq_attention_dense_lse over the 4680-key chunk alone"},
+        }
         line = {
             "metric": METRIC,
             "value": world * w.history_tokens / (ms_step / 1e3),
@@ -449,6 +508,7 @@ def run_gpu(args):
                          "traffic": ATTN_NCU_TRAFFIC_BYTES,
                          "traffic_unit": "bytes per launch (ncu dram__bytes_read.sum + dram__bytes_write.sum)"},
             "rows": rows,
+            "next_rows": next_rows,
             "clocks": clk,
             "gpu_launches": pipe.launches_per_step * args.steps,
             "wall_s_timed_region": wall,

@@ -18,6 +18,9 @@
  *  - attention over the compressed history with the reconstruction done on
  *    demand, and log-sum-exp merging of partial results (NanoKV page,
  *    Fig. 4(a,d); QuantWM, Fig. 9).
+ *  - the current chunk's full attention: the compressed history together
+ *    with uncompressed keys (the chunk itself, raw protected tokens; NanoKV
+ *    page, Table 4) under one softmax, by the same LSE merging.
  *
  * Conventions for every call:
  *  - All tensor pointers are DEVICE pointers owned by the caller; the library
@@ -79,7 +82,8 @@ typedef enum {
     KVQ_OP_FIT = 0,
     KVQ_OP_ENCODE = 1,
     KVQ_OP_DECODE = 2,
-    KVQ_OP_ATTENTION = 3
+    KVQ_OP_ATTENTION = 3,
+    KVQ_OP_LAYER_ATTENTION = 4
 } kvq_op;
 
 /* Codec of one K or V branch.  K and V are described separately, which is
@@ -113,7 +117,10 @@ KVQ_API kvq_status kvq_encoded_sizes(const kvq_codec_desc *desc, int64_t num_tok
                              size_t *code_bytes, size_t *meta_bytes);
 
 /* Device workspace (bytes) an operation needs for these sizes; 0 means the
- * call accepts workspace = NULL.  Tq is used by KVQ_OP_ATTENTION only. */
+ * call accepts workspace = NULL.  Tq is used by KVQ_OP_ATTENTION and
+ * KVQ_OP_LAYER_ATTENTION only, and only H and d of desc matter for them.
+ * KVQ_OP_ATTENTION also sizes kvq_attention_dense_lse's optional workspace
+ * (pass a desc with the same H and d). */
 KVQ_API kvq_status kvq_workspace_size(kvq_op op, const kvq_codec_desc *desc, int64_t num_tokens,
                               int64_t num_queries, size_t *bytes);
 
@@ -242,6 +249,52 @@ KVQ_API kvq_status kvq_attention_lse(const void *q, int64_t num_queries, const k
                              const kvq_compressed_view *v, int64_t t_begin, int64_t t_end, float softmax_scale,
                              void *o_out, kvq_dtype o_dtype, float *lse_out, void *workspace,
                              size_t workspace_bytes, kvq_stream_t stream);
+
+/*
+ * Dense-mode attention: the same computation as kvq_attention_lse over keys
+ * [t_begin, t_end) of UNCOMPRESSED bf16 keys and values -- the current
+ * chunk's own keys, or raw protected history tokens such as attention sinks
+ * and a recent window (NanoKV page, Table 4: protection keeps extra
+ * historical tokens uncompressed) -- so that its partial result can be merged
+ * with the compressed history's by LSE (NanoKV page, Fig. 4(d)).
+ *   q [Tq][H][d] bf16;  k, v [num_keys][H][d] bf16 (may be NULL when the
+ *   range is empty);  o_out [Tq][H][d] (o_dtype);  lse_out [H][Tq] float.
+ * Logits are exact bf16 products accumulated in binary32 (no lo part); v is
+ * widened to fp16 for the tensor cores (exact for |v| in [2^-14, 65504];
+ * larger magnitudes saturate) and P is rounded to fp16, as in
+ * kvq_attention_lse.  No mask: every query sees every key of the range.
+ * d in {64, 128} (KVQ_ERR_UNSUPPORTED otherwise); all pointers 16-byte
+ * aligned.  Workspace: optional, as for kvq_attention_lse, sized by
+ * kvq_workspace_size(KVQ_OP_ATTENTION, desc with this H and d, 0, Tq).
+ */
+KVQ_API kvq_status kvq_attention_dense_lse(const void *q, int64_t num_queries, const void *k, const void *v,
+                                           int64_t num_keys, int32_t num_heads, int32_t head_dim, int64_t t_begin,
+                                           int64_t t_end, float softmax_scale, void *o_out, kvq_dtype o_dtype,
+                                           float *lse_out, void *workspace, size_t workspace_bytes,
+                                           kvq_stream_t stream);
+
+/*
+ * Full-layer attention of the current chunk: its queries attend to history
+ * tokens [t_begin, t_end) of a compressed K and V (per-head codec, as in
+ * kvq_attention_lse) AND to num_cur uncompressed bf16 keys and values (the
+ * chunk itself, plus any raw protected tokens the caller places there), with
+ * one softmax over all of them:
+ *   o_i = sum_j softmax(s_i)_j v_j over both key sets, lse_i = ln sum_j exp(s_ij).
+ * Computed as two partial attentions (compressed and dense) written as
+ * binary32 partials to the workspace and merged by LSE (NanoKV page,
+ * Fig. 4(a,d)).
+ *   q [Tq][H][d] bf16; k_cur, v_cur [num_cur][H][d] bf16 (NULL allowed when
+ *   num_cur = 0); o_out [Tq][H][d] (o_dtype); lse_out [H][Tq] float.
+ * If both key sets are empty, o = 0 and lse = -inf.
+ * Workspace (required, 16-byte aligned): at least
+ * kvq_workspace_size(KVQ_OP_LAYER_ATTENTION, k_hist desc, T, Tq) bytes, else
+ * KVQ_ERR_WORKSPACE.  Other requirements as for kvq_attention_lse.
+ */
+KVQ_API kvq_status kvq_layer_attention(const void *q, int64_t num_queries, const kvq_compressed_view *k_hist,
+                                       const kvq_compressed_view *v_hist, int64_t t_begin, int64_t t_end,
+                                       const void *k_cur, const void *v_cur, int64_t num_cur, float softmax_scale,
+                                       void *o_out, kvq_dtype o_dtype, float *lse_out, void *workspace,
+                                       size_t workspace_bytes, kvq_stream_t stream);
 
 /*
  * Merge n partial attention results over disjoint history parts by their

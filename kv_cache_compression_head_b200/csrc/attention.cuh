@@ -4,7 +4,10 @@
 // A compressed K or V history is read through CodecView: idx, packed codes,
 // {s, z} pairs and the bf16 centres, from which the kernels rebuild
 // k^ = mu[idx] + (q - z) s on the fly (NanoKV page, Fig. 4(a,b); QuantWM,
-// Fig. 9: on-demand reconstruction).
+// Fig. 9: on-demand reconstruction).  In dense mode the same kernels read
+// uncompressed bf16 keys and values instead: the current chunk and the raw
+// protected tokens (sinks, recent window) whose partial result is merged with
+// the compressed history's by LSE (NanoKV page, Fig. 4(d) and Table 4).
 #pragma once
 
 #include "codec.cuh"
@@ -28,6 +31,9 @@ struct AttnArgs {
     int64_t Tq;
     int H;
     CodecView k, v;
+    const uint16_t *k_dense;  // dense mode: keys [Tk][H][D] bf16 (k, v unused)
+    const uint16_t *v_dense;  // dense mode: values [Tk][H][D] bf16
+    int dense;
     int64_t t_begin, t_end;
     float scale_log2;  // softmax scale * log2(e)
     void *o_out;

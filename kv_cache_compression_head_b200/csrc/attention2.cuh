@@ -10,7 +10,9 @@
 //               history tile rebuild k^ (bf16 hi + lo tiles) and v^ (fp16
 //               tile) from codes, {s, z}, idx and the bf16 centres straight
 //               into the 128-byte-swizzled operand layout; two threads per
-//               history row, one per half of the channels.
+//               history row, one per half of the channels.  Dense mode
+//               (uncompressed bf16 K and V): the rows are copied instead, K
+//               has no lo tile and V is widened to fp16.
 //   warp 8      MMA issuer (one thread): S_i = Q_i K_hi^T + Q_i K_lo^T into
 //               TMEM for both query tiles, then O_i += P_i V^ (fp16) once the
 //               softmax has published P_i.
@@ -182,6 +184,52 @@ __device__ __forceinline__ void a2_dequant(const CodecView &cv, int h, int64_t t
         a2_dequant_half<D, 4, SPLIT>(cv, h, tok, valid, half, tile, tile_lo, row);
 }
 
+// Dense mode: channels [d/2 half, d/2 half + d/2) of row `tok` of an
+// uncompressed bf16 [Tk][H][D] array into the swizzled tile -- keys as they
+// are (the K hi tile; no lo part), values (VALUE) widened to fp16.
+template <int D, bool VALUE>
+__device__ __forceinline__ void a2_dense_half(const uint16_t *x, int H, int h, int64_t tok, bool valid, int half,
+                                              uint8_t *tile, uint32_t row)
+{
+    constexpr int kUnits = D / 16;
+    const int u0 = half * kUnits;
+    uint4 w[kUnits];
+    const uint4 *src = reinterpret_cast<const uint4 *>(x + (tok * H + h) * D) + u0;
+#pragma unroll
+    for (int uu = 0; uu < kUnits; ++uu)
+        w[uu] = valid ? __ldg(src + uu) : make_uint4(0, 0, 0, 0);
+#pragma unroll
+    for (int uu = 0; uu < kUnits; ++uu) {
+        if (VALUE)
+            w[uu] = make_uint4(pack_f16x2_sat(bf16_lo(w[uu].x), bf16_hi(w[uu].x)),
+                               pack_f16x2_sat(bf16_lo(w[uu].y), bf16_hi(w[uu].y)),
+                               pack_f16x2_sat(bf16_lo(w[uu].z), bf16_hi(w[uu].z)),
+                               pack_f16x2_sat(bf16_lo(w[uu].w), bf16_hi(w[uu].w)));
+        *reinterpret_cast<uint4 *>(tile + sw128_unit_offset(row, u0 + uu, 128)) = w[uu];
+    }
+}
+
+// One history row's half of the K operand (hi, lo) or of the V operand,
+// rebuilt from the compressed view or copied in dense mode.
+template <int D>
+__device__ __forceinline__ void a2_fill_k(const AttnArgs &a, int h, int64_t tok, int half, uint8_t *hi, uint8_t *lo,
+                                          uint32_t row)
+{
+    if (a.dense)
+        a2_dense_half<D, false>(a.k_dense, a.H, h, tok, tok < a.t_end, half, hi, row);
+    else
+        a2_dequant<D, true>(a.k, h, tok, tok < a.t_end, half, hi, lo, row);
+}
+
+template <int D>
+__device__ __forceinline__ void a2_fill_v(const AttnArgs &a, int h, int64_t tok, int half, uint8_t *tile, uint32_t row)
+{
+    if (a.dense)
+        a2_dense_half<D, true>(a.v_dense, a.H, h, tok, tok < a.t_end, half, tile, row);
+    else
+        a2_dequant<D, false>(a.v, h, tok, tok < a.t_end, half, tile, nullptr, row);
+}
+
 __device__ __forceinline__ void tmem_st32(uint32_t taddr, const float *v)
 {
     asm volatile(
@@ -326,7 +374,7 @@ __global__ void __launch_bounds__(kA2Threads, 1) attention2_kernel(AttnArgs a)
         if (ntiles > 0) {
             {
                 const int64_t tok = a.t_begin + r;
-                a2_dequant<D, true>(a.k, h, tok, tok < a.t_end, half, slot(0, 0), slot(0, 1), r);
+                a2_fill_k<D>(a, h, tok, half, slot(0, 0), slot(0, 1), r);
                 fence_proxy_async_smem();
                 mbar_arrive(bar(B_KFULL0));
             }
@@ -334,13 +382,13 @@ __global__ void __launch_bounds__(kA2Threads, 1) attention2_kernel(AttnArgs a)
                 if (j >= 1 && !a2_wait(bar(B_PVDONE), (uint32_t)((j - 1) & 1), abort_flag))
                     break;
                 const int64_t tok = a.t_begin + (int64_t)j * 128 + r;
-                a2_dequant<D, false>(a.v, h, tok, tok < a.t_end, half, smem + L::offV, nullptr, r);
+                a2_fill_v<D>(a, h, tok, half, smem + L::offV, r);
                 fence_proxy_async_smem();
                 mbar_arrive(bar(B_VFULL));
                 if (j + 1 < ntiles) {
                     const int s = (j + 1) & 1;
                     const int64_t tk = tok + 128;
-                    a2_dequant<D, true>(a.k, h, tk, tk < a.t_end, half, slot(s, 0), slot(s, 1), r);
+                    a2_fill_k<D>(a, h, tk, half, slot(s, 0), slot(s, 1), r);
                     fence_proxy_async_smem();
                     mbar_arrive(bar(s ? B_KFULL1 : B_KFULL0));
                 }
@@ -354,6 +402,7 @@ __global__ void __launch_bounds__(kA2Threads, 1) attention2_kernel(AttnArgs a)
             const uint32_t aQ[2] = {smem_u32(smem + L::offQ0), smem_u32(smem + L::offQ1)};
             const uint32_t aV = smem_u32(smem + L::offV);
             const uint32_t tS[2] = {tmem, tmem + 128}, tO[2] = {tmem + 256, tmem + 256 + D};
+            const int last_part = a.dense ? 0 : 1;  // dense keys have no lo part
             bool ok = a2_wait(bar(B_QREADY), 0, abort_flag);
             for (int j = 0; ok && j < ntiles; ++j) {
                 const int s = j & 1;
@@ -366,6 +415,8 @@ __global__ void __launch_bounds__(kA2Threads, 1) attention2_kernel(AttnArgs a)
                 // longer read and can take P_0; S_1 completes last (K_lo -> P_1)
 #pragma unroll
                 for (int part = 0; part < 2; ++part) {
+                    if (part > last_part)
+                        break;
 #pragma unroll
                     for (int qt = 0; qt < 2; ++qt) {
 #pragma unroll
@@ -374,7 +425,7 @@ __global__ void __launch_bounds__(kA2Threads, 1) attention2_kernel(AttnArgs a)
                             umma_ss(tS[qt], sdesc_sw128(aQ[qt] + off, 16, 1024),
                                     sdesc_sw128((part ? aKl : aKh) + off, 16, 1024), idescS, (part | ks) ? 1u : 0u);
                         }
-                        if (part == 1)
+                        if (part == last_part)
                             umma_commit(bar(qt ? B_SFULL1 : B_SFULL0));
                     }
                 }

@@ -27,6 +27,11 @@
 // S(j,i).  tcgen05 MMAs of one issuer run in order, so S(j+1,i) overwrites
 // P(j,i) in TMEM only after P V(j,i) has read it.
 //
+// Dense mode (uncompressed bf16 K and V, e.g. the current chunk): the same
+// pipeline with the staged rows copied straight into their slots; S takes
+// the K hi MMAs only and V is widened in place from bf16 to fp16 (exact in
+// fp16's normal range).
+//
 // Producers: each thread rebuilds 4 units (32 channels) of one K row and of
 // one V row per tile.  Two tiles ahead it stages, with per-thread
 // asynchronous copies, the centre rows of its units directly into their
@@ -265,6 +270,35 @@ __device__ __forceinline__ void ap_read_stage(const uint8_t *stage_cw, const uin
     }
 }
 
+// Dense mode: stage units [u0, u0 + 4) of row `tok` of a bf16 [Tk][H][128]
+// key or value array straight into their swizzled slots.
+__device__ __forceinline__ void ap_stage_dense(const uint16_t *x, int H, int h, int64_t tok, int u0, uint32_t tile,
+                                               const uint32_t *off)
+{
+    const uint16_t *src = x + (tok * H + h) * 128 + u0 * 8;
+#pragma unroll
+    for (int uu = 0; uu < 4; ++uu)
+        cp_async16(tile + off[uu], src + uu * 8);
+}
+
+// Dense mode, once the staged copies have landed: rows past the end become
+// zeros; V units (VALUE) are widened in place from bf16 to fp16.
+template <bool VALUE>
+__device__ __forceinline__ void ap_finish_dense(uint8_t *tile, const uint32_t *off, bool valid)
+{
+#pragma unroll
+    for (int uu = 0; uu < 4; ++uu) {
+        uint4 *dst = reinterpret_cast<uint4 *>(tile + off[uu]);
+        if (!valid) {
+            *dst = make_uint4(0, 0, 0, 0);
+        } else if (VALUE) {
+            const uint4 w = *dst;
+            *dst = make_uint4(pack_f16x2_sat(bf16_lo(w.x), bf16_hi(w.x)), pack_f16x2_sat(bf16_lo(w.y), bf16_hi(w.y)),
+                              pack_f16x2_sat(bf16_lo(w.z), bf16_hi(w.z)), pack_f16x2_sat(bf16_lo(w.w), bf16_hi(w.w)));
+        }
+    }
+}
+
 // Make the warp's generic-proxy writes visible to the tensor core, then one
 // lane arrives on the leader's barrier (cluster address).
 __device__ __forceinline__ void ap_publish(uint32_t lead_bar)
@@ -278,8 +312,9 @@ __device__ __forceinline__ void ap_publish(uint32_t lead_bar)
 // Producer loop over tiles i: rebuild K(i) and V(i), then stage K(i + 2)
 // once the QK of tile i - 1 has freed its stage and V(i + 2) once its P V
 // has.  One commit group per staging step (empty past the end), so "all but
-// the newest two groups" is always the pair K(i), V(i).
-template <int BK, int BV>
+// the newest two groups" is always the pair K(i), V(i).  DENSE: bf16 K and V
+// rows instead of codes (BK, BV unused).
+template <int BK, int BV, bool DENSE>
 __device__ __forceinline__ void ap_produce(const AttnArgs &a, int h, uint32_t rank, int tid, int ntiles,
                                            uint8_t *smem, uint64_t *bars, volatile int *abort_flag)
 {
@@ -307,24 +342,40 @@ __device__ __forceinline__ void ap_produce(const AttnArgs &a, int h, uint32_t ra
     auto ktok = [&](int i) { return a.t_begin + (int64_t)i * 128 + 64 * rank + krow; };
     auto vtok = [&](int i) { return a.t_begin + (int64_t)i * 128 + vrow; };
     auto kidx = [&](int i) {
-        const int64_t t = ktok(i);
-        return (i < ntiles && t < a.t_end) ? (int)__ldg(a.k.idx + (int64_t)h * a.k.T + t) : 0;
+        if constexpr (DENSE) {
+            return 0;
+        } else {
+            const int64_t t = ktok(i);
+            return (i < ntiles && t < a.t_end) ? (int)__ldg(a.k.idx + (int64_t)h * a.k.T + t) : 0;
+        }
     };
     auto vidx = [&](int i) {
-        const int64_t t = vtok(i);
-        return (i < ntiles && t < a.t_end) ? (int)__ldg(a.v.idx + (int64_t)h * a.v.T + t) : 0;
+        if constexpr (DENSE) {
+            return 0;
+        } else {
+            const int64_t t = vtok(i);
+            return (i < ntiles && t < a.t_end) ? (int)__ldg(a.v.idx + (int64_t)h * a.v.T + t) : 0;
+        }
     };
     auto stage_k = [&](int i, int j) {
         const int s = i % kAPStages;
-        if (ktok(i) < a.t_end)
-            ap_stage<BK>(a.k, h, ktok(i), j, ku0, smem_u32(khi(s)), koff, smem_u32(klo(s) + koff[0]),
-                         smem_u32(klo(s) + koff[1]));
+        if (ktok(i) < a.t_end) {
+            if constexpr (DENSE)
+                ap_stage_dense(a.k_dense, a.H, h, ktok(i), ku0, smem_u32(khi(s)), koff);
+            else
+                ap_stage<BK>(a.k, h, ktok(i), j, ku0, smem_u32(khi(s)), koff, smem_u32(klo(s) + koff[0]),
+                             smem_u32(klo(s) + koff[1]));
+        }
     };
     auto stage_v = [&](int i, int j) {
         const int s = i % kAPStages;
-        if (vtok(i) < a.t_end)
-            ap_stage<BV>(a.v, h, vtok(i), j, vu0, smem_u32(vst(s)), voff, smem_u32(klo(s) + koff[2]),
-                         smem_u32(klo(s) + koff[3]));
+        if (vtok(i) < a.t_end) {
+            if constexpr (DENSE)
+                ap_stage_dense(a.v_dense, a.H, h, vtok(i), vu0, smem_u32(vst(s)), voff);
+            else
+                ap_stage<BV>(a.v, h, vtok(i), j, vu0, smem_u32(vst(s)), voff, smem_u32(klo(s) + koff[2]),
+                             smem_u32(klo(s) + koff[3]));
+        }
     };
 
     // prologue: tiles 0 and 1
@@ -348,14 +399,21 @@ __device__ __forceinline__ void ap_produce(const AttnArgs &a, int h, uint32_t ra
         // two commit groups); V's staged words are read first: K lo is
         // overwritten by the K rebuild
         cp_async_wait<2>();
-        uint32_t kcw[4], vcw[4];
-        float2 ksz[4], vsz[4];
-        ap_read_stage<BK>(klo(s) + koff[0], klo(s) + koff[1], a.k.G, kcw, ksz);
-        ap_read_stage<BV>(klo(s) + koff[2], klo(s) + koff[3], a.v.G, vcw, vsz);
-        ap_rebuild<BK, true>(khi(s), klo(s), koff, kcw, ksz, ktok(i) < a.t_end);
-        ap_publish(lead(P_KFULL0 + s));
-        ap_rebuild<BV, false>(vst(s), nullptr, voff, vcw, vsz, vtok(i) < a.t_end);
-        ap_publish(lead(P_VFULL0 + s));
+        if constexpr (DENSE) {
+            ap_finish_dense<false>(khi(s), koff, ktok(i) < a.t_end);
+            ap_publish(lead(P_KFULL0 + s));
+            ap_finish_dense<true>(vst(s), voff, vtok(i) < a.t_end);
+            ap_publish(lead(P_VFULL0 + s));
+        } else {
+            uint32_t kcw[4], vcw[4];
+            float2 ksz[4], vsz[4];
+            ap_read_stage<BK>(klo(s) + koff[0], klo(s) + koff[1], a.k.G, kcw, ksz);
+            ap_read_stage<BV>(klo(s) + koff[2], klo(s) + koff[3], a.v.G, vcw, vsz);
+            ap_rebuild<BK, true>(khi(s), klo(s), koff, kcw, ksz, ktok(i) < a.t_end);
+            ap_publish(lead(P_KFULL0 + s));
+            ap_rebuild<BV, false>(vst(s), nullptr, voff, vcw, vsz, vtok(i) < a.t_end);
+            ap_publish(lead(P_VFULL0 + s));
+        }
         // (2) stage tile i + 2 into the stage of tile i - 1 once its QK (K) and
         // its P V (V) are done.  Issued after the publications above, whose
         // proxy fences then need not wait for these copies.
@@ -461,14 +519,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAPThreads, 1) atten
         }
         ap_publish(lead(P_QREADY));
         if (ntiles > 0) {
-            if (a.k.bits == 2 && a.v.bits == 2)
-                ap_produce<2, 2>(a, h, rank, tid, ntiles, smem, bars, abort_flag);
+            if (a.dense)
+                ap_produce<0, 0, true>(a, h, rank, tid, ntiles, smem, bars, abort_flag);
+            else if (a.k.bits == 2 && a.v.bits == 2)
+                ap_produce<2, 2, false>(a, h, rank, tid, ntiles, smem, bars, abort_flag);
             else if (a.k.bits == 2)
-                ap_produce<2, 4>(a, h, rank, tid, ntiles, smem, bars, abort_flag);
+                ap_produce<2, 4, false>(a, h, rank, tid, ntiles, smem, bars, abort_flag);
             else if (a.v.bits == 2)
-                ap_produce<4, 2>(a, h, rank, tid, ntiles, smem, bars, abort_flag);
+                ap_produce<4, 2, false>(a, h, rank, tid, ntiles, smem, bars, abort_flag);
             else
-                ap_produce<4, 4>(a, h, rank, tid, ntiles, smem, bars, abort_flag);
+                ap_produce<4, 4, false>(a, h, rank, tid, ntiles, smem, bars, abort_flag);
         }
     } else if (warp == kAPProducers / 32) {
         // ------------------------------------------------------------ MMA issuer (leader)
@@ -477,12 +537,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAPThreads, 1) atten
             constexpr uint32_t idescO = idesc_f32acc(256, D, false, false, true);
             const uint32_t aQ[2] = {smem_u32(smem + L::offQ), smem_u32(smem + L::offQ + L::kQ)};
             const uint32_t tS[2] = {tmem, tmem + 128}, tO[2] = {tmem + 256, tmem + 384};
+            const int nparts = a.dense ? 1 : 2;  // dense keys have no lo part
             // S(j, qt) = Q_qt (K_j hi + K_j lo)^T into tS[qt]
             auto issue_s = [&](int j, int qt) {
                 const int ks_ = j % kAPStages;
                 const uint32_t aK[2] = {smem_u32(ksl(ks_, 0)), smem_u32(ksl(ks_, 1))};
 #pragma unroll
                 for (int part = 0; part < 2; ++part) {
+                    if (part >= nparts)
+                        break;
 #pragma unroll
                     for (int ks = 0; ks < D / 16; ++ks) {
                         const uint32_t offa = (uint32_t)(ks >> 2) * (128u * 128u) + (uint32_t)(ks & 3) * 32u;

@@ -443,10 +443,24 @@ CodecView to_codec_view(const kvq_compressed_view *v)
 
 constexpr int kMaxAttnSplit = 4;
 
+// Partial-result buffers for `slots` binary32 partials: O slices
+// [slot][Tq][H][d], then (256-byte aligned) lse slices [slot][H][Tq].
+size_t partials_bytes(int slots, int H, int d, int64_t Tq)
+{
+    const size_t o = (size_t)slots * (size_t)Tq * H * d * 4;
+    return round_up(o, 256) + (size_t)slots * H * (size_t)Tq * 4;
+}
+
 size_t attention_workspace(const kvq_codec_desc *d, int64_t Tq)
 {
-    const size_t o = (size_t)kMaxAttnSplit * (size_t)Tq * d->num_heads * d->head_dim * 4;
-    return round_up(o, 256) + (size_t)kMaxAttnSplit * d->num_heads * (size_t)Tq * 4;
+    return partials_bytes(kMaxAttnSplit, d->num_heads, d->head_dim, Tq);
+}
+
+// Full-layer attention: up to kMaxAttnSplit partials for the compressed
+// history and as many for the dense keys.
+size_t layer_workspace(const kvq_codec_desc *d, int64_t Tq)
+{
+    return partials_bytes(2 * kMaxAttnSplit, d->num_heads, d->head_dim, Tq);
 }
 
 // Number of history sub-ranges for one attention call: the CTA count
@@ -520,6 +534,103 @@ kvq_status launch_attention2(const AttnArgs &a, cudaStream_t s)
     return launch_status();
 }
 
+
+// d = 128 runs on CTA pairs (512 query rows per pair), d = 64 on single CTAs.
+kvq_status launch_attention(const AttnArgs &a, int D, cudaStream_t s)
+{
+    return D == 128 ? launch_attention_pair(a, s) : launch_attention2<64>(a, s);
+}
+
+// Sub-ranges for one attention whose partials may go to a workspace.
+int attention_split_for(const AttnArgs &a, int D, int64_t span)
+{
+    const bool pair = D == 128;
+    return attention_splits(a.Tq, a.H, span, 1, 0, pair ? kAPRowsPerPair : kA2Rows, pair ? 2 : 1);
+}
+
+// Launch one attention with its key range split into `nsplit` sub-ranges,
+// writing binary32 partials: O to o_part[z] = o_part + z Tq H D and lse to
+// l_part + z H Tq, z < nsplit.
+kvq_status launch_attention_partials(AttnArgs a, int D, int nsplit, float *o_part, float *l_part, cudaStream_t s)
+{
+    a.o_out = o_part;
+    a.lse_out = l_part;
+    a.o_bf16 = 0;
+    a.nsplit = nsplit;
+    return launch_attention(a, D, s);
+}
+
+// One attention call into o_out / lse_out: unsplit, or split into partials
+// in the workspace and merged by LSE when that fills the GPU better.
+kvq_status attention_call(const AttnArgs &a, int D, void *workspace, size_t workspace_bytes, cudaStream_t s)
+{
+    const size_t need = partials_bytes(kMaxAttnSplit, a.H, D, a.Tq);
+    const int nsplit = (workspace && aligned16(workspace) && workspace_bytes >= need)
+                           ? attention_split_for(a, D, a.t_end - a.t_begin)
+                           : 1;
+    if (nsplit == 1)
+        return launch_attention(a, D, s);
+    float *o_part = static_cast<float *>(workspace);
+    float *l_part = reinterpret_cast<float *>(static_cast<uint8_t *>(workspace) +
+                                              round_up((size_t)kMaxAttnSplit * (size_t)a.Tq * a.H * D * 4, 256));
+    kvq_status st = launch_attention_partials(a, D, nsplit, o_part, l_part, s);
+    if (st != KVQ_OK)
+        return st;
+    MergeArgs m;
+    memset(&m, 0, sizeof m);
+    for (int z = 0; z < nsplit; ++z) {
+        m.o[z] = o_part + (int64_t)z * a.Tq * a.H * D;
+        m.lse[z] = l_part + (int64_t)z * a.H * a.Tq;
+    }
+    m.n = nsplit;
+    m.Tq = a.Tq;
+    m.H = a.H;
+    m.D = D;
+    m.o_out = a.o_out;
+    m.o_bf16 = a.o_bf16;
+    m.lse_out = a.lse_out;
+    launch_merge(m, s);
+    return launch_status();
+}
+
+// Checks shared by the compressed-history attention calls: two per-head
+// views with the same H, d and length, and [t_begin, t_end) inside them.
+kvq_status check_history_pair(const kvq_compressed_view *k, const kvq_compressed_view *v, int64_t t_begin,
+                              int64_t t_end)
+{
+    kvq_status st;
+    if ((st = check_view(k)) != KVQ_OK || (st = check_view(v)) != KVQ_OK)
+        return st;
+    if (k->desc.joint_rank > 0 || v->desc.joint_rank > 0)
+        return KVQ_ERR_UNSUPPORTED;
+    if (k->desc.num_heads != v->desc.num_heads || k->desc.head_dim != v->desc.head_dim ||
+        k->num_tokens != v->num_tokens)
+        return KVQ_ERR_INVALID_ARG;
+    if (t_begin < 0 || t_end < t_begin || t_end > k->num_tokens)
+        return KVQ_ERR_INVALID_ARG;
+    if (k->desc.num_heads > 65535)
+        return KVQ_ERR_UNSUPPORTED;
+    return KVQ_OK;
+}
+
+AttnArgs attn_args(const void *q, int64_t Tq, int H, int D, int64_t t_begin, int64_t t_end, float softmax_scale,
+                   void *o_out, kvq_dtype o_dtype, float *lse_out)
+{
+    AttnArgs a;
+    memset(&a, 0, sizeof a);
+    a.q = static_cast<const uint16_t *>(q);
+    a.Tq = Tq;
+    a.H = H;
+    a.t_begin = t_begin;
+    a.t_end = t_end;
+    const float scale = softmax_scale > 0.0f ? softmax_scale : 1.0f / sqrtf((float)D);
+    a.scale_log2 = scale * 1.4426950408889634f;
+    a.o_out = o_out;
+    a.o_bf16 = o_dtype == KVQ_BF16;
+    a.lse_out = lse_out;
+    a.nsplit = 1;
+    return a;
+}
 }  // namespace
 
 extern "C" {
@@ -576,6 +687,7 @@ kvq_status kvq_workspace_size(kvq_op op, const kvq_codec_desc *desc, int64_t T, 
     case KVQ_OP_ENCODE:
     case KVQ_OP_DECODE: *bytes = 0; return KVQ_OK;
     case KVQ_OP_ATTENTION: *bytes = attention_workspace(desc, Tq); return KVQ_OK;
+    case KVQ_OP_LAYER_ATTENTION: *bytes = layer_workspace(desc, Tq); return KVQ_OK;
     }
     return KVQ_ERR_INVALID_ARG;
 }
@@ -848,19 +960,10 @@ kvq_status kvq_attention_lse(const void *q, int64_t Tq, const kvq_compressed_vie
                              int64_t t_begin, int64_t t_end, float softmax_scale, void *o_out, kvq_dtype o_dtype,
                              float *lse_out, void *workspace, size_t workspace_bytes, kvq_stream_t stream)
 {
-    (void)workspace;
-    (void)workspace_bytes;
-    kvq_status st;
-    if ((st = check_view(k)) != KVQ_OK || (st = check_view(v)) != KVQ_OK)
+    kvq_status st = check_history_pair(k, v, t_begin, t_end);
+    if (st != KVQ_OK)
         return st;
-    if (k->desc.joint_rank > 0 || v->desc.joint_rank > 0)
-        return KVQ_ERR_UNSUPPORTED;
-    if (k->desc.num_heads != v->desc.num_heads || k->desc.head_dim != v->desc.head_dim ||
-        k->num_tokens != v->num_tokens)
-        return KVQ_ERR_INVALID_ARG;
-    if (Tq < 0 || t_begin < 0 || t_end < t_begin || t_end > k->num_tokens)
-        return KVQ_ERR_INVALID_ARG;
-    if (o_dtype != KVQ_F32 && o_dtype != KVQ_BF16)
+    if (Tq < 0 || (o_dtype != KVQ_F32 && o_dtype != KVQ_BF16))
         return KVQ_ERR_INVALID_ARG;
     if (Tq == 0)
         return KVQ_OK;
@@ -869,57 +972,89 @@ kvq_status kvq_attention_lse(const void *q, int64_t Tq, const kvq_compressed_vie
     if (!aligned16(q) || !aligned16(o_out) || !aligned16(lse_out))
         return KVQ_ERR_ALIGNMENT;
     const int D = k->desc.head_dim;
-    AttnArgs a;
-    a.q = static_cast<const uint16_t *>(q);
-    a.Tq = Tq;
-    a.H = k->desc.num_heads;
+    AttnArgs a = attn_args(q, Tq, k->desc.num_heads, D, t_begin, t_end, softmax_scale, o_out, o_dtype, lse_out);
     a.k = to_codec_view(k);
     a.v = to_codec_view(v);
-    a.t_begin = t_begin;
-    a.t_end = t_end;
-    const float scale = softmax_scale > 0.0f ? softmax_scale : 1.0f / sqrtf((float)D);
-    a.scale_log2 = scale * 1.4426950408889634f;
-    a.o_out = o_out;
-    a.o_bf16 = o_dtype == KVQ_BF16;
-    a.lse_out = lse_out;
-    a.nsplit = 1;
+    return attention_call(a, D, workspace, workspace_bytes, reinterpret_cast<cudaStream_t>(stream));
+}
+
+kvq_status kvq_attention_dense_lse(const void *q, int64_t Tq, const void *k, const void *v, int64_t num_keys,
+                                   int32_t H, int32_t d, int64_t t_begin, int64_t t_end, float softmax_scale,
+                                   void *o_out, kvq_dtype o_dtype, float *lse_out, void *workspace,
+                                   size_t workspace_bytes, kvq_stream_t stream)
+{
+    if (H < 1 || Tq < 0 || num_keys < 0 || t_begin < 0 || t_end < t_begin || t_end > num_keys)
+        return KVQ_ERR_INVALID_ARG;
+    if (!supported_dim(d) || H > 65535)
+        return KVQ_ERR_UNSUPPORTED;
+    if (o_dtype != KVQ_F32 && o_dtype != KVQ_BF16)
+        return KVQ_ERR_INVALID_ARG;
+    if (Tq == 0)
+        return KVQ_OK;
+    if (!q || !o_out || !lse_out || (t_end > t_begin && (!k || !v)))
+        return KVQ_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(o_out) || !aligned16(lse_out) || !aligned16(k) || !aligned16(v))
+        return KVQ_ERR_ALIGNMENT;
+    AttnArgs a = attn_args(q, Tq, H, d, t_begin, t_end, softmax_scale, o_out, o_dtype, lse_out);
+    a.dense = 1;
+    a.k_dense = static_cast<const uint16_t *>(k);
+    a.v_dense = static_cast<const uint16_t *>(v);
+    return attention_call(a, d, workspace, workspace_bytes, reinterpret_cast<cudaStream_t>(stream));
+}
+
+kvq_status kvq_layer_attention(const void *q, int64_t Tq, const kvq_compressed_view *k_hist,
+                               const kvq_compressed_view *v_hist, int64_t t_begin, int64_t t_end, const void *k_cur,
+                               const void *v_cur, int64_t num_cur, float softmax_scale, void *o_out,
+                               kvq_dtype o_dtype, float *lse_out, void *workspace, size_t workspace_bytes,
+                               kvq_stream_t stream)
+{
+    kvq_status st = check_history_pair(k_hist, v_hist, t_begin, t_end);
+    if (st != KVQ_OK)
+        return st;
+    if (Tq < 0 || num_cur < 0 || (o_dtype != KVQ_F32 && o_dtype != KVQ_BF16))
+        return KVQ_ERR_INVALID_ARG;
+    if (Tq == 0)
+        return KVQ_OK;
+    if (!q || !o_out || !lse_out || (num_cur > 0 && (!k_cur || !v_cur)))
+        return KVQ_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(o_out) || !aligned16(lse_out) || !aligned16(k_cur) || !aligned16(v_cur) ||
+        !aligned16(workspace))
+        return KVQ_ERR_ALIGNMENT;
+    const int H = k_hist->desc.num_heads, D = k_hist->desc.head_dim;
+    if (!workspace || workspace_bytes < layer_workspace(&k_hist->desc, Tq))
+        return KVQ_ERR_WORKSPACE;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    const size_t need = attention_workspace(&k->desc, Tq);
-    // d = 128 runs on CTA pairs (512 query rows per pair), d = 64 on single CTAs
-    const bool pair = D == 128;
-    auto launch = [&](const AttnArgs &x) {
-        return pair ? launch_attention_pair(x, s) : launch_attention2<64>(x, s);
-    };
-    const int nsplit = (workspace && aligned16(workspace))
-                           ? attention_splits(Tq, a.H, t_end - t_begin, workspace_bytes, need,
-                                              pair ? kAPRowsPerPair : kA2Rows, pair ? 2 : 1)
-                           : 1;
-    if (nsplit == 1)
-        return launch(a);
-    // history split across CTAs: binary32 partials in the workspace, merged by LSE
+    AttnArgs hist = attn_args(q, Tq, H, D, t_begin, t_end, softmax_scale, o_out, o_dtype, lse_out);
+    hist.k = to_codec_view(k_hist);
+    hist.v = to_codec_view(v_hist);
+    AttnArgs cur = attn_args(q, Tq, H, D, 0, num_cur, softmax_scale, o_out, o_dtype, lse_out);
+    cur.dense = 1;
+    cur.k_dense = static_cast<const uint16_t *>(k_cur);
+    cur.v_dense = static_cast<const uint16_t *>(v_cur);
+    // partials: history in slots [0, nh), dense keys in [nh, nh + nc)
+    const int nh = attention_split_for(hist, D, t_end - t_begin);
+    const int nc = attention_split_for(cur, D, num_cur);
+    const int64_t slice = Tq * (int64_t)H * D;
     float *o_part = static_cast<float *>(workspace);
     float *l_part = reinterpret_cast<float *>(static_cast<uint8_t *>(workspace) +
-                                              round_up((size_t)kMaxAttnSplit * (size_t)Tq * a.H * D * 4, 256));
-    AttnArgs ap = a;
-    ap.o_out = o_part;
-    ap.lse_out = l_part;
-    ap.o_bf16 = 0;
-    ap.nsplit = nsplit;
-    st = launch(ap);
-    if (st != KVQ_OK)
+                                              round_up((size_t)(2 * kMaxAttnSplit) * (size_t)slice * 4, 256));
+    if ((st = launch_attention_partials(hist, D, nh, o_part, l_part, s)) != KVQ_OK)
+        return st;
+    if ((st = launch_attention_partials(cur, D, nc, o_part + nh * slice, l_part + (int64_t)nh * H * Tq, s)) !=
+        KVQ_OK)
         return st;
     MergeArgs m;
     memset(&m, 0, sizeof m);
-    for (int z = 0; z < nsplit; ++z) {
-        m.o[z] = o_part + (int64_t)z * Tq * a.H * D;
-        m.lse[z] = l_part + (int64_t)z * a.H * Tq;
+    for (int z = 0; z < nh + nc; ++z) {
+        m.o[z] = o_part + z * slice;
+        m.lse[z] = l_part + (int64_t)z * H * Tq;
     }
-    m.n = nsplit;
+    m.n = nh + nc;
     m.Tq = Tq;
-    m.H = a.H;
+    m.H = H;
     m.D = D;
     m.o_out = o_out;
-    m.o_bf16 = a.o_bf16;
+    m.o_bf16 = o_dtype == KVQ_BF16;
     m.lse_out = lse_out;
     launch_merge(m, s);
     return launch_status();

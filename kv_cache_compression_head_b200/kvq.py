@@ -34,11 +34,13 @@ KVQ_OP_FIT = 0
 KVQ_OP_ENCODE = 1
 KVQ_OP_DECODE = 2
 KVQ_OP_ATTENTION = 3
+KVQ_OP_LAYER_ATTENTION = 4
 
 EXPORTED = (
     "kvq_status_string", "kvq_encoded_sizes", "kvq_workspace_size", "kvq_fit_centroids",
     "kvq_fit_centroids_static", "kvq_encode",
-    "kvq_joint_coefficients", "kvq_decode", "kvq_attention_lse", "kvq_lse_merge", "kvq_last_device_status",
+    "kvq_joint_coefficients", "kvq_decode", "kvq_attention_lse", "kvq_attention_dense_lse", "kvq_layer_attention",
+    "kvq_lse_merge", "kvq_last_device_status",
 )
 
 
@@ -76,6 +78,10 @@ def _load():
         "kvq_joint_coefficients": [pdesc, vp, ctypes.c_int, i64, vp, vp, vp, vp, vp, sz, vp],
         "kvq_decode": [pview, vp, ctypes.c_int, vp, sz, vp],
         "kvq_attention_lse": [vp, i64, pview, pview, i64, i64, ctypes.c_float, vp, ctypes.c_int, vp, vp, sz, vp],
+        "kvq_attention_dense_lse": [vp, i64, vp, vp, i64, i32, i32, i64, i64, ctypes.c_float, vp, ctypes.c_int, vp,
+                                    vp, sz, vp],
+        "kvq_layer_attention": [vp, i64, pview, pview, i64, i64, vp, vp, i64, ctypes.c_float, vp, ctypes.c_int, vp,
+                                vp, sz, vp],
         "kvq_lse_merge": [i32, ctypes.POINTER(vp), ctypes.POINTER(vp), i64, i32, i32, vp, ctypes.c_int, vp, vp],
         "kvq_last_device_status": [vp],
     }
@@ -248,6 +254,41 @@ def kvq_attention_lse(q: torch.Tensor, k: Compressed, v: Compressed, o_out: torc
                                   softmax_scale, _ptr(o_out), _dtype_code(o_out), _ptr(lse_out), _ptr(workspace),
                                   workspace.numel() if workspace is not None else 0, _stream(stream)),
            "kvq_attention_lse")
+
+
+def kvq_attention_dense_lse(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, o_out: torch.Tensor,
+                            lse_out: torch.Tensor, t_begin: int = 0, t_end: Optional[int] = None,
+                            softmax_scale: float = 0.0, workspace: Optional[torch.Tensor] = None, stream=None) -> None:
+    """Attention over uncompressed bf16 keys/values k, v [Tk][H][d]."""
+    Tk, H, d = k.shape
+    if t_end is None:
+        t_end = Tk
+    _check(_lib.kvq_attention_dense_lse(_ptr(q), q.shape[0], _ptr(k), _ptr(v), Tk, H, d, t_begin, t_end,
+                                        softmax_scale, _ptr(o_out), _dtype_code(o_out), _ptr(lse_out),
+                                        _ptr(workspace), workspace.numel() if workspace is not None else 0,
+                                        _stream(stream)),
+           "kvq_attention_dense_lse")
+
+
+def kvq_layer_attention(q: torch.Tensor, k_hist: Compressed, v_hist: Compressed, k_cur: Optional[torch.Tensor],
+                        v_cur: Optional[torch.Tensor], o_out: torch.Tensor, lse_out: torch.Tensor,
+                        workspace: Optional[torch.Tensor] = None, t_begin: int = 0, t_end: Optional[int] = None,
+                        softmax_scale: float = 0.0, stream=None) -> None:
+    """One softmax over the compressed history and the uncompressed keys
+    k_cur, v_cur [Tc][H][d] (the current chunk and any raw protected tokens).
+    The call needs a workspace; one is allocated when none is given."""
+    if t_end is None:
+        t_end = k_hist.num_tokens
+    if workspace is None:
+        workspace = alloc_workspace(KVQ_OP_LAYER_ATTENTION, k_hist.codec, k_hist.num_tokens, q.device,
+                                    num_queries=q.shape[0])
+    n_cur = 0 if k_cur is None else k_cur.shape[0]
+    kv, vv = k_hist.view(), v_hist.view()
+    _check(_lib.kvq_layer_attention(_ptr(q), q.shape[0], ctypes.byref(kv), ctypes.byref(vv), t_begin, t_end,
+                                    _ptr(k_cur), _ptr(v_cur), n_cur, softmax_scale, _ptr(o_out), _dtype_code(o_out),
+                                    _ptr(lse_out), _ptr(workspace), workspace.numel() if workspace is not None else 0,
+                                    _stream(stream)),
+           "kvq_layer_attention")
 
 
 def kvq_lse_merge(o_parts: Sequence[torch.Tensor], lse_parts: Sequence[torch.Tensor], o_out: torch.Tensor,

@@ -32,6 +32,7 @@ __all__ = [
     "workload",
     "make_history",
     "make_queries",
+    "make_chunk",
     "make_orthonormal_encoder",
     "bf16_bits_from_f64",
     "bf16_bits_to_f32",
@@ -248,6 +249,21 @@ def make_queries(w: Workload, max_tokens: Optional[int] = None) -> np.ndarray:
     frames = _frames_for(w, 2, Tq, False)
     ww = dataclasses.replace(w, dtype="bf16")
     return _collect(ww, frames, Tq, w.num_heads, w.head_dim, max_tokens)
+
+
+def make_chunk(w: Workload, which: str, max_tokens: Optional[int] = None) -> np.ndarray:
+    """The current chunk's own keys ('K') or values ('V'), [Tq][H][d]: the
+    Tq tokens that follow the history in the same random stream (the next
+    frames of the same process), uncompressed, in the workload dtype."""
+    stream = {"K": 0, "V": 1}[which]
+    T, Tq = w.history_tokens, w.query_tokens
+    if w.generator == "smooth":
+        ww = dataclasses.replace(w, frames=w.frames + -(-Tq // w.tokens_per_frame))
+        frames = _frames_for(ww, stream, ww.history_tokens, True)
+    else:
+        frames = _frames_for(w, stream, T + Tq, True)
+    out = _collect(w, frames, T + Tq, w.num_heads, w.head_dim, None)[T:]
+    return np.ascontiguousarray(out if max_tokens is None else out[:max_tokens])
 
 
 def make_orthonormal_encoder(w: Workload, seed_stream: int = 3) -> np.ndarray:

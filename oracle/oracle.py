@@ -18,6 +18,10 @@ Functions and the passages they follow:
   log-sum-exp of the logits (NanoKV page, Fig. 4(a,d)).
 * ``lse_merge``: combination of partial attention results over history parts
   by their log-sum-exp (NanoKV page, Fig. 4(d)).
+* ``layer_attention``: the current chunk's full attention -- one softmax over
+  the reconstructed history and the uncompressed keys of the chunk itself
+  (and of any raw protected tokens; NanoKV page, Table 4), written as plain
+  attention over the union of both key sets (NanoKV page, Fig. 4(a,d)).
 * ``stored_bytes_per_token_head`` / ``bits_per_value``: storage accounting.
 """
 
@@ -229,7 +233,8 @@ def attention(q: np.ndarray, k: np.ndarray, v: np.ndarray, scale: Optional[float
               rows: Optional[np.ndarray] = None) -> Tuple[np.ndarray, np.ndarray]:
     """Softmax attention of queries over a (reconstructed) history.
 
-    q [Tq][H][d] (bf16 bits or float), k, v [T][H][d] float32 reconstructions.
+    q [Tq][H][d] (bf16 bits or float), k, v [T][H][d] float32 reconstructions
+    (or bf16 bits: uncompressed keys and values).
     Logits s_ij = scale * q_i . k_j with scale = 1/sqrt(d) unless given; no
     mask (the history strictly precedes the current chunk).
     Returns O [n][H][d] float64 and lse [H][n] float64 (natural log), where n
@@ -239,8 +244,8 @@ def attention(q: np.ndarray, k: np.ndarray, v: np.ndarray, scale: Optional[float
     qf = _widen(q)
     if rows is not None:
         qf = qf[rows]
-    kf = k.astype(np.float64)
-    vf = v.astype(np.float64)
+    kf = _widen(k)
+    vf = _widen(v)
     n, H, d = qf.shape
     T = kf.shape[0]
     sc = 1.0 / math.sqrt(d) if scale is None else float(scale)
@@ -256,6 +261,20 @@ def attention(q: np.ndarray, k: np.ndarray, v: np.ndarray, scale: Optional[float
         O[:, h, :] = (p @ vf[:, h, :]) / l
         lse[h, :] = (m + np.log(l))[:, 0]
     return O, lse
+
+
+def layer_attention(q: np.ndarray, k_hist: np.ndarray, v_hist: np.ndarray, k_cur: np.ndarray, v_cur: np.ndarray,
+                    scale: Optional[float] = None, rows: Optional[np.ndarray] = None) -> Tuple[np.ndarray, np.ndarray]:
+    """Full attention of the current chunk's queries: one softmax over the
+    history keys k_hist [T][H][d] (float32 reconstructions) together with the
+    uncompressed keys k_cur [Tc][H][d] (bf16 bits or float), values likewise.
+    The plain definition: attention over the union of the two key sets (the
+    order of keys does not change a softmax-weighted sum).  Returns O [n][H][d]
+    and lse [H][n] as ``attention`` does.
+    """
+    k = np.concatenate([_widen(k_hist), _widen(k_cur)], axis=0)
+    v = np.concatenate([_widen(v_hist), _widen(v_cur)], axis=0)
+    return attention(q, k, v, scale, rows)
 
 
 def lse_merge(o_parts: Sequence[np.ndarray], lse_parts: Sequence[np.ndarray]) -> Tuple[np.ndarray, np.ndarray]:

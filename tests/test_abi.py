@@ -134,6 +134,50 @@ def test_bad_pointers_and_sizes_rejected_on_host(K):
     assert K.workspace_size(K.KVQ_OP_ENCODE, K.Codec(12, 128, 256, 4, 32, 192), 32760) == 0
 
 
+def test_dense_and_layer_attention_rejected_on_host(K):
+    A = 1 << 20
+    f0 = ctypes.c_float(0)
+    dense = lambda *a: _err(K, "kvq_attention_dense_lse", *a)
+    # range outside the keys, unsupported head dim, too many heads, bad dtype
+    assert dense(A, 10, A, A, 100, 12, 128, 0, 101, f0, A, K.KVQ_F32, A, None, 0, None) == K.KVQ_ERR_INVALID_ARG
+    assert dense(A, 10, A, A, 100, 12, 96, 0, 100, f0, A, K.KVQ_F32, A, None, 0, None) == K.KVQ_ERR_UNSUPPORTED
+    assert dense(A, 10, A, A, 100, 70000, 128, 0, 100, f0, A, K.KVQ_F32, A, None, 0, None) \
+        == K.KVQ_ERR_UNSUPPORTED
+    assert dense(A, 10, A, A, 100, 0, 128, 0, 100, f0, A, K.KVQ_F32, A, None, 0, None) == K.KVQ_ERR_INVALID_ARG
+    assert dense(A, 10, A, A, 100, 12, 128, 0, 100, f0, A, 7, A, None, 0, None) == K.KVQ_ERR_INVALID_ARG
+    # null keys with a non-empty range; misaligned values
+    assert dense(A, 10, None, A, 100, 12, 128, 0, 100, f0, A, K.KVQ_F32, A, None, 0, None) \
+        == K.KVQ_ERR_INVALID_ARG
+    assert dense(A, 10, A, A + 2, 100, 12, 128, 0, 100, f0, A, K.KVQ_F32, A, None, 0, None) == K.KVQ_ERR_ALIGNMENT
+    assert dense(None, 0, None, None, 0, 12, 128, 0, 0, f0, None, K.KVQ_F32, None, None, 0, None) == K.KVQ_OK
+
+    d = K.CodecDesc(12, 128, 256, 2, 16, 0)
+    v = K.CompressedView(d, 1000, A, A, A, A, None)
+    dj = K.CompressedView(K.CodecDesc(12, 128, 256, 4, 32, 192), 1000, A, A, A, A, A)
+    layer = lambda *a: _err(K, "kvq_layer_attention", *a)
+    need = K.workspace_size(K.KVQ_OP_LAYER_ATTENTION, K.Codec(12, 128, 256, 2, 16), 1000, 10)
+    # eight binary32 partials of O [10][12][128] and of lse [12][10]
+    assert need == 8 * 10 * 12 * 128 * 4 + 8 * 12 * 10 * 4
+    ok_args = (A, 10, ctypes.byref(v), ctypes.byref(v), 0, 1000, A, A, 50, f0, A, K.KVQ_F32, A)
+    # workspace missing or short
+    assert layer(*ok_args, None, 0, None) == K.KVQ_ERR_WORKSPACE
+    assert layer(*ok_args, A, need - 1, None) == K.KVQ_ERR_WORKSPACE
+    assert layer(*ok_args[:-1], A + 4, A, need, None) == K.KVQ_ERR_ALIGNMENT
+    # joint history, history range outside it, chunk keys missing, negative chunk length
+    assert layer(A, 10, ctypes.byref(dj), ctypes.byref(dj), 0, 1000, A, A, 50, f0, A, K.KVQ_F32, A, A, need,
+                 None) == K.KVQ_ERR_UNSUPPORTED
+    assert layer(A, 10, ctypes.byref(v), ctypes.byref(v), 0, 1001, A, A, 50, f0, A, K.KVQ_F32, A, A, need,
+                 None) == K.KVQ_ERR_INVALID_ARG
+    assert layer(A, 10, ctypes.byref(v), ctypes.byref(v), 0, 1000, None, A, 50, f0, A, K.KVQ_F32, A, A, need,
+                 None) == K.KVQ_ERR_INVALID_ARG
+    assert layer(A, 10, ctypes.byref(v), ctypes.byref(v), 0, 1000, A, A, -1, f0, A, K.KVQ_F32, A, A, need,
+                 None) == K.KVQ_ERR_INVALID_ARG
+    assert layer(A, 10, ctypes.byref(v), ctypes.byref(v), 0, 1000, A, A + 8, 50, f0, A, K.KVQ_F32, A, A, need,
+                 None) == K.KVQ_ERR_ALIGNMENT
+    assert layer(None, 0, ctypes.byref(v), ctypes.byref(v), 0, 1000, None, None, 0, f0, None, K.KVQ_F32, None,
+                 None, 0, None) == K.KVQ_OK
+
+
 def test_binding_refuses_to_load_without_the_library(tmp_path):
     """A copy of the package without libkvq.so: importing the binding raises
     (the product path has no fallback)."""

@@ -444,3 +444,74 @@ def test_merge_with_empty_parts():
     assert np.allclose(o, o1, atol=1e-15) and np.allclose(l, l1, atol=1e-15)
     o, l = O.lse_merge([o_empty, o_empty], [l_empty, l_empty])
     assert np.all(l == -np.inf) and np.all(o == 0)
+
+
+# ----------------------------------------------------------------------------
+# full-layer attention: compressed history + uncompressed current chunk
+# ----------------------------------------------------------------------------
+
+def test_layer_attention_matches_library_sdpa_over_all_keys():
+    """One softmax over history and chunk keys: torch's SDPA over the union
+    (chunk keys first, history after -- a different order from the oracle's)
+    and scipy's logsumexp of the logits."""
+    from scipy.special import logsumexp
+
+    rng = np.random.default_rng(21)
+    Tq, T, Tc, H, d = 29, 211, 45, 3, 64
+    q = _bf16(rng.normal(size=(Tq, H, d)))
+    kh = (rng.normal(size=(T, H, d)) * 1.5).astype(np.float32)
+    vh = rng.normal(size=(T, H, d)).astype(np.float32)
+    kc = _bf16(rng.normal(size=(Tc, H, d)) * 1.5)
+    vc = _bf16(rng.normal(size=(Tc, H, d)))
+    o, lse = O.layer_attention(q, kh, vh, kc, vc)
+    kall = np.concatenate([_widen(kc), kh]).astype(np.float64)
+    vall = np.concatenate([_widen(vc), vh]).astype(np.float64)
+    qt = torch.from_numpy(_widen(q).astype(np.float64)).permute(1, 0, 2)
+    ref = torch.nn.functional.scaled_dot_product_attention(
+        qt, torch.from_numpy(kall).permute(1, 0, 2), torch.from_numpy(vall).permute(1, 0, 2)).permute(1, 0, 2)
+    assert np.max(np.abs(o - ref.numpy())) < 1e-12
+    s = np.einsum("qhd,khd->hqk", _widen(q).astype(np.float64), kall) / math.sqrt(d)
+    assert np.max(np.abs(lse - logsumexp(s, axis=2))) < 1e-12
+
+
+def test_layer_attention_reads_chunk_as_bf16_and_handles_empty_sets():
+    rng = np.random.default_rng(22)
+    Tq, T, Tc, H, d = 9, 40, 17, 2, 64
+    q = _bf16(rng.normal(size=(Tq, H, d)))
+    kh = rng.normal(size=(T, H, d)).astype(np.float32)
+    vh = rng.normal(size=(T, H, d)).astype(np.float32)
+    kc = _bf16(rng.normal(size=(Tc, H, d)))
+    vc = _bf16(rng.normal(size=(Tc, H, d)))
+    # bf16 bits and the same values as float32 give the same result
+    o1, l1 = O.layer_attention(q, kh, vh, kc, vc)
+    o2, l2 = O.layer_attention(q, kh, vh, _widen(kc), _widen(vc))
+    assert np.array_equal(o1, o2) and np.array_equal(l1, l2)
+    # empty chunk: the history alone; empty history: the chunk alone
+    none = np.zeros((0, H, d), np.float32)
+    oh, lh = O.layer_attention(q, kh, vh, none, none)
+    oa, la = O.attention(q, kh, vh)
+    assert np.array_equal(oh, oa) and np.array_equal(lh, la)
+    oc, lc = O.layer_attention(q, none, none, kc, vc)
+    s = np.einsum("qhd,khd->hqk", _widen(q).astype(np.float64), _widen(kc).astype(np.float64)) / 8.0
+    m = s.max(axis=2, keepdims=True)
+    assert np.allclose(lc, (m + np.log(np.exp(s - m).sum(axis=2, keepdims=True)))[..., 0], atol=1e-13)
+    # both empty: O = 0, lse = -inf
+    oz, lz = O.layer_attention(q, none, none, none, none)
+    assert np.all(oz == 0) and np.all(lz == -np.inf)
+
+
+def test_layer_attention_is_the_merge_of_history_and_chunk():
+    """Splitting the keys into the history part and the chunk part and
+    merging by LSE gives the layer result (the identity the GPU path uses)."""
+    rng = np.random.default_rng(23)
+    Tq, T, Tc, H, d = 12, 130, 33, 2, 128
+    q = _bf16(rng.normal(size=(Tq, H, d)))
+    kh = (rng.normal(size=(T, H, d)) * 2).astype(np.float32)
+    vh = rng.normal(size=(T, H, d)).astype(np.float32)
+    kc = _bf16(rng.normal(size=(Tc, H, d)) * 2)
+    vc = _bf16(rng.normal(size=(Tc, H, d)))
+    o, lse = O.layer_attention(q, kh, vh, kc, vc)
+    ph = O.attention(q, kh, vh)
+    pc = O.attention(q, kc, vc)
+    om, lm = O.lse_merge([ph[0], pc[0]], [ph[1], pc[1]])
+    assert np.max(np.abs(o - om)) < 1e-12 and np.max(np.abs(lse - lm)) < 1e-12

@@ -46,8 +46,9 @@ HISTORY_BLOCKS = 2
 FLUSH_BYTES = 256 << 20
 # DRAM bytes (read + write) of one attention_pair_kernel launch of this
 # workload, from the ncu capture summarised in profiles/attention_pair_wan13b.md;
-# None whenever the kernel has changed since that capture.
-ATTN_NCU_TRAFFIC_BYTES = 56_144_640 + 37_984_000
+# None whenever the kernel has changed since that capture.  The last capture
+# (92.6 MB per launch) predates the per-codec instantiation of the kernel.
+ATTN_NCU_TRAFFIC_BYTES = None
 
 
 def _joint():
@@ -502,8 +503,8 @@ def run_gpu(args):
                        "heads": w.num_heads, "head_dim": w.head_dim, "centroids": w.num_centroids,
                        "bits_k": w.bits_k, "bits_v": w.bits_v, "group": w.group_size,
                        "parallelism": f"replicas x{world}", "l2": "flushed (256 MiB write) before each step"},
-            "roofline": {"kernel": "attention_pair_kernel (time of the whole kvq_attention_lse call, incl. its "
-                                   "in-call LSE merge)", "bound": "tensor", "achieved": attn_tflops,
+            "roofline": {"kernel": "attention_pair_kernel<2, 2, false> (time of the whole kvq_attention_lse call, "
+                                   "incl. its in-call LSE merge)", "bound": "tensor", "achieved": attn_tflops,
                          "peak": tfl, "unit": "TFLOP/s", "frac": attn_tflops / tfl, "peak_kind": peak_kind,
                          "traffic": ATTN_NCU_TRAFFIC_BYTES,
                          "traffic_unit": "bytes per launch (ncu dram__bytes_read.sum + dram__bytes_write.sum)"},

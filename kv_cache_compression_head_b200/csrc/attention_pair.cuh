@@ -441,6 +441,9 @@ __device__ __forceinline__ void ap_produce(const AttnArgs &a, int h, uint32_t ra
     cp_async_wait<0>();
 }
 
+// One instantiation per (K bits, V bits) of a compressed history, and one for
+// dense keys and values (BK = BV = 0), so that each carries only its producer.
+template <int BK, int BV, bool DENSE>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAPThreads, 1) attention_pair_kernel(AttnArgs a)
 {
     constexpr int D = 128;
@@ -518,18 +521,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAPThreads, 1) atten
             }
         }
         ap_publish(lead(P_QREADY));
-        if (ntiles > 0) {
-            if (a.dense)
-                ap_produce<0, 0, true>(a, h, rank, tid, ntiles, smem, bars, abort_flag);
-            else if (a.k.bits == 2 && a.v.bits == 2)
-                ap_produce<2, 2, false>(a, h, rank, tid, ntiles, smem, bars, abort_flag);
-            else if (a.k.bits == 2)
-                ap_produce<2, 4, false>(a, h, rank, tid, ntiles, smem, bars, abort_flag);
-            else if (a.v.bits == 2)
-                ap_produce<4, 2, false>(a, h, rank, tid, ntiles, smem, bars, abort_flag);
-            else
-                ap_produce<4, 4, false>(a, h, rank, tid, ntiles, smem, bars, abort_flag);
-        }
+        if (ntiles > 0)
+            ap_produce<BK, BV, DENSE>(a, h, rank, tid, ntiles, smem, bars, abort_flag);
     } else if (warp == kAPProducers / 32) {
         // ------------------------------------------------------------ MMA issuer (leader)
         if (rank == 0 && lane == 0 && ntiles > 0) {
@@ -537,15 +530,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAPThreads, 1) atten
             constexpr uint32_t idescO = idesc_f32acc(256, D, false, false, true);
             const uint32_t aQ[2] = {smem_u32(smem + L::offQ), smem_u32(smem + L::offQ + L::kQ)};
             const uint32_t tS[2] = {tmem, tmem + 128}, tO[2] = {tmem + 256, tmem + 384};
-            const int nparts = a.dense ? 1 : 2;  // dense keys have no lo part
+            constexpr int nparts = DENSE ? 1 : 2;  // dense keys have no lo part
             // S(j, qt) = Q_qt (K_j hi + K_j lo)^T into tS[qt]
             auto issue_s = [&](int j, int qt) {
                 const int ks_ = j % kAPStages;
                 const uint32_t aK[2] = {smem_u32(ksl(ks_, 0)), smem_u32(ksl(ks_, 1))};
 #pragma unroll
-                for (int part = 0; part < 2; ++part) {
-                    if (part >= nparts)
-                        break;
+                for (int part = 0; part < nparts; ++part) {
 #pragma unroll
                     for (int ks = 0; ks < D / 16; ++ks) {
                         const uint32_t offa = (uint32_t)(ks >> 2) * (128u * 128u) + (uint32_t)(ks & 3) * 32u;

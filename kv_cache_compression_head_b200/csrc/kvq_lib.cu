@@ -497,22 +497,32 @@ void launch_merge(const MergeArgs &m, cudaStream_t s)
         lse_merge_kernel<64><<<dim3((unsigned)ceil_div(m.Tq, 256 / 16), (unsigned)m.H), 256, 0, s>>>(m);
 }
 
-kvq_status launch_attention_pair(const AttnArgs &a, cudaStream_t s)
+template <int BK, int BV, bool DENSE>
+kvq_status launch_attention_pair_t(const AttnArgs &a, cudaStream_t s)
 {
     static bool configured[64] = {};
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64)
         return KVQ_ERR_CUDA;
     if (!configured[dev]) {
-        if (cudaFuncSetAttribute(attention_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        if (cudaFuncSetAttribute(attention_pair_kernel<BK, BV, DENSE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  (int)APSmem::kLaunchBytes) != cudaSuccess)
             return KVQ_ERR_CUDA;
         configured[dev] = true;
     }
     const dim3 grid((unsigned)(2 * ceil_div(a.Tq, kAPRowsPerPair)), (unsigned)a.H,
                     (unsigned)(a.nsplit > 1 ? a.nsplit : 1));
-    attention_pair_kernel<<<grid, kAPThreads, APSmem::kLaunchBytes, s>>>(a);
+    attention_pair_kernel<BK, BV, DENSE><<<grid, kAPThreads, APSmem::kLaunchBytes, s>>>(a);
     return launch_status();
+}
+
+kvq_status launch_attention_pair(const AttnArgs &a, cudaStream_t s)
+{
+    if (a.dense)
+        return launch_attention_pair_t<0, 0, true>(a, s);
+    if (a.k.bits == 2)
+        return a.v.bits == 2 ? launch_attention_pair_t<2, 2, false>(a, s) : launch_attention_pair_t<2, 4, false>(a, s);
+    return a.v.bits == 2 ? launch_attention_pair_t<4, 2, false>(a, s) : launch_attention_pair_t<4, 4, false>(a, s);
 }
 
 template <int D>

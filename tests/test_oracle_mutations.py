@@ -2,7 +2,9 @@
 mistake in a copy of the C oracle (a dropped term, a flipped sign, a wrong
 index or bit order, a wrong tie rule, a skipped rounding), builds it, points
 the oracle wrapper at it and checks that at least one pin of
-tests/test_oracle_pins.py fails.  CPU only; the real oracle is restored after
+tests/test_oracle_pins.py fails.  The NumPy attention, merge and full-layer
+attention get the same treatment: a mutated copy of the function's source
+replaces it while the pins run.  CPU only; the real oracle is restored after
 every case."""
 
 import inspect
@@ -76,3 +78,41 @@ def test_pins_catch_planted_mistake(name, old, new):
 def test_unmutated_oracle_passes_every_pin():
     for _, pin in _pins():
         pin()
+
+
+# (function in oracle.py, name, text in its source, replacement): mistakes
+# planted in the NumPy attention, merge and full-layer attention
+PY_MUTATIONS = [
+    ("attention", "softmax scale dropped", "@ kf[:, h, :].T) * sc", "@ kf[:, h, :].T)"),
+    ("attention", "keys of head 0 for every head", "qf[:, h, :] @ kf[:, h, :].T", "qf[:, h, :] @ kf[:, 0, :].T"),
+    ("attention", "output not normalised", "O[:, h, :] = (p @ vf[:, h, :]) / l", "O[:, h, :] = (p @ vf[:, h, :])"),
+    ("attention", "lse without the max shift", "lse[h, :] = (m + np.log(l))[:, 0]", "lse[h, :] = (np.log(l))[:, 0]"),
+    ("lse_merge", "merge weights not normalised", "w / np.where(finite, tot, 1.0)[None]", "w"),
+    ("lse_merge", "merged lse without the max", "msafe + np.log(np.where(finite, tot, 1.0))",
+     "np.log(np.where(finite, tot, 1.0))"),
+    ("layer_attention", "chunk keys and values ignored",
+     "k = np.concatenate([_widen(k_hist), _widen(k_cur)], axis=0)\n    v = np.concatenate([_widen(v_hist), "
+     "_widen(v_cur)], axis=0)", "k = _widen(k_hist)\n    v = _widen(v_hist)"),
+    ("layer_attention", "chunk values read as raw bf16 bits", "_widen(v_cur)], axis=0)",
+     "v_cur.astype(np.float64)], axis=0)"),
+]
+
+
+@pytest.mark.parametrize("fn,name,old,new", PY_MUTATIONS, ids=[m[1] for m in PY_MUTATIONS])
+def test_pins_catch_planted_mistake_in_numpy_oracle(fn, name, old, new):
+    src = inspect.getsource(getattr(O, fn))
+    assert src.count(old) == 1, f"mutation site not unique or missing: {name}"
+    scope = {}
+    exec(compile(src.replace(old, new), O.__file__, "exec"), O.__dict__, scope)
+    saved = getattr(O, fn)
+    failed = []
+    try:
+        setattr(O, fn, scope[fn])
+        for pin_name, pin in _pins():
+            try:
+                pin()
+            except (AssertionError, RuntimeError, ValueError, FloatingPointError):
+                failed.append(pin_name)
+    finally:
+        setattr(O, fn, saved)
+    assert failed, f"no pin fails with the planted mistake: {name}"

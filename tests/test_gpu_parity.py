@@ -4,8 +4,10 @@ the same seeded inputs.
 Bar: centroid indices, packed codes and {scale, zero} bits identical; fitted
 centres identical; per-head reconstruction identical in binary32; attention
 within relative Frobenius 1e-2 and max abs 3e-2 of the oracle, LSE within
-1e-3.  Full-size workloads are checked on sampled token-heads / query rows
-that the oracle computes one by one; small shapes are checked in full.
+1e-3.  The tiny and the Wan-1.3B-like workloads are checked on every
+token-head, query row and head; the 14B-like layer and the sweep points on
+sampled token-heads and query rows that the oracle computes one by one; small
+edge shapes in full.
 """
 
 import numpy as np
@@ -140,53 +142,55 @@ def wan():
     return w, xk, xv, q, seeds_k, seeds_v
 
 
-def test_wan_encode_full_size_sampled(wan):
+def test_wan_encode_decode_full_size(wan):
+    """Every token-head of the Wan-1.3B-like history (12 heads x 32,760 tokens,
+    K and V): idx, codes and {s, z} bit-exact, and the reconstruction bit-exact
+    in binary32."""
     K = _K()
     w, xk, xv, q, seeds_k, seeds_v = wan
     T, H, d = xk.shape
-    for x, cent, bits, seed in ((xk, seeds_k, w.bits_k, 1), (xv, seeds_v, w.bits_v, 2)):
+    for x, cent, bits in ((xk, seeds_k, w.bits_k), (xv, seeds_v, w.bits_v)):
         codec = K.Codec(H, d, w.num_centroids, bits, w.group_size)
         comp = _gpu_encode(codec, x, cent)
-        toks = _sample_tokens(T, 2048, seed)
-        idx_r, codes_r, meta_r = O.encode(np.ascontiguousarray(x[toks]), cent, bits, w.group_size)
-        _assert_encoded_equal(comp, H, T, d, bits, w.group_size, idx_r, codes_r, meta_r, tokens=toks)
+        idx_r, codes_r, meta_r = O.encode(x, cent, bits, w.group_size)
+        _assert_encoded_equal(comp, H, T, d, bits, w.group_size, idx_r, codes_r, meta_r)
+        dec = torch.empty((T, H, d), dtype=torch.float32, device="cuda")
+        K.kvq_decode(comp, dec)
+        dref = O.decode(idx_r, codes_r, meta_r, cent, bits, w.group_size)
+        assert np.array_equal(f32_bits(dec), f32_bits(dref)), "decode differs"
     _status_ok()
 
 
-def test_wan_fit_full_size_two_heads(wan):
+def test_wan_fit_full_size(wan):
+    """Centres of all 12 heads after the benchmark's 2 k-means rounds, K and V,
+    bit-exact."""
     K = _K()
-    w, xk, *_ = wan
+    w, xk, xv, *_ = wan
     T, H, d = xk.shape
-    codec = K.Codec(H, d, w.num_centroids, w.bits_k, w.group_size)
-    cent = torch.empty((H, w.num_centroids, d), dtype=torch.bfloat16, device="cuda")
-    K.kvq_fit_centroids(codec, to_dev(xk), w.kmeans_iters, cent)
-    heads = [0, 7]
-    ref = O.fit(np.ascontiguousarray(xk[:, heads]), w.num_centroids, w.kmeans_iters)
-    assert np.array_equal(bits_u16(cent)[heads], ref)
+    for x, bits in ((xk, w.bits_k), (xv, w.bits_v)):
+        codec = K.Codec(H, d, w.num_centroids, bits, w.group_size)
+        cent = torch.empty((H, w.num_centroids, d), dtype=torch.bfloat16, device="cuda")
+        K.kvq_fit_centroids(codec, to_dev(x), w.kmeans_iters, cent)
+        ref = O.fit(x, w.num_centroids, w.kmeans_iters)
+        assert np.array_equal(bits_u16(cent), ref), f"centres differ in {np.sum(bits_u16(cent) != ref)} values"
     _status_ok()
 
 
-def test_wan_attention_full_size_sampled(wan):
+def test_wan_attention_full_size(wan):
+    """All 4,680 query rows of all 12 heads over the whole 32,760-token
+    compressed history, unsplit and with the history split inside the call."""
     K = _K()
     w, xk, xv, q, seeds_k, seeds_v = wan
     T, H, d = xk.shape
     ck = _gpu_encode(K.Codec(H, d, w.num_centroids, w.bits_k, w.group_size), xk, seeds_k)
     cv = _gpu_encode(K.Codec(H, d, w.num_centroids, w.bits_v, w.group_size), xv, seeds_v)
     o, lse = _attention(q, ck, cv)
-    o_s, lse_s = _attention(q, ck, cv, split=True)  # history split inside the call
-    heads = [3, 11]
-    rows = _sample_tokens(w.query_tokens, 256, 5)
-    sub = lambda a: np.ascontiguousarray(a[:, heads])
-    dk = O.decode(*O.encode(sub(xk), seeds_k[heads], w.bits_k, w.group_size), seeds_k[heads], w.bits_k,
-                  w.group_size)
-    dv = O.decode(*O.encode(sub(xv), seeds_v[heads], w.bits_v, w.group_size), seeds_v[heads], w.bits_v,
-                  w.group_size)
-    o_ref, lse_ref = O.attention(sub(q), dk, dv, rows=rows)
-    o_g = o.cpu().numpy()[rows][:, heads]
-    l_g = lse.cpu().numpy()[heads][:, rows]
-    assert_attention_close(o_g, l_g, o_ref, lse_ref, "wan full")
-    assert_attention_close(o_s.cpu().numpy()[rows][:, heads], lse_s.cpu().numpy()[heads][:, rows], o_ref, lse_ref,
-                           "wan full, split history")
+    o_s, lse_s = _attention(q, ck, cv, split=True)
+    dk = O.decode(*O.encode(xk, seeds_k, w.bits_k, w.group_size), seeds_k, w.bits_k, w.group_size)
+    dv = O.decode(*O.encode(xv, seeds_v, w.bits_v, w.group_size), seeds_v, w.bits_v, w.group_size)
+    o_ref, lse_ref = O.attention(q, dk, dv)
+    assert_attention_close(o.cpu().numpy(), lse.cpu().numpy(), o_ref, lse_ref, "wan full")
+    assert_attention_close(o_s.cpu().numpy(), lse_s.cpu().numpy(), o_ref, lse_ref, "wan full, split history")
     _status_ok()
 
 

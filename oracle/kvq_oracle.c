@@ -31,6 +31,14 @@
  *    QuantWM, Fig. 9 (packed storage, on-demand reconstruction).
  *  - joint head-channel linear encoder/decoder with INT4 coefficients, centres
  *    added back after decoding: NanoKV page, abstract and Fig. 4(a,b).
+ *  - query-sensitive centre selection (QSAC): QuantWM, Sec. 4.1 -- per-head
+ *    channel weights w_c from the historical queries' second moments (the
+ *    diagonal of M_h), a query-weighted distance that picks top-M candidate
+ *    centres, then the candidate whose residual groups minimise the expected
+ *    squared logit error sum_g (sum_{c in g} w_c) R_g^2 (the Widrow
+ *    approximation with its common factor 1 / (12 (2^b - 1)^2) dropped);
+ *    M = 4 (QuantWM, Table 11); w = 1 before any query has been seen
+ *    (QuantWM, the appendix paragraph on the cold start).
  *
  * Readings taken where the pages are silent (each mirrored by the CUDA
  * library and listed in the design notes):
@@ -47,7 +55,12 @@
  *    smallest normal binary32, is "degenerate": s = |min|, z = -sign(min),
  *    codes 0, which decodes to exactly min (and to 0 when min == 0);
  *  - decode: x^_c = mu_c + (q_c - z) * s with the subtraction, multiply and
- *    add each rounded to binary32.
+ *    add each rounded to binary32;
+ *  - QSAC arithmetic in binary32, channel order, no FMA: weighted distance
+ *    acc += w_c * (e_c * e_c); group weight W_g = sum of w_c in channel order;
+ *    R_g = max - min of the group's residuals; score += W_g * (R_g * R_g) over
+ *    groups in order; candidates ranked by (distance, index); the final
+ *    choice is the lowest score, ties to the better-ranked candidate.
  */
 
 #include <float.h>
@@ -421,6 +434,171 @@ int kvqo_decode(const uint16_t *idx, const uint8_t *codes, const float *meta, co
                 out[(t * H + h) * (int64_t)d + c] = mu + kvqo_dequant(q[c], s, z);
             }
         }
+        free(q);
+    }
+    return rc;
+}
+
+/* ------------------------------------------------------------------------ */
+/* query-sensitive centre selection (QSAC)                                   */
+/* ------------------------------------------------------------------------ */
+
+/* Query-weighted squared distance sum_c w_c (x_c - mu_c)^2, binary32. */
+float kvqo_weighted_distance(const float *x, const float *mu, const float *w, int d)
+{
+    float total = 0.0f;
+    for (int c = 0; c < d; ++c) {
+        const float diff = x[c] - mu[c];
+        const float diff2 = diff * diff;
+        const float term = w[c] * diff2;
+        total = total + term;
+    }
+    return total;
+}
+
+/* QSAC score of one residual: sum over groups of W_g * R_g^2, binary32. */
+float kvqo_qsac_score(const float *r, const float *w, int d, int G)
+{
+    float score = 0.0f;
+    for (int g = 0; g < d / G; ++g) {
+        float lo = r[g * G], hi = r[g * G], wg = 0.0f;
+        for (int c = g * G; c < (g + 1) * G; ++c) {
+            if (r[c] < lo)
+                lo = r[c];
+            if (r[c] > hi)
+                hi = r[c];
+            wg = wg + w[c];
+        }
+        const float range = hi - lo;
+        const float range2 = range * range;
+        const float term = wg * range2;
+        score = score + term;
+    }
+    return score;
+}
+
+/* Centre chosen by QSAC for one vector.  mu [C][d] binary32, w [d].  cand
+ * (M entries) receives the candidates in rank order. */
+static int qsac_choose(const float *x, const float *mu, const float *w, int C, int d, int G, int M, int *cand,
+                       float *cand_dist, float *r)
+{
+    int m = M < C ? M : C;
+    /* top-m by (distance, index): insertion into a sorted list */
+    int n = 0;
+    for (int j = 0; j < C; ++j) {
+        const float dj = kvqo_weighted_distance(x, mu + (int64_t)j * d, w, d);
+        int pos = n;
+        while (pos > 0 && dj < cand_dist[pos - 1])
+            --pos;
+        if (pos >= m)
+            continue;
+        int last = n < m ? n : m - 1;
+        for (int k = last; k > pos; --k) {
+            cand[k] = cand[k - 1];
+            cand_dist[k] = cand_dist[k - 1];
+        }
+        cand[pos] = j;
+        cand_dist[pos] = dj;
+        if (n < m)
+            ++n;
+    }
+    int choice = cand[0];
+    float best = 0.0f;
+    for (int k = 0; k < m; ++k) {
+        const float *mj = mu + (int64_t)cand[k] * d;
+        for (int c = 0; c < d; ++c)
+            r[c] = x[c] - mj[c];
+        const float sc = kvqo_qsac_score(r, w, d, G);
+        if (k == 0 || sc < best) {
+            best = sc;
+            choice = cand[k];
+        }
+    }
+    return choice;
+}
+
+/*
+ * QSAC assignment of one K history.  w: [H][d] binary32 channel weights.
+ * idx [H][T] (out); cand (optional) [H][T][M] the ranked candidates (-1 where
+ * C < M).
+ */
+int kvqo_qsac_assign(const void *x, int x_is_bf16, int64_t T, int H, int d, const uint16_t *cent, int C,
+                     const float *w, int G, int M, uint16_t *idx, int32_t *cand_out)
+{
+    if (T < 0 || H <= 0 || d <= 0 || C <= 0 || C > 65536 || M <= 0 || G <= 0 || d % G != 0)
+        return KVQO_EINVAL;
+    int rc = KVQO_OK;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int h = 0; h < H; ++h) {
+        float *mu = (float *)malloc(sizeof(float) * (size_t)C * d);
+        float *xv = (float *)malloc(sizeof(float) * (size_t)d);
+        float *r = (float *)malloc(sizeof(float) * (size_t)d);
+        int *cand = (int *)malloc(sizeof(int) * (size_t)M);
+        float *cdist = (float *)malloc(sizeof(float) * (size_t)M);
+        if (!mu || !xv || !r || !cand || !cdist) {
+            rc = KVQO_ENOMEM;
+        } else {
+            widen_centres(cent + (int64_t)h * C * d, C, d, mu);
+            for (int64_t t = 0; t < T; ++t) {
+                gather_token(x, x_is_bf16, H, d, t, h, xv);
+                for (int k = 0; k < M; ++k)
+                    cand[k] = -1;
+                const int j = qsac_choose(xv, mu, w + (int64_t)h * d, C, d, G, M, cand, cdist, r);
+                idx[(int64_t)h * T + t] = (uint16_t)j;
+                if (cand_out)
+                    for (int k = 0; k < M; ++k)
+                        cand_out[((int64_t)h * T + t) * M + k] = cand[k];
+            }
+        }
+        free(mu);
+        free(xv);
+        free(r);
+        free(cand);
+        free(cdist);
+    }
+    return rc;
+}
+
+/*
+ * Residual quantisation against GIVEN centre indices (the QSAC choice):
+ * codes and {s, z} exactly as kvqo_encode writes them for that index.
+ */
+int kvqo_encode_given(const void *x, int x_is_bf16, int64_t T, int H, int d, const uint16_t *cent, int C,
+                      int bits, int G, const uint16_t *idx, uint8_t *codes, float *meta)
+{
+    if (T < 0 || !check_codec(H, d, C, bits, G))
+        return KVQO_EINVAL;
+    const int cb = d * bits / 8, ng = d / G;
+    int rc = KVQO_OK;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int h = 0; h < H; ++h) {
+        float *xv = (float *)malloc(sizeof(float) * (size_t)d);
+        float *res = (float *)malloc(sizeof(float) * (size_t)d);
+        uint8_t *q = (uint8_t *)malloc((size_t)d);
+        if (!xv || !res || !q) {
+            rc = KVQO_ENOMEM;
+        } else {
+            for (int64_t t = 0; t < T; ++t) {
+                const int64_t th = (int64_t)h * T + t;
+                const int j = idx[th];
+                if (j >= C) {
+                    rc = KVQO_EINVAL;
+                    break;
+                }
+                gather_token(x, x_is_bf16, H, d, t, h, xv);
+                for (int c = 0; c < d; ++c)
+                    res[c] = xv[c] - bf16_widen(cent[((int64_t)h * C + j) * d + c]);
+                for (int g = 0; g < ng; ++g) {
+                    float sg, zg;
+                    kvqo_quant_group(res + g * G, G, bits, &sg, &zg, q + g * G);
+                    meta[(th * ng + g) * 2 + 0] = sg;
+                    meta[(th * ng + g) * 2 + 1] = zg;
+                }
+                kvqo_pack(q, d, bits, codes + th * cb);
+            }
+        }
+        free(xv);
+        free(res);
         free(q);
     }
     return rc;

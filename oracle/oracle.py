@@ -23,6 +23,16 @@ Functions and the passages they follow:
   (and of any raw protected tokens; NanoKV page, Table 4), written as plain
   attention over the union of both key sets (NanoKV page, Fig. 4(a,d)).
 * ``stored_bytes_per_token_head`` / ``bits_per_value``: storage accounting.
+* ``query_moments``, ``qsac_weights``, ``weighted_distance``, ``qsac_score``,
+  ``qsac_assign``, ``qsac_encode``: QuantWM's query-sensitive centre selection
+  (Sec. 4.1): per-head second moments of the historical queries, their
+  diagonal as channel weights, top-M candidates by the weighted distance, the
+  final centre by the expected squared logit error of its quantised residual.
+* ``psac_basis``, ``psac_coefficients``, ``attention_psac``: QuantWM's
+  principal-subspace logit correction (the PSAC section after Sec. 4.1;
+  r = 8, Table 9): the remaining key error
+  projected on the top-r eigenvectors of the query second moments, added back
+  to the logits.
 """
 
 from __future__ import annotations
@@ -58,6 +68,12 @@ def _load():
     lib.kvqo_joint_decode.argtypes = [vp, vp, vp, vp, vp, i64, i32, i32, i32, i32, i32, i32, vp]
     lib.kvqo_distance.argtypes = [vp, vp, i32]
     lib.kvqo_distance.restype = ctypes.c_float
+    lib.kvqo_weighted_distance.argtypes = [vp, vp, vp, i32]
+    lib.kvqo_weighted_distance.restype = ctypes.c_float
+    lib.kvqo_qsac_score.argtypes = [vp, vp, i32, i32]
+    lib.kvqo_qsac_score.restype = ctypes.c_float
+    lib.kvqo_qsac_assign.argtypes = [vp, i32, i64, i32, i32, vp, i32, vp, i32, i32, vp, vp]
+    lib.kvqo_encode_given.argtypes = [vp, i32, i64, i32, i32, vp, i32, i32, i32, vp, vp, vp]
     lib.kvqo_quant_group.argtypes = [vp, i32, i32, vp, vp, vp]
     lib.kvqo_dequant.argtypes = [ctypes.c_uint8, ctypes.c_float, ctypes.c_float]
     lib.kvqo_dequant.restype = ctypes.c_float
@@ -296,6 +312,108 @@ def lse_merge(o_parts: Sequence[np.ndarray], lse_parts: Sequence[np.ndarray]) ->
     wn = np.where(finite[None], w / np.where(finite, tot, 1.0)[None], 0.0)
     O = np.einsum("nht,nthd->thd", wn, Os)
     return O, lse
+
+
+# ----------------------------------------------------------------------------
+# QuantWM: query-sensitive centre selection (QSAC) and principal-subspace
+# logit correction (PSAC)
+# ----------------------------------------------------------------------------
+
+def query_moments(q: np.ndarray) -> np.ndarray:
+    """M_h = mean over the observed query tokens of q q^T, per head (binary64).
+
+    q [n][H][d] (bf16 bits or float) -> [H][d][d].  These are the historical
+    query statistics both QSAC and PSAC read (QuantWM, Sec. 4.1)."""
+    qf = _widen(q)
+    n = qf.shape[0]
+    return np.einsum("nhc,nhe->hce", qf, qf) / max(n, 1)
+
+
+def qsac_weights(moments: Optional[np.ndarray], H: int, d: int) -> np.ndarray:
+    """Channel weights w_{h,c} = [M_h]_cc rounded to binary32; all ones before
+    any query has been observed (cold start)."""
+    if moments is None:
+        return np.ones((H, d), np.float32)
+    return np.ascontiguousarray(np.einsum("hcc->hc", moments).astype(np.float32))
+
+
+def weighted_distance(x: np.ndarray, mu: np.ndarray, w: np.ndarray) -> float:
+    """QSAC's query-weighted distance sum_c w_c (x_c - mu_c)^2 in binary32."""
+    x = np.ascontiguousarray(x, dtype=np.float32)
+    mu = np.ascontiguousarray(mu, dtype=np.float32)
+    w = np.ascontiguousarray(w, dtype=np.float32)
+    return float(_load().kvqo_weighted_distance(_ptr(x), _ptr(mu), _ptr(w), x.shape[0]))
+
+
+def qsac_score(r: np.ndarray, w: np.ndarray, group: int) -> float:
+    """QSAC score of one residual: sum over groups of (sum of w_c) * R_g^2."""
+    r = np.ascontiguousarray(r, dtype=np.float32)
+    w = np.ascontiguousarray(w, dtype=np.float32)
+    return float(_load().kvqo_qsac_score(_ptr(r), _ptr(w), r.shape[0], group))
+
+
+def qsac_assign(x: np.ndarray, cent: np.ndarray, w: np.ndarray, group: int, M: int = 4,
+                return_candidates: bool = False):
+    """idx [H][T] chosen by QSAC; optionally the ranked candidates [H][T][M]
+    (-1 where there are fewer than M centres).  x [T][H][d], cent [H][C][d]
+    bf16 bits, w [H][d] binary32."""
+    x, xb = _x_arg(x)
+    T, H, d = x.shape
+    C = cent.shape[1]
+    cent = np.ascontiguousarray(cent, dtype=np.uint16)
+    w = np.ascontiguousarray(w, dtype=np.float32)
+    idx = np.zeros((H, T), np.uint16)
+    cand = np.zeros((H, T, M), np.int32)
+    _check(_load().kvqo_qsac_assign(_ptr(x), xb, T, H, d, _ptr(cent), C, _ptr(w), group, M, _ptr(idx),
+                                    _ptr(cand)), "qsac_assign")
+    return (idx, cand) if return_candidates else idx
+
+
+def qsac_encode(x: np.ndarray, cent: np.ndarray, w: np.ndarray, bits: int, group: int, M: int = 4):
+    """encode with the QSAC centre choice: (idx, codes, meta) in the layouts
+    of ``encode``."""
+    idx = qsac_assign(x, cent, w, group, M)
+    x, xb = _x_arg(x)
+    T, H, d = x.shape
+    C = cent.shape[1]
+    cent = np.ascontiguousarray(cent, dtype=np.uint16)
+    codes = np.zeros((H, T, d * bits // 8), np.uint8)
+    meta = np.zeros((H, T, d // group, 2), np.float32)
+    _check(_load().kvqo_encode_given(_ptr(x), xb, T, H, d, _ptr(cent), C, bits, group, _ptr(idx), _ptr(codes),
+                                     _ptr(meta)), "encode_given")
+    return idx, codes, meta
+
+
+def psac_basis(moments: np.ndarray, r: int) -> np.ndarray:
+    """U_r [H][d][r]: eigenvectors of M_h for its r largest eigenvalues, in
+    decreasing order (numpy.linalg.eigh), each with its largest-magnitude
+    component made positive."""
+    H, d, _ = moments.shape
+    U = np.zeros((H, d, r), np.float64)
+    for h in range(H):
+        lam, vec = np.linalg.eigh(moments[h])
+        order = np.argsort(-lam, kind="stable")[:r]
+        V = vec[:, order]
+        sign = np.sign(V[np.argmax(np.abs(V), axis=0), np.arange(r)])
+        U[h] = V * np.where(sign == 0, 1.0, sign)[None, :]
+    return U
+
+
+def psac_coefficients(x: np.ndarray, k_hat: np.ndarray, U: np.ndarray) -> np.ndarray:
+    """C [T][H][r] = (k - k^) U_r per head: the remaining key error along the
+    principal query directions, stored in binary32.  x the original keys
+    (bf16 bits or float), k_hat the reconstruction [T][H][d]."""
+    e = _widen(x) - _widen(k_hat)
+    return np.einsum("thd,hdr->thr", e, U).astype(np.float32)
+
+
+def attention_psac(q: np.ndarray, k_hat: np.ndarray, v: np.ndarray, U: np.ndarray, coef: np.ndarray,
+                   scale: Optional[float] = None, rows: Optional[np.ndarray] = None) -> Tuple[np.ndarray, np.ndarray]:
+    """Attention with PSAC's corrected logits s_ij = scale (q_i . k^_j +
+    (q_i U_r) . C_j); otherwise as ``attention``.  Equivalent to attention over
+    the corrected keys k^_j + U_r C_j, which is how it is evaluated."""
+    kc = _widen(k_hat) + np.einsum("hdr,thr->thd", U, coef.astype(np.float64))
+    return attention(q, kc, v, scale, rows)
 
 
 # ----------------------------------------------------------------------------

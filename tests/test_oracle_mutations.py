@@ -38,6 +38,12 @@ MUTATIONS = [
     ("joint residual not rounded to bf16", "res[h * d + c] = bf16_widen(bf16_round(e));", "res[h * d + c] = e;"),
     ("joint decoder forgets the centre", "out[(t * H + h) * (int64_t)d + c] = mu + (float)acc;",
      "out[(t * H + h) * (int64_t)d + c] = (float)acc;"),
+    ("QSAC distance without the channel weight", "const float term = w[c] * diff2;", "const float term = diff2;"),
+    ("QSAC score without the group weight", "const float term = wg * range2;", "const float term = range2;"),
+    ("QSAC group range without its minimum", "const float range = hi - lo;", "const float range = hi;"),
+    ("QSAC score ties to the worse-ranked candidate", "if (k == 0 || sc < best) {", "if (k == 0 || sc <= best) {"),
+    ("QSAC ranking ties to the higher index", "while (pos > 0 && dj < cand_dist[pos - 1])",
+     "while (pos > 0 && dj <= cand_dist[pos - 1])"),
 ]
 
 
@@ -95,6 +101,13 @@ PY_MUTATIONS = [
      "_widen(v_cur)], axis=0)", "k = _widen(k_hist)\n    v = _widen(v_hist)"),
     ("layer_attention", "chunk values read as raw bf16 bits", "_widen(v_cur)], axis=0)",
      "v_cur.astype(np.float64)], axis=0)"),
+    ("query_moments", "query moments not averaged", "/ max(n, 1)", ""),
+    ("psac_basis", "PSAC keeps the smallest eigenvalues", 'np.argsort(-lam, kind="stable")',
+     'np.argsort(lam, kind="stable")'),
+    ("psac_coefficients", "PSAC error with the wrong sign", "e = _widen(x) - _widen(k_hat)",
+     "e = _widen(k_hat) - _widen(x)"),
+    ("attention_psac", "PSAC correction dropped", 'kc = _widen(k_hat) + np.einsum("hdr,thr->thd", U, coef.astype(np.float64))',
+     "kc = _widen(k_hat)"),
 ]
 
 

@@ -515,3 +515,159 @@ def test_layer_attention_is_the_merge_of_history_and_chunk():
     pc = O.attention(q, kc, vc)
     om, lm = O.lse_merge([ph[0], pc[0]], [ph[1], pc[1]])
     assert np.max(np.abs(o - om)) < 1e-12 and np.max(np.abs(lse - lm)) < 1e-12
+
+
+# ----------------------------------------------------------------------------
+# QuantWM: query-sensitive centre selection (QSAC), principal-subspace logit
+# correction (PSAC)
+# ----------------------------------------------------------------------------
+
+def test_qsac_worked_example():
+    g = _golden("qsac_worked_example.json")
+    x = np.array(g["x"], np.float32)
+    cent = _bf16(np.array(g["centres"], np.float32))[None]          # [1][C][d]
+    G = g["group"]
+    for case in g["cases"]:
+        w = np.array(case["w"], np.float32)
+        mus = _widen(cent[0])
+        assert [O.weighted_distance(x, mu, w) for mu in mus] == case["distance"]
+        assert [O.qsac_score(x - mu, w, G) for mu in mus] == case["score"]
+        for M, want in case["choice"].items():
+            idx, cand = O.qsac_assign(x[None, None], cent, w[None], G, int(M), return_candidates=True)
+            assert int(idx[0, 0]) == want, (case["note"], M)
+            ranked = [int(c) for c in cand[0, 0] if c >= 0]
+            assert ranked == [j for j in np.argsort(case["rank"])][: min(int(M), 3)]
+
+
+def test_qsac_unit_weights_one_candidate_is_plain_nearest_centre():
+    """w = 1 and M = 1 reduce QSAC to the plain nearest-centre encode."""
+    rng = np.random.default_rng(31)
+    x = _bf16(rng.normal(size=(400, 3, 64)) * rng.uniform(0.5, 2, size=(1, 3, 64)))
+    cent = O.fit(x[:32], 32, 0)
+    w = O.qsac_weights(None, 3, 64)
+    assert np.array_equal(O.qsac_assign(x, cent, w, 16, 1), O.assign(x, cent))
+    for a, b in zip(O.qsac_encode(x, cent, w, 2, 16, 1), O.encode(x, cent, 2, 16)):
+        assert np.array_equal(a, b)
+
+
+def test_qsac_against_exact_rational_selection():
+    """Candidates and choice against exact rational arithmetic (tiny random
+    problems; cases whose exact values come within 1e-4 relative of a tie are
+    skipped, since binary32 may then order them either way)."""
+    rng = np.random.default_rng(32)
+    checked = 0
+    for trial in range(40):
+        d, G, C, M = 8, 4, 6, 3
+        x = rng.normal(size=d).astype(np.float32)
+        mus = _widen(_bf16(rng.normal(size=(C, d))))
+        w = rng.uniform(0.1, 4.0, size=d).astype(np.float32)
+        X = [Fraction(float(v)) for v in x]
+        W = [Fraction(float(v)) for v in w]
+        D = [sum(W[c] * (X[c] - Fraction(float(mu[c]))) ** 2 for c in range(d)) for mu in mus]
+        order = sorted(range(C), key=lambda j: (D[j], j))
+        gaps = [abs(D[order[k + 1]] - D[order[k]]) / max(D[order[k]], Fraction(1, 10 ** 9)) for k in range(M)]
+        if min(gaps) < Fraction(1, 10 ** 4):
+            continue
+        S = {}
+        for j in order[:M]:
+            r = [X[c] - Fraction(float(mus[j][c])) for c in range(d)]
+            S[j] = sum(sum(W[g * G:(g + 1) * G]) * (max(r[g * G:(g + 1) * G]) - min(r[g * G:(g + 1) * G])) ** 2
+                       for g in range(d // G))
+        best = min(order[:M], key=lambda j: (S[j], order.index(j)))
+        others = [S[j] for j in order[:M] if j != best]
+        if others and min(abs(s - S[best]) for s in others) < Fraction(1, 10 ** 4) * max(S[best], Fraction(1)):
+            continue
+        idx, cand = O.qsac_assign(x[None, None], _bf16(mus)[None], w[None], G, M, return_candidates=True)
+        assert [int(c) for c in cand[0, 0]] == order[:M]
+        assert int(idx[0, 0]) == best
+        checked += 1
+    assert checked >= 25
+
+
+def test_qsac_power_of_two_weight_scaling_keeps_the_choice():
+    rng = np.random.default_rng(33)
+    x = _bf16(rng.normal(size=(200, 2, 32)))
+    cent = O.fit(x[:16], 16, 0)
+    w = rng.uniform(0.2, 3.0, size=(2, 32)).astype(np.float32)
+    base = O.qsac_assign(x, cent, w, 16, 4)
+    for k in (-3, 5):
+        assert np.array_equal(O.qsac_assign(x, cent, (w * np.float32(2.0 ** k)).astype(np.float32), 16, 4), base)
+
+
+def test_query_moments_and_weights_closed_form():
+    """Queries along coordinate axes: M_h is diagonal with the mean squares;
+    the QSAC weights are that diagonal; no statistics gives unit weights."""
+    n, H, d = 6, 2, 4
+    q = np.zeros((n, H, d), np.float32)
+    for t in range(n):
+        q[t, :, t % d] = t + 1.0
+    M = O.query_moments(q)
+    want = np.zeros((H, d))
+    for t in range(n):
+        want[:, t % d] += (t + 1.0) ** 2 / n
+    assert np.allclose(M, np.stack([np.diag(want[h]) for h in range(H)]), atol=0, rtol=1e-15)
+    assert np.array_equal(O.qsac_weights(M, H, d), want.astype(np.float32))
+    assert np.array_equal(O.qsac_weights(None, H, d), np.ones((H, d), np.float32))
+
+
+def _psac_case(seed, r):
+    rng = np.random.default_rng(seed)
+    Tq, T, H, d = 12, 80, 2, 16
+    q_hist = _bf16(rng.normal(size=(300, H, d)) * np.linspace(3, 0.2, d)[None, None])
+    q = _bf16(rng.normal(size=(Tq, H, d)))
+    k = _bf16(rng.normal(size=(T, H, d)))
+    k_hat = (_widen(k) + rng.normal(size=(T, H, d)).astype(np.float32) * 0.1).astype(np.float32)
+    v = rng.normal(size=(T, H, d)).astype(np.float32)
+    M = O.query_moments(q_hist)
+    U = O.psac_basis(M, r)
+    return q, k, k_hat, v, M, U
+
+
+def test_psac_basis_is_the_principal_query_subspace():
+    q, k, k_hat, v, M, U = _psac_case(34, 5)
+    for h in range(M.shape[0]):
+        assert np.allclose(U[h].T @ U[h], np.eye(5), atol=1e-12)
+        lam = np.einsum("dr,de,er->r", U[h], M[h], U[h])
+        assert np.all(np.diff(lam) <= 1e-12)                          # decreasing
+        assert np.allclose(M[h] @ U[h], U[h] * lam[None], atol=1e-10)  # eigenvectors
+        top = np.sort(np.linalg.eigvalsh(M[h]))[::-1][:5]
+        assert np.allclose(lam, top, rtol=1e-12)
+        assert np.all(U[h][np.argmax(np.abs(U[h]), axis=0), np.arange(5)] > 0)
+
+
+def test_psac_full_rank_restores_the_exact_logits():
+    """r = d: k^ + U U^T (k - k^) = k, so the corrected attention is the
+    attention over the original keys (up to the binary32 storage of C)."""
+    q, k, k_hat, v, M, U = _psac_case(35, 16)
+    coef = O.psac_coefficients(k, k_hat, U)
+    o, lse = O.attention_psac(q, k_hat, v, U, coef)
+    o_ref, lse_ref = O.attention(q, k, v)
+    assert np.max(np.abs(o - o_ref)) < 1e-5 and np.max(np.abs(lse - lse_ref)) < 1e-5
+
+
+def test_psac_rank_zero_and_queries_in_the_subspace():
+    """r = 0 leaves the plain attention over k^; a query inside span(U_r) sees
+    its exact logits q . k, whatever the error outside that span."""
+    q, k, k_hat, v, M, U = _psac_case(36, 4)
+    Tq, H, d = q.shape
+    o0, l0 = O.attention_psac(q, k_hat, v, U[:, :, :0], O.psac_coefficients(k, k_hat, U[:, :, :0]))
+    oa, la = O.attention(q, k_hat, v)
+    assert np.array_equal(o0, oa) and np.array_equal(l0, la)
+    a = np.random.default_rng(37).normal(size=(Tq, H, 4))
+    q_in = np.einsum("hdr,thr->thd", U, a)                              # queries in span(U_r), float64
+    coef = O.psac_coefficients(k, k_hat, U)
+    o, lse = O.attention_psac(q_in, k_hat, v, U, coef)
+    o_ref, lse_ref = O.attention(q_in, k, v)
+    assert np.max(np.abs(lse - lse_ref)) < 1e-5 and np.max(np.abs(o - o_ref)) < 1e-5
+
+
+def test_qsac_ties_follow_index_order():
+    """Three centres at the same weighted distance and with the same score:
+    they rank by index and the lowest index is chosen."""
+    x = np.zeros((1, 1, 4), np.float32)
+    cent = _bf16(np.eye(4, dtype=np.float32)[:3])[None]
+    w = np.ones((1, 4), np.float32)
+    idx, cand = O.qsac_assign(x, cent, w, 2, 3, return_candidates=True)
+    assert [int(c) for c in cand[0, 0]] == [0, 1, 2] and int(idx[0, 0]) == 0
+    idx, cand = O.qsac_assign(x, cent[:, ::-1].copy(), w, 2, 2, return_candidates=True)
+    assert [int(c) for c in cand[0, 0]] == [0, 1] and int(idx[0, 0]) == 0

@@ -17,6 +17,13 @@ events.  The headline value is history tokens per second of whole steps,
 summed over ranks.  ``--impl reference`` times the CPU oracle instead on a
 bounded sample of the same workload.
 
+Beside the step (after its timed region, L2 flushed before each call) the
+line's ``next_rows`` reports the current chunk's full-layer attention --
+the compressed history plus the chunk's own 4,680 uncompressed keys under one
+softmax (kvq_layer_attention) -- and its dense part alone
+(kvq_attention_dense_lse), each as mean device time and TFLOP/s of
+4 Tq keys d H flops.
+
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
 """
 

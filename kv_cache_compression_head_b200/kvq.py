@@ -123,6 +123,14 @@ def _dtype_code(t: torch.Tensor) -> int:
     raise TypeError(f"unsupported dtype {t.dtype}")
 
 
+def _need_bf16(what: str, *ts: Optional[torch.Tensor]) -> None:
+    """The C ABI takes queries, dense keys and values as raw bf16 bits; a
+    tensor of another dtype would be misread, so it is refused here."""
+    for t in ts:
+        if t is not None and t.dtype != torch.bfloat16:
+            raise TypeError(f"{what}: expected bfloat16, got {t.dtype}")
+
+
 # ----------------------------------------------------------------------------
 # descriptors
 # ----------------------------------------------------------------------------
@@ -247,6 +255,7 @@ def kvq_decode(comp: Compressed, x_out: torch.Tensor, workspace: Optional[torch.
 def kvq_attention_lse(q: torch.Tensor, k: Compressed, v: Compressed, o_out: torch.Tensor, lse_out: torch.Tensor,
                       t_begin: int = 0, t_end: Optional[int] = None, softmax_scale: float = 0.0,
                       workspace: Optional[torch.Tensor] = None, stream=None) -> None:
+    _need_bf16("kvq_attention_lse", q)
     if t_end is None:
         t_end = k.num_tokens
     kv, vv = k.view(), v.view()
@@ -260,6 +269,7 @@ def kvq_attention_dense_lse(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, o
                             lse_out: torch.Tensor, t_begin: int = 0, t_end: Optional[int] = None,
                             softmax_scale: float = 0.0, workspace: Optional[torch.Tensor] = None, stream=None) -> None:
     """Attention over uncompressed bf16 keys/values k, v [Tk][H][d]."""
+    _need_bf16("kvq_attention_dense_lse", q, k, v)
     Tk, H, d = k.shape
     if t_end is None:
         t_end = Tk
@@ -277,6 +287,7 @@ def kvq_layer_attention(q: torch.Tensor, k_hist: Compressed, v_hist: Compressed,
     """One softmax over the compressed history and the uncompressed keys
     k_cur, v_cur [Tc][H][d] (the current chunk and any raw protected tokens).
     The call needs a workspace; one is allocated when none is given."""
+    _need_bf16("kvq_layer_attention", q, k_cur, v_cur)
     if t_end is None:
         t_end = k_hist.num_tokens
     if workspace is None:

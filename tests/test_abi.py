@@ -178,6 +178,27 @@ def test_dense_and_layer_attention_rejected_on_host(K):
                  None, 0, None) == K.KVQ_OK
 
 
+def test_binding_refuses_non_bf16_queries_keys_values(K):
+    """Queries and dense keys/values cross the ABI as raw bf16 bits; the
+    binding refuses other dtypes before calling the library."""
+    import torch
+
+    f = torch.zeros((4, 2, 64), dtype=torch.float32)
+    b = torch.zeros((4, 2, 64), dtype=torch.bfloat16)
+    o = torch.zeros((4, 2, 64))
+    lse = torch.zeros((2, 4))
+    with pytest.raises(TypeError):
+        K.kvq_attention_dense_lse(f, b, b, o, lse)
+    with pytest.raises(TypeError):
+        K.kvq_attention_dense_lse(b, b, f, o, lse)
+    codec = K.Codec(2, 64, 4, 2, 16)
+    comp = K.Compressed(codec, 4, b, b, b, b)
+    with pytest.raises(TypeError):
+        K.kvq_attention_lse(f, comp, comp, o, lse)
+    with pytest.raises(TypeError):
+        K.kvq_layer_attention(b, comp, comp, f, b, o, lse, workspace=b)
+
+
 def test_binding_refuses_to_load_without_the_library(tmp_path):
     """A copy of the package without libkvq.so: importing the binding raises
     (the product path has no fallback)."""

@@ -1,30 +1,39 @@
 #!/usr/bin/env python
 """Benchmark of the compressed-KV hot path on B200.
 
-One step = one pass of every step of the path over the Wan-1.3B-like layer
-(12 heads x 128, bf16, history 21 frames x 1,560 = 32,760 tokens, query chunk
-4,680 tokens, 256 centroids per head, K INT2 / V INT2, group 16):
+The headline step runs every step of the path over the 14B-like layer, the
+largest workload that fits one GPU: 40 heads x 128, bf16; a history of
+60 frames x 1,560 = 93,600 tokens; a query chunk of 4,680 tokens; 512
+centroids per head; K INT4 / V INT2; group 32.  The step is
 
   fit centroids (K, V; 2 k-means rounds) -> encode (K, V) -> decode (K, V)
-  -> joint head-channel code of the same history (K, V: rank 192, INT4,
-     group 32, orthonormal W_enc): encode, then decode
-  -> attention of the chunk over the compressed history in 2 blocks
-  -> LSE merge of the 2 partial results.
+  -> joint head-channel code (K, V: rank 192, INT4, group 32, orthonormal
+     W_enc; encode, then decode) of the joint workload's 32,760-token,
+     12-head history, which is the shape the joint code is defined on
+  -> attention of the chunk over the compressed history in 8 blocks
+  -> LSE merge of the 8 partial results.
+
+After the headline, the Wan-1.3B-like step (12 heads, 32,760 history tokens,
+C = 256, K2V2, group 16, 2 blocks) is timed the same way and reported under
+``config2``.  Next to the steps (after their timed regions, L2 flushed before
+each call), ``next_rows`` reports the Wan-like chunk's full-layer attention:
+the compressed history plus the chunk's own 4,680 uncompressed keys under one
+softmax (kvq_layer_attention), and its dense part alone
+(kvq_attention_dense_lse).
 
 Inputs are seeded synthetic tensors resident in HBM before timing starts;
 L2 is flushed (256 MiB write) before every timed step, outside the step's
 events.  The headline value is history tokens per second of whole steps,
-summed over ranks.  ``--impl reference`` times the CPU oracle instead on a
-bounded sample of the same workload.
+summed over ranks.
 
-Beside the step (after its timed region, L2 flushed before each call) the
-line's ``next_rows`` reports the current chunk's full-layer attention --
-the compressed history plus the chunk's own 4,680 uncompressed keys under one
-softmax (kvq_layer_attention) -- and its dense part alone
-(kvq_attention_dense_lse), each as mean device time and TFLOP/s of
-4 Tq keys d H flops.
+``--impl reference`` times the CPU oracle instead: every step runs the oracle
+on a bounded sample of the headline workload; ``ms_per_step`` is the wall
+time of that sample and ``value`` the full step's rate extrapolated from it.
+``--sweep PATH`` times encode, decode and attention on a covering set of the
+12-head sweep points and writes one JSON line per point to PATH.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+                    [--sweep PATH]
 """
 
 from __future__ import annotations
@@ -48,31 +57,26 @@ if ROOT not in sys.path:
 
 METRIC = "encode history-tokens/s (HBM GB/s) and compressed-KV attention TFLOP/s, 1×B200"
 UNIT = "history-tokens/s"
-WORKLOAD = "wan13b"
-HISTORY_BLOCKS = 2
+HEADLINE = "14b"
+SECONDARY = "wan13b"
+JOINT = "joint"
 FLUSH_BYTES = 256 << 20
-# DRAM bytes (read + write) of one attention_pair_kernel launch of this
-# workload, from the ncu capture summarised in profiles/attention_pair_wan13b.md;
-# None whenever the kernel has changed since that capture.  The last capture
-# (92.6 MB per launch) predates the per-codec instantiation of the kernel.
+# DRAM bytes (read + write) of one attention kernel launch of the headline
+# workload, from an ncu capture of the current kernel; None whenever the
+# kernel has changed since that capture.
 ATTN_NCU_TRAFFIC_BYTES = None
-
-
-def _joint():
-    """The joint head-channel workload (same history shape as WORKLOAD)."""
-    from kv_cache_compression_head_b200 import synth
-
-    return synth.workload("joint")
 
 
 def parse_args():
     p = argparse.ArgumentParser()
     p.add_argument("--gpus", type=int, default=1)
-    p.add_argument("--steps", type=int, default=50)
-    p.add_argument("--warmup", type=int, default=5)
+    p.add_argument("--steps", type=int, default=20)
+    p.add_argument("--warmup", type=int, default=3)
     p.add_argument("--impl", default="kvq", choices=["kvq", "reference"])
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--no-secondary", action="store_true")
+    p.add_argument("--sweep", default=None, help="write per-point sweep timings (JSON lines) to this path")
     return p.parse_args()
 
 
@@ -120,7 +124,8 @@ def barrier(world):
 class ClockSampler:
     """SM clock, power and clock-event reasons sampled every few milliseconds
     by a background thread through NVML (read-only queries) between start()
-    and stop(); falls back to `nvidia-smi -lms` where NVML is unavailable."""
+    and stop().  Without NVML the line records "NVML unavailable" and no
+    clock figures."""
 
     PERIOD_S = 0.005
     REASONS = (("hw_slowdown", "nvmlClocksEventReasonHwSlowdown"),
@@ -195,46 +200,111 @@ def measured_peaks():
 
 
 # ----------------------------------------------------------------------------
-# algorithmic work per step (roofline numerators)
+# algorithmic work (roofline numerators)
 # ----------------------------------------------------------------------------
 
+def stored_bytes(d, bits, G):
+    """Bytes encode writes per token-head: packed codes, {s, z} pairs, index."""
+    return d * bits // 8 + 8 * (d // G) + 2
+
+
 def work_model(w):
+    """Algorithmic bytes and flops of one step's rows on workload w."""
     T, H, d, Tq, C, G = w.history_tokens, w.num_heads, w.head_dim, w.query_tokens, w.num_centroids, w.group_size
     th = T * H
+    blocks = w.history_blocks
+    enc_bytes = sum(th * (2 * d + stored_bytes(d, b, G)) for b in (w.bits_k, w.bits_v))
+    dec_bytes = sum(th * (stored_bytes(d, b, G) + 2 * d) for b in (w.bits_k, w.bits_v))
+    return {
+        "encode_bytes": enc_bytes,
+        # the assignment filter, X mu^T: 2 C d flop per token-head (K and V)
+        "encode_flops": 2 * th * 2.0 * C * d,
+        "decode_bytes": dec_bytes,
+        "attention_flops": 4.0 * Tq * T * d * H,
+        "merge_bytes": (blocks + 1) * Tq * H * d * 4 + (blocks + 1) * Tq * H * 4,
+        # per k-means round and token-head: the assignment reads x and writes
+        # its index, the update reads x and the index (K and V)
+        "fit_bytes": 2 * w.kmeans_iters * th * (2 * d + 2 + 2 * d + 2),
+    }
 
-    def stored(bits):  # bytes written per token-head by encode
-        return d * bits // 8 + 8 * (d // G) + 2
 
-    enc_bytes = sum(th * (2 * d + stored(b)) for b in (w.bits_k, w.bits_v))
-    dec_bytes = sum(th * (stored(b) + 2 * d) for b in (w.bits_k, w.bits_v))  # read compressed, write bf16
-    attn_flops = 4.0 * Tq * T * d * H
-    merge_bytes = (HISTORY_BLOCKS + 1) * Tq * H * d * 4 + (HISTORY_BLOCKS + 1) * Tq * H * 4
-    # fit, per k-means round and token-head: the assignment reads x and writes
-    # its index, the accumulation reads x and the index (K and V)
-    fit_bytes = 2 * w.kmeans_iters * th * (2 * d + 2 + 2 * d + 2)
-    # joint code, K and V: the assignment pass reads x and writes idx; the
-    # projection pass reads x and idx and writes r*b/8 code bytes and r/G
-    # {s, z} pairs per token; the decoder reads those and writes bf16 x^
-    wj = _joint()
-    jstored = wj.joint_rank * wj.bits_k // 8 + 8 * (wj.joint_rank // wj.joint_group)
-    joint_enc_bytes = 2 * T * (2 * (2 * H * d + 2 * H) + jstored)
-    joint_dec_bytes = 2 * T * (2 * H + jstored + 2 * H * d)
-    joint_flops = 2 * T * 2.0 * H * d * wj.joint_rank  # one GEMM per direction, K and V
-    return {"encode_bytes": enc_bytes, "decode_bytes": dec_bytes, "attention_flops": attn_flops,
-            "merge_bytes": merge_bytes, "fit_bytes": fit_bytes, "joint_enc_bytes": joint_enc_bytes,
-            "joint_dec_bytes": joint_dec_bytes, "joint_gemm_flops": joint_flops}
+def joint_work_model(wj):
+    """Joint code of K and V: x read once, idx and the coefficient codes and
+    {s, z} written (the encoder); the decoder reads those and writes bf16."""
+    T, H, d, r = wj.history_tokens, wj.num_heads, wj.head_dim, wj.joint_rank
+    jstored = r * wj.bits_k // 8 + 8 * (r // wj.joint_group)
+    return {"joint_enc_bytes": 2 * T * (2 * H * d + 2 * H + jstored),
+            "joint_dec_bytes": 2 * T * (2 * H + jstored + 2 * H * d),
+            # one GEMM per direction and branch, plus the assignment filter
+            "joint_gemm_flops": 2 * T * 2.0 * H * d * r,
+            "joint_filter_flops": 2 * T * H * 2.0 * wj.num_centroids * d}
 
 
 # ----------------------------------------------------------------------------
 # GPU arm
 # ----------------------------------------------------------------------------
 
+def to_device_bf16(a, device):
+    import torch
+
+    return torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).to(device)
+
+
+def pinned_bf16(a):
+    import torch
+
+    return torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).pin_memory()
+
+
+class JointRows:
+    """The joint head-channel code (rows a4 and its decoder) on the joint
+    workload's history: centres fitted once at set-up (not timed), then per
+    step the joint encode and decode of K and V."""
+
+    def __init__(self, device):
+        import torch
+
+        from kv_cache_compression_head_b200 import kvq as K
+        from kv_cache_compression_head_b200 import synth
+
+        self.K = K
+        wj = synth.workload(JOINT)
+        self.w = wj
+        T, H, d = wj.history_tokens, wj.num_heads, wj.head_dim
+        bf = torch.bfloat16
+        self.x = [to_device_bf16(synth.make_history(wj, which), device) for which in ("K", "V")]
+        fit_codec = K.Codec(H, d, wj.num_centroids, 2, 16)
+        self.cent = [torch.empty((H, wj.num_centroids, d), dtype=bf, device=device) for _ in range(2)]
+        for x, c in zip(self.x, self.cent):
+            K.kvq_fit_centroids(fit_codec, x, wj.kmeans_iters, c)
+        self.codec = [K.Codec(H, d, wj.num_centroids, b, wj.joint_group, wj.joint_rank)
+                      for b in (wj.bits_k, wj.bits_v)]
+        w_enc = synth.make_orthonormal_encoder(wj)
+        self.w_enc = to_device_bf16(w_enc, device)
+        self.w_dec = self.w_enc.t().contiguous()
+        self.enc = [K.alloc_encoded(c, T, device) for c in self.codec]
+        self.comp = [K.Compressed(c, T, self.cent[i], *self.enc[i], w_dec=self.w_dec)
+                     for i, c in enumerate(self.codec)]
+        self.dec = [torch.empty((T, H, d), dtype=bf, device=device) for _ in range(2)]
+        self.launches = 2 * 2 + 2  # per branch: assignment + projection; decoder
+
+    def encode(self):
+        for i in range(2):
+            self.K.kvq_encode(self.codec[i], self.x[i], self.cent[i], *self.enc[i], w_enc=self.w_enc)
+
+    def decode(self):
+        for i in range(2):
+            self.K.kvq_decode(self.comp[i], self.dec[i])
+
+    def outputs(self):
+        return [t for e in self.enc for t in e]
+
+
 class Pipeline:
-    """Device buffers and the per-step call sequence through the public API."""
+    """Device buffers of one workload and its per-step call sequence through
+    the public API."""
 
-    ROWS = ("fit", "encode", "decode", "joint_encode", "joint_decode", "attention", "merge")
-
-    def __init__(self, w, device):
+    def __init__(self, w, device, joint=None, layer=False):
         import torch
 
         from kv_cache_compression_head_b200 import kvq as K
@@ -242,7 +312,9 @@ class Pipeline:
         self.K = K
         self.w = w
         self.dev = device
+        self.joint = joint
         T, H, d, Tq = w.history_tokens, w.num_heads, w.head_dim, w.query_tokens
+        self.blocks = w.history_blocks if w.history_blocks > 1 else 2
         self.codec_k = K.Codec(H, d, w.num_centroids, w.bits_k, w.group_size)
         self.codec_v = K.Codec(H, d, w.num_centroids, w.bits_v, w.group_size)
         bf = torch.bfloat16
@@ -254,42 +326,47 @@ class Pipeline:
         self.ws = K.alloc_workspace(K.KVQ_OP_FIT, self.codec_k, T, device)
         self.ws_attn = K.alloc_workspace(K.KVQ_OP_ATTENTION, self.codec_k, T, device, num_queries=Tq)
         self.dec = [torch.empty((T, H, d), dtype=bf, device=device) for _ in range(2)]
-        self.o_parts = [torch.empty((Tq, H, d), dtype=torch.float32, device=device) for _ in range(HISTORY_BLOCKS)]
-        self.l_parts = [torch.empty((H, Tq), dtype=torch.float32, device=device) for _ in range(HISTORY_BLOCKS)]
+        self.o_parts = [torch.empty((Tq, H, d), dtype=torch.float32, device=device) for _ in range(self.blocks)]
+        self.l_parts = [torch.empty((H, Tq), dtype=torch.float32, device=device) for _ in range(self.blocks)]
         self.o = torch.empty((Tq, H, d), dtype=bf, device=device)
         self.lse = torch.empty((H, Tq), dtype=torch.float32, device=device)
-        self.edges = [T * i // HISTORY_BLOCKS for i in range(HISTORY_BLOCKS + 1)]
+        self.edges = [T * i // self.blocks for i in range(self.blocks + 1)]
         self.comp = [K.Compressed(c, T, self.cent[i], *self.enc[i])
                      for i, c in enumerate((self.codec_k, self.codec_v))]
-        # joint head-channel code of the same history (same centres)
-        from kv_cache_compression_head_b200 import synth
+        self.layer = layer
+        if layer:
+            # full-layer attention (outside the step): the chunk's own keys and
+            # values follow the history; one call = compressed part + dense
+            # part + their merge
+            self.kc = torch.empty((Tq, H, d), dtype=bf, device=device)
+            self.vc = torch.empty((Tq, H, d), dtype=bf, device=device)
+            self.ws_layer = K.alloc_workspace(K.KVQ_OP_LAYER_ATTENTION, self.codec_k, T, device, num_queries=Tq)
+            self.o_layer = torch.empty((Tq, H, d), dtype=bf, device=device)
+            self.lse_layer = torch.empty((H, Tq), dtype=torch.float32, device=device)
+        # fit: seed + (assign + 7 sort/update kernels) per round, K and V;
+        # encode 1; decode 1 (K and V); attention: one launch per block plus
+        # the call's own merge when it splits the range; final merge 1
+        self.launches_per_step = (2 * (1 + 8 * w.kmeans_iters) + 2 + 2 + 2 * self.blocks + 1
+                                  + (joint.launches if joint is not None else 0))
 
-        wj = _joint()
-        self.codec_j = [K.Codec(H, d, w.num_centroids, b, wj.joint_group, wj.joint_rank)
-                        for b in (wj.bits_k, wj.bits_v)]
-        w_enc = synth.make_orthonormal_encoder(wj)
-        self.w_enc = torch.from_numpy(w_enc.view(np.int16)).view(bf).to(device)
-        self.w_dec = self.w_enc.t().contiguous()
-        self.enc_j = [K.alloc_encoded(c, T, device) for c in self.codec_j]
-        self.comp_j = [K.Compressed(c, T, self.cent[i], *self.enc_j[i], w_dec=self.w_dec)
-                       for i, c in enumerate(self.codec_j)]
-        # full-layer attention (outside the step): the chunk's own keys and
-        # values follow the history; one call = compressed part + dense part
-        # + their merge
-        self.kc = torch.empty((Tq, H, d), dtype=bf, device=device)
-        self.vc = torch.empty((Tq, H, d), dtype=bf, device=device)
-        self.ws_layer = K.alloc_workspace(K.KVQ_OP_LAYER_ATTENTION, self.codec_k, T, device, num_queries=Tq)
-        self.o_layer = torch.empty((Tq, H, d), dtype=bf, device=device)
-        self.lse_layer = torch.empty((H, Tq), dtype=torch.float32, device=device)
-        # fit: seed + (assign + 4 sort + 3 update kernels) per round; encode 1;
-        # decode 1; joint encode 2 (assign, projection), joint decode 1;
-        # attention 2 per block (split + its merge); final merge 1 -- K and V
-        self.launches_per_step = (2 * (1 + 8 * w.kmeans_iters) + 2 + 2 + 2 * 2 + 2 + 2 * HISTORY_BLOCKS + 1)
+    @property
+    def rows(self):
+        r = ["fit", "encode", "decode"]
+        if self.joint is not None:
+            r += ["joint_encode", "joint_decode"]
+        return tuple(r + ["attention", "merge"])
+
+    def load_inputs(self, hk, hv, hq):
+        self.xk.copy_(hk)
+        self.xv.copy_(hv)
+        self.q.copy_(hq)
 
     def outputs(self):
         outs = [self.o, self.lse]
         for i in range(2):
-            outs += [self.cent[i], *self.enc[i], *self.enc_j[i]]
+            outs += [self.cent[i], *self.enc[i]]
+        if self.joint is not None:
+            outs += self.joint.outputs()
         return outs
 
     def step(self, ev=None):
@@ -312,16 +389,15 @@ class Pipeline:
         K.kvq_decode(self.comp[0], self.dec[0])
         K.kvq_decode(self.comp[1], self.dec[1])
         mark("decode", 1)
-        mark("joint_encode", 0)
-        K.kvq_encode(self.codec_j[0], self.xk, self.cent[0], *self.enc_j[0], w_enc=self.w_enc)
-        K.kvq_encode(self.codec_j[1], self.xv, self.cent[1], *self.enc_j[1], w_enc=self.w_enc)
-        mark("joint_encode", 1)
-        mark("joint_decode", 0)
-        K.kvq_decode(self.comp_j[0], self.dec[0])
-        K.kvq_decode(self.comp_j[1], self.dec[1])
-        mark("joint_decode", 1)
+        if self.joint is not None:
+            mark("joint_encode", 0)
+            self.joint.encode()
+            mark("joint_encode", 1)
+            mark("joint_decode", 0)
+            self.joint.decode()
+            mark("joint_decode", 1)
         mark("attention", 0)
-        for b in range(HISTORY_BLOCKS):
+        for b in range(self.blocks):
             K.kvq_attention_lse(self.q, self.comp[0], self.comp[1], self.o_parts[b], self.l_parts[b],
                                 t_begin=self.edges[b], t_end=self.edges[b + 1], workspace=self.ws_attn)
         mark("attention", 1)
@@ -329,6 +405,9 @@ class Pipeline:
         K.kvq_lse_merge(self.o_parts, self.l_parts, self.o, self.lse)
         mark("merge", 1)
 
+    def attention_block(self, b):
+        self.K.kvq_attention_lse(self.q, self.comp[0], self.comp[1], self.o_parts[b], self.l_parts[b],
+                                 t_begin=self.edges[b], t_end=self.edges[b + 1], workspace=self.ws_attn)
 
     def layer_attention(self):
         self.K.kvq_layer_attention(self.q, self.comp[0], self.comp[1], self.kc, self.vc, self.o_layer,
@@ -356,6 +435,126 @@ def time_calls(fn, reps, warmup, flush):
     return statistics.mean(a.elapsed_time(b) for a, b in ev)
 
 
+def check_status(K, when):
+    st = K.kvq_last_device_status()
+    if st != 0:
+        raise RuntimeError(f"device status {when}: {K.status_string(st)}")
+
+
+def time_steps(pipe, steps, warmup, flush, world, device, sample_clocks=None):
+    """Warm-up, then `steps` timed steps between barriers; returns per-row
+    mean ms, mean step ms (max over ranks), wall seconds and clocks."""
+    import torch
+
+    for _ in range(warmup):
+        flush.zero_()
+        pipe.step()
+    torch.cuda.synchronize()
+    check_status(pipe.K, "after warm-up")
+    ev = [{r: (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for r in pipe.rows}
+          for _ in range(steps)]
+    barrier(world)
+    torch.cuda.synchronize()
+    if sample_clocks is not None:
+        sample_clocks.start()
+    t_wall = time.perf_counter()
+    for k in range(steps):
+        flush.zero_()
+        pipe.step(ev[k])
+    torch.cuda.synchronize()
+    wall = time.perf_counter() - t_wall
+    barrier(world)
+    clk = sample_clocks.stop() if sample_clocks is not None else None
+    check_status(pipe.K, "after timing")
+    first, last = pipe.rows[0], pipe.rows[-1]
+    row_ms = {r: statistics.mean(e[r][0].elapsed_time(e[r][1]) for e in ev) for r in pipe.rows}
+    step_ms = statistics.mean(e[first][0].elapsed_time(e[last][1]) for e in ev)
+    return row_ms, max_over_ranks(step_ms, world, device), wall, clk
+
+
+def time_e2e(pipe, host_inputs, steps, world, device):
+    """The step through the public API with pinned host inputs copied in and
+    every result copied back inside the timed region."""
+    import torch
+
+    hk, hv, hq = host_inputs
+    outs = pipe.outputs()
+    host_outs = [torch.empty(o.shape, dtype=o.dtype, pin_memory=True) for o in outs]
+    h2d = sum(t.numel() * t.element_size() for t in (hk, hv, hq))
+    d2h = sum(t.numel() * t.element_size() for t in outs)
+    e_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    for k in range(steps + 1):  # first pass untimed
+        if k > 0:
+            e_ev[k - 1][0].record()
+        pipe.xk.copy_(hk, non_blocking=True)
+        pipe.xv.copy_(hv, non_blocking=True)
+        pipe.q.copy_(hq, non_blocking=True)
+        pipe.step()
+        for ho, o in zip(host_outs, outs):
+            ho.copy_(o, non_blocking=True)
+        if k > 0:
+            e_ev[k - 1][1].record()
+    torch.cuda.synchronize()
+    check_status(pipe.K, "after the end-to-end steps")
+    e2e_ms = max_over_ranks(statistics.mean(a.elapsed_time(b) for a, b in e_ev), world, device)
+    return {"value": world * pipe.w.history_tokens / (e2e_ms / 1e3), "unit": UNIT, "ms_per_step": e2e_ms,
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+            "what": "the whole step through the Python binding of the C ABI; the history, the queries and "
+                    "every result (centres, idx, codes, {s, z}, joint codes, O, LSE) cross PCIe each step"}
+
+
+def row_report(pipe, row_ms, hbm, tfl):
+    """Per-row ms and roofline fractions of one workload's step."""
+    w = pipe.w
+    wm = work_model(w)
+    gbps = lambda b, ms: b / (ms / 1e3) / 1e9
+    tflops = lambda f, ms: f / (ms / 1e3) / 1e12
+    enc_hbm = gbps(wm["encode_bytes"], row_ms["encode"])
+    enc_tc = tflops(wm["encode_flops"], row_ms["encode"])
+    attn = tflops(wm["attention_flops"], row_ms["attention"])
+    enc_hbm_roof_ms = wm["encode_bytes"] / (hbm * 1e9) * 1e3
+    enc_tc_roof_ms = wm["encode_flops"] / (tfl * 1e12) * 1e3
+    rows = {
+        "fit": {"ms": row_ms["fit"], "gbps": gbps(wm["fit_bytes"], row_ms["fit"]),
+                "hbm_frac": gbps(wm["fit_bytes"], row_ms["fit"]) / hbm},
+        "encode": {"ms": row_ms["encode"], "tokens_per_s": w.history_tokens / (row_ms["encode"] / 1e3),
+                   "gbps": enc_hbm, "hbm_frac": enc_hbm / hbm,
+                   "filter_tflops": enc_tc, "tensor_frac": enc_tc / tfl,
+                   "binding_roof": "tensor" if enc_tc_roof_ms > enc_hbm_roof_ms else "hbm",
+                   "roof_ms": max(enc_tc_roof_ms, enc_hbm_roof_ms),
+                   "roof_frac": max(enc_tc_roof_ms, enc_hbm_roof_ms) / row_ms["encode"]},
+        "decode": {"ms": row_ms["decode"], "gbps": gbps(wm["decode_bytes"], row_ms["decode"]),
+                   "hbm_frac": gbps(wm["decode_bytes"], row_ms["decode"]) / hbm},
+        "attention": {"ms": row_ms["attention"], "launches": pipe.blocks, "tflops": attn, "frac": attn / tfl},
+        "merge": {"ms": row_ms["merge"], "gbps": gbps(wm["merge_bytes"], row_ms["merge"]),
+                  "hbm_frac": gbps(wm["merge_bytes"], row_ms["merge"]) / hbm},
+    }
+    if pipe.joint is not None:
+        jm = joint_work_model(pipe.joint.w)
+        je, jd = row_ms["joint_encode"], row_ms["joint_decode"]
+        rows["joint_encode"] = {"ms": je, "gbps": gbps(jm["joint_enc_bytes"], je),
+                                "hbm_frac": gbps(jm["joint_enc_bytes"], je) / hbm,
+                                "tflops": tflops(jm["joint_gemm_flops"] / 2 + jm["joint_filter_flops"], je),
+                                "tensor_frac": tflops(jm["joint_gemm_flops"] / 2 + jm["joint_filter_flops"], je) / tfl,
+                                "workload": "joint (12 heads, 32,760 tokens, rank 192, K4V4, G 32)"}
+        rows["joint_decode"] = {"ms": jd, "gbps": gbps(jm["joint_dec_bytes"], jd),
+                                "hbm_frac": gbps(jm["joint_dec_bytes"], jd) / hbm,
+                                "gemm_tflops": tflops(jm["joint_gemm_flops"] / 2, jd),
+                                "workload": "joint (12 heads, 32,760 tokens, rank 192, K4V4, G 32)"}
+    return rows
+
+
+def workload_config(w, world, extra=""):
+    return {"workload": f"{w.name}-like layer: {w.num_heads} heads x {w.head_dim}, history {w.history_tokens} "
+                        f"tokens ({w.frames} frames x {w.tokens_per_frame}), query chunk {w.query_tokens}, "
+                        f"C={w.num_centroids}, K{w.bits_k}V{w.bits_v}, group {w.group_size}, fit "
+                        f"{w.kmeans_iters} rounds, {max(w.history_blocks, 2)} history blocks{extra}",
+            "history_tokens": w.history_tokens, "query_tokens": w.query_tokens, "heads": w.num_heads,
+            "head_dim": w.head_dim, "centroids": w.num_centroids, "bits_k": w.bits_k, "bits_v": w.bits_v,
+            "group": w.group_size, "history_blocks": max(w.history_blocks, 2),
+            "parallelism": f"replicas x{world}", "l2": "flushed (256 MiB write) before each step"}
+
+
 def run_gpu(args):
     import torch
 
@@ -365,131 +564,67 @@ def run_gpu(args):
     torch.cuda.set_device(local)
     device = torch.device("cuda", local)
     init_dist(world, "nccl")
-    w = synth.workload(WORKLOAD)
-
-    # seeded inputs: generated on the host, staged in pinned memory
-    hk = synth.make_history(w, "K")
-    hv = synth.make_history(w, "V")
-    hq = synth.make_queries(w)
-    pin = lambda a: torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).pin_memory()
-    pk, pv, pq = pin(hk), pin(hv), pin(hq)
-
-    pipe = Pipeline(w, device)
-    pipe.xk.copy_(pk)
-    pipe.xv.copy_(pv)
-    pipe.q.copy_(pq)
-    pipe.kc.copy_(pin(synth.make_chunk(w, "K")))
-    pipe.vc.copy_(pin(synth.make_chunk(w, "V")))
+    hbm, tfl, peak_kind = measured_peaks()
     flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=device)
-    torch.cuda.synchronize()
 
-    for _ in range(args.warmup):
-        flush.zero_()
-        pipe.step()
+    # ---- headline: the 14B-like layer, with the joint rows on their workload
+    w = synth.workload(HEADLINE)
+    hk, hv, hq = (pinned_bf16(synth.make_history(w, "K")), pinned_bf16(synth.make_history(w, "V")),
+                  pinned_bf16(synth.make_queries(w)))
+    joint = JointRows(device)
+    pipe = Pipeline(w, device, joint=joint)
+    pipe.load_inputs(hk, hv, hq)
     torch.cuda.synchronize()
-    st = pipe.K.kvq_last_device_status()
-    if st != 0:
-        raise RuntimeError(f"device status after warm-up: {pipe.K.status_string(st)}")
-
-    ev = [{r: (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for r in Pipeline.ROWS}
-          for _ in range(args.steps)]
     clocks = ClockSampler(local)
-    barrier(world)
-    torch.cuda.synchronize()
-    clocks.start()
-    t_wall = time.perf_counter()
-    for k in range(args.steps):
-        flush.zero_()
-        pipe.step(ev[k])
-    torch.cuda.synchronize()
-    wall = time.perf_counter() - t_wall
-    barrier(world)
-    clk = clocks.stop()
-    st = pipe.K.kvq_last_device_status()
-    if st != 0:
-        raise RuntimeError(f"device status after timing: {pipe.K.status_string(st)}")
+    row_ms, ms_step, wall, clk = time_steps(pipe, args.steps, args.warmup, flush, world, device, clocks)
+    rows = row_report(pipe, row_ms, hbm, tfl)
+    # the attention launches of one step, one block per call: mean time per call
+    attn_call_ms = max_over_ranks(
+        statistics.mean(time_calls(lambda b=b: pipe.attention_block(b), max(3, args.steps // 4), 1, flush)
+                        for b in range(pipe.blocks)), world, device)
+    e2e = None if args.no_e2e else time_e2e(pipe, (hk, hv, hq), args.steps, world, device)
+    launches = pipe.launches_per_step * args.steps
+    del pipe, hk, hv, hq
+    torch.cuda.empty_cache()
 
-    # next to the step: the current chunk's full-layer attention (compressed
-    # history + its own uncompressed keys, merged by LSE) and the dense part
-    # alone, on the step's freshly encoded history
-    layer_ms = max_over_ranks(time_calls(pipe.layer_attention, args.steps, args.warmup, flush), world, device)
-    dense_ms = max_over_ranks(time_calls(pipe.dense_attention, args.steps, args.warmup, flush), world, device)
-    st = pipe.K.kvq_last_device_status()
-    if st != 0:
-        raise RuntimeError(f"device status after the layer attention: {pipe.K.status_string(st)}")
-
-    row_ms = {r: [e[r][0].elapsed_time(e[r][1]) for e in ev] for r in Pipeline.ROWS}
-    step_ms = [ev[k]["fit"][0].elapsed_time(ev[k]["merge"][1]) for k in range(args.steps)]
-    ms_step_local = statistics.mean(step_ms)
-    ms_step = max_over_ranks(ms_step_local, world, device)
-    row_mean = {r: statistics.mean(v) for r, v in row_ms.items()}
-
-    # end-to-end through the public API with host buffers
-    e2e = None
-    if not args.no_e2e:
-        outs = pipe.outputs()
-        host_outs = [torch.empty(o.shape, dtype=o.dtype, pin_memory=True) for o in outs]
-        h2d = sum(t.numel() * t.element_size() for t in (pk, pv, pq))
-        d2h = sum(t.numel() * t.element_size() for t in outs)
-        e_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-                for _ in range(args.steps)]
-        for k in range(args.steps + 1):  # first pass untimed
-            if k > 0:
-                e_ev[k - 1][0].record()
-            pipe.xk.copy_(pk, non_blocking=True)
-            pipe.xv.copy_(pv, non_blocking=True)
-            pipe.q.copy_(pq, non_blocking=True)
-            pipe.step()
-            for ho, o in zip(host_outs, outs):
-                ho.copy_(o, non_blocking=True)
-            if k > 0:
-                e_ev[k - 1][1].record()
+    # ---- the Wan-1.3B-like step, then its chunk's full-layer attention
+    secondary = None
+    next_rows = None
+    if not args.no_secondary:
+        w2 = synth.workload(SECONDARY)
+        p2 = Pipeline(w2, device, layer=True)
+        p2.load_inputs(pinned_bf16(synth.make_history(w2, "K")), pinned_bf16(synth.make_history(w2, "V")),
+                       pinned_bf16(synth.make_queries(w2)))
+        p2.kc.copy_(pinned_bf16(synth.make_chunk(w2, "K")))
+        p2.vc.copy_(pinned_bf16(synth.make_chunk(w2, "V")))
         torch.cuda.synchronize()
-        e2e_ms = max_over_ranks(statistics.mean(a.elapsed_time(b) for a, b in e_ev), world, device)
-        e2e = {"value": world * w.history_tokens / (e2e_ms / 1e3), "unit": UNIT, "ms_per_step": e2e_ms,
-               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
-
-    if rank == 0:
-        wm = work_model(w)
-        hbm, tfl, peak_kind = measured_peaks()
-        attn_launch_ms = row_mean["attention"] / HISTORY_BLOCKS
-        attn_launch_flops = wm["attention_flops"] / HISTORY_BLOCKS
-        attn_tflops = attn_launch_flops / (attn_launch_ms / 1e3) / 1e12
-        enc_gbps = wm["encode_bytes"] / (row_mean["encode"] / 1e3) / 1e9
-        dec_gbps = wm["decode_bytes"] / (row_mean["decode"] / 1e3) / 1e9
-        merge_gbps = wm["merge_bytes"] / (row_mean["merge"] / 1e3) / 1e9
-        fit_gbps = wm["fit_bytes"] / (row_mean["fit"] / 1e3) / 1e9
-        jenc_gbps = wm["joint_enc_bytes"] / (row_mean["joint_encode"] / 1e3) / 1e9
-        jdec_gbps = wm["joint_dec_bytes"] / (row_mean["joint_decode"] / 1e3) / 1e9
-        jdec_tflops = wm["joint_gemm_flops"] / 2 / (row_mean["joint_decode"] / 1e3) / 1e12
-        jenc_tflops = wm["joint_gemm_flops"] / 2 / (row_mean["joint_encode"] / 1e3) / 1e12
-        rows = {
-            "fit": {"ms": row_mean["fit"], "gbps": fit_gbps, "hbm_frac": fit_gbps / hbm},
-            "encode": {"ms": row_mean["encode"], "tokens_per_s": w.history_tokens / (row_mean["encode"] / 1e3),
-                       "gbps": enc_gbps, "hbm_frac": enc_gbps / hbm},
-            "decode": {"ms": row_mean["decode"], "gbps": dec_gbps, "hbm_frac": dec_gbps / hbm},
-            "joint_encode": {"ms": row_mean["joint_encode"], "gbps": jenc_gbps, "hbm_frac": jenc_gbps / hbm,
-                             "gemm_tflops": jenc_tflops},
-            "joint_decode": {"ms": row_mean["joint_decode"], "gbps": jdec_gbps, "hbm_frac": jdec_gbps / hbm,
-                             "gemm_tflops": jdec_tflops},
-            "attention": {"ms": row_mean["attention"], "launches": HISTORY_BLOCKS, "tflops": attn_tflops,
-                          "frac": attn_tflops / tfl},
-            "merge": {"ms": row_mean["merge"], "gbps": merge_gbps, "hbm_frac": merge_gbps / hbm},
-        }
-        Tq, H, d = w.query_tokens, w.num_heads, w.head_dim
-        layer_flops = 4.0 * Tq * (w.history_tokens + Tq) * d * H
+        r2, ms2, _, _ = time_steps(p2, args.steps, args.warmup, flush, world, device)
+        secondary = {"value": world * w2.history_tokens / (ms2 / 1e3), "unit": UNIT, "ms_per_step": ms2,
+                     "config": workload_config(w2, world), "rows": row_report(p2, r2, hbm, tfl)}
+        layer_ms = max_over_ranks(time_calls(p2.layer_attention, args.steps, args.warmup, flush), world, device)
+        dense_ms = max_over_ranks(time_calls(p2.dense_attention, args.steps, args.warmup, flush), world, device)
+        check_status(p2.K, "after the layer attention")
+        Tq, H, d = w2.query_tokens, w2.num_heads, w2.head_dim
+        layer_flops = 4.0 * Tq * (w2.history_tokens + Tq) * d * H
         dense_flops = 4.0 * Tq * Tq * d * H
         next_rows = {
-            "layer_attention": {"ms": layer_ms, "calls": 1, "keys": w.history_tokens + Tq,
+            "layer_attention": {"ms": layer_ms, "calls": 1, "keys": w2.history_tokens + Tq,
                                 "tflops": layer_flops / (layer_ms / 1e3) / 1e12,
                                 "frac": layer_flops / (layer_ms / 1e3) / 1e12 / tfl,
-                                "what": "kvq_layer_attention: 32760 compressed history keys + the 4680-key chunk "
-                                        "(bf16), one softmax, LSE merge inside the call"},
+                                "what": "kvq_layer_attention on the Wan-like layer: 32760 compressed history "
+                                        "keys + the 4680-key chunk (bf16), one softmax, LSE merge in the call"},
             "dense_attention": {"ms": dense_ms, "calls": 1, "keys": Tq,
                                 "tflops": dense_flops / (dense_ms / 1e3) / 1e12,
                                 "frac": dense_flops / (dense_ms / 1e3) / 1e12 / tfl,
-                                "what": "kvq_attention_dense_lse over the 4680-key chunk alone"},
+                                "what": "kvq_attention_dense_lse over the Wan-like 4680-key chunk alone"},
         }
+        launches += p2.launches_per_step * args.steps
+        del p2
+        torch.cuda.empty_cache()
+
+    if rank == 0:
+        wm = work_model(w)
+        attn_tflops = wm["attention_flops"] / pipe_blocks(w) / (attn_call_ms / 1e3) / 1e12
         line = {
             "metric": METRIC,
             "value": world * w.history_tokens / (ms_step / 1e3),
@@ -503,22 +638,21 @@ def run_gpu(args):
             "vs_baseline": None,
             "dtype": "bf16",
             "data": "synthetic (seeded AR(1) frames + heavy-tailed outlier channels)",
-            "config": {"workload": "wan13b-like layer: 12 heads x 128, history 32760 tokens (21 frames x 1560), "
-                                   "query chunk 4680, C=256, K2V2, group 16, fit 2 rounds, 2 history blocks; "
-                                   "joint code of the same history: rank 192, K4V4, group 32",
-                       "history_tokens": w.history_tokens, "query_tokens": w.query_tokens,
-                       "heads": w.num_heads, "head_dim": w.head_dim, "centroids": w.num_centroids,
-                       "bits_k": w.bits_k, "bits_v": w.bits_v, "group": w.group_size,
-                       "parallelism": f"replicas x{world}", "l2": "flushed (256 MiB write) before each step"},
-            "roofline": {"kernel": "attention_pair_kernel<2, 2, false> (time of the whole kvq_attention_lse call, "
-                                   "incl. its in-call LSE merge)", "bound": "tensor", "achieved": attn_tflops,
-                         "peak": tfl, "unit": "TFLOP/s", "frac": attn_tflops / tfl, "peak_kind": peak_kind,
+            "config": workload_config(w, world, extra="; the step also runs the joint head-channel code "
+                                                      "(rank 192, K4V4, group 32) of the joint workload's "
+                                                      "32,760-token, 12-head history"),
+            "roofline": {"kernel": "compressed-history attention, one kvq_attention_lse call per history block "
+                                   "(11,700 keys; incl. the call's own LSE merge of its sub-ranges)",
+                         "bound": "tensor", "achieved": attn_tflops, "peak": tfl, "unit": "TFLOP/s",
+                         "frac": attn_tflops / tfl, "peak_kind": f"{peak_kind} (bf16 dense, burst)",
                          "traffic": ATTN_NCU_TRAFFIC_BYTES,
-                         "traffic_unit": "bytes per launch (ncu dram__bytes_read.sum + dram__bytes_write.sum)"},
+                         "traffic_unit": "bytes per launch (ncu dram__bytes_read.sum + dram__bytes_write.sum)",
+                         "ms_per_launch": attn_call_ms},
             "rows": rows,
+            "config2": secondary,
             "next_rows": next_rows,
             "clocks": clk,
-            "gpu_launches": pipe.launches_per_step * args.steps,
+            "gpu_launches": launches,
             "wall_s_timed_region": wall,
             "e2e": e2e,
         }
@@ -528,23 +662,110 @@ def run_gpu(args):
     barrier(world)
 
 
+def pipe_blocks(w):
+    return w.history_blocks if w.history_blocks > 1 else 2
+
+
+# ----------------------------------------------------------------------------
+# sweep: encode, decode and attention per point (covering set)
+# ----------------------------------------------------------------------------
+
+def sweep_points():
+    """A covering set of the 12-head sweep: every (b_K, b_V), every G, every
+    C and every T of 4k-128k appear; both query-chunk lengths appear."""
+    Ts = [4096, 8192, 16384, 32768, 65536, 131072]
+    pts = []
+    combos = [(2, 2, 16, 64), (2, 4, 32, 256), (4, 2, 64, 1024), (4, 4, 16, 256), (2, 2, 64, 256),
+              (4, 4, 32, 64)]
+    for i, T in enumerate(Ts):
+        bk, bv, G, C = combos[i % len(combos)]
+        pts.append((T, 4680 if i % 2 == 0 else 1560, bk, bv, G, C))
+    pts.append((131072, 4680, 2, 2, 16, 1024))
+    pts.append((4096, 1560, 4, 4, 64, 1024))
+    return pts
+
+
+def run_sweep(args):
+    import torch
+
+    from kv_cache_compression_head_b200 import kvq as K
+    from kv_cache_compression_head_b200 import synth
+
+    device = torch.device("cuda", 0)
+    torch.cuda.set_device(device)
+    hbm, tfl, _ = measured_peaks()
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=device)
+    base = synth.sweep_point(131072, 4680, 2, 2, 16, 256)
+    full_k = to_device_bf16(synth.make_history(base, "K"), device)
+    full_v = to_device_bf16(synth.make_history(base, "V"), device)
+    full_q = to_device_bf16(synth.make_queries(base), device)
+    with open(args.sweep, "w") as out:
+        for (T, Tq, bk, bv, G, C) in sweep_points():
+            w = synth.sweep_point(T, Tq, bk, bv, G, C)
+            H, d = w.num_heads, w.head_dim
+            xk, xv, q = full_k[:T].contiguous(), full_v[:T].contiguous(), full_q[:Tq].contiguous()
+            ck, cv = K.Codec(H, d, C, bk, G), K.Codec(H, d, C, bv, G)
+            cent = [torch.empty((H, C, d), dtype=torch.bfloat16, device=device) for _ in range(2)]
+            ws = K.alloc_workspace(K.KVQ_OP_FIT, ck, T, device)
+            K.kvq_fit_centroids(ck, xk, 2, cent[0], ws)
+            K.kvq_fit_centroids(cv, xv, 2, cent[1], ws)
+            enc = [K.alloc_encoded(c, T, device) for c in (ck, cv)]
+            comp = [K.Compressed(c, T, cent[i], *enc[i]) for i, c in enumerate((ck, cv))]
+            dec = torch.empty((T, H, d), dtype=torch.bfloat16, device=device)
+            o = torch.empty((Tq, H, d), dtype=torch.float32, device=device)
+            lse = torch.empty((H, Tq), dtype=torch.float32, device=device)
+            ws_a = K.alloc_workspace(K.KVQ_OP_ATTENTION, ck, T, device, num_queries=Tq)
+
+            def encode():
+                K.kvq_encode(ck, xk, cent[0], *enc[0])
+                K.kvq_encode(cv, xv, cent[1], *enc[1])
+
+            def decode():
+                K.kvq_decode(comp[0], dec)
+                K.kvq_decode(comp[1], dec)
+
+            def attention():
+                K.kvq_attention_lse(q, comp[0], comp[1], o, lse, workspace=ws_a)
+
+            reps = 10
+            enc_ms = time_calls(encode, reps, 3, flush)
+            dec_ms = time_calls(decode, reps, 3, flush)
+            att_ms = time_calls(attention, reps, 3, flush)
+            check_status(K, f"after sweep point {w.name}")
+            wm = work_model(w)
+            rec = {"point": {"T": T, "Tq": Tq, "bits_k": bk, "bits_v": bv, "group": G, "centroids": C},
+                   "encode_ms": enc_ms, "encode_gbps": wm["encode_bytes"] / enc_ms / 1e6,
+                   "encode_hbm_frac": wm["encode_bytes"] / enc_ms / 1e6 / hbm,
+                   "encode_filter_tflops": wm["encode_flops"] / enc_ms / 1e9,
+                   "decode_ms": dec_ms, "decode_gbps": wm["decode_bytes"] / dec_ms / 1e6,
+                   "decode_hbm_frac": wm["decode_bytes"] / dec_ms / 1e6 / hbm,
+                   "attention_ms": att_ms, "attention_tflops": wm["attention_flops"] / att_ms / 1e9,
+                   "attention_frac": wm["attention_flops"] / att_ms / 1e9 / tfl}
+            out.write(json.dumps(rec) + "\n")
+            out.flush()
+            print(json.dumps(rec), flush=True)
+            del xk, xv, q, cent, ws, enc, comp, dec, o, lse, ws_a
+            torch.cuda.empty_cache()
+
+
 # ----------------------------------------------------------------------------
 # CPU oracle: baseline leg and reference arm
 # ----------------------------------------------------------------------------
 
-CPU_SAMPLE_T = 4096
+CPU_SAMPLE_T = 2048
 CPU_SAMPLE_TQ = 256
+CPU_REPEATS = 3
 
 
 def oracle_step_times(w):
     """Time the oracle on a bounded sample of the workload: fit+encode+decode
     of the first CPU_SAMPLE_T history tokens (all heads, K and V) and attention
-    (2 blocks) + merge of CPU_SAMPLE_TQ queries over them.  Returns the
-    extrapolated seconds of one full step and the raw sample times."""
+    over the same number of blocks + merge of CPU_SAMPLE_TQ queries over them.
+    Returns (wall seconds of the sample, its extrapolation to one full step)."""
     from kv_cache_compression_head_b200 import synth
     from oracle import oracle as O
 
-    Ts, Tqs = CPU_SAMPLE_T, CPU_SAMPLE_TQ
+    Ts, Tqs = min(CPU_SAMPLE_T, w.history_tokens), min(CPU_SAMPLE_TQ, w.query_tokens)
     xk = synth.make_history(w, "K", max_tokens=Ts)
     xv = synth.make_history(w, "V", max_tokens=Ts)
     q = synth.make_queries(w, max_tokens=Tqs)
@@ -555,26 +776,34 @@ def oracle_step_times(w):
         e = O.encode(x, cent, bits, w.group_size)
         decs.append(O.decode(*e, cent, bits, w.group_size))
     t1 = time.perf_counter()
-    edges = [Ts * i // HISTORY_BLOCKS for i in range(HISTORY_BLOCKS + 1)]
+    nb = pipe_blocks(w)
+    edges = [Ts * i // nb for i in range(nb + 1)]
     parts = [O.attention(q, decs[0][a:b], decs[1][a:b]) for a, b in zip(edges[:-1], edges[1:])]
     O.lse_merge([p[0] for p in parts], [p[1] for p in parts])
     t2 = time.perf_counter()
     codec_s, attn_s = t1 - t0, t2 - t1
     full = codec_s * (w.history_tokens / Ts) + attn_s * (w.history_tokens * w.query_tokens) / (Ts * Tqs)
-    return full, codec_s, attn_s
+    return t2 - t0, full
 
 
 def _omp_threads():
     return int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
 
 
+def _sample_text(w):
+    return (f"fit+encode+decode of {min(CPU_SAMPLE_T, w.history_tokens)}/{w.history_tokens} history tokens "
+            f"({w.num_heads} heads, K and V, C={w.num_centroids}) and attention ({pipe_blocks(w)} blocks)+merge "
+            f"of {min(CPU_SAMPLE_TQ, w.query_tokens)}/{w.query_tokens} queries over them; scaled per history "
+            f"token and per query x history token to the full step")
+
+
 def cpu_baseline(w):
-    full, codec_s, attn_s = oracle_step_times(w)
-    return {"value": w.history_tokens / full, "unit": UNIT, "cores": _omp_threads(), "kind": "oracle",
-            "sample": f"fit+encode+decode of {CPU_SAMPLE_T}/{w.history_tokens} history tokens (12 heads, K and V): "
-                      f"{codec_s:.2f}s; attention (2 blocks)+merge of {CPU_SAMPLE_TQ}/{w.query_tokens} queries "
-                      f"over them: {attn_s:.2f}s; scaled per history token and per query x history token",
-            "extrapolated_s_per_step": full}
+    runs = [oracle_step_times(w) for _ in range(CPU_REPEATS)]
+    rates = sorted(w.history_tokens / full for _, full in runs)
+    return {"value": statistics.median(rates), "unit": UNIT, "cores": _omp_threads(), "kind": "oracle",
+            "repeats": CPU_REPEATS, "min": rates[0], "max": rates[-1],
+            "spread": (rates[-1] - rates[0]) / statistics.median(rates),
+            "sample": _sample_text(w), "sample_s": statistics.median(s for s, _ in runs)}
 
 
 def run_reference(args):
@@ -585,26 +814,28 @@ def run_reference(args):
         return
     from kv_cache_compression_head_b200 import synth
 
-    w = synth.workload(WORKLOAD)
+    w = synth.workload(HEADLINE)
     for _ in range(args.warmup):
         oracle_step_times(w)
-    fulls = []
+    samples, fulls = [], []
     t_wall = time.perf_counter()
     for _ in range(args.steps):
-        fulls.append(oracle_step_times(w)[0])
+        s, full = oracle_step_times(w)
+        samples.append(s)
+        fulls.append(full)
     wall = time.perf_counter() - t_wall
-    s = statistics.mean(fulls)
-    value = w.history_tokens / s
+    value = w.history_tokens / statistics.median(fulls)
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": s * 1e3, "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "f32/f64 (CPU oracle)", "data": "synthetic",
-        "config": {"workload": "wan13b-like layer (bounded sample per step, extrapolated)",
-                   "history_tokens": w.history_tokens, "query_tokens": w.query_tokens,
-                   "parallelism": "rank 0 only"},
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": wall / args.steps * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32/f64 (CPU oracle)",
+        "data": "synthetic",
+        "config": {**workload_config(w, world), "parallelism": "rank 0 only",
+                   "sample": "each step runs the bounded sample below; value is the full step's rate "
+                             "extrapolated from it"},
+        "extrapolated_ms_per_full_step": statistics.median(fulls) * 1e3,
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": _omp_threads(), "kind": "oracle",
-                         "sample": f"each step: fit+encode+decode of {CPU_SAMPLE_T} history tokens and attention "
-                                   f"of {CPU_SAMPLE_TQ} queries over them, extrapolated to the full step"},
+                         "sample": _sample_text(w)},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
         "wall_s_timed_region": wall,
     }
@@ -615,6 +846,9 @@ def main():
     args = parse_args()
     if args.warmup < 0 or args.steps < 1:
         raise SystemExit("need --steps >= 1 and --warmup >= 0")
+    if args.sweep:
+        run_sweep(args)
+        return
     if args.impl == "reference":
         run_reference(args)
     else:

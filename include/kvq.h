@@ -165,8 +165,10 @@ KVQ_API kvq_status kvq_fit_centroids(const kvq_codec_desc *desc, const void *x, 
  *    events.  Sums and counts are cleared at the start of every round, so
  *    no state carries over from an earlier call.
  *  - The first call on each device looks up the array's device address
- *    (cudaGetSymbolAddress with that device current); make that first call
- *    before any stream capture.
+ *    (cudaGetSymbolAddress with that device current) and caches it; make
+ *    that first call before any stream capture.  The cache is not refreshed
+ *    by a cudaDeviceReset: do not use this call across a device reset in one
+ *    process.
  * Other arguments, validation and results are those of kvq_fit_centroids.
  */
 KVQ_API kvq_status kvq_fit_centroids_static(const kvq_codec_desc *desc, const void *x, kvq_dtype x_dtype,

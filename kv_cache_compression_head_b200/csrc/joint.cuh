@@ -10,8 +10,8 @@
 //   per row, Eq. 1 on each group of G coefficients -> packed codes, {s, z}
 // The A operand (R) is built in shared memory by the CTA's threads, 64
 // channels per K-block; W_enc [H d][r] (r contiguous) is the MN-major B
-// operand.  Two stages: the threads build K-block k+1 while the MMAs of block
-// k run.
+// operand.  A ring of four stages: TMA brings K-blocks up to three ahead while
+// the threads rebuild block k in place and the MMAs of earlier blocks run.
 //
 // Decoder, per 128-token tile and 128 output channels (one head):
 //   c^[t][n] = (q - z) s                       (binary32, the quantiser's grid)

@@ -4,6 +4,8 @@
 #include <cuda.h>
 #include <cudaTypedefs.h>
 #include <math.h>
+
+#include <atomic>
 #include <stdint.h>
 #include <stdio.h>
 #include <stdlib.h>
@@ -807,23 +809,27 @@ static __device__ __align__(256) unsigned char g_fit_static_scratch[KVQ_FIT_STAT
 
 namespace {
 
+// The address is cached per device.  Two host threads making their first call
+// at the same time both look it up and store the same value; the atomics make
+// that well defined.  The cache is not refreshed after cudaDeviceReset, so the
+// library must not be used across a device reset in one process.
 void *fit_static_scratch(kvq_status *st)
 {
-    static void *by_device[64] = {};
+    static std::atomic<void *> by_device[64];
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) {
         *st = KVQ_ERR_CUDA;
         return nullptr;
     }
-    if (!by_device[dev]) {
-        void *p = nullptr;
+    void *p = by_device[dev].load(std::memory_order_acquire);
+    if (!p) {
         if (cudaGetSymbolAddress(&p, g_fit_static_scratch) != cudaSuccess || !p) {
             *st = KVQ_ERR_CUDA;
             return nullptr;
         }
-        by_device[dev] = p;
+        by_device[dev].store(p, std::memory_order_release);
     }
-    return by_device[dev];
+    return p;
 }
 
 }  // namespace

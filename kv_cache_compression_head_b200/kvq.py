@@ -123,12 +123,81 @@ def _dtype_code(t: torch.Tensor) -> int:
     raise TypeError(f"unsupported dtype {t.dtype}")
 
 
-def _need_bf16(what: str, *ts: Optional[torch.Tensor]) -> None:
-    """The C ABI takes queries, dense keys and values as raw bf16 bits; a
-    tensor of another dtype would be misread, so it is refused here."""
+_IDX_DTYPES = (torch.int16, getattr(torch, "uint16", torch.int16))
+
+
+def _want(what: str, t: Optional[torch.Tensor], dtypes, shape=None, numel=None, min_numel=None) -> None:
+    """Refuse a tensor the library would misread or overrun.
+
+    The C ABI takes raw pointers, so a wrong dtype, shape, stride or device
+    would become an out-of-bounds access on the GPU rather than an error.
+    Checked here: present, dtype, shape / element count, contiguity.  The
+    device is checked by _on_cuda once every tensor of a call has passed
+    these."""
+    if t is None:
+        raise ValueError(f"{what}: tensor required")
+    dtypes = dtypes if isinstance(dtypes, tuple) else (dtypes,)
+    if t.dtype not in dtypes:
+        raise TypeError(f"{what}: expected {' or '.join(str(d) for d in dtypes)}, got {t.dtype}")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{what}: expected shape {tuple(shape)}, got {tuple(t.shape)}")
+    if numel is not None and t.numel() != numel:
+        raise ValueError(f"{what}: expected {numel} elements, got {t.numel()}")
+    if min_numel is not None and t.numel() < min_numel:
+        raise ValueError(f"{what}: expected at least {min_numel} elements, got {t.numel()}")
+    if not t.is_contiguous():
+        raise ValueError(f"{what}: expected a contiguous tensor")
+
+
+def _on_cuda(what: str, *ts) -> None:
+    """Every tensor given (None skipped; Compressed records expanded) lives on a CUDA device."""
     for t in ts:
-        if t is not None and t.dtype != torch.bfloat16:
-            raise TypeError(f"{what}: expected bfloat16, got {t.dtype}")
+        if isinstance(t, Compressed):
+            _on_cuda(what, t.centroids, t.idx, t.codes, t.meta, t.w_dec)
+        elif t is not None and not t.is_cuda:
+            raise ValueError(f"{what}: expected CUDA tensors, got one on {t.device}")
+
+
+_X_DTYPES = (torch.bfloat16, torch.float32)
+
+
+def _want_history(what: str, codec: "Codec", x: torch.Tensor) -> int:
+    """x [T][H][d] in bf16 or float32; returns T."""
+    if x is None or x.dim() != 3:
+        raise ValueError(f"{what}: expected a [T][H][d] tensor")
+    _want(what, x, _X_DTYPES, shape=(x.shape[0], codec.num_heads, codec.head_dim))
+    return x.shape[0]
+
+
+def _want_encoded(what: str, codec: "Codec", num_tokens: int, idx, codes, meta) -> None:
+    ib, cb, mb = encoded_sizes(codec, num_tokens)
+    _want(f"{what} idx", idx, _IDX_DTYPES, numel=ib // 2)
+    _want(f"{what} codes", codes, torch.uint8, numel=cb)
+    _want(f"{what} meta", meta, torch.float32, numel=mb // 4)
+
+
+def _want_workspace(what: str, ws: Optional[torch.Tensor]) -> None:
+    if ws is not None:
+        _want(f"{what} workspace", ws, torch.uint8)
+
+
+def _want_compressed(what: str, comp: "Compressed") -> None:
+    c = comp.codec
+    _want(f"{what} centroids", comp.centroids, torch.bfloat16, shape=(c.num_heads, c.num_centroids, c.head_dim))
+    _want_encoded(what, c, comp.num_tokens, comp.idx, comp.codes, comp.meta)
+    if comp.w_dec is not None:
+        _want(f"{what} w_dec", comp.w_dec, torch.bfloat16, shape=(c.joint_rank, c.num_heads * c.head_dim))
+
+
+def _want_attention_io(what: str, q: torch.Tensor, H: int, d: int, o_out, lse_out) -> int:
+    """q [Tq][H][d] bf16, o_out [Tq][H][d] bf16/float32, lse_out [H][Tq] float32; returns Tq."""
+    if q is None or q.dim() != 3:
+        raise ValueError(f"{what}: expected queries [Tq][H][d]")
+    Tq = q.shape[0]
+    _want(f"{what} q", q, torch.bfloat16, shape=(Tq, H, d))
+    _want(f"{what} o_out", o_out, _X_DTYPES, shape=(Tq, H, d))
+    _want(f"{what} lse_out", lse_out, torch.float32, shape=(H, Tq))
+    return Tq
 
 
 # ----------------------------------------------------------------------------
@@ -206,9 +275,13 @@ def alloc_workspace(op: int, codec: Codec, num_tokens: int, device, num_queries:
 
 def kvq_fit_centroids(codec: Codec, x: torch.Tensor, iters: int, centroids_out: torch.Tensor,
                       workspace: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
-    T = x.shape[0]
+    T = _want_history("kvq_fit_centroids x", codec, x)
+    _want("kvq_fit_centroids centroids_out", centroids_out, torch.bfloat16,
+          shape=(codec.num_heads, codec.num_centroids, codec.head_dim))
     if workspace is None:
         workspace = alloc_workspace(KVQ_OP_FIT, codec, T, x.device)
+    _want_workspace("kvq_fit_centroids", workspace)
+    _on_cuda("kvq_fit_centroids", x, centroids_out, workspace)
     d = codec.c()
     _check(_lib.kvq_fit_centroids(ctypes.byref(d), _ptr(x), _dtype_code(x), T, iters, _ptr(centroids_out),
                                   _ptr(workspace), workspace.numel() if workspace is not None else 0,
@@ -219,6 +292,10 @@ def kvq_fit_centroids(codec: Codec, x: torch.Tensor, iters: int, centroids_out: 
 def kvq_fit_centroids_static(codec: Codec, x: torch.Tensor, iters: int, centroids_out: torch.Tensor,
                              stream=None) -> torch.Tensor:
     """kvq_fit_centroids with the library's fixed device scratch (no workspace)."""
+    _want_history("kvq_fit_centroids_static x", codec, x)
+    _want("kvq_fit_centroids_static centroids_out", centroids_out, torch.bfloat16,
+          shape=(codec.num_heads, codec.num_centroids, codec.head_dim))
+    _on_cuda("kvq_fit_centroids_static", x, centroids_out)
     d = codec.c()
     _check(_lib.kvq_fit_centroids_static(ctypes.byref(d), _ptr(x), _dtype_code(x), x.shape[0], iters,
                                          _ptr(centroids_out), _stream(stream)), "kvq_fit_centroids_static")
@@ -228,6 +305,14 @@ def kvq_fit_centroids_static(codec: Codec, x: torch.Tensor, iters: int, centroid
 def kvq_encode(codec: Codec, x: torch.Tensor, centroids: torch.Tensor, idx: torch.Tensor, codes: torch.Tensor,
                meta: torch.Tensor, w_enc: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None,
                stream=None) -> None:
+    T = _want_history("kvq_encode x", codec, x)
+    _want("kvq_encode centroids", centroids, torch.bfloat16,
+          shape=(codec.num_heads, codec.num_centroids, codec.head_dim))
+    _want_encoded("kvq_encode", codec, T, idx, codes, meta)
+    if w_enc is not None:
+        _want("kvq_encode w_enc", w_enc, torch.bfloat16, shape=(codec.num_heads * codec.head_dim, codec.joint_rank))
+    _want_workspace("kvq_encode", workspace)
+    _on_cuda("kvq_encode", x, centroids, idx, codes, meta, w_enc, workspace)
     d = codec.c()
     _check(_lib.kvq_encode(ctypes.byref(d), _ptr(x), _dtype_code(x), x.shape[0], _ptr(centroids), _ptr(w_enc),
                            _ptr(idx), _ptr(codes), _ptr(meta), _ptr(workspace),
@@ -237,6 +322,15 @@ def kvq_encode(codec: Codec, x: torch.Tensor, centroids: torch.Tensor, idx: torc
 def kvq_joint_coefficients(codec: Codec, x: torch.Tensor, centroids: torch.Tensor, w_enc: torch.Tensor,
                            idx: torch.Tensor, coef_out: torch.Tensor, workspace: Optional[torch.Tensor] = None,
                            stream=None) -> None:
+    T = _want_history("kvq_joint_coefficients x", codec, x)
+    _want("kvq_joint_coefficients centroids", centroids, torch.bfloat16,
+          shape=(codec.num_heads, codec.num_centroids, codec.head_dim))
+    _want("kvq_joint_coefficients w_enc", w_enc, torch.bfloat16,
+          shape=(codec.num_heads * codec.head_dim, codec.joint_rank))
+    _want("kvq_joint_coefficients idx", idx, _IDX_DTYPES, numel=codec.num_heads * T)
+    _want("kvq_joint_coefficients coef_out", coef_out, torch.float32, shape=(T, codec.joint_rank))
+    _want_workspace("kvq_joint_coefficients", workspace)
+    _on_cuda("kvq_joint_coefficients", x, centroids, w_enc, idx, coef_out, workspace)
     d = codec.c()
     _check(_lib.kvq_joint_coefficients(ctypes.byref(d), _ptr(x), _dtype_code(x), x.shape[0], _ptr(centroids),
                                        _ptr(w_enc), _ptr(idx), _ptr(coef_out), _ptr(workspace),
@@ -246,6 +340,11 @@ def kvq_joint_coefficients(codec: Codec, x: torch.Tensor, centroids: torch.Tenso
 
 def kvq_decode(comp: Compressed, x_out: torch.Tensor, workspace: Optional[torch.Tensor] = None,
                stream=None) -> torch.Tensor:
+    _want_compressed("kvq_decode", comp)
+    c = comp.codec
+    _want("kvq_decode x_out", x_out, _X_DTYPES, shape=(comp.num_tokens, c.num_heads, c.head_dim))
+    _want_workspace("kvq_decode", workspace)
+    _on_cuda("kvq_decode", comp, x_out, workspace)
     v = comp.view()
     _check(_lib.kvq_decode(ctypes.byref(v), _ptr(x_out), _dtype_code(x_out), _ptr(workspace),
                            workspace.numel() if workspace is not None else 0, _stream(stream)), "kvq_decode")
@@ -255,7 +354,11 @@ def kvq_decode(comp: Compressed, x_out: torch.Tensor, workspace: Optional[torch.
 def kvq_attention_lse(q: torch.Tensor, k: Compressed, v: Compressed, o_out: torch.Tensor, lse_out: torch.Tensor,
                       t_begin: int = 0, t_end: Optional[int] = None, softmax_scale: float = 0.0,
                       workspace: Optional[torch.Tensor] = None, stream=None) -> None:
-    _need_bf16("kvq_attention_lse", q)
+    _want_compressed("kvq_attention_lse k", k)
+    _want_compressed("kvq_attention_lse v", v)
+    _want_attention_io("kvq_attention_lse", q, k.codec.num_heads, k.codec.head_dim, o_out, lse_out)
+    _want_workspace("kvq_attention_lse", workspace)
+    _on_cuda("kvq_attention_lse", q, k, v, o_out, lse_out, workspace)
     if t_end is None:
         t_end = k.num_tokens
     kv, vv = k.view(), v.view()
@@ -269,8 +372,14 @@ def kvq_attention_dense_lse(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, o
                             lse_out: torch.Tensor, t_begin: int = 0, t_end: Optional[int] = None,
                             softmax_scale: float = 0.0, workspace: Optional[torch.Tensor] = None, stream=None) -> None:
     """Attention over uncompressed bf16 keys/values k, v [Tk][H][d]."""
-    _need_bf16("kvq_attention_dense_lse", q, k, v)
+    if k is None or k.dim() != 3:
+        raise ValueError("kvq_attention_dense_lse: expected keys [Tk][H][d]")
     Tk, H, d = k.shape
+    _want("kvq_attention_dense_lse k", k, torch.bfloat16)
+    _want("kvq_attention_dense_lse v", v, torch.bfloat16, shape=(Tk, H, d))
+    _want_attention_io("kvq_attention_dense_lse", q, H, d, o_out, lse_out)
+    _want_workspace("kvq_attention_dense_lse", workspace)
+    _on_cuda("kvq_attention_dense_lse", q, k, v, o_out, lse_out, workspace)
     if t_end is None:
         t_end = Tk
     _check(_lib.kvq_attention_dense_lse(_ptr(q), q.shape[0], _ptr(k), _ptr(v), Tk, H, d, t_begin, t_end,
@@ -287,12 +396,22 @@ def kvq_layer_attention(q: torch.Tensor, k_hist: Compressed, v_hist: Compressed,
     """One softmax over the compressed history and the uncompressed keys
     k_cur, v_cur [Tc][H][d] (the current chunk and any raw protected tokens).
     The call needs a workspace; one is allocated when none is given."""
-    _need_bf16("kvq_layer_attention", q, k_cur, v_cur)
+    _want_compressed("kvq_layer_attention k_hist", k_hist)
+    _want_compressed("kvq_layer_attention v_hist", v_hist)
+    H, dh = k_hist.codec.num_heads, k_hist.codec.head_dim
+    _want_attention_io("kvq_layer_attention", q, H, dh, o_out, lse_out)
+    if k_cur is not None or v_cur is not None:
+        if k_cur is None or v_cur is None or k_cur.dim() != 3:
+            raise ValueError("kvq_layer_attention: k_cur and v_cur are given together as [Tc][H][d]")
+        _want("kvq_layer_attention k_cur", k_cur, torch.bfloat16, shape=(k_cur.shape[0], H, dh))
+        _want("kvq_layer_attention v_cur", v_cur, torch.bfloat16, shape=tuple(k_cur.shape))
     if t_end is None:
         t_end = k_hist.num_tokens
     if workspace is None:
         workspace = alloc_workspace(KVQ_OP_LAYER_ATTENTION, k_hist.codec, k_hist.num_tokens, q.device,
                                     num_queries=q.shape[0])
+    _want_workspace("kvq_layer_attention", workspace)
+    _on_cuda("kvq_layer_attention", q, k_hist, v_hist, k_cur, v_cur, o_out, lse_out, workspace)
     n_cur = 0 if k_cur is None else k_cur.shape[0]
     kv, vv = k_hist.view(), v_hist.view()
     _check(_lib.kvq_layer_attention(_ptr(q), q.shape[0], ctypes.byref(kv), ctypes.byref(vv), t_begin, t_end,
@@ -305,7 +424,17 @@ def kvq_layer_attention(q: torch.Tensor, k_hist: Compressed, v_hist: Compressed,
 def kvq_lse_merge(o_parts: Sequence[torch.Tensor], lse_parts: Sequence[torch.Tensor], o_out: torch.Tensor,
                   lse_out: torch.Tensor, stream=None) -> None:
     n = len(o_parts)
+    if n < 1 or len(lse_parts) != n:
+        raise ValueError("kvq_lse_merge: need matching, non-empty lists of partial outputs and LSEs")
+    if o_parts[0].dim() != 3:
+        raise ValueError("kvq_lse_merge: partial outputs are [Tq][H][d]")
     Tq, H, d = o_parts[0].shape
+    for i, (o, l) in enumerate(zip(o_parts, lse_parts)):
+        _want(f"kvq_lse_merge o_parts[{i}]", o, torch.float32, shape=(Tq, H, d))
+        _want(f"kvq_lse_merge lse_parts[{i}]", l, torch.float32, shape=(H, Tq))
+    _want("kvq_lse_merge o_out", o_out, _X_DTYPES, shape=(Tq, H, d))
+    _want("kvq_lse_merge lse_out", lse_out, torch.float32, shape=(H, Tq))
+    _on_cuda("kvq_lse_merge", *o_parts, *lse_parts, o_out, lse_out)
     arr_o = (ctypes.c_void_p * n)(*[t.data_ptr() for t in o_parts])
     arr_l = (ctypes.c_void_p * n)(*[t.data_ptr() for t in lse_parts])
     _check(_lib.kvq_lse_merge(n, arr_o, arr_l, Tq, H, d, _ptr(o_out), _dtype_code(o_out), _ptr(lse_out),

@@ -438,8 +438,3 @@ def compression_ratio(bits: int, group: int, meta_bits_per_group: int, base_bits
 def joint_nominal_ratio(channels: int, rank: int, coef_bits: int = 4, base_bits: int = 16) -> float:
     """Nominal coefficient compression: channels*16 / (rank*coef_bits)."""
     return channels * base_bits / (rank * coef_bits)
-
-
-def kv_cache_bytes(layers: int, tokens: int, width: int, bits: int = 16) -> float:
-    """Uncompressed K+V storage: 2 * L * T * C * bits / 8 bytes."""
-    return 2 * layers * tokens * width * bits / 8

@@ -191,12 +191,78 @@ def test_binding_refuses_non_bf16_queries_keys_values(K):
         K.kvq_attention_dense_lse(f, b, b, o, lse)
     with pytest.raises(TypeError):
         K.kvq_attention_dense_lse(b, b, f, o, lse)
-    codec = K.Codec(2, 64, 4, 2, 16)
-    comp = K.Compressed(codec, 4, b, b, b, b)
+    comp = _cpu_compressed(K, K.Codec(2, 64, 4, 2, 16), 4)
     with pytest.raises(TypeError):
         K.kvq_attention_lse(f, comp, comp, o, lse)
     with pytest.raises(TypeError):
-        K.kvq_layer_attention(b, comp, comp, f, b, o, lse, workspace=b)
+        K.kvq_layer_attention(b, comp, comp, f, b, o, lse, workspace=torch.zeros(16, dtype=torch.uint8))
+
+
+def _cpu_compressed(K, codec, T):
+    """A compressed record of the right dtypes and sizes, on the CPU."""
+    import torch
+
+    ib, cb, mb = K.encoded_sizes(codec, T)
+    cent = torch.zeros((codec.num_heads, codec.num_centroids, codec.head_dim), dtype=torch.bfloat16)
+    return K.Compressed(codec, T, cent, torch.zeros(ib // 2, dtype=torch.int16), torch.zeros(cb, dtype=torch.uint8),
+                        torch.zeros(mb // 4, dtype=torch.float32))
+
+
+def test_binding_checks_every_tensor_before_the_library(K):
+    """Every wrapper checks dtype, shape, contiguity and device of each tensor
+    before a pointer reaches the library: a float32 LSE buffer, a view of the
+    wrong head count or a CPU tensor would otherwise be read or written out of
+    bounds on the GPU.  With correct dtypes and shapes, CPU tensors are refused
+    for not being on a CUDA device."""
+    import torch
+
+    H, d, C, T, Tq = 2, 64, 4, 8, 4
+    codec = K.Codec(H, d, C, 2, 16)
+    comp = _cpu_compressed(K, codec, T)
+    bf = torch.bfloat16
+    q = torch.zeros((Tq, H, d), dtype=bf)
+    o = torch.zeros((Tq, H, d))
+    lse = torch.zeros((H, Tq))
+    x = torch.zeros((T, H, d), dtype=bf)
+    cent = torch.zeros((H, C, d), dtype=bf)
+    idx, codes, meta = comp.idx, comp.codes, comp.meta
+
+    def raises(exc, fn, *a, match=None, **kw):
+        with pytest.raises(exc, match=match):
+            fn(*a, **kw)
+
+    # attention: wrong LSE dtype, wrong head count in the output, CPU tensors
+    raises(TypeError, K.kvq_attention_lse, q, comp, comp, o, lse.to(bf))
+    raises(ValueError, K.kvq_attention_lse, q, comp, comp, torch.zeros((Tq, H + 1, d)), lse, match="shape")
+    raises(ValueError, K.kvq_attention_lse, q.transpose(0, 1).contiguous().transpose(0, 1), comp, comp, o, lse,
+           match="contiguous")
+    raises(ValueError, K.kvq_attention_lse, q, comp, comp, o, lse, match="CUDA")
+    raises(ValueError, K.kvq_attention_lse, q, _cpu_compressed(K, K.Codec(H, d, C, 4, 16), T - 1), comp, o,
+           torch.zeros((H, Tq)), match="CUDA")
+    bad = K.Compressed(codec, T, cent, idx, codes[:-1], meta)
+    raises(ValueError, K.kvq_attention_lse, q, bad, comp, o, lse, match="elements")
+    raises(ValueError, K.kvq_attention_dense_lse, q, x, x[:, :, :32], o, lse, match="shape")
+    raises(ValueError, K.kvq_attention_dense_lse, q, x, x, o, lse, match="CUDA")
+    raises(ValueError, K.kvq_layer_attention, q, comp, comp, x, x[:1], o, lse, match="shape")
+    raises(ValueError, K.kvq_layer_attention, q, comp, comp, x, None, o, lse, match="together")
+    # codec calls
+    raises(ValueError, K.kvq_fit_centroids, codec, x[:, :1], 2, cent, match="shape")
+    raises(TypeError, K.kvq_fit_centroids, codec, x, 2, cent.float())
+    raises(ValueError, K.kvq_fit_centroids_static, codec, x, 2, cent, match="CUDA")
+    raises(TypeError, K.kvq_encode, codec, x.to(torch.float16), cent, idx, codes, meta)
+    raises(TypeError, K.kvq_encode, codec, x, cent, idx.int(), codes, meta)
+    raises(ValueError, K.kvq_encode, codec, x, cent, idx, codes, meta[:-2], match="elements")
+    raises(ValueError, K.kvq_encode, codec, x, cent, idx, codes, meta, match="CUDA")
+    jc = K.Codec(H, d, C, 4, 32, 64)
+    raises(ValueError, K.kvq_joint_coefficients, jc, x, cent, torch.zeros((H * d, 32), dtype=bf), idx,
+           torch.zeros((T, 64)), match="shape")
+    raises(ValueError, K.kvq_decode, comp, torch.zeros((T - 1, H, d)), match="shape")
+    raises(ValueError, K.kvq_decode, comp, torch.zeros((T, H, d)), match="CUDA")
+    # merge: binary32 parts only, matching shapes
+    raises(TypeError, K.kvq_lse_merge, [o.to(bf), o], [lse, lse], o, lse)
+    raises(ValueError, K.kvq_lse_merge, [o, o], [lse, lse[:, :2]], o, lse, match="shape")
+    raises(ValueError, K.kvq_lse_merge, [o, o], [lse], o, lse, match="matching")
+    raises(ValueError, K.kvq_lse_merge, [o, o], [lse, lse], o, lse, match="CUDA")
 
 
 def test_binding_refuses_to_load_without_the_library(tmp_path):

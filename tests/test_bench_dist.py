@@ -48,7 +48,7 @@ def _reference_worker(rank: int, world: int, port: int, out_dir: str):
 
     import bench
 
-    bench.oracle_step_times = lambda w: (0.25, None)  # stands in for the oracle's timing
+    bench.oracle_step_times = lambda w: (0.25, 0.5)  # stands in for the oracle's timing
     args = type("A", (), {"steps": 2, "warmup": 1, "impl": "reference"})()
     buf = io.StringIO()
     with contextlib.redirect_stdout(buf):
@@ -69,6 +69,7 @@ def test_reference_arm_prints_on_rank0_only(tmp_path):
     assert len(lines) == 1
     rec = json.loads(lines[0])
     assert rec["impl"] == "reference" and rec["n_gpus"] == 2
-    assert rec["ms_per_step"] == pytest.approx(250.0)
+    assert rec["extrapolated_ms_per_full_step"] == pytest.approx(500.0)
+    assert rec["ms_per_step"] < 250.0  # the wall time it ran, not the stand-in figure
     assert rec["e2e"]["h2d_bytes_per_step"] == 0 and rec["cpu_baseline"]["kind"] == "oracle"
     assert (tmp_path / "r1.txt").read_text() == ""

@@ -7,23 +7,37 @@
 // bit-identical to the exact kernel in codec.cuh: the tensor cores only narrow
 // the search, the decision is taken by the specified binary32 distance.
 //
-// For a tile of 128 tokens of head h:
-//   1. TMA loads the tile X [128][d] (bf16, 128-byte swizzle) from [T][H][d];
-//   2. one thread issues P = X mu^T (M=128, N=C, K=d, fp32 in TMEM); the
-//      centres of the head stay resident in shared memory for every tile the
-//      CTA processes;
-//   3. two threads per token (one per half of the TMEM columns and of the
-//      channels) compute v_j = |mu_j|^2 - 2 p_j, the row minimum m and the
-//      candidate window  v_j <= m + kappa (|x| + max_j |mu_j|)^2,  which
-//      provably contains the specified argmin: kappa covers the tensor-core
-//      accumulation error, the rounding of |mu_j|^2 and of v_j, the rounding
-//      of the specified distance and the index bits carried in v.  When the
-//      second smallest v lies outside the window the smallest is the answer;
-//      when only the two smallest lie inside it, the two threads of the token
-//      each score one of them with the specified distance; otherwise the
-//      whole window is re-scored (lowest index wins ties everywhere);
-//   4. the residual against the chosen centre is quantised (Eq. 1) per group
-//      and packed, each thread covering its half of the channels.
+// Certified candidate set.  With R_j = |x| + |mu_j|, the tensor-core value
+// v~_j = |mu_j|^2 - 2 x.mu_j (binary32 norms, fp32 MMA accumulation, one
+// rounded FMA) is within tau R_j^2 of the exact |x - mu_j|^2 - |x|^2, and the
+// specified binary32 distance D_j is within gamma_{d+2} R_j^2 of the exact
+// squared distance.  Hence the specified argmin j* satisfies, for every j,
+//   L_j* <= U_j,   L_j = v~_j - k R_j^2,   U_j = v~_j + k R_j^2,
+// k = tau + gamma_{d+2} (plus margins for the rounding of L and the index
+// bits carried in v).  The scan ranks centres by L (three smallest kept) and
+// takes U of the first as the threshold: every centre with L <= U(first) is a
+// candidate, a superset of {j : L_j <= min U}.  The bound is per centre, so a
+// far-off centre with a large norm does not widen anyone's window.
+//
+// Persistent, warp-specialised kernel.  The (head, 128-token tile) units of
+// the whole call are split into equal contiguous ranges, one per CTA (one CTA
+// per SM), so a CTA changes head at most a few times; at each change the
+// CTA reloads that head's centres into shared memory.  Roles:
+//   warp 17 (TMA): loads X tiles [128][d] (bf16, 128-byte swizzle) from
+//     [T][H][d] into a ring of stages, as far ahead as the ring allows;
+//   warp 16 (MMA): one thread issues P = X mu^T (M = 128, K = d, fp32 in
+//     TMEM) in sub-units of up to 256 centre columns; tiles alternate between
+//     two epilogue groups, each with its own 256-column TMEM accumulator, so
+//     the tensor core fills one group's accumulator while the other reads;
+//   warps 0-7 and 8-15 (two epilogue groups, even and odd tiles): two threads
+//     per token (one per half of the TMEM columns and of the channels) compute
+//     L_j, keep the three smallest, release the accumulator, and decide: one
+//     candidate: done; two: the two threads of the token score one each with
+//     the specified distance; three or more: the warp pair scores every
+//     centre of the head with the specified distance (rare).  Lowest index
+//     wins ties everywhere.  Then the residual against the chosen centre is
+//     quantised (Eq. 1) per group and packed, each thread covering its half
+//     of the channels, and the X stage is released.
 #pragma once
 
 #include <cuda.h>
@@ -34,29 +48,39 @@
 namespace kvq {
 
 constexpr int kFltRows = 128;
-constexpr int kFltThreads = 256;
+constexpr int kFltGroupThreads = 256;            // one epilogue group: 8 warps
+constexpr int kFltMmaWarp = 16, kFltTmaWarp = 17;
+constexpr int kFltThreads = 576;
 constexpr int kFltMaxC = 512;
+constexpr int kFltAccCols = 256;                 // columns of one group's TMEM accumulator
+constexpr int kFltMaxStages = 4;
 
 struct FilterArgs {
     int64_t T;
     int H;
     int C;
     int Cpad;          // C rounded up to a multiple of 32
-    int tmem_cols;     // power of two >= max(32, Cpad)
+    int stages;        // X tiles in the ring (2 .. kFltMaxStages)
+    int64_t ntiles;    // 128-token tiles per head
     const uint16_t *cent;
     uint16_t *idx;
     uint8_t *codes;
     float *meta;
     int assign_only;
-    float kappa;       // window = kappa * (|x| + M)^2
+    float kappa;       // k of the certified bound (see above)
 };
 
-constexpr uint32_t kFltPairBytes = 7168u;  // pair exchange: float4 [2][128] | int [2][128] | float4 [128]
+// pair exchange of one epilogue group, two slots by tile parity:
+// float4 [2][2][128] | int [2][2][128] | float4 [128]
+constexpr uint32_t kFltPairBytes = 12288u;
 
-__host__ __device__ constexpr uint32_t flt_smem_bytes(int D, int Cpad)
+__host__ __device__ constexpr uint32_t flt_tile_bytes(int D) { return (uint32_t)(D * 2 * kFltRows); }
+
+__host__ __device__ constexpr uint32_t flt_smem_bytes(int D, int Cpad, int stages)
 {
-    // X tile | centres | norms | pair exchange | 2 barriers + slots
-    return (uint32_t)(D * 2 * kFltRows) + (uint32_t)(Cpad * D * 2) + (uint32_t)(Cpad * 4) + kFltPairBytes + 64u;
+    // X ring | centres | A_j, |mu_j| | pair exchange x 2 groups | barriers + slots
+    return (uint32_t)stages * flt_tile_bytes(D) + (uint32_t)(Cpad * D * 2) + (uint32_t)(Cpad * 8) +
+           2u * kFltPairBytes + 256u;
 }
 
 // Insert (v, c) into the ascending list (b1, c1) <= (b2, c2) <= (b3, c3);
@@ -107,94 +131,105 @@ __device__ __forceinline__ float spec_distance_smem(const uint8_t *sX, const uin
 }
 
 // Residual r = x - mu[best] of channels [half*CH, half*CH + CH) of one token,
-// read from the swizzled tiles, quantised per group (Eq. 1) and packed.  Two
-// passes over shared memory (min/max, then codes) keep r out of registers.
-// Group min/max use strict comparisons in channel order, as specified.
+// read from the swizzled tiles, quantised per group (Eq. 1) and packed.  Three
+// phases over all of the thread's groups at once, so that the groups' chains
+// (min/max, the two IEEE divisions of Eq. 1, the codes) run side by side:
+// (1) min and max of every group, (2) Eq. 1 parameters of every group,
+// (3) codes, re-reading the residuals from shared memory.  Group min/max are
+// those of a strict scan in channel order; the two differ only in the sign
+// of a zero extreme, for which the group is rescanned in order.
 template <int CH, int BITS, int G>
 __device__ __forceinline__ void encode_residual_smem(const uint8_t *sX, const uint8_t *sMu, int Cpad, int row,
                                                      int best, int half, uint8_t *codes_dst, float2 *meta_dst)
 {
     constexpr int kPerWord = 32 / BITS;
     constexpr int kWords = CH * BITS / 32;
+    constexpr int NG = CH / G;
+    // residual of the 8 channels of unit uu (0 .. CH/8) of this thread's half
+    auto unit_residual = [&](int uu, float *r8) {
+        const int u = half * (CH / 8) + uu;
+        const uint4 xw = *reinterpret_cast<const uint4 *>(sX + sw128_unit_offset(row, u, kFltRows));
+        const uint4 mw = *reinterpret_cast<const uint4 *>(sMu + sw128_unit_offset(best, u, Cpad));
+        const uint32_t xa[4] = {xw.x, xw.y, xw.z, xw.w}, ma[4] = {mw.x, mw.y, mw.z, mw.w};
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            const float2 d = sub2(make_float2(bf16_lo(xa[k]), bf16_hi(xa[k])), make_float2(bf16_lo(ma[k]), bf16_hi(ma[k])));
+            r8[2 * k] = d.x;
+            r8[2 * k + 1] = d.y;
+        }
+    };
+    // (1) min / max of every group
+    float mn[NG], mx[NG];
+#pragma unroll
+    for (int g = 0; g < NG; ++g) {
+        float r8[8];
+        unit_residual(g * (G / 8), r8);
+        float a = fminf(r8[0], r8[1]), b = fmaxf(r8[0], r8[1]);
+#pragma unroll
+        for (int c = 2; c < 8; c += 2) {
+            a = fmin3(a, r8[c], r8[c + 1]);
+            b = fmax3(b, r8[c], r8[c + 1]);
+        }
+#pragma unroll
+        for (int uu = 1; uu < G / 8; ++uu) {
+            unit_residual(g * (G / 8) + uu, r8);
+#pragma unroll
+            for (int c = 0; c < 8; c += 2) {
+                a = fmin3(a, r8[c], r8[c + 1]);
+                b = fmax3(b, r8[c], r8[c + 1]);
+            }
+        }
+        mn[g] = a;
+        mx[g] = b;
+    }
+#pragma unroll
+    for (int g = 0; g < NG; ++g) {
+        if (mn[g] == 0.0f || mx[g] == 0.0f) {
+            // a zero extreme: take its sign exactly as the ordered strict scan does
+            float a = 0.0f, b = 0.0f;
+            for (int uu = 0; uu < G / 8; ++uu) {
+                float r8[8];
+                unit_residual(g * (G / 8) + uu, r8);
+                for (int c = 0; c < 8; ++c) {
+                    if (uu == 0 && c == 0) {
+                        a = r8[0];
+                        b = r8[0];
+                    } else {
+                        if (r8[c] < a) a = r8[c];
+                        if (r8[c] > b) b = r8[c];
+                    }
+                }
+            }
+            mn[g] = a;
+            mx[g] = b;
+        }
+    }
+    // (2) Eq. 1 parameters of every group
+    GroupQ gq[NG];
+    GroupFast gf[NG];
+#pragma unroll
+    for (int g = 0; g < NG; ++g)
+        gq[g] = group_params(mn[g], mx[g], BITS);
+#pragma unroll
+    for (int g = 0; g < NG; ++g) {
+        gf[g] = group_fast(gq[g], mn[g], mx[g]);
+        meta_dst[g] = make_float2(gq[g].s, gq[g].z);
+    }
+    // (3) codes
     uint32_t words[kWords];
 #pragma unroll
     for (int w = 0; w < kWords; ++w)
         words[w] = 0u;
 #pragma unroll
-    for (int g = 0; g < CH / G; ++g) {
-        if constexpr (G <= 32) {
-            // the group's residuals stay in registers
-            float r[G];
-#pragma unroll
-            for (int uu = 0; uu < G / 8; ++uu) {
-                const int u = half * (CH / 8) + g * (G / 8) + uu;
-                const uint4 xw = *reinterpret_cast<const uint4 *>(sX + sw128_unit_offset(row, u, kFltRows));
-                const uint4 mw = *reinterpret_cast<const uint4 *>(sMu + sw128_unit_offset(best, u, Cpad));
-                const uint32_t xa[4] = {xw.x, xw.y, xw.z, xw.w}, ma[4] = {mw.x, mw.y, mw.z, mw.w};
-#pragma unroll
-                for (int k = 0; k < 4; ++k) {
-                    const float2 d = sub2(make_float2(bf16_lo(xa[k]), bf16_hi(xa[k])),
-                                          make_float2(bf16_lo(ma[k]), bf16_hi(ma[k])));
-                    r[uu * 8 + 2 * k] = d.x;
-                    r[uu * 8 + 2 * k + 1] = d.y;
-                }
-            }
-            float mn = fminf(r[0], r[1]), mx = fmaxf(r[0], r[1]);
-#pragma unroll
-            for (int c = 2; c < G; c += 2) {
-                mn = fmin3(mn, r[c], r[c + 1]);
-                mx = fmax3(mx, r[c], r[c + 1]);
-            }
-            if (mn == 0.0f || mx == 0.0f) {
-                // a zero extreme: take its sign exactly as the ordered strict scan does
-                mn = r[0];
-                mx = r[0];
-#pragma unroll
-                for (int c = 1; c < G; ++c) {
-                    if (r[c] < mn) mn = r[c];
-                    if (r[c] > mx) mx = r[c];
-                }
-            }
-            const GroupQ gq = group_params(mn, mx, BITS);
-            meta_dst[g] = make_float2(gq.s, gq.z);
-            quant_group_into<G, BITS>(r, gq, mn, mx, words, g * G);
-            continue;
-        }
-        float mn = 0.0f, mx = 0.0f;
+    for (int g = 0; g < NG; ++g) {
 #pragma unroll
         for (int uu = 0; uu < G / 8; ++uu) {
-            const int u = half * (CH / 8) + g * (G / 8) + uu;
-            const uint4 xw = *reinterpret_cast<const uint4 *>(sX + sw128_unit_offset(row, u, kFltRows));
-            const uint4 mw = *reinterpret_cast<const uint4 *>(sMu + sw128_unit_offset(best, u, Cpad));
-            const uint32_t xa[4] = {xw.x, xw.y, xw.z, xw.w}, ma[4] = {mw.x, mw.y, mw.z, mw.w};
+            float r8[8];
+            unit_residual(g * (G / 8) + uu, r8);
 #pragma unroll
             for (int k = 0; k < 8; ++k) {
-                const float r = __fsub_rn((k & 1) ? bf16_hi(xa[k >> 1]) : bf16_lo(xa[k >> 1]),
-                                          (k & 1) ? bf16_hi(ma[k >> 1]) : bf16_lo(ma[k >> 1]));
-                if (uu == 0 && k == 0) {
-                    mn = r;
-                    mx = r;
-                } else {
-                    if (r < mn) mn = r;
-                    if (r > mx) mx = r;
-                }
-            }
-        }
-        const GroupQ gq = group_params(mn, mx, BITS);
-        meta_dst[g] = make_float2(gq.s, gq.z);
-        const GroupFast gf = group_fast(gq, mn, mx);
-#pragma unroll
-        for (int uu = 0; uu < G / 8; ++uu) {
-            const int u = half * (CH / 8) + g * (G / 8) + uu;
-            const uint4 xw = *reinterpret_cast<const uint4 *>(sX + sw128_unit_offset(row, u, kFltRows));
-            const uint4 mw = *reinterpret_cast<const uint4 *>(sMu + sw128_unit_offset(best, u, Cpad));
-            const uint32_t xa[4] = {xw.x, xw.y, xw.z, xw.w}, ma[4] = {mw.x, mw.y, mw.z, mw.w};
-#pragma unroll
-            for (int k = 0; k < 8; ++k) {
-                const float r = __fsub_rn((k & 1) ? bf16_hi(xa[k >> 1]) : bf16_lo(xa[k >> 1]),
-                                          (k & 1) ? bf16_hi(ma[k >> 1]) : bf16_lo(ma[k >> 1]));
                 const int c = g * G + uu * 8 + k;
-                words[c / kPerWord] += (gf.fast ? quant_code_fast<BITS>(r, gf) : quant_code(r, gq, BITS))
+                words[c / kPerWord] += (gf[g].fast ? quant_code_fast<BITS>(r8[k], gf[g]) : quant_code(r8[k], gq[g], BITS))
                                        << ((c % kPerWord) * BITS);
             }
         }
@@ -212,295 +247,474 @@ __device__ __forceinline__ void encode_residual_smem(const uint8_t *sX, const ui
     }
 }
 
+// Bounded mbarrier wait that also gives up at once when another role of the
+// CTA has given up (abort flag in shared memory); on its own expiry it raises
+// the device status and sets the flag.
+__device__ __forceinline__ bool flt_wait(uint32_t bar, uint32_t parity, volatile int *abort)
+{
+    for (uint32_t i = 0; i < kSpinLimit; ++i) {
+        if (mbar_try_wait(bar, parity))
+            return true;
+        if ((i & 255u) == 255u && *abort)
+            return false;
+    }
+    raise_status(DEVSTAT_TIMEOUT);
+    *abort = 1;
+    return false;
+}
+
+// Specified binary32 distances of row `row` of the X tile to the centres
+// j = j0 + 64 m (m = 0, 1, ...) below C, two chains at a time; returns the
+// smallest (distance, index), lowest index on ties.
+template <int D>
+__device__ __forceinline__ void flt_bruteforce_part(const uint8_t *sX, const uint8_t *sMu, int Cpad, int C, int row,
+                                                    int j0, float &bd, int &bj)
+{
+    bd = INFINITY;
+    bj = -1;
+    for (int j = j0; j < C; j += 128) {
+        const int j2 = j + 64;
+        const float da = spec_distance_smem<D>(sX, sMu, Cpad, row, j);
+        const float db = j2 < C ? spec_distance_smem<D>(sX, sMu, Cpad, row, j2) : INFINITY;
+        if (bj < 0 || da < bd) {
+            bd = da;
+            bj = j;
+        }
+        if (j2 < C && db < bd) {
+            bd = db;
+            bj = j2;
+        }
+    }
+}
+
+// Named barrier 1 + 4 g + q over the 64 threads of one row group (warps w and
+// w + 4 of epilogue group g).
+__device__ __forceinline__ void flt_pair_sync(int g, int q)
+{
+    switch ((g << 2) | (q & 3)) {
+    case 0: named_barrier_sync<1>(64); break;
+    case 1: named_barrier_sync<2>(64); break;
+    case 2: named_barrier_sync<3>(64); break;
+    case 3: named_barrier_sync<4>(64); break;
+    case 4: named_barrier_sync<5>(64); break;
+    case 5: named_barrier_sync<6>(64); break;
+    case 6: named_barrier_sync<7>(64); break;
+    default: named_barrier_sync<8>(64); break;
+    }
+}
+
+// L'_j of 32 columns (L_j + k |x|^2, the same shift for every j of the row),
+// with the chunk-local index in the low 5 mantissa bits, merged into the three
+// smallest of two independent chains.
+__device__ __forceinline__ void flt_scan_chunk(const float *p, const float *sA, const float *sM, float nB, float &a1,
+                                               float &a2, float &a3, float &e1, float &e2, float &e3)
+{
+    auto pair_into = [](float pa, float pb, float &m1, float &m2, float &m3) {
+        // sort the pair, then merge it into the three smallest (k-th smallest
+        // of two sorted lists = min over i + j = k of max(a_i, b_j))
+        const float lo = fminf(pa, pb), hi = fmaxf(pa, pb);
+        const float n3 = fmin3(m3, fmaxf(m2, lo), fmaxf(m1, hi));
+        const float n2 = fmin3(fmaxf(m1, lo), m2, hi);
+        m1 = fminf(m1, lo);
+        m2 = n2;
+        m3 = n3;
+    };
+    const float4 *A4 = reinterpret_cast<const float4 *>(sA);
+    const float4 *M4 = reinterpret_cast<const float4 *>(sM);
+#pragma unroll
+    for (int i4 = 0; i4 < 8; ++i4) {
+        const float4 av = A4[i4], mv = M4[i4];
+        // L' = (A_j - 2 p_j) - 2 k |x| |mu_j|, pairs of columns at a time
+        const float2 t01 = fma2(make_float2(-2.0f, -2.0f), make_float2(p[4 * i4], p[4 * i4 + 1]),
+                                make_float2(av.x, av.y));
+        const float2 t23 = fma2(make_float2(-2.0f, -2.0f), make_float2(p[4 * i4 + 2], p[4 * i4 + 3]),
+                                make_float2(av.z, av.w));
+        const float2 l01 = fma2(make_float2(nB, nB), make_float2(mv.x, mv.y), t01);
+        const float2 l23 = fma2(make_float2(nB, nB), make_float2(mv.z, mv.w), t23);
+        const uint32_t i = (uint32_t)(i4 * 4);
+        const float pk0 = __uint_as_float((__float_as_uint(l01.x) & ~31u) | i);
+        const float pk1 = __uint_as_float((__float_as_uint(l01.y) & ~31u) | (i + 1));
+        const float pk2 = __uint_as_float((__float_as_uint(l23.x) & ~31u) | (i + 2));
+        const float pk3 = __uint_as_float((__float_as_uint(l23.y) & ~31u) | (i + 3));
+        pair_into(pk0, pk1, a1, a2, a3);
+        pair_into(pk2, pk3, e1, e2, e3);
+    }
+}
+
+// tcgen05.ld of 32 columns without the wait (the caller waits once for all
+// loads in flight with tmem_ld_wait).
+__device__ __forceinline__ void tmem_ld32_nowait(uint32_t taddr, uint32_t *r)
+{
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]),
+          "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]),
+          "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]),
+          "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+        : "r"(taddr));
+}
+
+__device__ __forceinline__ void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+
 template <int D, int BITS, int G>
-__global__ void __launch_bounds__(kFltThreads, 2)
+__global__ void __launch_bounds__(kFltThreads, 1)
     encode_filter_kernel(const __grid_constant__ CUtensorMap tmap_x, FilterArgs a)
 {
     static_assert(G <= D / 2, "a group must lie inside one half of the channels");
-    constexpr int CH = D / 2;             // channels per thread
-    constexpr int kMaxChunks = kFltMaxC / 32 / 2;
+    constexpr int CH = D / 2;             // channels per epilogue thread
+    constexpr int kSubChunks = kFltAccCols / 32;
 
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    const int Cpad = a.Cpad;
-    uint8_t *sX = smem;
-    uint8_t *sMu = smem + D * 2 * kFltRows;
-    float *sNrm = reinterpret_cast<float *>(sMu + Cpad * D * 2);
-    float4 *sPair = reinterpret_cast<float4 *>(sNrm + Cpad);               // [2][128] {|x|^2 part, top 3}
-    int *sPairC = reinterpret_cast<int *>(sPair + 2 * 128);                  // [2][128] top-3 chunk ids
-    float4 *sWin = reinterpret_cast<float4 *>(sPairC + 2 * 128);             // [128] exact winners / distances
-    uint64_t *bars = reinterpret_cast<uint64_t *>(reinterpret_cast<uint8_t *>(sPair) + kFltPairBytes);
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 2);
-    uint32_t *sMaxNrm = tmem_slot + 1;
+    const int Cpad = a.Cpad, S = a.stages;
+    const uint32_t tile_bytes = flt_tile_bytes(D);
+    uint8_t *sXring = smem;
+    uint8_t *sMu = smem + S * tile_bytes;
+    float *sA = reinterpret_cast<float *>(sMu + Cpad * D * 2);  // A_j = N_j - k |mu_j|^2 (inf past C)
+    float *sM = sA + Cpad;                                      // |mu_j| (0 past C)
+    uint8_t *sPairBase = reinterpret_cast<uint8_t *>(sM + Cpad);
+    uint64_t *bars = reinterpret_cast<uint64_t *>(sPairBase + 2 * kFltPairBytes);
+    // bars: xfull[4] xempty[4] afull[2] aempty[2] drain
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 13);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 2);
+    auto xfull = [&](int st) { return smem_u32(bars + st); };
+    auto xempty = [&](int st) { return smem_u32(bars + kFltMaxStages + st); };
+    auto afull = [&](int g) { return smem_u32(bars + 2 * kFltMaxStages + g); };
+    auto aempty = [&](int g) { return smem_u32(bars + 2 * kFltMaxStages + 2 + g); };
+    const uint32_t bar_drain = smem_u32(bars + 2 * kFltMaxStages + 4);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int half = warp >> 2;
-    const int row = (warp & 3) * 32 + lane;
-    const int h = blockIdx.y;
-    const uint32_t bar_x = smem_u32(bars), bar_m = smem_u32(bars + 1);
 
     if (warp == 0)
-        tmem_alloc(smem_u32(tmem_slot), a.tmem_cols);
+        tmem_alloc(smem_u32(tmem_slot), 2 * kFltAccCols);
     if (tid == 0) {
-        mbar_init(bar_x, 1);
-        mbar_init(bar_m, 1);
-        fence_mbar_init();
-        *sMaxNrm = 0u;
-    }
-    __syncthreads();
-
-    // centres of head h -> swizzled K-major tile [D/64][Cpad][128 B]; norms
-    const uint16_t *cent_h = a.cent + (int64_t)h * a.C * D;
-    for (int e = tid; e < Cpad * (D / 8); e += kFltThreads) {
-        const int j = e / (D / 8), u = e % (D / 8);
-        const uint4 w = j < a.C ? __ldg(reinterpret_cast<const uint4 *>(cent_h + (int64_t)j * D) + u)
-                                : make_uint4(0, 0, 0, 0);
-        *reinterpret_cast<uint4 *>(sMu + sw128_unit_offset(j, u, Cpad)) = w;
-    }
-    for (int j = tid; j < Cpad; j += kFltThreads) {
-        float nrm = INFINITY;
-        if (j < a.C) {
-            nrm = 0.0f;
-            for (int u = 0; u < D / 8; ++u) {
-                float m8[8];
-                load_bf16x8(cent_h + (int64_t)j * D + u * 8, m8);
-#pragma unroll
-                for (int k = 0; k < 8; ++k)
-                    nrm = fmaf(m8[k], m8[k], nrm);
-            }
-            atomicMax(sMaxNrm, __float_as_uint(nrm));
+        for (int st = 0; st < kFltMaxStages; ++st) {
+            mbar_init(xfull(st), 1);
+            mbar_init(xempty(st), kFltGroupThreads / 32);
         }
-        sNrm[j] = nrm;
+        for (int g = 0; g < 2; ++g) {
+            mbar_init(afull(g), 1);
+            mbar_init(aempty(g), kFltGroupThreads / 32);
+        }
+        mbar_init(bar_drain, 1);
+        *abort_flag = 0;
+        fence_mbar_init();
     }
-    fence_proxy_async_smem();
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
-    const float Mnorm = sqrtf(__uint_as_float(*sMaxNrm));
-    const uint32_t lane_off = ((uint32_t)(warp & 3) * 32u) << 16;
-    const uint32_t aX = smem_u32(sX), aMu = smem_u32(sMu);
+    const uint32_t aMu = smem_u32(sMu);
 
-    // this thread's 32-column chunks of the TMEM row
-    const int nchunks = Cpad / 32;
-    const int c_lo = half == 0 ? 0 : (nchunks + 1) / 2;
-    const int c_hi = half == 0 ? (nchunks + 1) / 2 : nchunks;
+    const int nsub = (Cpad + kFltAccCols - 1) / kFltAccCols;
+    const int64_t units = (int64_t)a.H * a.ntiles;
+    const int64_t u_begin = (int64_t)blockIdx.x * units / gridDim.x;
+    const int64_t u_end = (int64_t)(blockIdx.x + 1) * units / gridDim.x;
 
-    const int64_t ntiles = (a.T + kFltRows - 1) / kFltRows;
-    uint32_t ph_x = 0, ph_m = 0;
-    bool ok = true;
-    for (int64_t tile = blockIdx.x; tile < ntiles; tile += gridDim.x) {
-        const int64_t t0 = tile * kFltRows;
-        if (tid == 0) {
-            mbar_arrive_expect_tx(bar_x, D * 2 * kFltRows);
-#pragma unroll
-            for (int ch = 0; ch < D / 64; ++ch)
-                tma_load_3d(aX + ch * (kFltRows * 128), &tmap_x, bar_x, ch * 64, h, (int)t0);
+    // epilogue thread geometry: group, row (TMEM lane) and half of columns /
+    // channels
+    const int grp = warp >> 3, w8 = warp & 7;
+    const int half = w8 >> 2;
+    const int row = (w8 & 3) * 32 + lane;
+    const uint32_t lane_off = ((uint32_t)(w8 & 3) * 32u) << 16;
+    float4 *sPair2 = reinterpret_cast<float4 *>(sPairBase + grp * kFltPairBytes);  // [2][2][128]
+    int *sPairC2 = reinterpret_cast<int *>(sPair2 + 2 * 2 * 128);                   // [2][2][128]
+    float4 *sWin = reinterpret_cast<float4 *>(sPairC2 + 2 * 2 * 128);               // [128]
+
+    int64_t tile_seq = 0;  // tiles this CTA has handled (X ring position, group = parity)
+    uint32_t mma_issued = 0;
+    for (int64_t u = u_begin; u < u_end;) {
+        const int h = (int)(u / a.ntiles);
+        const int64_t seg_end = min(u_end, (int64_t)(h + 1) * a.ntiles);
+        const int64_t tile0 = u - (int64_t)h * a.ntiles;
+        const int n = (int)(seg_end - u);
+
+        // ---- centres of head h -> swizzled K-major tile [D/64][Cpad][128 B];
+        // A_j and |mu_j|
+        __syncthreads();  // the previous segment is fully consumed
+        const uint16_t *cent_h = a.cent + (int64_t)h * a.C * D;
+        for (int e = tid; e < Cpad * (D / 8); e += kFltThreads) {
+            const int j = e / (D / 8), uu = e % (D / 8);
+            const uint4 w = j < a.C ? __ldg(reinterpret_cast<const uint4 *>(cent_h + (int64_t)j * D) + uu)
+                                    : make_uint4(0, 0, 0, 0);
+            *reinterpret_cast<uint4 *>(sMu + sw128_unit_offset(j, uu, Cpad)) = w;
         }
-        ok = mbar_wait(bar_x, ph_x) && ok;
-        ph_x ^= 1u;
-        if (tid == 0) {
-            tc_fence_after();
-            for (int n0 = 0; n0 < Cpad; n0 += 256) {
-                const int N = min(256, Cpad - n0);
-                const uint32_t idesc = idesc_f32acc(128, N, true, false, false);
+        for (int j = tid; j < Cpad; j += kFltThreads) {
+            float A = INFINITY, m = 0.0f;
+            if (j < a.C) {
+                float nrm = 0.0f;
+                for (int uu = 0; uu < D / 8; ++uu) {
+                    float m8[8];
+                    load_bf16x8(cent_h + (int64_t)j * D + uu * 8, m8);
 #pragma unroll
-                for (int ks = 0; ks < D / 16; ++ks) {
-                    const uint32_t aoff = (uint32_t)(ks >> 2) * (kFltRows * 128u) + (uint32_t)(ks & 3) * 32u;
-                    const uint32_t boff =
-                        (uint32_t)(ks >> 2) * (uint32_t)(Cpad * 128) + (uint32_t)n0 * 128u + (uint32_t)(ks & 3) * 32u;
-                    umma_ss(tmem + (uint32_t)n0, sdesc_sw128(aX + aoff, 16, 1024), sdesc_sw128(aMu + boff, 16, 1024),
-                            idesc, ks > 0 ? 1u : 0u);
+                    for (int k = 0; k < 8; ++k)
+                        nrm = fmaf(m8[k], m8[k], nrm);
                 }
+                m = sqrtf(nrm);
+                A = fmaf(-a.kappa, nrm, nrm);
             }
-            umma_commit(bar_m);
+            sA[j] = A;
+            sM[j] = m;
         }
-        ok = mbar_wait(bar_m, ph_m) && ok;
-        ph_m ^= 1u;
+        fence_proxy_async_smem();
+        tc_fence_before();
+        __syncthreads();
         tc_fence_after();
 
-        // (1) |x|^2 over this thread's channel half
-        float xx = 0.0f;
+        if (warp == kFltTmaWarp) {
+            // ------------------------------------------------------------ TMA
+            if (lane == 0) {
+                for (int k = 0; k < n && !*abort_flag; ++k) {
+                    const int64_t seq = tile_seq + k;
+                    const int st = (int)(seq % S);
+                    if (seq >= S && !flt_wait(xempty(st), (uint32_t)(((seq / S) - 1) & 1), abort_flag))
+                        break;
+                    const uint32_t dst = smem_u32(sXring + st * tile_bytes);
+                    mbar_arrive_expect_tx(xfull(st), tile_bytes);
+                    const int t0 = (int)((tile0 + k) * kFltRows);
 #pragma unroll
-        for (int u = half * (CH / 8); u < (half + 1) * (CH / 8); ++u) {
-            const uint4 w = *reinterpret_cast<const uint4 *>(sX + sw128_unit_offset(row, u, kFltRows));
-            const uint32_t wa[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-            for (int k = 0; k < 4; ++k) {
-                xx = fmaf(bf16_lo(wa[k]), bf16_lo(wa[k]), xx);
-                xx = fmaf(bf16_hi(wa[k]), bf16_hi(wa[k]), xx);
-            }
-        }
-        // (2) v_j = |mu_j|^2 - 2 p_j over this thread's chunks.  The chunk-local
-        // column index rides in the low 5 mantissa bits of v, so one pass keeps
-        // the three smallest values (the window below absorbs the <= 31 ulp
-        // this perturbs v); chunk ids are kept beside them.
-        float b1 = INFINITY, b2 = INFINITY, b3 = INFINITY;
-        int k1 = 0, k2 = 0, k3 = 0;
-#pragma unroll
-        for (int k = 0; k < kMaxChunks; ++k) {
-            const int c = c_lo + k;
-            if (c < c_hi) {
-                float p[32];
-                tmem_ld32(tmem + lane_off + (uint32_t)(c * 32), p);
-                // two independent chains (pairs 4q and 4q + 2 / 4q + 1 and 4q + 3
-                // of the chunk) so consecutive updates do not wait on each other
-                float a1 = INFINITY, a2 = INFINITY, a3 = INFINITY;
-                float c1 = INFINITY, c2 = INFINITY, c3 = INFINITY;
-                const float4 *nrm4 = reinterpret_cast<const float4 *>(sNrm + c * 32);
-                auto pair_into = [](float pa, float pb, float &m1, float &m2, float &m3) {
-                    // sort the pair, then merge it into the three smallest
-                    // (k-th smallest of two sorted lists = min over i + j = k
-                    // of max(a_i, b_j))
-                    const float lo = fminf(pa, pb), hi = fmaxf(pa, pb);
-                    const float n3 = fmin3(m3, fmaxf(m2, lo), fmaxf(m1, hi));
-                    const float n2 = fmin3(fmaxf(m1, lo), m2, hi);
-                    m1 = fminf(m1, lo);
-                    m2 = n2;
-                    m3 = n3;
-                };
-#pragma unroll
-                for (int i4 = 0; i4 < 8; ++i4) {
-                    const float4 n4 = nrm4[i4];
-                    const float nn[4] = {n4.x, n4.y, n4.z, n4.w};
-                    float pk[4];
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const int i = i4 * 4 + e;
-                        const float v = fmaf(-2.0f, p[i], nn[e]);
-                        pk[e] = __uint_as_float((__float_as_uint(v) & ~31u) | (uint32_t)i);
-                    }
-                    pair_into(pk[0], pk[1], a1, a2, a3);
-                    pair_into(pk[2], pk[3], c1, c2, c3);
-                }
-                // merge the two chains' three smallest
-                const float m1 = fminf(a1, c1);
-                const float m2 = fmin3(a2, fmaxf(a1, c1), c2);
-                const float m3 = fminf(fmin3(a3, fmaxf(a2, c1), fmaxf(a1, c2)), c3);
-                top3_insert(m1, c, b1, k1, b2, k2, b3, k3);
-                top3_insert(m2, c, b1, k1, b2, k2, b3, k3);
-                top3_insert(m3, c, b1, k1, b2, k2, b3, k3);
-            }
-        }
-        // (3) exchange with the partner thread of this row (warps w and w+4);
-        // both threads then hold the row's three smallest values, half-0
-        // entries first on equal values
-        sPair[half * 128 + row] = make_float4(xx, b1, b2, b3);
-        sPairC[half * 128 + row] = k1 | (k2 << 8) | (k3 << 16);
-        named_barrier_sync_q(warp & 3, 64);
-        const float4 other = sPair[(half ^ 1) * 128 + row];
-        const int oc = sPairC[(half ^ 1) * 128 + row];
-        float g1, g2, g3;
-        int h1, h2, h3;
-        {
-            // list of half 0, then insert half 1's entries
-            const bool h0 = half == 0;
-            g1 = h0 ? b1 : other.y;
-            g2 = h0 ? b2 : other.z;
-            g3 = h0 ? b3 : other.w;
-            const int cc = h0 ? (k1 | (k2 << 8) | (k3 << 16)) : oc;
-            h1 = cc & 0xff;
-            h2 = (cc >> 8) & 0xff;
-            h3 = (cc >> 16) & 0xff;
-            const int dc = h0 ? oc : (k1 | (k2 << 8) | (k3 << 16));
-            top3_insert(h0 ? other.y : b1, dc & 0xff, g1, h1, g2, h2, g3, h3);
-            top3_insert(h0 ? other.z : b2, (dc >> 8) & 0xff, g1, h1, g2, h2, g3, h3);
-            top3_insert(h0 ? other.w : b3, (dc >> 16) & 0xff, g1, h1, g2, h2, g3, h3);
-        }
-        const float xn = sqrtf(xx + other.x);
-        const float thr = g1 + a.kappa * (xn + Mnorm) * (xn + Mnorm);
-        int best = h1 * 32 + (int)(__float_as_uint(g1) & 31u);
-        const bool finite = thr < INFINITY;
-        const bool pair_case = finite && !(g2 > thr) && g3 > thr;    // two candidates
-        const bool wide_case = !finite || (!(g2 > thr) && !(g3 > thr));  // three or more
-        // two candidates: each thread of the pair scores one with the specified
-        // distance; the smaller wins, the lower index on a tie
-        if (__any_sync(0xffffffffu, pair_case)) {
-            const int j1 = best, j2 = h2 * 32 + (int)(__float_as_uint(g2) & 31u);
-            float dmine = 0.0f;
-            if (pair_case)
-                dmine = spec_distance_smem<D>(sX, sMu, Cpad, row, half == 0 ? j1 : j2);
-            if (pair_case) {
-                if (half == 0)
-                    sWin[row].x = dmine;
-            }
-            named_barrier_sync_q(warp & 3, 64);
-            if (pair_case) {
-                const float d1 = half == 0 ? dmine : sWin[row].x;
-                const float d2 = half == 0 ? 0.0f : dmine;
-                if (half == 1) {
-                    const int lo = j1 < j2 ? j1 : j2;
-                    const int hi = j1 < j2 ? j2 : j1;
-                    const float dlo = j1 < j2 ? d1 : d2, dhi = j1 < j2 ? d2 : d1;
-                    sWin[row].y = __int_as_float(dhi < dlo ? hi : lo);
+                    for (int ch = 0; ch < D / 64; ++ch)
+                        tma_load_3d(dst + ch * (kFltRows * 128), &tmap_x, xfull(st), ch * 64, h, t0);
                 }
             }
-            named_barrier_sync_q(warp & 3, 64);
-            if (pair_case)
-                best = __float_as_int(sWin[row].y);
-        }
-        // three or more candidates (rare): re-score the window (or every centre
-        // when the window is not finite) with the specified distance.  Each
-        // thread of the pair scans its own half of the columns in increasing
-        // index order; the lower half wins ties.  Both warps of the pair see
-        // the same flags, so they take the branch together.
-        if (__any_sync(0xffffffffu, wide_case)) {
-            float bd = INFINITY;
-            int bj = -1;
-            for (int c = c_lo; c < c_hi; ++c) {
-                float p[32];
-                tmem_ld32(tmem + lane_off + (uint32_t)(c * 32), p);
-                uint32_t cand = 0u;
+        } else if (warp == kFltMmaWarp) {
+            // ------------------------------------------------------------ MMA
+            // issue order: for each pair of consecutive tiles (one per group),
+            // sub-unit 0 of both, then sub-unit 1 of both, ... so neither
+            // group's accumulator release holds up the other's MMAs
+            if (lane == 0) {
+                bool ok = true;
+                for (int kb = 0; ok && kb < n; kb += 2) {
+                    for (int sub = 0; ok && sub < nsub; ++sub) {
+                        for (int kk = kb; ok && kk < kb + 2 && kk < n; ++kk) {
+                            const int64_t seq = tile_seq + kk;
+                            const int st = (int)(seq % S);
+                            const int g = (int)(seq & 1);
+                            if (sub == 0 && !(ok = flt_wait(xfull(st), (uint32_t)((seq / S) & 1), abort_flag)))
+                                break;
+                            const int64_t gsub = (seq >> 1) * nsub + sub;  // group g's sub-unit count
+                            if (gsub >= 1 && !(ok = flt_wait(aempty(g), (uint32_t)((gsub - 1) & 1), abort_flag)))
+                                break;
+                            tc_fence_after();
+                            const uint32_t aX = smem_u32(sXring + st * tile_bytes);
+                            const int n0 = sub * kFltAccCols;
+                            const int N = min(kFltAccCols, Cpad - n0);
+                            const uint32_t idesc = idesc_f32acc(128, N, true, false, false);
 #pragma unroll
-                for (int i = 0; i < 32; ++i) {
-                    const int j = c * 32 + i;
-                    const float v = fmaf(-2.0f, p[i], sNrm[j]);
-                    if (wide_case && j < a.C && (!finite || v <= thr))
-                        cand |= 1u << i;
-                }
-                while (cand) {  // increasing index order
-                    const int i = __ffs(cand) - 1;
-                    cand &= cand - 1u;
-                    const int j = c * 32 + i;
-                    const float dj = spec_distance_smem<D>(sX, sMu, Cpad, row, j);
-                    if (bj < 0 || dj < bd) {
-                        bd = dj;
-                        bj = j;
+                            for (int ks = 0; ks < D / 16; ++ks) {
+                                const uint32_t aoff =
+                                    (uint32_t)(ks >> 2) * (kFltRows * 128u) + (uint32_t)(ks & 3) * 32u;
+                                const uint32_t boff = (uint32_t)(ks >> 2) * (uint32_t)(Cpad * 128) +
+                                                      (uint32_t)n0 * 128u + (uint32_t)(ks & 3) * 32u;
+                                umma_ss(tmem + (uint32_t)(g * kFltAccCols), sdesc_sw128(aX + aoff, 16, 1024),
+                                        sdesc_sw128(aMu + boff, 16, 1024), idesc, ks > 0 ? 1u : 0u);
+                            }
+                            umma_commit(afull(g));
+                            ++mma_issued;
+                        }
                     }
                 }
             }
-            reinterpret_cast<float2 *>(sWin + row)[half] = make_float2(bd, __int_as_float(bj));
-            named_barrier_sync_q(warp & 3, 64);
-            if (wide_case) {
-                const float4 w = sWin[row];
-                const int j0 = __float_as_int(w.y), j1 = __float_as_int(w.w);
-                best = (j0 < 0 || (j1 >= 0 && w.z < w.x)) ? j1 : j0;
-            }
-        }
-        if (best < 0 || best >= a.C)
-            best = 0;  // unreachable for finite inputs
+        } else {
+            // ------------------------------------------------------------ epilogue group grp
+            bool ok = true;
+            for (int k = 0; k < n; ++k) {
+                const int64_t seq = tile_seq + k;
+                if ((int)(seq & 1) != grp)
+                    continue;
+                const int st = (int)(seq % S);
+                const uint8_t *sX = sXring + st * tile_bytes;
+                float4 *sPair = sPair2 + ((seq >> 1) & 1) * 256;
+                int *sPairC = sPairC2 + ((seq >> 1) & 1) * 256;
+                ok = ok && __all_sync(0xffffffffu, flt_wait(xfull(st), (uint32_t)((seq / S) & 1), abort_flag));
+                // (1) |x|^2 over this thread's channel half
+                float xx = 0.0f;
+                if (ok) {
+#pragma unroll
+                    for (int uu = half * (CH / 8); uu < (half + 1) * (CH / 8); ++uu) {
+                        const uint4 w = *reinterpret_cast<const uint4 *>(sX + sw128_unit_offset(row, uu, kFltRows));
+                        const uint32_t wa[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+                        for (int q = 0; q < 4; ++q) {
+                            xx = fmaf(bf16_lo(wa[q]), bf16_lo(wa[q]), xx);
+                            xx = fmaf(bf16_hi(wa[q]), bf16_hi(wa[q]), xx);
+                        }
+                    }
+                }
+                // both threads of the row need |x|: exchange the halves
+                sPair[half * 128 + row].x = xx;
+                flt_pair_sync(grp, w8 & 3);
+                const float xn = sqrtf(xx + sPair[(half ^ 1) * 128 + row].x);
+                const float nB = -2.0f * a.kappa * xn;
+                // (2) L'_j over this thread's chunks of every sub-unit; the
+                // chunk-local column index rides in the low 5 mantissa bits,
+                // so one pass keeps the three smallest values (the margin in k
+                // absorbs the <= 31 ulp this perturbs them); global chunk ids
+                // are kept beside them
+                float b1 = INFINITY, b2 = INFINITY, b3 = INFINITY;
+                int k1 = 0, k2 = 0, k3 = 0;
+                for (int sub = 0; sub < nsub; ++sub) {
+                    const int64_t gsub = (seq >> 1) * nsub + sub;
+                    ok = ok && __all_sync(0xffffffffu, flt_wait(afull(grp), (uint32_t)(gsub & 1), abort_flag));
+                    if (!ok)
+                        break;
+                    tc_fence_after();
+                    const int n0 = sub * kFltAccCols;
+                    const int nch = min(kSubChunks, (Cpad - n0) / 32);
+                    const int c_lo = half == 0 ? 0 : (nch + 1) / 2;
+                    const int c_hi = half == 0 ? (nch + 1) / 2 : nch;
+                    const uint32_t tbase = tmem + lane_off + (uint32_t)(grp * kFltAccCols);
+#pragma unroll
+                    for (int kk = 0; kk < kSubChunks / 2; ++kk) {
+                        const int c = c_lo + kk;
+                        if (c < c_hi) {
+                            uint32_t pw[32];
+                            tmem_ld32_nowait(tbase + (uint32_t)(c * 32), pw);
+                            tmem_ld_wait();
+                            float a1 = INFINITY, a2 = INFINITY, a3 = INFINITY;
+                            float e1 = INFINITY, e2 = INFINITY, e3 = INFINITY;
+                            flt_scan_chunk(reinterpret_cast<const float *>(pw), sA + n0 + c * 32, sM + n0 + c * 32, nB,
+                                           a1, a2, a3, e1, e2, e3);
+                            const int gc = sub * kSubChunks + c;
+                            top3_insert(fminf(a1, e1), gc, b1, k1, b2, k2, b3, k3);
+                            top3_insert(fmin3(a2, fmaxf(a1, e1), e2), gc, b1, k1, b2, k2, b3, k3);
+                            top3_insert(fminf(fmin3(a3, fmaxf(a2, e1), fmaxf(a1, e2)), e3), gc, b1, k1, b2, k2, b3, k3);
+                        }
+                    }
+                    // accumulator read: the MMA may overwrite it
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0)
+                        mbar_arrive(aempty(grp));
+                }
+                // (3) exchange with the partner thread of this row (warps w and
+                // w+4 of the group); both then hold the row's three smallest
+                // values, half-0 entries first on equal values.  Both warps
+                // always meet here and carry their status (bit 31) along, so
+                // every later named barrier is taken by both or by neither.
+                sPair[half * 128 + row] = make_float4(xx, b1, b2, b3);
+                sPairC[half * 128 + row] = (k1 | (k2 << 8) | (k3 << 16)) | (ok ? 0 : (int)0x80000000u);
+                flt_pair_sync(grp, w8 & 3);
+                const int oc_raw = sPairC[(half ^ 1) * 128 + row];
+                ok = ok && oc_raw >= 0;
+                if (ok) {
+                    const float4 other = sPair[(half ^ 1) * 128 + row];
+                    const int oc = oc_raw;
+                    float g1, g2, g3;
+                    int h1, h2, h3;
+                    {
+                        const bool h0 = half == 0;
+                        g1 = h0 ? b1 : other.y;
+                        g2 = h0 ? b2 : other.z;
+                        g3 = h0 ? b3 : other.w;
+                        const int cc = h0 ? (k1 | (k2 << 8) | (k3 << 16)) : oc;
+                        h1 = cc & 0xff;
+                        h2 = (cc >> 8) & 0xff;
+                        h3 = (cc >> 16) & 0xff;
+                        const int dc = h0 ? oc : (k1 | (k2 << 8) | (k3 << 16));
+                        top3_insert(h0 ? other.y : b1, dc & 0xff, g1, h1, g2, h2, g3, h3);
+                        top3_insert(h0 ? other.z : b2, (dc >> 8) & 0xff, g1, h1, g2, h2, g3, h3);
+                        top3_insert(h0 ? other.w : b3, (dc >> 16) & 0xff, g1, h1, g2, h2, g3, h3);
+                    }
+                    int best = h1 * 32 + (int)(__float_as_uint(g1) & 31u);
+                    // threshold: U'(best) = L'(best) + 2 k (|x| + |mu_best|)^2
+                    const float r1 = xn + sM[min(best, Cpad - 1)];
+                    const float thr = g1 + 2.0f * a.kappa * r1 * r1;
+                    const bool finite = thr < INFINITY;
+                    const bool pair_case = finite && !(g2 > thr) && g3 > thr;        // two candidates
+                    const bool wide_case = !finite || (!(g2 > thr) && !(g3 > thr));  // three or more
+                    // two candidates: each thread of the pair scores one with the
+                    // specified distance; the smaller wins, the lower index on a tie
+                    if (__any_sync(0xffffffffu, pair_case)) {
+                        const int j1 = best, j2 = h2 * 32 + (int)(__float_as_uint(g2) & 31u);
+                        float dmine = 0.0f;
+                        if (pair_case) {
+                            dmine = spec_distance_smem<D>(sX, sMu, Cpad, row, half == 0 ? j1 : j2);
+                            if (half == 0)
+                                sWin[row].x = dmine;
+                        }
+                        flt_pair_sync(grp, w8 & 3);
+                        if (pair_case && half == 1) {
+                            const float d1 = sWin[row].x, d2 = dmine;
+                            const int lo = j1 < j2 ? j1 : j2;
+                            const int hi = j1 < j2 ? j2 : j1;
+                            const float dlo = j1 < j2 ? d1 : d2, dhi = j1 < j2 ? d2 : d1;
+                            sWin[row].y = __int_as_float(dhi < dlo ? hi : lo);
+                        }
+                        flt_pair_sync(grp, w8 & 3);
+                        if (pair_case)
+                            best = __float_as_int(sWin[row].y);
+                    }
+                    // three or more candidates (rare): the two warps of this row
+                    // group score every centre of the head for each such row,
+                    // lane-parallel over the centres, and take the smallest
+                    // (distance, index).  Both warps see the same flags.
+                    uint32_t wide = __ballot_sync(0xffffffffu, wide_case);
+                    while (wide) {
+                        const int wl = __ffs(wide) - 1;
+                        wide &= wide - 1u;
+                        const int wrow = (w8 & 3) * 32 + wl;
+                        float bd;
+                        int bj;
+                        flt_bruteforce_part<D>(sX, sMu, Cpad, a.C, wrow, half * 32 + lane, bd, bj);
+#pragma unroll
+                        for (int off = 16; off > 0; off >>= 1) {
+                            const float od = __shfl_xor_sync(0xffffffffu, bd, off);
+                            const int oj = __shfl_xor_sync(0xffffffffu, bj, off);
+                            if (oj >= 0 && (bj < 0 || od < bd || (od == bd && oj < bj))) {
+                                bd = od;
+                                bj = oj;
+                            }
+                        }
+                        if (lane == 0)
+                            reinterpret_cast<float2 *>(sWin + wrow)[half] = make_float2(bd, __int_as_float(bj));
+                        flt_pair_sync(grp, w8 & 3);
+                        if (lane == wl) {
+                            const float4 wv = sWin[wrow];
+                            const int j0 = __float_as_int(wv.y), jj1 = __float_as_int(wv.w);
+                            best = (j0 < 0 || (jj1 >= 0 && (wv.z < wv.x || (wv.z == wv.x && jj1 < j0)))) ? jj1 : j0;
+                        }
+                        flt_pair_sync(grp, w8 & 3);
+                    }
+                    if (best < 0 || best >= a.C)
+                        best = 0;  // unreachable for finite inputs
 
-        // (4) residual + Eq. 1 + packing for this thread's channel half
-        const int64_t t = t0 + row;
-        if (t < a.T) {
-            const int64_t th = (int64_t)h * a.T + t;
-            if (half == 0)
-                a.idx[th] = (uint16_t)best;
-            if (!a.assign_only)
-                encode_residual_smem<CH, BITS, G>(sX, sMu, Cpad, row, best, half,
-                                                  a.codes + th * (D * BITS / 8) + half * (CH * BITS / 8),
-                                                  reinterpret_cast<float2 *>(a.meta) + th * (D / G) + half * (CH / G));
+                    // (4) residual + Eq. 1 + packing for this thread's channel half
+                    const int64_t t = (tile0 + k) * kFltRows + row;
+                    if (t < a.T) {
+                        const int64_t th = (int64_t)h * a.T + t;
+                        if (half == 0)
+                            a.idx[th] = (uint16_t)best;
+                        if (!a.assign_only)
+                            encode_residual_smem<CH, BITS, G>(
+                                sX, sMu, Cpad, row, best, half, a.codes + th * (D * BITS / 8) + half * (CH * BITS / 8),
+                                reinterpret_cast<float2 *>(a.meta) + th * (D / G) + half * (CH / G));
+                    }
+                }
+                // X stage read: the TMA may refill it
+                __syncwarp();
+                if (lane == 0)
+                    mbar_arrive(xempty(st));
+            }
         }
-        tc_fence_before();
-        ok = __syncthreads_and(ok) != 0;
-        if (!ok)
-            break;
+        tile_seq += n;
+        u = seg_end;
+    }
+    // drain: every MMA issued has completed before TMEM is freed
+    if (warp == kFltMmaWarp && lane == 0 && mma_issued > 0) {
+        umma_commit(bar_drain);
+        uint32_t spins = 0;
+        while (!mbar_try_wait(bar_drain, 0) && ++spins < kSpinLimit) {
+        }
     }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     if (warp == 0)
-        tmem_dealloc(tmem, a.tmem_cols);
+        tmem_dealloc(tmem, 2 * kFltAccCols);
 }
 
 }  // namespace kvq

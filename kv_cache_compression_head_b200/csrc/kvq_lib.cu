@@ -141,30 +141,35 @@ bool filter_applies(int D, int C, int G, bool x_bf16)
     return x_bf16 && C <= kFltMaxC && G <= D / 2 && (D == 64 || D == 128);
 }
 
+// X stages that fit beside the centres (2 .. kFltMaxStages).
+int filter_stages(int D, int Cpad)
+{
+    const uint32_t budget = 227u * 1024u - 1024u;
+    const uint32_t fixed = flt_smem_bytes(D, Cpad, 0);
+    const int fit = fixed < budget ? (int)((budget - fixed) / flt_tile_bytes(D)) : 0;
+    return fit < 2 ? 2 : (fit > kFltMaxStages ? kFltMaxStages : fit);
+}
+
 template <int D, int BITS, int G>
 kvq_status launch_filter_t(const CUtensorMap &m, const FilterArgs &a, cudaStream_t s)
 {
-    const uint32_t smem = flt_smem_bytes(D, a.Cpad) + 1024;
-    static bool configured[64] = {};
+    const uint32_t smem = flt_smem_bytes(D, a.Cpad, a.stages) + 1024;
+    static std::atomic<bool> configured[64];
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64)
         return KVQ_ERR_CUDA;
-    if (!configured[dev]) {
+    if (!configured[dev].load()) {
         if (cudaFuncSetAttribute(encode_filter_kernel<D, BITS, G>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  227 * 1024) != cudaSuccess)
             return KVQ_ERR_CUDA;
-        configured[dev] = true;
+        configured[dev].store(true);
     }
-    // CTAs per SM: bounded by shared memory and by TMEM (512 columns)
-    const int by_smem = (int)((228u * 1024u) / (smem + 1024u));
-    const int by_tmem = 512 / a.tmem_cols;
-    const int per_sm = max(1, min(min(by_smem, by_tmem), 8));
-    const int64_t ntiles = (a.T + kFltRows - 1) / kFltRows;
-    // one resident wave: per_sm CTAs on every SM, split evenly across heads
-    const int64_t want = ((int64_t)per_sm * sm_count()) / a.H > 0 ? ((int64_t)per_sm * sm_count()) / a.H : 1;
-    const int64_t gx64 = ntiles < want ? ntiles : want;
-    const unsigned gx = (unsigned)(gx64 > 0 ? gx64 : 1);
-    encode_filter_kernel<D, BITS, G><<<dim3(gx, (unsigned)a.H), kFltThreads, smem, s>>>(m, a);
+    // persistent: one CTA per SM (the two 256-column accumulators take all of
+    // TMEM), each with an equal contiguous share of the (head, tile) units
+    const int64_t units = (int64_t)a.H * a.ntiles;
+    const int64_t sms = sm_count();
+    const unsigned grid = (unsigned)(units < sms ? units : sms);
+    encode_filter_kernel<D, BITS, G><<<grid, kFltThreads, smem, s>>>(m, a);
     return launch_status();
 }
 
@@ -182,17 +187,23 @@ kvq_status launch_filter_g(int G, const CUtensorMap &m, const FilterArgs &a, cud
     }
 }
 
-// Window factor of the certified candidate set (see encode_filter.cuh):
-// kappa = 4 (eps_tc + gamma_d + 2u + gamma_{d+2}), eps_tc = d 2^-21 bounding
-// the tensor-core accumulation error relative to sum |x_c mu_c|.
-// Plus 2^-16 for the column index carried in the low 5 mantissa bits of v
-// (<= 31 ulp each on the smallest and on the compared value, |v| <= (|x|+M)^2).
+// k of the certified candidate set (see encode_filter.cuh), with R_j =
+// |x| + |mu_j| and u = 2^-24:
+//  - every computed L'_j is within rho R_j^2 of its exact value, rho =
+//    gamma_d (the binary32 centre norm) + eps_tc / 2 (the tensor-core dot
+//    product, eps_tc = d 2^-21 relative to sum |x_c mu_c| <= |x||mu_j| <=
+//    R_j^2 / 4, taken twice) + 129 u (the roundings of A_j, of the two FMAs
+//    and of |x|, and the <= 31 ulp of the column index carried in L');
+//  - the specified distance is within gamma_{d+3} R_j^2 of the exact one.
+// k >= rho + gamma_{d+3} suffices; the factor 1.25 and 2^-20 cover the
+// relative error of the threshold's own (|x| + |mu|)^2.
 float filter_kappa(int D)
 {
     const double u = ldexp(1.0, -24);
     const double eps_tc = D * ldexp(1.0, -21);
-    const double g_d = D * u / (1.0 - D * u), g_d2 = (D + 2) * u / (1.0 - (D + 2) * u);
-    return (float)(4.0 * (eps_tc + g_d + 2.0 * u + g_d2) + ldexp(1.0, -16));
+    auto gamma = [&](int n) { return n * u / (1.0 - n * u); };
+    const double rho = gamma(D) + eps_tc / 2.0 + 129.0 * u;
+    return (float)(1.25 * (rho + gamma(D + 3)) + ldexp(1.0, -20));
 }
 
 kvq_status launch_encode_filter(int D, int bits, int G, const void *x, const EncodeArgs &e, cudaStream_t s)
@@ -205,10 +216,8 @@ kvq_status launch_encode_filter(int D, int bits, int G, const void *x, const Enc
     a.H = e.H;
     a.C = e.C;
     a.Cpad = (e.C + 31) / 32 * 32;
-    int cols = 32;
-    while (cols < a.Cpad)
-        cols <<= 1;
-    a.tmem_cols = cols;
+    a.stages = filter_stages(D, a.Cpad);
+    a.ntiles = (e.T + kFltRows - 1) / kFltRows;
     a.cent = e.cent;
     a.idx = e.idx;
     a.codes = e.codes;

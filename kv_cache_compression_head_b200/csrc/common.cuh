@@ -197,6 +197,20 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const void *tmap, uint
         : "memory");
 }
 
+// TMA gather of four rows of a 2-D tensor map whose box is one row high (128
+// bytes of bf16 with 128-byte swizzle here): rows r0..r3 at column c0 land as
+// four consecutive 128-byte rows at `dst`, completing on the mbarrier.  No
+// multicast.
+__device__ __forceinline__ void tma_gather4(uint32_t dst, const void *tmap, uint32_t bar, int c0, int r0, int r1,
+                                            int r2, int r3)
+{
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes [%0], [%1, {%2, "
+        "%3, %4, %5, %6}], [%7];" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(tmap)), "r"(c0), "r"(r0), "r"(r1), "r"(r2), "r"(r3), "r"(bar)
+        : "memory");
+}
+
 // Bounded wait for phase `parity` of an mbarrier.  On expiry the device status
 // word records a timeout and false is returned; callers then stop issuing work.
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity)
@@ -214,6 +228,23 @@ template <int ID>
 __device__ __forceinline__ void named_barrier_sync(int count)
 {
     asm volatile("bar.sync %0, %1;" ::"n"(ID), "r"(count) : "memory");
+}
+
+// Named barrier ID over `count` threads that also returns the AND of `pred`
+// over all of them, so the threads take one decision together.
+template <int ID>
+__device__ __forceinline__ bool named_barrier_and(int count, bool pred)
+{
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\t"
+        "setp.ne.u32 p, %1, 0;\n\t"
+        "bar.red.and.pred q, %2, %3, p;\n\t"
+        "selp.u32 %0, 1, 0, q;\n\t}"
+        : "=r"(r)
+        : "r"((uint32_t)pred), "n"(ID), "r"(count)
+        : "memory");
+    return r != 0;
 }
 
 // Named barrier 1 + q (q = 0..3) over `count` threads.
@@ -311,6 +342,24 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float *v)
     for (int i = 0; i < 32; ++i)
         v[i] = __uint_as_float(r[i]);
 }
+
+// tcgen05.ld of 32 columns without the wait (the caller waits once for all
+// loads in flight with tmem_ld_wait).
+__device__ __forceinline__ void tmem_ld32_nowait(uint32_t taddr, uint32_t *r)
+{
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]),
+          "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]),
+          "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]),
+          "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+        : "r"(taddr));
+}
+
+__device__ __forceinline__ void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 
 // ---------------------------------------------------------------------------
 // 128-byte swizzled operand tiles

@@ -14,6 +14,7 @@
 #include "attention.cuh"
 #include "attention2.cuh"
 #include "attention_pair.cuh"
+#include "attention_tma.cuh"
 #include "codec.cuh"
 #include "common.cuh"
 #include "encode_filter.cuh"
@@ -527,10 +528,75 @@ kvq_status launch_attention_pair_t(const AttnArgs &a, cudaStream_t s)
     return launch_status();
 }
 
+// 2-D tensor map over rows of `row_bytes` bytes (dims innermost first).
+bool encode_2d(CUtensorMap *m, CUtensorMapDataType dt, const void *base, uint64_t inner, uint64_t rows,
+               uint64_t row_bytes, uint32_t box_inner, uint32_t box_rows, CUtensorMapSwizzle sw)
+{
+    PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
+    if (!enc || !base)
+        return false;
+    cuuint64_t dims[2] = {(cuuint64_t)inner, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)row_bytes};
+    cuuint32_t box[2] = {box_inner, box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    return enc(m, dt, 2, const_cast<void *>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// Tensor maps of a compressed K/V history for attention_tma_kernel (d = 128).
+bool make_attn_maps(AttnMaps *m, const AttnArgs &a)
+{
+    const uint64_t rows = (uint64_t)a.H * (uint64_t)a.k.T;
+    const CodecView &k = a.k, &v = a.v;
+    const uint32_t vm_box = v.G == 64 ? 4u : (uint32_t)(64 / v.G) * 2u;
+    return encode_2d(&m->kc, CU_TENSOR_MAP_DATA_TYPE_UINT8, k.codes, 16u * k.bits, rows, 16u * k.bits,
+                     16u * k.bits, 64, CU_TENSOR_MAP_SWIZZLE_NONE) &&
+           encode_2d(&m->km, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, k.meta, 2u * (128 / k.G), rows, 8u * (128 / k.G),
+                     2u * (128 / k.G), 64, CU_TENSOR_MAP_SWIZZLE_NONE) &&
+           encode_2d(&m->vc, CU_TENSOR_MAP_DATA_TYPE_UINT8, v.codes, 16u * v.bits, rows, 16u * v.bits,
+                     8u * v.bits, 128, CU_TENSOR_MAP_SWIZZLE_NONE) &&
+           encode_2d(&m->vm, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, v.meta, 2u * (128 / v.G), rows, 8u * (128 / v.G), vm_box,
+                     128, CU_TENSOR_MAP_SWIZZLE_NONE) &&
+           encode_2d(&m->kcent, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, k.cent, 128, (uint64_t)a.H * k.C, 256, 64, 1,
+                     CU_TENSOR_MAP_SWIZZLE_128B) &&
+           encode_2d(&m->vcent, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, v.cent, 128, (uint64_t)a.H * v.C, 256, 64, 1,
+                     CU_TENSOR_MAP_SWIZZLE_128B);
+}
+
+template <int BK, int BV>
+kvq_status launch_attention_tma_t(const AttnArgs &a, cudaStream_t s)
+{
+    static std::atomic<bool> configured[64];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64)
+        return KVQ_ERR_CUDA;
+    if (!configured[dev].load()) {
+        if (cudaFuncSetAttribute(attention_tma_kernel<BK, BV>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)APSmem::kLaunchBytes) != cudaSuccess)
+            return KVQ_ERR_CUDA;
+        configured[dev].store(true);
+    }
+    AttnMaps maps;
+    if (!make_attn_maps(&maps, a))
+        return KVQ_ERR_CUDA;
+    const dim3 grid((unsigned)(2 * ceil_div(a.Tq, kAPRowsPerPair)), (unsigned)a.H,
+                    (unsigned)(a.nsplit > 1 ? a.nsplit : 1));
+    attention_tma_kernel<BK, BV><<<grid, kATThreads, APSmem::kLaunchBytes, s>>>(maps, a);
+    return launch_status();
+}
+
 kvq_status launch_attention_pair(const AttnArgs &a, cudaStream_t s)
 {
     if (a.dense)
         return launch_attention_pair_t<0, 0, true>(a, s);
+    // compressed history with keys to read: every byte staged by TMA (row
+    // coordinates are 32-bit); an empty range needs no staging
+    if (a.t_end > a.t_begin && (int64_t)a.H * a.k.T < (int64_t)INT32_MAX &&
+        (int64_t)a.H * (a.k.C > a.v.C ? a.k.C : a.v.C) < (int64_t)INT32_MAX) {
+        if (a.k.bits == 2)
+            return a.v.bits == 2 ? launch_attention_tma_t<2, 2>(a, s) : launch_attention_tma_t<2, 4>(a, s);
+        return a.v.bits == 2 ? launch_attention_tma_t<4, 2>(a, s) : launch_attention_tma_t<4, 4>(a, s);
+    }
     if (a.k.bits == 2)
         return a.v.bits == 2 ? launch_attention_pair_t<2, 2, false>(a, s) : launch_attention_pair_t<2, 4, false>(a, s);
     return a.v.bits == 2 ? launch_attention_pair_t<4, 2, false>(a, s) : launch_attention_pair_t<4, 4, false>(a, s);

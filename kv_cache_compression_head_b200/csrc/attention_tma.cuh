@@ -26,7 +26,7 @@
 // all completing on the stage's fill barrier.  The producers (8 warps) wait
 // on that barrier, copy their code words and {s, z} to registers, meet at a
 // named barrier (the K lo writes overwrite the staged words), rebuild their
-// units in place and publish them with a proxy fence.  They have no copies of
+// units of K and V in place and publish both behind one proxy fence.  They have no copies of
 // their own in flight, so the fence does not wait on memory.
 //
 // Barriers (parity = use count & 1): those of attention_pair.cuh plus
@@ -186,9 +186,14 @@ __device__ __forceinline__ void at_produce(const AttnArgs &a, uint32_t rank, int
         if (!named_barrier_and<5>(kAPProducers, filled))
             return;
         ap_rebuild<BK, true>(khi(s), klo(s), koff, kcw, ksz, t0 + 64 * rank + krow < a.t_end);
-        ap_publish(lead(P_KFULL0 + s));
         ap_rebuild<BV, false>(vst(s), nullptr, voff, vcw, vsz, t0 + vrow < a.t_end);
-        ap_publish(lead(P_VFULL0 + s));
+        // one proxy fence for both tiles (a fence costs more than a rebuild)
+        fence_proxy_async_smem();
+        __syncwarp();
+        if ((threadIdx.x & 31) == 0) {
+            mbar_arrive_cluster(lead(P_KFULL0 + s));
+            mbar_arrive_cluster(lead(P_VFULL0 + s));
+        }
     }
 }
 

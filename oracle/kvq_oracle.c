@@ -56,6 +56,15 @@
  *    codes 0, which decodes to exactly min (and to 0 when min == 0);
  *  - decode: x^_c = mu_c + (q_c - z) * s with the subtraction, multiply and
  *    add each rounded to binary32;
+ *  - compact {s, z} (16-bit scale and zero per group, the b + 1 bits per value
+ *    of TempoKV, Table 1, at G = 32): s is formed as above, then rounded to
+ *    binary16 (nearest, ties to even, magnitudes past the largest finite
+ *    binary16 saturating to it); inv = 1/s16 and z = rint(-min * inv) use the
+ *    rounded scale, z is rounded to binary16 in the same way, and the codes
+ *    are q = clamp(rint(r * inv) + z16, 0, 2^b - 1), so that encode and decode
+ *    use the stored values.  A degenerate group, or one whose scale rounds to
+ *    zero in binary16, stores s16 = binary16(|min|), z16 = -sign(min) and
+ *    codes 0 (decoding to min rounded to binary16);
  *  - QSAC arithmetic in binary32, channel order, no FMA: weighted distance
  *    acc += w_c * (e_c * e_c); group weight W_g = sum of w_c in channel order;
  *    R_g = max - min of the group's residuals; score += W_g * (R_g * R_g) over
@@ -98,6 +107,60 @@ static uint16_t bf16_round(float f)
 }
 
 uint16_t kvqo_bf16_round(float f) { return bf16_round(f); }
+
+/* ------------------------------------------------------------------------ */
+/* binary16 storage conversions (compact {s, z})                             */
+/* ------------------------------------------------------------------------ */
+
+/*
+ * binary32 -> binary16 by the IEEE 754 definition: round to nearest, ties to
+ * even, gradual underflow to subnormals; a magnitude that would round to
+ * infinity (>= 65520) saturates to the largest finite value 65504; NaN gives
+ * the quiet NaN 0x7e00 with the sign kept.
+ */
+uint16_t kvqo_f16_round(float f)
+{
+    uint32_t u;
+    memcpy(&u, &f, sizeof u);
+    const uint32_t sign = (u >> 16) & 0x8000u;
+    const uint32_t a = u & 0x7fffffffu;
+    if (a > 0x7f800000u)
+        return (uint16_t)(sign | 0x7e00u);
+    if (a >= 0x477ff000u) /* 65520 and above, infinity included */
+        return (uint16_t)(sign | 0x7bffu);
+    if (a >= 0x38800000u) { /* 2^-14 and above: a normal binary16 */
+        const uint32_t exp = (a >> 23) - 112u, mant = a & 0x7fffffu;
+        uint32_t h = (exp << 10) | (mant >> 13);
+        const uint32_t rem = mant & 0x1fffu; /* the 13 bits dropped */
+        if (rem > 0x1000u || (rem == 0x1000u && (h & 1u)))
+            h += 1u; /* a carry into the exponent is the correct result */
+        return (uint16_t)(sign | h);
+    }
+    /* subnormal or zero: a multiple of 2^-24; |f| 2^24 is exact in binary32 */
+    float t;
+    memcpy(&t, &a, sizeof t);
+    t = rintf(t * 16777216.0f); /* ties to even (the default rounding mode) */
+    return (uint16_t)(sign | (uint32_t)t);
+}
+
+/* binary16 -> binary32 (exact). */
+float kvqo_f16_widen(uint16_t h)
+{
+    const uint32_t sign = ((uint32_t)h & 0x8000u) << 16;
+    const uint32_t e = (h >> 10) & 0x1fu, m = h & 0x3ffu;
+    float f;
+    if (e == 0) {
+        f = (float)m * (1.0f / 16777216.0f); /* m 2^-24, exact */
+        uint32_t v;
+        memcpy(&v, &f, sizeof v);
+        v |= sign;
+        memcpy(&f, &v, sizeof f);
+        return f;
+    }
+    uint32_t v = sign | (e == 31 ? (0xffu << 23) | (m << 13) : ((e + 112u) << 23) | (m << 13));
+    memcpy(&f, &v, sizeof f);
+    return f;
+}
 
 /* x is either binary32 ([n]) or bf16 bit patterns ([n]); returns binary32. */
 static float load_x(const void *x, int x_is_bf16, int64_t i)
@@ -309,6 +372,52 @@ void kvqo_quant_group(const float *r, int G, int bits, float *s_out, float *z_ou
     *z_out = z;
 }
 
+/*
+ * Eq. 1 with 16-bit {s, z} (the compact reading in the header): writes the
+ * binary16 bits of s and z and G codes computed with the stored values.
+ */
+void kvqo_quant_group16(const float *r, int G, int bits, uint16_t *s_out, uint16_t *z_out, uint8_t *q)
+{
+    float mn = r[0], mx = r[0];
+    for (int c = 1; c < G; ++c) {
+        if (r[c] < mn)
+            mn = r[c];
+        if (r[c] > mx)
+            mx = r[c];
+    }
+    const float qmax = (float)((1 << bits) - 1);
+    float s = 0.0f;
+    if (mx != mn)
+        s = (mx - mn) / qmax;
+    const uint16_t s16 = kvqo_f16_round(s);
+    if (mx == mn || !(s >= FLT_MIN) || (s16 & 0x7fffu) == 0u) {
+        if (mn == 0.0f) {
+            *s_out = 0u;
+            *z_out = 0u;
+        } else {
+            *s_out = kvqo_f16_round(fabsf(mn));
+            *z_out = (mn > 0.0f) ? 0xbc00u /* -1 */ : 0x3c00u /* +1 */;
+        }
+        for (int c = 0; c < G; ++c)
+            q[c] = 0;
+        return;
+    }
+    const float sf = kvqo_f16_widen(s16);
+    const float inv = 1.0f / sf;
+    const uint16_t z16 = kvqo_f16_round(rintf(-mn * inv));
+    const float zf = kvqo_f16_widen(z16);
+    for (int c = 0; c < G; ++c) {
+        float v = rintf(r[c] * inv) + zf;
+        if (v < 0.0f)
+            v = 0.0f;
+        if (v > qmax)
+            v = qmax;
+        q[c] = (uint8_t)v;
+    }
+    *s_out = s16;
+    *z_out = z16;
+}
+
 /* x^ = (q - z) * s, each step rounded to binary32. */
 float kvqo_dequant(uint8_t q, float s, float z)
 {
@@ -430,6 +539,84 @@ int kvqo_decode(const uint16_t *idx, const uint8_t *codes, const float *meta, co
                 int g = c / G;
                 float s = meta[(th * ng + g) * 2 + 0];
                 float z = meta[(th * ng + g) * 2 + 1];
+                float mu = bf16_widen(cent[((int64_t)h * C + j) * d + c]);
+                out[(t * H + h) * (int64_t)d + c] = mu + kvqo_dequant(q[c], s, z);
+            }
+        }
+        free(q);
+    }
+    return rc;
+}
+
+/*
+ * kvqo_encode with 16-bit {s, z}: meta16 [H][T][d/G][2] binary16 bits
+ * {s, z}; everything else as kvqo_encode.
+ */
+int kvqo_encode16(const void *x, int x_is_bf16, int64_t T, int H, int d, const uint16_t *cent, int C, int bits,
+                  int G, uint16_t *idx, uint8_t *codes, uint16_t *meta16)
+{
+    if (T < 0 || !check_codec(H, d, C, bits, G))
+        return KVQO_EINVAL;
+    const int cb = d * bits / 8, ng = d / G;
+    int rc = KVQO_OK;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int h = 0; h < H; ++h) {
+        float *mu = (float *)malloc(sizeof(float) * (size_t)C * d);
+        float *xv = (float *)malloc(sizeof(float) * (size_t)d);
+        float *r = (float *)malloc(sizeof(float) * (size_t)d);
+        uint8_t *q = (uint8_t *)malloc((size_t)d);
+        if (!mu || !xv || !r || !q) {
+            rc = KVQO_ENOMEM;
+        } else {
+            widen_centres(cent + (int64_t)h * C * d, C, d, mu);
+            for (int64_t t = 0; t < T; ++t) {
+                int64_t th = (int64_t)h * T + t;
+                gather_token(x, x_is_bf16, H, d, t, h, xv);
+                int j = nearest(xv, mu, C, d, NULL);
+                idx[th] = (uint16_t)j;
+                for (int c = 0; c < d; ++c)
+                    r[c] = xv[c] - mu[(int64_t)j * d + c];
+                for (int g = 0; g < ng; ++g)
+                    kvqo_quant_group16(r + g * G, G, bits, &meta16[(th * ng + g) * 2 + 0],
+                                       &meta16[(th * ng + g) * 2 + 1], q + g * G);
+                kvqo_pack(q, d, bits, codes + th * cb);
+            }
+        }
+        free(mu);
+        free(xv);
+        free(r);
+        free(q);
+    }
+    return rc;
+}
+
+/* kvqo_decode for 16-bit {s, z}: x^ = mu + (q - z16) * s16 in binary32. */
+int kvqo_decode16(const uint16_t *idx, const uint8_t *codes, const uint16_t *meta16, const uint16_t *cent,
+                  int64_t T, int H, int d, int C, int bits, int G, float *out)
+{
+    if (T < 0 || !check_codec(H, d, C, bits, G))
+        return KVQO_EINVAL;
+    const int cb = d * bits / 8, ng = d / G;
+    int rc = KVQO_OK;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int h = 0; h < H; ++h) {
+        uint8_t *q = (uint8_t *)malloc((size_t)d);
+        if (!q) {
+            rc = KVQO_ENOMEM;
+            continue;
+        }
+        for (int64_t t = 0; t < T; ++t) {
+            int64_t th = (int64_t)h * T + t;
+            int j = idx[th];
+            if (j >= C) {
+                rc = KVQO_EINVAL;
+                break;
+            }
+            kvqo_unpack(codes + th * cb, d, bits, q);
+            for (int c = 0; c < d; ++c) {
+                int g = c / G;
+                float s = kvqo_f16_widen(meta16[(th * ng + g) * 2 + 0]);
+                float z = kvqo_f16_widen(meta16[(th * ng + g) * 2 + 1]);
                 float mu = bf16_widen(cent[((int64_t)h * C + j) * d + c]);
                 out[(t * H + h) * (int64_t)d + c] = mu + kvqo_dequant(q[c], s, z);
             }

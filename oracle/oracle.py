@@ -81,6 +81,13 @@ def _load():
     lib.kvqo_unpack.argtypes = [vp, i32, i32, vp]
     lib.kvqo_bf16_round.argtypes = [ctypes.c_float]
     lib.kvqo_bf16_round.restype = ctypes.c_uint16
+    lib.kvqo_f16_round.argtypes = [ctypes.c_float]
+    lib.kvqo_f16_round.restype = ctypes.c_uint16
+    lib.kvqo_f16_widen.argtypes = [ctypes.c_uint16]
+    lib.kvqo_f16_widen.restype = ctypes.c_float
+    lib.kvqo_quant_group16.argtypes = [vp, i32, i32, vp, vp, vp]
+    lib.kvqo_encode16.argtypes = [vp, i32, i64, i32, i32, vp, i32, i32, i32, vp, vp, vp]
+    lib.kvqo_decode16.argtypes = [vp, vp, vp, vp, i64, i32, i32, i32, i32, i32, vp]
     _lib = lib
     return lib
 
@@ -146,6 +153,26 @@ def bf16_round(f: float) -> int:
     return int(_load().kvqo_bf16_round(f))
 
 
+def f16_round(f: float) -> int:
+    """binary32 -> binary16 bits: nearest, ties to even, subnormals, saturating
+    at 65504 (the compact {s, z} storage)."""
+    return int(_load().kvqo_f16_round(f))
+
+
+def f16_widen(h: int) -> float:
+    return float(_load().kvqo_f16_widen(h))
+
+
+def quant_group16(r: np.ndarray, bits: int) -> Tuple[int, int, np.ndarray]:
+    """Eq. 1 on one group with 16-bit {s, z}: (s16 bits, z16 bits, codes)."""
+    r = np.ascontiguousarray(r, dtype=np.float32)
+    s = np.zeros(1, np.uint16)
+    z = np.zeros(1, np.uint16)
+    q = np.zeros(r.shape[0], np.uint8)
+    _load().kvqo_quant_group16(_ptr(r), r.shape[0], bits, _ptr(s), _ptr(z), _ptr(q))
+    return int(s[0]), int(z[0]), q
+
+
 # ----------------------------------------------------------------------------
 # codec
 # ----------------------------------------------------------------------------
@@ -184,6 +211,31 @@ def encode(x: np.ndarray, cent: np.ndarray, bits: int, group: int):
     _check(_load().kvqo_encode(_ptr(x), xb, T, H, d, _ptr(cent), C, bits, group,
                                _ptr(idx), _ptr(codes), _ptr(meta)), "encode")
     return idx, codes, meta
+
+
+def encode16(x: np.ndarray, cent: np.ndarray, bits: int, group: int):
+    """encode with 16-bit {s, z}: (idx, codes, meta16 [H][T][d/G][2] binary16 bits as u16)."""
+    x, xb = _x_arg(x)
+    T, H, d = x.shape
+    C = cent.shape[1]
+    cent = np.ascontiguousarray(cent, dtype=np.uint16)
+    idx = np.zeros((H, T), np.uint16)
+    codes = np.zeros((H, T, d * bits // 8), np.uint8)
+    meta = np.zeros((H, T, d // group, 2), np.uint16)
+    _check(_load().kvqo_encode16(_ptr(x), xb, T, H, d, _ptr(cent), C, bits, group,
+                                 _ptr(idx), _ptr(codes), _ptr(meta)), "encode16")
+    return idx, codes, meta
+
+
+def decode16(idx: np.ndarray, codes: np.ndarray, meta16: np.ndarray, cent: np.ndarray,
+             bits: int, group: int) -> np.ndarray:
+    """Reconstruction [T][H][d] float32 from the 16-bit {s, z} form."""
+    H, T = idx.shape
+    C, d = cent.shape[1], cent.shape[2]
+    out = np.zeros((T, H, d), np.float32)
+    args = [np.ascontiguousarray(a) for a in (idx, codes, meta16, cent)]
+    _check(_load().kvqo_decode16(*(_ptr(a) for a in args), T, H, d, C, bits, group, _ptr(out)), "decode16")
+    return out
 
 
 def decode(idx: np.ndarray, codes: np.ndarray, meta: np.ndarray, cent: np.ndarray,

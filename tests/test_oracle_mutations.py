@@ -44,6 +44,13 @@ MUTATIONS = [
     ("QSAC score ties to the worse-ranked candidate", "if (k == 0 || sc < best) {", "if (k == 0 || sc <= best) {"),
     ("QSAC ranking ties to the higher index", "while (pos > 0 && dj < cand_dist[pos - 1])",
      "while (pos > 0 && dj <= cand_dist[pos - 1])"),
+    ("compact codec takes 1/s from the unrounded scale", "const float inv = 1.0f / sf;", "const float inv = 1.0f / s;"),
+    ("binary16 rounding truncates", "if (rem > 0x1000u || (rem == 0x1000u && (h & 1u)))\n            h += 1u;",
+     "(void)rem;"),
+    ("binary16 overflow goes to infinity", "return (uint16_t)(sign | 0x7bffu);", "return (uint16_t)(sign | 0x7c00u);"),
+    ("compact codec keeps a scale that rounds to zero", " || (s16 & 0x7fffu) == 0u", ""),
+    ("compact decode forgets the zero point", "float z = kvqo_f16_widen(meta16[(th * ng + g) * 2 + 1]);",
+     "float z = 0.0f;"),
 ]
 
 

@@ -11,6 +11,7 @@ import numpy as np
 import pytest
 import torch
 
+from kv_cache_compression_head_b200 import synth
 from oracle import oracle as O
 
 GOLDEN = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden")
@@ -671,3 +672,106 @@ def test_qsac_ties_follow_index_order():
     assert [int(c) for c in cand[0, 0]] == [0, 1, 2] and int(idx[0, 0]) == 0
     idx, cand = O.qsac_assign(x, cent[:, ::-1].copy(), w, 2, 2, return_candidates=True)
     assert [int(c) for c in cand[0, 0]] == [0, 1] and int(idx[0, 0]) == 0
+
+# ----------------------------------------------------------------------------
+# compact 16-bit {s, z} (TempoKV, Table 1: b + 1 bits per value at G = 32)
+# ----------------------------------------------------------------------------
+
+def test_f16_round_golden():
+    g = _golden("eq1_f16_worked_examples.json")
+    for case in g["round"]:
+        assert O.f16_round(case["f"]) == case["h"], case["note"]
+
+
+def test_f16_round_matches_numpy_in_range():
+    """numpy's float16 conversion (round to nearest even, gradual underflow)
+    is an independent implementation; they agree wherever numpy does not
+    overflow, and numpy's widening agrees on every finite pattern."""
+    rng = np.random.default_rng(61)
+    vals = np.concatenate([
+        rng.normal(size=4000) * 10.0 ** rng.uniform(-9, 4.8, size=4000),
+        (rng.integers(0, 4096, size=2000) + rng.choice([0.25, 0.5, 0.75], size=2000)) * 2.0 ** -24,
+        rng.uniform(-65519, 65519, size=2000),
+    ]).astype(np.float32)
+    vals = vals[np.abs(vals) < 65520.0]  # numpy rounds these to infinity; the oracle saturates
+    want = vals.astype(np.float16).view(np.uint16)
+    got = np.array([O.f16_round(float(v)) for v in vals], np.uint16)
+    assert np.array_equal(got, want), f"differs at {vals[got != want][:5]}"
+    bits = np.arange(0, 65536, dtype=np.uint32).astype(np.uint16)
+    fin = np.isfinite(bits.view(np.float16))
+    widened = np.array([O.f16_widen(int(b)) for b in bits[fin]], np.float32)
+    assert np.array_equal(widened.view(np.uint32), bits[fin].view(np.float16).astype(np.float32).view(np.uint32))
+
+
+def test_eq1_f16_worked_examples():
+    g = _golden("eq1_f16_worked_examples.json")
+    for case in g["groups"]:
+        s16, z16, q = O.quant_group16(np.array(case["r"], np.float32), case["bits"])
+        assert (s16, z16) == (case["s16"], case["z16"]), case["note"]
+        assert q.tolist() == case["q"], case["note"]
+        dec = [O.dequant(int(qq), O.f16_widen(s16), O.f16_widen(z16)) for qq in q]
+        assert dec == case["decoded"], case["note"]
+
+
+def test_eq1_f16_error_bound():
+    """For groups whose zero point is stored exactly (min <= 0 <= max keeps it
+    in [0, 2^b - 1]), every residual decodes within s16/2 + (2^b - 1)|s - s16|
+    (the grid of the rounded scale may stop short of max) plus binary32
+    rounding."""
+    rng = np.random.default_rng(62)
+    for trial in range(400):
+        bits = (2, 4)[trial % 2]
+        G = (16, 32, 64)[trial % 3]
+        r = (rng.normal(size=G) * 10.0 ** rng.uniform(-3, 2)).astype(np.float32)
+        r[0], r[1] = -abs(r[0]), abs(r[1])
+        s16, z16, q = O.quant_group16(r, bits)
+        s_exact = (np.float32(r.max()) - np.float32(r.min())) / np.float32((1 << bits) - 1)
+        sf, zf = O.f16_widen(s16), O.f16_widen(z16)
+        assert zf == np.rint(zf) and 0 <= zf <= (1 << bits) - 1
+        dec = np.array([O.dequant(int(qq), sf, zf) for qq in q], np.float64)
+        bound = sf / 2 + ((1 << bits) - 1) * abs(float(s_exact) - sf) + 4 * np.spacing(np.abs(r).max())
+        assert np.all(np.abs(dec - r.astype(np.float64)) <= bound)
+
+
+def test_eq1_f16_equals_binary32_codec_when_scale_is_a_half():
+    """Groups whose binary32 scale is itself a binary16 value and whose zero
+    point is small: the compact codec stores the same s and z and the same
+    codes as the binary32 one."""
+    rng = np.random.default_rng(63)
+    for trial in range(200):
+        bits = (2, 4)[trial % 2]
+        qmax = (1 << bits) - 1
+        s = np.float32(np.float16(2.0 ** rng.integers(-8, 4) * rng.integers(1, 1024) / 512.0))
+        mn = -np.float32(rng.integers(0, qmax + 1)) * s
+        r = (mn + rng.integers(0, qmax * 4 + 1, size=32).astype(np.float32) * s / np.float32(4.0)).astype(np.float32)
+        r[0], r[1] = mn, mn + np.float32(qmax) * s
+        if np.float32(r.max() - r.min()) / np.float32(qmax) != s:
+            continue
+        s32, z32, q32 = O.quant_group(r, bits)
+        s16, z16, q16 = O.quant_group16(r, bits)
+        assert O.f16_widen(s16) == s32 and O.f16_widen(z16) == z32
+        assert np.array_equal(q16, q32)
+
+
+def test_encode16_decode16_storage_and_bound():
+    """The compact codec on a history: the same centre indices as the binary32
+    codec, half the metadata bytes (4 per group against 8), and every value
+    decoded within the per-group bound of the compact quantiser."""
+    rng = np.random.default_rng(64)
+    T, H, d, C = 300, 2, 64, 8
+    x = synth.bf16_bits_from_f64(rng.normal(size=(T, H, d)) * rng.uniform(0.5, 3, size=(1, H, d)))
+    cent = O.fit(x, C, 2)
+    for bits, G in ((2, 16), (4, 32)):
+        idx, codes, meta = O.encode(x, cent, bits, G)
+        idx16, codes16, meta16 = O.encode16(x, cent, bits, G)
+        assert np.array_equal(idx16, idx)
+        assert meta16.nbytes * 2 == meta.nbytes
+        dec = O.decode16(idx16, codes16, meta16, cent, bits, G).astype(np.float64)
+        xf = synth.bf16_bits_to_f32(x).astype(np.float64)
+        s32 = meta[..., 0].astype(np.float64)
+        s16 = np.vectorize(O.f16_widen)(meta16[..., 0]).astype(np.float64)
+        z16 = np.vectorize(O.f16_widen)(meta16[..., 1])
+        exact_z = (z16 == np.rint(z16)) & (np.abs(z16) <= 2048)
+        bound = s16 / 2 + ((1 << bits) - 1) * np.abs(s32 - s16) + 1e-6 * (1 + np.abs(xf).max())
+        err = np.abs(dec - xf).transpose(1, 0, 2).reshape(H, T, d // G, G).max(axis=3)
+        assert np.all(err[exact_z] <= bound[exact_z])

@@ -41,7 +41,8 @@
  *      codes (per-head) [H][T][d*b/8]    uint8, code of channel c of a byte
  *                                         holds bits (c % (8/b)) * b ..; low
  *                                         bits first
- *      meta  (per-head) [H][T][d/G][2]   float {scale s, zero z}
+ *      meta  (per-head) [H][T][d/G][2]   {scale s, zero z}: float, or
+ *                                         binary16 bits (meta_format)
  *      codes (joint)    [T][r*b/8]       meta (joint) [T][r/G][2]
  *      queries q        [Tq][H][d]       bf16;  output o [Tq][H][d]
  *      lse              [H][Tq]          float, natural logarithm
@@ -78,6 +79,12 @@ typedef enum {
 
 typedef enum { KVQ_F32 = 0, KVQ_BF16 = 1 } kvq_dtype;
 
+/* Storage of the per-group {scale, zero} pair (kvq_codec_desc.meta_format). */
+typedef enum {
+    KVQ_META_F32 = 0, /* binary32 {s, z}: 8 bytes per group */
+    KVQ_META_F16 = 1  /* binary16 {s, z}: 4 bytes per group (see kvq_encode) */
+} kvq_meta_format;
+
 typedef enum {
     KVQ_OP_FIT = 0,
     KVQ_OP_ENCODE = 1,
@@ -95,6 +102,7 @@ typedef struct {
     int32_t bits;          /* b: 2 or 4 */
     int32_t group_size;    /* G: multiple of 8 dividing d (per-head) or r (joint) */
     int32_t joint_rank;    /* 0: per-head codec; r > 0: joint head-channel code */
+    int32_t meta_format;   /* kvq_meta_format; 0 (binary32) when zero-initialised */
 } kvq_codec_desc;
 
 /* A compressed K or V history as produced by kvq_encode (read-only view). */
@@ -104,7 +112,7 @@ typedef struct {
     const void *centroids;  /* [H][C][d] bf16 */
     const uint16_t *idx;    /* [H][T] */
     const uint8_t *codes;   /* per-head [H][T][d*b/8]; joint [T][r*b/8] */
-    const float *meta;      /* per-head [H][T][d/G][2]; joint [T][r/G][2] */
+    const void *meta;       /* per-head [H][T][d/G][2]; joint [T][r/G][2] (meta_format) */
     const void *w_dec;      /* joint only: decoder [r][H*d] bf16; else NULL */
 } kvq_compressed_view;
 
@@ -186,6 +194,13 @@ KVQ_API kvq_status kvq_fit_centroids_static(const kvq_codec_desc *desc, const vo
  *   q = clamp(rint(r/s) + z, 0, 2^b - 1) with 1/s formed once per group
  *   (TempoKV, Sec. 3.1, Eq. 1); a zero-range (or underflowing) group stores
  *   s = |min|, z = -sign(min), q = 0.  Codes packed low bits first.
+ *   Compact {s, z} (meta_format = KVQ_META_F16; the b + 1 bits per value of
+ *   TempoKV, Table 1, at G = 32): s is rounded to binary16 (nearest, ties to
+ *   even, saturating at 65504), 1/s and z are formed from the rounded scale,
+ *   z is rounded to binary16 likewise, and the codes use the stored values;
+ *   a zero-range group, or one whose scale rounds to zero, stores
+ *   s = binary16(|min|), z = -sign(min), q = 0.  Per-head codec only (the
+ *   joint codec returns KVQ_ERR_UNSUPPORTED).
  * Joint codec (desc->joint_rank = r > 0, w_enc = [H*d][r] bf16):
  *   idx as above per head; the residual of all H*d channels of a token is
  *   rounded to bf16 and projected, c = R W_enc (tensor-core GEMM, binary32
@@ -199,7 +214,7 @@ KVQ_API kvq_status kvq_fit_centroids_static(const kvq_codec_desc *desc, const vo
  * arguments are accepted and ignored).
  */
 KVQ_API kvq_status kvq_encode(const kvq_codec_desc *desc, const void *x, kvq_dtype x_dtype, int64_t num_tokens,
-                      const void *centroids, const void *w_enc, uint16_t *idx, uint8_t *codes, float *meta,
+                      const void *centroids, const void *w_enc, uint16_t *idx, uint8_t *codes, void *meta,
                       void *workspace, size_t workspace_bytes, kvq_stream_t stream);
 
 /*
@@ -218,7 +233,8 @@ KVQ_API kvq_status kvq_joint_coefficients(const kvq_codec_desc *desc, const void
  * Reconstruct a history from its compressed view (NanoKV page, Fig. 4(b):
  * the decoder reconstructs the residual and adds back the centres).
  * Per-head: x^ = mu[idx] + (q - z) * s, each step rounded to binary32
- * (subtract, multiply, add; no FMA), then stored as float or bf16 (RNE).
+ * (subtract, multiply, add; no FMA), then stored as float or bf16 (RNE);
+ * with compact {s, z} the binary16 values are widened first.
  * Joint: c^ = (q - z) s (binary32); R^ = c^ W_dec (tensor-core GEMM: c^ is
  *   carried as a bf16 high part plus a bf16 remainder, about 16 significant
  *   bits, against bf16 W_dec with binary32 accumulation); x^ = mu[idx] + R^
@@ -239,8 +255,10 @@ KVQ_API kvq_status kvq_decode(const kvq_compressed_view *view, void *x_out, kvq_
  * k^ and v^ are rounded to bf16 for the tensor cores; logits, softmax and the
  * output accumulate in binary32.  No mask: the history precedes the chunk.
  *   q     [Tq][H][d] bf16;  o_out [Tq][H][d] (o_dtype);  lse_out [H][Tq]
- * k and v must have the same H, d and num_tokens; their bits, group sizes and
- * centroid counts may differ.  An empty range gives o = 0, lse = -inf.
+ * k and v must have the same H, d and num_tokens; their bits, group sizes,
+ * centroid counts and meta formats may differ.  Compact {s, z} needs d = 128
+ * (KVQ_ERR_UNSUPPORTED for d = 64).  An empty range gives o = 0,
+ * lse = -inf.
  * Workspace (optional): with at least kvq_workspace_size(KVQ_OP_ATTENTION, k
  * desc, T, Tq) bytes (16-byte aligned), the call may split the history range
  * into up to 4 sub-ranges processed by separate CTAs when that fills the GPU

@@ -19,11 +19,12 @@ struct CodecView {
     const uint16_t *cent;  // [H][C][D] bf16
     const uint16_t *idx;   // [H][T]
     const uint8_t *codes;  // [H][T][D*bits/8]
-    const float *meta;     // [H][T][D/G][2]
+    const void *meta;      // [H][T][D/G][2] float, or binary16 when meta16
     int64_t T;
     int C;
     int bits;
     int G;
+    int meta16;
 };
 
 struct AttnArgs {

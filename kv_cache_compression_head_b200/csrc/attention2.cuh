@@ -136,7 +136,7 @@ __device__ __forceinline__ void a2_dequant_half(const CodecView &cv, int h, int6
         for (int uu = 0; uu < kUnits; ++uu)
             cws[uu] = __ldg(cr + uu);
     }
-    const float2 *meta_row = reinterpret_cast<const float2 *>(cv.meta) + th * (D / cv.G);
+    const float2 *meta_row = static_cast<const float2 *>(cv.meta) + th * (D / cv.G);  // binary32 {s, z} only
     constexpr float kTwoB = (float)(1 << BITS);
 #pragma unroll
     for (int uu = 0; uu < kUnits; ++uu) {

@@ -235,7 +235,7 @@ __device__ __forceinline__ void ap_stage(const CodecView &cv, int h, int64_t tok
         cp_async8(stage_cw, cv.codes + th * (D / 4) + u0 * 2);
     else
         cp_async16(stage_cw, cv.codes + th * (D / 2) + u0 * 4);
-    const float *meta = cv.meta + (th * (D / cv.G) + (u0 * 8) / cv.G) * 2;
+    const float *meta = static_cast<const float *>(cv.meta) + (th * (D / cv.G) + (u0 * 8) / cv.G) * 2;  // binary32 {s, z}
     if (cv.G == 16)
         cp_async16(stage_sz, meta);
     else

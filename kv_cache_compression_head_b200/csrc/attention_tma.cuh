@@ -19,6 +19,9 @@
 //  - tiled TMA loads of the tile's packed codes and {s, z} pairs into the
 //    stage's K lo slot (the CTA's 64 K rows whole; the CTA's channel half of
 //    all 128 V rows), from 2-D views [H T][row bytes] of the codec arrays;
+//    compact binary16 {s, z} rows (8 to 32 bytes, too narrow for a tiled
+//    copy at G = 64) are read by the loader lanes instead and stored before
+//    the fill barrier's arrival, which releases them to the producers;
 //  - TMA gathers (tile::gather4) of the centre rows mu_h[idx] straight into
 //    their 128-byte-swizzled operand rows: both 64-channel halves of the 64 K
 //    rows into K hi, this CTA's channel half of the 128 V rows into V, four
@@ -81,8 +84,12 @@ __device__ __forceinline__ void at_load(const AttnArgs &a, const AttnMaps &m, in
     auto klo = [&](int s) { return smem_u32(smem + L::offK + (uint32_t)(2 * s + 1) * L::kKh); };
     auto vst = [&](int s) { return smem_u32(smem + L::offV + (uint32_t)s * L::kV); };
     const int Gk = a.k.G, Gv = a.v.G;
-    const uint32_t bytes = 16384u + 16384u + 64u * 16u * BK + 64u * (uint32_t)(128 / Gk) * 8u + 128u * 8u * BV +
-                           128u * (uint32_t)at_vm_row_bytes(Gv);
+    const bool k16 = a.k.meta16 != 0, v16 = a.v.meta16 != 0;
+    const uint32_t bytes = 16384u + 16384u + 64u * 16u * BK + (k16 ? 0u : 64u * (uint32_t)(128 / Gk) * 8u) +
+                           128u * 8u * BV + (v16 ? 0u : 128u * (uint32_t)at_vm_row_bytes(Gv));
+    // compact {s, z}: whole rows of 4 (128/G) bytes, in 8-byte words
+    const int kw_row = (128 / Gk) / 2, vw_row = (128 / Gv) / 2;  // words per row
+    const int kw_lane = 64 * kw_row / 32, vw_lane = 128 * vw_row / 32;
     const int vc_x = (int)rank * 8 * BV;
     const int vm_x = Gv == 64 ? 0 : (int)rank * (64 / Gv) * 2;
     const int64_t rowK = (int64_t)h * a.k.T, rowV = (int64_t)h * a.v.T;
@@ -109,12 +116,53 @@ __device__ __forceinline__ void at_load(const AttnArgs &a, const AttnMaps &m, in
             kr[q] = centK + ik;
             vr[q] = centV + iv;
         }
+        uint2 km16[8], vm16[16];
+        if (k16) {
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+                const int w = lane + 32 * q;
+                km16[q] = make_uint2(0u, 0u);
+                if (q < kw_lane) {
+                    const int64_t t = t0 + 64 * rank + w / kw_row;
+                    if (t < a.k.T)
+                        km16[q] = __ldg(static_cast<const uint2 *>(a.k.meta) + (rowK + t) * kw_row + w % kw_row);
+                }
+            }
+        }
+        if (v16) {
+#pragma unroll
+            for (int q = 0; q < 16; ++q) {
+                const int w = lane + 32 * q;
+                vm16[q] = make_uint2(0u, 0u);
+                if (q < vw_lane) {
+                    const int64_t t = t0 + w / vw_row;
+                    if (t < a.v.T)
+                        vm16[q] = __ldg(static_cast<const uint2 *>(a.v.meta) + (rowV + t) * vw_row + w % vw_row);
+                }
+            }
+        }
         if (i >= kAPStages) {
             const uint32_t par = (uint32_t)(((i / kAPStages) - 1) & 1);
             ok = __all_sync(0xffffffffu, ap_wait(bar(P_KFREE0 + s), par, abort_flag) &&
                                              ap_wait(bar(P_VFREE0 + s), par, abort_flag));
             if (!ok)
                 break;
+        }
+        {
+            uint8_t *lo_p = smem + L::offK + (uint32_t)(2 * s + 1) * L::kKh;
+            if (k16) {
+#pragma unroll
+                for (int q = 0; q < 8; ++q)
+                    if (q < kw_lane)
+                        reinterpret_cast<uint2 *>(lo_p + kATStKm)[lane + 32 * q] = km16[q];
+            }
+            if (v16) {
+#pragma unroll
+                for (int q = 0; q < 16; ++q)
+                    if (q < vw_lane)
+                        reinterpret_cast<uint2 *>(lo_p + kATStVm)[lane + 32 * q] = vm16[q];
+            }
+            __syncwarp();  // the lanes' stores precede lane 0's arrival (release)
         }
         if (lane == 0)
             mbar_arrive_expect_tx(bar(AT_FILL0 + s), bytes);
@@ -123,9 +171,11 @@ __device__ __forceinline__ void at_load(const AttnArgs &a, const AttnMaps &m, in
         if (lane == 0) {
             const int rk = (int)(rowK + t0 + 64 * rank), rv = (int)(rowV + t0);
             tma_load_2d(klo(s) + kATStKc, &m.kc, fill, 0, rk);
-            tma_load_2d(klo(s) + kATStKm, &m.km, fill, 0, rk);
+            if (!k16)
+                tma_load_2d(klo(s) + kATStKm, &m.km, fill, 0, rk);
             tma_load_2d(klo(s) + kATStVc, &m.vc, fill, vc_x, rv);
-            tma_load_2d(klo(s) + kATStVm, &m.vm, fill, vm_x, rv);
+            if (!v16)
+                tma_load_2d(klo(s) + kATStVm, &m.vm, fill, vm_x, rv);
         }
         tma_gather4(khi(s) + (uint32_t)(lane >> 4) * 8192u + (uint32_t)(lane & 15) * 512u, &m.kcent, fill,
                     (lane >> 4) * 64, kr[0], kr[1], kr[2], kr[3]);
@@ -137,6 +187,39 @@ __device__ __forceinline__ void at_load(const AttnArgs &a, const AttnMaps &m, in
         uint32_t spins = 0;
         while (!mbar_try_wait(bar(AT_FILL0 + i % kAPStages), (uint32_t)((i / kAPStages) & 1)) && ++spins < kSpinLimit) {
         }
+    }
+}
+
+// Code words and per-unit {s, z} of 4 units from the staging slots: binary32
+// pairs (as ap_read_stage) or, with compact metadata, binary16 pairs widened.
+template <int BITS>
+__device__ __forceinline__ void at_read_stage(const uint8_t *stage_cw, const uint8_t *stage_sz, int G, bool meta16,
+                                              uint32_t *cw, float2 *sz)
+{
+    if (!meta16) {
+        ap_read_stage<BITS>(stage_cw, stage_sz, G, cw, sz);
+        return;
+    }
+    if (BITS == 2) {
+        const uint2 w = *reinterpret_cast<const uint2 *>(stage_cw);
+        cw[0] = w.x & 0xffffu;
+        cw[1] = w.x >> 16;
+        cw[2] = w.y & 0xffffu;
+        cw[3] = w.y >> 16;
+    } else {
+        const uint4 w = *reinterpret_cast<const uint4 *>(stage_cw);
+        cw[0] = w.x;
+        cw[1] = w.y;
+        cw[2] = w.z;
+        cw[3] = w.w;
+    }
+    if (G == 16) {
+        const uint2 m = *reinterpret_cast<const uint2 *>(stage_sz);
+        sz[0] = sz[1] = make_float2(f16_widen(m.x), f16_widen(m.x >> 16));
+        sz[2] = sz[3] = make_float2(f16_widen(m.y), f16_widen(m.y >> 16));
+    } else {
+        const uint32_t m = *reinterpret_cast<const uint32_t *>(stage_sz);
+        sz[0] = sz[1] = sz[2] = sz[3] = make_float2(f16_widen(m), f16_widen(m >> 16));
     }
 }
 
@@ -164,12 +247,21 @@ __device__ __forceinline__ void at_produce(const AttnArgs &a, uint32_t rank, int
         koff[uu] = sw128_unit_offset(krow, 4 * kq + uu, 64);
         voff[uu] = sw128_unit_offset(vrow, 4 * vh + uu, 128);
     }
-    const uint32_t kmRow = (uint32_t)(128 / Gk) * 8u;
+    const bool k16 = a.k.meta16 != 0, v16 = a.v.meta16 != 0;
     const uint32_t kcw_off = kATStKc + krow * 16u * BK + (uint32_t)kq * 4u * BK;
-    const uint32_t ksz_off = kATStKm + krow * kmRow + (uint32_t)(Gk == 16 ? 16 * kq : Gk == 32 ? 8 * kq : 8 * (kq >> 1));
     const uint32_t vcw_off = kATStVc + vrow * 8u * BV + (uint32_t)vh * 4u * BV;
-    const uint32_t vsz_off = kATStVm + vrow * (uint32_t)at_vm_row_bytes(Gv) +
-                             (uint32_t)(Gv == 16 ? 16 * vh : Gv == 32 ? 8 * vh : 8 * (int)rank);
+    uint32_t ksz_off, vsz_off;
+    if (k16)  // whole binary16 rows of 4 (128/G) bytes; this thread's groups
+        ksz_off = kATStKm + krow * (uint32_t)(4 * (128 / Gk)) + (uint32_t)(4 * ((32 * kq) / Gk));
+    else
+        ksz_off = kATStKm + krow * (uint32_t)(128 / Gk) * 8u +
+                  (uint32_t)(Gk == 16 ? 16 * kq : Gk == 32 ? 8 * kq : 8 * (kq >> 1));
+    if (v16)  // whole rows; the groups of channels 64 rank + 32 vh ..
+        vsz_off = kATStVm + vrow * (uint32_t)(4 * (128 / Gv)) +
+                  (uint32_t)(4 * ((64 * (int)rank + 32 * vh) / Gv));
+    else
+        vsz_off = kATStVm + vrow * (uint32_t)at_vm_row_bytes(Gv) +
+                  (uint32_t)(Gv == 16 ? 16 * vh : Gv == 32 ? 8 * vh : 8 * (int)rank);
     for (int i = 0; i < ntiles; ++i) {
         const int s = i % kAPStages;
         const bool filled = ap_wait(bar(AT_FILL0 + s), (uint32_t)((i / kAPStages) & 1), abort_flag);
@@ -178,8 +270,8 @@ __device__ __forceinline__ void at_produce(const AttnArgs &a, uint32_t rank, int
         float2 ksz[4], vsz[4];
         const uint8_t *lo = klo(s);
         if (filled) {
-            ap_read_stage<BK>(lo + kcw_off, lo + ksz_off, Gk, kcw, ksz);
-            ap_read_stage<BV>(lo + vcw_off, lo + vsz_off, Gv, vcw, vsz);
+            at_read_stage<BK>(lo + kcw_off, lo + ksz_off, Gk, k16, kcw, ksz);
+            at_read_stage<BV>(lo + vcw_off, lo + vsz_off, Gv, v16, vcw, vsz);
         }
         // every staged word is in registers (the K lo writes below overwrite
         // them); all producers arrive, and all leave if any wait gave up

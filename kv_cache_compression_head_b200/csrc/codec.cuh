@@ -71,6 +71,84 @@ __device__ __forceinline__ uint32_t quant_code(float r, const GroupQ &g, int bit
     return (uint32_t)v;
 }
 
+// binary32 -> binary16 bits: round to nearest, ties to even, saturating at
+// the largest finite value (cvt .satfinite); and back (exact).
+__device__ __forceinline__ uint16_t f16_round_sat(float f)
+{
+    uint32_t r;
+    asm("cvt.rn.satfinite.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(0.0f), "f"(f));
+    return (uint16_t)(r & 0xffffu);
+}
+
+__device__ __forceinline__ float f16_widen(uint32_t h)
+{
+    float f;
+    asm("{\n\t.reg .b16 t;\n\tcvt.u16.u32 t, %1;\n\tcvt.f32.f16 %0, t;\n\t}" : "=f"(f) : "r"(h & 0xffffu));
+    return f;
+}
+
+// Eq. 1 parameters with compact 16-bit {s, z}: s rounded to binary16, 1/s and
+// z formed from the rounded scale, z rounded to binary16; the returned s and
+// z are the stored values widened, and *packed = s16 | z16 << 16.  A group
+// whose scale rounds to zero is stored as degenerate.
+__device__ __forceinline__ GroupQ group_params16(float mn, float mx, int bits, uint32_t *packed)
+{
+    const float qmax = (float)((1 << bits) - 1);
+    GroupQ g;
+    g.degenerate = true;
+    g.inv = 0.0f;
+    float s = 0.0f;
+    if (mx != mn)
+        s = __fdiv_rn(__fsub_rn(mx, mn), qmax);
+    const uint16_t sh = f16_round_sat(s);
+    if (mx == mn || !(s >= FLT_MIN) || (sh & 0x7fffu) == 0u) {
+        if (mn == 0.0f) {
+            g.s = 0.0f;
+            g.z = 0.0f;
+            *packed = 0u;
+        } else {
+            const uint16_t ah = f16_round_sat(fabsf(mn));
+            const uint16_t zh = (mn > 0.0f) ? 0xbc00u : 0x3c00u;
+            g.s = f16_widen(ah);
+            g.z = (mn > 0.0f) ? -1.0f : 1.0f;
+            *packed = (uint32_t)ah | ((uint32_t)zh << 16);
+        }
+        return g;
+    }
+    g.degenerate = false;
+    g.s = f16_widen(sh);
+    g.inv = __fdiv_rn(1.0f, g.s);
+    const uint16_t zh = f16_round_sat(rintf(__fmul_rn(-mn, g.inv)));
+    g.z = f16_widen(zh);
+    *packed = (uint32_t)sh | ((uint32_t)zh << 16);
+    return g;
+}
+
+// Eq. 1 parameters of a group in the storage format (meta16: compact
+// 16-bit {s, z}), stored at group index g of this token-head's meta row.
+__device__ __forceinline__ GroupQ group_params_store(float mn, float mx, int bits, bool meta16, void *meta_row, int g)
+{
+    if (meta16) {
+        uint32_t packed;
+        const GroupQ gq = group_params16(mn, mx, bits, &packed);
+        static_cast<uint32_t *>(meta_row)[g] = packed;
+        return gq;
+    }
+    const GroupQ gq = group_params(mn, mx, bits);
+    static_cast<float2 *>(meta_row)[g] = make_float2(gq.s, gq.z);
+    return gq;
+}
+
+// {s, z} of group g of a meta row in either storage format, as binary32.
+__device__ __forceinline__ float2 load_sz(const void *meta_row, int g, bool meta16)
+{
+    if (meta16) {
+        const uint32_t w = static_cast<const uint32_t *>(meta_row)[g];
+        return make_float2(f16_widen(w), f16_widen(w >> 16));
+    }
+    return static_cast<const float2 *>(meta_row)[g];
+}
+
 // Eq. 1 codes of a group whose every |r * inv| is below 2^22 (checked once
 // per group), without the conversion unit: t + 1.5 2^23 rounds t to the
 // nearest integer, ties to even -- rint(t) -- in the low significand bits, so
@@ -151,7 +229,7 @@ __device__ __forceinline__ void load_bf16x8(const uint16_t *p, float *out)
 // channels the Eq. 1 parameters, then packed codes (low bits first) and the
 // {s, z} pairs.  codes_row must be 16-byte aligned (D*BITS/8 is 16, 32 or 64).
 template <int D, int BITS, int G>
-__device__ __forceinline__ void encode_residual_row(const float *r, uint8_t *codes_row, float2 *meta_row)
+__device__ __forceinline__ void encode_residual_row(const float *r, uint8_t *codes_row, void *meta_row, bool meta16)
 {
     constexpr int kWords = D * BITS / 32;
     uint32_t words[kWords];
@@ -166,8 +244,7 @@ __device__ __forceinline__ void encode_residual_row(const float *r, uint8_t *cod
             if (r[c] < mn) mn = r[c];
             if (r[c] > mx) mx = r[c];
         }
-        const GroupQ gq = group_params(mn, mx, BITS);
-        meta_row[g] = make_float2(gq.s, gq.z);
+        const GroupQ gq = group_params_store(mn, mx, BITS, meta16, meta_row, g);
         quant_group_into<G, BITS>(r + g * G, gq, mn, mx, words, g * G);
     }
     uint4 *dst = reinterpret_cast<uint4 *>(codes_row);
@@ -195,8 +272,9 @@ struct EncodeArgs {
     const uint16_t *cent;  // [H][C][D] bf16
     uint16_t *idx;         // [H][T]
     uint8_t *codes;        // [H][T][D*bits/8] (may be null when assign_only)
-    float *meta;           // [H][T][D/G][2]
+    void *meta;            // [H][T][D/G][2] float, or binary16 when meta16
     int assign_only;
+    int meta16;
 };
 
 template <int D, int BITS, int G>
@@ -266,7 +344,7 @@ __global__ void __launch_bounds__(kDirectTokens) encode_direct_kernel(EncodeArgs
     }
     const int64_t th = (int64_t)h * a.T + t;
     encode_residual_row<D, BITS, G>(xr, a.codes + th * (D * BITS / 8),
-                                    reinterpret_cast<float2 *>(a.meta) + th * (D / G));
+                                    static_cast<uint8_t *>(a.meta) + th * (D / G) * (a.meta16 ? 4 : 8), a.meta16 != 0);
 }
 
 // ---------------------------------------------------------------------------
@@ -276,7 +354,7 @@ struct DecodeArgs {
     const uint16_t *cent;
     const uint16_t *idx;
     const uint8_t *codes;
-    const float *meta;
+    const void *meta;
     int64_t T;
     int H;
     int D;
@@ -285,6 +363,7 @@ struct DecodeArgs {
     int G;
     void *out;
     int out_bf16;
+    int meta16;
 };
 
 // One block per (tile of 256 / (D/8) tokens, head); thread = 8 channels of
@@ -307,7 +386,8 @@ __global__ void __launch_bounds__(256) decode_kernel(DecodeArgs a)
         j = 0;
     }
     const int c0 = u * 8;
-    const float2 sz = reinterpret_cast<const float2 *>(a.meta)[th * (D / a.G) + c0 / a.G];
+    const float2 sz = load_sz(static_cast<const uint8_t *>(a.meta) + th * (D / a.G) * (a.meta16 ? 4 : 8), c0 / a.G,
+                              a.meta16 != 0);
     uint32_t cw;
     if (a.bits == 2)
         cw = *reinterpret_cast<const uint16_t *>(a.codes + th * (D / 4) + c0 / 4);

@@ -65,8 +65,9 @@ struct FilterArgs {
     const uint16_t *cent;
     uint16_t *idx;
     uint8_t *codes;
-    float *meta;
+    void *meta;        // [H][T][d/G][2] float, or binary16 when meta16
     int assign_only;
+    int meta16;
     float kappa;       // k of the certified bound (see above)
 };
 
@@ -140,7 +141,8 @@ __device__ __forceinline__ float spec_distance_smem(const uint8_t *sX, const uin
 // of a zero extreme, for which the group is rescanned in order.
 template <int CH, int BITS, int G>
 __device__ __forceinline__ void encode_residual_smem(const uint8_t *sX, const uint8_t *sMu, int Cpad, int row,
-                                                     int best, int half, uint8_t *codes_dst, float2 *meta_dst)
+                                                     int best, int half, uint8_t *codes_dst, void *meta_dst,
+                                                     bool meta16)
 {
     constexpr int kPerWord = 32 / BITS;
     constexpr int kWords = CH * BITS / 32;
@@ -209,12 +211,10 @@ __device__ __forceinline__ void encode_residual_smem(const uint8_t *sX, const ui
     GroupFast gf[NG];
 #pragma unroll
     for (int g = 0; g < NG; ++g)
-        gq[g] = group_params(mn[g], mx[g], BITS);
+        gq[g] = group_params_store(mn[g], mx[g], BITS, meta16, meta_dst, g);
 #pragma unroll
-    for (int g = 0; g < NG; ++g) {
+    for (int g = 0; g < NG; ++g)
         gf[g] = group_fast(gq[g], mn[g], mx[g]);
-        meta_dst[g] = make_float2(gq[g].s, gq[g].z);
-    }
     // (3) codes
     uint32_t words[kWords];
 #pragma unroll
@@ -674,7 +674,8 @@ __global__ void __launch_bounds__(kFltThreads, 1)
                         if (!a.assign_only)
                             encode_residual_smem<CH, BITS, G>(
                                 sX, sMu, Cpad, row, best, half, a.codes + th * (D * BITS / 8) + half * (CH * BITS / 8),
-                                reinterpret_cast<float2 *>(a.meta) + th * (D / G) + half * (CH / G));
+                                static_cast<uint8_t *>(a.meta) + (th * (D / G) + half * (CH / G)) * (a.meta16 ? 4 : 8),
+                                a.meta16 != 0);
                     }
                 }
                 // X stage read: the TMA may refill it

@@ -48,6 +48,10 @@ kvq_status check_desc(const kvq_codec_desc *d, bool allow_joint)
         return KVQ_ERR_INVALID_ARG;
     if (d->joint_rank > 0 && !allow_joint)
         return KVQ_ERR_UNSUPPORTED;
+    if (d->meta_format != KVQ_META_F32 && d->meta_format != KVQ_META_F16)
+        return KVQ_ERR_INVALID_ARG;
+    if (d->meta_format == KVQ_META_F16 && d->joint_rank > 0)
+        return KVQ_ERR_UNSUPPORTED;  // compact {s, z} is a per-head codec format
     const int span = d->joint_rank > 0 ? d->joint_rank : d->head_dim;
     if (d->group_size < 8 || d->group_size % 8 != 0 || span % d->group_size != 0)
         return KVQ_ERR_INVALID_ARG;
@@ -224,6 +228,7 @@ kvq_status launch_encode_filter(int D, int bits, int G, const void *x, const Enc
     a.codes = e.codes;
     a.meta = e.meta;
     a.assign_only = e.assign_only;
+    a.meta16 = e.meta16;
     a.kappa = filter_kappa(D);
     if (D == 128)
         return bits == 2 ? launch_filter_g<128, 2>(G, m, a, s) : launch_filter_g<128, 4>(G, m, a, s);
@@ -335,7 +340,7 @@ kvq_status launch_joint_decode(const JointDecArgs &a, const void *w_dec, cudaStr
 // Validates and runs the joint encoder: per-head assignment into idx, then the
 // projection + quantisation (codes/meta) and/or the binary32 coefficients.
 kvq_status joint_encode_call(const kvq_codec_desc *desc, const void *x, kvq_dtype x_dtype, int64_t T,
-                             const void *centroids, const void *w_enc, uint16_t *idx, uint8_t *codes, float *meta,
+                             const void *centroids, const void *w_enc, uint16_t *idx, uint8_t *codes, void *meta,
                              float *coef_out, cudaStream_t s)
 {
     if (x_dtype != KVQ_BF16)
@@ -377,7 +382,7 @@ kvq_status joint_encode_call(const kvq_codec_desc *desc, const void *x, kvq_dtyp
     a.bits = desc->bits;
     a.G = desc->group_size;
     a.codes = codes;
-    a.meta = meta;
+    a.meta = static_cast<float *>(meta);
     a.coef_out = coef_out;
     return launch_joint_encode(a, s);
 }
@@ -446,6 +451,7 @@ CodecView to_codec_view(const kvq_compressed_view *v)
     cv.idx = v->idx;
     cv.codes = v->codes;
     cv.meta = v->meta;
+    cv.meta16 = v->desc.meta_format == KVQ_META_F16;
     cv.T = v->num_tokens;
     cv.C = v->desc.num_centroids;
     cv.bits = v->desc.bits;
@@ -549,14 +555,17 @@ bool make_attn_maps(AttnMaps *m, const AttnArgs &a)
     const uint64_t rows = (uint64_t)a.H * (uint64_t)a.k.T;
     const CodecView &k = a.k, &v = a.v;
     const uint32_t vm_box = v.G == 64 ? 4u : (uint32_t)(64 / v.G) * 2u;
+    // compact binary16 {s, z} is read by the loader lanes: no map
+    memset(&m->km, 0, sizeof m->km);
+    memset(&m->vm, 0, sizeof m->vm);
     return encode_2d(&m->kc, CU_TENSOR_MAP_DATA_TYPE_UINT8, k.codes, 16u * k.bits, rows, 16u * k.bits,
                      16u * k.bits, 64, CU_TENSOR_MAP_SWIZZLE_NONE) &&
-           encode_2d(&m->km, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, k.meta, 2u * (128 / k.G), rows, 8u * (128 / k.G),
-                     2u * (128 / k.G), 64, CU_TENSOR_MAP_SWIZZLE_NONE) &&
+           (k.meta16 || encode_2d(&m->km, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, k.meta, 2u * (128 / k.G), rows,
+                                  8u * (128 / k.G), 2u * (128 / k.G), 64, CU_TENSOR_MAP_SWIZZLE_NONE)) &&
            encode_2d(&m->vc, CU_TENSOR_MAP_DATA_TYPE_UINT8, v.codes, 16u * v.bits, rows, 16u * v.bits,
                      8u * v.bits, 128, CU_TENSOR_MAP_SWIZZLE_NONE) &&
-           encode_2d(&m->vm, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, v.meta, 2u * (128 / v.G), rows, 8u * (128 / v.G), vm_box,
-                     128, CU_TENSOR_MAP_SWIZZLE_NONE) &&
+           (v.meta16 || encode_2d(&m->vm, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, v.meta, 2u * (128 / v.G), rows,
+                                  8u * (128 / v.G), vm_box, 128, CU_TENSOR_MAP_SWIZZLE_NONE)) &&
            encode_2d(&m->kcent, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, k.cent, 128, (uint64_t)a.H * k.C, 256, 64, 1,
                      CU_TENSOR_MAP_SWIZZLE_128B) &&
            encode_2d(&m->vcent, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, v.cent, 128, (uint64_t)a.H * v.C, 256, 64, 1,
@@ -597,6 +606,8 @@ kvq_status launch_attention_pair(const AttnArgs &a, cudaStream_t s)
             return a.v.bits == 2 ? launch_attention_tma_t<2, 2>(a, s) : launch_attention_tma_t<2, 4>(a, s);
         return a.v.bits == 2 ? launch_attention_tma_t<4, 2>(a, s) : launch_attention_tma_t<4, 4>(a, s);
     }
+    if ((a.k.meta16 || a.v.meta16) && a.t_end > a.t_begin)
+        return KVQ_ERR_UNSUPPORTED;  // only the TMA-staged kernel reads compact {s, z}
     if (a.k.bits == 2)
         return a.v.bits == 2 ? launch_attention_pair_t<2, 2, false>(a, s) : launch_attention_pair_t<2, 4, false>(a, s);
     return a.v.bits == 2 ? launch_attention_pair_t<4, 2, false>(a, s) : launch_attention_pair_t<4, 4, false>(a, s);
@@ -697,6 +708,8 @@ kvq_status check_history_pair(const kvq_compressed_view *k, const kvq_compressed
         return KVQ_ERR_INVALID_ARG;
     if (k->desc.num_heads > 65535)
         return KVQ_ERR_UNSUPPORTED;
+    if (k->desc.head_dim != 128 && (k->desc.meta_format == KVQ_META_F16 || v->desc.meta_format == KVQ_META_F16))
+        return KVQ_ERR_UNSUPPORTED;  // compact {s, z} is read by the d = 128 kernel only
     return KVQ_OK;
 }
 
@@ -752,7 +765,7 @@ kvq_status kvq_encoded_sizes(const kvq_codec_desc *desc, int64_t T, size_t *idx_
         mb = (size_t)T * (r / desc->group_size) * 8;
     } else {
         cb = H * (size_t)T * d * desc->bits / 8;
-        mb = H * (size_t)T * (d / desc->group_size) * 8;
+        mb = H * (size_t)T * (d / desc->group_size) * (desc->meta_format == KVQ_META_F16 ? 4 : 8);
     }
     if (idx_bytes) *idx_bytes = ib;
     if (code_bytes) *code_bytes = cb;
@@ -929,7 +942,7 @@ kvq_status kvq_fit_centroids_static(const kvq_codec_desc *desc, const void *x, k
 }
 
 kvq_status kvq_encode(const kvq_codec_desc *desc, const void *x, kvq_dtype x_dtype, int64_t T,
-                      const void *centroids, const void *w_enc, uint16_t *idx, uint8_t *codes, float *meta,
+                      const void *centroids, const void *w_enc, uint16_t *idx, uint8_t *codes, void *meta,
                       void *workspace, size_t workspace_bytes, kvq_stream_t stream)
 {
     (void)workspace;
@@ -967,6 +980,7 @@ kvq_status kvq_encode(const kvq_codec_desc *desc, const void *x, kvq_dtype x_dty
     e.codes = codes;
     e.meta = meta;
     e.assign_only = 0;
+    e.meta16 = desc->meta_format == KVQ_META_F16;
     return launch_encode(desc->head_dim, e, reinterpret_cast<cudaStream_t>(stream));
 }
 
@@ -1014,7 +1028,7 @@ kvq_status kvq_decode(const kvq_compressed_view *view, void *x_out, kvq_dtype ou
         j.cent = static_cast<const uint16_t *>(view->centroids);
         j.idx = view->idx;
         j.codes = view->codes;
-        j.meta = view->meta;
+        j.meta = static_cast<const float *>(view->meta);
         j.T = view->num_tokens;
         j.H = view->desc.num_heads;
         j.D = view->desc.head_dim;
@@ -1039,6 +1053,7 @@ kvq_status kvq_decode(const kvq_compressed_view *view, void *x_out, kvq_dtype ou
     a.G = view->desc.group_size;
     a.out = x_out;
     a.out_bf16 = out_dtype == KVQ_BF16;
+    a.meta16 = view->desc.meta_format == KVQ_META_F16;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     if (a.D == 128)
         decode_kernel<128><<<dim3((unsigned)ceil_div(a.T, 256 / 16), (unsigned)a.H), 256, 0, s>>>(a);

@@ -30,6 +30,9 @@ KVQ_ERR_DEVICE_TIMEOUT = 6
 KVQ_F32 = 0
 KVQ_BF16 = 1
 
+KVQ_META_F32 = 0
+KVQ_META_F16 = 1
+
 KVQ_OP_FIT = 0
 KVQ_OP_ENCODE = 1
 KVQ_OP_DECODE = 2
@@ -52,7 +55,8 @@ class KvqError(RuntimeError):
 
 class CodecDesc(ctypes.Structure):
     _fields_ = [("num_heads", ctypes.c_int32), ("head_dim", ctypes.c_int32), ("num_centroids", ctypes.c_int32),
-                ("bits", ctypes.c_int32), ("group_size", ctypes.c_int32), ("joint_rank", ctypes.c_int32)]
+                ("bits", ctypes.c_int32), ("group_size", ctypes.c_int32), ("joint_rank", ctypes.c_int32),
+                ("meta_format", ctypes.c_int32)]
 
 
 class CompressedView(ctypes.Structure):
@@ -173,7 +177,10 @@ def _want_encoded(what: str, codec: "Codec", num_tokens: int, idx, codes, meta) 
     ib, cb, mb = encoded_sizes(codec, num_tokens)
     _want(f"{what} idx", idx, _IDX_DTYPES, numel=ib // 2)
     _want(f"{what} codes", codes, torch.uint8, numel=cb)
-    _want(f"{what} meta", meta, torch.float32, numel=mb // 4)
+    if codec.meta_format == KVQ_META_F16:
+        _want(f"{what} meta", meta, torch.float16, numel=mb // 2)
+    else:
+        _want(f"{what} meta", meta, torch.float32, numel=mb // 4)
 
 
 def _want_workspace(what: str, ws: Optional[torch.Tensor]) -> None:
@@ -206,7 +213,8 @@ def _want_attention_io(what: str, q: torch.Tensor, H: int, d: int, o_out, lse_ou
 
 @dataclasses.dataclass
 class Codec:
-    """One K or V branch: heads, head dim, centroids, bits, group size, joint rank."""
+    """One K or V branch: heads, head dim, centroids, bits, group size, joint
+    rank, and the storage of {scale, zero} (KVQ_META_F32 or KVQ_META_F16)."""
 
     num_heads: int
     head_dim: int
@@ -214,10 +222,11 @@ class Codec:
     bits: int
     group_size: int
     joint_rank: int = 0
+    meta_format: int = KVQ_META_F32
 
     def c(self) -> CodecDesc:
         return CodecDesc(self.num_heads, self.head_dim, self.num_centroids, self.bits, self.group_size,
-                         self.joint_rank)
+                         self.joint_rank, self.meta_format)
 
 
 @dataclasses.dataclass
@@ -229,7 +238,7 @@ class Compressed:
     centroids: torch.Tensor  # [H][C][d] bf16
     idx: torch.Tensor        # [H][T] int16 (uint16 bits)
     codes: torch.Tensor      # uint8
-    meta: torch.Tensor       # float32
+    meta: torch.Tensor       # float32, or float16 with compact {s, z}
     w_dec: Optional[torch.Tensor] = None
 
     def view(self) -> CompressedView:
@@ -258,7 +267,10 @@ def alloc_encoded(codec: Codec, num_tokens: int, device) -> Tuple[torch.Tensor, 
     ib, cb, mb = encoded_sizes(codec, num_tokens)
     idx = torch.empty(ib // 2, dtype=torch.int16, device=device)
     codes = torch.empty(cb, dtype=torch.uint8, device=device)
-    meta = torch.empty(mb // 4, dtype=torch.float32, device=device)
+    if codec.meta_format == KVQ_META_F16:
+        meta = torch.empty(mb // 2, dtype=torch.float16, device=device)
+    else:
+        meta = torch.empty(mb // 4, dtype=torch.float32, device=device)
     return idx, codes, meta
 
 

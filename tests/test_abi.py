@@ -280,3 +280,31 @@ def test_binding_refuses_to_load_without_the_library(tmp_path):
                        capture_output=True, text=True, env={**os.environ, "PYTHONPATH": str(tmp_path)})
     assert r.returncode != 0
     assert "ImportError" in r.stderr and "libkvq.so not built" in r.stderr
+
+
+def test_compact_meta_sizes_and_refusals(K):
+    """Compact 16-bit {s, z}: 4 metadata bytes per group (TempoKV, Table 1:
+    b + 1 bits per value at G = 32, i.e. 5.33x for INT2 and 3.20x for INT4
+    against bf16); an unknown format is an invalid argument; the joint codec
+    and the d = 64 attention refuse the compact format before any launch."""
+    import ctypes
+
+    for bits, ratio in ((2, 16 / 3), (4, 16 / 5)):
+        d16 = K.CodecDesc(12, 128, 256, bits, 32, 0, K.KVQ_META_F16)
+        ib, cb, mb = ctypes.c_size_t(), ctypes.c_size_t(), ctypes.c_size_t()
+        assert K._lib.kvq_encoded_sizes(ctypes.byref(d16), 1000, ctypes.byref(ib), ctypes.byref(cb),
+                                        ctypes.byref(mb)) == K.KVQ_OK
+        assert mb.value == 12 * 1000 * (128 // 32) * 4
+        values = 12 * 1000 * 128
+        assert abs(16 * values / ((cb.value + mb.value) * 8) - ratio) < 1e-12
+    bad = K.CodecDesc(12, 128, 256, 2, 32, 0, 2)
+    sz = ctypes.c_size_t()
+    assert K._lib.kvq_encoded_sizes(ctypes.byref(bad), 10, None, None, None) == K.KVQ_ERR_INVALID_ARG
+    joint16 = K.CodecDesc(12, 128, 256, 4, 32, 192, K.KVQ_META_F16)
+    assert K._lib.kvq_encoded_sizes(ctypes.byref(joint16), 10, None, None, None) == K.KVQ_ERR_UNSUPPORTED
+    A = 1 << 20  # a 16-byte aligned fake address: validation fails before any use
+    v64 = K.CompressedView(K.CodecDesc(2, 64, 16, 2, 32, 0, K.KVQ_META_F16), 100, A, A, A, A, None)
+    o = ctypes.c_void_p(A)
+    assert K._lib.kvq_attention_lse(A, 10, ctypes.byref(v64), ctypes.byref(v64), 0, 100, ctypes.c_float(0.0), o,
+                                    K.KVQ_F32, A, None, 0, None) == K.KVQ_ERR_UNSUPPORTED
+    del sz

@@ -218,6 +218,34 @@ KVQ_API kvq_status kvq_encode(const kvq_codec_desc *desc, const void *x, kvq_dty
                       void *workspace, size_t workspace_bytes, kvq_stream_t stream);
 
 /*
+ * Encode one K history with QuantWM's query-sensitive centre selection
+ * (QSAC; QuantWM: Temporally Consistent 2-Bit KV Cache Quantization for Video
+ * World Models, Sec. 4.1).  Per token-head:
+ *   d_j   = sum_c w_c (x_c - mu_jc)^2 in binary32, each operation rounded, in
+ *           channel order; the M smallest by (d_j, j) are the candidates;
+ *   score = sum over groups g of W_g R_g^2 (binary32, group order), W_g the
+ *           sum of the group's w_c in channel order, R_g = max - min of the
+ *           group's residual x - mu_j (the Widrow factor 1/(12 (2^b - 1)^2)
+ *           is common to all candidates and dropped);
+ *   idx   = the candidate with the lowest score, ties to the better-ranked;
+ *   codes and {s, z} of x - mu[idx] exactly as kvq_encode writes them.
+ *   w       [H][d] binary32 channel weights: the diagonal of the head's
+ *           second-moment matrix of the queries seen so far (all ones
+ *           before any query; QuantWM, cold start); device pointer, 16-byte
+ *           aligned.  Computing them is the caller's (they come from the
+ *           model's queries, not from this history).
+ *   M       1 .. 8 candidates (QuantWM, Table 11: M = 4); M = 1 is the plain
+ *           nearest centre under the weighted distance.
+ * Per-head codec only (joint_rank = 0) with binary32 {s, z} (meta_format
+ * KVQ_META_F32; KVQ_ERR_UNSUPPORTED otherwise), d in {64, 128}; x float or
+ * bf16; outputs and other requirements as for kvq_encode.  Runs on CUDA cores with
+ * the specified arithmetic, so idx, codes and {s, z} are bit-exact.
+ */
+KVQ_API kvq_status kvq_encode_qsac(const kvq_codec_desc *desc, const void *x, kvq_dtype x_dtype, int64_t num_tokens,
+                                   const void *centroids, const float *w, int32_t M, uint16_t *idx, uint8_t *codes,
+                                   void *meta, kvq_stream_t stream);
+
+/*
  * Joint codec only: the binary32 coefficient matrix c = R W_enc [T][r] that
  * kvq_encode quantises, and idx [H][T].  Lets a caller quantise the same
  * coefficients independently: they are bit-identical to the ones kvq_encode
@@ -269,6 +297,46 @@ KVQ_API kvq_status kvq_attention_lse(const void *q, int64_t num_queries, const k
                              const kvq_compressed_view *v, int64_t t_begin, int64_t t_end, float softmax_scale,
                              void *o_out, kvq_dtype o_dtype, float *lse_out, void *workspace,
                              size_t workspace_bytes, kvq_stream_t stream);
+
+/*
+ * PSAC coefficients of a compressed K history (QuantWM: Temporally Consistent
+ * 2-Bit KV Cache Quantization for Video World Models, Sec. 4.2, principal
+ * query-subspace attention correction; rank 8 as in its Table 9):
+ *   C[h][t] = (k_t - k^_t) U_h   for every token t < num_tokens, head h,
+ * k the original keys, k^ their reconstruction from `k` (the value
+ * kvq_decode writes in binary32), U_h [d][8] the head's basis: the leading
+ * eigenvectors of its query second-moment matrix, computed by the caller
+ * from the model's queries.  Per token-head: e_c = k_c - k^_c in binary32,
+ * each C_r accumulated by binary32 FMAs in channel order.
+ *   k       per-head codec view (joint_rank = 0; KVQ_ERR_UNSUPPORTED
+ *           otherwise), d in {64, 128}, either {s, z} format;
+ *   x       [T][H][d] original keys, float or bf16 (x_dtype), 16-byte aligned;
+ *   U       [H][d][8] float, 16-byte aligned;  rank must be 8
+ *           (KVQ_ERR_UNSUPPORTED otherwise);
+ *   coef_out [H][T][8] float, 16-byte aligned (caller-owned, 32 bytes per
+ *           token-head: the stored cost of the correction).
+ * An index past C sets KVQ_ERR_INVALID_ARG in the device status word (centre
+ * 0 is used).  T = 0 returns KVQ_OK without touching memory.
+ */
+KVQ_API kvq_status kvq_psac_coefficients(const kvq_compressed_view *k, const void *x, kvq_dtype x_dtype,
+                                         const float *U, int32_t rank, float *coef_out, kvq_stream_t stream);
+
+/*
+ * kvq_attention_lse with PSAC's corrected logits (QuantWM, Sec. 4.2):
+ *   s_ij = scale (q_i . k^_j + (q_i U_h) . C_j) = scale q_i . (k^_j + U_h C_j),
+ * evaluated as attention over the corrected keys: the kernel adds
+ * sum_r U_h[c][r] C_j[r] (binary32) to every rebuilt key value before it
+ * splits the key into its bf16 high and low parts; everything else is as in
+ * kvq_attention_lse.  U [H][128][8] and coef [H][T][8] float (as written by
+ * kvq_psac_coefficients for the same K history), both 16-byte aligned; rank
+ * must be 8 and d 128 (KVQ_ERR_UNSUPPORTED otherwise, also when H T or H C
+ * reaches 2^31).  Workspace as for kvq_attention_lse.
+ */
+KVQ_API kvq_status kvq_attention_psac_lse(const void *q, int64_t num_queries, const kvq_compressed_view *k,
+                                          const kvq_compressed_view *v, const float *U, const float *coef,
+                                          int32_t rank, int64_t t_begin, int64_t t_end, float softmax_scale,
+                                          void *o_out, kvq_dtype o_dtype, float *lse_out, void *workspace,
+                                          size_t workspace_bytes, kvq_stream_t stream);
 
 /*
  * Dense-mode attention: the same computation as kvq_attention_lse over keys

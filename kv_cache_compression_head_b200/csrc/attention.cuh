@@ -42,6 +42,8 @@ struct AttnArgs {
     float *lse_out;  // [H][Tq]
     int nsplit;      // > 1: blockIdx.z selects a sub-range; o_out / lse_out
                      // then hold nsplit float partials [z][Tq][H][D], [z][H][Tq]
+    const float *psac_u;     // PSAC: basis [H][D][8] (NULL: no correction)
+    const float *psac_coef;  // PSAC: coefficients [H][T][8] of the K history
 };
 
 }  // namespace kvq

@@ -32,6 +32,12 @@
 // units of K and V in place and publish both behind one proxy fence.  They have no copies of
 // their own in flight, so the fence does not wait on memory.
 //
+// PSAC (QuantWM, Sec. 4.2; rank 8, Table 9): with a basis U_h [d][8] and
+// per-key coefficients C [H][T][8], the logits are those of the corrected
+// keys k^ + U_h C; the loader stages each tile's coefficient rows with a
+// tiled load beside the codes, and the producers add U_h C (binary32, U_h
+// resident in shared memory) to every rebuilt K value before the hi/lo split.
+//
 // Barriers (parity = use count & 1): those of attention_pair.cuh plus
 // fill[s] (1 arrival with the stage's byte count, completed by the TMA
 // traffic; local to each CTA).  The loader waits kfree[s] and vfree[s] (the
@@ -62,10 +68,20 @@ struct AttnMaps {
     CUtensorMap vm;     // V {s, z}  [H T][2 128/G_V] f32,   box {half row (>= 16 B), 128}
     CUtensorMap kcent;  // K centres [H C_K][128] bf16,      box {64, 1}, 128-byte swizzle
     CUtensorMap vcent;  // V centres [H C_V][128] bf16,      box {64, 1}, 128-byte swizzle
+    CUtensorMap kpc;    // PSAC coefficients [H T][8] f32,   box {8, 64} (when used)
 };
 
 // Offsets of the staged words inside a stage's K lo slot (16 KB).
 constexpr uint32_t kATStKc = 0, kATStKm = 4096, kATStVc = 8192, kATStVm = 12288;
+
+// Shared memory beyond the pair kernel's layout: the PSAC basis of the head
+// [128][8] binary32 and one coefficient tile [64][8] per stage.
+struct ATSmem {
+    static constexpr uint32_t offU = APSmem::kBytes;
+    static constexpr uint32_t offC = offU + 128 * 8 * 4;
+    static constexpr uint32_t kBytes = offC + kAPStages * 64 * 8 * 4;
+    static constexpr uint32_t kLaunchBytes = kBytes + 1024;
+};
 
 enum { AT_FILL0 = P_COUNT, AT_COUNT = AT_FILL0 + kAPStages };
 
@@ -85,8 +101,9 @@ __device__ __forceinline__ void at_load(const AttnArgs &a, const AttnMaps &m, in
     auto vst = [&](int s) { return smem_u32(smem + L::offV + (uint32_t)s * L::kV); };
     const int Gk = a.k.G, Gv = a.v.G;
     const bool k16 = a.k.meta16 != 0, v16 = a.v.meta16 != 0;
+    const bool psac = a.psac_coef != nullptr;
     const uint32_t bytes = 16384u + 16384u + 64u * 16u * BK + (k16 ? 0u : 64u * (uint32_t)(128 / Gk) * 8u) +
-                           128u * 8u * BV + (v16 ? 0u : 128u * (uint32_t)at_vm_row_bytes(Gv));
+                           128u * 8u * BV + (v16 ? 0u : 128u * (uint32_t)at_vm_row_bytes(Gv)) + (psac ? 2048u : 0u);
     // compact {s, z}: whole rows of 4 (128/G) bytes, in 8-byte words
     const int kw_row = (128 / Gk) / 2, vw_row = (128 / Gv) / 2;  // words per row
     const int kw_lane = 64 * kw_row / 32, vw_lane = 128 * vw_row / 32;
@@ -176,6 +193,8 @@ __device__ __forceinline__ void at_load(const AttnArgs &a, const AttnMaps &m, in
             tma_load_2d(klo(s) + kATStVc, &m.vc, fill, vc_x, rv);
             if (!v16)
                 tma_load_2d(klo(s) + kATStVm, &m.vm, fill, vm_x, rv);
+            if (psac)
+                tma_load_2d(smem_u32(smem + ATSmem::offC + (uint32_t)s * 2048u), &m.kpc, fill, 0, rk);
         }
         tma_gather4(khi(s) + (uint32_t)(lane >> 4) * 8192u + (uint32_t)(lane & 15) * 512u, &m.kcent, fill,
                     (lane >> 4) * 64, kr[0], kr[1], kr[2], kr[3]);
@@ -220,6 +239,61 @@ __device__ __forceinline__ void at_read_stage(const uint8_t *stage_cw, const uin
     } else {
         const uint32_t m = *reinterpret_cast<const uint32_t *>(stage_sz);
         sz[0] = sz[1] = sz[2] = sz[3] = make_float2(f16_widen(m), f16_widen(m >> 16));
+    }
+}
+
+// K rebuild with the PSAC correction: as ap_rebuild<BITS, true>, with
+// sum_r U[c][r] C[r] added to each value (binary32) before the hi/lo split.
+// Units uu cover channels ch0 + 8 uu .. + 7.
+template <int BITS>
+__device__ __forceinline__ void at_rebuild_k_psac(uint8_t *tile, uint8_t *lo, const uint32_t *off, const uint32_t *cw,
+                                                  const float2 *sz, bool valid, const float *sU, const float *Crow,
+                                                  int ch0)
+{
+    constexpr float kTwoB = (float)(1 << BITS);
+    const float4 c0 = reinterpret_cast<const float4 *>(Crow)[0], c1 = reinterpret_cast<const float4 *>(Crow)[1];
+#pragma unroll
+    for (int uu = 0; uu < 4; ++uu) {
+        uint4 *dst = reinterpret_cast<uint4 *>(tile + off[uu]);
+        if (!valid) {
+            *dst = make_uint4(0, 0, 0, 0);
+            *reinterpret_cast<uint4 *>(lo + off[uu]) = make_uint4(0, 0, 0, 0);
+            continue;
+        }
+        const uint4 mw = *dst;
+        const float sc = kTwoB * sz[uu].x;
+        const float nb = -__fmul_rn(kTwoB + sz[uu].y, sz[uu].x);
+        const uint32_t ma[4] = {mw.x, mw.y, mw.z, mw.w};
+        uint32_t hi[4], lw[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            const float2 f = make_float2(code_as_unit_float<BITS>(cw[uu], 2 * k),
+                                         code_as_unit_float<BITS>(cw[uu], 2 * k + 1));
+            const float2 b = add2(make_float2(bf16_lo(ma[k]), bf16_hi(ma[k])), make_float2(nb, nb));
+            float2 val = fma2(f, make_float2(sc, sc), b);
+            float corr[2];
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+                const float *u = sU + (ch0 + 8 * uu + 2 * k + e) * 8;
+                const float4 u0 = reinterpret_cast<const float4 *>(u)[0], u1 = reinterpret_cast<const float4 *>(u)[1];
+                float acc = u0.x * c0.x;
+                acc = fmaf(u0.y, c0.y, acc);
+                acc = fmaf(u0.z, c0.z, acc);
+                acc = fmaf(u0.w, c0.w, acc);
+                acc = fmaf(u1.x, c1.x, acc);
+                acc = fmaf(u1.y, c1.y, acc);
+                acc = fmaf(u1.z, c1.z, acc);
+                corr[e] = fmaf(u1.w, c1.w, acc);
+            }
+            val = add2(val, make_float2(corr[0], corr[1]));
+            const uint32_t a0 = __float_as_uint(val.x) & 0xffff0000u;
+            const uint32_t a1 = __float_as_uint(val.y) & 0xffff0000u;
+            hi[k] = __byte_perm(a0, a1, 0x7632);
+            const float2 d = sub2(val, make_float2(__uint_as_float(a0), __uint_as_float(a1)));
+            lw[k] = pack_bf16x2(d.x, d.y);
+        }
+        *dst = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+        *reinterpret_cast<uint4 *>(lo + off[uu]) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
     }
 }
 
@@ -273,11 +347,16 @@ __device__ __forceinline__ void at_produce(const AttnArgs &a, uint32_t rank, int
             at_read_stage<BK>(lo + kcw_off, lo + ksz_off, Gk, k16, kcw, ksz);
             at_read_stage<BV>(lo + vcw_off, lo + vsz_off, Gv, v16, vcw, vsz);
         }
+        const float *crow = reinterpret_cast<const float *>(smem + ATSmem::offC + (uint32_t)s * 2048u) + krow * 8;
         // every staged word is in registers (the K lo writes below overwrite
         // them); all producers arrive, and all leave if any wait gave up
         if (!named_barrier_and<5>(kAPProducers, filled))
             return;
-        ap_rebuild<BK, true>(khi(s), klo(s), koff, kcw, ksz, t0 + 64 * rank + krow < a.t_end);
+        if (a.psac_coef)
+            at_rebuild_k_psac<BK>(khi(s), klo(s), koff, kcw, ksz, t0 + 64 * rank + krow < a.t_end,
+                                  reinterpret_cast<const float *>(smem + ATSmem::offU), crow, 32 * kq);
+        else
+            ap_rebuild<BK, true>(khi(s), klo(s), koff, kcw, ksz, t0 + 64 * rank + krow < a.t_end);
         ap_rebuild<BV, false>(vst(s), nullptr, voff, vcw, vsz, t0 + vrow < a.t_end);
         // one proxy fence for both tiles (a fence costs more than a rebuild)
         fence_proxy_async_smem();
@@ -441,6 +520,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kATThreads, 1)
                 const uint4 w = valid ? __ldg(reinterpret_cast<const uint4 *>(src) + u) : make_uint4(0, 0, 0, 0);
                 *reinterpret_cast<uint4 *>(dst + sw128_unit_offset(r, u, 128)) = w;
             }
+        }
+        if (a.psac_u) {  // the head's PSAC basis; read by producers after their first named barrier
+            const float4 *src = reinterpret_cast<const float4 *>(a.psac_u + (int64_t)h * D * 8);
+            float4 *dst = reinterpret_cast<float4 *>(smem + ATSmem::offU);
+            dst[tid] = __ldg(src + tid);
         }
         ap_publish(lead(P_QREADY));
         if (ntiles > 0)

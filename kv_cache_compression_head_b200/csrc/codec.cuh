@@ -348,6 +348,166 @@ __global__ void __launch_bounds__(kDirectTokens) encode_direct_kernel(EncodeArgs
 }
 
 // ---------------------------------------------------------------------------
+// QSAC (QuantWM, Sec. 4.1): query-sensitive centre selection, exact on CUDA
+// cores.  One thread per token; a block covers 128 tokens of one head and
+// streams the head's centres through shared memory (binary32) in chunks.
+//  - weighted distance sum_c w_c ((x_c - mu_c)^2), every operation rounded
+//    separately in channel order; the M smallest by (distance, index) are
+//    kept (strict comparisons while scanning centres in index order);
+//  - score of each candidate: sum over groups of W_g R_g^2, W_g the sum of
+//    the group's w_c in channel order, R_g = max - min of the group's
+//    residual (strict scans); the lowest score wins, ties to the better-
+//    ranked candidate (QuantWM, Table 11: M = 4; the Widrow factor
+//    1 / (12 (2^b - 1)^2) is common to all candidates and dropped);
+//  - the chosen centre's residual is quantised exactly as the plain encode.
+// ---------------------------------------------------------------------------
+constexpr int kQsacMaxM = 8;
+
+struct QsacArgs {
+    EncodeArgs e;     // history, centres, outputs (assign_only unused)
+    const float *w;   // [H][D] channel weights, binary32
+    int M;            // candidates, 1 .. kQsacMaxM
+};
+
+template <int D, int BITS, int G>
+__global__ void __launch_bounds__(kDirectTokens) qsac_encode_kernel(QsacArgs q)
+{
+    const EncodeArgs &a = q.e;
+    __shared__ __align__(16) float s_mu[kDirectChunk * D];
+    __shared__ __align__(16) float s_w[D];
+    const int h = blockIdx.y;
+    const int64_t t = (int64_t)blockIdx.x * kDirectTokens + threadIdx.x;
+    const bool active = t < a.T;
+    for (int c = threadIdx.x; c < D; c += kDirectTokens)
+        s_w[c] = q.w[(int64_t)h * D + c];
+
+    float xr[D];
+    if (active) {
+#pragma unroll
+        for (int c = 0; c < D; c += 8)
+            load_x8(a.x, a.x_bf16, (t * a.H + h) * D + c, xr + c);
+    } else {
+#pragma unroll
+        for (int c = 0; c < D; ++c)
+            xr[c] = 0.0f;
+    }
+    const int m = q.M < a.C ? q.M : a.C;
+    float cd[kQsacMaxM];
+    int cand[kQsacMaxM];
+#pragma unroll
+    for (int k = 0; k < kQsacMaxM; ++k) {
+        cd[k] = INFINITY;
+        cand[k] = -1;
+    }
+    const uint16_t *cent_h = a.cent + (int64_t)h * a.C * D;
+    for (int j0 = 0; j0 < a.C; j0 += kDirectChunk) {
+        const int nj = min(kDirectChunk, a.C - j0);
+        __syncthreads();
+        for (int e = threadIdx.x * 8; e < nj * D; e += kDirectTokens * 8)
+            load_bf16x8(cent_h + (int64_t)j0 * D + e, s_mu + e);
+        __syncthreads();
+        if (active) {
+            for (int jj = 0; jj < nj; ++jj) {
+                const float4 *mu4 = reinterpret_cast<const float4 *>(s_mu + jj * D);
+                const float4 *w4 = reinterpret_cast<const float4 *>(s_w);
+                float acc = 0.0f;
+#pragma unroll
+                for (int c4 = 0; c4 < D / 4; ++c4) {
+                    const float4 mv = mu4[c4], wv = w4[c4];
+                    const float mm[4] = {mv.x, mv.y, mv.z, mv.w}, ww[4] = {wv.x, wv.y, wv.z, wv.w};
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) {
+                        const float e = __fsub_rn(xr[4 * c4 + k], mm[k]);
+                        acc = __fadd_rn(acc, __fmul_rn(ww[k], __fmul_rn(e, e)));
+                    }
+                }
+                const int j = j0 + jj;
+                // insert (acc, j) into the ascending lists (an empty slot
+                // takes any value, infinite ones included); equal distances
+                // keep the earlier (lower-index) entry first
+#pragma unroll
+                for (int k = kQsacMaxM - 1; k >= 1; --k) {
+                    if (k < m) {
+                        if (acc < cd[k - 1]) {
+                            cd[k] = cd[k - 1];
+                            cand[k] = cand[k - 1];
+                        } else if (cand[k - 1] >= 0 && (cand[k] < 0 || acc < cd[k])) {
+                            cd[k] = acc;
+                            cand[k] = j;
+                        }
+                    }
+                }
+                if (cand[0] < 0 || acc < cd[0]) {
+                    cd[0] = acc;
+                    cand[0] = j;
+                }
+            }
+        }
+    }
+    if (!active)
+        return;
+    // scores of the candidates; the group weights do not depend on the centre
+    float wg[D / G];
+#pragma unroll
+    for (int g = 0; g < D / G; ++g) {
+        float acc = 0.0f;
+#pragma unroll
+        for (int c = g * G; c < (g + 1) * G; ++c)
+            acc = __fadd_rn(acc, s_w[c]);
+        wg[g] = acc;
+    }
+    int choice = cand[0] < 0 ? 0 : cand[0];
+    float best = 0.0f;
+#pragma unroll
+    for (int k = 0; k < kQsacMaxM; ++k) {
+        if (k < m && cand[k] >= 0) {
+            const uint16_t *mu_row = cent_h + (int64_t)cand[k] * D;
+            float score = 0.0f;
+#pragma unroll
+            for (int g = 0; g < D / G; ++g) {
+                float lo = 0.0f, hi = 0.0f;
+#pragma unroll
+                for (int c = g * G; c < (g + 1) * G; c += 8) {
+                    float m8[8];
+                    load_bf16x8(mu_row + c, m8);
+#pragma unroll
+                    for (int kk = 0; kk < 8; ++kk) {
+                        const float r = __fsub_rn(xr[c + kk], m8[kk]);
+                        if (c + kk == g * G) {
+                            lo = r;
+                            hi = r;
+                        } else {
+                            if (r < lo) lo = r;
+                            if (r > hi) hi = r;
+                        }
+                    }
+                }
+                const float range = __fsub_rn(hi, lo);
+                score = __fadd_rn(score, __fmul_rn(wg[g], __fmul_rn(range, range)));
+            }
+            if (k == 0 || score < best) {
+                best = score;
+                choice = cand[k];
+            }
+        }
+    }
+    a.idx[(int64_t)h * a.T + t] = (uint16_t)choice;
+    // residual against the chosen centre, quantised as the plain encode does
+    const uint16_t *mu_row = cent_h + (int64_t)choice * D;
+#pragma unroll
+    for (int c = 0; c < D; c += 8) {
+        float m8[8];
+        load_bf16x8(mu_row + c, m8);
+#pragma unroll
+        for (int k = 0; k < 8; ++k)
+            xr[c + k] = __fsub_rn(xr[c + k], m8[k]);
+    }
+    const int64_t th = (int64_t)h * a.T + t;
+    encode_residual_row<D, BITS, G>(xr, a.codes + th * (D * BITS / 8),
+                                    static_cast<uint8_t *>(a.meta) + th * (D / G) * (a.meta16 ? 4 : 8), a.meta16 != 0);
+}
+
+// ---------------------------------------------------------------------------
 // Per-head reconstruction: one thread per 8 channels of a token-head.
 // ---------------------------------------------------------------------------
 struct DecodeArgs {
@@ -421,6 +581,80 @@ __global__ void __launch_bounds__(256) decode_kernel(DecodeArgs a)
         *reinterpret_cast<float4 *>(dst) = make_float4(v[0], v[1], v[2], v[3]);
         *reinterpret_cast<float4 *>(dst + 4) = make_float4(v[4], v[5], v[6], v[7]);
     }
+}
+
+// ---------------------------------------------------------------------------
+// PSAC coefficients (QuantWM, Sec. 4.2: principal query-subspace attention
+// correction): C[t][h] = (x - x^)[t][h] U_h, the part of the key's
+// reconstruction error along the r = 8 leading eigenvectors of the head's
+// query second-moment matrix.  One thread per token-head; x^ is formed as
+// decode_kernel forms it (binary32), e = x - x^ in binary32, the r dot
+// products accumulate in binary32 FMAs in channel order.
+// ---------------------------------------------------------------------------
+constexpr int kPsacRank = 8;
+
+struct PsacCoefArgs {
+    DecodeArgs d;     // the compressed K history (out / out_bf16 unused)
+    const void *x;    // original keys [T][H][D], float or bf16
+    int x_bf16;
+    const float *U;   // [H][D][8]
+    float *coef;      // [H][T][8]
+};
+
+template <int D>
+__global__ void __launch_bounds__(128) psac_coef_kernel(PsacCoefArgs p)
+{
+    const DecodeArgs &a = p.d;
+    __shared__ __align__(16) float sU[D * kPsacRank];
+    const int h = blockIdx.y;
+    for (int e = threadIdx.x; e < D * kPsacRank; e += 128)
+        sU[e] = p.U[(int64_t)h * D * kPsacRank + e];
+    __syncthreads();
+    const int64_t t = (int64_t)blockIdx.x * 128 + threadIdx.x;
+    if (t >= a.T)
+        return;
+    const int64_t th = (int64_t)h * a.T + t;
+    int j = a.idx[th];
+    if (j >= a.C) {
+        raise_status(DEVSTAT_BAD_INDEX);
+        j = 0;
+    }
+    const uint8_t *meta_row = static_cast<const uint8_t *>(a.meta) + th * (D / a.G) * (a.meta16 ? 4 : 8);
+    const uint32_t mask = (1u << a.bits) - 1u;
+    float acc[kPsacRank];
+#pragma unroll
+    for (int r = 0; r < kPsacRank; ++r)
+        acc[r] = 0.0f;
+#pragma unroll 1
+    for (int c0 = 0; c0 < D; c0 += 8) {
+        const float2 sz = load_sz(meta_row, c0 / a.G, a.meta16 != 0);
+        uint32_t cw;
+        if (a.bits == 2)
+            cw = *reinterpret_cast<const uint16_t *>(a.codes + th * (D / 4) + c0 / 4);
+        else
+            cw = *reinterpret_cast<const uint32_t *>(a.codes + th * (D / 2) + c0 / 2);
+        float mu[8], xv[8];
+        load_bf16x8(a.cent + ((int64_t)h * a.C + j) * D + c0, mu);
+        load_x8(p.x, p.x_bf16, (t * a.H + h) * D + c0, xv);
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+            const float xh = dequant_spec((cw >> (k * a.bits)) & mask, sz.x, sz.y, mu[k]);
+            const float e = __fsub_rn(xv[k], xh);
+            const float4 u0 = *reinterpret_cast<const float4 *>(sU + (c0 + k) * kPsacRank);
+            const float4 u1 = *reinterpret_cast<const float4 *>(sU + (c0 + k) * kPsacRank + 4);
+            acc[0] = fmaf(e, u0.x, acc[0]);
+            acc[1] = fmaf(e, u0.y, acc[1]);
+            acc[2] = fmaf(e, u0.z, acc[2]);
+            acc[3] = fmaf(e, u0.w, acc[3]);
+            acc[4] = fmaf(e, u1.x, acc[4]);
+            acc[5] = fmaf(e, u1.y, acc[5]);
+            acc[6] = fmaf(e, u1.z, acc[6]);
+            acc[7] = fmaf(e, u1.w, acc[7]);
+        }
+    }
+    float4 *dst = reinterpret_cast<float4 *>(p.coef + th * kPsacRank);
+    dst[0] = make_float4(acc[0], acc[1], acc[2], acc[3]);
+    dst[1] = make_float4(acc[4], acc[5], acc[6], acc[7]);
 }
 
 // ---------------------------------------------------------------------------

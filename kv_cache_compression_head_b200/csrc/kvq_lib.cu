@@ -558,6 +558,7 @@ bool make_attn_maps(AttnMaps *m, const AttnArgs &a)
     // compact binary16 {s, z} is read by the loader lanes: no map
     memset(&m->km, 0, sizeof m->km);
     memset(&m->vm, 0, sizeof m->vm);
+    memset(&m->kpc, 0, sizeof m->kpc);
     return encode_2d(&m->kc, CU_TENSOR_MAP_DATA_TYPE_UINT8, k.codes, 16u * k.bits, rows, 16u * k.bits,
                      16u * k.bits, 64, CU_TENSOR_MAP_SWIZZLE_NONE) &&
            (k.meta16 || encode_2d(&m->km, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, k.meta, 2u * (128 / k.G), rows,
@@ -569,7 +570,9 @@ bool make_attn_maps(AttnMaps *m, const AttnArgs &a)
            encode_2d(&m->kcent, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, k.cent, 128, (uint64_t)a.H * k.C, 256, 64, 1,
                      CU_TENSOR_MAP_SWIZZLE_128B) &&
            encode_2d(&m->vcent, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, v.cent, 128, (uint64_t)a.H * v.C, 256, 64, 1,
-                     CU_TENSOR_MAP_SWIZZLE_128B);
+                     CU_TENSOR_MAP_SWIZZLE_128B) &&
+           (!a.psac_coef || encode_2d(&m->kpc, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, a.psac_coef, 8, rows, 32, 8, 64,
+                                      CU_TENSOR_MAP_SWIZZLE_NONE));
 }
 
 template <int BK, int BV>
@@ -581,7 +584,7 @@ kvq_status launch_attention_tma_t(const AttnArgs &a, cudaStream_t s)
         return KVQ_ERR_CUDA;
     if (!configured[dev].load()) {
         if (cudaFuncSetAttribute(attention_tma_kernel<BK, BV>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)APSmem::kLaunchBytes) != cudaSuccess)
+                                 (int)ATSmem::kLaunchBytes) != cudaSuccess)
             return KVQ_ERR_CUDA;
         configured[dev].store(true);
     }
@@ -590,7 +593,7 @@ kvq_status launch_attention_tma_t(const AttnArgs &a, cudaStream_t s)
         return KVQ_ERR_CUDA;
     const dim3 grid((unsigned)(2 * ceil_div(a.Tq, kAPRowsPerPair)), (unsigned)a.H,
                     (unsigned)(a.nsplit > 1 ? a.nsplit : 1));
-    attention_tma_kernel<BK, BV><<<grid, kATThreads, APSmem::kLaunchBytes, s>>>(maps, a);
+    attention_tma_kernel<BK, BV><<<grid, kATThreads, ATSmem::kLaunchBytes, s>>>(maps, a);
     return launch_status();
 }
 
@@ -606,8 +609,8 @@ kvq_status launch_attention_pair(const AttnArgs &a, cudaStream_t s)
             return a.v.bits == 2 ? launch_attention_tma_t<2, 2>(a, s) : launch_attention_tma_t<2, 4>(a, s);
         return a.v.bits == 2 ? launch_attention_tma_t<4, 2>(a, s) : launch_attention_tma_t<4, 4>(a, s);
     }
-    if ((a.k.meta16 || a.v.meta16) && a.t_end > a.t_begin)
-        return KVQ_ERR_UNSUPPORTED;  // only the TMA-staged kernel reads compact {s, z}
+    if ((a.k.meta16 || a.v.meta16 || a.psac_coef) && a.t_end > a.t_begin)
+        return KVQ_ERR_UNSUPPORTED;  // only the TMA-staged kernel reads compact {s, z} and PSAC terms
     if (a.k.bits == 2)
         return a.v.bits == 2 ? launch_attention_pair_t<2, 2, false>(a, s) : launch_attention_pair_t<2, 4, false>(a, s);
     return a.v.bits == 2 ? launch_attention_pair_t<4, 2, false>(a, s) : launch_attention_pair_t<4, 4, false>(a, s);
@@ -984,6 +987,55 @@ kvq_status kvq_encode(const kvq_codec_desc *desc, const void *x, kvq_dtype x_dty
     return launch_encode(desc->head_dim, e, reinterpret_cast<cudaStream_t>(stream));
 }
 
+kvq_status kvq_encode_qsac(const kvq_codec_desc *desc, const void *x, kvq_dtype x_dtype, int64_t T,
+                           const void *centroids, const float *w, int32_t M, uint16_t *idx, uint8_t *codes,
+                           void *meta, kvq_stream_t stream)
+{
+    kvq_status st = check_desc(desc, false);
+    if (st != KVQ_OK)
+        return st;
+    if (T < 0 || (x_dtype != KVQ_F32 && x_dtype != KVQ_BF16) || M < 1 || M > kQsacMaxM)
+        return KVQ_ERR_INVALID_ARG;
+    if (desc->meta_format != KVQ_META_F32 || desc->num_heads > 65535)
+        return KVQ_ERR_UNSUPPORTED;
+    if (T == 0)
+        return KVQ_OK;
+    if (!x || !centroids || !w || !idx || !codes || !meta)
+        return KVQ_ERR_INVALID_ARG;
+    if (!aligned16(x) || !aligned16(centroids) || !aligned16(w) || !aligned16(codes) || !aligned16(meta) ||
+        (reinterpret_cast<uintptr_t>(idx) & 1u))
+        return KVQ_ERR_ALIGNMENT;
+    QsacArgs q;
+    memset(&q, 0, sizeof q);
+    q.e.x = x;
+    q.e.x_bf16 = x_dtype == KVQ_BF16;
+    q.e.T = T;
+    q.e.H = desc->num_heads;
+    q.e.C = desc->num_centroids;
+    q.e.bits = desc->bits;
+    q.e.G = desc->group_size;
+    q.e.cent = static_cast<const uint16_t *>(centroids);
+    q.e.idx = idx;
+    q.e.codes = codes;
+    q.e.meta = meta;
+    q.w = w;
+    q.M = M;
+    const dim3 grid((unsigned)ceil_div(T, kDirectTokens), (unsigned)desc->num_heads);
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    const int D = desc->head_dim, B = desc->bits, G = desc->group_size;
+#define KVQ_QSAC(DD, BB, GG)                                                          \
+    if (D == DD && B == BB && G == GG) {                                              \
+        qsac_encode_kernel<DD, BB, GG><<<grid, kDirectTokens, 0, s>>>(q);             \
+        return launch_status();                                                       \
+    }
+    KVQ_QSAC(128, 2, 16) KVQ_QSAC(128, 2, 32) KVQ_QSAC(128, 2, 64)
+    KVQ_QSAC(128, 4, 16) KVQ_QSAC(128, 4, 32) KVQ_QSAC(128, 4, 64)
+    KVQ_QSAC(64, 2, 16) KVQ_QSAC(64, 2, 32) KVQ_QSAC(64, 2, 64)
+    KVQ_QSAC(64, 4, 16) KVQ_QSAC(64, 4, 32) KVQ_QSAC(64, 4, 64)
+#undef KVQ_QSAC
+    return KVQ_ERR_UNSUPPORTED;
+}
+
 kvq_status kvq_joint_coefficients(const kvq_codec_desc *desc, const void *x, kvq_dtype x_dtype, int64_t T,
                                   const void *centroids, const void *w_enc, uint16_t *idx, float *coef_out,
                                   void *workspace, size_t workspace_bytes, kvq_stream_t stream)
@@ -1082,6 +1134,81 @@ kvq_status kvq_attention_lse(const void *q, int64_t Tq, const kvq_compressed_vie
     a.k = to_codec_view(k);
     a.v = to_codec_view(v);
     return attention_call(a, D, workspace, workspace_bytes, reinterpret_cast<cudaStream_t>(stream));
+}
+
+kvq_status kvq_attention_psac_lse(const void *q, int64_t Tq, const kvq_compressed_view *k,
+                                  const kvq_compressed_view *v, const float *U, const float *coef, int32_t rank,
+                                  int64_t t_begin, int64_t t_end, float softmax_scale, void *o_out, kvq_dtype o_dtype,
+                                  float *lse_out, void *workspace, size_t workspace_bytes, kvq_stream_t stream)
+{
+    kvq_status st = check_history_pair(k, v, t_begin, t_end);
+    if (st != KVQ_OK)
+        return st;
+    if (Tq < 0 || (o_dtype != KVQ_F32 && o_dtype != KVQ_BF16))
+        return KVQ_ERR_INVALID_ARG;
+    if (rank != kPsacRank || k->desc.head_dim != 128)
+        return KVQ_ERR_UNSUPPORTED;
+    const int H = k->desc.num_heads;
+    const int Cmax = k->desc.num_centroids > v->desc.num_centroids ? k->desc.num_centroids : v->desc.num_centroids;
+    if ((int64_t)H * k->num_tokens >= (int64_t)INT32_MAX || (int64_t)H * Cmax >= (int64_t)INT32_MAX)
+        return KVQ_ERR_UNSUPPORTED;
+    if (Tq == 0)
+        return KVQ_OK;
+    if (!q || !o_out || !lse_out || !U || !coef)
+        return KVQ_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(o_out) || !aligned16(lse_out) || !aligned16(U) || !aligned16(coef))
+        return KVQ_ERR_ALIGNMENT;
+    AttnArgs a = attn_args(q, Tq, H, 128, t_begin, t_end, softmax_scale, o_out, o_dtype, lse_out);
+    a.k = to_codec_view(k);
+    a.v = to_codec_view(v);
+    a.psac_u = U;
+    a.psac_coef = coef;
+    return attention_call(a, 128, workspace, workspace_bytes, reinterpret_cast<cudaStream_t>(stream));
+}
+
+kvq_status kvq_psac_coefficients(const kvq_compressed_view *k, const void *x, kvq_dtype x_dtype, const float *U,
+                                 int32_t rank, float *coef_out, kvq_stream_t stream)
+{
+    kvq_status st = check_view(k);
+    if (st != KVQ_OK)
+        return st;
+    if (k->desc.joint_rank > 0 || rank != kPsacRank)
+        return KVQ_ERR_UNSUPPORTED;
+    if (x_dtype != KVQ_F32 && x_dtype != KVQ_BF16)
+        return KVQ_ERR_INVALID_ARG;
+    if (k->num_tokens == 0)
+        return KVQ_OK;
+    if (!x || !U || !coef_out)
+        return KVQ_ERR_INVALID_ARG;
+    if (!aligned16(x) || !aligned16(U) || !aligned16(coef_out))
+        return KVQ_ERR_ALIGNMENT;
+    if (k->desc.num_heads > 65535)
+        return KVQ_ERR_UNSUPPORTED;
+    PsacCoefArgs p;
+    DecodeArgs &a = p.d;
+    memset(&p, 0, sizeof p);
+    a.cent = static_cast<const uint16_t *>(k->centroids);
+    a.idx = k->idx;
+    a.codes = k->codes;
+    a.meta = k->meta;
+    a.T = k->num_tokens;
+    a.H = k->desc.num_heads;
+    a.D = k->desc.head_dim;
+    a.C = k->desc.num_centroids;
+    a.bits = k->desc.bits;
+    a.G = k->desc.group_size;
+    a.meta16 = k->desc.meta_format == KVQ_META_F16;
+    p.x = x;
+    p.x_bf16 = x_dtype == KVQ_BF16;
+    p.U = U;
+    p.coef = coef_out;
+    const dim3 grid((unsigned)ceil_div(a.T, 128), (unsigned)a.H);
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (a.D == 128)
+        psac_coef_kernel<128><<<grid, 128, 0, s>>>(p);
+    else
+        psac_coef_kernel<64><<<grid, 128, 0, s>>>(p);
+    return launch_status();
 }
 
 kvq_status kvq_attention_dense_lse(const void *q, int64_t Tq, const void *k, const void *v, int64_t num_keys,

@@ -41,8 +41,9 @@ KVQ_OP_LAYER_ATTENTION = 4
 
 EXPORTED = (
     "kvq_status_string", "kvq_encoded_sizes", "kvq_workspace_size", "kvq_fit_centroids",
-    "kvq_fit_centroids_static", "kvq_encode",
-    "kvq_joint_coefficients", "kvq_decode", "kvq_attention_lse", "kvq_attention_dense_lse", "kvq_layer_attention",
+    "kvq_fit_centroids_static", "kvq_encode", "kvq_encode_qsac",
+    "kvq_joint_coefficients", "kvq_decode", "kvq_psac_coefficients", "kvq_attention_lse", "kvq_attention_psac_lse",
+    "kvq_attention_dense_lse", "kvq_layer_attention",
     "kvq_lse_merge", "kvq_last_device_status",
 )
 
@@ -79,9 +80,13 @@ def _load():
         "kvq_fit_centroids": [pdesc, vp, ctypes.c_int, i64, i32, vp, vp, sz, vp],
         "kvq_fit_centroids_static": [pdesc, vp, ctypes.c_int, i64, i32, vp, vp],
         "kvq_encode": [pdesc, vp, ctypes.c_int, i64, vp, vp, vp, vp, vp, vp, sz, vp],
+        "kvq_encode_qsac": [pdesc, vp, ctypes.c_int, i64, vp, vp, i32, vp, vp, vp, vp],
         "kvq_joint_coefficients": [pdesc, vp, ctypes.c_int, i64, vp, vp, vp, vp, vp, sz, vp],
         "kvq_decode": [pview, vp, ctypes.c_int, vp, sz, vp],
         "kvq_attention_lse": [vp, i64, pview, pview, i64, i64, ctypes.c_float, vp, ctypes.c_int, vp, vp, sz, vp],
+        "kvq_psac_coefficients": [pview, vp, ctypes.c_int, vp, i32, vp, vp],
+        "kvq_attention_psac_lse": [vp, i64, pview, pview, vp, vp, i32, i64, i64, ctypes.c_float, vp, ctypes.c_int, vp,
+                                   vp, sz, vp],
         "kvq_attention_dense_lse": [vp, i64, vp, vp, i64, i32, i32, i64, i64, ctypes.c_float, vp, ctypes.c_int, vp,
                                     vp, sz, vp],
         "kvq_layer_attention": [vp, i64, pview, pview, i64, i64, vp, vp, i64, ctypes.c_float, vp, ctypes.c_int, vp,
@@ -331,6 +336,21 @@ def kvq_encode(codec: Codec, x: torch.Tensor, centroids: torch.Tensor, idx: torc
                            workspace.numel() if workspace is not None else 0, _stream(stream)), "kvq_encode")
 
 
+def kvq_encode_qsac(codec: Codec, x: torch.Tensor, centroids: torch.Tensor, w: torch.Tensor, idx: torch.Tensor,
+                    codes: torch.Tensor, meta: torch.Tensor, M: int = 4, stream=None) -> None:
+    """Encode with QuantWM's query-sensitive centre selection; w [H][d]
+    float32 channel weights (the queries' second moments' diagonal)."""
+    T = _want_history("kvq_encode_qsac x", codec, x)
+    _want("kvq_encode_qsac centroids", centroids, torch.bfloat16,
+          shape=(codec.num_heads, codec.num_centroids, codec.head_dim))
+    _want("kvq_encode_qsac w", w, torch.float32, shape=(codec.num_heads, codec.head_dim))
+    _want_encoded("kvq_encode_qsac", codec, T, idx, codes, meta)
+    _on_cuda("kvq_encode_qsac", x, centroids, w, idx, codes, meta)
+    d = codec.c()
+    _check(_lib.kvq_encode_qsac(ctypes.byref(d), _ptr(x), _dtype_code(x), T, _ptr(centroids), _ptr(w), M, _ptr(idx),
+                                _ptr(codes), _ptr(meta), _stream(stream)), "kvq_encode_qsac")
+
+
 def kvq_joint_coefficients(codec: Codec, x: torch.Tensor, centroids: torch.Tensor, w_enc: torch.Tensor,
                            idx: torch.Tensor, coef_out: torch.Tensor, workspace: Optional[torch.Tensor] = None,
                            stream=None) -> None:
@@ -378,6 +398,47 @@ def kvq_attention_lse(q: torch.Tensor, k: Compressed, v: Compressed, o_out: torc
                                   softmax_scale, _ptr(o_out), _dtype_code(o_out), _ptr(lse_out), _ptr(workspace),
                                   workspace.numel() if workspace is not None else 0, _stream(stream)),
            "kvq_attention_lse")
+
+
+PSAC_RANK = 8
+
+
+def kvq_psac_coefficients(k: Compressed, x: torch.Tensor, U: torch.Tensor, coef_out: torch.Tensor,
+                          stream=None) -> None:
+    """QuantWM's PSAC coefficients C [H][T][8] = (k - k^) U_h of a K history;
+    x [T][H][d] the original keys, U [H][d][8] float32."""
+    _want_compressed("kvq_psac_coefficients k", k)
+    c = k.codec
+    _want("kvq_psac_coefficients x", x, _X_DTYPES, shape=(k.num_tokens, c.num_heads, c.head_dim))
+    _want("kvq_psac_coefficients U", U, torch.float32, shape=(c.num_heads, c.head_dim, PSAC_RANK))
+    _want("kvq_psac_coefficients coef_out", coef_out, torch.float32, shape=(c.num_heads, k.num_tokens, PSAC_RANK))
+    _on_cuda("kvq_psac_coefficients", k, x, U, coef_out)
+    kv = k.view()
+    _check(_lib.kvq_psac_coefficients(ctypes.byref(kv), _ptr(x), _dtype_code(x), _ptr(U), PSAC_RANK, _ptr(coef_out),
+                                      _stream(stream)), "kvq_psac_coefficients")
+
+
+def kvq_attention_psac_lse(q: torch.Tensor, k: Compressed, v: Compressed, U: torch.Tensor, coef: torch.Tensor,
+                           o_out: torch.Tensor, lse_out: torch.Tensor, t_begin: int = 0, t_end: Optional[int] = None,
+                           softmax_scale: float = 0.0, workspace: Optional[torch.Tensor] = None,
+                           stream=None) -> None:
+    """kvq_attention_lse over the PSAC-corrected keys k^ + U_h C (d = 128)."""
+    _want_compressed("kvq_attention_psac_lse k", k)
+    _want_compressed("kvq_attention_psac_lse v", v)
+    c = k.codec
+    _want_attention_io("kvq_attention_psac_lse", q, c.num_heads, c.head_dim, o_out, lse_out)
+    _want("kvq_attention_psac_lse U", U, torch.float32, shape=(c.num_heads, c.head_dim, PSAC_RANK))
+    _want("kvq_attention_psac_lse coef", coef, torch.float32, shape=(c.num_heads, k.num_tokens, PSAC_RANK))
+    _want_workspace("kvq_attention_psac_lse", workspace)
+    _on_cuda("kvq_attention_psac_lse", q, k, v, U, coef, o_out, lse_out, workspace)
+    if t_end is None:
+        t_end = k.num_tokens
+    kv, vv = k.view(), v.view()
+    _check(_lib.kvq_attention_psac_lse(_ptr(q), q.shape[0], ctypes.byref(kv), ctypes.byref(vv), _ptr(U), _ptr(coef),
+                                       PSAC_RANK, t_begin, t_end, softmax_scale, _ptr(o_out), _dtype_code(o_out),
+                                       _ptr(lse_out), _ptr(workspace),
+                                       workspace.numel() if workspace is not None else 0, _stream(stream)),
+           "kvq_attention_psac_lse")
 
 
 def kvq_attention_dense_lse(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, o_out: torch.Tensor,

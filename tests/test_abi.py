@@ -308,3 +308,40 @@ def test_compact_meta_sizes_and_refusals(K):
     assert K._lib.kvq_attention_lse(A, 10, ctypes.byref(v64), ctypes.byref(v64), 0, 100, ctypes.c_float(0.0), o,
                                     K.KVQ_F32, A, None, 0, None) == K.KVQ_ERR_UNSUPPORTED
     del sz
+
+
+def test_quantwm_entry_points_rejected_on_host(K):
+    """QSAC encode and the PSAC calls refuse bad arguments before any launch:
+    candidate counts outside 1..8, compact {s, z} or a joint codec for QSAC,
+    a PSAC rank other than 8, d = 64 PSAC attention, misaligned bases."""
+    A = 1 << 20
+    f0 = ctypes.c_float(0)
+    d = K.CodecDesc(12, 128, 256, 2, 16, 0)
+    qsac = lambda desc, *a: _err(K, "kvq_encode_qsac", ctypes.byref(desc), *a)
+    ok = (A, K.KVQ_BF16, 100, A, A)
+    assert qsac(d, *ok, 0, A, A, A, None) == K.KVQ_ERR_INVALID_ARG
+    assert qsac(d, *ok, 9, A, A, A, None) == K.KVQ_ERR_INVALID_ARG
+    assert qsac(d, A, K.KVQ_BF16, 100, A, None, 4, A, A, A, None) == K.KVQ_ERR_INVALID_ARG
+    assert qsac(d, A, K.KVQ_BF16, 100, A, A + 4, 4, A, A, A, None) == K.KVQ_ERR_ALIGNMENT
+    assert qsac(K.CodecDesc(12, 128, 256, 2, 16, 0, K.KVQ_META_F16), *ok, 4, A, A, A, None) \
+        == K.KVQ_ERR_UNSUPPORTED
+    assert qsac(K.CodecDesc(12, 128, 256, 4, 32, 192), *ok, 4, A, A, A, None) == K.KVQ_ERR_UNSUPPORTED
+    assert qsac(d, A, K.KVQ_BF16, 0, A, A, 4, A, A, A, None) == K.KVQ_OK
+
+    v = K.CompressedView(d, 1000, A, A, A, A, None)
+    coef = lambda view, *a: _err(K, "kvq_psac_coefficients", ctypes.byref(view), *a)
+    assert coef(v, A, K.KVQ_BF16, A, 4, A, None) == K.KVQ_ERR_UNSUPPORTED
+    assert coef(v, A, K.KVQ_BF16, A + 8, 8, A, None) == K.KVQ_ERR_ALIGNMENT
+    assert coef(v, A, K.KVQ_BF16, A, 8, None, None) == K.KVQ_ERR_INVALID_ARG
+    assert coef(v, A, 7, A, 8, A, None) == K.KVQ_ERR_INVALID_ARG
+    vj = K.CompressedView(K.CodecDesc(12, 128, 256, 4, 32, 192), 1000, A, A, A, A, A)
+    assert coef(vj, A, K.KVQ_BF16, A, 8, A, None) == K.KVQ_ERR_UNSUPPORTED
+    assert coef(K.CompressedView(d, 0, A, A, A, A, None), None, K.KVQ_BF16, None, 8, None, None) == K.KVQ_OK
+
+    att = lambda kv, vv, *a: _err(K, "kvq_attention_psac_lse", A, 10, ctypes.byref(kv), ctypes.byref(vv), *a)
+    assert att(v, v, A, A, 4, 0, 1000, f0, A, K.KVQ_F32, A, None, 0, None) == K.KVQ_ERR_UNSUPPORTED
+    assert att(v, v, A, None, 8, 0, 1000, f0, A, K.KVQ_F32, A, None, 0, None) == K.KVQ_ERR_INVALID_ARG
+    assert att(v, v, A, A + 4, 8, 0, 1000, f0, A, K.KVQ_F32, A, None, 0, None) == K.KVQ_ERR_ALIGNMENT
+    assert att(v, v, A, A, 8, 0, 1001, f0, A, K.KVQ_F32, A, None, 0, None) == K.KVQ_ERR_INVALID_ARG
+    v64 = K.CompressedView(K.CodecDesc(12, 64, 256, 2, 16, 0), 1000, A, A, A, A, None)
+    assert att(v64, v64, A, A, 8, 0, 1000, f0, A, K.KVQ_F32, A, None, 0, None) == K.KVQ_ERR_UNSUPPORTED

@@ -28,6 +28,13 @@ Functions and the passages they follow:
   (Sec. 4.1): per-head second moments of the historical queries, their
   diagonal as channel weights, top-M candidates by the weighted distance, the
   final centre by the expected squared logit error of its quantised residual.
+* ``bf16_bits``, ``fast_maps_analytical``, ``fast_reduce_queries``,
+  ``fast_attention``, ``fast_history_mac_ratio``: NanoKV-Fast's
+  mixed-dimensional attention (NanoKV page, abstract, Fig. 4(a,d), Tables 6,
+  8 and 11): queries reduced into a head's low-dimensional space, attention
+  there over keys and values decoded straight into that space from the
+  stored coefficients, outputs restored to the head dimension before the
+  LSE merge.
 * ``psac_basis``, ``psac_coefficients``, ``attention_psac``: QuantWM's
   principal-subspace logit correction (the PSAC section after Sec. 4.1;
   r = 8, Table 9): the remaining key error
@@ -466,6 +473,89 @@ def attention_psac(q: np.ndarray, k_hat: np.ndarray, v: np.ndarray, U: np.ndarra
     the corrected keys k^_j + U_r C_j, which is how it is evaluated."""
     kc = _widen(k_hat) + np.einsum("hdr,thr->thd", U, coef.astype(np.float64))
     return attention(q, kc, v, scale, rows)
+
+
+# ----------------------------------------------------------------------------
+# NanoKV-Fast: mixed-dimensional attention on the joint code
+# ----------------------------------------------------------------------------
+
+def bf16_bits(a: np.ndarray) -> np.ndarray:
+    """Round-to-nearest-even of real values (float64, or float32 widened) to
+    bf16, as bit patterns [uint16].  Values past the largest finite bf16
+    round to infinity; the subnormal range keeps the fixed 2^-133 spacing."""
+    a = np.asarray(a, np.float64)
+    m, e = np.frexp(a)                       # a = m 2^e, 0.5 <= |m| < 1
+    e = np.maximum(e, -125)                  # bf16 normals start at 2^-126
+    q = np.rint(np.ldexp(a, 8 - e))          # 8 significant bits, ties to even
+    r = np.ldexp(q, e - 8)
+    with np.errstate(over="ignore"):
+        f = r.astype(np.float32)             # exact unless past the range (-> inf)
+    return (f.view(np.uint32) >> 16).astype(np.uint16)
+
+
+def fast_maps_analytical(w_dec: np.ndarray, cent: np.ndarray, d_low: int):
+    """Analytical low-dimensional maps of one branch (the "analytical
+    initialization" row of Table 8), per head h of the joint decoder W_dec
+    [r][H d] (bf16 bits or float) and the centres [H][C][d]:
+
+      P_h     [d][d_low]  the d_low leading right singular vectors of the head's
+                          decoder slice W_dec[:, h d:(h+1) d] (numpy.linalg.svd,
+                          descending singular values), each with its
+                          largest-magnitude component made positive;
+      W_low   [r][H d_low] the folded decoder, W_dec,h P_h per head;
+      c_low   [H][C][d_low] the centres in the low space, mu_h P_h.
+
+    Keys use their branch's P_h to reduce queries; values use theirs, P_h^T,
+    to restore outputs.  Returned in float64; the resident copies are bf16."""
+    W = _widen(np.asarray(w_dec))
+    cf = _widen(np.asarray(cent))
+    H, C, d = cf.shape
+    r = W.shape[0]
+    P = np.zeros((H, d, d_low))
+    W_low = np.zeros((r, H * d_low))
+    c_low = np.zeros((H, C, d_low))
+    for h in range(H):
+        Wh = W[:, h * d:(h + 1) * d]
+        _, _, vt = np.linalg.svd(Wh, full_matrices=True)
+        V = vt[:d_low].T                                        # [d][d_low]
+        sign = np.sign(V[np.argmax(np.abs(V), axis=0), np.arange(d_low)])
+        V = V * np.where(sign == 0, 1.0, sign)[None, :]
+        P[h] = V
+        W_low[:, h * d_low:(h + 1) * d_low] = Wh @ V
+        c_low[h] = cf[h] @ V
+    return P, W_low, c_low
+
+
+def fast_reduce_queries(q: np.ndarray, P: np.ndarray) -> np.ndarray:
+    """Queries reduced into each head's low space, q_h P_h, rounded to bf16
+    (the model's activation type): q [Tq][H][d], P [H][d][d_low] (bf16 bits
+    or float) -> [Tq][H][d_low] bf16 bits."""
+    return bf16_bits(np.einsum("thc,hcl->thl", _widen(q), _widen(P)))
+
+
+def fast_attention(q: np.ndarray, k_low: np.ndarray, v_low: np.ndarray, P: np.ndarray, R: np.ndarray,
+                   scale: Optional[float] = None, rows: Optional[np.ndarray] = None) -> Tuple[np.ndarray, np.ndarray]:
+    """NanoKV-Fast's low-dimensional history attention of one head set
+    (NanoKV page, Fig. 4(d)): the queries are reduced, q_low = bf16(q_h P_h);
+    attention runs in the low space over k_low, v_low [T][H][d_low] with the
+    softmax scale of the full head dimension (the low-space logits stand in
+    for q . k), and the output is restored, O_h = O_low,h R_h with R [H][d_low][d].
+    Returns O [n][H][d] and lse [H][n] as ``attention`` does."""
+    d = _widen(P).shape[1]
+    q_low = fast_reduce_queries(q, P)
+    sc = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    o_low, lse = attention(q_low, k_low, v_low, sc, rows)
+    return np.einsum("thl,hld->thd", o_low, _widen(R)), lse
+
+
+def fast_history_mac_ratio(dim_counts: dict, d: int = 128) -> float:
+    """History-attention MACs of the deployed head dims relative to full
+    dimension, when every head-layer attends its whole history at its own
+    dim d_h: both Q K^T and P V scale with d_h, so the ratio is
+    sum_h count_h d_h / (sum_h count_h d) (NanoKV page, Table 6's counts)."""
+    num = sum(int(n) * int(dh) for dh, n in dim_counts.items())
+    den = sum(int(n) for n in dim_counts.values()) * d
+    return num / den
 
 
 # ----------------------------------------------------------------------------

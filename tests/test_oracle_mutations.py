@@ -113,6 +113,15 @@ PY_MUTATIONS = [
      'np.argsort(lam, kind="stable")'),
     ("psac_coefficients", "PSAC error with the wrong sign", "e = _widen(x) - _widen(k_hat)",
      "e = _widen(k_hat) - _widen(x)"),
+    ("bf16_bits", "bf16 rounding truncates", "q = np.rint(np.ldexp(a, 8 - e))", "q = np.trunc(np.ldexp(a, 8 - e))"),
+    ("fast_maps_analytical", "analytical maps keep the smallest singular vectors", "V = vt[:d_low].T",
+     "V = vt[-d_low:].T"),
+    ("fast_reduce_queries", "reduced queries left unrounded",
+     'return bf16_bits(np.einsum("thc,hcl->thl", _widen(q), _widen(P)))',
+     'return np.einsum("thc,hcl->thl", _widen(q), _widen(P))'),
+    ("fast_attention", "softmax scale of the low dimension", "d = _widen(P).shape[1]", "d = _widen(P).shape[2]"),
+    ("fast_attention", "output restored with the query map", "_widen(R))", "np.transpose(_widen(P), (0, 2, 1)))"),
+    ("fast_history_mac_ratio", "MACs not weighted by the head dim", "int(n) * int(dh)", "int(n) * d"),
     ("attention_psac", "PSAC correction dropped", 'kc = _widen(k_hat) + np.einsum("hdr,thr->thd", U, coef.astype(np.float64))',
      "kc = _widen(k_hat)"),
 ]

@@ -775,3 +775,161 @@ def test_encode16_decode16_storage_and_bound():
         bound = s16 / 2 + ((1 << bits) - 1) * np.abs(s32 - s16) + 1e-6 * (1 + np.abs(xf).max())
         err = np.abs(dec - xf).transpose(1, 0, 2).reshape(H, T, d // G, G).max(axis=3)
         assert np.all(err[exact_z] <= bound[exact_z])
+
+
+# ----------------------------------------------------------------------------
+# NanoKV-Fast: mixed-dimensional attention (NanoKV page, Fig. 4(d), Tables 6,
+# 8, 9, 11)
+# ----------------------------------------------------------------------------
+
+def test_bf16_bits_rounds_to_nearest_even():
+    """Against torch's float32 -> bf16 conversion (random values, every
+    binade's ties, subnormals, overflow) and hand-worked float64 cases that
+    float32 cannot hold: a value just above a tie rounds up, exact ties go to
+    the even neighbour."""
+    rng = np.random.default_rng(5)
+    a = (rng.standard_normal(20000) * np.exp2(rng.integers(-140, 128, 20000))).astype(np.float32)
+    ties = (np.float32(1.0) + np.float32(2.0 ** -8) * np.arange(1, 64, 2, dtype=np.float32)).astype(np.float32)
+    a = np.concatenate([a, ties, -ties, np.float32([0.0, -0.0, 3.0e38, 3.4e38, -3.4e38, 1e-40, 2.0 ** -133])])
+    with np.errstate(over="ignore"):
+        assert np.array_equal(O.bf16_bits(a), _bf16(a))
+    assert O.bf16_bits(np.array([1 + 2.0 ** -8 + 2.0 ** -40]))[0] == 0x3F81   # above the tie: up
+    assert O.bf16_bits(np.array([1 + 2.0 ** -8]))[0] == 0x3F80                # tie: even (down)
+    assert O.bf16_bits(np.array([1 + 3 * 2.0 ** -8]))[0] == 0x3F82            # tie: even (up)
+    assert O.bf16_bits(np.array([-(1 + 2.0 ** -8 - 2.0 ** -45)]))[0] == 0xBF80
+    assert O.bf16_bits(np.array([3 * 2.0 ** -134]))[0] == 0x0002              # subnormal tie: even
+
+
+def _fast_case(seed, T=37, Tq=11, H=2, d=64):
+    rng = np.random.default_rng(seed)
+    q = _bf16(rng.standard_normal((Tq, H, d)) * 0.5)
+    k = _bf16(rng.standard_normal((T, H, d)))
+    v = _bf16(rng.standard_normal((T, H, d)))
+    return q, k, v
+
+
+def test_fast_attention_identity_maps_are_full_attention():
+    """d_low = d with identity maps: the reduction and restoration change
+    nothing, so the result is exactly ``attention`` over the same keys."""
+    q, k, v = _fast_case(1)
+    H, d = q.shape[1], q.shape[2]
+    I = np.broadcast_to(np.eye(d), (H, d, d))
+    o, lse = O.fast_attention(q, k, v, _bf16(I), _bf16(I))
+    o_ref, lse_ref = O.attention(q, k, v)
+    assert np.array_equal(o, o_ref) and np.array_equal(lse, lse_ref)
+
+
+def test_fast_attention_channel_selection_is_brute_force():
+    """P_h picks d_low channels (entries +-2, exact in bf16), R_h puts them
+    back scaled by 1/2: the low-space logits are 2 q_c k'_c summed over the
+    picked channels, the softmax scale is that of the FULL head dimension, and
+    the output lands on the picked channels only -- checked against a direct
+    loop over keys."""
+    q, k, v = _fast_case(2, T=19, Tq=5, d=64)
+    Tq, H, d = q.shape
+    dl = 16
+    rng = np.random.default_rng(3)
+    P = np.zeros((H, d, dl))
+    R = np.zeros((H, dl, d))
+    picks = []
+    for h in range(H):
+        sel = rng.choice(d, dl, replace=False)
+        sgn = rng.choice([-1.0, 1.0], dl)
+        P[h, sel, np.arange(dl)] = 2.0 * sgn
+        R[h, np.arange(dl), sel] = 0.5 * sgn
+        picks.append((sel, sgn))
+    k_low = np.zeros((k.shape[0], H, dl), np.float32)
+    v_low = np.zeros((v.shape[0], H, dl), np.float32)
+    kf, vf, qf = _widen(k), _widen(v), _widen(q).astype(np.float64)
+    for h, (sel, sgn) in enumerate(picks):
+        k_low[:, h] = kf[:, h][:, sel]
+        v_low[:, h] = vf[:, h][:, sel]
+    o, lse = O.fast_attention(q, _bf16(k_low), _bf16(v_low), _bf16(P), _bf16(R))
+    for i in range(Tq):
+        for h, (sel, sgn) in enumerate(picks):
+            s = np.array([sum(2.0 * sgn[j] * qf[i, h, sel[j]] * k_low[t, h, j] for j in range(dl))
+                          for t in range(k.shape[0])]) / math.sqrt(d)
+            m = s.max()
+            p = np.exp(s - m)
+            want = np.zeros(d)
+            for j in range(dl):
+                want[sel[j]] = 0.5 * sgn[j] * float(np.dot(p, v_low[:, h, j])) / p.sum()
+            assert np.allclose(o[i, h], want, rtol=1e-12, atol=1e-12)
+            assert abs(lse[h, i] - (m + math.log(p.sum()))) < 1e-12
+
+
+def test_fast_attention_in_the_span_equals_full_attention():
+    """With orthonormal maps whose entries are exact in bf16 (Hadamard columns
+    / 8, d = 64) and queries, keys and values inside their span, the reduced
+    attention IS the full attention: q P P^T k = q k."""
+    Tq, T, H, d, dl = 6, 29, 2, 64, 16
+    Hd = np.array([[1.0]])
+    while Hd.shape[0] < d:
+        Hd = np.block([[Hd, Hd], [Hd, -Hd]])
+    P = np.stack([Hd[:, 3:3 + dl] / 8.0, Hd[:, 40:40 + dl] / 8.0])      # [H][d][dl], orthonormal columns
+    rng = np.random.default_rng(4)
+    small = lambda *s: rng.integers(-4, 5, s).astype(np.float64) / 4.0
+    q_low, k_low, v_low = small(Tq, H, dl), small(T, H, dl), small(T, H, dl)
+    q = np.einsum("thl,hdl->thd", q_low, P)        # in the span; exact dyadic values
+    k = np.einsum("thl,hdl->thd", k_low, P)
+    v = np.einsum("thl,hdl->thd", v_low, P)
+    assert np.array_equal(_widen(_bf16(q)).astype(np.float64), q)   # q itself is a bf16 tensor
+    o, lse = O.fast_attention(_bf16(q), k_low.astype(np.float32), v_low.astype(np.float32), _bf16(P),
+                              _bf16(np.transpose(P, (0, 2, 1))))
+    o_ref, lse_ref = O.attention(q, k, v)
+    assert np.allclose(o, o_ref, rtol=0, atol=1e-12) and np.allclose(lse, lse_ref, rtol=0, atol=1e-12)
+
+
+def test_fast_maps_analytical_properties():
+    """Per head: P_h has orthonormal columns ordered by descending singular
+    value of the decoder slice; W_low = W_h P_h and c_low = mu_h P_h; when the
+    slice has rank <= d_low the folded decoder loses nothing, W_low P_h^T =
+    W_h, and the leading vector carries the largest singular value."""
+    rng = np.random.default_rng(6)
+    r, H, d, C, dl = 24, 2, 64, 5, 16
+    base = _bf16(rng.standard_normal((10, H * d)) / 8.0)
+    w_dec = base[rng.integers(0, 10, r)]             # 24 rows copied from 10: rank <= 10 < dl, exactly
+    cent = _bf16(rng.standard_normal((H, C, d)))
+    P, W_low, c_low = O.fast_maps_analytical(w_dec, cent, dl)
+    W = _widen(w_dec).astype(np.float64)
+    for h in range(H):
+        Wh = W[:, h * d:(h + 1) * d]
+        assert np.allclose(P[h].T @ P[h], np.eye(dl), atol=1e-12)
+        assert np.allclose(W_low[:, h * dl:(h + 1) * dl], Wh @ P[h], atol=1e-12)
+        assert np.allclose(c_low[h], _widen(cent[h]).astype(np.float64) @ P[h], atol=1e-12)
+        assert np.allclose(W_low[:, h * dl:(h + 1) * dl] @ P[h].T, Wh, atol=1e-9)
+        gains = np.linalg.norm(Wh @ P[h], axis=0)
+        assert np.all(np.diff(gains[:10]) <= 1e-9) and abs(gains[0] - np.linalg.norm(Wh, 2)) < 1e-9
+        assert np.all(P[h][np.argmax(np.abs(P[h]), axis=0), np.arange(dl)] > 0)
+
+
+def test_fast_mac_accounting_against_tables_6_9_11():
+    """Table 6's head-layer counts add up to Table 9's layers x heads; with
+    every head-layer attending its whole history at its deployed dim the
+    history MACs fall to sum count d_h / (sum count 128), a bound Table 11's
+    saving (which routes some history at full dimension, Table 7) stays
+    under; and Table 11's overall saving is the product of its two columns."""
+    for m in _golden("nanokv_fast_tables.json")["models"]:
+        dims = {int(k): v for k, v in m["dims"].items()}
+        assert sum(dims.values()) == m["layers"] * m["heads"]
+        ratio = O.fast_history_mac_ratio(dims, m["head_dim"])
+        assert m["history_saved_pct"] <= 100.0 * (1.0 - ratio)
+        assert abs(m["historical_share_pct"] * m["history_saved_pct"] / 100.0 - m["all_saved_pct"]) < 0.006
+    hy32 = _golden("nanokv_fast_tables.json")["models"][1]
+    assert O.fast_history_mac_ratio({int(k): v for k, v in hy32["dims"].items()}) == 0.5
+    assert O.fast_history_mac_ratio({64: 3}) == 0.5 and O.fast_history_mac_ratio({128: 1}) == 1.0
+
+
+def test_fast_reduce_queries_rounds_the_exact_sum_once():
+    """q_h P_h is formed exactly and rounded to bf16 once, to nearest even:
+    with q = (1, 2^-8) the columns (1, 1), (1, 3), (1, 1 + 2^-7) and (-1, -1)
+    give 1 + 2^-8 (a tie: down to 1), 1 + 3 2^-8 (a tie: up), 1 + 2^-8 +
+    2^-15 (above the tie: up) and -(1 + 2^-8); a second head uses its own map."""
+    q = _bf16(np.array([[[1.0, 2.0 ** -8], [2.0, 0.0]]]))                       # [1][2][2]
+    P = np.zeros((2, 2, 4))
+    P[0] = np.array([[1.0, 1.0, 1.0, -1.0], [1.0, 3.0, 1.0 + 2.0 ** -7, -1.0]])
+    P[1] = np.array([[0.5, 0.0, 3.0, 1.0], [7.0, 1.0, 1.0, 1.0]])
+    got = O.fast_reduce_queries(q, _bf16(P))
+    assert got.dtype == np.uint16 and got.shape == (1, 2, 4)
+    assert [int(b) for b in got[0, 0]] == [0x3F80, 0x3F82, 0x3F81, 0xBF80]
+    assert [float(x) for x in _widen(got[0, 1])] == [1.0, 0.0, 6.0, 2.0]

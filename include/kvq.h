@@ -339,6 +339,42 @@ KVQ_API kvq_status kvq_attention_psac_lse(const void *q, int64_t num_queries, co
                                           size_t workspace_bytes, kvq_stream_t stream);
 
 /*
+ * NanoKV-Fast low-dimensional history attention (NanoKV page, abstract,
+ * Fig. 4(a,d); per-head attention dims, Table 6): for each head h with its
+ * low dim d_low,
+ *   q_low = bf16(q_h P_h)                  queries reduced into the low space
+ *                                           (binary64 sums, correctly rounded
+ *                                           to bf16: RNE of the exact sum);
+ *   s_ij  = scale q_low,i . k_low,j         scale = softmax_scale if > 0, else
+ *                                           1/sqrt(d): the FULL head dimension;
+ *   o_low = softmax_j(s) v_low,  lse = ln sum_j exp(s_ij)  (as
+ *           kvq_attention_dense_lse, binary32 partials);
+ *   o_h   = o_low R_h                       restored to d channels (binary32).
+ *   q      [Tq][H][d] bf16;
+ *   k_low, v_low [num_keys][H][d_low] bf16: the history decoded straight into
+ *           the low space -- kvq_decode of a joint view whose head_dim is
+ *           d_low, whose centres are mu_h P_h and whose w_dec holds the folded
+ *           decoder W_dec,h P_h (per branch; the V branch folds its own maps);
+ *   P      [H][d][d_low] bf16 (query maps), R [H][d_low][d] bf16 (output maps);
+ *   o_out  [Tq][H][d] (o_dtype);  lse_out [H][Tq] float (natural log).
+ * d, d_low in {64, 128}, d_low <= d (KVQ_ERR_UNSUPPORTED otherwise; heads at
+ * 32 or 96 dims run at 64 or 128 with zero-padded maps).  Keys
+ * [t_begin, t_end) of the history; all pointers 16-byte aligned.
+ * Workspace (required): at least the q_low and o_low buffers, 6 Tq H d_low
+ * bytes rounded up; with kvq_fast_attention_workspace_size() bytes the
+ * attention may also split the key range as kvq_attention_lse does.
+ */
+KVQ_API kvq_status kvq_fast_attention_lse(const void *q, int64_t num_queries, const void *k_low, const void *v_low,
+                                          int64_t num_keys, int32_t num_heads, int32_t head_dim, int32_t d_low,
+                                          const void *P, const void *R, int64_t t_begin, int64_t t_end,
+                                          float softmax_scale, void *o_out, kvq_dtype o_dtype, float *lse_out,
+                                          void *workspace, size_t workspace_bytes, kvq_stream_t stream);
+
+/* Workspace bytes for kvq_fast_attention_lse with room to split. */
+KVQ_API kvq_status kvq_fast_attention_workspace_size(int32_t num_heads, int32_t head_dim, int32_t d_low,
+                                                     int64_t num_queries, size_t *bytes);
+
+/*
  * Dense-mode attention: the same computation as kvq_attention_lse over keys
  * [t_begin, t_end) of UNCOMPRESSED bf16 keys and values -- the current
  * chunk's own keys, or raw protected history tokens such as attention sinks

@@ -18,6 +18,7 @@
 #include "codec.cuh"
 #include "common.cuh"
 #include "encode_filter.cuh"
+#include "fast.cuh"
 #include "joint.cuh"
 #include "merge.cuh"
 
@@ -1164,6 +1165,118 @@ kvq_status kvq_attention_psac_lse(const void *q, int64_t Tq, const kvq_compresse
     a.psac_u = U;
     a.psac_coef = coef;
     return attention_call(a, 128, workspace, workspace_bytes, reinterpret_cast<cudaStream_t>(stream));
+}
+
+}  // extern "C"
+
+namespace {
+
+// NanoKV-Fast workspace: q_low bf16 [Tq][H][d_low] and o_low float
+// [Tq][H][d_low] (each 256-byte aligned), then optional split partials.
+size_t fast_base_bytes(int H, int dl, int64_t Tq)
+{
+    return round_up((size_t)Tq * H * dl * 2, 256) + round_up((size_t)Tq * H * dl * 4, 256);
+}
+
+template <int DIN, int DOUT, bool IN_BF16>
+kvq_status launch_fast_map(const FastMapArgs &f, cudaStream_t s)
+{
+    constexpr int kSmem = DIN * DOUT * 4;
+    static std::atomic<bool> configured[64];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64)
+        return KVQ_ERR_CUDA;
+    if (!configured[dev].load()) {
+        if (cudaFuncSetAttribute(fast_map_kernel<DIN, DOUT, IN_BF16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 kSmem) != cudaSuccess)
+            return KVQ_ERR_CUDA;
+        configured[dev].store(true);
+    }
+    const dim3 grid((unsigned)ceil_div(f.Tq, kFastThreads), (unsigned)f.H);
+    fast_map_kernel<DIN, DOUT, IN_BF16><<<grid, kFastThreads, kSmem, s>>>(f);
+    return launch_status();
+}
+
+kvq_status launch_fast_reduce(const FastMapArgs &f, int d, int dl, cudaStream_t s)
+{
+    if (d == 128)
+        return dl == 128 ? launch_fast_map<128, 128, true>(f, s) : launch_fast_map<128, 64, true>(f, s);
+    return launch_fast_map<64, 64, true>(f, s);
+}
+
+kvq_status launch_fast_restore(const FastMapArgs &f, int d, int dl, cudaStream_t s)
+{
+    if (d == 128)
+        return dl == 128 ? launch_fast_map<128, 128, false>(f, s) : launch_fast_map<64, 128, false>(f, s);
+    return launch_fast_map<64, 64, false>(f, s);
+}
+
+bool fast_dims_ok(int d, int dl) { return supported_dim(d) && supported_dim(dl) && dl <= d; }
+
+}  // namespace
+
+extern "C" {
+
+kvq_status kvq_fast_attention_workspace_size(int32_t H, int32_t d, int32_t d_low, int64_t Tq, size_t *bytes)
+{
+    if (!bytes || H < 1 || Tq < 0)
+        return KVQ_ERR_INVALID_ARG;
+    if (!fast_dims_ok(d, d_low) || H > 65535)
+        return KVQ_ERR_UNSUPPORTED;
+    *bytes = fast_base_bytes(H, d_low, Tq) + partials_bytes(kMaxAttnSplit, H, d_low, Tq);
+    return KVQ_OK;
+}
+
+kvq_status kvq_fast_attention_lse(const void *q, int64_t Tq, const void *k_low, const void *v_low, int64_t num_keys,
+                                  int32_t H, int32_t d, int32_t d_low, const void *P, const void *R, int64_t t_begin,
+                                  int64_t t_end, float softmax_scale, void *o_out, kvq_dtype o_dtype, float *lse_out,
+                                  void *workspace, size_t workspace_bytes, kvq_stream_t stream)
+{
+    if (H < 1 || Tq < 0 || num_keys < 0 || t_begin < 0 || t_end < t_begin || t_end > num_keys)
+        return KVQ_ERR_INVALID_ARG;
+    if (!fast_dims_ok(d, d_low) || H > 65535)
+        return KVQ_ERR_UNSUPPORTED;
+    if (o_dtype != KVQ_F32 && o_dtype != KVQ_BF16)
+        return KVQ_ERR_INVALID_ARG;
+    if (Tq == 0)
+        return KVQ_OK;
+    if (!q || !P || !R || !o_out || !lse_out || (t_end > t_begin && (!k_low || !v_low)))
+        return KVQ_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(P) || !aligned16(R) || !aligned16(o_out) || !aligned16(lse_out) ||
+        !aligned16(k_low) || !aligned16(v_low) || !aligned16(workspace))
+        return KVQ_ERR_ALIGNMENT;
+    const size_t base = fast_base_bytes(H, d_low, Tq);
+    if (!workspace || workspace_bytes < base)
+        return KVQ_ERR_WORKSPACE;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    uint8_t *ws = static_cast<uint8_t *>(workspace);
+    uint16_t *q_low = reinterpret_cast<uint16_t *>(ws);
+    float *o_low = reinterpret_cast<float *>(ws + round_up((size_t)Tq * H * d_low * 2, 256));
+    // (1) queries into the low space, rounded to bf16
+    FastMapArgs f;
+    f.in = q;
+    f.map = static_cast<const uint16_t *>(P);
+    f.out = q_low;
+    f.Tq = Tq;
+    f.H = H;
+    f.out_bf16 = 1;
+    kvq_status st = launch_fast_reduce(f, d, d_low, s);
+    if (st != KVQ_OK)
+        return st;
+    // (2) attention in the low space with the full head dimension's scale
+    const float scale = softmax_scale > 0.0f ? softmax_scale : 1.0f / sqrtf((float)d);
+    AttnArgs a = attn_args(q_low, Tq, H, d_low, t_begin, t_end, scale, o_low, KVQ_F32, lse_out);
+    a.dense = 1;
+    a.k_dense = static_cast<const uint16_t *>(k_low);
+    a.v_dense = static_cast<const uint16_t *>(v_low);
+    if ((st = attention_call(a, d_low, ws + base, workspace_bytes - base, s)) != KVQ_OK)
+        return st;
+    // (3) outputs restored to the head dimension
+    f.in = o_low;
+    f.map = static_cast<const uint16_t *>(R);
+    f.out = o_out;
+    f.out_bf16 = o_dtype == KVQ_BF16;
+    return launch_fast_restore(f, d, d_low, s);
 }
 
 kvq_status kvq_psac_coefficients(const kvq_compressed_view *k, const void *x, kvq_dtype x_dtype, const float *U,

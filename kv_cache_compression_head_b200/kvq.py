@@ -43,7 +43,7 @@ EXPORTED = (
     "kvq_status_string", "kvq_encoded_sizes", "kvq_workspace_size", "kvq_fit_centroids",
     "kvq_fit_centroids_static", "kvq_encode", "kvq_encode_qsac",
     "kvq_joint_coefficients", "kvq_decode", "kvq_psac_coefficients", "kvq_attention_lse", "kvq_attention_psac_lse",
-    "kvq_attention_dense_lse", "kvq_layer_attention",
+    "kvq_attention_dense_lse", "kvq_fast_attention_lse", "kvq_fast_attention_workspace_size", "kvq_layer_attention",
     "kvq_lse_merge", "kvq_last_device_status",
 )
 
@@ -87,6 +87,9 @@ def _load():
         "kvq_psac_coefficients": [pview, vp, ctypes.c_int, vp, i32, vp, vp],
         "kvq_attention_psac_lse": [vp, i64, pview, pview, vp, vp, i32, i64, i64, ctypes.c_float, vp, ctypes.c_int, vp,
                                    vp, sz, vp],
+        "kvq_fast_attention_lse": [vp, i64, vp, vp, i64, i32, i32, i32, vp, vp, i64, i64, ctypes.c_float, vp,
+                                   ctypes.c_int, vp, vp, sz, vp],
+        "kvq_fast_attention_workspace_size": [i32, i32, i32, i64, ctypes.POINTER(sz)],
         "kvq_attention_dense_lse": [vp, i64, vp, vp, i64, i32, i32, i64, i64, ctypes.c_float, vp, ctypes.c_int, vp,
                                     vp, sz, vp],
         "kvq_layer_attention": [vp, i64, pview, pview, i64, i64, vp, vp, i64, ctypes.c_float, vp, ctypes.c_int, vp,
@@ -460,6 +463,41 @@ def kvq_attention_dense_lse(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, o
                                         _ptr(workspace), workspace.numel() if workspace is not None else 0,
                                         _stream(stream)),
            "kvq_attention_dense_lse")
+
+
+def fast_attention_workspace(num_heads: int, head_dim: int, d_low: int, num_queries: int, device) -> torch.Tensor:
+    n = ctypes.c_size_t()
+    _check(_lib.kvq_fast_attention_workspace_size(num_heads, head_dim, d_low, num_queries, ctypes.byref(n)),
+           "kvq_fast_attention_workspace_size")
+    return torch.empty(max(1, n.value), dtype=torch.uint8, device=device)
+
+
+def kvq_fast_attention_lse(q: torch.Tensor, k_low: torch.Tensor, v_low: torch.Tensor, P: torch.Tensor,
+                           R: torch.Tensor, o_out: torch.Tensor, lse_out: torch.Tensor, workspace: torch.Tensor,
+                           t_begin: int = 0, t_end: Optional[int] = None, softmax_scale: float = 0.0,
+                           stream=None) -> None:
+    """NanoKV-Fast: attention in each head's low space over k_low, v_low
+    [Tk][H][d_low] (bf16), queries reduced by P [H][d][d_low], outputs
+    restored by R [H][d_low][d] (both bf16)."""
+    if k_low is None or k_low.dim() != 3:
+        raise ValueError("kvq_fast_attention_lse: expected low-space keys [Tk][H][d_low]")
+    Tk, H, dl = k_low.shape
+    if q is None or q.dim() != 3:
+        raise ValueError("kvq_fast_attention_lse: expected queries [Tq][H][d]")
+    d = q.shape[2]
+    _want("kvq_fast_attention_lse k_low", k_low, torch.bfloat16)
+    _want("kvq_fast_attention_lse v_low", v_low, torch.bfloat16, shape=(Tk, H, dl))
+    _want("kvq_fast_attention_lse P", P, torch.bfloat16, shape=(H, d, dl))
+    _want("kvq_fast_attention_lse R", R, torch.bfloat16, shape=(H, dl, d))
+    _want_attention_io("kvq_fast_attention_lse", q, H, d, o_out, lse_out)
+    _want_workspace("kvq_fast_attention_lse", workspace)
+    _on_cuda("kvq_fast_attention_lse", q, k_low, v_low, P, R, o_out, lse_out, workspace)
+    if t_end is None:
+        t_end = Tk
+    _check(_lib.kvq_fast_attention_lse(_ptr(q), q.shape[0], _ptr(k_low), _ptr(v_low), Tk, H, d, dl, _ptr(P), _ptr(R),
+                                       t_begin, t_end, softmax_scale, _ptr(o_out), _dtype_code(o_out), _ptr(lse_out),
+                                       _ptr(workspace), workspace.numel() if workspace is not None else 0,
+                                       _stream(stream)), "kvq_fast_attention_lse")
 
 
 def kvq_layer_attention(q: torch.Tensor, k_hist: Compressed, v_hist: Compressed, k_cur: Optional[torch.Tensor],

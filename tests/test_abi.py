@@ -345,3 +345,28 @@ def test_quantwm_entry_points_rejected_on_host(K):
     assert att(v, v, A, A, 8, 0, 1001, f0, A, K.KVQ_F32, A, None, 0, None) == K.KVQ_ERR_INVALID_ARG
     v64 = K.CompressedView(K.CodecDesc(12, 64, 256, 2, 16, 0), 1000, A, A, A, A, None)
     assert att(v64, v64, A, A, 8, 0, 1000, f0, A, K.KVQ_F32, A, None, 0, None) == K.KVQ_ERR_UNSUPPORTED
+
+
+def test_fast_attention_rejected_on_host(K):
+    """kvq_fast_attention_lse refuses before any launch: low dims outside
+    {64, 128} or above d, a missing or short workspace, misaligned maps, a
+    key range outside the keys; zero queries is a no-op."""
+    A = 1 << 20
+    f0 = ctypes.c_float(0)
+    need = 6 * 10 * 12 * 64
+    fast = lambda *a: _err(K, "kvq_fast_attention_lse", *a)
+    ok = lambda d, dl, ws=A, nws=1 << 20, P=A, t1=100: fast(A, 10, A, A, 100, 12, d, dl, P, A, 0, t1, f0, A,
+                                                         K.KVQ_F32, A, ws, nws, None)
+    assert ok(128, 32) == K.KVQ_ERR_UNSUPPORTED
+    assert ok(128, 96) == K.KVQ_ERR_UNSUPPORTED
+    assert ok(64, 128) == K.KVQ_ERR_UNSUPPORTED
+    assert ok(128, 64, ws=None, nws=0) == K.KVQ_ERR_WORKSPACE
+    assert ok(128, 64, nws=need - 1) == K.KVQ_ERR_WORKSPACE
+    assert ok(128, 64, P=A + 2) == K.KVQ_ERR_ALIGNMENT
+    assert ok(128, 64, t1=101) == K.KVQ_ERR_INVALID_ARG
+    assert fast(None, 0, None, None, 0, 12, 128, 64, None, None, 0, 0, f0, None, K.KVQ_F32, None, None, 0,
+                None) == K.KVQ_OK
+    n = ctypes.c_size_t()
+    assert K._lib.kvq_fast_attention_workspace_size(12, 128, 64, 10, ctypes.byref(n)) == K.KVQ_OK
+    assert n.value >= need
+    assert K._lib.kvq_fast_attention_workspace_size(12, 128, 32, 10, ctypes.byref(n)) == K.KVQ_ERR_UNSUPPORTED

@@ -19,7 +19,10 @@ C = 256, K2V2, group 16, 2 blocks) is timed the same way and reported under
 each call), ``next_rows`` reports the Wan-like chunk's full-layer attention:
 the compressed history plus the chunk's own 4,680 uncompressed keys under one
 softmax (kvq_layer_attention), and its dense part alone
-(kvq_attention_dense_lse).
+(kvq_attention_dense_lse); QuantWM's QSAC encode, PSAC coefficients and PSAC
+attention on the Wan-like layer; and NanoKV-Fast on the joint workload (the
+history decoded into a 64-dim space per head, low-space attention with query
+reduction and output restoration) beside its full-dimensional counterpart.
 
 Inputs are seeded synthetic tensors resident in HBM before timing starts;
 L2 is flushed (256 MiB write) before every timed step, outside the step's
@@ -418,6 +421,115 @@ class Pipeline:
                                        workspace=self.ws_attn)
 
 
+def quantwm_rows(p2, steps, warmup, flush, world, device, tfl, hbm):
+    """QuantWM's two additions on the Wan-like layer (its K history, after the
+    timed steps have fitted and encoded it): the QSAC encode (M = 4, channel
+    weights from the chunk's queries) beside the plain encode, the PSAC
+    coefficients, and the PSAC attention per history block beside the plain
+    one.  Basis U: the 8 leading eigenvectors of the queries' second moments
+    (set-up, not timed)."""
+    import torch
+
+    K, w = p2.K, p2.w
+    T, H, d, Tq = w.history_tokens, w.num_heads, w.head_dim, w.query_tokens
+    qf = p2.q.float()
+    Mq = torch.einsum("thc,the->hce", qf, qf) / Tq
+    wts = torch.diagonal(Mq, dim1=1, dim2=2).contiguous()
+    U = torch.linalg.eigh(Mq.double())[1][:, :, -8:].flip(-1).float().contiguous()
+    idx, codes, meta = K.alloc_encoded(p2.codec_k, T, device)
+    coef = torch.empty((H, T, 8), dtype=torch.float32, device=device)
+    qsac_ms = max_over_ranks(time_calls(lambda: K.kvq_encode_qsac(p2.codec_k, p2.xk, p2.cent[0], wts, idx, codes,
+                                                                  meta, M=4), steps, warmup, flush), world, device)
+    plain_ms = max_over_ranks(time_calls(lambda: K.kvq_encode(p2.codec_k, p2.xk, p2.cent[0], idx, codes, meta),
+                                         steps, warmup, flush), world, device)
+    coef_ms = max_over_ranks(time_calls(lambda: K.kvq_psac_coefficients(p2.comp[0], p2.xk, U, coef), steps, warmup,
+                                        flush), world, device)
+    o, lse = p2.o_parts[0], p2.l_parts[0]
+    e = p2.edges
+
+    def psac_blocks():
+        for b in range(p2.blocks):
+            K.kvq_attention_psac_lse(p2.q, p2.comp[0], p2.comp[1], U, coef, o, lse, t_begin=e[b], t_end=e[b + 1],
+                                     workspace=p2.ws_attn)
+
+    def plain_blocks():
+        for b in range(p2.blocks):
+            K.kvq_attention_lse(p2.q, p2.comp[0], p2.comp[1], o, lse, t_begin=e[b], t_end=e[b + 1],
+                                workspace=p2.ws_attn)
+
+    psac_ms = max_over_ranks(time_calls(psac_blocks, steps, warmup, flush), world, device)
+    base_ms = max_over_ranks(time_calls(plain_blocks, steps, warmup, flush), world, device)
+    check_status(K, "after the QuantWM rows")
+    flops = 4.0 * Tq * T * d * H
+    coef_bytes = T * H * (d * 2 + d * w.bits_k / 8 + (d // w.group_size) * 8 + 2 + 8 * 4)
+    return {
+        "qsac_encode": {"ms": qsac_ms, "plain_encode_ms": plain_ms, "M": 4,
+                        "what": "kvq_encode_qsac of the Wan-like K history (32760 x 12 x 128, C = 256, INT2 "
+                                "G = 16): exact weighted distances to every centre on CUDA cores, top-4, "
+                                "group-range score"},
+        "psac_coefficients": {"ms": coef_ms, "gbs": coef_bytes / (coef_ms / 1e3) / 1e9,
+                              "frac": coef_bytes / (coef_ms / 1e3) / 1e9 / hbm,
+                              "what": "kvq_psac_coefficients: reads x (bf16) and the compressed K, writes 8 "
+                                      "binary32 per token-head"},
+        "psac_attention": {"ms": psac_ms, "plain_ms": base_ms, "calls": p2.blocks,
+                           "tflops": flops / (psac_ms / 1e3) / 1e12, "frac": flops / (psac_ms / 1e3) / 1e12 / tfl,
+                           "what": "kvq_attention_psac_lse over the Wan-like history (2 blocks), beside "
+                                   "kvq_attention_lse on the same blocks"},
+    }
+
+
+def fast_rows(joint, steps, warmup, flush, world, device, tfl, d_low=64):
+    """NanoKV-Fast on the joint workload: its K and V joint codes decoded
+    straight into a 64-dim space per head (folded analytical maps, set up
+    with torch, not timed) and the low-space attention with query reduction
+    and output restoration, beside the full-dimensional decode + dense
+    attention of the same history."""
+    import torch
+
+    from kv_cache_compression_head_b200 import synth
+
+    K, wj = joint.K, joint.w
+    T, H, d, Tq, r = wj.history_tokens, wj.num_heads, wj.head_dim, wj.query_tokens, wj.joint_rank
+    q = torch.from_numpy(synth.make_queries(wj).view(np.int16)).to(device).view(torch.bfloat16)
+    Wf = joint.w_dec.float().view(r, H, d)
+    P = torch.stack([torch.linalg.svd(Wf[:, h].double(), full_matrices=True)[2][:d_low].t() for h in range(H)])
+    lows, dec_low, dec_full = [], [], []
+    for i in range(2):
+        Wl = torch.einsum("rhd,hdl->rhl", Wf.double(), P).reshape(r, H * d_low).to(torch.bfloat16).contiguous()
+        cl = torch.einsum("hcd,hdl->hcl", joint.cent[i].double(), P).to(torch.bfloat16).contiguous()
+        codec = K.Codec(H, d_low, wj.num_centroids, joint.codec[i].bits, wj.joint_group, r)
+        lows.append(K.Compressed(codec, T, cl, *joint.enc[i], w_dec=Wl))
+        dec_low.append(torch.empty((T, H, d_low), dtype=torch.bfloat16, device=device))
+        dec_full.append(torch.empty((T, H, d), dtype=torch.bfloat16, device=device))
+    Pb = P.to(torch.bfloat16).contiguous()
+    Rb = P.transpose(1, 2).to(torch.bfloat16).contiguous()
+    o = torch.empty((Tq, H, d), dtype=torch.float32, device=device)
+    lse = torch.empty((H, Tq), dtype=torch.float32, device=device)
+    fws = K.fast_attention_workspace(H, d, d_low, Tq, device)
+    aws = K.alloc_workspace(K.KVQ_OP_ATTENTION, joint.codec[0], T, device, num_queries=Tq)
+    low_dec_ms = max_over_ranks(time_calls(lambda: [K.kvq_decode(lows[i], dec_low[i]) for i in range(2)], steps,
+                                           warmup, flush), world, device)
+    low_att_ms = max_over_ranks(time_calls(lambda: K.kvq_fast_attention_lse(q, dec_low[0], dec_low[1], Pb, Rb, o, lse,
+                                                                            fws), steps, warmup, flush), world, device)
+    full_dec_ms = max_over_ranks(time_calls(lambda: [K.kvq_decode(joint.comp[i], dec_full[i]) for i in range(2)],
+                                            steps, warmup, flush), world, device)
+    full_att_ms = max_over_ranks(time_calls(lambda: K.kvq_attention_dense_lse(q, dec_full[0], dec_full[1], o, lse,
+                                                                              workspace=aws), steps, warmup, flush),
+                                 world, device)
+    check_status(K, "after the NanoKV-Fast rows")
+    fl_low = 4.0 * Tq * T * d_low * H
+    fl_full = 4.0 * Tq * T * d * H
+    return {"nanokv_fast": {
+        "d_low": d_low, "decode_ms": low_dec_ms, "attention_ms": low_att_ms,
+        "attention_tflops": fl_low / (low_att_ms / 1e3) / 1e12,
+        "attention_frac": fl_low / (low_att_ms / 1e3) / 1e12 / tfl,
+        "full_decode_ms": full_dec_ms, "full_attention_ms": full_att_ms,
+        "full_attention_tflops": fl_full / (full_att_ms / 1e3) / 1e12,
+        "history_macs_ratio": d_low / d,
+        "what": "joint workload (32760 keys, 12 heads x 128, rank 192, INT4): low-space decode of K and V "
+                "(d_low = 64) + kvq_fast_attention_lse, beside the full decode + kvq_attention_dense_lse"}}
+
+
 def time_calls(fn, reps, warmup, flush):
     """Mean device time (ms) of fn() over reps calls, L2 flushed before each."""
     import torch
@@ -618,6 +730,8 @@ def run_gpu(args):
                                 "frac": dense_flops / (dense_ms / 1e3) / 1e12 / tfl,
                                 "what": "kvq_attention_dense_lse over the Wan-like 4680-key chunk alone"},
         }
+        next_rows.update(quantwm_rows(p2, args.steps, args.warmup, flush, world, device, tfl, hbm))
+        next_rows.update(fast_rows(joint, args.steps, args.warmup, flush, world, device, tfl))
         launches += p2.launches_per_step * args.steps
         del p2
         torch.cuda.empty_cache()

@@ -80,6 +80,8 @@ def parse_args():
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-secondary", action="store_true")
     p.add_argument("--sweep", default=None, help="write per-point sweep timings (JSON lines) to this path")
+    p.add_argument("--workload", default=HEADLINE, choices=["14b", "wan13b"],
+                   help="the step's workload (14b: the headline; wan13b: a smaller case for profiling)")
     return p.parse_args()
 
 
@@ -680,7 +682,7 @@ def run_gpu(args):
     flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=device)
 
     # ---- headline: the 14B-like layer, with the joint rows on their workload
-    w = synth.workload(HEADLINE)
+    w = synth.workload(args.workload)
     hk, hv, hq = (pinned_bf16(synth.make_history(w, "K")), pinned_bf16(synth.make_history(w, "V")),
                   pinned_bf16(synth.make_queries(w)))
     joint = JointRows(device)

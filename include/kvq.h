@@ -436,6 +436,22 @@ KVQ_API kvq_status kvq_lse_merge(int32_t n_parts, const float *const *o_parts, c
                          kvq_dtype o_dtype, float *lse_out, kvq_stream_t stream);
 
 /*
+ * Test hook for the give-up path of the bounded waits.  Sets, for the current
+ * device, how many times a waiting role of the encode filter (kvq_encode with
+ * a bf16 history and C <= 512, the fit's assignment passes) and of the d = 128
+ * attention kernels (kvq_attention_lse, kvq_attention_psac_lse, the dense and
+ * full-layer attention) polls an mbarrier before it gives up, raising
+ * KVQ_ERR_DEVICE_TIMEOUT in the status word and stopping the kernel's work
+ * (its outputs are then undefined).  KVQ_WAIT_LIMIT_DEFAULT (the value at load
+ * time, a wait of well under a few seconds) restores normal operation; 0 makes
+ * every such wait give up at once.  Waits that drain the kernel's own copies
+ * and tensor-core work before it exits are not affected.  Synchronous; applies
+ * to kernels launched afterwards.
+ */
+#define KVQ_WAIT_LIMIT_DEFAULT 4194304u
+KVQ_API kvq_status kvq_set_wait_limit(uint32_t polls);
+
+/*
  * Synchronise `stream`, then read and clear this device's status word.
  * Returns KVQ_ERR_DEVICE_TIMEOUT if any kernel since the last read gave up a
  * bounded wait (its outputs are then undefined), KVQ_ERR_CUDA if the stream

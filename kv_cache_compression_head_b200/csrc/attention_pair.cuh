@@ -122,7 +122,8 @@ __device__ __forceinline__ bool mbar_try_wait_cluster(uint32_t bar, uint32_t par
 
 __device__ __forceinline__ bool ap_wait(uint32_t bar, uint32_t parity, volatile int *abort)
 {
-    for (uint32_t i = 0; i < kSpinLimit; ++i) {
+    const uint32_t limit = c_wait_limit;
+    for (uint32_t i = 0; i < limit; ++i) {
         if (mbar_try_wait_cluster(bar, parity))
             return true;
         if ((i & 255u) == 255u && *abort)
@@ -131,6 +132,15 @@ __device__ __forceinline__ bool ap_wait(uint32_t bar, uint32_t parity, volatile 
     raise_status(DEVSTAT_TIMEOUT);
     *abort = 1;
     return false;
+}
+
+// After a give-up: wait (bounded, ignoring the abort flag) for the leader's
+// final commit, which it issues on every path once the CTA pair has work.
+__device__ __forceinline__ void ap_drain_ofull(uint32_t bar)
+{
+    uint32_t spins = 0;
+    while (!mbar_try_wait_cluster(bar, 0) && ++spins < kSpinLimit) {
+    }
 }
 
 __device__ __forceinline__ void umma2_ss(uint32_t d, uint64_t adesc, uint64_t bdesc, uint32_t idesc, uint32_t acc)
@@ -666,6 +676,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAPThreads, 1) atten
             __all_sync(0xffffffffu, ntiles > 0 && ok && ap_wait(bar(P_OFULL), 0, abort_flag));
         if (have)
             tc_fence_after();
+        else if (ntiles > 0)
+            ap_drain_ofull(bar(P_OFULL));  // the leader's last commit lands before this CTA exits
         const bool empty = !(l > 0.0f);
         const float inv_l = empty ? 0.0f : 1.0f / l;
 #pragma unroll 1

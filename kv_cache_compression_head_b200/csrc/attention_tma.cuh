@@ -653,6 +653,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kATThreads, 1)
             __all_sync(0xffffffffu, ntiles > 0 && ok && ap_wait(bar(P_OFULL), 0, abort_flag));
         if (have)
             tc_fence_after();
+        else if (ntiles > 0)
+            ap_drain_ofull(bar(P_OFULL));  // the leader's last commit lands before this CTA exits
         const bool empty = !(l > 0.0f);
         const float inv_l = empty ? 0.0f : 1.0f / l;
 #pragma unroll 1

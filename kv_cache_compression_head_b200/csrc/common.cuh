@@ -27,6 +27,12 @@ __device__ __forceinline__ void raise_status(unsigned bits) { atomicOr(&g_device
 // well under a few seconds.
 constexpr uint32_t kSpinLimit = 1u << 22;
 
+// Polls a give-up wait makes before it gives up: kSpinLimit unless lowered
+// through kvq_set_wait_limit, which a test uses to take the give-up path on
+// purpose.  The waits that drain copies and MMAs before a CTA exits keep
+// kSpinLimit, so a give-up never leaves asynchronous work in flight.
+__constant__ uint32_t c_wait_limit = kSpinLimit;
+
 // ---------------------------------------------------------------------------
 // small numeric helpers
 // ---------------------------------------------------------------------------

@@ -252,7 +252,8 @@ __device__ __forceinline__ void encode_residual_smem(const uint8_t *sX, const ui
 // the device status and sets the flag.
 __device__ __forceinline__ bool flt_wait(uint32_t bar, uint32_t parity, volatile int *abort)
 {
-    for (uint32_t i = 0; i < kSpinLimit; ++i) {
+    const uint32_t limit = c_wait_limit;
+    for (uint32_t i = 0; i < limit; ++i) {
         if (mbar_try_wait(bar, parity))
             return true;
         if ((i & 255u) == 255u && *abort)
@@ -409,6 +410,7 @@ __global__ void __launch_bounds__(kFltThreads, 1)
 
     int64_t tile_seq = 0;  // tiles this CTA has handled (X ring position, group = parity)
     uint32_t mma_issued = 0;
+    int64_t tma_last = -1;  // TMA lane: the last tile whose X load it issued
     for (int64_t u = u_begin; u < u_end;) {
         const int h = (int)(u / a.ntiles);
         const int64_t seg_end = min(u_end, (int64_t)(h + 1) * a.ntiles);
@@ -461,6 +463,7 @@ __global__ void __launch_bounds__(kFltThreads, 1)
 #pragma unroll
                     for (int ch = 0; ch < D / 64; ++ch)
                         tma_load_3d(dst + ch * (kFltRows * 128), &tmap_x, xfull(st), ch * 64, h, t0);
+                    tma_last = seq;
                 }
             }
         } else if (warp == kFltMmaWarp) {
@@ -687,7 +690,16 @@ __global__ void __launch_bounds__(kFltThreads, 1)
         tile_seq += n;
         u = seg_end;
     }
-    // drain: every MMA issued has completed before TMEM is freed
+    // drain: the X loads of the last tiles issued have landed (after a
+    // give-up nobody else waits for them) before the CTA may exit ...
+    if (warp == kFltTmaWarp && lane == 0) {
+        for (int64_t seq = tma_last - S + 1 < 0 ? 0 : tma_last - S + 1; seq <= tma_last; ++seq) {
+            uint32_t spins = 0;
+            while (!mbar_try_wait(xfull((int)(seq % S)), (uint32_t)((seq / S) & 1)) && ++spins < kSpinLimit) {
+            }
+        }
+    }
+    // ... and every MMA issued has completed before TMEM is freed
     if (warp == kFltMmaWarp && lane == 0 && mma_issued > 0) {
         umma_commit(bar_drain);
         uint32_t spins = 0;

@@ -1217,6 +1217,13 @@ bool fast_dims_ok(int d, int dl) { return supported_dim(d) && supported_dim(dl) 
 
 extern "C" {
 
+kvq_status kvq_set_wait_limit(uint32_t polls)
+{
+    if (cudaMemcpyToSymbol(c_wait_limit, &polls, sizeof polls) != cudaSuccess)
+        return KVQ_ERR_CUDA;
+    return KVQ_OK;
+}
+
 kvq_status kvq_fast_attention_workspace_size(int32_t H, int32_t d, int32_t d_low, int64_t Tq, size_t *bytes)
 {
     if (!bytes || H < 1 || Tq < 0)

@@ -44,6 +44,7 @@ EXPORTED = (
     "kvq_fit_centroids_static", "kvq_encode", "kvq_encode_qsac",
     "kvq_joint_coefficients", "kvq_decode", "kvq_psac_coefficients", "kvq_attention_lse", "kvq_attention_psac_lse",
     "kvq_attention_dense_lse", "kvq_fast_attention_lse", "kvq_fast_attention_workspace_size", "kvq_layer_attention",
+    "kvq_set_wait_limit",
     "kvq_lse_merge", "kvq_last_device_status",
 )
 
@@ -90,6 +91,7 @@ def _load():
         "kvq_fast_attention_lse": [vp, i64, vp, vp, i64, i32, i32, i32, vp, vp, i64, i64, ctypes.c_float, vp,
                                    ctypes.c_int, vp, vp, sz, vp],
         "kvq_fast_attention_workspace_size": [i32, i32, i32, i64, ctypes.POINTER(sz)],
+        "kvq_set_wait_limit": [ctypes.c_uint32],
         "kvq_attention_dense_lse": [vp, i64, vp, vp, i64, i32, i32, i64, i64, ctypes.c_float, vp, ctypes.c_int, vp,
                                     vp, sz, vp],
         "kvq_layer_attention": [vp, i64, pview, pview, i64, i64, vp, vp, i64, ctypes.c_float, vp, ctypes.c_int, vp,
@@ -404,6 +406,13 @@ def kvq_attention_lse(q: torch.Tensor, k: Compressed, v: Compressed, o_out: torc
 
 
 PSAC_RANK = 8
+KVQ_WAIT_LIMIT_DEFAULT = 4194304
+
+
+def kvq_set_wait_limit(polls: int) -> None:
+    """Test hook: polls before a bounded wait of the encode filter or the
+    d = 128 attention kernels gives up (KVQ_WAIT_LIMIT_DEFAULT restores)."""
+    _check(_lib.kvq_set_wait_limit(int(polls)), "kvq_set_wait_limit")
 
 
 def kvq_psac_coefficients(k: Compressed, x: torch.Tensor, U: torch.Tensor, coef_out: torch.Tensor,

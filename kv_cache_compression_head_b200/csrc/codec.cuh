@@ -308,15 +308,19 @@ __global__ void __launch_bounds__(kDirectTokens) encode_direct_kernel(EncodeArgs
         if (active) {
             for (int jj = 0; jj < nj; ++jj) {
                 const float4 *mu4 = reinterpret_cast<const float4 *>(s_mu + jj * D);
+                // e_c e_c of two channels at a time (packed binary32 operations
+                // round each lane as the scalar ones do), summed in channel order
                 float acc = 0.0f;
 #pragma unroll
                 for (int c4 = 0; c4 < D / 4; ++c4) {
                     const float4 m = mu4[c4];
-                    float e;
-                    e = __fsub_rn(xr[4 * c4 + 0], m.x); acc = __fadd_rn(acc, __fmul_rn(e, e));
-                    e = __fsub_rn(xr[4 * c4 + 1], m.y); acc = __fadd_rn(acc, __fmul_rn(e, e));
-                    e = __fsub_rn(xr[4 * c4 + 2], m.z); acc = __fadd_rn(acc, __fmul_rn(e, e));
-                    e = __fsub_rn(xr[4 * c4 + 3], m.w); acc = __fadd_rn(acc, __fmul_rn(e, e));
+                    const float2 e01 = sub2(make_float2(xr[4 * c4], xr[4 * c4 + 1]), make_float2(m.x, m.y));
+                    const float2 e23 = sub2(make_float2(xr[4 * c4 + 2], xr[4 * c4 + 3]), make_float2(m.z, m.w));
+                    const float2 q01 = mul2(e01, e01), q23 = mul2(e23, e23);
+                    acc = __fadd_rn(acc, q01.x);
+                    acc = __fadd_rn(acc, q01.y);
+                    acc = __fadd_rn(acc, q23.x);
+                    acc = __fadd_rn(acc, q23.y);
                 }
                 const int j = j0 + jj;
                 if (j == 0 || acc < best) {
@@ -410,16 +414,21 @@ __global__ void __launch_bounds__(kDirectTokens) qsac_encode_kernel(QsacArgs q)
             for (int jj = 0; jj < nj; ++jj) {
                 const float4 *mu4 = reinterpret_cast<const float4 *>(s_mu + jj * D);
                 const float4 *w4 = reinterpret_cast<const float4 *>(s_w);
+                // the terms w_c (e_c e_c) of two channels at a time (packed
+                // binary32 operations round each lane as the scalar ones do),
+                // summed one by one in channel order
                 float acc = 0.0f;
 #pragma unroll
                 for (int c4 = 0; c4 < D / 4; ++c4) {
                     const float4 mv = mu4[c4], wv = w4[c4];
-                    const float mm[4] = {mv.x, mv.y, mv.z, mv.w}, ww[4] = {wv.x, wv.y, wv.z, wv.w};
-#pragma unroll
-                    for (int k = 0; k < 4; ++k) {
-                        const float e = __fsub_rn(xr[4 * c4 + k], mm[k]);
-                        acc = __fadd_rn(acc, __fmul_rn(ww[k], __fmul_rn(e, e)));
-                    }
+                    const float2 e01 = sub2(make_float2(xr[4 * c4], xr[4 * c4 + 1]), make_float2(mv.x, mv.y));
+                    const float2 e23 = sub2(make_float2(xr[4 * c4 + 2], xr[4 * c4 + 3]), make_float2(mv.z, mv.w));
+                    const float2 t01 = mul2(make_float2(wv.x, wv.y), mul2(e01, e01));
+                    const float2 t23 = mul2(make_float2(wv.z, wv.w), mul2(e23, e23));
+                    acc = __fadd_rn(acc, t01.x);
+                    acc = __fadd_rn(acc, t01.y);
+                    acc = __fadd_rn(acc, t23.x);
+                    acc = __fadd_rn(acc, t23.y);
                 }
                 const int j = j0 + jj;
                 // insert (acc, j) into the ascending lists (an empty slot

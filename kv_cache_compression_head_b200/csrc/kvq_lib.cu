@@ -598,14 +598,21 @@ kvq_status launch_attention_tma_t(const AttnArgs &a, cudaStream_t s)
     return launch_status();
 }
 
+// The compressed d = 128 history goes to the TMA-staged kernel when its row
+// coordinates fit the 32-bit tensor-map coordinates and the range is not empty.
+bool uses_tma_attention(const AttnArgs &a, int D)
+{
+    return D == 128 && !a.dense && a.t_end > a.t_begin && (int64_t)a.H * a.k.T < (int64_t)INT32_MAX &&
+           (int64_t)a.H * (a.k.C > a.v.C ? a.k.C : a.v.C) < (int64_t)INT32_MAX;
+}
+
 kvq_status launch_attention_pair(const AttnArgs &a, cudaStream_t s)
 {
     if (a.dense)
         return launch_attention_pair_t<0, 0, true>(a, s);
     // compressed history with keys to read: every byte staged by TMA (row
     // coordinates are 32-bit); an empty range needs no staging
-    if (a.t_end > a.t_begin && (int64_t)a.H * a.k.T < (int64_t)INT32_MAX &&
-        (int64_t)a.H * (a.k.C > a.v.C ? a.k.C : a.v.C) < (int64_t)INT32_MAX) {
+    if (uses_tma_attention(a, 128)) {
         if (a.k.bits == 2)
             return a.v.bits == 2 ? launch_attention_tma_t<2, 2>(a, s) : launch_attention_tma_t<2, 4>(a, s);
         return a.v.bits == 2 ? launch_attention_tma_t<4, 2>(a, s) : launch_attention_tma_t<4, 4>(a, s);

@@ -13,6 +13,10 @@ the joint workload.
   a 131,072-token history.
 * joint workload: the decoder at full size (32,760 tokens, both branches,
   K4V4 rank 192) on sampled tokens, within the decoder's derived bound.
+* the next rows at the sizes the benchmark times them: QSAC encode of the
+  whole Wan-like K history (sampled tiles, bit-exact), PSAC attention over the
+  whole Wan-like history in 2 blocks merged by LSE (512 rows per head), and
+  NanoKV-Fast on the whole joint workload (512 rows per head).
 """
 
 import numpy as np
@@ -205,3 +209,106 @@ def test_joint_decode_full_size_sampled():
 
 def _widen(bits: np.ndarray) -> np.ndarray:
     return synth.bf16_bits_to_f32(bits).astype(np.float64)
+
+
+# ---------------------------------------------------------------------------
+# the next rows at the sizes the benchmark times them
+# ---------------------------------------------------------------------------
+
+@pytest.fixture(scope="module")
+def wan_full():
+    w = synth.workload("wan13b")
+    return w, synth.make_history(w, "K"), synth.make_history(w, "V"), synth.make_queries(w)
+
+
+def test_qsac_full_size_sampled(wan_full):
+    """QSAC encode (M = 4) of the whole Wan-like K history (32,760 x 12,
+    C = 256, INT2 G16, weights from the chunk's queries), bit-exact on a
+    seeded 1/16 of the tiles of every head."""
+    K = _K()
+    w, xk, _, q = wan_full
+    T, H, d = xk.shape
+    C, G = w.num_centroids, w.group_size
+    cent = O.fit(xk[:C], C, 0)
+    wts = O.qsac_weights(O.query_moments(q), H, d)
+    codec = K.Codec(H, d, C, w.bits_k, G)
+    idx, codes, meta = K.alloc_encoded(codec, T, "cuda")
+    K.kvq_encode_qsac(codec, to_dev(xk), to_dev(cent), to_dev(wts), idx, codes, meta, M=4)
+    assert K.kvq_last_device_status() == K.KVQ_OK
+    toks = _tiles_sample(T, 1.0 / 16, 21)
+    idx_r, codes_r, meta_r = O.qsac_encode(np.ascontiguousarray(xk[toks]), cent, wts, w.bits_k, G, 4)
+    assert np.array_equal(bits_u16(idx).reshape(H, T)[:, toks], idx_r)
+    assert np.array_equal(u8(codes).reshape(H, T, d * w.bits_k // 8)[:, toks], codes_r)
+    assert np.array_equal(f32_bits(meta).reshape(H, T, d // G, 2)[:, toks], f32_bits(meta_r))
+
+
+def test_psac_attention_full_size_sampled(wan_full):
+    """PSAC attention over the whole Wan-like history in the benchmark's 2
+    blocks (split calls, merged by LSE), fed the oracle's coefficients, on 512
+    query rows of every head."""
+    K = _K()
+    w, xk, xv, q = wan_full
+    T, H, d = xk.shape
+    C, G = w.num_centroids, w.group_size
+    comps, decs = [], []
+    for x, bits in ((xk, w.bits_k), (xv, w.bits_v)):
+        cent = O.fit(x[:C], C, 0)
+        codec = K.Codec(H, d, C, bits, G)
+        comps.append(_gpu_encode(codec, to_dev(x), cent))
+        decs.append(O.decode(*O.encode(x, cent, bits, G), cent, bits, G))
+    U = O.psac_basis(O.query_moments(q), 8).astype(np.float32)
+    coef = O.psac_coefficients(xk, decs[0], U.astype(np.float64))
+    coef_d = to_dev(np.ascontiguousarray(coef.transpose(1, 0, 2)))
+    qd, Ud = to_dev(q), to_dev(U)
+    ws = K.alloc_workspace(K.KVQ_OP_ATTENTION, comps[0].codec, T, "cuda", num_queries=q.shape[0])
+    edges = [0, T // 2, T]
+    parts = []
+    for a, b in zip(edges[:-1], edges[1:]):
+        o = torch.empty(q.shape, dtype=torch.float32, device="cuda")
+        lse = torch.empty((H, q.shape[0]), dtype=torch.float32, device="cuda")
+        K.kvq_attention_psac_lse(qd, comps[0], comps[1], Ud, coef_d, o, lse, t_begin=a, t_end=b, workspace=ws)
+        parts.append((o, lse))
+    om, lm = torch.empty_like(parts[0][0]), torch.empty_like(parts[0][1])
+    K.kvq_lse_merge([p[0] for p in parts], [p[1] for p in parts], om, lm)
+    assert K.kvq_last_device_status() == K.KVQ_OK
+    rows = _rows_sample(q.shape[0], 512, 22)
+    o_ref, lse_ref = O.attention_psac(q, decs[0], decs[1], U.astype(np.float64), coef, rows=rows)
+    assert_attention_close(om.cpu().numpy()[rows], lm.cpu().numpy()[:, rows], o_ref, lse_ref, "psac full size")
+
+
+def test_fast_attention_full_size_sampled():
+    """NanoKV-Fast on the whole joint workload (32,760 keys, 12 heads, 4,680
+    queries, d_low = 64): the GPU decodes both branches into the low space,
+    then attends there; 512 query rows of every head against the oracle's
+    low-space decode and fast_attention."""
+    K = _K()
+    w = synth.workload("joint")
+    H, d, r, G, C = w.num_heads, w.head_dim, w.joint_rank, w.joint_group, w.num_centroids
+    dl = 64
+    w_enc = synth.make_orthonormal_encoder(w)
+    w_dec = np.ascontiguousarray(w_enc.T)
+    q = synth.make_queries(w)
+    lows, lows_ref, Ps = [], [], []
+    for which, bits in (("K", w.bits_k), ("V", w.bits_v)):
+        x = synth.make_history(w, which)
+        T = x.shape[0]
+        cent = O.fit(x[:C], C, 0)
+        idx, codes, meta, _ = O.joint_encode(x, cent, w_enc, bits, G)
+        P, W_low, c_low = O.fast_maps_analytical(w_dec, cent, dl)
+        Pb, Wb, cb = O.bf16_bits(P), O.bf16_bits(W_low), O.bf16_bits(c_low)
+        lows_ref.append(O.bf16_bits(O.joint_decode(idx, codes, meta, cb, Wb, bits, G)))
+        comp = K.Compressed(K.Codec(H, dl, C, bits, G, r), T, to_dev(cb), to_dev(idx.view(np.int16)),
+                            to_dev(codes), to_dev(meta), w_dec=to_dev(Wb))
+        out = torch.empty((T, H, dl), dtype=torch.bfloat16, device="cuda")
+        K.kvq_decode(comp, out)
+        lows.append(out)
+        Ps.append(Pb)
+    R = np.ascontiguousarray(np.transpose(Ps[1], (0, 2, 1)))
+    o = torch.empty((q.shape[0], H, d), dtype=torch.float32, device="cuda")
+    lse = torch.empty((H, q.shape[0]), dtype=torch.float32, device="cuda")
+    K.kvq_fast_attention_lse(to_dev(q), lows[0], lows[1], to_dev(Ps[0]), to_dev(R), o, lse,
+                             K.fast_attention_workspace(H, d, dl, q.shape[0], "cuda"))
+    assert K.kvq_last_device_status() == K.KVQ_OK
+    rows = _rows_sample(q.shape[0], 512, 23)
+    o_ref, lse_ref = O.fast_attention(q, lows_ref[0], lows_ref[1], Ps[0], R, rows=rows)
+    assert_attention_close(o.cpu().numpy()[rows], lse.cpu().numpy()[:, rows], o_ref, lse_ref, "fast full size")

@@ -93,7 +93,7 @@ __global__ void __launch_bounds__(kFastThreads) fast_map_kernel(FastMapArgs a)
     const int64_t row = t * a.H + h;
     const void *in_row = IN_BF16 ? static_cast<const void *>(static_cast<const uint16_t *>(a.in) + row * DIN)
                                  : static_cast<const void *>(static_cast<const float *>(a.in) + row * DIN);
-    if (IN_BF16) {
+    if constexpr (IN_BF16) {
 #pragma unroll 1
         for (int o0 = 0; o0 < DOUT; o0 += 32) {
             double acc[32];
@@ -126,8 +126,7 @@ __global__ void __launch_bounds__(kFastThreads) fast_map_kernel(FastMapArgs a)
                                      pack_bf16x2(round_odd_f32(acc[8 * j8 + 4]), round_odd_f32(acc[8 * j8 + 5])),
                                      pack_bf16x2(round_odd_f32(acc[8 * j8 + 6]), round_odd_f32(acc[8 * j8 + 7])));
         }
-        return;
-    }
+    } else {
 #pragma unroll 1
     for (int o0 = 0; o0 < DOUT; o0 += 64) {
         float acc[64];
@@ -165,6 +164,7 @@ __global__ void __launch_bounds__(kFastThreads) fast_map_kernel(FastMapArgs a)
             for (int j4 = 0; j4 < 16; ++j4)
                 dst[j4] = make_float4(acc[4 * j4], acc[4 * j4 + 1], acc[4 * j4 + 2], acc[4 * j4 + 3]);
         }
+    }
     }
 }
 

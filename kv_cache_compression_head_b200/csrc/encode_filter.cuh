@@ -222,15 +222,27 @@ __device__ __forceinline__ void encode_residual_smem(const uint8_t *sX, const ui
         words[w] = 0u;
 #pragma unroll
     for (int g = 0; g < NG; ++g) {
+        if (gf[g].fast) {  // one branch per group, not per value
 #pragma unroll
-        for (int uu = 0; uu < G / 8; ++uu) {
-            float r8[8];
-            unit_residual(g * (G / 8) + uu, r8);
+            for (int uu = 0; uu < G / 8; ++uu) {
+                float r8[8];
+                unit_residual(g * (G / 8) + uu, r8);
 #pragma unroll
-            for (int k = 0; k < 8; ++k) {
-                const int c = g * G + uu * 8 + k;
-                words[c / kPerWord] += (gf[g].fast ? quant_code_fast<BITS>(r8[k], gf[g]) : quant_code(r8[k], gq[g], BITS))
-                                       << ((c % kPerWord) * BITS);
+                for (int k = 0; k < 8; ++k) {
+                    const int c = g * G + uu * 8 + k;
+                    words[c / kPerWord] += quant_code_fast<BITS>(r8[k], gf[g]) << ((c % kPerWord) * BITS);
+                }
+            }
+        } else {
+#pragma unroll
+            for (int uu = 0; uu < G / 8; ++uu) {
+                float r8[8];
+                unit_residual(g * (G / 8) + uu, r8);
+#pragma unroll
+                for (int k = 0; k < 8; ++k) {
+                    const int c = g * G + uu * 8 + k;
+                    words[c / kPerWord] += quant_code(r8[k], gq[g], BITS) << ((c % kPerWord) * BITS);
+                }
             }
         }
     }

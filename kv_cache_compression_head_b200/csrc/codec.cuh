@@ -723,6 +723,8 @@ struct FitSortArgs {
     unsigned *abs_min;       // [H] bits of the smallest nonzero |x| (+inf: none)
     int *redo;               // [H][C]
     int track;               // segsum also updates abs_max / abs_min
+    unsigned *bkt_max;       // [H][C] bits of the largest |x| of the round's bucket
+    unsigned *bkt_minv;      // [H][C] ~bits of its smallest nonzero |x| (0: none)
 };
 
 // mu_j = bf16(x_j) for the first C tokens; the update totals start cleared.
@@ -742,8 +744,11 @@ __global__ void __launch_bounds__(256) fit_seed_kernel(FitArgs a, FitSortArgs fs
     const __nv_bfloat16 b = __float2bfloat16_rn(v);
     a.cent[gid] = *reinterpret_cast<const uint16_t *>(&b);
     fs.sums[gid] = 0.0;
-    if (c == 0)
+    if (c == 0) {
         fs.redo[hj] = 0;
+        fs.bkt_max[hj] = 0u;
+        fs.bkt_minv[hj] = 0u;
+    }
     if (c == 0 && j == 0) {
         fs.abs_max[h] = 0u;
         fs.abs_min[h] = 0x7f800000u;
@@ -916,6 +921,7 @@ __global__ void __launch_bounds__(256) fit_segsum_kernel(FitSortArgs a)
 
     double acc[kPer];
     unsigned amax = 0u, amin = 0x7f800000u;
+    unsigned rmax = 0u, rmin = 0x7f800000u;  // |x| bounds of the current run (bucket)
     int cur = -1;
 #pragma unroll
     for (int k = 0; k < kPer; ++k)
@@ -927,6 +933,15 @@ __global__ void __launch_bounds__(256) fit_segsum_kernel(FitSortArgs a)
             atomicAdd(dst + k, acc[k]);
             acc[k] = 0.0;
         }
+        // the run's bounds join the bucket's (the run is the whole warp's)
+        const unsigned bmax = __reduce_max_sync(0xffffffffu, rmax);
+        const unsigned bmin = __reduce_min_sync(0xffffffffu, rmin);
+        if (lane == 0) {
+            atomicMax(a.bkt_max + (int64_t)h * a.C + cur, bmax);
+            atomicMax(a.bkt_minv + (int64_t)h * a.C + cur, ~bmin);
+        }
+        rmax = 0u;
+        rmin = 0x7f800000u;
     };
     // the next 32 slots' token ids are fetched one round ahead; a round's rows
     // are requested before its centre indices are consumed
@@ -963,8 +978,10 @@ __global__ void __launch_bounds__(256) fit_segsum_kernel(FitSortArgs a)
 #pragma unroll
                 for (int k = 0; k < kPer; ++k) {
                     acc[k] = __dadd_rn(acc[k], (double)v[b][k]);
+                    const unsigned u = __float_as_uint(v[b][k]) & 0x7fffffffu;
+                    rmax = max(rmax, u);
+                    rmin = min(rmin, u ? u : 0x7f800000u);
                     if (a.track) {
-                        const unsigned u = __float_as_uint(v[b][k]) & 0x7fffffffu;
                         amax = max(amax, u);
                         amin = min(amin, u ? u : 0x7f800000u);
                     }
@@ -1000,11 +1017,16 @@ __global__ void __launch_bounds__(256) fit_finalize_kernel(FitSortArgs a)
     const int64_t hj = (int64_t)h * a.C + j;
     const int *bs = a.bucket_start + (int64_t)h * (a.C + 1);
     const int n = bs[j + 1] - bs[j];
-    // every partial sum is a multiple of 2^L below 2^(53 + L) in magnitude
+    // every partial sum is a multiple of 2^L below 2^(53 + L) in magnitude,
+    // L from the head's smallest nonzero |x| or from the bucket's own (every
+    // value is a multiple of its own ulp, hence of that of the smallest)
     const unsigned amin = a.abs_min[h];
     const int L = (int)(amin >> 23) - (a.x_bf16 ? 134 : 150);
+    const unsigned bmin = ~a.bkt_minv[hj];
+    const int Lb = (int)(bmin >> 23) - (a.x_bf16 ? 134 : 150);
     const bool exact =
-        amin >= 0x7f800000u || (double)n * (double)__uint_as_float(a.abs_max[h]) <= ldexp(1.0, 52 + L);
+        amin >= 0x7f800000u || (double)n * (double)__uint_as_float(a.abs_max[h]) <= ldexp(1.0, 52 + L) ||
+        bmin >= 0x7f800000u || (double)n * (double)__uint_as_float(a.bkt_max[hj]) <= ldexp(1.0, 52 + Lb);
     double *sum = a.sums + hj * D + lane * kPer;
     if (n > 0 && exact) {
         uint16_t *dst = a.cent + hj * D + lane * kPer;
@@ -1017,8 +1039,12 @@ __global__ void __launch_bounds__(256) fit_finalize_kernel(FitSortArgs a)
 #pragma unroll
     for (int k = 0; k < kPer; ++k)
         sum[k] = 0.0;
-    if (lane == 0)
+    __syncwarp();  // every lane has read the bucket's bounds
+    if (lane == 0) {
         a.redo[hj] = (n > 0 && !exact) ? 1 : 0;
+        a.bkt_max[hj] = 0u;
+        a.bkt_minv[hj] = 0u;
+    }
 }
 
 // One warp per (head, centre) marked by fit_finalize; lane l owns channels

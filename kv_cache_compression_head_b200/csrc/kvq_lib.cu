@@ -391,7 +391,7 @@ kvq_status joint_encode_call(const kvq_codec_desc *desc, const void *x, kvq_dtyp
 // Fit workspace: idx [H][T] u16 | per-chunk centre counts [H][nch][C] i32 |
 // bucket starts [H][C+1] i32 | token order [H][T] i32.
 struct FitLayout {
-    size_t idx, counts, starts, order, sums, bounds, redo, total;
+    size_t idx, counts, starts, order, sums, bounds, redo, bkt, total;
     int nchunks;
 };
 
@@ -409,7 +409,8 @@ FitLayout fit_layout(const kvq_codec_desc *d, int64_t T)
     L.sums = L.order + round_up(H * (size_t)T * 4, 256);
     L.bounds = L.sums + round_up(H * C * (size_t)d->head_dim * 8, 256);
     L.redo = L.bounds + round_up(H * 8, 256);
-    L.total = L.redo + H * C * 4;
+    L.bkt = L.redo + round_up(H * C * 4, 256);
+    L.total = L.bkt + H * C * 8;
     return L;
 }
 
@@ -849,6 +850,8 @@ kvq_status kvq_fit_centroids(const kvq_codec_desc *desc, const void *x, kvq_dtyp
     fs.abs_min = fs.abs_max + H;
     fs.track = 1;
     fs.redo = reinterpret_cast<int *>(ws + Lw.redo);
+    fs.bkt_max = reinterpret_cast<unsigned *>(ws + Lw.bkt);
+    fs.bkt_minv = fs.bkt_max + (size_t)H * C;
 
     const int64_t n_cent = (int64_t)H * C * D;
     fit_seed_kernel<<<(unsigned)ceil_div(n_cent, 256), 256, 0, s>>>(f, fs);

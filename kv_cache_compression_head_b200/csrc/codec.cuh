@@ -306,26 +306,37 @@ __global__ void __launch_bounds__(kDirectTokens) encode_direct_kernel(EncodeArgs
             load_bf16x8(cent_h + (int64_t)j0 * D + e, s_mu + e);
         __syncthreads();
         if (active) {
-            for (int jj = 0; jj < nj; ++jj) {
-                const float4 *mu4 = reinterpret_cast<const float4 *>(s_mu + jj * D);
-                // e_c e_c of two channels at a time (packed binary32 operations
-                // round each lane as the scalar ones do), summed in channel order
-                float acc = 0.0f;
+            // four centres at a time: four independent sequential sums keep
+            // the adders busy (each sum alone is one dependent chain of D adds)
+            for (int jq = 0; jq < nj; jq += 4) {
+                float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
 #pragma unroll
                 for (int c4 = 0; c4 < D / 4; ++c4) {
-                    const float4 m = mu4[c4];
-                    const float2 e01 = sub2(make_float2(xr[4 * c4], xr[4 * c4 + 1]), make_float2(m.x, m.y));
-                    const float2 e23 = sub2(make_float2(xr[4 * c4 + 2], xr[4 * c4 + 3]), make_float2(m.z, m.w));
-                    const float2 q01 = mul2(e01, e01), q23 = mul2(e23, e23);
-                    acc = __fadd_rn(acc, q01.x);
-                    acc = __fadd_rn(acc, q01.y);
-                    acc = __fadd_rn(acc, q23.x);
-                    acc = __fadd_rn(acc, q23.y);
+                    const float2 x01 = make_float2(xr[4 * c4], xr[4 * c4 + 1]);
+                    const float2 x23 = make_float2(xr[4 * c4 + 2], xr[4 * c4 + 3]);
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        // rows past nj hold stale centres of the chunk buffer; their sums are dropped
+                        const float4 m = reinterpret_cast<const float4 *>(s_mu + (jq + q) * D)[c4];
+                        // e_c e_c of two channels at a time (packed binary32
+                        // operations round each lane as the scalar ones do),
+                        // summed in channel order
+                        const float2 e01 = sub2(x01, make_float2(m.x, m.y));
+                        const float2 e23 = sub2(x23, make_float2(m.z, m.w));
+                        const float2 q01 = mul2(e01, e01), q23 = mul2(e23, e23);
+                        acc[q] = __fadd_rn(acc[q], q01.x);
+                        acc[q] = __fadd_rn(acc[q], q01.y);
+                        acc[q] = __fadd_rn(acc[q], q23.x);
+                        acc[q] = __fadd_rn(acc[q], q23.y);
+                    }
                 }
-                const int j = j0 + jj;
-                if (j == 0 || acc < best) {
-                    best = acc;
-                    best_j = j;
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    const int j = j0 + jq + q;
+                    if (jq + q < nj && (j == 0 || acc[q] < best)) {
+                        best = acc[q];
+                        best_j = j;
+                    }
                 }
             }
         }

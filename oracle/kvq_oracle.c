@@ -56,6 +56,12 @@
  *    codes 0, which decodes to exactly min (and to 0 when min == 0);
  *  - decode: x^_c = mu_c + (q_c - z) * s with the subtraction, multiply and
  *    add each rounded to binary32;
+ *  - second residual stage (QVG's progressive residual quantisation, named
+ *    by TempoKV, Sec. 2, without its steps; NanoKV page, Table 4 evaluates
+ *    QVG with one stage): stage 2 quantises what stage 1 leaves,
+ *    e_c = r_c - (q1_c - z1) s1 (binary32), with Eq. 1 on the same groups and
+ *    bit width; decode x^_c = (mu_c + (q1_c - z1) s1) + (q2_c - z2) s2, each
+ *    operation rounded to binary32;
  *  - compact {s, z} (16-bit scale and zero per group, the b + 1 bits per value
  *    of TempoKV, Table 1, at G = 32): s is formed as above, then rounded to
  *    binary16 (nearest, ties to even, magnitudes past the largest finite
@@ -622,6 +628,112 @@ int kvqo_decode16(const uint16_t *idx, const uint8_t *codes, const uint16_t *met
             }
         }
         free(q);
+    }
+    return rc;
+}
+
+/* ------------------------------------------------------------------------ */
+/* second residual stage                                                     */
+/* ------------------------------------------------------------------------ */
+
+/*
+ * kvqo_encode followed by a second stage: idx, codes and meta exactly as
+ * kvqo_encode writes them; then, per group, the stage-1 error
+ * e = r - (q1 - z1) s1 and its Eq. 1 form in codes2 [H][T][d*bits/8] and
+ * meta2 [H][T][d/G][2].
+ */
+int kvqo_encode2(const void *x, int x_is_bf16, int64_t T, int H, int d, const uint16_t *cent, int C, int bits,
+                 int G, uint16_t *idx, uint8_t *codes, float *meta, uint8_t *codes2, float *meta2)
+{
+    if (T < 0 || !check_codec(H, d, C, bits, G))
+        return KVQO_EINVAL;
+    const int cb = d * bits / 8, ng = d / G;
+    int rc = KVQO_OK;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int h = 0; h < H; ++h) {
+        float *mu = (float *)malloc(sizeof(float) * (size_t)C * d);
+        float *xv = (float *)malloc(sizeof(float) * (size_t)d);
+        float *r = (float *)malloc(sizeof(float) * (size_t)d);
+        float *e = (float *)malloc(sizeof(float) * (size_t)d);
+        uint8_t *q = (uint8_t *)malloc((size_t)d);
+        if (!mu || !xv || !r || !e || !q) {
+            rc = KVQO_ENOMEM;
+        } else {
+            widen_centres(cent + (int64_t)h * C * d, C, d, mu);
+            for (int64_t t = 0; t < T; ++t) {
+                int64_t th = (int64_t)h * T + t;
+                gather_token(x, x_is_bf16, H, d, t, h, xv);
+                int j = nearest(xv, mu, C, d, NULL);
+                idx[th] = (uint16_t)j;
+                for (int c = 0; c < d; ++c)
+                    r[c] = xv[c] - mu[(int64_t)j * d + c];
+                /* stage 1 */
+                for (int g = 0; g < ng; ++g) {
+                    float s1, z1;
+                    kvqo_quant_group(r + g * G, G, bits, &s1, &z1, q + g * G);
+                    meta[(th * ng + g) * 2 + 0] = s1;
+                    meta[(th * ng + g) * 2 + 1] = z1;
+                    for (int c = g * G; c < (g + 1) * G; ++c)
+                        e[c] = r[c] - kvqo_dequant(q[c], s1, z1);
+                }
+                kvqo_pack(q, d, bits, codes + th * cb);
+                /* stage 2: the error stage 1 leaves */
+                for (int g = 0; g < ng; ++g) {
+                    float s2, z2;
+                    kvqo_quant_group(e + g * G, G, bits, &s2, &z2, q + g * G);
+                    meta2[(th * ng + g) * 2 + 0] = s2;
+                    meta2[(th * ng + g) * 2 + 1] = z2;
+                }
+                kvqo_pack(q, d, bits, codes2 + th * cb);
+            }
+        }
+        free(mu);
+        free(xv);
+        free(r);
+        free(e);
+        free(q);
+    }
+    return rc;
+}
+
+/* Reconstruction from both stages: (mu + (q1 - z1) s1) + (q2 - z2) s2. */
+int kvqo_decode2(const uint16_t *idx, const uint8_t *codes, const float *meta, const uint8_t *codes2,
+                 const float *meta2, const uint16_t *cent, int64_t T, int H, int d, int C, int bits, int G,
+                 float *out)
+{
+    if (T < 0 || !check_codec(H, d, C, bits, G))
+        return KVQO_EINVAL;
+    const int cb = d * bits / 8, ng = d / G;
+    int rc = KVQO_OK;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int h = 0; h < H; ++h) {
+        uint8_t *q1 = (uint8_t *)malloc((size_t)d);
+        uint8_t *q2 = (uint8_t *)malloc((size_t)d);
+        if (!q1 || !q2) {
+            rc = KVQO_ENOMEM;
+            free(q1);
+            free(q2);
+            continue;
+        }
+        for (int64_t t = 0; t < T; ++t) {
+            int64_t th = (int64_t)h * T + t;
+            int j = idx[th];
+            if (j >= C) {
+                rc = KVQO_EINVAL;
+                break;
+            }
+            kvqo_unpack(codes + th * cb, d, bits, q1);
+            kvqo_unpack(codes2 + th * cb, d, bits, q2);
+            for (int c = 0; c < d; ++c) {
+                int g = c / G;
+                float mu = bf16_widen(cent[((int64_t)h * C + j) * d + c]);
+                float stage1 = mu + kvqo_dequant(q1[c], meta[(th * ng + g) * 2], meta[(th * ng + g) * 2 + 1]);
+                out[(t * H + h) * (int64_t)d + c] =
+                    stage1 + kvqo_dequant(q2[c], meta2[(th * ng + g) * 2], meta2[(th * ng + g) * 2 + 1]);
+            }
+        }
+        free(q1);
+        free(q2);
     }
     return rc;
 }

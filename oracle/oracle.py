@@ -11,6 +11,9 @@ Functions and the passages they follow:
 * ``assign``, ``fit``, ``encode``, ``decode``: centroid-residual codec -- see
   the header of kvq_oracle.c (QuantWM Sec. 4.1; TempoKV Sec. 3.1 Eq. 1 and
   Sec. 3.3 Eq. 2; CORAL-KV Sec. 2; NanoKV page Tables 4-5).
+* ``encode2``, ``decode2``: a second residual stage (QVG's progressive
+  residual quantisation, named by TempoKV Sec. 2; the reading in the header
+  of kvq_oracle.c).
 * ``joint_encode``, ``joint_decode``, ``quant_rows``: joint head-channel
   encoder/decoder with INT4 coefficients (NanoKV page, abstract, Fig. 4(b)).
 * ``attention``: softmax attention of the current chunk's queries over the
@@ -70,6 +73,8 @@ def _load():
     lib.kvqo_fit.argtypes = [vp, i32, i64, i32, i32, i32, i32, vp, vp]
     lib.kvqo_encode.argtypes = [vp, i32, i64, i32, i32, vp, i32, i32, i32, vp, vp, vp]
     lib.kvqo_decode.argtypes = [vp, vp, vp, vp, i64, i32, i32, i32, i32, i32, vp]
+    lib.kvqo_encode2.argtypes = [vp, i32, i64, i32, i32, vp, i32, i32, i32, vp, vp, vp, vp, vp]
+    lib.kvqo_decode2.argtypes = [vp, vp, vp, vp, vp, vp, i64, i32, i32, i32, i32, i32, vp]
     lib.kvqo_quant_rows.argtypes = [vp, i64, i32, i32, i32, vp, vp]
     lib.kvqo_joint_encode.argtypes = [vp, i32, i64, i32, i32, vp, i32, vp, i32, i32, i32, vp, vp, vp, vp]
     lib.kvqo_joint_decode.argtypes = [vp, vp, vp, vp, vp, i64, i32, i32, i32, i32, i32, i32, vp]
@@ -242,6 +247,34 @@ def decode16(idx: np.ndarray, codes: np.ndarray, meta16: np.ndarray, cent: np.nd
     out = np.zeros((T, H, d), np.float32)
     args = [np.ascontiguousarray(a) for a in (idx, codes, meta16, cent)]
     _check(_load().kvqo_decode16(*(_ptr(a) for a in args), T, H, d, C, bits, group, _ptr(out)), "decode16")
+    return out
+
+
+def encode2(x: np.ndarray, cent: np.ndarray, bits: int, group: int):
+    """encode with a second residual stage: (idx, codes, meta, codes2, meta2);
+    the first three exactly as ``encode``, the stage-2 arrays in the same
+    layouts (the reading in kvq_oracle.c's header)."""
+    x, xb = _x_arg(x)
+    T, H, d = x.shape
+    C = cent.shape[1]
+    cent = np.ascontiguousarray(cent, dtype=np.uint16)
+    idx = np.zeros((H, T), np.uint16)
+    codes = np.zeros((H, T, d * bits // 8), np.uint8)
+    meta = np.zeros((H, T, d // group, 2), np.float32)
+    codes2 = np.zeros_like(codes)
+    meta2 = np.zeros_like(meta)
+    _check(_load().kvqo_encode2(_ptr(x), xb, T, H, d, _ptr(cent), C, bits, group, _ptr(idx), _ptr(codes),
+                                _ptr(meta), _ptr(codes2), _ptr(meta2)), "encode2")
+    return idx, codes, meta, codes2, meta2
+
+
+def decode2(idx, codes, meta, codes2, meta2, cent, bits: int, group: int) -> np.ndarray:
+    """Reconstruction [T][H][d] float32 from both residual stages."""
+    H, T = idx.shape
+    C, d = cent.shape[1], cent.shape[2]
+    out = np.zeros((T, H, d), np.float32)
+    args = [np.ascontiguousarray(a) for a in (idx, codes, meta, codes2, meta2, cent)]
+    _check(_load().kvqo_decode2(*(_ptr(a) for a in args), T, H, d, C, bits, group, _ptr(out)), "decode2")
     return out
 
 

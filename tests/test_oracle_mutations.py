@@ -44,6 +44,12 @@ MUTATIONS = [
     ("QSAC score ties to the worse-ranked candidate", "if (k == 0 || sc < best) {", "if (k == 0 || sc <= best) {"),
     ("QSAC ranking ties to the higher index", "while (pos > 0 && dj < cand_dist[pos - 1])",
      "while (pos > 0 && dj <= cand_dist[pos - 1])"),
+    ("second stage error with the wrong sign", "e[c] = r[c] - kvqo_dequant(q[c], s1, z1);",
+     "e[c] = kvqo_dequant(q[c], s1, z1) - r[c];"),
+    ("second stage quantises the residual again", "kvqo_quant_group(e + g * G, G, bits, &s2, &z2, q + g * G);",
+     "kvqo_quant_group(r + g * G, G, bits, &s2, &z2, q + g * G);"),
+    ("two-stage decode drops the second stage",
+     "stage1 + kvqo_dequant(q2[c], meta2[(th * ng + g) * 2], meta2[(th * ng + g) * 2 + 1]);", "stage1;"),
     ("compact codec takes 1/s from the unrounded scale", "const float inv = 1.0f / sf;", "const float inv = 1.0f / s;"),
     ("binary16 rounding truncates", "if (rem > 0x1000u || (rem == 0x1000u && (h & 1u)))\n            h += 1u;",
      "(void)rem;"),

@@ -933,3 +933,60 @@ def test_fast_reduce_queries_rounds_the_exact_sum_once():
     assert got.dtype == np.uint16 and got.shape == (1, 2, 4)
     assert [int(b) for b in got[0, 0]] == [0x3F80, 0x3F82, 0x3F81, 0xBF80]
     assert [float(x) for x in _widen(got[0, 1])] == [1.0, 0.0, 6.0, 2.0]
+
+
+# ----------------------------------------------------------------------------
+# second residual stage (QVG's progressive residual quantisation; the reading
+# in the oracle's header)
+# ----------------------------------------------------------------------------
+
+def test_encode2_worked_examples():
+    for case in _golden("eq1_two_stage_worked_examples.json")["cases"]:
+        x = np.array(case["x"], np.float32)[None, None, :]
+        cent = np.zeros((1, 1, 4), np.uint16)
+        idx, codes, meta, codes2, meta2 = O.encode2(x, cent, case["bits"], 4)
+        assert [float(v) for v in meta[0, 0, 0]] == [case["s1"], case["z1"]]
+        assert O.unpack(codes[0, 0], 4, case["bits"]).tolist() == case["q1"]
+        s2, z2 = (float(v) for v in meta2[0, 0, 0])
+        assert s2 == np.float32(case["s2"]) and z2 == case["z2"] and math.copysign(1.0, z2) == \
+            math.copysign(1.0, case["z2"])
+        assert O.unpack(codes2[0, 0], 4, case["bits"]).tolist() == case["q2"]
+        out = O.decode2(idx, codes, meta, codes2, meta2, cent, case["bits"], 4)
+        assert out[0, 0].tolist() == case["x_hat"]
+
+
+def test_encode2_stage_one_is_encode_and_error_bound():
+    """The stage-1 arrays are exactly ``encode``'s; every value is within half
+    a stage-2 step (plus the rounding of the two additions) of its
+    reconstruction, and the stage-2 step is at most the stage-1 step over
+    2^b - 1, so two stages never do worse than one."""
+    rng = np.random.default_rng(41)
+    for bits, G in ((2, 16), (4, 32), (2, 64)):
+        x = (rng.standard_normal((120, 3, 64)) * np.exp(rng.uniform(-3, 3, (120, 3, 1)))).astype(np.float32)
+        cent = O.fit(x, 16, 1)
+        e1 = O.encode(x, cent, bits, G)
+        idx, codes, meta, codes2, meta2 = O.encode2(x, cent, bits, G)
+        for a, b in zip((idx, codes, meta), e1):
+            assert np.array_equal(a, b)
+        xh1 = O.decode(*e1, cent, bits, G).astype(np.float64)
+        xh2 = O.decode2(idx, codes, meta, codes2, meta2, cent, bits, G).astype(np.float64)
+        s1 = np.repeat(meta[:, :, :, 0], G, axis=2).transpose(1, 0, 2).astype(np.float64)
+        s2 = np.repeat(meta2[:, :, :, 0], G, axis=2).transpose(1, 0, 2).astype(np.float64)
+        z2 = np.repeat(meta2[:, :, :, 1], G, axis=2).transpose(1, 0, 2)
+        err2 = np.abs(xh2 - x)
+        ulp = 2.0 ** -22 * (np.abs(x) + np.abs(xh1 - x) + 1e-30)
+        live = z2 == np.rint(z2)  # every group, degenerate ones included, has an integer zero
+        assert np.all(err2[live] <= s2[live] / 2 + ulp[live] + 2.0 ** -23 * s1[live])
+        assert np.all(s2 <= s1 / ((1 << bits) - 1) * (1 + 2.0 ** -20) + 1e-37)
+        assert np.abs(xh2 - x).mean() < np.abs(xh1 - x).mean()
+
+
+def test_encode2_residual_on_the_stage_one_grid_leaves_nothing():
+    """Residuals that stage 1 represents exactly leave e = 0: stage 2 is the
+    zero-range group (s2 = 0, z2 = 0, codes 0) and the reconstruction is the
+    stage-1 one."""
+    x = np.array([[[0.0, 0.5, 1.0, 1.5, 1.5, 0.0, 1.0, 0.5]]], np.float32)
+    cent = np.zeros((1, 1, 8), np.uint16)
+    idx, codes, meta, codes2, meta2 = O.encode2(x, cent, 2, 8)
+    assert np.all(meta2 == 0.0) and np.all(codes2 == 0)
+    assert np.array_equal(O.decode2(idx, codes, meta, codes2, meta2, cent, 2, 8), x)

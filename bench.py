@@ -22,7 +22,8 @@ softmax (kvq_layer_attention), and its dense part alone
 (kvq_attention_dense_lse); QuantWM's QSAC encode, PSAC coefficients and PSAC
 attention on the Wan-like layer; and NanoKV-Fast on the joint workload (the
 history decoded into a 64-dim space per head, low-space attention with query
-reduction and output restoration) beside its full-dimensional counterpart.
+reduction and output restoration) beside its full-dimensional counterpart;
+and the second residual stage's encode and decode on the Wan-like layer.
 
 Inputs are seeded synthetic tensors resident in HBM before timing starts;
 L2 is flushed (256 MiB write) before every timed step, outside the step's
@@ -483,6 +484,40 @@ def quantwm_rows(p2, steps, warmup, flush, world, device, tfl, hbm):
     }
 
 
+def stages_rows(p2, steps, warmup, flush, world, device, hbm):
+    """The second residual stage on the Wan-like layer (its K and V histories
+    and fitted centres): the two-stage encode beside the one-stage encode, and
+    the two-stage decode beside the one-stage decode."""
+    import torch
+
+    K, w = p2.K, p2.w
+    T = w.history_tokens
+    codecs = [K.Codec(c.num_heads, c.head_dim, c.num_centroids, c.bits, c.group_size, 0, K.KVQ_META_F32, 2)
+              for c in (p2.codec_k, p2.codec_v)]
+    enc = []
+    for c in codecs:
+        idx, codes, meta = K.alloc_encoded(c, T, device)
+        enc.append((idx, codes, meta, torch.empty_like(codes), torch.empty_like(meta)))
+    xs = (p2.xk, p2.xv)
+
+    def encode2():
+        for i in range(2):
+            K.kvq_encode_stages(codecs[i], xs[i], p2.cent[i], *enc[i])
+
+    enc_ms = max_over_ranks(time_calls(encode2, steps, warmup, flush), world, device)
+    comps = [K.Compressed(codecs[i], T, p2.cent[i], *enc[i][:3], codes2=enc[i][3], meta2=enc[i][4]) for i in range(2)]
+    dec_ms = max_over_ranks(time_calls(lambda: [K.kvq_decode(comps[i], p2.dec[i]) for i in range(2)], steps, warmup,
+                                       flush), world, device)
+    check_status(K, "after the two-stage rows")
+    H, d = w.num_heads, w.head_dim
+    dec_bytes = sum(T * H * (2 + 2 * (d * c.bits // 8 + 8 * d // c.group_size) + 2 * d) for c in codecs)
+    return {"two_stage": {"encode_ms": enc_ms, "decode_ms": dec_ms,
+                          "decode_gbs": dec_bytes / (dec_ms / 1e3) / 1e9,
+                          "decode_frac": dec_bytes / (dec_ms / 1e3) / 1e9 / hbm,
+                          "what": "second residual stage on the Wan-like layer (K and V, INT2 G16 twice): "
+                                  "kvq_encode_stages (exact CUDA-core path) and the two-stage kvq_decode to bf16"}}
+
+
 def fast_rows(joint, steps, warmup, flush, world, device, tfl, d_low=64):
     """NanoKV-Fast on the joint workload: its K and V joint codes decoded
     straight into a 64-dim space per head (folded analytical maps, set up
@@ -767,6 +802,7 @@ def run_gpu(args):
         }
         next_rows.update(quantwm_rows(p2, args.steps, args.warmup, flush, world, device, tfl, hbm))
         next_rows.update(fast_rows(joint, args.steps, args.warmup, flush, world, device, tfl))
+        next_rows.update(stages_rows(p2, args.steps, args.warmup, flush, world, device, hbm))
         launches += p2.launches_per_step * args.steps
         del p2
         torch.cuda.empty_cache()

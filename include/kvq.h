@@ -103,6 +103,9 @@ typedef struct {
     int32_t group_size;    /* G: multiple of 8 dividing d (per-head) or r (joint) */
     int32_t joint_rank;    /* 0: per-head codec; r > 0: joint head-channel code */
     int32_t meta_format;   /* kvq_meta_format; 0 (binary32) when zero-initialised */
+    int32_t residual_stages; /* 0 or 1: one residual stage; 2: a second stage
+                              * (kvq_encode_stages; per-head codec with binary32
+                              * {s, z} only) */
 } kvq_codec_desc;
 
 /* A compressed K or V history as produced by kvq_encode (read-only view). */
@@ -114,6 +117,8 @@ typedef struct {
     const uint8_t *codes;   /* per-head [H][T][d*b/8]; joint [T][r*b/8] */
     const void *meta;       /* per-head [H][T][d/G][2]; joint [T][r/G][2] (meta_format) */
     const void *w_dec;      /* joint only: decoder [r][H*d] bf16; else NULL */
+    const uint8_t *codes2;  /* residual_stages = 2: stage-2 codes, laid out as codes */
+    const float *meta2;     /* residual_stages = 2: stage-2 {s, z}, laid out as meta */
 } kvq_compressed_view;
 
 /* Human-readable name of a status code (static string, never NULL). */
@@ -216,6 +221,25 @@ KVQ_API kvq_status kvq_fit_centroids_static(const kvq_codec_desc *desc, const vo
 KVQ_API kvq_status kvq_encode(const kvq_codec_desc *desc, const void *x, kvq_dtype x_dtype, int64_t num_tokens,
                       const void *centroids, const void *w_enc, uint16_t *idx, uint8_t *codes, void *meta,
                       void *workspace, size_t workspace_bytes, kvq_stream_t stream);
+
+/*
+ * Encode with two residual stages (desc->residual_stages = 2).  The reading
+ * of QVG's progressive residual quantisation, which TempoKV (Sec. 2) names
+ * without giving its steps (NanoKV page, Table 4 evaluates QVG with one
+ * stage): idx, codes and meta exactly as kvq_encode writes them; then, per
+ * group, the error stage 1 leaves, e_c = r_c - (q_c - z) s (binary32), is
+ * quantised again with Eq. 1 on the same groups and bit width into codes2
+ * and meta2 (the same sizes and layouts as codes and meta).  kvq_decode of a
+ * view carrying codes2 / meta2 reconstructs (mu + (q1 - z1) s1) + (q2 - z2) s2,
+ * each operation rounded to binary32.  Per-head codec with binary32 {s, z}
+ * (KVQ_ERR_UNSUPPORTED otherwise); runs on the exact CUDA-core path for any
+ * history type and C; all arrays 16-byte aligned.  The attention calls refuse
+ * two-stage views (KVQ_ERR_UNSUPPORTED): decode them and use
+ * kvq_attention_dense_lse.
+ */
+KVQ_API kvq_status kvq_encode_stages(const kvq_codec_desc *desc, const void *x, kvq_dtype x_dtype, int64_t num_tokens,
+                                     const void *centroids, uint16_t *idx, uint8_t *codes, float *meta,
+                                     uint8_t *codes2, float *meta2, kvq_stream_t stream);
 
 /*
  * Encode one K history with QuantWM's query-sensitive centre selection

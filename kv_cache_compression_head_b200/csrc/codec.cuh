@@ -228,8 +228,10 @@ __device__ __forceinline__ void load_bf16x8(const uint16_t *p, float *out)
 // Quantise a residual row of D channels held in registers: per group of G
 // channels the Eq. 1 parameters, then packed codes (low bits first) and the
 // {s, z} pairs.  codes_row must be 16-byte aligned (D*BITS/8 is 16, 32 or 64).
-template <int D, int BITS, int G>
-__device__ __forceinline__ void encode_residual_row(const float *r, uint8_t *codes_row, void *meta_row, bool meta16)
+// ERR: also replace every r_c by the error this stage leaves,
+// r_c - (q_c - z) s (binary32; the input of a second residual stage).
+template <int D, int BITS, int G, bool ERR = false>
+__device__ __forceinline__ void encode_residual_row(float *r, uint8_t *codes_row, void *meta_row, bool meta16)
 {
     constexpr int kWords = D * BITS / 32;
     uint32_t words[kWords];
@@ -246,6 +248,11 @@ __device__ __forceinline__ void encode_residual_row(const float *r, uint8_t *cod
         }
         const GroupQ gq = group_params_store(mn, mx, BITS, meta16, meta_row, g);
         quant_group_into<G, BITS>(r + g * G, gq, mn, mx, words, g * G);
+        if constexpr (ERR) {
+#pragma unroll
+            for (int c = g * G; c < (g + 1) * G; ++c)
+                r[c] = __fsub_rn(r[c], __fmul_rn(__fsub_rn((float)quant_code(r[c], gq, BITS), gq.z), gq.s));
+        }
     }
     uint4 *dst = reinterpret_cast<uint4 *>(codes_row);
 #pragma unroll
@@ -275,6 +282,8 @@ struct EncodeArgs {
     void *meta;            // [H][T][D/G][2] float, or binary16 when meta16
     int assign_only;
     int meta16;
+    uint8_t *codes2;       // second residual stage (exact path only): as codes,
+    float *meta2;          // and as meta (binary32); NULL: one stage
 };
 
 template <int D, int BITS, int G>
@@ -358,8 +367,16 @@ __global__ void __launch_bounds__(kDirectTokens) encode_direct_kernel(EncodeArgs
             xr[c + k] = __fsub_rn(xr[c + k], m8[k]);
     }
     const int64_t th = (int64_t)h * a.T + t;
-    encode_residual_row<D, BITS, G>(xr, a.codes + th * (D * BITS / 8),
-                                    static_cast<uint8_t *>(a.meta) + th * (D / G) * (a.meta16 ? 4 : 8), a.meta16 != 0);
+    if (a.codes2) {
+        // two residual stages: the error stage 1 leaves, quantised again
+        encode_residual_row<D, BITS, G, true>(xr, a.codes + th * (D * BITS / 8),
+                                              static_cast<uint8_t *>(a.meta) + th * (D / G) * 8, false);
+        encode_residual_row<D, BITS, G>(xr, a.codes2 + th * (D * BITS / 8), a.meta2 + th * (D / G) * 2, false);
+    } else {
+        encode_residual_row<D, BITS, G>(xr, a.codes + th * (D * BITS / 8),
+                                        static_cast<uint8_t *>(a.meta) + th * (D / G) * (a.meta16 ? 4 : 8),
+                                        a.meta16 != 0);
+    }
 }
 
 // ---------------------------------------------------------------------------
@@ -544,6 +561,8 @@ struct DecodeArgs {
     void *out;
     int out_bf16;
     int meta16;
+    const uint8_t *codes2;  // second residual stage (binary32 {s, z} only); NULL: one stage
+    const float *meta2;
 };
 
 // One block per (tile of 256 / (D/8) tokens, head); thread = 8 channels of
@@ -590,6 +609,14 @@ __global__ void __launch_bounds__(256) decode_kernel(DecodeArgs a)
 #pragma unroll
         for (int k = 0; k < 8; ++k)
             v[k] = dequant_spec((cw >> (k * a.bits)) & mask, sz.x, sz.y, mu[k]);
+    }
+    if (a.codes2) {  // + (q2 - z2) s2
+        const float2 sz2 = reinterpret_cast<const float2 *>(a.meta2)[th * (D / a.G) + c0 / a.G];
+        const uint32_t cw2 = a.bits == 2 ? *reinterpret_cast<const uint16_t *>(a.codes2 + th * (D / 4) + c0 / 4)
+                                         : *reinterpret_cast<const uint32_t *>(a.codes2 + th * (D / 2) + c0 / 2);
+#pragma unroll
+        for (int k = 0; k < 8; ++k)
+            v[k] = __fadd_rn(v[k], __fmul_rn(__fsub_rn((float)((cw2 >> (k * a.bits)) & mask), sz2.y), sz2.x));
     }
     const int64_t o = (t * a.H + h) * D + c0;
     if (a.out_bf16) {

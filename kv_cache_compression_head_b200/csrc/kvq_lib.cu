@@ -53,6 +53,11 @@ kvq_status check_desc(const kvq_codec_desc *d, bool allow_joint)
         return KVQ_ERR_INVALID_ARG;
     if (d->meta_format == KVQ_META_F16 && d->joint_rank > 0)
         return KVQ_ERR_UNSUPPORTED;  // compact {s, z} is a per-head codec format
+    if (d->residual_stages < 0)
+        return KVQ_ERR_INVALID_ARG;
+    if (d->residual_stages > 2 ||
+        (d->residual_stages == 2 && (d->joint_rank > 0 || d->meta_format != KVQ_META_F32)))
+        return KVQ_ERR_UNSUPPORTED;
     const int span = d->joint_rank > 0 ? d->joint_rank : d->head_dim;
     if (d->group_size < 8 || d->group_size % 8 != 0 || span % d->group_size != 0)
         return KVQ_ERR_INVALID_ARG;
@@ -713,6 +718,8 @@ kvq_status check_history_pair(const kvq_compressed_view *k, const kvq_compressed
         return st;
     if (k->desc.joint_rank > 0 || v->desc.joint_rank > 0)
         return KVQ_ERR_UNSUPPORTED;
+    if (k->desc.residual_stages == 2 || v->desc.residual_stages == 2)
+        return KVQ_ERR_UNSUPPORTED;  // two-stage histories: decode, then dense attention
     if (k->desc.num_heads != v->desc.num_heads || k->desc.head_dim != v->desc.head_dim ||
         k->num_tokens != v->num_tokens)
         return KVQ_ERR_INVALID_ARG;
@@ -981,7 +988,10 @@ kvq_status kvq_encode(const kvq_codec_desc *desc, const void *x, kvq_dtype x_dty
     if (!aligned16(x) || !aligned16(centroids) || !aligned16(codes) || !aligned16(meta) ||
         (reinterpret_cast<uintptr_t>(idx) & 1u))
         return KVQ_ERR_ALIGNMENT;
+    if (desc->residual_stages == 2)
+        return KVQ_ERR_INVALID_ARG;  // two stages write two code sets: kvq_encode_stages
     EncodeArgs e;
+    memset(&e, 0, sizeof e);
     e.x = x;
     e.x_bf16 = x_dtype == KVQ_BF16;
     e.T = T;
@@ -998,6 +1008,44 @@ kvq_status kvq_encode(const kvq_codec_desc *desc, const void *x, kvq_dtype x_dty
     return launch_encode(desc->head_dim, e, reinterpret_cast<cudaStream_t>(stream));
 }
 
+kvq_status kvq_encode_stages(const kvq_codec_desc *desc, const void *x, kvq_dtype x_dtype, int64_t T,
+                             const void *centroids, uint16_t *idx, uint8_t *codes, float *meta, uint8_t *codes2,
+                             float *meta2, kvq_stream_t stream)
+{
+    kvq_status st = check_desc(desc, false);
+    if (st != KVQ_OK)
+        return st;
+    if (desc->residual_stages != 2)
+        return KVQ_ERR_INVALID_ARG;
+    if (T < 0 || (x_dtype != KVQ_F32 && x_dtype != KVQ_BF16))
+        return KVQ_ERR_INVALID_ARG;
+    if (desc->num_heads > 65535)
+        return KVQ_ERR_UNSUPPORTED;
+    if (T == 0)
+        return KVQ_OK;
+    if (!x || !centroids || !idx || !codes || !meta || !codes2 || !meta2)
+        return KVQ_ERR_INVALID_ARG;
+    if (!aligned16(x) || !aligned16(centroids) || !aligned16(codes) || !aligned16(meta) || !aligned16(codes2) ||
+        !aligned16(meta2) || (reinterpret_cast<uintptr_t>(idx) & 1u))
+        return KVQ_ERR_ALIGNMENT;
+    EncodeArgs e;
+    memset(&e, 0, sizeof e);
+    e.x = x;
+    e.x_bf16 = x_dtype == KVQ_BF16;
+    e.T = T;
+    e.H = desc->num_heads;
+    e.C = desc->num_centroids;
+    e.bits = desc->bits;
+    e.G = desc->group_size;
+    e.cent = static_cast<const uint16_t *>(centroids);
+    e.idx = idx;
+    e.codes = codes;
+    e.meta = meta;
+    e.codes2 = codes2;
+    e.meta2 = meta2;
+    return launch_encode_direct(desc->head_dim, e, reinterpret_cast<cudaStream_t>(stream));
+}
+
 kvq_status kvq_encode_qsac(const kvq_codec_desc *desc, const void *x, kvq_dtype x_dtype, int64_t T,
                            const void *centroids, const float *w, int32_t M, uint16_t *idx, uint8_t *codes,
                            void *meta, kvq_stream_t stream)
@@ -1007,7 +1055,7 @@ kvq_status kvq_encode_qsac(const kvq_codec_desc *desc, const void *x, kvq_dtype 
         return st;
     if (T < 0 || (x_dtype != KVQ_F32 && x_dtype != KVQ_BF16) || M < 1 || M > kQsacMaxM)
         return KVQ_ERR_INVALID_ARG;
-    if (desc->meta_format != KVQ_META_F32 || desc->num_heads > 65535)
+    if (desc->meta_format != KVQ_META_F32 || desc->residual_stages == 2 || desc->num_heads > 65535)
         return KVQ_ERR_UNSUPPORTED;
     if (T == 0)
         return KVQ_OK;
@@ -1104,6 +1152,15 @@ kvq_status kvq_decode(const kvq_compressed_view *view, void *x_out, kvq_dtype ou
         return launch_joint_decode(j, view->w_dec, reinterpret_cast<cudaStream_t>(stream));
     }
     DecodeArgs a;
+    memset(&a, 0, sizeof a);
+    if (view->desc.residual_stages == 2) {
+        if (!view->codes2 || !view->meta2)
+            return KVQ_ERR_INVALID_ARG;
+        if (!aligned16(view->codes2) || !aligned16(view->meta2))
+            return KVQ_ERR_ALIGNMENT;
+        a.codes2 = view->codes2;
+        a.meta2 = view->meta2;
+    }
     a.cent = static_cast<const uint16_t *>(view->centroids);
     a.idx = view->idx;
     a.codes = view->codes;
@@ -1302,7 +1359,7 @@ kvq_status kvq_psac_coefficients(const kvq_compressed_view *k, const void *x, kv
     kvq_status st = check_view(k);
     if (st != KVQ_OK)
         return st;
-    if (k->desc.joint_rank > 0 || rank != kPsacRank)
+    if (k->desc.joint_rank > 0 || k->desc.residual_stages == 2 || rank != kPsacRank)
         return KVQ_ERR_UNSUPPORTED;
     if (x_dtype != KVQ_F32 && x_dtype != KVQ_BF16)
         return KVQ_ERR_INVALID_ARG;

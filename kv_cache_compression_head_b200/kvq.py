@@ -41,7 +41,7 @@ KVQ_OP_LAYER_ATTENTION = 4
 
 EXPORTED = (
     "kvq_status_string", "kvq_encoded_sizes", "kvq_workspace_size", "kvq_fit_centroids",
-    "kvq_fit_centroids_static", "kvq_encode", "kvq_encode_qsac",
+    "kvq_fit_centroids_static", "kvq_encode", "kvq_encode_qsac", "kvq_encode_stages",
     "kvq_joint_coefficients", "kvq_decode", "kvq_psac_coefficients", "kvq_attention_lse", "kvq_attention_psac_lse",
     "kvq_attention_dense_lse", "kvq_fast_attention_lse", "kvq_fast_attention_workspace_size", "kvq_layer_attention",
     "kvq_set_wait_limit",
@@ -58,13 +58,13 @@ class KvqError(RuntimeError):
 class CodecDesc(ctypes.Structure):
     _fields_ = [("num_heads", ctypes.c_int32), ("head_dim", ctypes.c_int32), ("num_centroids", ctypes.c_int32),
                 ("bits", ctypes.c_int32), ("group_size", ctypes.c_int32), ("joint_rank", ctypes.c_int32),
-                ("meta_format", ctypes.c_int32)]
+                ("meta_format", ctypes.c_int32), ("residual_stages", ctypes.c_int32)]
 
 
 class CompressedView(ctypes.Structure):
     _fields_ = [("desc", CodecDesc), ("num_tokens", ctypes.c_int64), ("centroids", ctypes.c_void_p),
                 ("idx", ctypes.c_void_p), ("codes", ctypes.c_void_p), ("meta", ctypes.c_void_p),
-                ("w_dec", ctypes.c_void_p)]
+                ("w_dec", ctypes.c_void_p), ("codes2", ctypes.c_void_p), ("meta2", ctypes.c_void_p)]
 
 
 def _load():
@@ -82,6 +82,7 @@ def _load():
         "kvq_fit_centroids_static": [pdesc, vp, ctypes.c_int, i64, i32, vp, vp],
         "kvq_encode": [pdesc, vp, ctypes.c_int, i64, vp, vp, vp, vp, vp, vp, sz, vp],
         "kvq_encode_qsac": [pdesc, vp, ctypes.c_int, i64, vp, vp, i32, vp, vp, vp, vp],
+        "kvq_encode_stages": [pdesc, vp, ctypes.c_int, i64, vp, vp, vp, vp, vp, vp, vp],
         "kvq_joint_coefficients": [pdesc, vp, ctypes.c_int, i64, vp, vp, vp, vp, vp, sz, vp],
         "kvq_decode": [pview, vp, ctypes.c_int, vp, sz, vp],
         "kvq_attention_lse": [vp, i64, pview, pview, i64, i64, ctypes.c_float, vp, ctypes.c_int, vp, vp, sz, vp],
@@ -167,7 +168,7 @@ def _on_cuda(what: str, *ts) -> None:
     """Every tensor given (None skipped; Compressed records expanded) lives on a CUDA device."""
     for t in ts:
         if isinstance(t, Compressed):
-            _on_cuda(what, t.centroids, t.idx, t.codes, t.meta, t.w_dec)
+            _on_cuda(what, t.centroids, t.idx, t.codes, t.meta, t.w_dec, t.codes2, t.meta2)
         elif t is not None and not t.is_cuda:
             raise ValueError(f"{what}: expected CUDA tensors, got one on {t.device}")
 
@@ -204,6 +205,9 @@ def _want_compressed(what: str, comp: "Compressed") -> None:
     _want_encoded(what, c, comp.num_tokens, comp.idx, comp.codes, comp.meta)
     if comp.w_dec is not None:
         _want(f"{what} w_dec", comp.w_dec, torch.bfloat16, shape=(c.joint_rank, c.num_heads * c.head_dim))
+    if c.residual_stages == 2 or comp.codes2 is not None or comp.meta2 is not None:
+        _want(f"{what} codes2", comp.codes2, torch.uint8, numel=comp.codes.numel())
+        _want(f"{what} meta2", comp.meta2, torch.float32, numel=comp.meta.numel())
 
 
 def _want_attention_io(what: str, q: torch.Tensor, H: int, d: int, o_out, lse_out) -> int:
@@ -233,10 +237,11 @@ class Codec:
     group_size: int
     joint_rank: int = 0
     meta_format: int = KVQ_META_F32
+    residual_stages: int = 1
 
     def c(self) -> CodecDesc:
         return CodecDesc(self.num_heads, self.head_dim, self.num_centroids, self.bits, self.group_size,
-                         self.joint_rank, self.meta_format)
+                         self.joint_rank, self.meta_format, self.residual_stages)
 
 
 @dataclasses.dataclass
@@ -250,10 +255,13 @@ class Compressed:
     codes: torch.Tensor      # uint8
     meta: torch.Tensor       # float32, or float16 with compact {s, z}
     w_dec: Optional[torch.Tensor] = None
+    codes2: Optional[torch.Tensor] = None  # second residual stage: as codes
+    meta2: Optional[torch.Tensor] = None   # and as meta (float32)
 
     def view(self) -> CompressedView:
         return CompressedView(self.codec.c(), self.num_tokens, _ptr(self.centroids), _ptr(self.idx),
-                              _ptr(self.codes), _ptr(self.meta), _ptr(self.w_dec))
+                              _ptr(self.codes), _ptr(self.meta), _ptr(self.w_dec), _ptr(self.codes2),
+                              _ptr(self.meta2))
 
 
 def encoded_sizes(codec: Codec, num_tokens: int) -> Tuple[int, int, int]:
@@ -354,6 +362,24 @@ def kvq_encode_qsac(codec: Codec, x: torch.Tensor, centroids: torch.Tensor, w: t
     d = codec.c()
     _check(_lib.kvq_encode_qsac(ctypes.byref(d), _ptr(x), _dtype_code(x), T, _ptr(centroids), _ptr(w), M, _ptr(idx),
                                 _ptr(codes), _ptr(meta), _stream(stream)), "kvq_encode_qsac")
+
+
+def kvq_encode_stages(codec: Codec, x: torch.Tensor, centroids: torch.Tensor, idx: torch.Tensor,
+                      codes: torch.Tensor, meta: torch.Tensor, codes2: torch.Tensor, meta2: torch.Tensor,
+                      stream=None) -> None:
+    """Encode with two residual stages (codec.residual_stages == 2): the
+    stage-2 arrays have the shapes and types of codes and meta."""
+    T = _want_history("kvq_encode_stages x", codec, x)
+    _want("kvq_encode_stages centroids", centroids, torch.bfloat16,
+          shape=(codec.num_heads, codec.num_centroids, codec.head_dim))
+    _want_encoded("kvq_encode_stages", codec, T, idx, codes, meta)
+    _want("kvq_encode_stages codes2", codes2, torch.uint8, numel=codes.numel())
+    _want("kvq_encode_stages meta2", meta2, torch.float32, numel=meta.numel())
+    _on_cuda("kvq_encode_stages", x, centroids, idx, codes, meta, codes2, meta2)
+    d = codec.c()
+    _check(_lib.kvq_encode_stages(ctypes.byref(d), _ptr(x), _dtype_code(x), T, _ptr(centroids), _ptr(idx),
+                                  _ptr(codes), _ptr(meta), _ptr(codes2), _ptr(meta2), _stream(stream)),
+           "kvq_encode_stages")
 
 
 def kvq_joint_coefficients(codec: Codec, x: torch.Tensor, centroids: torch.Tensor, w_enc: torch.Tensor,

@@ -370,3 +370,33 @@ def test_fast_attention_rejected_on_host(K):
     assert K._lib.kvq_fast_attention_workspace_size(12, 128, 64, 10, ctypes.byref(n)) == K.KVQ_OK
     assert n.value >= need
     assert K._lib.kvq_fast_attention_workspace_size(12, 128, 32, 10, ctypes.byref(n)) == K.KVQ_ERR_UNSUPPORTED
+
+
+def test_two_stage_codec_refusals_on_host(K):
+    """A second residual stage: only through kvq_encode_stages, per-head codec
+    with binary32 {s, z}; the attention calls and QSAC / PSAC refuse two-stage
+    views; decode needs the stage-2 arrays."""
+    A = 1 << 20
+    f0 = ctypes.c_float(0)
+    d2 = K.CodecDesc(12, 128, 256, 2, 16, 0, K.KVQ_META_F32, 2)
+    sizes = lambda desc: K._lib.kvq_encoded_sizes(ctypes.byref(desc), 10, None, None, None)
+    assert sizes(d2) == K.KVQ_OK
+    assert sizes(K.CodecDesc(12, 128, 256, 2, 16, 0, K.KVQ_META_F16, 2)) == K.KVQ_ERR_UNSUPPORTED
+    assert sizes(K.CodecDesc(12, 128, 256, 4, 32, 192, K.KVQ_META_F32, 2)) == K.KVQ_ERR_UNSUPPORTED
+    assert sizes(K.CodecDesc(12, 128, 256, 2, 16, 0, K.KVQ_META_F32, 3)) == K.KVQ_ERR_UNSUPPORTED
+    assert sizes(K.CodecDesc(12, 128, 256, 2, 16, 0, K.KVQ_META_F32, -1)) == K.KVQ_ERR_INVALID_ARG
+    assert _err(K, "kvq_encode", ctypes.byref(d2), A, K.KVQ_BF16, 100, A, None, A, A, A, None, 0, None) \
+        == K.KVQ_ERR_INVALID_ARG
+    stages = lambda desc, *a: _err(K, "kvq_encode_stages", ctypes.byref(desc), A, K.KVQ_BF16, 100, A, *a, None)
+    assert stages(K.CodecDesc(12, 128, 256, 2, 16, 0), A, A, A, A, A) == K.KVQ_ERR_INVALID_ARG
+    assert stages(d2, A, A, A, None, A) == K.KVQ_ERR_INVALID_ARG
+    assert stages(d2, A, A, A, A + 8, A) == K.KVQ_ERR_ALIGNMENT
+    v2 = K.CompressedView(d2, 1000, A, A, A, A, None, None, None)
+    assert _err(K, "kvq_decode", ctypes.byref(v2), A, K.KVQ_F32, None, 0, None) == K.KVQ_ERR_INVALID_ARG
+    v2 = K.CompressedView(d2, 1000, A, A, A, A, None, A, A)
+    v1 = K.CompressedView(K.CodecDesc(12, 128, 256, 2, 16, 0), 1000, A, A, A, A, None)
+    assert _err(K, "kvq_attention_lse", A, 10, ctypes.byref(v2), ctypes.byref(v1), 0, 1000, f0, A, K.KVQ_F32, A,
+                None, 0, None) == K.KVQ_ERR_UNSUPPORTED
+    assert _err(K, "kvq_psac_coefficients", ctypes.byref(v2), A, K.KVQ_BF16, A, 8, A, None) == K.KVQ_ERR_UNSUPPORTED
+    assert _err(K, "kvq_encode_qsac", ctypes.byref(d2), A, K.KVQ_BF16, 100, A, A, 4, A, A, A, None) \
+        == K.KVQ_ERR_UNSUPPORTED

@@ -515,7 +515,7 @@ def stages_rows(p2, steps, warmup, flush, world, device, hbm):
                           "decode_gbs": dec_bytes / (dec_ms / 1e3) / 1e9,
                           "decode_frac": dec_bytes / (dec_ms / 1e3) / 1e9 / hbm,
                           "what": "second residual stage on the Wan-like layer (K and V, INT2 G16 twice): "
-                                  "kvq_encode_stages (exact CUDA-core path) and the two-stage kvq_decode to bf16"}}
+                                  "kvq_encode_stages (tensor-core filter) and the two-stage kvq_decode to bf16"}}
 
 
 def fast_rows(joint, steps, warmup, flush, world, device, tfl, d_low=64):

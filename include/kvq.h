@@ -232,8 +232,10 @@ KVQ_API kvq_status kvq_encode(const kvq_codec_desc *desc, const void *x, kvq_dty
  * and meta2 (the same sizes and layouts as codes and meta).  kvq_decode of a
  * view carrying codes2 / meta2 reconstructs (mu + (q1 - z1) s1) + (q2 - z2) s2,
  * each operation rounded to binary32.  Per-head codec with binary32 {s, z}
- * (KVQ_ERR_UNSUPPORTED otherwise); runs on the exact CUDA-core path for any
- * history type and C; all arrays 16-byte aligned.  The attention calls refuse
+ * (KVQ_ERR_UNSUPPORTED otherwise); all arrays 16-byte aligned.  Runs where
+ * kvq_encode does (the tensor-core filter for bf16 histories and the C it
+ * takes, else the exact CUDA-core kernel), with identical results on both
+ * paths.  The attention calls refuse
  * two-stage views (KVQ_ERR_UNSUPPORTED): decode them and use
  * kvq_attention_dense_lse.
  */

@@ -282,7 +282,7 @@ struct EncodeArgs {
     void *meta;            // [H][T][D/G][2] float, or binary16 when meta16
     int assign_only;
     int meta16;
-    uint8_t *codes2;       // second residual stage (exact path only): as codes,
+    uint8_t *codes2;       // second residual stage: as codes,
     float *meta2;          // and as meta (binary32); NULL: one stage
 };
 

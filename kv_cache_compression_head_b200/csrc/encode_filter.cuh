@@ -69,6 +69,8 @@ struct FilterArgs {
     int assign_only;
     int meta16;
     float kappa;       // k of the certified bound (see above)
+    uint8_t *codes2;   // second residual stage (kernel instantiated with TWO):
+    float *meta2;      // as codes, and as meta in binary32
 };
 
 // pair exchange of one epilogue group, two slots by tile parity:
@@ -131,41 +133,29 @@ __device__ __forceinline__ float spec_distance_smem(const uint8_t *sX, const uin
     return acc;
 }
 
-// Residual r = x - mu[best] of channels [half*CH, half*CH + CH) of one token,
-// read from the swizzled tiles, quantised per group (Eq. 1) and packed.  Three
-// phases over all of the thread's groups at once, so that the groups' chains
-// (min/max, the two IEEE divisions of Eq. 1, the codes) run side by side:
-// (1) min and max of every group, (2) Eq. 1 parameters of every group,
-// (3) codes, re-reading the residuals from shared memory.  Group min/max are
-// those of a strict scan in channel order; the two differ only in the sign
-// of a zero extreme, for which the group is rescanned in order.
-template <int CH, int BITS, int G>
-__device__ __forceinline__ void encode_residual_smem(const uint8_t *sX, const uint8_t *sMu, int Cpad, int row,
-                                                     int best, int half, uint8_t *codes_dst, void *meta_dst,
-                                                     bool meta16)
+// One residual stage of channels [half*CH, half*CH + CH) of one token: the
+// values come from val(uu, v8) (the 8 channels of unit uu of the half; group
+// g holds units g G/8 .. (g + 1) G/8 - 1), are quantised per group (Eq. 1)
+// and packed.  Three phases over all of the thread's groups at once, so that
+// the groups' chains (min/max, the two IEEE divisions of Eq. 1, the codes)
+// run side by side: (1) min and max of every group, (2) Eq. 1 parameters of
+// every group, (3) codes, asking val again.  Group min/max are those of a
+// strict scan in channel order; the two differ only in the sign of a zero
+// extreme, for which the group is rescanned in order.  The groups'
+// parameters are copied to gq_out / gf_out unless these are null.
+template <int CH, int BITS, int G, class Val>
+__device__ __forceinline__ void quantise_half(const Val &val, uint8_t *codes_dst, void *meta_dst, bool meta16,
+                                              GroupQ *gq_out, GroupFast *gf_out)
 {
     constexpr int kPerWord = 32 / BITS;
     constexpr int kWords = CH * BITS / 32;
     constexpr int NG = CH / G;
-    // residual of the 8 channels of unit uu (0 .. CH/8) of this thread's half
-    auto unit_residual = [&](int uu, float *r8) {
-        const int u = half * (CH / 8) + uu;
-        const uint4 xw = *reinterpret_cast<const uint4 *>(sX + sw128_unit_offset(row, u, kFltRows));
-        const uint4 mw = *reinterpret_cast<const uint4 *>(sMu + sw128_unit_offset(best, u, Cpad));
-        const uint32_t xa[4] = {xw.x, xw.y, xw.z, xw.w}, ma[4] = {mw.x, mw.y, mw.z, mw.w};
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-            const float2 d = sub2(make_float2(bf16_lo(xa[k]), bf16_hi(xa[k])), make_float2(bf16_lo(ma[k]), bf16_hi(ma[k])));
-            r8[2 * k] = d.x;
-            r8[2 * k + 1] = d.y;
-        }
-    };
     // (1) min / max of every group
     float mn[NG], mx[NG];
 #pragma unroll
     for (int g = 0; g < NG; ++g) {
         float r8[8];
-        unit_residual(g * (G / 8), r8);
+        val(g * (G / 8), r8);
         float a = fminf(r8[0], r8[1]), b = fmaxf(r8[0], r8[1]);
 #pragma unroll
         for (int c = 2; c < 8; c += 2) {
@@ -174,7 +164,7 @@ __device__ __forceinline__ void encode_residual_smem(const uint8_t *sX, const ui
         }
 #pragma unroll
         for (int uu = 1; uu < G / 8; ++uu) {
-            unit_residual(g * (G / 8) + uu, r8);
+            val(g * (G / 8) + uu, r8);
 #pragma unroll
             for (int c = 0; c < 8; c += 2) {
                 a = fmin3(a, r8[c], r8[c + 1]);
@@ -191,7 +181,7 @@ __device__ __forceinline__ void encode_residual_smem(const uint8_t *sX, const ui
             float a = 0.0f, b = 0.0f;
             for (int uu = 0; uu < G / 8; ++uu) {
                 float r8[8];
-                unit_residual(g * (G / 8) + uu, r8);
+                val(g * (G / 8) + uu, r8);
                 for (int c = 0; c < 8; ++c) {
                     if (uu == 0 && c == 0) {
                         a = r8[0];
@@ -226,7 +216,7 @@ __device__ __forceinline__ void encode_residual_smem(const uint8_t *sX, const ui
 #pragma unroll
             for (int uu = 0; uu < G / 8; ++uu) {
                 float r8[8];
-                unit_residual(g * (G / 8) + uu, r8);
+                val(g * (G / 8) + uu, r8);
 #pragma unroll
                 for (int k = 0; k < 8; ++k) {
                     const int c = g * G + uu * 8 + k;
@@ -237,7 +227,7 @@ __device__ __forceinline__ void encode_residual_smem(const uint8_t *sX, const ui
 #pragma unroll
             for (int uu = 0; uu < G / 8; ++uu) {
                 float r8[8];
-                unit_residual(g * (G / 8) + uu, r8);
+                val(g * (G / 8) + uu, r8);
 #pragma unroll
                 for (int k = 0; k < 8; ++k) {
                     const int c = g * G + uu * 8 + k;
@@ -256,6 +246,57 @@ __device__ __forceinline__ void encode_residual_smem(const uint8_t *sX, const ui
 #pragma unroll
         for (int v = 0; v < kWords; ++v)
             dst[v] = words[v];
+    }
+    if (gq_out) {
+#pragma unroll
+        for (int g = 0; g < NG; ++g) {
+            gq_out[g] = gq[g];
+            gf_out[g] = gf[g];
+        }
+    }
+}
+
+// Residual r = x - mu[best] of channels [half*CH, half*CH + CH) of one token,
+// read from the swizzled tiles, quantised per group (Eq. 1) and packed.  With
+// TWO, a second residual stage follows: the error e = r - (q - z) s the first
+// stage leaves (each operation rounded in binary32) is quantised on the same
+// groups with the same code width into codes2_dst / meta2_dst (binary32
+// {s, z}).
+template <int CH, int BITS, int G, bool TWO>
+__device__ __forceinline__ void encode_residual_smem(const uint8_t *sX, const uint8_t *sMu, int Cpad, int row,
+                                                     int best, int half, uint8_t *codes_dst, void *meta_dst,
+                                                     bool meta16, uint8_t *codes2_dst, float *meta2_dst)
+{
+    constexpr int NG = CH / G;
+    // residual of the 8 channels of unit uu of this thread's half
+    auto residual = [&](int uu, float *r8) {
+        const int u = half * (CH / 8) + uu;
+        const uint4 xw = *reinterpret_cast<const uint4 *>(sX + sw128_unit_offset(row, u, kFltRows));
+        const uint4 mw = *reinterpret_cast<const uint4 *>(sMu + sw128_unit_offset(best, u, Cpad));
+        const uint32_t xa[4] = {xw.x, xw.y, xw.z, xw.w}, ma[4] = {mw.x, mw.y, mw.z, mw.w};
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            const float2 d = sub2(make_float2(bf16_lo(xa[k]), bf16_hi(xa[k])), make_float2(bf16_lo(ma[k]), bf16_hi(ma[k])));
+            r8[2 * k] = d.x;
+            r8[2 * k + 1] = d.y;
+        }
+    };
+    GroupQ gq[NG];
+    GroupFast gf[NG];
+    quantise_half<CH, BITS, G>(residual, codes_dst, meta_dst, meta16, TWO ? gq : nullptr, TWO ? gf : nullptr);
+    if constexpr (TWO) {
+        // error of the first stage: the code again (quant_code_fast equals
+        // quant_code), then r - (q - z) s
+        auto error = [&](int uu, float *e8) {
+            const int g = uu / (G / 8);
+            residual(uu, e8);
+#pragma unroll
+            for (int k = 0; k < 8; ++k) {
+                const uint32_t q = gf[g].fast ? quant_code_fast<BITS>(e8[k], gf[g]) : quant_code(e8[k], gq[g], BITS);
+                e8[k] = __fsub_rn(e8[k], __fmul_rn(__fsub_rn((float)q, gq[g].z), gq[g].s));
+            }
+        };
+        quantise_half<CH, BITS, G>(error, codes2_dst, meta2_dst, false, nullptr, nullptr);
     }
 }
 
@@ -355,7 +396,7 @@ __device__ __forceinline__ void flt_scan_chunk(const float *p, const float *sA, 
 }
 
 
-template <int D, int BITS, int G>
+template <int D, int BITS, int G, bool TWO>
 __global__ void __launch_bounds__(kFltThreads, 1)
     encode_filter_kernel(const __grid_constant__ CUtensorMap tmap_x, FilterArgs a)
 {
@@ -687,10 +728,12 @@ __global__ void __launch_bounds__(kFltThreads, 1)
                         if (half == 0)
                             a.idx[th] = (uint16_t)best;
                         if (!a.assign_only)
-                            encode_residual_smem<CH, BITS, G>(
+                            encode_residual_smem<CH, BITS, G, TWO>(
                                 sX, sMu, Cpad, row, best, half, a.codes + th * (D * BITS / 8) + half * (CH * BITS / 8),
                                 static_cast<uint8_t *>(a.meta) + (th * (D / G) + half * (CH / G)) * (a.meta16 ? 4 : 8),
-                                a.meta16 != 0);
+                                a.meta16 != 0,
+                                TWO ? a.codes2 + th * (D * BITS / 8) + half * (CH * BITS / 8) : nullptr,
+                                TWO ? a.meta2 + (th * (D / G) + half * (CH / G)) * 2 : nullptr);
                     }
                 }
                 // X stage read: the TMA may refill it

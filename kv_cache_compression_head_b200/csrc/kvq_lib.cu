@@ -161,7 +161,7 @@ int filter_stages(int D, int Cpad)
     return fit < 2 ? 2 : (fit > kFltMaxStages ? kFltMaxStages : fit);
 }
 
-template <int D, int BITS, int G>
+template <int D, int BITS, int G, bool TWO>
 kvq_status launch_filter_t(const CUtensorMap &m, const FilterArgs &a, cudaStream_t s)
 {
     const uint32_t smem = flt_smem_bytes(D, a.Cpad, a.stages) + 1024;
@@ -170,7 +170,7 @@ kvq_status launch_filter_t(const CUtensorMap &m, const FilterArgs &a, cudaStream
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64)
         return KVQ_ERR_CUDA;
     if (!configured[dev].load()) {
-        if (cudaFuncSetAttribute(encode_filter_kernel<D, BITS, G>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        if (cudaFuncSetAttribute(encode_filter_kernel<D, BITS, G, TWO>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  227 * 1024) != cudaSuccess)
             return KVQ_ERR_CUDA;
         configured[dev].store(true);
@@ -180,7 +180,7 @@ kvq_status launch_filter_t(const CUtensorMap &m, const FilterArgs &a, cudaStream
     const int64_t units = (int64_t)a.H * a.ntiles;
     const int64_t sms = sm_count();
     const unsigned grid = (unsigned)(units < sms ? units : sms);
-    encode_filter_kernel<D, BITS, G><<<grid, kFltThreads, smem, s>>>(m, a);
+    encode_filter_kernel<D, BITS, G, TWO><<<grid, kFltThreads, smem, s>>>(m, a);
     return launch_status();
 }
 
@@ -188,11 +188,11 @@ template <int D, int BITS>
 kvq_status launch_filter_g(int G, const CUtensorMap &m, const FilterArgs &a, cudaStream_t s)
 {
     switch (G) {
-    case 16: return launch_filter_t<D, BITS, 16>(m, a, s);
-    case 32: return launch_filter_t<D, BITS, 32>(m, a, s);
+    case 16: return a.codes2 ? launch_filter_t<D, BITS, 16, true>(m, a, s) : launch_filter_t<D, BITS, 16, false>(m, a, s);
+    case 32: return a.codes2 ? launch_filter_t<D, BITS, 32, true>(m, a, s) : launch_filter_t<D, BITS, 32, false>(m, a, s);
     case 64:
         if constexpr (D >= 128)
-            return launch_filter_t<D, BITS, 64>(m, a, s);
+            return a.codes2 ? launch_filter_t<D, BITS, 64, true>(m, a, s) : launch_filter_t<D, BITS, 64, false>(m, a, s);
         return KVQ_ERR_UNSUPPORTED;
     default: return KVQ_ERR_UNSUPPORTED;
     }
@@ -236,6 +236,8 @@ kvq_status launch_encode_filter(int D, int bits, int G, const void *x, const Enc
     a.assign_only = e.assign_only;
     a.meta16 = e.meta16;
     a.kappa = filter_kappa(D);
+    a.codes2 = e.codes2;
+    a.meta2 = e.meta2;
     if (D == 128)
         return bits == 2 ? launch_filter_g<128, 2>(G, m, a, s) : launch_filter_g<128, 4>(G, m, a, s);
     return bits == 2 ? launch_filter_g<64, 2>(G, m, a, s) : launch_filter_g<64, 4>(G, m, a, s);
@@ -1043,7 +1045,7 @@ kvq_status kvq_encode_stages(const kvq_codec_desc *desc, const void *x, kvq_dtyp
     e.meta = meta;
     e.codes2 = codes2;
     e.meta2 = meta2;
-    return launch_encode_direct(desc->head_dim, e, reinterpret_cast<cudaStream_t>(stream));
+    return launch_encode(desc->head_dim, e, reinterpret_cast<cudaStream_t>(stream));
 }
 
 kvq_status kvq_encode_qsac(const kvq_codec_desc *desc, const void *x, kvq_dtype x_dtype, int64_t T,

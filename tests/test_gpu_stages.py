@@ -3,7 +3,10 @@ residual quantisation, named by TempoKV Sec. 2) against the oracle's encode2 /
 decode2: centre indices, both stages' codes and {s, z} bit-exact, the binary32
 two-stage reconstruction bit-exact and its bf16 output the round-to-nearest-
 even of it; bf16 and float32 histories, d = 64 and 128, both code widths,
-every group size; a ragged token count; the whole Wan-like K history."""
+every group size; a ragged token count; the whole Wan-like K history.  bf16
+histories with C <= 512 run on the tensor-core filter, the others on the
+exact CUDA-core kernel; the cases cover both, and one history is run through
+both (bf16 and its exact float32 widening) with identical outputs."""
 
 import numpy as np
 import pytest
@@ -62,6 +65,10 @@ def _check(x, cent, bits, G, got):
     ("14b", 700, 2, 2, 64, 600, False),
     ("tiny", 1024, 2, 4, 16, 16, True),
     ("tiny", 333, 2, 2, 32, 7, False),
+    ("14b", 901, 2, 4, 64, 300, False),     # filter, d = 128, INT4 G64
+    ("14b", 515, 2, 4, 16, 512, False),     # filter, the largest C it takes
+    ("tiny", 517, 2, 4, 16, 64, False),     # filter, d = 64
+    ("tiny", 129, 2, 2, 16, 33, False),     # filter, d = 64, INT2 G16
 ])
 def test_two_stage_encode_decode_bit_exact(name, T, H, bits, G, C, f32):
     w = synth.workload(name)
@@ -82,3 +89,16 @@ def test_two_stage_full_wan_history():
     x = synth.make_history(w, "K")
     cent = O.fit(x[:w.num_centroids], w.num_centroids, 0)
     _check(x, cent, w.bits_k, w.group_size, _run(x, cent, w.bits_k, w.group_size))
+
+
+def test_two_stage_filter_and_exact_paths_agree():
+    """The same Wan-like history as bf16 (filter) and as its float32 widening
+    (exact kernel): every output identical."""
+    w = synth.workload("wan13b")
+    x = np.ascontiguousarray(synth.make_history(w, "K", max_tokens=2050)[:, :4])
+    cent = O.fit(x[:128], 128, 0)
+    a = _run(x, cent, 2, 16)
+    b = _run(synth.bf16_bits_to_f32(x), cent, 2, 16)
+    for u, v in zip(a[:5], b[:5]):
+        assert torch.equal(u, v)
+    assert np.array_equal(f32_bits(a[5]), f32_bits(b[5]))

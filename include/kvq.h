@@ -169,7 +169,7 @@ KVQ_API kvq_status kvq_fit_centroids(const kvq_codec_desc *desc, const void *x, 
  *
  *  - Limit: the scratch kvq_workspace_size(KVQ_OP_FIT, desc, T, ...) reports
  *    must not exceed KVQ_FIT_STATIC_SCRATCH_BYTES (16 MiB: e.g. 12 heads x
- *    32,760 tokens x 256 centres x 128 channels needs 7.1 MB); larger requests return
+ *    32,760 tokens x 256 centres x 128 channels needs 7.9 MB); larger requests return
  *    KVQ_ERR_WORKSPACE before anything is launched.
  *  - The array is one per GPU that loads the library and is held until the
  *    process exits.  Every call on a device shares it: two calls whose work

@@ -730,6 +730,7 @@ struct FitArgs {
 //   fit_scan:    per (head, centre), per-chunk bases and totals    [H][C][nch], [H][C]
 //   fit_starts:  per head, bucket starts (prefix of the totals)    [H][C+1]
 //   fit_scatter: per (head, chunk), stable placement of token ids  order[H][T]
+//                and of their centres                               order_j[H][T]
 //   fit_segsum:  one warp per 64 consecutive slots of the sorted order: per
 //                run of one centre, binary64 sums per channel, added to the
 //                centre's totals with atomics (exact sums are order
@@ -756,6 +757,7 @@ struct FitSortArgs {
     int *chunk_counts;       // [H][C][nchunks] (counts, then bases)
     int *bucket_start;       // [H][C + 1]
     int *order;              // [H][T]
+    uint16_t *order_j;       // [H][T] centre of each slot of order
     double *sums;            // [H][C][D]
     unsigned *abs_max;       // [H] bits of the largest |x|
     unsigned *abs_min;       // [H] bits of the smallest nonzero |x| (+inf: none)
@@ -912,8 +914,10 @@ __global__ void __launch_bounds__(32) fit_scatter_kernel(FitSortArgs a)
         if (on && lane == leader)
             s_cur[j] += __popc(peers);
         __syncwarp();
-        if (on)
+        if (on) {
             a.order[(int64_t)h * a.T + slot] = (int)t;
+            a.order_j[(int64_t)h * a.T + slot] = (uint16_t)j;
+        }
     }
 }
 
@@ -942,10 +946,50 @@ __device__ __forceinline__ void fit_load_row(const FitSortArgs &a, int h, int64_
     }
 }
 
-template <int D>
-__global__ void __launch_bounds__(256) fit_segsum_kernel(FitSortArgs a)
+// Raw words of lane l's kPer channels of token t (bf16: kPer / 2 words,
+// binary32: kPer words), loaded as one vector.
+template <int D, bool BF16>
+struct FitRow {
+    static constexpr int kPer = D / 32;
+    static constexpr int kWords = BF16 ? kPer / 2 : kPer;
+    uint32_t w[kWords];
+
+    __device__ __forceinline__ void load(const FitSortArgs &a, int h, int64_t t, int lane)
+    {
+        const int64_t e = (t * a.H + h) * D + lane * kPer;
+        const uint32_t *p = BF16 ? reinterpret_cast<const uint32_t *>(static_cast<const uint16_t *>(a.x) + e)
+                                 : reinterpret_cast<const uint32_t *>(static_cast<const float *>(a.x) + e);
+        if constexpr (kWords == 4) {
+            const uint4 v = __ldg(reinterpret_cast<const uint4 *>(p));
+            w[0] = v.x; w[1] = v.y; w[2] = v.z; w[3] = v.w;
+        } else if constexpr (kWords == 2) {
+            const uint2 v = __ldg(reinterpret_cast<const uint2 *>(p));
+            w[0] = v.x; w[1] = v.y;
+        } else {
+            w[0] = __ldg(p);
+        }
+    }
+    __device__ __forceinline__ float value(int k) const
+    {
+        if constexpr (BF16)
+            return (k & 1) ? bf16_hi(w[k >> 1]) : bf16_lo(w[k >> 1]);
+        else
+            return __uint_as_float(w[k]);
+    }
+};
+
+// One warp per kFitSegSlots consecutive slots of the sorted order.  The
+// slots' token ids and centres are read coalesced up front (lane l holds
+// slots l and 32 + l), so no load waits on another; rows are then gathered
+// kBatch at a time, kept as raw words until used, and summed in slot order.
+// 64 registers (4 blocks of 256 per SM) keep more gathers in flight per SM
+// than a larger batch at lower occupancy.
+template <int D, bool BF16>
+__global__ void __launch_bounds__(256, 4) fit_segsum_kernel(FitSortArgs a)
 {
+    static_assert(kFitSegSlots == 64, "two slots per lane");
     constexpr int kPer = D / 32;
+    constexpr int kBatch = 8;
     const int lane = threadIdx.x & 31;
     const int64_t segs = (a.T + kFitSegSlots - 1) / kFitSegSlots;
     const int64_t gw = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
@@ -953,9 +997,11 @@ __global__ void __launch_bounds__(256) fit_segsum_kernel(FitSortArgs a)
         return;
     const int h = (int)(gw / segs);
     const int64_t i0 = (gw % segs) * kFitSegSlots;
-    const int64_t i1 = min(a.T, i0 + kFitSegSlots);
-    const int *ord = a.order + (int64_t)h * a.T;
-    const uint16_t *idx = a.idx + (int64_t)h * a.T;
+    const int nb = (int)min((int64_t)kFitSegSlots, a.T - i0);
+    const int *ord = a.order + (int64_t)h * a.T + i0;
+    const uint16_t *oj = a.order_j + (int64_t)h * a.T + i0;
+    const int tA = lane < nb ? ord[lane] : 0, tB = 32 + lane < nb ? ord[32 + lane] : 0;
+    const int jA = lane < nb ? (int)oj[lane] : -1, jB = 32 + lane < nb ? (int)oj[32 + lane] : -1;
 
     double acc[kPer];
     unsigned amax = 0u, amin = 0x7f800000u;
@@ -981,48 +1027,37 @@ __global__ void __launch_bounds__(256) fit_segsum_kernel(FitSortArgs a)
         rmax = 0u;
         rmin = 0x7f800000u;
     };
-    // the next 32 slots' token ids are fetched one round ahead; a round's rows
-    // are requested before its centre indices are consumed
-    int t_next = (i0 + lane < i1) ? ord[i0 + lane] : 0;
-    for (int64_t ib = i0; ib < i1; ib += 32) {
-        const int nb = (int)min((int64_t)32, i1 - ib);
-        const int t_l = t_next;
-        t_next = (ib + 32 + lane < i1) ? ord[ib + 32 + lane] : 0;
-        const int j_l = lane < nb ? (int)idx[t_l] : -1;
-        for (int b0 = 0; b0 < nb; b0 += 8) {
-            float v[8][kPer];
-            int jj[8];
+#pragma unroll 1
+    for (int b0 = 0; b0 < nb; b0 += kBatch) {
+        // a batch lies within one half (kBatch divides 32)
+        const int t_src = b0 < 32 ? tA : tB, j_src = b0 < 32 ? jA : jB;
+        FitRow<D, BF16> rows[kBatch];
 #pragma unroll
-            for (int b = 0; b < 8; ++b) {
-                const int t = __shfl_sync(0xffffffffu, t_l, (b0 + b) & 31);
-                if (b0 + b < nb)
-                    fit_load_row<D>(a, h, t, lane, v[b]);
+        for (int b = 0; b < kBatch; ++b) {
+            const int t = __shfl_sync(0xffffffffu, t_src, (b0 + b) & 31);
+            if (b0 + b < nb)
+                rows[b].load(a, h, t, lane);
+        }
+#pragma unroll
+        for (int b = 0; b < kBatch; ++b) {
+            const int j = __shfl_sync(0xffffffffu, j_src, (b0 + b) & 31);
+            if (b0 + b >= nb)
+                break;
+            if (j != cur) {
+                if (cur >= 0)
+                    flush();
+                cur = j;
             }
 #pragma unroll
-            for (int b = 0; b < 8; ++b) {
-                jj[b] = __shfl_sync(0xffffffffu, j_l, (b0 + b) & 31);
-                if (b0 + b >= nb)
-                    jj[b] = -1;
-            }
-#pragma unroll
-            for (int b = 0; b < 8; ++b) {
-                if (jj[b] < 0)
-                    break;
-                if (jj[b] != cur) {
-                    if (cur >= 0)
-                        flush();
-                    cur = jj[b];
-                }
-#pragma unroll
-                for (int k = 0; k < kPer; ++k) {
-                    acc[k] = __dadd_rn(acc[k], (double)v[b][k]);
-                    const unsigned u = __float_as_uint(v[b][k]) & 0x7fffffffu;
-                    rmax = max(rmax, u);
-                    rmin = min(rmin, u ? u : 0x7f800000u);
-                    if (a.track) {
-                        amax = max(amax, u);
-                        amin = min(amin, u ? u : 0x7f800000u);
-                    }
+            for (int k = 0; k < kPer; ++k) {
+                const float v = rows[b].value(k);
+                acc[k] = __dadd_rn(acc[k], (double)v);
+                const unsigned u = __float_as_uint(v) & 0x7fffffffu;
+                rmax = max(rmax, u);
+                rmin = min(rmin, u ? u : 0x7f800000u);
+                if (a.track) {
+                    amax = max(amax, u);
+                    amin = min(amin, u ? u : 0x7f800000u);
                 }
             }
         }

@@ -398,7 +398,7 @@ kvq_status joint_encode_call(const kvq_codec_desc *desc, const void *x, kvq_dtyp
 // Fit workspace: idx [H][T] u16 | per-chunk centre counts [H][nch][C] i32 |
 // bucket starts [H][C+1] i32 | token order [H][T] i32.
 struct FitLayout {
-    size_t idx, counts, starts, order, sums, bounds, redo, bkt, total;
+    size_t idx, counts, starts, order, order_j, sums, bounds, redo, bkt, total;
     int nchunks;
 };
 
@@ -413,7 +413,8 @@ FitLayout fit_layout(const kvq_codec_desc *d, int64_t T)
     L.counts = round_up(H * (size_t)T * 2, 256);
     L.starts = L.counts + round_up(H * (size_t)L.nchunks * C * 4, 256);
     L.order = L.starts + round_up(H * (C + 1) * 4, 256);
-    L.sums = L.order + round_up(H * (size_t)T * 4, 256);
+    L.order_j = L.order + round_up(H * (size_t)T * 4, 256);
+    L.sums = L.order_j + round_up(H * (size_t)T * 2, 256);
     L.bounds = L.sums + round_up(H * C * (size_t)d->head_dim * 8, 256);
     L.redo = L.bounds + round_up(H * 8, 256);
     L.bkt = L.redo + round_up(H * C * 4, 256);
@@ -854,6 +855,7 @@ kvq_status kvq_fit_centroids(const kvq_codec_desc *desc, const void *x, kvq_dtyp
     fs.chunk_counts = reinterpret_cast<int *>(ws + Lw.counts);
     fs.bucket_start = reinterpret_cast<int *>(ws + Lw.starts);
     fs.order = reinterpret_cast<int *>(ws + Lw.order);
+    fs.order_j = reinterpret_cast<uint16_t *>(ws + Lw.order_j);
     fs.sums = reinterpret_cast<double *>(ws + Lw.sums);
     fs.abs_max = reinterpret_cast<unsigned *>(ws + Lw.bounds);
     fs.abs_min = fs.abs_max + H;
@@ -895,11 +897,17 @@ kvq_status kvq_fit_centroids(const kvq_codec_desc *desc, const void *x, kvq_dtyp
         const unsigned cent_blocks = (unsigned)ceil_div(warps * 32, 256);
         fs.track = it == 0 ? 1 : 0;  // the head bounds need one pass over x
         if (D == 128) {
-            fit_segsum_kernel<128><<<seg_blocks, 256, 0, s>>>(fs);
+            if (fs.x_bf16)
+                fit_segsum_kernel<128, true><<<seg_blocks, 256, 0, s>>>(fs);
+            else
+                fit_segsum_kernel<128, false><<<seg_blocks, 256, 0, s>>>(fs);
             fit_finalize_kernel<128><<<cent_blocks, 256, 0, s>>>(fs);
             fit_bucket_update_kernel<128><<<cent_blocks, 256, 0, s>>>(fs);
         } else {
-            fit_segsum_kernel<64><<<seg_blocks, 256, 0, s>>>(fs);
+            if (fs.x_bf16)
+                fit_segsum_kernel<64, true><<<seg_blocks, 256, 0, s>>>(fs);
+            else
+                fit_segsum_kernel<64, false><<<seg_blocks, 256, 0, s>>>(fs);
             fit_finalize_kernel<64><<<cent_blocks, 256, 0, s>>>(fs);
             fit_bucket_update_kernel<64><<<cent_blocks, 256, 0, s>>>(fs);
         }

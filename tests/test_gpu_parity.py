@@ -378,3 +378,19 @@ def test_fit_token_order_sums_with_inexact_binary64():
         K.kvq_fit_centroids(codec, to_dev(x), it, cent)
         assert np.array_equal(bits_u16(cent), O.fit(x, C, it))
     _status_ok()
+
+
+@pytest.mark.parametrize("d,T,H,C,it", [(128, 2051, 3, 37, 2), (64, 777, 2, 64, 1)])
+def test_fit_float32_history(d, T, H, C, it):
+    """kvq_fit_centroids over a float32 history (the binary32 row gathers of
+    the centre sums; L from 24-bit significands) bit-exact against the oracle,
+    a ragged token count included."""
+    K = _K()
+    rng = np.random.default_rng(d * 1000 + T)
+    x = (rng.normal(size=(T, H, d)) * rng.uniform(0.2, 5, size=(1, H, d))).astype(np.float32)
+    x[::97] *= np.float32(2.0 ** -20)     # a spread of exponents in every head
+    codec = K.Codec(H, d, C, 2, 16)
+    cent = torch.empty((H, C, d), dtype=torch.bfloat16, device="cuda")
+    K.kvq_fit_centroids(codec, to_dev(x), it, cent)
+    assert np.array_equal(bits_u16(cent), O.fit(x, C, it))
+    _status_ok()

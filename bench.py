@@ -66,12 +66,15 @@ SECONDARY = "wan13b"
 JOINT = "joint"
 FLUSH_BYTES = 256 << 20
 # DRAM bytes (read + write) of one attention kernel launch of the headline
-# workload, from an ncu capture of the current kernel (dram__bytes_read.sum +
-# dram__bytes_write.sum of the first two history-block launches of a timed
-# step: 352.7 and 349.6 MB, against 329 MB of algorithmic bytes -- the
-# block's compressed K and V, the centres, Q and the binary32 partials of its
-# two sub-ranges); None whenever the kernel has changed since that capture.
-ATTN_NCU_TRAFFIC_BYTES = 351.1e6
+# workload from an ncu capture (dram__bytes_read.sum + dram__bytes_write.sum of
+# the first two history-block launches of a timed step: 352.7 and 349.6 MB,
+# against 329 MB of algorithmic bytes -- the block's compressed K and V, the
+# centres, Q and the binary32 partials of its two sub-ranges).  The kernel has
+# changed since (its bounded waits read their poll limit from constant memory;
+# its softmax warps drain the last commit after a give-up), so the line
+# reports traffic as null and the captured figure beside it, labelled.
+ATTN_NCU_TRAFFIC_BYTES = None
+ATTN_NCU_TRAFFIC_BEFORE_CHANGE = 351.1e6
 
 
 def parse_args():
@@ -832,6 +835,9 @@ def run_gpu(args):
                          "frac": attn_tflops / tfl, "peak_kind": f"{peak_kind} (bf16 dense, burst)",
                          "traffic": ATTN_NCU_TRAFFIC_BYTES,
                          "traffic_unit": "bytes per launch (ncu dram__bytes_read.sum + dram__bytes_write.sum)",
+                         "traffic_before_change": ATTN_NCU_TRAFFIC_BEFORE_CHANGE,
+                         "traffic_note": "captured before the give-up changes (wait limit read from constant "
+                                         "memory, drain after a give-up); not re-captured since",
                          "ms_per_launch": attn_call_ms},
             "rows": rows,
             "config2": secondary,

@@ -57,6 +57,8 @@ MUTATIONS = [
     ("compact codec keeps a scale that rounds to zero", " || (s16 & 0x7fffu) == 0u", ""),
     ("compact decode forgets the zero point", "float z = kvqo_f16_widen(meta16[(th * ng + g) * 2 + 1]);",
      "float z = 0.0f;"),
+    ("bf16 rounding ties away from zero", "u += 0x7fffu + keep_lsb;", "u += 0x8000u + 0u * keep_lsb;"),
+    ("bf16 rounding truncates", "u += 0x7fffu + keep_lsb;", "u += 0u * keep_lsb;"),
 ]
 
 

@@ -677,6 +677,32 @@ def test_qsac_ties_follow_index_order():
 # compact 16-bit {s, z} (TempoKV, Table 1: b + 1 bits per value at G = 32)
 # ----------------------------------------------------------------------------
 
+def test_bf16_round_matches_torch_and_hand_cases():
+    """binary32 -> bf16 (centres, joint residual): torch's conversion is an
+    independent round-to-nearest-even implementation; they agree on random
+    values over the whole exponent range, on exact ties, subnormals and on
+    overflow to infinity.  Hand cases: 1 + 2^-8 is a tie and goes to the even
+    neighbour 1.0 (0x3f80); 1 + 3 2^-8 goes up to 1 + 2^-6 (0x3f82); -0 keeps
+    its sign; a NaN stays a NaN."""
+    rng = np.random.default_rng(67)
+    mant = rng.integers(0, 1 << 23, size=6000, dtype=np.uint32)
+    expo = rng.integers(0, 255, size=6000, dtype=np.uint32)
+    sign = rng.integers(0, 2, size=6000, dtype=np.uint32)
+    u = (sign << 31) | (expo << 23) | mant
+    ties = (rng.integers(0, 1 << 16, size=2000, dtype=np.uint32) << 16) | np.uint32(0x8000)
+    ties = ties[((ties >> 23) & 0xFF) != 0xFF]
+    vals = np.concatenate([u, ties]).view(np.float32)
+    want = torch.from_numpy(vals.copy()).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    got = np.array([O.bf16_round(float(v)) for v in vals], np.uint16)
+    assert np.array_equal(got, want), f"differs at {vals[got != want][:5]}"
+    assert O.bf16_round(1.0 + 2.0 ** -8) == 0x3F80
+    assert O.bf16_round(1.0 + 3 * 2.0 ** -8) == 0x3F82
+    assert O.bf16_round(-0.0) == 0x8000
+    assert O.bf16_round(3.4e38) == 0x7F80                      # rounds past the largest bf16
+    nan = O.bf16_round(float("nan"))
+    assert (nan & 0x7F80) == 0x7F80 and (nan & 0x007F) != 0
+
+
 def test_f16_round_golden():
     g = _golden("eq1_f16_worked_examples.json")
     for case in g["round"]:

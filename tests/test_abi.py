@@ -22,7 +22,8 @@ def K():
 
 
 def _declared():
-    src = open(os.path.join(ROOT, "include", "kvq.h")).read()
+    with open(os.path.join(ROOT, "include", "kvq.h")) as f:
+        src = f.read()
     return sorted(set(re.findall(r"KVQ_API\s+[\w\s\*]*?\b(kvq_\w+)\s*\(", src)))
 
 

@@ -78,7 +78,8 @@ def _build_mutant(src: str, out_dir: str) -> str:
 
 @pytest.mark.parametrize("name,old,new", MUTATIONS, ids=[m[0] for m in MUTATIONS])
 def test_pins_catch_planted_mistake(name, old, new):
-    src = open(OB.SRC).read()
+    with open(OB.SRC) as f:
+        src = f.read()
     assert src.count(old) == 1, f"mutation site not unique or missing: {name}"
     saved_path, saved_lib = O._LIB_PATH, O._lib
     failed = []

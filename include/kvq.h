@@ -70,7 +70,7 @@ typedef struct CUstream_st *kvq_stream_t;
 typedef enum {
     KVQ_OK = 0,
     KVQ_ERR_INVALID_ARG = 1,    /* null pointer, bad size or shape */
-    KVQ_ERR_UNSUPPORTED = 2,    /* a valid request this build does not serve */
+    KVQ_ERR_UNSUPPORTED = 2,    /* a valid request the library does not serve */
     KVQ_ERR_ALIGNMENT = 3,      /* a pointer is not 16-byte aligned */
     KVQ_ERR_WORKSPACE = 4,      /* workspace missing or smaller than required */
     KVQ_ERR_CUDA = 5,           /* a CUDA runtime call or launch failed */
